@@ -12,7 +12,7 @@ __all__ = ["workloads", "ops"]
 
 
 def __getattr__(name):
-    if name == "ops":
-        from . import ops
-        return ops
+    if name in ("ops", "build"):
+        import importlib
+        return importlib.import_module(f"{__name__}.{name}")
     raise AttributeError(name)

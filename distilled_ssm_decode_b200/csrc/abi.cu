@@ -1,0 +1,200 @@
+// abi.cu -- the extern "C" entry points of libhyena_b200 (declared in include/hyena.h).
+//
+// Every entry point validates its arguments on the host and returns a
+// negative hyena_status before enqueuing anything when a check fails.  No
+// entry point allocates, frees or synchronises; all work goes on `stream`.
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace hyena;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+bool is_pow2(long long x) { return x > 0 && (x & (x - 1)) == 0; }
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA; }
+
+int check_common(int H, int d, int Dch) {
+    if (H < 1 || Dch < 0) return HYENA_ERR_SHAPE;
+    if (Dch % H != 0) return HYENA_ERR_SHAPE;
+    if (d < 1 || d > HYENA_MAX_MODES) return HYENA_ERR_SHAPE;
+    return HYENA_OK;
+}
+
+// Prefill workspace layout: [h: H*L f32][spectra: H*N c64][four-step planes][state partials]
+struct PrefillWs {
+    size_t h_off, spec_off, four_off, state_off, total;
+};
+
+PrefillWs prefill_ws(int B, int L, int Dch, int H, int d, int fft_len) {
+    PrefillWs w{};
+    const int N = fft_internal_len(fft_len);
+    const int ch = Dch / H;
+    w.h_off = 0;
+    w.spec_off = align_up((size_t)H * L * sizeof(float));
+    w.four_off = w.spec_off + align_up(spectrum_ws_bytes(H, N));
+    w.state_off = w.four_off + align_up(fourstep_ws_bytes(B, Dch, ch, N));
+    w.total = w.state_off + (N > kFusedMaxN ? align_up(state_ws_bytes(B, L, Dch, d)) : 0);
+    return w;
+}
+
+int check_prefill_shape(int B, int L, int Dch, int H, int d, int fft_len) {
+    if (B < 0 || L < 0) return HYENA_ERR_SHAPE;
+    int st = check_common(H, d, Dch);
+    if (st != HYENA_OK) return st;
+    if (!is_pow2(fft_len) || (long long)fft_len < 2LL * L - 1) return HYENA_ERR_SHAPE;
+    if (fft_len > kMaxFFT) return HYENA_ERR_UNSUPPORTED;
+    const int ch = Dch / H;
+    const long long slots = (ch % 2 == 0) ? Dch / 2 : Dch;
+    if (B > 65535) return HYENA_ERR_UNSUPPORTED;
+    if (fft_internal_len(fft_len) > kFusedMaxN && (long long)B * slots > 65535) return HYENA_ERR_UNSUPPORTED;
+    return HYENA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *hyena_status_string(int status) {
+    switch (status) {
+        case HYENA_OK: return "ok";
+        case HYENA_ERR_ARG: return "invalid argument (null pointer or unknown dtype)";
+        case HYENA_ERR_SHAPE: return "invalid shape (negative size, Dch % H != 0, d out of range, or bad fft_len)";
+        case HYENA_ERR_ALIGN: return "pointer misaligned for the required layout";
+        case HYENA_ERR_WORKSPACE: return "workspace missing or too small";
+        case HYENA_ERR_UNSUPPORTED: return "size outside what this build implements";
+        case HYENA_ERR_CUDA: return "CUDA launch or runtime error";
+        default: return "unknown status";
+    }
+}
+
+int hyena_abi_version(void) { return (1 << 16) | 0; }
+
+int hyena_filter_from_modes(const float *lambda, const float *R, const float *Dskip, int H, int d,
+                            int L, float *h_out, hyena_stream_t stream) {
+    if (H < 0 || L < 0 || d < 1 || d > HYENA_MAX_MODES) return HYENA_ERR_SHAPE;
+    if (H > 65535) return HYENA_ERR_UNSUPPORTED;
+    if (H == 0 || L == 0) return HYENA_OK;
+    if (!lambda || !R || !Dskip || !h_out) return HYENA_ERR_ARG;
+    if (!aligned(lambda, 8) || !aligned(R, 8) || !aligned(Dskip, 4) || !aligned(h_out, 4))
+        return HYENA_ERR_ALIGN;
+    return cuda_status(launch_filter(reinterpret_cast<const float2 *>(lambda),
+                                     reinterpret_cast<const float2 *>(R), Dskip, H, d, L, h_out,
+                                     (cudaStream_t)stream));
+}
+
+size_t hyena_filter_spectrum_workspace_bytes(int H, int L, int fft_len) {
+    if (H < 0 || L < 0 || !is_pow2(fft_len)) return 0;
+    return align_up(spectrum_ws_bytes(H, fft_len));
+}
+
+int hyena_filter_spectrum(const float *h, int H, int L, int fft_len, float *spec_out, void *workspace,
+                          size_t ws_bytes, hyena_stream_t stream) {
+    if (H < 0 || L < 0 || !is_pow2(fft_len) || fft_len < L || fft_len < 2) return HYENA_ERR_SHAPE;
+    if (fft_len < kMinFFT || fft_len > kMaxFFT || H > 65535) return HYENA_ERR_UNSUPPORTED;
+    if (H == 0) return HYENA_OK;
+    if (!h || !spec_out || !workspace) return HYENA_ERR_ARG;
+    if (!aligned(h, 4) || !aligned(spec_out, 8) || !aligned(workspace, kAlign)) return HYENA_ERR_ALIGN;
+    if (ws_bytes < hyena_filter_spectrum_workspace_bytes(H, L, fft_len)) return HYENA_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    float2 *perm = static_cast<float2 *>(workspace);
+    cudaError_t e = launch_spectrum_perm(h, H, L, fft_len, perm, 1.0f, s);
+    if (e != cudaSuccess) return HYENA_ERR_CUDA;
+    return cuda_status(launch_spectrum_natural(perm, H, fft_len, reinterpret_cast<float2 *>(spec_out), s));
+}
+
+size_t hyena_prefill_workspace_bytes(int B, int L, int Dch, int H, int d, int fft_len) {
+    if (check_prefill_shape(B, L, Dch, H, d, fft_len) != HYENA_OK) return 0;
+    return prefill_ws(B, L, Dch, H, d, fft_len).total;
+}
+
+int hyena_prefill(const void *q, const void *k, const void *v, int dtype, int B, int L, int Dch,
+                  int H, int d, int fft_len, const float *lambda, const float *R, const float *Dskip,
+                  void *y, float *state_out, void *workspace, size_t ws_bytes,
+                  hyena_stream_t stream) {
+    if (dtype != HYENA_F32 && dtype != HYENA_BF16) return HYENA_ERR_ARG;
+    int st = check_prefill_shape(B, L, Dch, H, d, fft_len);
+    if (st != HYENA_OK) return st;
+    if (B == 0 || Dch == 0) return HYENA_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (!state_out || !lambda || !R || !Dskip) return HYENA_ERR_ARG;
+    if (!aligned(state_out, 8) || !aligned(lambda, 8) || !aligned(R, 8) || !aligned(Dskip, 4))
+        return HYENA_ERR_ALIGN;
+    if (L == 0)
+        return cuda_status(cudaMemsetAsync(state_out, 0, (size_t)B * d * Dch * 2 * sizeof(float), s));
+    if (!q || !k || !v || !y || !workspace) return HYENA_ERR_ARG;
+    const size_t ab = (dtype == HYENA_BF16) ? 2 : 4;
+    if (!aligned(q, 2 * ab) || !aligned(k, 2 * ab) || !aligned(v, 2 * ab) || !aligned(y, 2 * ab) ||
+        !aligned(workspace, kAlign))
+        return HYENA_ERR_ALIGN;
+    const PrefillWs w = prefill_ws(B, L, Dch, H, d, fft_len);
+    if (ws_bytes < w.total) return HYENA_ERR_WORKSPACE;
+    char *ws = static_cast<char *>(workspace);
+    float *h = reinterpret_cast<float *>(ws + w.h_off);
+    float2 *spec = reinterpret_cast<float2 *>(ws + w.spec_off);
+    const int N = fft_internal_len(fft_len);
+    const float2 *lam2 = reinterpret_cast<const float2 *>(lambda);
+    cudaError_t e = launch_filter(lam2, reinterpret_cast<const float2 *>(R), Dskip, H, d, L, h, s);
+    if (e != cudaSuccess) return HYENA_ERR_CUDA;
+    // the inverse transform is unnormalised: fold its 1/N into the spectrum
+    e = launch_spectrum_perm(h, H, L, N, spec, 1.0f / (float)N, s);
+    if (e != cudaSuccess) return HYENA_ERR_CUDA;
+    e = launch_prefill_fft(q, k, v, dtype, B, L, Dch, H, d, N, spec, lam2, y, state_out,
+                           ws + w.four_off, w.total - w.four_off, s);
+    return cuda_status(e);
+}
+
+size_t hyena_prompt_state_workspace_bytes(int B, int L, int Dch, int d) {
+    if (B < 0 || L < 0 || Dch < 0 || d < 1 || d > HYENA_MAX_MODES) return 0;
+    return align_up(state_ws_bytes(B, L, Dch, d));
+}
+
+int hyena_prompt_state(const void *k, const void *v, int dtype, int B, int L, int Dch, int H, int d,
+                       const float *lambda, float *state_out, void *workspace, size_t ws_bytes,
+                       hyena_stream_t stream) {
+    if (dtype != HYENA_F32 && dtype != HYENA_BF16) return HYENA_ERR_ARG;
+    if (B < 0 || L < 0) return HYENA_ERR_SHAPE;
+    int st = check_common(H, d, Dch);
+    if (st != HYENA_OK) return st;
+    if (B > 65535) return HYENA_ERR_UNSUPPORTED;
+    if (B == 0 || Dch == 0) return HYENA_OK;
+    if (!state_out || !lambda) return HYENA_ERR_ARG;
+    if (!aligned(state_out, 8) || !aligned(lambda, 8)) return HYENA_ERR_ALIGN;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (L == 0)
+        return cuda_status(cudaMemsetAsync(state_out, 0, (size_t)B * d * Dch * 2 * sizeof(float), s));
+    if (!k || !v || !workspace) return HYENA_ERR_ARG;
+    const size_t ab = (dtype == HYENA_BF16) ? 2 : 4;
+    if (!aligned(k, ab) || !aligned(v, ab) || !aligned(workspace, kAlign)) return HYENA_ERR_ALIGN;
+    if (ws_bytes < hyena_prompt_state_workspace_bytes(B, L, Dch, d)) return HYENA_ERR_WORKSPACE;
+    return cuda_status(launch_prompt_state(k, v, dtype, B, L, Dch, H, d,
+                                           reinterpret_cast<const float2 *>(lambda), state_out,
+                                           workspace, s));
+}
+
+int hyena_decode_step(const void *q, const void *k, const void *v, int dtype, int B, int Dch, int H,
+                      int d, const float *lambda, const float *R, const float *Dskip, float *state,
+                      void *y, hyena_stream_t stream) {
+    if (dtype != HYENA_F32 && dtype != HYENA_BF16) return HYENA_ERR_ARG;
+    if (B < 0) return HYENA_ERR_SHAPE;
+    int st = check_common(H, d, Dch);
+    if (st != HYENA_OK) return st;
+    if (B == 0 || Dch == 0) return HYENA_OK;
+    if (!q || !k || !v || !y || !state || !lambda || !R || !Dskip) return HYENA_ERR_ARG;
+    const size_t ab = (dtype == HYENA_BF16) ? 2 : 4;
+    if (!aligned(q, ab) || !aligned(k, ab) || !aligned(v, ab) || !aligned(y, ab) ||
+        !aligned(state, 8) || !aligned(lambda, 8) || !aligned(R, 8) || !aligned(Dskip, 4))
+        return HYENA_ERR_ALIGN;
+    return cuda_status(launch_decode_step(q, k, v, dtype, B, Dch, H, d,
+                                          reinterpret_cast<const float2 *>(lambda),
+                                          reinterpret_cast<const float2 *>(R), Dskip, state, y,
+                                          (cudaStream_t)stream));
+}
+
+}  // extern "C"

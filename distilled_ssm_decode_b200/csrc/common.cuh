@@ -1,0 +1,72 @@
+// common.cuh -- small device helpers shared by the libhyena_b200 kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/hyena.h"
+
+namespace hyena {
+
+// ---------------------------------------------------------------- activations
+// Activation element types.  Loads widen to fp32; stores round to nearest-even.
+struct ActF32 {
+    using T = float;
+    static constexpr int bytes = 4;
+    __device__ __forceinline__ static float ld(const T *p) { return __ldg(p); }
+    __device__ __forceinline__ static void st(T *p, float x) { *p = x; }
+    // two consecutive channels
+    __device__ __forceinline__ static float2 ld2(const T *p) {
+        return __ldg(reinterpret_cast<const float2 *>(p));
+    }
+    __device__ __forceinline__ static void st2(T *p, float a, float b) {
+        *reinterpret_cast<float2 *>(p) = make_float2(a, b);
+    }
+};
+
+struct ActBF16 {
+    using T = __nv_bfloat16;
+    static constexpr int bytes = 2;
+    __device__ __forceinline__ static float ld(const T *p) { return __bfloat162float(*p); }
+    __device__ __forceinline__ static void st(T *p, float x) { *p = __float2bfloat16_rn(x); }
+    __device__ __forceinline__ static float2 ld2(const T *p) {
+        unsigned int w = __ldg(reinterpret_cast<const unsigned int *>(p));
+        // bf16 -> fp32 is exact: the bf16 bits are the high half of the fp32 word
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+    __device__ __forceinline__ static void st2(T *p, float a, float b) {
+        __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+        *reinterpret_cast<__nv_bfloat162 *>(p) = v;
+    }
+};
+
+// ---------------------------------------------------------------- complex fp32
+__device__ __forceinline__ float2 cmul(float2 a, float2 b) {
+    return make_float2(fmaf(a.x, b.x, -a.y * b.y), fmaf(a.x, b.y, a.y * b.x));
+}
+__device__ __forceinline__ float2 cmulc(float2 a, float2 b) {  // a * conj(b)
+    return make_float2(fmaf(a.x, b.x, a.y * b.y), fmaf(a.y, b.x, -a.x * b.y));
+}
+__device__ __forceinline__ float2 cadd(float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); }
+__device__ __forceinline__ float2 csub(float2 a, float2 b) { return make_float2(a.x - b.x, a.y - b.y); }
+__device__ __forceinline__ float2 cscale(float2 a, float s) { return make_float2(a.x * s, a.y * s); }
+
+// ---------------------------------------------------------------- complex fp64
+struct cd { double x, y; };
+__device__ __forceinline__ cd cdmul(cd a, cd b) {
+    return cd{fma(a.x, b.x, -a.y * b.y), fma(a.x, b.y, a.y * b.x)};
+}
+// lambda^m by binary powering in fp64 (m >= 0; lambda^0 = 1 also for lambda = 0).
+__device__ __forceinline__ cd cdpow(cd lam, long long m) {
+    cd r{1.0, 0.0};
+    cd b = lam;
+    while (m > 0) {
+        if (m & 1) r = cdmul(r, b);
+        b = cdmul(b, b);
+        m >>= 1;
+    }
+    return r;
+}
+
+}  // namespace hyena

@@ -1,0 +1,49 @@
+// kernels.h -- internal launchers of libhyena_b200 (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace hyena {
+
+// Largest FFT handled by one CTA in shared memory; longer transforms take the
+// four-step route through the workspace.
+constexpr int kFusedMaxN = 16384;
+// Size of the inner (shared-memory) transform of the four-step route.
+constexpr int kFourStepN2 = 8192;
+constexpr int kMaxFFT = 1 << 17;
+// FFT lengths below this are raised to it internally (same result).
+constexpr int kMinFFT = 64;
+
+inline int fft_internal_len(int fft_len) { return fft_len < kMinFFT ? kMinFFT : fft_len; }
+
+// filter.cu
+cudaError_t launch_filter(const float2 *lam, const float2 *R, const float *Dskip,
+                          int H, int d, int L, float *h, cudaStream_t s);
+
+// prefill_fft.cu
+size_t spectrum_ws_bytes(int H, int N);               // digit-reversed spectra (+ four-step scratch)
+// scale multiplies the transform (1/N for the convolution, 1 for the plain DFT)
+cudaError_t launch_spectrum_perm(const float *h, int H, int L, int N, float2 *spec_perm,
+                                 float scale, cudaStream_t s);
+cudaError_t launch_spectrum_natural(const float2 *spec_perm, int H, int N, float2 *out,
+                                    cudaStream_t s);
+size_t fourstep_ws_bytes(int B, int Dch, int ch, int N);
+cudaError_t launch_prefill_fft(const void *q, const void *k, const void *v, int dtype,
+                               int B, int L, int Dch, int H, int d, int N,
+                               const float2 *spec_perm, const float2 *lam,
+                               void *y, float *state_out, void *scratch, size_t scratch_bytes,
+                               cudaStream_t s);
+
+// state.cu
+size_t state_ws_bytes(int B, int L, int Dch, int d);
+cudaError_t launch_prompt_state(const void *k, const void *v, int dtype, int B, int L, int Dch,
+                                int H, int d, const float2 *lam, float *state_out,
+                                void *scratch, cudaStream_t s);
+
+// decode.cu
+cudaError_t launch_decode_step(const void *q, const void *k, const void *v, int dtype,
+                               int B, int Dch, int H, int d, const float2 *lam, const float2 *R,
+                               const float *Dskip, float *state, void *y, cudaStream_t s);
+
+}  // namespace hyena

@@ -1,0 +1,115 @@
+// state.cu -- prompt -> recurrent-state reduction (Vandermonde contraction).
+//
+// s[b][n][c] = sum_{j<L} lambda_n^(L-1-j) u[b][j][c],  u = k * v:
+// the O(d)-per-channel state that lets generation continue in O(1) per token
+// after a prompt ("Laughing Hyena Distillery", nubint.ai review, "Main
+// findings"; the recurrence is the modal SSM of "Proposed method").
+//
+// Kernel 1: one thread per (batch, channel, prompt segment) runs Horner's rule
+// over its segment for every mode (acc <- acc * lambda + u), then scales by
+// lambda^(L - segment end) (fp64 binary powering) and writes a partial state.
+// Kernel 2 adds the partials of each (b, n, c) in segment order, so the result
+// does not depend on scheduling.  Consecutive threads take consecutive
+// channels, so every token row is read coalesced.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace hyena {
+
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kModeChunk = 16;
+
+int choose_nseg(int B, int L, int Dch) {
+    const long long want = 148LL * 1024;   // threads to cover the GPU
+    long long cols = (long long)B * Dch;
+    long long nseg = (want + cols - 1) / cols;
+    long long maxseg = (L + 63) / 64;      // keep segments >= 64 tokens
+    if (nseg > maxseg) nseg = maxseg;
+    if (nseg < 1) nseg = 1;
+    return (int)nseg;
+}
+
+template <class Act>
+__global__ void __launch_bounds__(kThreads)
+state_partial_kernel(const typename Act::T *__restrict__ k, const typename Act::T *__restrict__ v,
+                     int L, int Dch, int ch, int d, int seglen, const float2 *__restrict__ lam,
+                     float2 *__restrict__ part /* [B][nseg][d][Dch] */) {
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= Dch) return;
+    const int g = blockIdx.y, b = blockIdx.z, nseg = gridDim.y;
+    const int hd = c / ch;
+    const int j0 = g * seglen, j1 = min(L, j0 + seglen);
+    for (int n0 = 0; n0 < d; n0 += kModeChunk) {
+        float2 l[kModeChunk], a[kModeChunk];
+#pragma unroll
+        for (int i = 0; i < kModeChunk; ++i) {
+            l[i] = (n0 + i < d) ? __ldg(&lam[(size_t)hd * d + n0 + i]) : make_float2(0.f, 0.f);
+            a[i] = make_float2(0.f, 0.f);
+        }
+        for (int j = j0; j < j1; ++j) {
+            const size_t o = ((size_t)b * L + j) * Dch + c;
+            const float u = Act::ld(k + o) * Act::ld(v + o);
+#pragma unroll
+            for (int i = 0; i < kModeChunk; ++i)
+                a[i] = make_float2(fmaf(a[i].x, l[i].x, fmaf(-a[i].y, l[i].y, u)),
+                                   fmaf(a[i].x, l[i].y, a[i].y * l[i].x));
+        }
+#pragma unroll
+        for (int i = 0; i < kModeChunk; ++i) {
+            const int n = n0 + i;
+            if (n >= d) break;
+            float2 r = make_float2(0.f, 0.f);
+            if (j1 > j0) {
+                const cd pw = cdpow(cd{l[i].x, l[i].y}, (long long)(L - j1));
+                r = cmul(a[i], make_float2((float)pw.x, (float)pw.y));
+            }
+            part[(((size_t)b * nseg + g) * d + n) * Dch + c] = r;
+        }
+    }
+}
+
+__global__ void state_sum_kernel(const float2 *__restrict__ part, int nseg, int d, int Dch,
+                                 float2 *__restrict__ state) {
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= Dch) return;
+    const int n = blockIdx.y, b = blockIdx.z;
+    float2 s = make_float2(0.f, 0.f);
+    for (int g = 0; g < nseg; ++g) s = cadd(s, part[(((size_t)b * nseg + g) * d + n) * Dch + c]);
+    state[((size_t)b * d + n) * Dch + c] = s;
+}
+
+}  // namespace
+
+size_t state_ws_bytes(int B, int L, int Dch, int d) {
+    if (L <= 0) return 0;
+    return (size_t)B * choose_nseg(B, L, Dch) * d * Dch * sizeof(float2);
+}
+
+cudaError_t launch_prompt_state(const void *k, const void *v, int dtype, int B, int L, int Dch,
+                                int H, int d, const float2 *lam, float *state_out, void *scratch,
+                                cudaStream_t s) {
+    if (B == 0 || Dch == 0) return cudaSuccess;
+    if (L == 0) return cudaMemsetAsync(state_out, 0, (size_t)B * d * Dch * 2 * sizeof(float), s);
+    const int ch = Dch / H;
+    const int nseg = choose_nseg(B, L, Dch);
+    const int seglen = (L + nseg - 1) / nseg;
+    float2 *part = static_cast<float2 *>(scratch);
+    dim3 grid((Dch + kThreads - 1) / kThreads, nseg, B);
+    if (dtype == HYENA_BF16)
+        state_partial_kernel<ActBF16><<<grid, kThreads, 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v), L, Dch, ch,
+            d, seglen, lam, part);
+    else
+        state_partial_kernel<ActF32><<<grid, kThreads, 0, s>>>(
+            static_cast<const float *>(k), static_cast<const float *>(v), L, Dch, ch, d, seglen, lam,
+            part);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    dim3 g2((Dch + 255) / 256, d, B);
+    state_sum_kernel<<<g2, 256, 0, s>>>(part, nseg, d, Dch, reinterpret_cast<float2 *>(state_out));
+    return cudaGetLastError();
+}
+
+}  // namespace hyena

@@ -1,0 +1,189 @@
+"""Python binding of libhyena_b200 (argument marshalling only).
+
+Every function here passes device pointers, sizes and the current CUDA stream
+to the C ABI declared in ``include/hyena.h``; all arithmetic runs in the
+library's CUDA kernels.  There is no fallback: if the shared library is
+missing or cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhyena_b200.so")
+
+HYENA_F32, HYENA_BF16 = 0, 1
+_DT = {torch.float32: HYENA_F32, torch.bfloat16: HYENA_BF16}
+
+_lock = threading.Lock()
+_lib = None
+
+_vp, _fp, _i, _sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+
+# name -> (restype, argtypes)
+SIGNATURES = {
+    "hyena_status_string": (ctypes.c_char_p, [_i]),
+    "hyena_abi_version": (_i, []),
+    "hyena_filter_from_modes": (_i, [_fp, _fp, _fp, _i, _i, _i, _fp, _vp]),
+    "hyena_filter_spectrum_workspace_bytes": (_sz, [_i, _i, _i]),
+    "hyena_filter_spectrum": (_i, [_fp, _i, _i, _i, _fp, _vp, _sz, _vp]),
+    "hyena_prefill_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "hyena_prefill": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp, _fp,
+                           _vp, _sz, _vp]),
+    "hyena_prompt_state_workspace_bytes": (_sz, [_i, _i, _i, _i]),
+    "hyena_prompt_state": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _fp, _fp, _vp, _sz, _vp]),
+    "hyena_decode_step": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _fp, _fp, _fp, _fp, _vp, _vp]),
+}
+
+
+class HyenaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: status {status} ({status_string(status)})")
+        self.status = status
+
+
+def lib():
+    """The loaded ctypes library (raises if the CUDA library is missing)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"libhyena_b200.so not found at {LIB_PATH}; build it with "
+                    "`python -m distilled_ssm_decode_b200.build` (there is no CPU fallback)")
+            L = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                f = getattr(L, name)
+                f.restype = res
+                f.argtypes = args
+            _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().hyena_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise HyenaError(fn, status)
+
+
+def _ptr(t: torch.Tensor):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream(device=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _cuda(t: torch.Tensor, name: str, dtype=None) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _params(lam, R, Dskip):
+    lam = _cuda(lam, "lam", torch.float32)
+    R = _cuda(R, "R", torch.float32)
+    Dskip = _cuda(Dskip, "Dskip", torch.float32)
+    if lam.dim() != 3 or lam.shape[-1] != 2 or R.shape != lam.shape or Dskip.shape != lam.shape[:1]:
+        raise ValueError("lam, R must be [H][d][2] float32 and Dskip [H]")
+    return lam, R, Dskip
+
+
+def _act_dtype(t: torch.Tensor) -> int:
+    if t.dtype not in _DT:
+        raise TypeError(f"activations must be float32 or bfloat16, got {t.dtype}")
+    return _DT[t.dtype]
+
+
+# ------------------------------------------------------------------ operations
+def filter_from_modes(lam, R, Dskip, L: int) -> torch.Tensor:
+    """h [H][L] float32: h_0 = Dskip, h_j = Re sum_n R_n lam_n^(j-1)."""
+    lam, R, Dskip = _params(lam, R, Dskip)
+    H, d = lam.shape[0], lam.shape[1]
+    h = torch.empty((H, L), dtype=torch.float32, device=lam.device)
+    _check("hyena_filter_from_modes",
+           lib().hyena_filter_from_modes(_ptr(lam), _ptr(R), _ptr(Dskip), H, d, L, _ptr(h),
+                                         _stream(lam.device)))
+    return h
+
+
+def filter_spectrum(h, fft_len: int) -> torch.Tensor:
+    """complex64 [H][fft_len/2+1]: DFT of each row of h zero-padded to fft_len."""
+    h = _cuda(h, "h", torch.float32)
+    H, L = h.shape
+    out = torch.empty((H, fft_len // 2 + 1, 2), dtype=torch.float32, device=h.device)
+    nbytes = lib().hyena_filter_spectrum_workspace_bytes(H, L, fft_len)
+    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=h.device)
+    _check("hyena_filter_spectrum",
+           lib().hyena_filter_spectrum(_ptr(h), H, L, fft_len, _ptr(out), _ptr(ws), nbytes,
+                                       _stream(h.device)))
+    return torch.view_as_complex(out)
+
+
+def prefill_workspace_bytes(B, L, Dch, H, d, fft_len) -> int:
+    return int(lib().hyena_prefill_workspace_bytes(B, L, Dch, H, d, fft_len))
+
+
+def prefill(q, k, v, lam, R, Dskip, fft_len: int, y=None, state=None, workspace=None):
+    """FFT prefill.  q,k,v [B][L][Dch] -> (y [B][L][Dch], state float32 [B][d][Dch][2])."""
+    lam, R, Dskip = _params(lam, R, Dskip)
+    q, k, v = _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v")
+    dt = _act_dtype(q)
+    B, L, Dch = q.shape
+    H, d = lam.shape[0], lam.shape[1]
+    if y is None:
+        y = torch.empty_like(q)
+    if state is None:
+        state = torch.empty((B, d, Dch, 2), dtype=torch.float32, device=q.device)
+    nbytes = prefill_workspace_bytes(B, L, Dch, H, d, fft_len)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    _check("hyena_prefill",
+           lib().hyena_prefill(_ptr(q), _ptr(k), _ptr(v), dt, B, L, Dch, H, d, fft_len,
+                               _ptr(lam), _ptr(R), _ptr(Dskip), _ptr(y), _ptr(state),
+                               _ptr(workspace), workspace.numel(), _stream(q.device)))
+    return y, state
+
+
+def prompt_state(k, v, lam, H: int, state=None):
+    """state float32 [B][d][Dch][2] = sum_j lam^(L-1-j) k_j v_j (standalone reduction)."""
+    lam = _cuda(lam, "lam", torch.float32)
+    k, v = _cuda(k, "k"), _cuda(v, "v")
+    dt = _act_dtype(k)
+    B, L, Dch = k.shape
+    d = lam.shape[1]
+    if state is None:
+        state = torch.empty((B, d, Dch, 2), dtype=torch.float32, device=k.device)
+    nbytes = int(lib().hyena_prompt_state_workspace_bytes(B, L, Dch, d))
+    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=k.device)
+    _check("hyena_prompt_state",
+           lib().hyena_prompt_state(_ptr(k), _ptr(v), dt, B, L, Dch, H, d, _ptr(lam), _ptr(state),
+                                    _ptr(ws), ws.numel(), _stream(k.device)))
+    return state
+
+
+def decode_step(q, k, v, lam, R, Dskip, state, y=None):
+    """One decode step: q,k,v [B][Dch]; state [B][d][Dch][2] updated in place; returns y."""
+    lam, R, Dskip = _params(lam, R, Dskip)
+    q, k, v = _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v")
+    state = _cuda(state, "state", torch.float32)
+    dt = _act_dtype(q)
+    B, Dch = q.shape
+    H, d = lam.shape[0], lam.shape[1]
+    if y is None:
+        y = torch.empty_like(q)
+    _check("hyena_decode_step",
+           lib().hyena_decode_step(_ptr(q), _ptr(k), _ptr(v), dt, B, Dch, H, d, _ptr(lam), _ptr(R),
+                                   _ptr(Dskip), _ptr(state), _ptr(y), _stream(q.device)))
+    return y

@@ -1,0 +1,173 @@
+/*
+ * hyena.h -- C ABI of libhyena_b200: the gated modal long convolution on B200.
+ *
+ * The operator (order-2 Hyena block; "Hyena processes long sequences 100x
+ * faster than FlashAttention", lequren.com, sections "Hyena層次結構" and
+ * "Hyena塊": a long convolution whose filter is as long as the input, between
+ * element-wise gates):
+ *
+ *     u_t = k_t * v_t,    z_t = sum_{j<=t} h_{t-j} u_j,    y_t = q_t * z_t
+ *
+ * with one filter per head shared by the head's Dch/H channels (weight tying,
+ * "Laughing Hyena Distillery", nubint.ai review, "Proposed method", and the
+ * abstract on the CoChat page), given in modal state-space form (the
+ * low-order SSM extracted from each convolution, same sources):
+ *
+ *     h_0 = Dskip,    h_j = Re sum_{n<d} R_n lambda_n^(j-1)   (j >= 1, |lambda_n| < 1)
+ *
+ * and its O(d)-state recurrent form for generation ("Main findings": O(d)
+ * memory and O(dK) time for K generated tokens):
+ *
+ *     y_t = q_t (Dskip u_t + Re sum_n R_n s_n),   then   s_n <- lambda_n s_n + u_t
+ *     prompt state:  s_n = sum_{j<L} lambda_n^(L-1-j) u_j
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Channel c belongs to head c / (Dch / H); Dch must be a multiple of H.
+ *  - Activations q, k, v, y: row-major [B][L][Dch] (prefill) or [B][Dch]
+ *    (decode), channel innermost, dtype HYENA_F32 (float) or HYENA_BF16
+ *    (bfloat16 bits).  All arithmetic is fp32; bf16 outputs are rounded to
+ *    nearest-even once, on store.
+ *  - Modal parameters (always fp32): lambda, R as [H][d][2] (re, im
+ *    interleaved complex64), Dskip as [H].
+ *  - Recurrent state: [B][d][Dch][2] complex64 (mode-major, channel
+ *    innermost, re/im interleaved), so that one mode of consecutive channels
+ *    is one contiguous run.
+ *  - Every pointer is DEVICE memory of the current CUDA device, owned by the
+ *    caller.  The library never allocates, frees or synchronises; work is
+ *    enqueued on `stream` (NULL = the legacy default stream) and returns
+ *    immediately.  Inputs must not alias outputs unless stated.
+ *  - Arguments are validated on the host before anything is enqueued; a
+ *    failed check returns a negative hyena_status and enqueues nothing.  A
+ *    launch failure returns HYENA_ERR_CUDA.  Not checked (would need a device
+ *    read): |lambda| < 1 and finiteness of the data.
+ *  - Empty problems (B == 0, Dch == 0, or L == 0 for the convolution) are
+ *    valid: nothing is read, and outputs that have no elements are left alone.
+ *    A prefill with L == 0 writes a zero state.
+ */
+#ifndef HYENA_B200_H
+#define HYENA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st *hyena_stream_t;
+
+typedef enum {
+    HYENA_OK = 0,
+    HYENA_ERR_ARG = -1,          /* NULL pointer, unknown dtype */
+    HYENA_ERR_SHAPE = -2,        /* negative size, Dch % H != 0, fft_len too short / not 2^k, d out of range */
+    HYENA_ERR_ALIGN = -3,        /* pointer not aligned as the layout requires */
+    HYENA_ERR_WORKSPACE = -4,    /* workspace NULL or smaller than the query says */
+    HYENA_ERR_UNSUPPORTED = -5,  /* valid operator, size outside what this build implements */
+    HYENA_ERR_CUDA = -6          /* a CUDA launch/runtime call failed */
+} hyena_status;
+
+typedef enum {
+    HYENA_F32 = 0,
+    HYENA_BF16 = 1
+} hyena_dtype;
+
+/* Largest number of poles per head the kernels accept. */
+#define HYENA_MAX_MODES 64
+
+/* Human-readable text for a hyena_status value (static storage, never NULL). */
+const char *hyena_status_string(int status);
+
+/* ABI version of this header: (major << 16) | minor. */
+int hyena_abi_version(void);
+
+/*
+ * Filter materialisation (modal form above; Laughing Hyena Distillery review,
+ * "Proposed method").
+ *   lambda, R : [H][d][2] fp32 device;  Dskip : [H] fp32 device
+ *   h_out     : [H][L] fp32 device, h_out[hd][0] = Dskip[hd],
+ *               h_out[hd][j] = Re sum_n R[hd][n] lambda[hd][n]^(j-1).
+ * Powers are formed in fp64 (binary powering of lambda, then a short run of
+ * multiplications), so lambda = 0 gives the 2-tap filter [Dskip, Re sum R].
+ * Requires H >= 0, 1 <= d <= HYENA_MAX_MODES, L >= 0.
+ */
+int hyena_filter_from_modes(const float *lambda, const float *R, const float *Dskip,
+                            int H, int d, int L, float *h_out, hyena_stream_t stream);
+
+/*
+ * Spectrum of each head's filter zero-padded to fft_len (the transform the
+ * FFT long convolution multiplies by; "Hyena層次結構": fast convolution
+ * without forming the full matrix):
+ *   spec_out[hd][f] = sum_{j<L} h[hd][j] exp(-2 pi i j f / fft_len),  f = 0..fft_len/2
+ *   h        : [H][L] fp32 device
+ *   spec_out : [H][fft_len/2+1][2] fp32 device (complex64)
+ * fft_len must be a power of two >= L; this build implements 64 <= fft_len
+ * <= 2^17 (HYENA_ERR_UNSUPPORTED otherwise).
+ * workspace: device scratch of hyena_filter_spectrum_workspace_bytes() bytes,
+ * 256-byte aligned.
+ */
+size_t hyena_filter_spectrum_workspace_bytes(int H, int L, int fft_len);
+int hyena_filter_spectrum(const float *h, int H, int L, int fft_len, float *spec_out,
+                          void *workspace, size_t ws_bytes, hyena_stream_t stream);
+
+/*
+ * Prefill by FFT long convolution: materialise the filter, transform it,
+ * convolve each channel's u = k*v causally through a zero-padded FFT of
+ * length fft_len, gate by q, and reduce the prompt to the recurrent state.
+ *   q, k, v, y : [B][L][Dch] activations (dtype), y written
+ *   state_out  : [B][d][Dch][2] fp32, overwritten with s_n = sum_j lambda_n^(L-1-j) u_j
+ *   fft_len    : power of two, >= 2L-1 (so the circular convolution equals the
+ *                linear one on the first L outputs).  Any such length gives the
+ *                same result up to rounding; lengths below 64 are raised to 64
+ *                internally.  This build implements fft_len <= 2^17, B <= 65535.
+ *                fft_len <= 16384 runs one fused kernel per channel pair with
+ *                the whole sequence in shared memory; longer transforms take a
+ *                four-step route through the workspace.
+ *   workspace  : device scratch, >= hyena_prefill_workspace_bytes(...) bytes,
+ *                256-byte aligned; contents on entry are ignored.
+ * Alignment: all activation pointers 4-byte aligned (bf16) / 8-byte (f32).
+ */
+size_t hyena_prefill_workspace_bytes(int B, int L, int Dch, int H, int d, int fft_len);
+int hyena_prefill(const void *q, const void *k, const void *v, int dtype,
+                  int B, int L, int Dch, int H, int d, int fft_len,
+                  const float *lambda, const float *R, const float *Dskip,
+                  void *y, float *state_out,
+                  void *workspace, size_t ws_bytes, hyena_stream_t stream);
+
+/*
+ * Prompt -> state reduction alone (the Vandermonde contraction over the
+ * prompt; "Main findings": the O(d) state that generation continues from):
+ *   state_out[b][n][c] = sum_{j<L} lambda[head(c)][n]^(L-1-j) k[b][j][c] v[b][j][c]
+ *   k, v      : [B][L][Dch] (dtype)
+ *   state_out : [B][d][Dch][2] fp32, overwritten (zero for L == 0).
+ *   workspace : device scratch, 256-byte aligned, of
+ *               hyena_prompt_state_workspace_bytes() bytes (partial states of
+ *               prompt segments, summed in a fixed order: deterministic).
+ */
+size_t hyena_prompt_state_workspace_bytes(int B, int L, int Dch, int d);
+int hyena_prompt_state(const void *k, const void *v, int dtype,
+                       int B, int L, int Dch, int H, int d,
+                       const float *lambda, float *state_out,
+                       void *workspace, size_t ws_bytes, hyena_stream_t stream);
+
+/*
+ * One O(1) decode step for a batch of sequences (one token per call):
+ *   y[b][c] = q[b][c] * (Dskip[h] u + Re sum_n R[h][n] s[b][n][c]),  u = k[b][c] v[b][c]
+ *   then    s[b][n][c] <- lambda[h][n] s[b][n][c] + u
+ * The output uses the state from before the update, so a prompt state from
+ * hyena_prefill followed by decode steps reproduces the full-length
+ * convolution.
+ *   q, k, v, y : [B][Dch] (dtype);  state : [B][d][Dch][2] fp32, updated in place.
+ * Alignment: state 8-byte aligned (16-byte for the vectorised path, taken when
+ * Dch is even and all pointers allow it).
+ */
+int hyena_decode_step(const void *q, const void *k, const void *v, int dtype,
+                      int B, int Dch, int H, int d,
+                      const float *lambda, const float *R, const float *Dskip,
+                      float *state, void *y, hyena_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HYENA_B200_H */

@@ -1,0 +1,134 @@
+"""C-ABI library checks that need no GPU.
+
+The library must load, export every function that include/hyena.h declares,
+and reject invalid arguments on the host (before any CUDA call) with the
+documented status codes.  Every call below fails validation, so nothing is
+enqueued and no CUDA context is created.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hyena.h")
+
+OK, ERR_ARG, ERR_SHAPE, ERR_ALIGN, ERR_WS, ERR_UNSUP, ERR_CUDA = 0, -1, -2, -3, -4, -5, -6
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from distilled_ssm_decode_b200 import build, ops
+    build.build()
+    return ops.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hyena_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("hyena_filter_from_modes", "hyena_prefill", "hyena_decode_step",
+                     "hyena_prefill_workspace_bytes", "hyena_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from distilled_ssm_decode_b200 import ops
+    out = subprocess.run(["nm", "-D", "--defined-only", ops.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (hyena_\w+)", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert hasattr(lib, n)
+
+
+def test_binding_signatures_cover_every_declared_symbol():
+    from distilled_ssm_decode_b200 import ops
+    assert set(declared_functions()) <= set(ops.SIGNATURES)
+
+
+def test_status_strings(lib):
+    for s in (OK, ERR_ARG, ERR_SHAPE, ERR_ALIGN, ERR_WS, ERR_UNSUP, ERR_CUDA, 12345):
+        assert lib.hyena_status_string(s)
+    assert lib.hyena_abi_version() >> 16 == 1
+
+
+FAKE = 1 << 40   # an aligned, never-dereferenced address: every call below fails validation first
+
+
+def _p(x=FAKE):
+    return ctypes.c_void_p(x)
+
+
+def prefill(lib, dtype=1, B=2, L=16, Dch=8, H=2, d=4, fft_len=32, ws=1 << 30, ptr=FAKE, wsptr=FAKE):
+    return lib.hyena_prefill(_p(ptr), _p(ptr), _p(ptr), dtype, B, L, Dch, H, d, fft_len, _p(ptr), _p(ptr),
+                             _p(ptr), _p(ptr), _p(ptr), _p(wsptr), ws, None)
+
+
+def test_prefill_validation(lib):
+    assert prefill(lib, dtype=7) == ERR_ARG
+    assert prefill(lib, Dch=9, H=2) == ERR_SHAPE          # Dch % H
+    assert prefill(lib, H=0) == ERR_SHAPE
+    assert prefill(lib, d=0) == ERR_SHAPE
+    assert prefill(lib, d=65) == ERR_SHAPE
+    assert prefill(lib, fft_len=24) == ERR_SHAPE          # not a power of two
+    assert prefill(lib, L=17, fft_len=32) == ERR_SHAPE    # < 2L-1
+    assert prefill(lib, B=-1) == ERR_SHAPE
+    assert prefill(lib, L=70000, fft_len=1 << 18) == ERR_UNSUP
+    assert prefill(lib, ws=0) == ERR_WS
+    assert prefill(lib, wsptr=FAKE + 8) == ERR_ALIGN       # workspace must be 256-byte aligned
+    assert prefill(lib, ptr=FAKE + 2) == ERR_ALIGN         # bf16 pairs need 4-byte alignment
+    assert prefill(lib, ptr=0) == ERR_ARG
+    # empty problems are valid and enqueue nothing
+    assert prefill(lib, B=0) == OK
+    assert prefill(lib, Dch=0) == OK
+
+
+def test_workspace_queries(lib):
+    assert lib.hyena_prefill_workspace_bytes(8, 4096, 1024, 8, 16, 8192) > 0
+    assert lib.hyena_prefill_workspace_bytes(8, 4096, 1024, 8, 16, 4096) == 0   # fft_len < 2L-1
+    four = lib.hyena_prefill_workspace_bytes(1, 65536, 768, 12, 16, 131072)
+    assert four >= 384 * 131072 * 8          # four-step planes for 384 channel pairs
+    assert lib.hyena_prompt_state_workspace_bytes(1, 65536, 768, 16) > 0
+    assert lib.hyena_filter_spectrum_workspace_bytes(4, 100, 256) >= 4 * 256 * 8
+
+
+def test_decode_validation(lib):
+    def call(dtype=1, B=4, Dch=8, H=2, d=4, ptr=FAKE, sptr=FAKE):
+        return lib.hyena_decode_step(_p(ptr), _p(ptr), _p(ptr), dtype, B, Dch, H, d, _p(ptr), _p(ptr),
+                                     _p(ptr), _p(sptr), _p(ptr), None)
+    assert call(dtype=3) == ERR_ARG
+    assert call(Dch=7, H=2) == ERR_SHAPE
+    assert call(d=0) == ERR_SHAPE
+    assert call(B=-2) == ERR_SHAPE
+    assert call(sptr=FAKE + 4) == ERR_ALIGN
+    assert call(ptr=0) == ERR_ARG
+    assert call(B=0) == OK
+
+
+def test_filter_and_state_validation(lib):
+    assert lib.hyena_filter_from_modes(_p(), _p(), _p(), 2, 0, 10, _p(), None) == ERR_SHAPE
+    assert lib.hyena_filter_from_modes(_p(), _p(), _p(), 2, 4, -1, _p(), None) == ERR_SHAPE
+    assert lib.hyena_filter_from_modes(_p(0), _p(), _p(), 2, 4, 10, _p(), None) == ERR_ARG
+    assert lib.hyena_filter_from_modes(_p(), _p(), _p(), 0, 4, 10, _p(), None) == OK
+    assert lib.hyena_filter_spectrum(_p(), 2, 10, 100, _p(), _p(), 1 << 20, None) == ERR_SHAPE
+    assert lib.hyena_filter_spectrum(_p(), 2, 10, 32, _p(), _p(), 1 << 20, None) == ERR_UNSUP
+    assert lib.hyena_filter_spectrum(_p(), 2, 10, 64, _p(), _p(), 0, None) == ERR_WS
+    assert lib.hyena_prompt_state(_p(), _p(), 1, 2, 10, 8, 3, 4, _p(), _p(), _p(), 1 << 20, None) == ERR_SHAPE
+    assert lib.hyena_prompt_state(_p(), _p(), 1, 2, 10, 8, 2, 4, _p(), _p(), _p(), 0, None) == ERR_WS
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    """The Python binding has no fallback: a missing library is an error, not a CPU path."""
+    from distilled_ssm_decode_b200 import ops
+    monkeypatch.setattr(ops, "_lib", None)
+    monkeypatch.setattr(ops, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        ops.lib()
