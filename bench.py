@@ -264,45 +264,66 @@ def run_ours(args):
     ops.lib()
 
     w = W.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.with_(B=args.batch)
+    has_pre, has_dec = w.L > 0, w.T > 0
     p = W.params(w)
     lam, R, D = p.lam_f32().to(dev), p.R_f32().to(dev), p.Dskip_f32().to(dev)
-    q_h, k_h, v_h = W.prefill_inputs(w)
-    dec_h = [W.decode_inputs(w, t) for t in range(w.T)]
-    dq_h = torch.stack([x[0] for x in dec_h])
-    dk_h = torch.stack([x[1] for x in dec_h])
-    dv_h = torch.stack([x[2] for x in dec_h])
-    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
-    dq, dk, dv = dq_h.to(dev), dk_h.to(dev), dv_h.to(dev)
-    y = torch.empty_like(q)
-    ydec = torch.empty_like(dq)
-    state = torch.empty((w.B, w.d, w.Dch, 2), dtype=torch.float32, device=dev)
-    ws = torch.empty(ops.prefill_workspace_bytes(w.B, w.L, w.Dch, w.H, w.d, w.fft_len),
-                     dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(dev)
+    state = torch.empty((w.B, w.d, w.Dch, 2), dtype=torch.float32, device=dev)
+
+    # ---- inputs (resident in HBM before the timed region)
+    host = {}
+    if has_pre:
+        host["q"], host["k"], host["v"] = W.prefill_inputs(w)
+        q, k, v = host["q"].to(dev), host["k"].to(dev), host["v"].to(dev)
+        y = torch.empty_like(q)
+        ws = torch.empty(ops.prefill_workspace_bytes(w.B, w.L, w.Dch, w.H, w.d, w.fft_len),
+                         dtype=torch.uint8, device=dev)
+    else:
+        state.copy_(torch.view_as_real(W.initial_state(w)).to(dev))
+    if has_dec:
+        pool = w.T if w.B * w.Dch * w.T <= (1 << 26) else 32
+        if pool == w.T:
+            dec = [W.decode_inputs(w, t) for t in range(w.T)]
+            host["dq"] = torch.stack([x[0] for x in dec])
+            host["dk"] = torch.stack([x[1] for x in dec])
+            host["dv"] = torch.stack([x[2] for x in dec])
+            dq, dk, dv = host["dq"].to(dev), host["dk"].to(dev), host["dv"].to(dev)
+        else:
+            dq, dk, dv = W.decode_pool_device(w, pool, device=dev)
+        ydec = torch.empty((w.T, w.B, w.Dch), dtype=w.torch_dtype, device=dev)
 
     def prefill():
         ops.prefill(q, k, v, lam, R, D, w.fft_len, y=y, state=state, workspace=ws)
 
     def decode_all():
         for t in range(w.T):
-            ops.decode_step(dq[t], dk[t], dv[t], lam, R, D, state, y=ydec[t])
+            i = t % dq.shape[0]
+            ops.decode_step(dq[i], dk[i], dv[i], lam, R, D, state, y=ydec[t])
 
+    g = None
     with torch.cuda.stream(stream):
-        prefill()
-        decode_all()
+        if has_pre:
+            prefill()
+        if has_dec:
+            decode_all()
     torch.cuda.synchronize(dev)
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        decode_all()
-    torch.cuda.synchronize(dev)
+    if has_dec:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            decode_all()
+        torch.cuda.synchronize(dev)
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        prefill()
+        if has_pre:
+            prefill()
         if ev is not None:
             ev[1].record(stream)
-        g.replay()
+        if has_dec:
+            g.replay()
         if ev is not None:
             ev[2].record(stream)
 
@@ -334,43 +355,54 @@ def run_ours(args):
 
     tokens_step = w.B * (w.L + w.T)
     value = world * tokens_step / (ms_per_step / 1e3)
-    pre_tok = world * w.B * w.L / (pre_ms / 1e3)
-    dec_tok = world * w.B * w.T / (dec_ms / 1e3)
     peak, peak_src = load_peaks()
     pb, db = algorithmic_bytes(w)
-    pre_gbs = pb / (pre_ms / 1e3) / 1e9
-    dec_launch_ms = dec_ms / max(w.T, 1)
-    dec_gbs = db / (dec_launch_ms / 1e3) / 1e9
-    roof_pre = {"kernel": "hyena_prefill (filter + spectrum + fused FFT conv/gate/state)",
-                "bound": "hbm", "achieved": pre_gbs, "peak": peak, "unit": "GB/s",
-                "frac": pre_gbs / peak, "peak_source": peak_src,
-                "algorithmic_bytes": pb, "launch_ms": pre_ms,
-                "traffic": ncu_traffic("prefill_fused", w.name)}
-    roof_dec = {"kernel": "hyena_decode_step", "bound": "hbm", "achieved": dec_gbs, "peak": peak,
-                "unit": "GB/s", "frac": dec_gbs / peak, "peak_source": peak_src,
-                "algorithmic_bytes": db, "launch_ms": dec_launch_ms,
-                "traffic": ncu_traffic("decode", w.name)}
-    dominant = roof_dec if dec_ms > pre_ms else roof_pre
+    roofs = []
+    out_pre = out_dec = None
+    if has_pre:
+        pre_gbs = pb / (pre_ms / 1e3) / 1e9
+        roofs.append({"kernel": "hyena_prefill (filter + spectrum + fused FFT conv/gate/state)",
+                      "bound": "hbm", "achieved": pre_gbs, "peak": peak, "unit": "GB/s",
+                      "frac": pre_gbs / peak, "peak_source": peak_src, "algorithmic_bytes": pb,
+                      "launch_ms": pre_ms, "total_ms": pre_ms,
+                      "traffic": ncu_traffic("prefill_fused", w.name)})
+        out_pre = {"tokens_per_s": world * w.B * w.L / (pre_ms / 1e3), "ms": pre_ms,
+                   "hbm_frac": pre_gbs / peak}
+    if has_dec:
+        dec_launch_ms = dec_ms / w.T
+        dec_gbs = db / (dec_launch_ms / 1e3) / 1e9
+        roofs.append({"kernel": "hyena_decode_step", "bound": "hbm", "achieved": dec_gbs,
+                      "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak,
+                      "peak_source": peak_src, "algorithmic_bytes": db,
+                      "launch_ms": dec_launch_ms, "total_ms": dec_ms,
+                      "traffic": ncu_traffic("decode", w.name)})
+        out_dec = {"tokens_per_s": world * w.B * w.T / (dec_ms / 1e3),
+                   "ms_per_token_step": dec_launch_ms, "hbm_frac": dec_gbs / peak}
+    dominant = max(roofs, key=lambda r: r["total_ms"])
 
     # ---- end to end: host (pinned) inputs, copies inside the timed region
     e2e = None
-    if not args.no_e2e:
-        pin = lambda t: t.pin_memory()  # noqa: E731
-        qp, kp, vp = pin(q_h), pin(k_h), pin(v_h)
-        dqp, dkp, dvp = pin(dq_h), pin(dk_h), pin(dv_h)
-        yp, ydp = torch.empty_like(qp).pin_memory(), torch.empty_like(dqp).pin_memory()
-        bi = sum(t.numel() * t.element_size() for t in (qp, kp, vp, dqp, dkp, dvp))
-        bo = yp.numel() * yp.element_size() + ydp.numel() * ydp.element_size()
+    if not args.no_e2e and all(x in host for x in ("q", "k", "v")) and \
+            (not has_dec or "dq" in host):
+        pins = {n: t.pin_memory() for n, t in host.items()}
+        dsts = {"q": q, "k": k, "v": v}
+        if has_dec:
+            dsts.update({"dq": dq, "dk": dk, "dv": dv})
+        yp = torch.empty_like(pins["q"]).pin_memory()
+        ydp = torch.empty(tuple(ydec.shape), dtype=ydec.dtype).pin_memory() if has_dec else None
+        bi = sum(t.numel() * t.element_size() for t in pins.values())
+        bo = yp.numel() * yp.element_size() + (ydp.numel() * ydp.element_size() if has_dec else 0)
 
         def e2e_step():
-            for dst, src in ((q, qp), (k, kp), (v, vp), (dq, dqp), (dk, dkp), (dv, dvp)):
-                dst.copy_(src, non_blocking=True)
+            for n, dst in dsts.items():
+                dst.copy_(pins[n], non_blocking=True)
             step()
             yp.copy_(y, non_blocking=True)
-            ydp.copy_(ydec, non_blocking=True)
+            if has_dec:
+                ydp.copy_(ydec, non_blocking=True)
 
         with torch.cuda.stream(stream):
-            for _ in range(max(1, min(args.warmup, 3))):
+            for _ in range(3):
                 e2e_step()
         torch.cuda.synchronize(dev)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -387,7 +419,7 @@ def run_ours(args):
 
     # ---- CPU baseline: the oracle on the host cores (rank 0, N = 1 only)
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and has_pre:
         import oracle
         oracle.build()
         sample = OracleSample(w)
@@ -400,19 +432,23 @@ def run_ours(args):
 
     if rank == 0:
         cfg = workload_config(w)
-        cfg["l2"] = ("prefill inputs larger than L2 (3 x %d MiB); decode state %.1f MiB stays "
-                     "L2-resident between steps, as in real decoding"
-                     % (q.numel() * q.element_size() >> 20, state.numel() * 4 / 2 ** 20))
+        if has_pre:
+            cfg["l2"] = ("prefill inputs larger than L2 (3 x %d MiB)"
+                         % (q.numel() * q.element_size() >> 20))
+        if has_dec:
+            st_mib = state.numel() * 4 / 2 ** 20
+            cfg["l2_decode"] = ("decode state %.1f MiB %s" % (
+                st_mib, "stays L2-resident between steps, as in real decoding" if st_mib < 100
+                else "is larger than L2"))
+            if dq.shape[0] != w.T:
+                cfg["decode_inputs"] = f"{dq.shape[0]} distinct device-drawn input sets, cycled"
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-                "data": "synthetic", "config": cfg,
-                "prefill": {"tokens_per_s": pre_tok, "ms": pre_ms, "hbm_frac": pre_gbs / peak},
-                "decode": {"tokens_per_s": dec_tok, "ms_per_token_step": dec_launch_ms,
-                           "hbm_frac": dec_gbs / peak},
-                "roofline": dominant, "roofline_all": [roof_pre, roof_dec],
+                "data": "synthetic", "config": cfg, "prefill": out_pre, "decode": out_dec,
+                "roofline": dominant, "roofline_all": roofs,
                 "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": args.steps * (3 + w.T), "clocks": clk}
+                "gpu_launches": args.steps * ((3 if has_pre else 0) + w.T), "clocks": clk}
         print(json.dumps(line), flush=True)
     del g
     import torch.distributed as dist
@@ -428,6 +464,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mid_bf16")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -69,4 +69,24 @@ __device__ __forceinline__ cd cdpow(cd lam, long long m) {
     return r;
 }
 
+// Number of trailing prompt tokens that the prompt -> state reduction needs:
+// with r = max_n |lambda_n| < 1, the tokens older than M contribute at most
+// max|u| * r^M / (1 - r) <= 2^-40 max|u| to any state entry (a geometric tail
+// far below fp32 resolution), so only the last M tokens are summed.
+// r == 0 gives M = 1 (lambda^0 = 1 is the only nonzero power); r >= 1 (outside
+// the stated |lambda| < 1 precondition) keeps the whole prompt.
+__device__ __forceinline__ int state_window(const float2 *lam_head, int d, int L) {
+    float r2 = 0.f;
+    for (int n = 0; n < d; ++n) {
+        const float2 l = lam_head[n];
+        r2 = fmaxf(r2, l.x * l.x + l.y * l.y);
+    }
+    if (r2 == 0.f) return L < 1 ? L : 1;
+    if (r2 >= 1.f) return L;
+    const double r = sqrt((double)r2);
+    const double m = (-40.0 * 0.69314718055994530942 + log1p(-r)) / log(r);
+    if (!(m < (double)L)) return L;
+    return (int)ceil(m) + 1;
+}
+
 }  // namespace hyena

@@ -12,8 +12,8 @@
 // writes d complex64 state entries, and writes y.  The vector kernel gives each
 // thread two adjacent channels, so one mode of the pair is one 16-byte load;
 // consecutive threads take consecutive pairs, so each mode row is read as
-// contiguous 128-byte lines.  All of a thread's modes are loaded before any
-// arithmetic so that up to 16 loads per thread are in flight.  When B * Dch is
+// contiguous 128-byte lines.  A thread's modes (up to 8 at a time) are loaded
+// before any arithmetic so that they are all in flight together.  When B * Dch is
 // small, NG threads share one pair (each takes every NG-th mode) and combine
 // their partial outputs with warp shuffles, so that small batches still put
 // enough loads in flight to cover memory latency.
@@ -25,9 +25,9 @@ namespace hyena {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kChunk = 16;   // modes per thread held in registers at once
 
-template <class Act>
+// MPT: modes held in registers per thread per iteration (all loaded before use).
+template <class Act, int MPT>
 __global__ void __launch_bounds__(kThreads)
 decode_vec_kernel(const typename Act::T *__restrict__ q, const typename Act::T *__restrict__ k,
                   const typename Act::T *__restrict__ v, int B, int Dch, int ch, int d, int lg_ng,
@@ -44,29 +44,30 @@ decode_vec_kernel(const typename Act::T *__restrict__ q, const typename Act::T *
     const int c = valid ? 2 * (int)(pair_id % pairs) : 0;
     const int hd = c / ch;
 
-    float ua = 0.f, ub = 0.f;
-    float2 qq = make_float2(0.f, 0.f);
-    if (valid) {
-        const size_t o = (size_t)b * Dch + c;
-        const float2 kk = Act::ld2(k + o), vv = Act::ld2(v + o);
-        qq = Act::ld2(q + o);
-        ua = kk.x * vv.x;
-        ub = kk.y * vv.y;
-    }
-    float acc_a = 0.f, acc_b = 0.f;
     const size_t srow = (size_t)Dch >> 1;                    // float4 per mode row
     float4 *sp = state + (size_t)b * d * srow + (c >> 1);
     const float2 *lh = lam + (size_t)hd * d;
     const float2 *rh = R + (size_t)hd * d;
-    for (int n0 = g; n0 < d; n0 += NG * kChunk) {
-        float4 s[kChunk];
+
+    float ua = 0.f, ub = 0.f;
+    float2 qq = make_float2(0.f, 0.f);
+    float acc_a = 0.f, acc_b = 0.f;
+    for (int n0 = g; n0 < d; n0 += NG * MPT) {
+        float4 s[MPT];
 #pragma unroll
-        for (int i = 0; i < kChunk; ++i) {
+        for (int i = 0; i < MPT; ++i) {
             const int n = n0 + i * NG;
             if (valid && n < d) s[i] = sp[(size_t)n * srow];
         }
+        if (n0 == g && valid) {   // activations: issued after the first state loads
+            const size_t o = (size_t)b * Dch + c;
+            const float2 kk = Act::ld2(k + o), vv = Act::ld2(v + o);
+            qq = Act::ld2(q + o);
+            ua = kk.x * vv.x;
+            ub = kk.y * vv.y;
+        }
 #pragma unroll
-        for (int i = 0; i < kChunk; ++i) {
+        for (int i = 0; i < MPT; ++i) {
             const int n = n0 + i * NG;
             if (valid && n < d) {
                 const float2 r = __ldg(&rh[n]);
@@ -118,11 +119,25 @@ decode_scalar_kernel(const typename Act::T *__restrict__ q, const typename Act::
     Act::st(y + o, Act::ld(q + o) * fmaf(__ldg(&Dskip[hd]), u, acc));
 }
 
-int choose_lg_ng(long long pairs, int d) {
+// Lanes per channel pair (NG) and modes per thread (MPT): enough threads to fill the GPU
+// (148 SMs x 2048), at most 16 lanes per pair, at most 8 modes in registers at once.
+void choose_split(long long pairs, int d, int *lg_ng, int *mpt) {
     const long long want = 148LL * 2048;
     int lg = 0;
     while ((pairs << lg) < want && (1 << (lg + 1)) <= 16 && (1 << (lg + 1)) <= d) ++lg;
-    return lg;
+    int per = (d + (1 << lg) - 1) >> lg;        // modes per lane
+    int m = 1;
+    while (m < per && m < 8) m <<= 1;
+    *lg_ng = lg;
+    *mpt = m;
+}
+
+template <class Act, int MPT>
+void launch_vec(unsigned blocks, cudaStream_t s, const typename Act::T *q, const typename Act::T *k,
+                const typename Act::T *v, int B, int Dch, int ch, int d, int lg, const float2 *lam,
+                const float2 *R, const float *Dskip, float *state, typename Act::T *y) {
+    decode_vec_kernel<Act, MPT><<<blocks, kThreads, 0, s>>>(q, k, v, B, Dch, ch, d, lg, lam, R, Dskip,
+                                                            reinterpret_cast<float4 *>(state), y);
 }
 
 template <class Act>
@@ -138,11 +153,16 @@ cudaError_t decode_launch(const void *q, const void *k, const void *v, int B, in
                        reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(y)) % (2 * Act::bytes) == 0);
     if (vec) {
         const long long pairs = (long long)B * (Dch / 2);
-        const int lg = choose_lg_ng(pairs, d);
+        int lg, mpt;
+        choose_split(pairs, d, &lg, &mpt);
         const long long threads = pairs << lg;
-        const long long blocks = (threads + kThreads - 1) / kThreads;
-        decode_vec_kernel<Act><<<(unsigned)blocks, kThreads, 0, s>>>(
-            qq, kk, vv, B, Dch, ch, d, lg, lam, R, Dskip, reinterpret_cast<float4 *>(state), yy);
+        const unsigned blocks = (unsigned)((threads + kThreads - 1) / kThreads);
+        switch (mpt) {
+            case 1: launch_vec<Act, 1>(blocks, s, qq, kk, vv, B, Dch, ch, d, lg, lam, R, Dskip, state, yy); break;
+            case 2: launch_vec<Act, 2>(blocks, s, qq, kk, vv, B, Dch, ch, d, lg, lam, R, Dskip, state, yy); break;
+            case 4: launch_vec<Act, 4>(blocks, s, qq, kk, vv, B, Dch, ch, d, lg, lam, R, Dskip, state, yy); break;
+            default: launch_vec<Act, 8>(blocks, s, qq, kk, vv, B, Dch, ch, d, lg, lam, R, Dskip, state, yy); break;
+        }
     } else {
         const long long threads = (long long)B * Dch;
         const long long blocks = (threads + kThreads - 1) / kThreads;

@@ -34,7 +34,8 @@ __device__ __forceinline__ int pad(int i) { return i + (i >> 4); }
 __host__ __device__ __forceinline__ int padded_len(int n) { return n + (n >> 4) + 1; }
 
 // exp(-2 pi i * num / den) for 0 <= num < den (den a power of two), fp32.
-__device__ __forceinline__ float2 expi_neg(long long num, long long den) {
+// The argument -2 num/den is exact in fp32 for den <= 2^24.
+__device__ __forceinline__ float2 expi_neg(int num, int den) {
     float s, c;
     sincospif(-2.0f * (float)num / (float)den, &s, &c);
     return make_float2(c, s);
@@ -135,7 +136,7 @@ __device__ __forceinline__ void dftR(float2 *x) {
 // w^k for k = 0..R-1 given the group's base angle num/den (w = exp(-2 pi i num/den)),
 // conjugated for the inverse.  Two accurate evaluations (w, w^4), the rest by products.
 template <int R, bool INV>
-__device__ __forceinline__ void twiddles(float2 *tw, long long num, long long den) {
+__device__ __forceinline__ void twiddles(float2 *tw, int num, int den) {
     float2 w1 = expi_neg(num, den);
     tw[0] = make_float2(1.f, 0.f);
     if constexpr (R >= 2) tw[1] = w1;
@@ -145,7 +146,7 @@ __device__ __forceinline__ void twiddles(float2 *tw, long long num, long long de
         tw[3] = cmul(w2, w1);
     }
     if constexpr (R >= 8) {
-        float2 w4 = expi_neg((num * 4) % den, den);
+        float2 w4 = expi_neg(num * 4, den);     // num < den / R, so 4 num < den
 #pragma unroll
         for (int k = 4; k < R; ++k) {
             float2 base = (k >= 12) ? cmul(cmul(w4, w4), w4) : (k >= 8 ? cmul(w4, w4) : w4);
@@ -165,11 +166,12 @@ __device__ __forceinline__ void twiddles(float2 *tw, long long num, long long de
 // the upper half zero).
 template <int R, bool HALF_IN>
 __device__ __forceinline__ void fwd_pass(float2 *buf, int N, int M, int tid, int nthr) {
-    const int s = M / R;
+    const int s = M / R;               // powers of two: index math by shifts and masks
+    const int lgs = __ffs(s) - 1;
     const int groups = N / R;
     for (int gi = tid; gi < groups; gi += nthr) {
-        const int i = gi % s;          // s is a power of two
-        const int base = (gi / s) * M + i;
+        const int i = gi & (s - 1);
+        const int base = ((gi >> lgs) * M) + i;
         float2 x[R];
 #pragma unroll
         for (int k = 0; k < R; ++k) {
@@ -194,10 +196,11 @@ __device__ __forceinline__ void fwd_pass(float2 *buf, int N, int M, int tid, int
 template <int R>
 __device__ __forceinline__ void inv_pass(float2 *buf, int N, int M, int tid, int nthr, int out_limit) {
     const int s = M / R;
+    const int lgs = __ffs(s) - 1;
     const int groups = N / R;
     for (int gi = tid; gi < groups; gi += nthr) {
-        const int i = gi % s;
-        const int base = (gi / s) * M + i;
+        const int i = gi & (s - 1);
+        const int base = ((gi >> lgs) * M) + i;
         float2 x[R];
 #pragma unroll
         for (int k = 0; k < R; ++k) x[k] = buf[pad(base + k * s)];

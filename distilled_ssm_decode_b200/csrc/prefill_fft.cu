@@ -32,10 +32,11 @@ using fft::padded_len;
 
 namespace {
 
-constexpr int kFusedThreads = 512;
+constexpr int kFusedThreads = 256;
+constexpr int kFusedMinBlocks = 3;   // three CTAs per SM: one loads while others compute
 
 int fused_threads(int N) {
-    int t = N / 16;
+    int t = N / 32;
     if (t < 64) t = 64;
     if (t > kFusedThreads) t = kFusedThreads;
     return t;
@@ -79,7 +80,7 @@ __global__ void spectrum_natural_kernel(const float2 *__restrict__ spec_perm, in
 // ------------------------------------------------------------------ fused prefill
 // grid (slots, B); slot = channel pair (paired) or single channel.
 template <class Act>
-__global__ void __launch_bounds__(kFusedThreads)
+__global__ void __launch_bounds__(kFusedThreads, kFusedMinBlocks)
 prefill_fused_kernel(const typename Act::T *__restrict__ q, const typename Act::T *__restrict__ k,
                      const typename Act::T *__restrict__ v, int L, int Dch, int ch, int d, int N,
                      int paired, const float2 *__restrict__ spec_perm,
@@ -93,32 +94,43 @@ prefill_fused_kernel(const typename Act::T *__restrict__ q, const typename Act::
     const int b = blockIdx.y;
     const int c0 = paired ? 2 * blockIdx.x : blockIdx.x;
     const int hd = c0 / ch;
-    const size_t rowbase = (size_t)b * L * Dch + c0;
+    const typename Act::T *kb = k + (size_t)b * L * Dch + c0;
+    const typename Act::T *vb = v + (size_t)b * L * Dch + c0;
 
-    // 1. gate-in: x_t = (k_a v_a, k_b v_b), zero padding up to N/2
-    for (int t = tid; t < N / 2; t += nthr) {
-        float2 x = make_float2(0.f, 0.f);
-        if (t < L) {
-            const size_t o = rowbase + (size_t)t * Dch;
-            if (paired) {
-                const float2 kk = Act::ld2(k + o), vv = Act::ld2(v + o);
-                x = make_float2(kk.x * vv.x, kk.y * vv.y);
-            } else {
-                x.x = Act::ld(k + o) * Act::ld(v + o);
+    // 1. gate-in: x_t = (k_a v_a, k_b v_b), zero padding up to N/2; four rows per
+    //    thread are loaded before any is used so that their latencies overlap
+    constexpr int U = 4;
+    for (int t0 = tid; t0 < N / 2; t0 += U * nthr) {
+        float2 kk[U], vv[U];
+#pragma unroll
+        for (int r = 0; r < U; ++r) {
+            const int t = t0 + r * nthr;
+            kk[r] = vv[r] = make_float2(0.f, 0.f);
+            if (t < L) {
+                const size_t o = (size_t)t * Dch;
+                if (paired) { kk[r] = Act::ld2(kb + o); vv[r] = Act::ld2(vb + o); }
+                else { kk[r].x = Act::ld(kb + o); vv[r].x = Act::ld(vb + o); }
             }
         }
-        buf[pad(t)] = x;
+#pragma unroll
+        for (int r = 0; r < U; ++r) {
+            const int t = t0 + r * nthr;
+            if (t < N / 2) buf[pad(t)] = make_float2(kk[r].x * vv[r].x, kk[r].y * vv[r].y);
+        }
     }
     __syncthreads();
 
-    // 2. prompt -> state: s_n = sum_j lambda_n^(L-1-j) x_j, by segments of the prompt.
-    //    Horner inside a segment, then scaled by lambda^(L - segment end) (fp64 power).
+    // 2. prompt -> state: s_n = sum_j lambda_n^(L-1-j) x_j over the last W tokens
+    //    (older ones weigh < 2^-40 max|u|), by segments: Horner inside a segment,
+    //    then scaled by lambda^(L - segment end) (fp64 power), segments summed in order.
+    const float2 *lh = lam + (size_t)hd * d;
+    const int jstart = L - state_window(lh, d, L);
     const int nseg = max(1, nthr / d);
-    const int seglen = (L + nseg - 1) / nseg;
+    const int seglen = (L - jstart + nseg - 1) / nseg;
     for (int w = tid; w < d * nseg; w += nthr) {
         const int n = w % d, g = w / d;
-        const float2 l = __ldg(&lam[(size_t)hd * d + n]);
-        const int j0 = g * seglen;
+        const float2 l = __ldg(&lh[n]);
+        const int j0 = jstart + g * seglen;
         const int j1 = min(L, j0 + seglen);
         float2 aa = make_float2(0.f, 0.f), ab = make_float2(0.f, 0.f);
         for (int j = j0; j < j1; ++j) {
@@ -142,8 +154,8 @@ prefill_fused_kernel(const typename Act::T *__restrict__ q, const typename Act::
             s.x += p.x; s.y += p.y; s.z += p.z; s.w += p.w;
         }
         float *so = state_out + (((size_t)b * d + n) * Dch + c0) * 2;
-        so[0] = s.x; so[1] = s.y;
-        if (paired) { so[2] = s.z; so[3] = s.w; }
+        *reinterpret_cast<float2 *>(so) = make_float2(s.x, s.y);   // state is 8-byte aligned
+        if (paired) *reinterpret_cast<float2 *>(so + 2) = make_float2(s.z, s.w);
     }
 
     // 3. forward transform, product with the head's spectrum (scaled by 1/N), inverse
@@ -154,14 +166,27 @@ prefill_fused_kernel(const typename Act::T *__restrict__ q, const typename Act::
     fft::inverse(buf, N, L);
 
     // 4. gate-out and store the first L outputs
-    for (int t = tid; t < L; t += nthr) {
-        const size_t o = rowbase + (size_t)t * Dch;
-        const float2 z = buf[pad(t)];
-        if (paired) {
-            const float2 qq = Act::ld2(q + o);
-            Act::st2(y + o, qq.x * z.x, qq.y * z.y);
-        } else {
-            Act::st(y + o, Act::ld(q + o) * z.x);
+    const typename Act::T *qb = q + (size_t)b * L * Dch + c0;
+    typename Act::T *yb = y + (size_t)b * L * Dch + c0;
+    for (int t0 = tid; t0 < L; t0 += U * nthr) {
+        float2 qq[U];
+#pragma unroll
+        for (int r = 0; r < U; ++r) {
+            const int t = t0 + r * nthr;
+            qq[r] = make_float2(0.f, 0.f);
+            if (t < L) {
+                if (paired) qq[r] = Act::ld2(qb + (size_t)t * Dch);
+                else qq[r].x = Act::ld(qb + (size_t)t * Dch);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < U; ++r) {
+            const int t = t0 + r * nthr;
+            if (t < L) {
+                const float2 z = buf[pad(t)];
+                if (paired) Act::st2(yb + (size_t)t * Dch, qq[r].x * z.x, qq[r].y * z.y);
+                else Act::st(yb + (size_t)t * Dch, qq[r].x * z.x);
+            }
         }
     }
 }
@@ -208,7 +233,7 @@ fourstep_fwd1_kernel(Src src, int N2, float2 *__restrict__ Y) {
     float2 *out = Y + (size_t)col * N + n2;
 #pragma unroll
     for (int k1 = 0; k1 < N1; ++k1) {
-        const float2 w = fft::expi_neg((long long)n2 * k1, N);
+        const float2 w = fft::expi_neg(n2 * k1, (int)N);
         out[(size_t)k1 * N2] = k1 ? cmul(x[k1], w) : x[k1];
     }
 }
@@ -252,7 +277,7 @@ fourstep_inv1_kernel(const float2 *__restrict__ Y, int N2, int L, int Dch, int n
     float2 x[N1];
 #pragma unroll
     for (int k1 = 0; k1 < N1; ++k1) {
-        const float2 w = fft::expi_neg((long long)n2 * k1, N);
+        const float2 w = fft::expi_neg(n2 * k1, (int)N);
         x[k1] = k1 ? cmulc(in[(size_t)k1 * N2], w) : in[0];
     }
     fft::dftR<N1, true>(x);

@@ -5,8 +5,10 @@
 // after a prompt ("Laughing Hyena Distillery", nubint.ai review, "Main
 // findings"; the recurrence is the modal SSM of "Proposed method").
 //
-// Kernel 1: one thread per (batch, channel, prompt segment) runs Horner's rule
-// over its segment for every mode (acc <- acc * lambda + u), then scales by
+// Only the last W tokens of the prompt are summed, W chosen per head so that
+// the older ones weigh at most 2^-40 max|u| (state_window in common.cuh).
+// Kernel 1: one thread per (batch, channel, segment of that window) runs Horner's
+// rule over its segment for every mode (acc <- acc * lambda + u), then scales by
 // lambda^(L - segment end) (fp64 binary powering) and writes a partial state.
 // Kernel 2 adds the partials of each (b, n, c) in segment order, so the result
 // does not depend on scheduling.  Consecutive threads take consecutive
@@ -34,13 +36,17 @@ int choose_nseg(int B, int L, int Dch) {
 template <class Act>
 __global__ void __launch_bounds__(kThreads)
 state_partial_kernel(const typename Act::T *__restrict__ k, const typename Act::T *__restrict__ v,
-                     int L, int Dch, int ch, int d, int seglen, const float2 *__restrict__ lam,
+                     int L, int Dch, int ch, int d, const float2 *__restrict__ lam,
                      float2 *__restrict__ part /* [B][nseg][d][Dch] */) {
     const int c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= Dch) return;
     const int g = blockIdx.y, b = blockIdx.z, nseg = gridDim.y;
     const int hd = c / ch;
-    const int j0 = g * seglen, j1 = min(L, j0 + seglen);
+    // the nseg segments cover this head's window [L - W, L)
+    const int W = state_window(lam + (size_t)hd * d, d, L);
+    const int jstart = L - W;
+    const int segw = (W + nseg - 1) / nseg;
+    const int j0 = jstart + g * segw, j1 = min(L, j0 + segw);
     for (int n0 = 0; n0 < d; n0 += kModeChunk) {
         float2 l[kModeChunk], a[kModeChunk];
 #pragma unroll
@@ -94,17 +100,15 @@ cudaError_t launch_prompt_state(const void *k, const void *v, int dtype, int B, 
     if (L == 0) return cudaMemsetAsync(state_out, 0, (size_t)B * d * Dch * 2 * sizeof(float), s);
     const int ch = Dch / H;
     const int nseg = choose_nseg(B, L, Dch);
-    const int seglen = (L + nseg - 1) / nseg;
     float2 *part = static_cast<float2 *>(scratch);
     dim3 grid((Dch + kThreads - 1) / kThreads, nseg, B);
     if (dtype == HYENA_BF16)
         state_partial_kernel<ActBF16><<<grid, kThreads, 0, s>>>(
             static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v), L, Dch, ch,
-            d, seglen, lam, part);
+            d, lam, part);
     else
         state_partial_kernel<ActF32><<<grid, kThreads, 0, s>>>(
-            static_cast<const float *>(k), static_cast<const float *>(v), L, Dch, ch, d, seglen, lam,
-            part);
+            static_cast<const float *>(k), static_cast<const float *>(v), L, Dch, ch, d, lam, part);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     dim3 g2((Dch + 255) / 256, d, B);

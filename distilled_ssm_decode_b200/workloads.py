@@ -158,6 +158,21 @@ def initial_state(w: Workload, B: Optional[int] = None, Dch: Optional[int] = Non
     return torch.view_as_complex(torch.from_numpy(np.ascontiguousarray(x)))
 
 
+def decode_pool_device(w: Workload, pool: int, B: Optional[int] = None, device="cuda",
+                       layer: int = 0):
+    """`pool` distinct decode-step inputs (q, k, v), each [pool][B][Dch], drawn N(0, 1) on
+    the device by torch's seeded generator.  For benchmarking large batches, where drawing
+    every step on the host would take minutes; parity tests use decode_inputs()."""
+    B = w.B if B is None else B
+    g = torch.Generator(device=device)
+    out = []
+    for tid in (T_DQ, T_DK, T_DV):
+        g.manual_seed(_seed(w, layer, tid))
+        x = torch.randn((pool, B, w.Dch), generator=g, device=device, dtype=torch.float32)
+        out.append(x.to(w.torch_dtype))
+    return tuple(out)
+
+
 def to_f64(t: torch.Tensor) -> np.ndarray:
     """Exact widening of a CPU tensor (fp32 / bf16 / complex64) to numpy float64/complex128."""
     if t.is_complex():

@@ -117,6 +117,9 @@ int hyena_filter_spectrum(const float *h, int H, int L, int fft_len, float *spec
  * length fft_len, gate by q, and reduce the prompt to the recurrent state.
  *   q, k, v, y : [B][L][Dch] activations (dtype), y written
  *   state_out  : [B][d][Dch][2] fp32, overwritten with s_n = sum_j lambda_n^(L-1-j) u_j
+ *                (summed over the last W tokens, W chosen per head from
+ *                r = max|lambda| so that the older tokens weigh at most
+ *                r^W/(1-r) max|u| <= 2^-40 max|u|, far below fp32 resolution)
  *   fft_len    : power of two, >= 2L-1 (so the circular convolution equals the
  *                linear one on the first L outputs).  Any such length gives the
  *                same result up to rounding; lengths below 64 are raised to 64
@@ -140,7 +143,8 @@ int hyena_prefill(const void *q, const void *k, const void *v, int dtype,
  * prompt; "Main findings": the O(d) state that generation continues from):
  *   state_out[b][n][c] = sum_{j<L} lambda[head(c)][n]^(L-1-j) k[b][j][c] v[b][j][c]
  *   k, v      : [B][L][Dch] (dtype)
- *   state_out : [B][d][Dch][2] fp32, overwritten (zero for L == 0).
+ *   state_out : [B][d][Dch][2] fp32, overwritten (zero for L == 0); the same
+ *               trailing-window rule as hyena_prefill applies.
  *   workspace : device scratch, 256-byte aligned, of
  *               hyena_prompt_state_workspace_bytes() bytes (partial states of
  *               prompt segments, summed in a fixed order: deterministic).

@@ -62,7 +62,7 @@ def test_filter_zero_pole_is_two_tap(oracle):
 @pytest.mark.parametrize("name,L,N,bins", [("tiny_f32", 256, 512, None),
                                            ("mid_bf16", 4096, 8192, 64),
                                            ("long_prefill_bf16", 65536, 131072, 64),
-                                           ("tiny_f32", 100, 64, None)])
+                                           ("tiny_f32", 50, 64, None)])
 def test_spectrum_parity(oracle, name, L, N, bins):
     w = W.WORKLOADS[name]
     p = W.params(w)
