@@ -250,6 +250,7 @@ def workload_config(w):
             "decode_steps": w.T, "activations": w.dtype, "parallelism": "data-parallel replicas"}
 
 
+
 # ------------------------------------------------------------------ our arm
 def run_ours(args):
     import torch
@@ -267,6 +268,10 @@ def run_ours(args):
     if args.batch:
         w = w.with_(B=args.batch)
     has_pre, has_dec = w.L > 0, w.T > 0
+    use_chunked = has_pre and args.prefill != "fft" and ops.lib().hyena_prefill_chunked_workspace_bytes(
+        w.B, w.L, w.Dch, w.H, w.d) > 0
+    if args.prefill == "chunked" and not use_chunked:
+        raise SystemExit(f"chunked prefill does not support workload {w.name}")
     p = W.params(w)
     lam, R, D = p.lam_f32().to(dev), p.R_f32().to(dev), p.Dskip_f32().to(dev)
     stream = torch.cuda.Stream(dev)
@@ -280,6 +285,9 @@ def run_ours(args):
         y = torch.empty_like(q)
         ws = torch.empty(ops.prefill_workspace_bytes(w.B, w.L, w.Dch, w.H, w.d, w.fft_len),
                          dtype=torch.uint8, device=dev)
+        if use_chunked:
+            ws_c = torch.empty(ops.prefill_chunked_workspace_bytes(w.B, w.L, w.Dch, w.H, w.d),
+                               dtype=torch.uint8, device=dev)
     else:
         state.copy_(torch.view_as_real(W.initial_state(w)).to(dev))
     if has_dec:
@@ -294,8 +302,13 @@ def run_ours(args):
             dq, dk, dv = W.decode_pool_device(w, pool, device=dev)
         ydec = torch.empty((w.T, w.B, w.Dch), dtype=w.torch_dtype, device=dev)
 
-    def prefill():
+    def prefill_fft():
         ops.prefill(q, k, v, lam, R, D, w.fft_len, y=y, state=state, workspace=ws)
+
+    def prefill_chunked():
+        ops.prefill_chunked(q, k, v, lam, R, D, y=y, state=state, workspace=ws_c)
+
+    prefill = prefill_chunked if use_chunked else prefill_fft
 
     def decode_all():
         for t in range(w.T):
@@ -378,6 +391,30 @@ def run_ours(args):
                       "traffic": ncu_traffic("decode", w.name)})
         out_dec = {"tokens_per_s": world * w.B * w.T / (dec_ms / 1e3),
                    "ms_per_token_step": dec_launch_ms, "hbm_frac": dec_gbs / peak}
+    if use_chunked:
+        roofs[0]["kernel"] = "hyena_prefill_chunked (tcgen05 chunked conv/gate/state)"
+        roofs[0]["traffic"] = ncu_traffic("prefill_chunk", w.name)
+        err = ops.chunked_error(ws_c, w.B, w.L, w.Dch, w.H, w.d)
+        if err:
+            raise SystemExit(f"chunked prefill kernel reported error {err}")
+    # the FFT route (zero-padded FFT long convolution) timed on the same inputs
+    fft_route = None
+    if has_pre and use_chunked and not args.no_fft_route:
+        fe = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                prefill_fft()
+            fe[0].record(stream)
+            for _ in range(args.steps):
+                prefill_fft()
+            fe[1].record(stream)
+        torch.cuda.synchronize(dev)
+        fms = reduce_max(fe[0].elapsed_time(fe[1]) / args.steps, dev)
+        fgbs = pb / (fms / 1e3) / 1e9
+        fft_route = {"kernel": "hyena_prefill (filter + spectrum + fused FFT conv/gate/state)",
+                     "fft_len": w.fft_len, "tokens_per_s": world * w.B * w.L / (fms / 1e3),
+                     "ms": fms, "achieved": fgbs, "frac": fgbs / peak, "unit": "GB/s",
+                     "traffic": ncu_traffic("prefill_fused", w.name)}
     dominant = max(roofs, key=lambda r: r["total_ms"])
 
     # ---- end to end: host (pinned) inputs, copies inside the timed region
@@ -430,9 +467,13 @@ def run_ours(args):
                           f"{channels} of {w.Dch} channels ({w.L}-token prompt + {w.T} decode "
                           f"tokens); {dt:.1f} s")}
 
+    # our kernels per step: chunked = constants + main; FFT = filter + spectrum + fused
+    # (four-step FFT beyond 16384 points: filter, 2 spectrum, 3 convolution, 2 state kernels)
+    pre_launches = 0 if not has_pre else (2 if use_chunked else (3 if w.fft_len <= 16384 else 8))
     if rank == 0:
         cfg = workload_config(w)
         if has_pre:
+            cfg["prefill_route"] = "chunked" if use_chunked else "fft"
             cfg["l2"] = ("prefill inputs larger than L2 (3 x %d MiB)"
                          % (q.numel() * q.element_size() >> 20))
         if has_dec:
@@ -446,9 +487,10 @@ def run_ours(args):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic", "config": cfg, "prefill": out_pre, "decode": out_dec,
+                "prefill_fft_route": fft_route,
                 "roofline": dominant, "roofline_all": roofs,
                 "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": args.steps * ((3 if has_pre else 0) + w.T), "clocks": clk}
+                "gpu_launches": args.steps * (pre_launches + w.T), "clocks": clk}
         print(json.dumps(line), flush=True)
     del g
     import torch.distributed as dist
@@ -465,6 +507,10 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mid_bf16")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size")
+    ap.add_argument("--prefill", choices=["auto", "chunked", "fft"], default="auto",
+                    help="prefill route: chunked tensor-core evaluation (auto when supported) or FFT")
+    ap.add_argument("--no-fft-route", action="store_true",
+                    help="skip the extra timing of the FFT route when the chunked route is used")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -150,6 +150,46 @@ int hyena_prefill(const void *q, const void *k, const void *v, int dtype, int B,
     return cuda_status(e);
 }
 
+static int check_chunked(int dtype, int B, int L, int Dch, int H, int d) {
+    if (dtype != HYENA_F32 && dtype != HYENA_BF16) return HYENA_ERR_ARG;
+    if (B < 0 || L < 0) return HYENA_ERR_SHAPE;
+    int st = check_common(H, d, Dch);
+    if (st != HYENA_OK) return st;
+    if (B > 65535 || !chunked_supported(dtype, Dch, H, d)) return HYENA_ERR_UNSUPPORTED;
+    return HYENA_OK;
+}
+
+size_t hyena_prefill_chunked_workspace_bytes(int B, int L, int Dch, int H, int d) {
+    if (check_chunked(HYENA_BF16, B, L, Dch, H, d) != HYENA_OK) return 0;
+    return chunked_ws_bytes(B, L, Dch, H, d);
+}
+
+size_t hyena_prefill_chunked_error_offset(int B, int L, int Dch, int H, int d) {
+    if (check_chunked(HYENA_BF16, B, L, Dch, H, d) != HYENA_OK) return 0;
+    return (size_t)chunked_error_offset(B, L, Dch, H, d);
+}
+
+int hyena_prefill_chunked(const void *q, const void *k, const void *v, int dtype, int B, int L, int Dch,
+                          int H, int d, const float *lambda, const float *R, const float *Dskip, void *y,
+                          float *state_out, void *workspace, size_t ws_bytes, hyena_stream_t stream) {
+    int st = check_chunked(dtype, B, L, Dch, H, d);
+    if (st != HYENA_OK) return st;
+    if (B == 0 || Dch == 0) return HYENA_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (!state_out || !lambda || !R || !Dskip) return HYENA_ERR_ARG;
+    if (!aligned(state_out, 8) || !aligned(lambda, 8) || !aligned(R, 8) || !aligned(Dskip, 4))
+        return HYENA_ERR_ALIGN;
+    if (L == 0)
+        return cuda_status(cudaMemsetAsync(state_out, 0, (size_t)B * d * Dch * 2 * sizeof(float), s));
+    if (!q || !k || !v || !y || !workspace) return HYENA_ERR_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(y, 16) || !aligned(workspace, kAlign))
+        return HYENA_ERR_ALIGN;
+    if (ws_bytes < chunked_ws_bytes(B, L, Dch, H, d)) return HYENA_ERR_WORKSPACE;
+    return cuda_status(launch_prefill_chunked(q, k, v, B, L, Dch, H, d, reinterpret_cast<const float2 *>(lambda),
+                                              reinterpret_cast<const float2 *>(R), Dskip, y, state_out,
+                                              workspace, s));
+}
+
 size_t hyena_prompt_state_workspace_bytes(int B, int L, int Dch, int d) {
     if (B < 0 || L < 0 || Dch < 0 || d < 1 || d > HYENA_MAX_MODES) return 0;
     return align_up(state_ws_bytes(B, L, Dch, d));

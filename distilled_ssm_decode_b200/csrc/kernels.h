@@ -35,6 +35,14 @@ cudaError_t launch_prefill_fft(const void *q, const void *k, const void *v, int 
                                void *y, float *state_out, void *scratch, size_t scratch_bytes,
                                cudaStream_t s);
 
+// prefill_chunked.cu (bf16 activations, heads of a multiple of 128 channels, d <= 16)
+bool chunked_supported(int dtype, int Dch, int H, int d);
+size_t chunked_ws_bytes(int B, int L, int Dch, int H, int d);
+int chunked_error_offset(int B, int L, int Dch, int H, int d);
+cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, int B, int L, int Dch,
+                                   int H, int d, const float2 *lam, const float2 *R, const float *Dskip,
+                                   void *y, float *state_out, void *ws, cudaStream_t s);
+
 // state.cu
 size_t state_ws_bytes(int B, int L, int Dch, int d);
 cudaError_t launch_prompt_state(const void *k, const void *v, int dtype, int B, int L, int Dch,

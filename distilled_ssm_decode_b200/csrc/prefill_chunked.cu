@@ -1,0 +1,669 @@
+// prefill_chunked.cu -- chunked modal prefill on tcgen05 tensor cores.
+//
+// The long convolution y = q * (h conv (k * v)) ("Hyena processes long
+// sequences 100x faster than FlashAttention", lequren.com, "Hyena層次結構")
+// with the modal filter h_0 = Dskip, h_j = Re sum_n R_n lambda_n^(j-1) of
+// "Laughing Hyena Distillery" (nubint.ai review, "Proposed method") is
+// evaluated chunk by chunk.  For a chunk of C tokens starting at c0, with
+// tau, iota in [0, C):
+//
+//   z[c0+tau] = sum_{iota<=tau} h_{tau-iota} u[c0+iota]            (intra-chunk Toeplitz)
+//             + Re sum_n R_n lambda_n^tau s_n(c0)                  (modal carry from the past)
+//   s_n(c0+C) = lambda_n^C s_n(c0) + sum_iota lambda_n^(C-1-iota) u[c0+iota]
+//
+// where s(c0) is the recurrent state after c0 tokens -- the same O(d) state the
+// decode step advances ("Main findings": O(d) memory per channel).  This is an
+// exact regrouping of the causal convolution (the carry term is the tail of the
+// sum over j < c0 with h_{t-j} = Re sum R lambda^(t-c0) lambda^(c0-1-j)), and
+// the prompt -> state reduction falls out as the last carry.
+//
+// Per chunk and 128-channel tile (one head, M = 128 = channels on the MMA
+// rows), three products run on the tensor cores in tf32 with fp32 accumulation
+// in tensor memory:
+//   D1[c][tau] = sum_iota U[c][iota] T[tau][iota]  +  sum_r S[c][r] A[tau][r]
+//   D2[c][r]   = sum_iota U[c][iota] V[r][iota]
+// with T[tau][iota] = h_{tau-iota} (iota <= tau), A = (Re, -Im) of R lambda^tau,
+// V = (Re, Im) of lambda^(C-1-iota), S = (Re, Im) of the state.  The chunk's
+// state update S <- lambda^C S + D2 runs on the CUDA cores in fp32 registers
+// (one thread per channel, the thread that owns TMEM lane c), and
+// y = q * D1 is gated and stored by the same thread.
+//
+// Work split: a sequence is cut into segments of whole chunks; each
+// (batch, channel tile, segment) item first runs a state-only pass (k, v and
+// the D2 product) to publish its segment's state contribution, then obtains the
+// state entering its segment by a decoupled look-back over its predecessors'
+// published contributions (bounded polls), then runs the full pass.  Items are
+// handed out by an atomic ticket in launch order, so an item only ever waits on
+// items already running; the state-only pass never waits, so the look-back
+// always ends.  k and v are read twice per item, the second time mostly from L2.
+//
+// Roles in a 192-thread CTA: warps 0-3 (one thread per channel) compute
+// u = k*v, the state and the gated output; warp 4 issues the TMA loads; warp 5
+// owns tensor memory and issues the MMAs.  Every wait is bounded; on timeout
+// the kernel records an error code, drains its copies and MMAs, frees tensor
+// memory and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace hyena {
+
+namespace {
+
+constexpr int kC = 64;             // tokens per chunk
+constexpr int kNC = 128;           // channels per tile (MMA M)
+constexpr int kMaxModes = 16;      // d <= 16 (KS = 2d rounded up to 16 <= 32)
+constexpr int kKSMax = 32;
+constexpr int kThreads = 192;
+constexpr int kTileBytes = kC * kNC * 2;          // one bf16 [C][128] activation tile (TMA box)
+constexpr uint32_t kTmemCols = 256;               // D1 x2 (64 cols each) + D2 x2 (32 each)
+
+// constant block per head (global, laid out exactly as in shared memory)
+constexpr int kTTBytes = kC * kC * 4;             // B operand of the Toeplitz product
+constexpr int kATBytes = kC * kKSMax * 4;         // B operand of the carry product
+constexpr int kVTBytes = kKSMax * kC * 4;         // B operand of the state product
+constexpr int kConstBytes = kTTBytes + kATBytes + kVTBytes + 2 * kMaxModes * 8;   // + lambda^C, lambda^Lseg
+constexpr int kConstStride = (kConstBytes + 255) & ~255;
+
+// shared memory map (offsets from a 1024-byte aligned base)
+constexpr int kSmTT = 0;
+constexpr int kSmAT = kSmTT + kTTBytes;
+constexpr int kSmVT = kSmAT + kATBytes;
+constexpr int kSmUT = kSmVT + kVTBytes;                       // 2 x [128][C] tf32
+constexpr int kUTBytes = kNC * kC * 4;
+constexpr int kSmST = kSmUT + 2 * kUTBytes;                   // [128][KS] tf32
+constexpr int kSTBytes = kNC * kKSMax * 4;
+constexpr int kSmKV = kSmST + kSTBytes;                       // 2 stages x {k, v}
+constexpr int kSmQ = kSmKV + 2 * 2 * kTileBytes;              // 2 stages x q (y staged in place)
+constexpr int kSmBar = kSmQ + 2 * kTileBytes;
+constexpr int kNumBars = 18;
+constexpr int kSmMisc = kSmBar + kNumBars * 8;
+constexpr int kSmemBytes = kSmMisc + 64 + 1024;               // + misc words + alignment slack
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+
+// barrier slots
+enum : int {
+    kBarKVFull = 0,    // [2] TMA k,v landed (1 arrival + tx)
+    kBarKVEmpty = 2,   // [2] k,v consumed (128)
+    kBarQFull = 4,     // [2] TMA q landed (1 + tx)
+    kBarQEmpty = 6,    // [2] q/y buffer free again (1)
+    kBarURdy = 8,      // [2] U operand written (128)
+    kBarSRdy = 10,     // state operand written (128)
+    kBarWDone = 11,    // [2] state product done (commit)
+    kBarYDone = 13,    // [2] output product done (commit)
+    kBarYStaged = 15,  // gated output staged for the store (128)
+    kBarPub = 16,      // segment state written to global (128)
+    kBarDrain = 17     // every MMA of the CTA finished (commit)
+};
+
+// byte offset of element (row, k) in a K-major, no-swizzle core-matrix tile whose K extent is K
+__host__ __device__ __forceinline__ int cm_off(int row, int k, int K) {
+    return (k >> 2) * 128 + (row >> 3) * (K * 32) + (row & 7) * 16 + (k & 3) * 4;
+}
+
+struct ChunkArgs {
+    int L, Dch, d, KS, ch;
+    int ntiles;          // channel tiles per sequence (Dch / 128)
+    int nchunks;         // chunks per sequence
+    int nseg, segc;      // segments per sequence, chunks per segment (all but the last)
+    const float2 *lam;   // [H][d]
+    const uint8_t *consts;
+    float *state_out;    // [B][d][Dch][2]
+    int *sched;          // [0] ticket counter, [1] error code
+    int *status;         // [items]: 0 none, 1 segment contribution, 2 inclusive state
+    float2 *agg;         // [items][d][128]
+    float2 *inc;         // [items][d][128]
+};
+
+enum : int { kErrWait = 1, kErrLookback = 2 };
+
+__device__ __forceinline__ void record_error(const ChunkArgs &a, volatile int *abort, int code) {
+    *abort = 1;
+    atomicCAS(a.sched + 1, 0, code);
+}
+
+// ------------------------------------------------------------------ per-head constants
+__global__ void __launch_bounds__(256)
+chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R,
+                    const float *__restrict__ Dskip, int d, int KS, int seg_tokens,
+                    uint8_t *__restrict__ consts) {
+    const int hd = blockIdx.x;
+    uint8_t *base = consts + (size_t)hd * kConstStride;
+    float *TT = reinterpret_cast<float *>(base);
+    float *AT = reinterpret_cast<float *>(base + kTTBytes);
+    float *VT = reinterpret_cast<float *>(base + kTTBytes + kATBytes);
+    float2 *lamC = reinterpret_cast<float2 *>(base + kTTBytes + kATBytes + kVTBytes);
+    float2 *lamS = lamC + kMaxModes;
+    __shared__ double hs[kC];
+    const float2 *lh = lam + (size_t)hd * d;
+    const float2 *rh = R + (size_t)hd * d;
+    // filter taps h_0 .. h_{C-1} in fp64
+    for (int j = threadIdx.x; j < kC; j += blockDim.x) {
+        double acc = 0.0;
+        if (j == 0) {
+            acc = Dskip[hd];
+        } else {
+            for (int n = 0; n < d; ++n) {
+                const cd p = cdpow(cd{lh[n].x, lh[n].y}, j - 1);
+                acc += (double)rh[n].x * p.x - (double)rh[n].y * p.y;
+            }
+        }
+        hs[j] = acc;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < kC * kC; e += blockDim.x) {
+        const int tau = e / kC, io = e % kC;
+        const float v = io <= tau ? (float)hs[tau - io] : 0.f;
+        TT[cm_off(tau, io, kC) / 4] = tc::to_tf32(v);
+    }
+    for (int e = threadIdx.x; e < kC * KS; e += blockDim.x) {
+        const int tau = e / KS, r = e % KS;
+        float v = 0.f;
+        if (r < 2 * d) {
+            const int n = r < d ? r : r - d;
+            const cd p = cdpow(cd{lh[n].x, lh[n].y}, tau);
+            const double re = (double)rh[n].x * p.x - (double)rh[n].y * p.y;
+            const double im = (double)rh[n].x * p.y + (double)rh[n].y * p.x;
+            v = r < d ? (float)re : (float)(-im);
+        }
+        AT[cm_off(tau, r, KS) / 4] = tc::to_tf32(v);
+    }
+    for (int e = threadIdx.x; e < KS * kC; e += blockDim.x) {
+        const int r = e / kC, io = e % kC;
+        float v = 0.f;
+        if (r < 2 * d) {
+            const int n = r < d ? r : r - d;
+            const cd p = cdpow(cd{lh[n].x, lh[n].y}, kC - 1 - io);
+            v = r < d ? (float)p.x : (float)p.y;
+        }
+        VT[cm_off(r, io, kC) / 4] = tc::to_tf32(v);
+    }
+    for (int n = threadIdx.x; n < kMaxModes; n += blockDim.x) {
+        cd pc{0.0, 0.0}, ps{0.0, 0.0};
+        if (n < d) {
+            pc = cdpow(cd{lh[n].x, lh[n].y}, kC);
+            ps = cdpow(cd{lh[n].x, lh[n].y}, seg_tokens);
+        }
+        lamC[n] = make_float2((float)pc.x, (float)pc.y);
+        lamS[n] = make_float2((float)ps.x, (float)ps.y);
+    }
+}
+
+
+// ------------------------------------------------------------------ main kernel
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_y,
+                     const ChunkArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = tc::smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    auto bar = [&](int slot) { return sbase + kSmBar + 8u * slot; };
+    volatile int *misc = reinterpret_cast<volatile int *>(sm + kSmMisc);   // item, abort, tmem, never
+    volatile int *abort = misc + 1;
+    volatile int *never = misc + 3;
+
+    if (tid == 0) {
+        misc[0] = atomicAdd(a.sched, 1);
+        misc[1] = 0;
+        misc[3] = 0;
+        const int counts[kNumBars] = {1, 1, 128, 128, 1, 1, 1, 1, 128, 128, 128, 1, 1, 1, 1, 128, 128, 1};
+        for (int i = 0; i < kNumBars; ++i) tc::mbar_init(bar(i), counts[i]);
+        tc::fence_mbar_init();
+    }
+    if (warp == 5) {
+        tc::tmem_alloc(tc::smem_u32((const void *)(misc + 2)), kTmemCols);
+        tc::tmem_relinquish();
+    }
+    __syncthreads();
+    const int item = misc[0];
+    const int unit = item / a.nseg, seg = item % a.nseg;
+    const int b = unit / a.ntiles, c0 = (unit % a.ntiles) * kNC;
+    const int hd = c0 / a.ch;
+    const int ck0 = seg * a.segc;
+    const int nck = min(a.nchunks, ck0 + a.segc) - ck0;
+    const bool last_seg = (seg == a.nseg - 1);
+    const bool phase1 = !last_seg;
+    const int n1 = phase1 ? nck : 0;                  // state-only iterations
+    const int d = a.d, KS = a.KS;
+
+    // per-head constants -> shared memory; zero the state operand (its padding columns stay 0)
+    {
+        const int4 *src = reinterpret_cast<const int4 *>(a.consts + (size_t)hd * kConstStride);
+        int4 *dst = reinterpret_cast<int4 *>(sm);
+        for (int i = tid; i < (kTTBytes + kATBytes + kVTBytes) / 16; i += kThreads) dst[i] = __ldg(src + i);
+        int4 *stz = reinterpret_cast<int4 *>(sm + kSmST);
+        for (int i = tid; i < kSTBytes / 16; i += kThreads) stz[i] = make_int4(0, 0, 0, 0);
+    }
+    tc::fence_proxy_async_smem();
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = (uint32_t)misc[2];
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ TMA producers
+        if (lane == 0) {            // k, v for every iteration (state-only pass, then full pass)
+            tc::prefetch_tensormap(&tm_k);
+            tc::prefetch_tensormap(&tm_v);
+            int it = 0;
+            for (; it < n1 + nck; ++it) {
+                const int s = it & 1;
+                if (!tc::mbar_wait(bar(kBarKVEmpty + s), ((it >> 1) & 1) ^ 1, abort)) {
+                    record_error(a, abort, kErrWait);
+                    break;
+                }
+                const int chunk = ck0 + (it < n1 ? it : it - n1);
+                const uint32_t dst = sbase + kSmKV + s * 2 * kTileBytes;
+                tc::mbar_expect_tx(bar(kBarKVFull + s), 2 * kTileBytes);
+                tc::tma_load_3d(dst, &tm_k, bar(kBarKVFull + s), c0, chunk * kC, b);
+                tc::tma_load_3d(dst + kTileBytes, &tm_v, bar(kBarKVFull + s), c0, chunk * kC, b);
+            }
+            if (*abort)
+                for (int j = max(0, it - 2); j < it; ++j)
+                    tc::mbar_wait(bar(kBarKVFull + (j & 1)), (j >> 1) & 1, never);
+        } else if (lane == 1) {     // q for the full pass (the buffer also stages y)
+            tc::prefetch_tensormap(&tm_q);
+            tc::prefetch_tensormap(&tm_y);
+            int j = 0;
+            for (; j < nck; ++j) {
+                const int s = j & 1;
+                if (!tc::mbar_wait(bar(kBarQEmpty + s), ((j >> 1) & 1) ^ 1, abort)) {
+                    record_error(a, abort, kErrWait);
+                    break;
+                }
+                tc::mbar_expect_tx(bar(kBarQFull + s), kTileBytes);
+                tc::tma_load_3d(sbase + kSmQ + s * kTileBytes, &tm_q, bar(kBarQFull + s), c0,
+                                (ck0 + j) * kC, b);
+            }
+            if (*abort)
+                for (int jj = max(0, j - 2); jj < j; ++jj)
+                    tc::mbar_wait(bar(kBarQFull + (jj & 1)), (jj >> 1) & 1, never);
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_y = tc::idesc_tf32(kNC, kC);
+            const uint32_t idesc_w = tc::idesc_tf32(kNC, KS);
+            for (int it = 0; it < n1 + nck && !*abort; ++it) {
+                const int ub = it & 1;
+                const uint32_t ut = sbase + kSmUT + ub * kUTBytes;
+                if (!tc::mbar_wait(bar(kBarURdy + ub), (it >> 1) & 1, abort)) {
+                    record_error(a, abort, kErrWait);
+                    break;
+                }
+                tc::tc_fence_after();
+                // D2 = U V^T: the chunk's contribution to the state
+                const uint32_t d2 = tmem + 2 * kC + ub * kKSMax;
+                for (int ks = 0; ks < kC / 8; ++ks)
+                    tc::mma_tf32(d2, tc::smem_desc(ut + ks * 256, 128, kC * 32),
+                                 tc::smem_desc(sbase + kSmVT + ks * 256, 128, kC * 32), idesc_w, ks > 0);
+                tc::mma_commit(bar(kBarWDone + ub));
+                if (it >= n1) {
+                    const int j = it - n1;
+                    if (!tc::mbar_wait(bar(kBarSRdy), j & 1, abort)) {
+                        record_error(a, abort, kErrWait);
+                        break;
+                    }
+                    tc::tc_fence_after();
+                    // D1 = U T^T + S A^T: intra-chunk Toeplitz product plus the modal carry
+                    const uint32_t d1 = tmem + (j & 1) * kC;
+                    for (int ks = 0; ks < kC / 8; ++ks)
+                        tc::mma_tf32(d1, tc::smem_desc(ut + ks * 256, 128, kC * 32),
+                                     tc::smem_desc(sbase + kSmTT + ks * 256, 128, kC * 32), idesc_y, ks > 0);
+                    for (int ks = 0; ks < KS / 8; ++ks)
+                        tc::mma_tf32(d1, tc::smem_desc(sbase + kSmST + ks * 256, 128, KS * 32),
+                                     tc::smem_desc(sbase + kSmAT + ks * 256, 128, KS * 32), idesc_y, 1);
+                    tc::mma_commit(bar(kBarYDone + (j & 1)));
+                }
+            }
+            tc::mma_commit(bar(kBarDrain));
+            tc::mbar_wait(bar(kBarDrain), 0, never);
+        }
+    } else {
+        // ------------------------------------------------------------ compute warps
+        const int c = tid;                        // channel within the tile == TMEM lane
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const float2 *lamC = reinterpret_cast<const float2 *>(a.consts + (size_t)hd * kConstStride +
+                                                              kTTBytes + kATBytes + kVTBytes);
+        const float2 *lamS = lamC + kMaxModes;
+        float2 lc[kMaxModes], st[kMaxModes];
+#pragma unroll
+        for (int n = 0; n < kMaxModes; ++n) {
+            lc[n] = n < d ? __ldg(&lamC[n]) : make_float2(0.f, 0.f);
+            st[n] = make_float2(0.f, 0.f);
+        }
+        bool ok = true;
+        int pub_phase = 0;
+        // keep every compute warp converged (tcgen05.ld is warp-collective): a step
+        // counts as done only if all 32 lanes finished it and nobody aborted
+        auto uni = [&](bool x) -> bool { return __all_sync(0xffffffffu, x && !*abort); };
+
+        // u = k*v of the chunk in kv stage (it & 1) -> U operand buffer (it & 1)
+        auto make_u = [&](int it, int chunk, bool release) -> bool {
+            if (!tc::mbar_wait(bar(kBarKVFull + (it & 1)), (it >> 1) & 1, abort)) return false;
+            const __nv_bfloat16 *kt = reinterpret_cast<const __nv_bfloat16 *>(sm + kSmKV + (it & 1) * 2 * kTileBytes);
+            const __nv_bfloat16 *vt = kt + kC * kNC;
+            uint8_t *ut = sm + kSmUT + (it & 1) * kUTBytes;
+            const int valid = a.L - chunk * kC;     // tokens of this chunk inside the prompt
+#pragma unroll 4
+            for (int i4 = 0; i4 < kC / 4; ++i4) {
+                float u[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int io = i4 * 4 + j;
+                    const float x = __bfloat162float(kt[io * kNC + c]) * __bfloat162float(vt[io * kNC + c]);
+                    u[j] = io < valid ? tc::to_tf32(x) : 0.f;
+                }
+                *reinterpret_cast<float4 *>(ut + cm_off(c, i4 * 4, kC)) = make_float4(u[0], u[1], u[2], u[3]);
+            }
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(bar(kBarURdy + (it & 1)));
+            if (release) tc::mbar_arrive(bar(kBarKVEmpty + (it & 1)));
+            return true;
+        };
+        // state operand (tf32): columns [0, d) real parts, [d, 2d) imaginary parts
+        auto write_state = [&]() {
+            uint8_t *stp = sm + kSmST;
+#pragma unroll
+            for (int n = 0; n < kMaxModes; ++n) {
+                if (n < d) {
+                    *reinterpret_cast<float *>(stp + cm_off(c, n, KS)) = tc::to_tf32(st[n].x);
+                    *reinterpret_cast<float *>(stp + cm_off(c, d + n, KS)) = tc::to_tf32(st[n].y);
+                }
+            }
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(bar(kBarSRdy));
+        };
+        // st <- lambda^C st + D2 of iteration it
+        auto advance_state = [&](int it) -> bool {
+            if (!tc::mbar_wait(bar(kBarWDone + (it & 1)), (it >> 1) & 1, abort)) return false;
+            tc::tc_fence_after();
+            float w[kKSMax];
+            const uint32_t taddr = tmem + lane_base + 2 * kC + (it & 1) * kKSMax;
+            tc::tmem_ld16(taddr, w);
+            if (KS > 16) tc::tmem_ld16(taddr + 16, w + 16);
+            tc::tmem_wait_ld();
+            tc::tc_fence_before();
+#pragma unroll
+            for (int n = 0; n < kMaxModes; ++n) {
+                if (n < d) {
+                    const float2 s = st[n];
+                    st[n] = make_float2(fmaf(lc[n].x, s.x, fmaf(-lc[n].y, s.y, w[n])),
+                                        fmaf(lc[n].x, s.y, fmaf(lc[n].y, s.x, w[d + n])));
+                }
+            }
+            return true;
+        };
+        // publish st to global for other items, then set the status word
+        auto publish = [&](float2 *dst, int code) -> bool {
+#pragma unroll
+            for (int n = 0; n < kMaxModes; ++n)
+                if (n < d) dst[(size_t)n * kNC + c] = st[n];
+            __threadfence();
+            tc::mbar_arrive(bar(kBarPub));
+            if (c == 0) {
+                if (!tc::mbar_wait(bar(kBarPub), pub_phase & 1, abort)) return false;
+                __threadfence();
+                atomicExch(a.status + item, code);
+            }
+            ++pub_phase;
+            return true;
+        };
+
+        // ---------------- state-only pass over the segment
+        if (phase1) {
+            ok = uni(make_u(0, ck0, true));
+            for (int i = 0; i < nck && ok; ++i) {
+                if (i + 1 < nck) ok = uni(make_u(i + 1, ck0 + i + 1, true));
+                if (ok) ok = uni(advance_state(i));
+            }
+            if (ok) ok = uni(publish((seg == 0 ? a.inc : a.agg) + (size_t)item * d * kNC, seg == 0 ? 2 : 1));
+            if (!ok) record_error(a, abort, kErrWait);
+        }
+        float2 sloc[kMaxModes];
+#pragma unroll
+        for (int n = 0; n < kMaxModes; ++n) { sloc[n] = st[n]; st[n] = make_float2(0.f, 0.f); }
+
+        // ---------------- look-back: the state entering this segment
+        if (ok && seg > 0) {
+            float2 lsg[kMaxModes], scale[kMaxModes];
+#pragma unroll
+            for (int n = 0; n < kMaxModes; ++n) {
+                lsg[n] = n < d ? __ldg(&lamS[n]) : make_float2(0.f, 0.f);
+                scale[n] = make_float2(1.f, 0.f);
+            }
+            for (int p = item - 1; p >= item - seg && ok; --p) {
+                int code = *(volatile int *)(a.status + p);
+                const unsigned long long t0 = tc::global_ns();
+                while (code == 0 && !*abort && tc::global_ns() - t0 < tc::kWaitNs) {
+                    __nanosleep(100);
+                    code = *(volatile int *)(a.status + p);
+                }
+                if (code == 0) {
+                    record_error(a, abort, kErrLookback);
+                    ok = false;
+                    break;
+                }
+                __threadfence();
+                const volatile float2 *src = (code == 2 ? a.inc : a.agg) + (size_t)p * d * kNC;
+#pragma unroll
+                for (int n = 0; n < kMaxModes; ++n) {
+                    if (n < d) {
+                        const float2 v = make_float2(src[(size_t)n * kNC + c].x, src[(size_t)n * kNC + c].y);
+                        st[n] = cadd(st[n], cmul(scale[n], v));
+                        scale[n] = cmul(scale[n], lsg[n]);
+                    }
+                }
+                if (code == 2) break;
+            }
+            if (ok && phase1) {
+                // inclusive state at the end of this segment: lambda^Lseg s_in + own contribution
+                float2 keep[kMaxModes];
+#pragma unroll
+                for (int n = 0; n < kMaxModes; ++n) {
+                    keep[n] = st[n];
+                    st[n] = cadd(cmul(lsg[n], st[n]), sloc[n]);
+                }
+                ok = publish(a.inc + (size_t)item * d * kNC, 2);
+#pragma unroll
+                for (int n = 0; n < kMaxModes; ++n) st[n] = keep[n];
+                if (!ok) record_error(a, abort, kErrWait);
+            }
+        }
+        ok = uni(ok);
+
+        // ---------------- full pass: outputs and state, starting from st = state entering the segment
+        if (ok) {
+            const int it0 = n1;
+            ok = uni(make_u(it0, ck0, ck0 != a.nchunks - 1));
+            if (ok) write_state();
+            for (int j = 0; j < nck && ok; ++j) {
+                const int it = it0 + j, chunk = ck0 + j;
+                if (j + 1 < nck) {
+                    if (!(ok = uni(make_u(it + 1, chunk + 1, chunk + 1 != a.nchunks - 1)))) break;
+                }
+                if (chunk != a.nchunks - 1) {
+                    if (!(ok = uni(advance_state(it)))) break;
+                } else {
+                    // last chunk of the prompt (possibly partial): exact fp32 Horner over its
+                    // tokens, st <- lambda^rem st + sum_{iota<rem} lambda^(rem-1-iota) u_iota
+                    const int rem = a.L - chunk * kC;
+                    const __nv_bfloat16 *kt = reinterpret_cast<const __nv_bfloat16 *>(sm + kSmKV + (it & 1) * 2 * kTileBytes);
+                    const __nv_bfloat16 *vt = kt + kC * kNC;
+                    float2 lm[kMaxModes], acc[kMaxModes];
+#pragma unroll
+                    for (int n = 0; n < kMaxModes; ++n) {
+                        lm[n] = n < d ? __ldg(&a.lam[(size_t)hd * d + n]) : make_float2(0.f, 0.f);
+                        acc[n] = make_float2(0.f, 0.f);
+                    }
+                    for (int io = 0; io < rem; ++io) {
+                        const float u = __bfloat162float(kt[io * kNC + c]) * __bfloat162float(vt[io * kNC + c]);
+#pragma unroll
+                        for (int n = 0; n < kMaxModes; ++n)
+                            acc[n] = make_float2(fmaf(acc[n].x, lm[n].x, fmaf(-acc[n].y, lm[n].y, u)),
+                                                 fmaf(acc[n].x, lm[n].y, acc[n].y * lm[n].x));
+                    }
+                    tc::mbar_arrive(bar(kBarKVEmpty + (it & 1)));
+#pragma unroll
+                    for (int n = 0; n < kMaxModes; ++n) {
+                        if (n < d) {
+                            const cd pw = cdpow(cd{lm[n].x, lm[n].y}, rem);
+                            st[n] = cadd(cmul(make_float2((float)pw.x, (float)pw.y), st[n]), acc[n]);
+                        }
+                    }
+                }
+                // output product of this chunk done: D1 ready, state operand free
+                if (!(ok = uni(tc::mbar_wait(bar(kBarYDone + (j & 1)), (j >> 1) & 1, abort)))) break;
+                tc::tc_fence_after();
+                if (j + 1 < nck) write_state();
+                // gate: y = q * D1, written in place of q, then one TMA store of the tile
+                if (!(ok = uni(tc::mbar_wait(bar(kBarQFull + (j & 1)), (j >> 1) & 1, abort)))) break;
+                __nv_bfloat16 *qy = reinterpret_cast<__nv_bfloat16 *>(sm + kSmQ + (j & 1) * kTileBytes);
+#pragma unroll
+                for (int k16 = 0; k16 < kC / 16; ++k16) {
+                    float z[16];
+                    tc::tmem_ld16(tmem + lane_base + (j & 1) * kC + k16 * 16, z);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) {
+                        const int tau = k16 * 16 + t;
+                        qy[tau * kNC + c] = __float2bfloat16_rn(__bfloat162float(qy[tau * kNC + c]) * z[t]);
+                    }
+                }
+                tc::tc_fence_before();
+                tc::fence_proxy_async_smem();
+                tc::mbar_arrive(bar(kBarYStaged));
+                if (c == 0) {
+                    ok = tc::mbar_wait(bar(kBarYStaged), j & 1, abort);
+                    if (ok) {
+                        tc::tma_store_3d(&tm_y, sbase + kSmQ + (j & 1) * kTileBytes, c0, chunk * kC, b);
+                        tc::bulk_commit();
+                        if (j >= 1) {
+                            // the previous tile's store has read its buffer: hand it back to the q loader
+                            tc::bulk_wait_read<1>();
+                            tc::mbar_arrive(bar(kBarQEmpty + ((j - 1) & 1)));
+                        }
+                    }
+                }
+                if (!(ok = uni(ok))) break;
+            }
+            if (!ok) record_error(a, abort, kErrWait);
+            if (c == 0) tc::bulk_wait<0>();
+            if (ok && last_seg) {
+                float2 *so = reinterpret_cast<float2 *>(a.state_out) + ((size_t)b * d) * a.Dch + c0 + c;
+#pragma unroll
+                for (int n = 0; n < kMaxModes; ++n)
+                    if (n < d) so[(size_t)n * a.Dch] = st[n];
+            }
+        } else {
+            record_error(a, abort, kErrWait);
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    if (warp == 5) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// [B][L][Dch] bf16 viewed as a 3-D tensor (Dch, L, B); box = 128 channels x C tokens x 1
+bool make_map(CUtensorMap *m, const void *base, int B, int L, int Dch) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)Dch, (cuuint64_t)L, (cuuint64_t)B};
+    cuuint64_t strides[2] = {(cuuint64_t)Dch * 2, (cuuint64_t)L * Dch * 2};
+    cuuint32_t box[3] = {(cuuint32_t)kNC, (cuuint32_t)kC, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct ChunkPlan {
+    int nchunks, nseg, segc, items;
+    size_t consts_off, sched_off, status_off, agg_off, inc_off, total;
+};
+
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+ChunkPlan plan(int B, int L, int Dch, int H, int d) {
+    ChunkPlan p{};
+    p.nchunks = (L + kC - 1) / kC;
+    const long long units = (long long)B * (Dch / kNC);
+    // enough items for ~2 waves of one CTA per SM, segments of at least 4 chunks
+    long long want = (2 * 148 + units - 1) / units;
+    long long maxseg = (p.nchunks + 3) / 4;
+    if (want > maxseg) want = maxseg;
+    if (want < 1) want = 1;
+    p.segc = (int)((p.nchunks + want - 1) / want);
+    p.nseg = (p.nchunks + p.segc - 1) / p.segc;
+    p.items = (int)(units * p.nseg);
+    p.consts_off = 0;
+    p.sched_off = al256((size_t)H * kConstStride);
+    p.status_off = p.sched_off + 256;
+    p.agg_off = p.status_off + al256((size_t)p.items * 4);
+    p.inc_off = p.agg_off + al256((size_t)p.items * d * kNC * 8);
+    p.total = p.inc_off + al256((size_t)p.items * d * kNC * 8);
+    return p;
+}
+
+}  // namespace
+
+bool chunked_supported(int dtype, int Dch, int H, int d) {
+    return dtype == HYENA_BF16 && H > 0 && Dch % H == 0 && (Dch / H) % kNC == 0 && d >= 1 && d <= kMaxModes;
+}
+
+size_t chunked_ws_bytes(int B, int L, int Dch, int H, int d) { return plan(B, L, Dch, H, d).total; }
+
+cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, int B, int L, int Dch,
+                                   int H, int d, const float2 *lam, const float2 *R, const float *Dskip,
+                                   void *y, float *state_out, void *ws, cudaStream_t s) {
+    const ChunkPlan p = plan(B, L, Dch, H, d);
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    const int KS = ((2 * d + 15) / 16) * 16;
+    cudaError_t e = cudaMemsetAsync(w + p.sched_off, 0, p.agg_off - p.sched_off, s);
+    if (e != cudaSuccess) return e;
+    chunk_consts_kernel<<<H, 256, 0, s>>>(lam, R, Dskip, d, KS, p.segc * kC, w + p.consts_off);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    CUtensorMap mq, mk, mv, my;
+    if (!make_map(&mq, q, B, L, Dch) || !make_map(&mk, k, B, L, Dch) || !make_map(&mv, v, B, L, Dch) ||
+        !make_map(&my, y, B, L, Dch))
+        return cudaErrorInvalidValue;
+    ChunkArgs a;
+    a.L = L; a.Dch = Dch; a.d = d; a.KS = KS; a.ch = Dch / H;
+    a.ntiles = Dch / kNC; a.nchunks = p.nchunks; a.nseg = p.nseg; a.segc = p.segc;
+    a.lam = lam;
+    a.consts = w + p.consts_off;
+    a.state_out = state_out;
+    a.sched = reinterpret_cast<int *>(w + p.sched_off);
+    a.status = reinterpret_cast<int *>(w + p.status_off);
+    a.agg = reinterpret_cast<float2 *>(w + p.agg_off);
+    a.inc = reinterpret_cast<float2 *>(w + p.inc_off);
+    e = cudaFuncSetAttribute(prefill_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    prefill_chunk_kernel<<<p.items, kThreads, kSmemBytes, s>>>(mq, mk, mv, my, a);
+    return cudaGetLastError();
+}
+
+int chunked_error_offset(int B, int L, int Dch, int H, int d) {
+    return (int)(plan(B, L, Dch, H, d).sched_off + 4);
+}
+
+}  // namespace hyena

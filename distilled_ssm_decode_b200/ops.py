@@ -34,6 +34,10 @@ SIGNATURES = {
     "hyena_prefill_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "hyena_prefill": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp, _fp,
                            _vp, _sz, _vp]),
+    "hyena_prefill_chunked_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "hyena_prefill_chunked_error_offset": (_sz, [_i, _i, _i, _i, _i]),
+    "hyena_prefill_chunked": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp, _fp,
+                                   _vp, _sz, _vp]),
     "hyena_prompt_state_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "hyena_prompt_state": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _fp, _fp, _vp, _sz, _vp]),
     "hyena_decode_step": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _fp, _fp, _fp, _fp, _vp, _vp]),
@@ -154,6 +158,40 @@ def prefill(q, k, v, lam, R, Dskip, fft_len: int, y=None, state=None, workspace=
                                _ptr(lam), _ptr(R), _ptr(Dskip), _ptr(y), _ptr(state),
                                _ptr(workspace), workspace.numel(), _stream(q.device)))
     return y, state
+
+
+def prefill_chunked_workspace_bytes(B, L, Dch, H, d) -> int:
+    return int(lib().hyena_prefill_chunked_workspace_bytes(B, L, Dch, H, d))
+
+
+def prefill_chunked(q, k, v, lam, R, Dskip, y=None, state=None, workspace=None):
+    """Chunked tensor-core prefill.  q,k,v bf16 [B][L][Dch] -> (y, state [B][d][Dch][2]).
+
+    Returns (y, state, workspace); the int32 at chunked_error_offset() of the
+    workspace is 0 after a successful run."""
+    lam, R, Dskip = _params(lam, R, Dskip)
+    q, k, v = _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v")
+    dt = _act_dtype(q)
+    B, L, Dch = q.shape
+    H, d = lam.shape[0], lam.shape[1]
+    if y is None:
+        y = torch.empty_like(q)
+    if state is None:
+        state = torch.empty((B, d, Dch, 2), dtype=torch.float32, device=q.device)
+    nbytes = prefill_chunked_workspace_bytes(B, L, Dch, H, d)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    _check("hyena_prefill_chunked",
+           lib().hyena_prefill_chunked(_ptr(q), _ptr(k), _ptr(v), dt, B, L, Dch, H, d, _ptr(lam),
+                                       _ptr(R), _ptr(Dskip), _ptr(y), _ptr(state), _ptr(workspace),
+                                       workspace.numel(), _stream(q.device)))
+    return y, state, workspace
+
+
+def chunked_error(workspace, B, L, Dch, H, d) -> int:
+    """The kernel's error word (synchronises): 0 when every bounded wait succeeded."""
+    off = int(lib().hyena_prefill_chunked_error_offset(B, L, Dch, H, d))
+    return int(workspace[off:off + 4].view(torch.int32).item())
 
 
 def prompt_state(k, v, lam, H: int, state=None):

@@ -139,6 +139,35 @@ int hyena_prefill(const void *q, const void *k, const void *v, int dtype,
                   void *workspace, size_t ws_bytes, hyena_stream_t stream);
 
 /*
+ * Prefill by chunked modal evaluation on the tensor cores: the same operator
+ * and outputs as hyena_prefill, computed as an exact regrouping of the causal
+ * convolution.  Per chunk of 64 tokens, the intra-chunk part is a Toeplitz
+ * product with the filter taps h_0..h_63 and the older tokens enter through the
+ * recurrent state: z_t = sum_{j in chunk, j<=t} h_{t-j} u_j
+ * + Re sum_n R_n lambda_n^(t-c0) s_n(c0), with s advanced chunk by chunk
+ * (s(c0+C) = lambda^C s(c0) + sum_j lambda^(c0+C-1-j) u_j); the last state is
+ * the prompt state.  (The "FFT (or chunked)" evaluation of the long
+ * convolution; the carry is the distilled recurrence of "Laughing Hyena
+ * Distillery", "Main findings".)  Products run in tf32 with fp32 accumulation;
+ * the state is carried in fp32.
+ *   Arguments as hyena_prefill, without fft_len.
+ *   Implemented for: dtype HYENA_BF16, Dch/H a multiple of 128, d <= 16, all
+ *   activation pointers 16-byte aligned; HYENA_ERR_UNSUPPORTED otherwise.
+ *   workspace: >= hyena_prefill_chunked_workspace_bytes() bytes, 256-byte aligned.
+ *   The int32 at byte offset hyena_prefill_chunked_error_offset() of the
+ *   workspace is 0 after a successful run; a nonzero value means a bounded
+ *   wait inside the kernel gave up (the outputs are then invalid).  Read it
+ *   after synchronising the stream if needed.
+ */
+size_t hyena_prefill_chunked_workspace_bytes(int B, int L, int Dch, int H, int d);
+size_t hyena_prefill_chunked_error_offset(int B, int L, int Dch, int H, int d);
+int hyena_prefill_chunked(const void *q, const void *k, const void *v, int dtype,
+                          int B, int L, int Dch, int H, int d,
+                          const float *lambda, const float *R, const float *Dskip,
+                          void *y, float *state_out,
+                          void *workspace, size_t ws_bytes, hyena_stream_t stream);
+
+/*
  * Prompt -> state reduction alone (the Vandermonde contraction over the
  * prompt; "Main findings": the O(d) state that generation continues from):
  *   state_out[b][n][c] = sum_{j<L} lambda[head(c)][n]^(L-1-j) k[b][j][c] v[b][j][c]

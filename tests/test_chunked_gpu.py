@@ -1,0 +1,118 @@
+"""GPU parity of the chunked tensor-core prefill (tcgen05) against the fp64 oracle.
+
+The chunked route regroups the causal convolution into 64-token chunks with the
+recurrent state carried between them; its outputs must match the oracle's
+direct convolution and prompt state within the bf16 tolerance (2e-2 of
+max|oracle|).  Shapes cover ragged prompts, prompts shorter than one chunk,
+several 128-channel tiles and heads, d from 1 to 16, and sequences split into
+many segments (which exercises the cross-segment state look-back).  Every run
+also checks the kernel's error word (0 = no bounded wait gave up).
+"""
+import numpy as np
+import pytest
+import torch
+
+from distilled_ssm_decode_b200 import ops
+from distilled_ssm_decode_b200 import workloads as W
+from parity_util import TOL, column_params, dev_params, gather_columns, rel_err, sample_columns, state_c128
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from distilled_ssm_decode_b200 import build
+    build.build()
+
+
+def _run(q, k, v, p):
+    lam, R, D = dev_params(p)
+    y, s, ws = ops.prefill_chunked(q.cuda(), k.cuda(), v.cuda(), lam, R, D)
+    B, L, Dch = q.shape
+    err = ops.chunked_error(ws, B, L, Dch, lam.shape[0], lam.shape[1])
+    assert err == 0, f"kernel error word {err}"
+    return y.cpu(), state_c128(s)
+
+
+CASES = [
+    # B, L, Dch, H, d
+    (1, 64, 128, 1, 16),      # one full chunk
+    (1, 1, 128, 1, 16),       # single token
+    (2, 63, 256, 2, 8),       # shorter than a chunk, two heads
+    (2, 65, 256, 1, 16),      # one chunk + 1 token; a head spans two channel tiles
+    (3, 300, 128, 1, 4),      # ragged, d = 4
+    (1, 1000, 384, 3, 1),     # d = 1
+    (1, 4096, 128, 1, 16),    # one tile: the sequence is split into many segments (look-back)
+    (2, 2048, 256, 2, 12),    # d not a multiple of 8
+]
+
+
+@pytest.mark.parametrize("B,L,Dch,H,d", CASES)
+def test_chunked_small_cases_full_compare(oracle, B, L, Dch, H, d):
+    w = W.Workload(300 + L + d, "case", B=B, L=L, Dch=Dch, H=H, d=d, dtype="bf16", fft_len=0, T=0)
+    p = W.params(w)
+    q, k, v = W.prefill_inputs(w)
+    y, s = _run(q, k, v, p)
+    qf, kf, vf = W.to_f64(q), W.to_f64(k), W.to_f64(v)
+    if L <= 1024:
+        h = oracle.filter_from_modes(p.lam, p.R, p.Dskip, L)
+        y_ref = oracle.conv_direct(qf, kf, vf, h, H=H)
+        s_ref = oracle.prompt_state(kf, vf, p.lam, H=H)
+    else:
+        y_ref, s_ref = oracle.recurrent(qf, kf, vf, p.lam, p.R, p.Dskip, H=H)
+    ey, es = rel_err(y.double().numpy(), y_ref), rel_err(s, s_ref)
+    assert ey <= TOL["bf16"] and es <= TOL["bf16"], (ey, es)
+
+
+@pytest.mark.parametrize("name,ncols", [("mid_bf16", 24), ("gen1p3b_bf16", 32)])
+def test_chunked_full_size_sampled(oracle, name, ncols):
+    w = W.WORKLOADS[name]
+    p = W.params(w)
+    q, k, v = W.prefill_inputs(w)
+    y, s = _run(q, k, v, p)
+    rng = np.random.default_rng(7)
+    bc = sample_columns(rng, w.B, w.Dch, ncols)
+    lam_c, R_c, D_c = column_params(p, w.H, w.Dch, [c for _, c in bc])
+    qc, kc, vc = gather_columns(q, bc), gather_columns(k, bc), gather_columns(v, bc)
+    h = oracle.filter_from_modes(lam_c, R_c, D_c, w.L)
+    y_ref = oracle.conv_direct(qc, kc, vc, h, H=len(bc))
+    s_ref = oracle.prompt_state(kc, vc, lam_c, H=len(bc))
+    ey = rel_err(gather_columns(y, bc), y_ref)
+    es = rel_err(np.stack([s[b, :, c] for b, c in bc], -1)[None], s_ref)
+    assert ey <= TOL["bf16"] and es <= TOL["bf16"], (ey, es)
+
+
+def test_chunked_matches_fft_route():
+    """Both prefill routes compute the same operator: outputs agree within the bf16 bar."""
+    w = W.WORKLOADS["mid_bf16"]
+    p = W.params(w)
+    q, k, v = (t.cuda() for t in W.prefill_inputs(w, B=2, L=2048, Dch=256))
+    lam, R, D = dev_params(p.__class__(p.lam[:2], p.R[:2], p.Dskip[:2]))
+    y1, s1, _ = ops.prefill_chunked(q, k, v, lam, R, D)
+    y2, s2 = ops.prefill(q, k, v, lam, R, D, 4096)
+    assert rel_err(y1.cpu().double().numpy(), y2.cpu().double().numpy()) <= TOL["bf16"]
+    assert rel_err(state_c128(s1), state_c128(s2)) <= 1e-3
+
+
+def test_chunked_is_deterministic():
+    w = W.WORKLOADS["gen1p3b_bf16"]
+    p = W.params(w)
+    q, k, v = (t.cuda() for t in W.prefill_inputs(w, B=4, L=512, Dch=256))
+    lam, R, D = dev_params(p.__class__(p.lam[:2], p.R[:2], p.Dskip[:2]))
+    y1, s1, _ = ops.prefill_chunked(q, k, v, lam, R, D)
+    y2, s2, _ = ops.prefill_chunked(q, k, v, lam, R, D)
+    assert torch.equal(y1, y2) and torch.equal(s1, s2)
+
+
+def test_chunked_unsupported_shapes_are_rejected():
+    lam = torch.zeros(2, 4, 2, device="cuda")
+    D = torch.zeros(2, device="cuda")
+    x32 = torch.zeros(1, 64, 256, device="cuda")
+    with pytest.raises(ops.HyenaError) as e:
+        ops.prefill_chunked(x32, x32, x32, lam, lam, D)          # fp32 activations
+    assert e.value.status == -5
+    x = torch.zeros(1, 64, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ops.HyenaError) as e:
+        ops.prefill_chunked(x, x, x, lam, lam, D)                # 64 channels per head
+    assert e.value.status == -5
