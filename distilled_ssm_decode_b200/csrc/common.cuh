@@ -5,7 +5,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-#include "../../include/hyena.h"
+#include "hyena.h"   // from include/ (on the -I path)
 
 namespace hyena {
 

@@ -53,13 +53,15 @@ namespace hyena {
 
 namespace {
 
-constexpr int kC = 64;             // tokens per chunk
+constexpr int kC = 32;             // tokens per chunk
 constexpr int kNC = 128;           // channels per tile (MMA M)
 constexpr int kMaxModes = 16;      // d <= 16 (KS = 2d rounded up to 16 <= 32)
 constexpr int kKSMax = 32;
 constexpr int kThreads = 192;
 constexpr int kTileBytes = kC * kNC * 2;          // one bf16 [C][128] activation tile (TMA box)
-constexpr uint32_t kTmemCols = 256;               // D1 x2 (64 cols each) + D2 x2 (32 each)
+constexpr int kKVStages = 4;                      // k,v prefetch depth (chunks)
+constexpr int kQStages = 4;                       // q (and staged y) buffers
+constexpr uint32_t kTmemCols = 128;               // D1 x2 (C cols each) + D2 x2 (32 each)
 
 // constant block per head (global, laid out exactly as in shared memory)
 constexpr int kTTBytes = kC * kC * 4;             // B operand of the Toeplitz product
@@ -74,29 +76,29 @@ constexpr int kSmAT = kSmTT + kTTBytes;
 constexpr int kSmVT = kSmAT + kATBytes;
 constexpr int kSmUT = kSmVT + kVTBytes;                       // 2 x [128][C] tf32
 constexpr int kUTBytes = kNC * kC * 4;
-constexpr int kSmST = kSmUT + 2 * kUTBytes;                   // [128][KS] tf32
+constexpr int kSmST = kSmUT + 2 * kUTBytes;                   // 2 x [128][KS] tf32
 constexpr int kSTBytes = kNC * kKSMax * 4;
-constexpr int kSmKV = kSmST + kSTBytes;                       // 2 stages x {k, v}
-constexpr int kSmQ = kSmKV + 2 * 2 * kTileBytes;              // 2 stages x q (y staged in place)
-constexpr int kSmBar = kSmQ + 2 * kTileBytes;
-constexpr int kNumBars = 18;
+constexpr int kSmKV = kSmST + 2 * kSTBytes;                   // kKVStages x {k, v}
+constexpr int kSmQ = kSmKV + kKVStages * 2 * kTileBytes;      // kQStages x q (y staged in place)
+constexpr int kSmBar = kSmQ + kQStages * kTileBytes;
+constexpr int kNumBars = 27;
 constexpr int kSmMisc = kSmBar + kNumBars * 8;
 constexpr int kSmemBytes = kSmMisc + 64 + 1024;               // + misc words + alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 // barrier slots
 enum : int {
-    kBarKVFull = 0,    // [2] TMA k,v landed (1 arrival + tx)
-    kBarKVEmpty = 2,   // [2] k,v consumed (128)
-    kBarQFull = 4,     // [2] TMA q landed (1 + tx)
-    kBarQEmpty = 6,    // [2] q/y buffer free again (1)
-    kBarURdy = 8,      // [2] U operand written (128)
-    kBarSRdy = 10,     // state operand written (128)
-    kBarWDone = 11,    // [2] state product done (commit)
-    kBarYDone = 13,    // [2] output product done (commit)
-    kBarYStaged = 15,  // gated output staged for the store (128)
-    kBarPub = 16,      // segment state written to global (128)
-    kBarDrain = 17     // every MMA of the CTA finished (commit)
+    kBarKVFull = 0,    // [4] TMA k,v landed (1 arrival + tx)
+    kBarKVEmpty = 4,   // [4] k,v consumed (128)
+    kBarQFull = 8,     // [4] TMA q landed (1 + tx)
+    kBarQEmpty = 12,   // [4] q/y buffer free again (1)
+    kBarURdy = 16,     // [2] U operand written (128)
+    kBarSRdy = 18,     // [2] state operand written (128)
+    kBarWDone = 20,    // [2] state product done (commit)
+    kBarYDone = 22,    // [2] output product done (commit)
+    kBarYStaged = 24,  // gated output staged for the store (128)
+    kBarPub = 25,      // segment state written to global (128)
+    kBarDrain = 26     // every MMA of the CTA finished (commit)
 };
 
 // byte offset of element (row, k) in a K-major, no-swizzle core-matrix tile whose K extent is K
@@ -211,7 +213,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         misc[0] = atomicAdd(a.sched, 1);
         misc[1] = 0;
         misc[3] = 0;
-        const int counts[kNumBars] = {1, 1, 128, 128, 1, 1, 1, 1, 128, 128, 128, 1, 1, 1, 1, 128, 128, 1};
+        const int counts[kNumBars] = {1, 1, 1, 1, 128, 128, 128, 128, 1, 1, 1, 1, 1, 1, 1, 1,
+                                      128, 128, 128, 128, 1, 1, 1, 1, 128, 128, 1};
         for (int i = 0; i < kNumBars; ++i) tc::mbar_init(bar(i), counts[i]);
         tc::fence_mbar_init();
     }
@@ -237,7 +240,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         int4 *dst = reinterpret_cast<int4 *>(sm);
         for (int i = tid; i < (kTTBytes + kATBytes + kVTBytes) / 16; i += kThreads) dst[i] = __ldg(src + i);
         int4 *stz = reinterpret_cast<int4 *>(sm + kSmST);
-        for (int i = tid; i < kSTBytes / 16; i += kThreads) stz[i] = make_int4(0, 0, 0, 0);
+        for (int i = tid; i < 2 * kSTBytes / 16; i += kThreads) stz[i] = make_int4(0, 0, 0, 0);
     }
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
@@ -252,8 +255,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             tc::prefetch_tensormap(&tm_v);
             int it = 0;
             for (; it < n1 + nck; ++it) {
-                const int s = it & 1;
-                if (!tc::mbar_wait(bar(kBarKVEmpty + s), ((it >> 1) & 1) ^ 1, abort)) {
+                const int s = it % kKVStages;
+                if (!tc::mbar_wait(bar(kBarKVEmpty + s), ((it / kKVStages) & 1) ^ 1, abort)) {
                     record_error(a, abort, kErrWait);
                     break;
                 }
@@ -264,15 +267,15 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 tc::tma_load_3d(dst + kTileBytes, &tm_v, bar(kBarKVFull + s), c0, chunk * kC, b);
             }
             if (*abort)
-                for (int j = max(0, it - 2); j < it; ++j)
-                    tc::mbar_wait(bar(kBarKVFull + (j & 1)), (j >> 1) & 1, never);
+                for (int j = max(0, it - kKVStages); j < it; ++j)
+                    tc::mbar_wait(bar(kBarKVFull + j % kKVStages), (j / kKVStages) & 1, never);
         } else if (lane == 1) {     // q for the full pass (the buffer also stages y)
             tc::prefetch_tensormap(&tm_q);
             tc::prefetch_tensormap(&tm_y);
             int j = 0;
             for (; j < nck; ++j) {
-                const int s = j & 1;
-                if (!tc::mbar_wait(bar(kBarQEmpty + s), ((j >> 1) & 1) ^ 1, abort)) {
+                const int s = j % kQStages;
+                if (!tc::mbar_wait(bar(kBarQEmpty + s), ((j / kQStages) & 1) ^ 1, abort)) {
                     record_error(a, abort, kErrWait);
                     break;
                 }
@@ -281,8 +284,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                                 (ck0 + j) * kC, b);
             }
             if (*abort)
-                for (int jj = max(0, j - 2); jj < j; ++jj)
-                    tc::mbar_wait(bar(kBarQFull + (jj & 1)), (jj >> 1) & 1, never);
+                for (int jj = max(0, j - kQStages); jj < j; ++jj)
+                    tc::mbar_wait(bar(kBarQFull + jj % kQStages), (jj / kQStages) & 1, never);
         }
     } else if (warp == 5) {
         // ------------------------------------------------------------ MMA issuer
@@ -305,7 +308,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 tc::mma_commit(bar(kBarWDone + ub));
                 if (it >= n1) {
                     const int j = it - n1;
-                    if (!tc::mbar_wait(bar(kBarSRdy), j & 1, abort)) {
+                    if (!tc::mbar_wait(bar(kBarSRdy + (j & 1)), (j >> 1) & 1, abort)) {
                         record_error(a, abort, kErrWait);
                         break;
                     }
@@ -315,8 +318,9 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     for (int ks = 0; ks < kC / 8; ++ks)
                         tc::mma_tf32(d1, tc::smem_desc(ut + ks * 256, 128, kC * 32),
                                      tc::smem_desc(sbase + kSmTT + ks * 256, 128, kC * 32), idesc_y, ks > 0);
+                    const uint32_t stb = sbase + kSmST + (j & 1) * kSTBytes;
                     for (int ks = 0; ks < KS / 8; ++ks)
-                        tc::mma_tf32(d1, tc::smem_desc(sbase + kSmST + ks * 256, 128, KS * 32),
+                        tc::mma_tf32(d1, tc::smem_desc(stb + ks * 256, 128, KS * 32),
                                      tc::smem_desc(sbase + kSmAT + ks * 256, 128, KS * 32), idesc_y, 1);
                     tc::mma_commit(bar(kBarYDone + (j & 1)));
                 }
@@ -345,8 +349,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 
         // u = k*v of the chunk in kv stage (it & 1) -> U operand buffer (it & 1)
         auto make_u = [&](int it, int chunk, bool release) -> bool {
-            if (!tc::mbar_wait(bar(kBarKVFull + (it & 1)), (it >> 1) & 1, abort)) return false;
-            const __nv_bfloat16 *kt = reinterpret_cast<const __nv_bfloat16 *>(sm + kSmKV + (it & 1) * 2 * kTileBytes);
+            if (!tc::mbar_wait(bar(kBarKVFull + it % kKVStages), (it / kKVStages) & 1, abort)) return false;
+            const __nv_bfloat16 *kt = reinterpret_cast<const __nv_bfloat16 *>(sm + kSmKV + (it % kKVStages) * 2 * kTileBytes);
             const __nv_bfloat16 *vt = kt + kC * kNC;
             uint8_t *ut = sm + kSmUT + (it & 1) * kUTBytes;
             const int valid = a.L - chunk * kC;     // tokens of this chunk inside the prompt
@@ -363,12 +367,12 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             }
             tc::fence_proxy_async_smem();
             tc::mbar_arrive(bar(kBarURdy + (it & 1)));
-            if (release) tc::mbar_arrive(bar(kBarKVEmpty + (it & 1)));
+            if (release) tc::mbar_arrive(bar(kBarKVEmpty + it % kKVStages));
             return true;
         };
-        // state operand (tf32): columns [0, d) real parts, [d, 2d) imaginary parts
-        auto write_state = [&]() {
-            uint8_t *stp = sm + kSmST;
+        // state operand (tf32) for chunk j: columns [0, d) real parts, [d, 2d) imaginary parts
+        auto write_state = [&](int j) {
+            uint8_t *stp = sm + kSmST + (j & 1) * kSTBytes;
 #pragma unroll
             for (int n = 0; n < kMaxModes; ++n) {
                 if (n < d) {
@@ -377,7 +381,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 }
             }
             tc::fence_proxy_async_smem();
-            tc::mbar_arrive(bar(kBarSRdy));
+            tc::mbar_arrive(bar(kBarSRdy + (j & 1)));
         };
         // st <- lambda^C st + D2 of iteration it
         auto advance_state = [&](int it) -> bool {
@@ -481,19 +485,23 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         if (ok) {
             const int it0 = n1;
             ok = uni(make_u(it0, ck0, ck0 != a.nchunks - 1));
-            if (ok) write_state();
+            if (ok) write_state(0);
             for (int j = 0; j < nck && ok; ++j) {
                 const int it = it0 + j, chunk = ck0 + j;
+                // next chunk's U operand (its buffer was freed when chunk j-1's products finished)
                 if (j + 1 < nck) {
                     if (!(ok = uni(make_u(it + 1, chunk + 1, chunk + 1 != a.nchunks - 1)))) break;
                 }
                 if (chunk != a.nchunks - 1) {
+                    // state after this chunk, then the next chunk's state operand, so that the
+                    // next output product can start while this chunk is gated and stored
                     if (!(ok = uni(advance_state(it)))) break;
+                    if (j + 1 < nck) write_state(j + 1);
                 } else {
                     // last chunk of the prompt (possibly partial): exact fp32 Horner over its
                     // tokens, st <- lambda^rem st + sum_{iota<rem} lambda^(rem-1-iota) u_iota
                     const int rem = a.L - chunk * kC;
-                    const __nv_bfloat16 *kt = reinterpret_cast<const __nv_bfloat16 *>(sm + kSmKV + (it & 1) * 2 * kTileBytes);
+                    const __nv_bfloat16 *kt = reinterpret_cast<const __nv_bfloat16 *>(sm + kSmKV + (it % kKVStages) * 2 * kTileBytes);
                     const __nv_bfloat16 *vt = kt + kC * kNC;
                     float2 lm[kMaxModes], acc[kMaxModes];
 #pragma unroll
@@ -508,7 +516,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                             acc[n] = make_float2(fmaf(acc[n].x, lm[n].x, fmaf(-acc[n].y, lm[n].y, u)),
                                                  fmaf(acc[n].x, lm[n].y, acc[n].y * lm[n].x));
                     }
-                    tc::mbar_arrive(bar(kBarKVEmpty + (it & 1)));
+                    tc::mbar_arrive(bar(kBarKVEmpty + it % kKVStages));
 #pragma unroll
                     for (int n = 0; n < kMaxModes; ++n) {
                         if (n < d) {
@@ -517,13 +525,12 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         }
                     }
                 }
-                // output product of this chunk done: D1 ready, state operand free
+                // gate: y = q * D1, written in place of q, then one TMA store of the tile
                 if (!(ok = uni(tc::mbar_wait(bar(kBarYDone + (j & 1)), (j >> 1) & 1, abort)))) break;
                 tc::tc_fence_after();
-                if (j + 1 < nck) write_state();
-                // gate: y = q * D1, written in place of q, then one TMA store of the tile
-                if (!(ok = uni(tc::mbar_wait(bar(kBarQFull + (j & 1)), (j >> 1) & 1, abort)))) break;
-                __nv_bfloat16 *qy = reinterpret_cast<__nv_bfloat16 *>(sm + kSmQ + (j & 1) * kTileBytes);
+                const int qs = j % kQStages;
+                if (!(ok = uni(tc::mbar_wait(bar(kBarQFull + qs), (j / kQStages) & 1, abort)))) break;
+                __nv_bfloat16 *qy = reinterpret_cast<__nv_bfloat16 *>(sm + kSmQ + qs * kTileBytes);
 #pragma unroll
                 for (int k16 = 0; k16 < kC / 16; ++k16) {
                     float z[16];
@@ -541,12 +548,12 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 if (c == 0) {
                     ok = tc::mbar_wait(bar(kBarYStaged), j & 1, abort);
                     if (ok) {
-                        tc::tma_store_3d(&tm_y, sbase + kSmQ + (j & 1) * kTileBytes, c0, chunk * kC, b);
+                        tc::tma_store_3d(&tm_y, sbase + kSmQ + qs * kTileBytes, c0, chunk * kC, b);
                         tc::bulk_commit();
                         if (j >= 1) {
                             // the previous tile's store has read its buffer: hand it back to the q loader
                             tc::bulk_wait_read<1>();
-                            tc::mbar_arrive(bar(kBarQEmpty + ((j - 1) & 1)));
+                            tc::mbar_arrive(bar(kBarQEmpty + (j - 1) % kQStages));
                         }
                     }
                 }
