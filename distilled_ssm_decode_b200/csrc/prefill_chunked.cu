@@ -55,10 +55,12 @@ namespace {
 
 constexpr int kC = 32;             // tokens per chunk
 constexpr int kNC = 128;           // channels per tile (MMA M)
-constexpr int kMaxModes = 16;      // d <= 16 (KS = 2d rounded up to 16 <= 32)
-constexpr int kKSMax = 32;
+constexpr int kMaxModes = 16;      // d <= 16
+constexpr int kKSMax = 32;         // state operand width: Re at [0,16), Im at [16,32)
+constexpr int kIm = 16;
 constexpr int kThreads = 192;
-constexpr int kTileBytes = kC * kNC * 2;          // one bf16 [C][128] activation tile (TMA box)
+constexpr int kTileBytes = kC * kNC * 2;          // one bf16 [C][128] activation tile
+constexpr int kHalfBytes = kTileBytes / 2;        // [C][64] half tile = one TMA box, 128-byte swizzled
 constexpr int kKVStages = 4;                      // k,v prefetch depth (chunks)
 constexpr int kQStages = 4;                       // q (and staged y) buffers
 constexpr uint32_t kTmemCols = 128;               // D1 x2 (C cols each) + D2 x2 (32 each)
@@ -106,8 +108,14 @@ __host__ __device__ __forceinline__ int cm_off(int row, int k, int K) {
     return (k >> 2) * 128 + (row >> 3) * (K * 32) + (row & 7) * 16 + (k & 3) * 4;
 }
 
+// byte offset of activation (token tau, channel c) in a [C][128] bf16 tile held as two
+// [C][64] halves written by TMA with 128-byte swizzling (16-byte chunk ^= row % 8)
+__device__ __forceinline__ int act_off(int tau, int c) {
+    return (c >> 6) * kHalfBytes + tau * 128 + ((((c & 63) >> 3) ^ (tau & 7)) << 4) + (c & 7) * 2;
+}
+
 struct ChunkArgs {
-    int L, Dch, d, KS, ch;
+    int L, Dch, d, ch;
     int ntiles;          // channel tiles per sequence (Dch / 128)
     int nchunks;         // chunks per sequence
     int nseg, segc;      // segments per sequence, chunks per segment (all but the last)
@@ -130,7 +138,7 @@ __device__ __forceinline__ void record_error(const ChunkArgs &a, volatile int *a
 // ------------------------------------------------------------------ per-head constants
 __global__ void __launch_bounds__(256)
 chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R,
-                    const float *__restrict__ Dskip, int d, int KS, int seg_tokens,
+                    const float *__restrict__ Dskip, int d, int seg_tokens,
                     uint8_t *__restrict__ consts) {
     const int hd = blockIdx.x;
     uint8_t *base = consts + (size_t)hd * kConstStride;
@@ -161,25 +169,26 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
         const float v = io <= tau ? (float)hs[tau - io] : 0.f;
         TT[cm_off(tau, io, kC) / 4] = tc::to_tf32(v);
     }
-    for (int e = threadIdx.x; e < kC * KS; e += blockDim.x) {
-        const int tau = e / KS, r = e % KS;
+    // columns r < 16: real parts of mode r; columns 16 + n: imaginary parts of mode n
+    for (int e = threadIdx.x; e < kC * kKSMax; e += blockDim.x) {
+        const int tau = e / kKSMax, r = e % kKSMax;
+        const int n = r & (kIm - 1);
         float v = 0.f;
-        if (r < 2 * d) {
-            const int n = r < d ? r : r - d;
+        if (n < d) {
             const cd p = cdpow(cd{lh[n].x, lh[n].y}, tau);
             const double re = (double)rh[n].x * p.x - (double)rh[n].y * p.y;
             const double im = (double)rh[n].x * p.y + (double)rh[n].y * p.x;
-            v = r < d ? (float)re : (float)(-im);
+            v = r < kIm ? (float)re : (float)(-im);
         }
-        AT[cm_off(tau, r, KS) / 4] = tc::to_tf32(v);
+        AT[cm_off(tau, r, kKSMax) / 4] = tc::to_tf32(v);
     }
-    for (int e = threadIdx.x; e < KS * kC; e += blockDim.x) {
+    for (int e = threadIdx.x; e < kKSMax * kC; e += blockDim.x) {
         const int r = e / kC, io = e % kC;
+        const int n = r & (kIm - 1);
         float v = 0.f;
-        if (r < 2 * d) {
-            const int n = r < d ? r : r - d;
+        if (n < d) {
             const cd p = cdpow(cd{lh[n].x, lh[n].y}, kC - 1 - io);
-            v = r < d ? (float)p.x : (float)p.y;
+            v = r < kIm ? (float)p.x : (float)p.y;
         }
         VT[cm_off(r, io, kC) / 4] = tc::to_tf32(v);
     }
@@ -232,7 +241,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const bool last_seg = (seg == a.nseg - 1);
     const bool phase1 = !last_seg;
     const int n1 = phase1 ? nck : 0;                  // state-only iterations
-    const int d = a.d, KS = a.KS;
+    const int d = a.d;
 
     // per-head constants -> shared memory; zero the state operand (its padding columns stay 0)
     {
@@ -263,8 +272,11 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int chunk = ck0 + (it < n1 ? it : it - n1);
                 const uint32_t dst = sbase + kSmKV + s * 2 * kTileBytes;
                 tc::mbar_expect_tx(bar(kBarKVFull + s), 2 * kTileBytes);
-                tc::tma_load_3d(dst, &tm_k, bar(kBarKVFull + s), c0, chunk * kC, b);
-                tc::tma_load_3d(dst + kTileBytes, &tm_v, bar(kBarKVFull + s), c0, chunk * kC, b);
+                for (int h = 0; h < 2; ++h) {
+                    tc::tma_load_3d(dst + h * kHalfBytes, &tm_k, bar(kBarKVFull + s), c0 + 64 * h, chunk * kC, b);
+                    tc::tma_load_3d(dst + kTileBytes + h * kHalfBytes, &tm_v, bar(kBarKVFull + s), c0 + 64 * h,
+                                    chunk * kC, b);
+                }
             }
             if (*abort)
                 for (int j = max(0, it - kKVStages); j < it; ++j)
@@ -280,8 +292,9 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     break;
                 }
                 tc::mbar_expect_tx(bar(kBarQFull + s), kTileBytes);
-                tc::tma_load_3d(sbase + kSmQ + s * kTileBytes, &tm_q, bar(kBarQFull + s), c0,
-                                (ck0 + j) * kC, b);
+                for (int h = 0; h < 2; ++h)
+                    tc::tma_load_3d(sbase + kSmQ + s * kTileBytes + h * kHalfBytes, &tm_q, bar(kBarQFull + s),
+                                    c0 + 64 * h, (ck0 + j) * kC, b);
             }
             if (*abort)
                 for (int jj = max(0, j - kQStages); jj < j; ++jj)
@@ -291,7 +304,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc_y = tc::idesc_tf32(kNC, kC);
-            const uint32_t idesc_w = tc::idesc_tf32(kNC, KS);
+            const uint32_t idesc_w = tc::idesc_tf32(kNC, kKSMax);
             for (int it = 0; it < n1 + nck && !*abort; ++it) {
                 const int ub = it & 1;
                 const uint32_t ut = sbase + kSmUT + ub * kUTBytes;
@@ -319,9 +332,9 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         tc::mma_tf32(d1, tc::smem_desc(ut + ks * 256, 128, kC * 32),
                                      tc::smem_desc(sbase + kSmTT + ks * 256, 128, kC * 32), idesc_y, ks > 0);
                     const uint32_t stb = sbase + kSmST + (j & 1) * kSTBytes;
-                    for (int ks = 0; ks < KS / 8; ++ks)
-                        tc::mma_tf32(d1, tc::smem_desc(stb + ks * 256, 128, KS * 32),
-                                     tc::smem_desc(sbase + kSmAT + ks * 256, 128, KS * 32), idesc_y, 1);
+                    for (int ks = 0; ks < kKSMax / 8; ++ks)
+                        tc::mma_tf32(d1, tc::smem_desc(stb + ks * 256, 128, kKSMax * 32),
+                                     tc::smem_desc(sbase + kSmAT + ks * 256, 128, kKSMax * 32), idesc_y, 1);
                     tc::mma_commit(bar(kBarYDone + (j & 1)));
                 }
             }
@@ -347,38 +360,50 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // counts as done only if all 32 lanes finished it and nobody aborted
         auto uni = [&](bool x) -> bool { return __all_sync(0xffffffffu, x && !*abort); };
 
-        // u = k*v of the chunk in kv stage (it & 1) -> U operand buffer (it & 1)
-        auto make_u = [&](int it, int chunk, bool release) -> bool {
+        // u = k*v of the chunk in kv stage -> U operand buffer (it & 1).  The k, v tiles are
+        // transposed on the way with ldmatrix: warp w covers channel groups 4w..4w+3 (8 channels
+        // each), and each lane receives token pairs of one channel, which is exactly the
+        // K-major row layout of the U operand.  Tokens past the prompt were zero-filled by TMA.
+        auto make_u = [&](int it, bool release) -> bool {
             if (!tc::mbar_wait(bar(kBarKVFull + it % kKVStages), (it / kKVStages) & 1, abort)) return false;
-            const __nv_bfloat16 *kt = reinterpret_cast<const __nv_bfloat16 *>(sm + kSmKV + (it % kKVStages) * 2 * kTileBytes);
-            const __nv_bfloat16 *vt = kt + kC * kNC;
+            const uint32_t kb = sbase + kSmKV + (it % kKVStages) * 2 * kTileBytes;
             uint8_t *ut = sm + kSmUT + (it & 1) * kUTBytes;
-            const int valid = a.L - chunk * kC;     // tokens of this chunk inside the prompt
-#pragma unroll 4
-            for (int i4 = 0; i4 < kC / 4; ++i4) {
-                float u[4];
+            const int r8 = lane & 7, mat = lane >> 3;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int io = i4 * 4 + j;
-                    const float x = __bfloat162float(kt[io * kNC + c]) * __bfloat162float(vt[io * kNC + c]);
-                    u[j] = io < valid ? tc::to_tf32(x) : 0.f;
+            for (int gi = 0; gi < 4; ++gi) {
+                const int g = 4 * warp + gi, cbase = 8 * g;
+                const int tau_row = 8 * mat + r8;               // row address supplied by this lane
+                const uint32_t off = (uint32_t)((cbase >> 6) * kHalfBytes + tau_row * 128 +
+                                                ((((cbase & 63) >> 3) ^ r8) << 4));
+                uint32_t kr[4], vr[4];
+                tc::ldsm_x4_trans(kb + off, kr);
+                tc::ldsm_x4_trans(kb + kTileBytes + off, vr);
+                const int ch = cbase + (lane >> 2);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const int tau = 8 * m + 2 * (lane & 3);
+                    const float u0 = __uint_as_float(kr[m] << 16) * __uint_as_float(vr[m] << 16);
+                    const float u1 = __uint_as_float(kr[m] & 0xffff0000u) * __uint_as_float(vr[m] & 0xffff0000u);
+                    *reinterpret_cast<float2 *>(ut + cm_off(ch, tau, kC)) = make_float2(tc::to_tf32(u0), tc::to_tf32(u1));
                 }
-                *reinterpret_cast<float4 *>(ut + cm_off(c, i4 * 4, kC)) = make_float4(u[0], u[1], u[2], u[3]);
             }
             tc::fence_proxy_async_smem();
             tc::mbar_arrive(bar(kBarURdy + (it & 1)));
             if (release) tc::mbar_arrive(bar(kBarKVEmpty + it % kKVStages));
             return true;
         };
-        // state operand (tf32) for chunk j: columns [0, d) real parts, [d, 2d) imaginary parts
+        // state operand (tf32) for chunk j: column n real part, column 16 + n imaginary part
         auto write_state = [&](int j) {
             uint8_t *stp = sm + kSmST + (j & 1) * kSTBytes;
 #pragma unroll
-            for (int n = 0; n < kMaxModes; ++n) {
-                if (n < d) {
-                    *reinterpret_cast<float *>(stp + cm_off(c, n, KS)) = tc::to_tf32(st[n].x);
-                    *reinterpret_cast<float *>(stp + cm_off(c, d + n, KS)) = tc::to_tf32(st[n].y);
-                }
+            for (int n4 = 0; n4 < kMaxModes / 4; ++n4) {
+                const int n = 4 * n4;
+                *reinterpret_cast<float4 *>(stp + cm_off(c, n, kKSMax)) =
+                    make_float4(tc::to_tf32(st[n].x), tc::to_tf32(st[n + 1].x), tc::to_tf32(st[n + 2].x),
+                                tc::to_tf32(st[n + 3].x));
+                *reinterpret_cast<float4 *>(stp + cm_off(c, kIm + n, kKSMax)) =
+                    make_float4(tc::to_tf32(st[n].y), tc::to_tf32(st[n + 1].y), tc::to_tf32(st[n + 2].y),
+                                tc::to_tf32(st[n + 3].y));
             }
             tc::fence_proxy_async_smem();
             tc::mbar_arrive(bar(kBarSRdy + (j & 1)));
@@ -390,7 +415,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             float w[kKSMax];
             const uint32_t taddr = tmem + lane_base + 2 * kC + (it & 1) * kKSMax;
             tc::tmem_ld16(taddr, w);
-            if (KS > 16) tc::tmem_ld16(taddr + 16, w + 16);
+            tc::tmem_ld16(taddr + 16, w + 16);
             tc::tmem_wait_ld();
             tc::tc_fence_before();
 #pragma unroll
@@ -398,7 +423,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 if (n < d) {
                     const float2 s = st[n];
                     st[n] = make_float2(fmaf(lc[n].x, s.x, fmaf(-lc[n].y, s.y, w[n])),
-                                        fmaf(lc[n].x, s.y, fmaf(lc[n].y, s.x, w[d + n])));
+                                        fmaf(lc[n].x, s.y, fmaf(lc[n].y, s.x, w[kIm + n])));
                 }
             }
             return true;
@@ -421,9 +446,9 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 
         // ---------------- state-only pass over the segment
         if (phase1) {
-            ok = uni(make_u(0, ck0, true));
+            ok = uni(make_u(0, true));
             for (int i = 0; i < nck && ok; ++i) {
-                if (i + 1 < nck) ok = uni(make_u(i + 1, ck0 + i + 1, true));
+                if (i + 1 < nck) ok = uni(make_u(i + 1, true));
                 if (ok) ok = uni(advance_state(i));
             }
             if (ok) ok = uni(publish((seg == 0 ? a.inc : a.agg) + (size_t)item * d * kNC, seg == 0 ? 2 : 1));
@@ -484,13 +509,13 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // ---------------- full pass: outputs and state, starting from st = state entering the segment
         if (ok) {
             const int it0 = n1;
-            ok = uni(make_u(it0, ck0, ck0 != a.nchunks - 1));
+            ok = uni(make_u(it0, ck0 != a.nchunks - 1));
             if (ok) write_state(0);
             for (int j = 0; j < nck && ok; ++j) {
                 const int it = it0 + j, chunk = ck0 + j;
                 // next chunk's U operand (its buffer was freed when chunk j-1's products finished)
                 if (j + 1 < nck) {
-                    if (!(ok = uni(make_u(it + 1, chunk + 1, chunk + 1 != a.nchunks - 1)))) break;
+                    if (!(ok = uni(make_u(it + 1, chunk + 1 != a.nchunks - 1)))) break;
                 }
                 if (chunk != a.nchunks - 1) {
                     // state after this chunk, then the next chunk's state operand, so that the
@@ -501,8 +526,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     // last chunk of the prompt (possibly partial): exact fp32 Horner over its
                     // tokens, st <- lambda^rem st + sum_{iota<rem} lambda^(rem-1-iota) u_iota
                     const int rem = a.L - chunk * kC;
-                    const __nv_bfloat16 *kt = reinterpret_cast<const __nv_bfloat16 *>(sm + kSmKV + (it % kKVStages) * 2 * kTileBytes);
-                    const __nv_bfloat16 *vt = kt + kC * kNC;
+                    const uint8_t *kt = sm + kSmKV + (it % kKVStages) * 2 * kTileBytes;
+                    const uint8_t *vt = kt + kTileBytes;
                     float2 lm[kMaxModes], acc[kMaxModes];
 #pragma unroll
                     for (int n = 0; n < kMaxModes; ++n) {
@@ -510,7 +535,9 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         acc[n] = make_float2(0.f, 0.f);
                     }
                     for (int io = 0; io < rem; ++io) {
-                        const float u = __bfloat162float(kt[io * kNC + c]) * __bfloat162float(vt[io * kNC + c]);
+                        const int o = act_off(io, c);
+                        const float u = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(kt + o)) *
+                                        __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(vt + o));
 #pragma unroll
                         for (int n = 0; n < kMaxModes; ++n)
                             acc[n] = make_float2(fmaf(acc[n].x, lm[n].x, fmaf(-acc[n].y, lm[n].y, u)),
@@ -530,7 +557,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 tc::tc_fence_after();
                 const int qs = j % kQStages;
                 if (!(ok = uni(tc::mbar_wait(bar(kBarQFull + qs), (j / kQStages) & 1, abort)))) break;
-                __nv_bfloat16 *qy = reinterpret_cast<__nv_bfloat16 *>(sm + kSmQ + qs * kTileBytes);
+                uint8_t *qy = sm + kSmQ + qs * kTileBytes;
 #pragma unroll
                 for (int k16 = 0; k16 < kC / 16; ++k16) {
                     float z[16];
@@ -539,7 +566,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
                     for (int t = 0; t < 16; ++t) {
                         const int tau = k16 * 16 + t;
-                        qy[tau * kNC + c] = __float2bfloat16_rn(__bfloat162float(qy[tau * kNC + c]) * z[t]);
+                        __nv_bfloat16 *e = reinterpret_cast<__nv_bfloat16 *>(qy + act_off(tau, c));
+                        *e = __float2bfloat16_rn(__bfloat162float(*e) * z[t]);
                     }
                 }
                 tc::tc_fence_before();
@@ -548,7 +576,9 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 if (c == 0) {
                     ok = tc::mbar_wait(bar(kBarYStaged), j & 1, abort);
                     if (ok) {
-                        tc::tma_store_3d(&tm_y, sbase + kSmQ + qs * kTileBytes, c0, chunk * kC, b);
+                        for (int h = 0; h < 2; ++h)
+                            tc::tma_store_3d(&tm_y, sbase + kSmQ + qs * kTileBytes + h * kHalfBytes, c0 + 64 * h,
+                                             chunk * kC, b);
                         tc::bulk_commit();
                         if (j >= 1) {
                             // the previous tile's store has read its buffer: hand it back to the q loader
@@ -596,10 +626,10 @@ bool make_map(CUtensorMap *m, const void *base, int B, int L, int Dch) {
     if (!enc) return false;
     cuuint64_t dims[3] = {(cuuint64_t)Dch, (cuuint64_t)L, (cuuint64_t)B};
     cuuint64_t strides[2] = {(cuuint64_t)Dch * 2, (cuuint64_t)L * Dch * 2};
-    cuuint32_t box[3] = {(cuuint32_t)kNC, (cuuint32_t)kC, 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)kC, 1};     // 64 channels = 128 bytes, the swizzle span
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -644,17 +674,17 @@ cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, 
                                    void *y, float *state_out, void *ws, cudaStream_t s) {
     const ChunkPlan p = plan(B, L, Dch, H, d);
     uint8_t *w = static_cast<uint8_t *>(ws);
-    const int KS = ((2 * d + 15) / 16) * 16;
+
     cudaError_t e = cudaMemsetAsync(w + p.sched_off, 0, p.agg_off - p.sched_off, s);
     if (e != cudaSuccess) return e;
-    chunk_consts_kernel<<<H, 256, 0, s>>>(lam, R, Dskip, d, KS, p.segc * kC, w + p.consts_off);
+    chunk_consts_kernel<<<H, 256, 0, s>>>(lam, R, Dskip, d, p.segc * kC, w + p.consts_off);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     CUtensorMap mq, mk, mv, my;
     if (!make_map(&mq, q, B, L, Dch) || !make_map(&mk, k, B, L, Dch) || !make_map(&mv, v, B, L, Dch) ||
         !make_map(&my, y, B, L, Dch))
         return cudaErrorInvalidValue;
     ChunkArgs a;
-    a.L = L; a.Dch = Dch; a.d = d; a.KS = KS; a.ch = Dch / H;
+    a.L = L; a.Dch = Dch; a.d = d; a.ch = Dch / H;
     a.ntiles = Dch / kNC; a.nchunks = p.nchunks; a.nseg = p.nseg; a.segc = p.segc;
     a.lam = lam;
     a.consts = w + p.consts_off;

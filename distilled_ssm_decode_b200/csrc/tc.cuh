@@ -172,6 +172,14 @@ __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Four 8x8 b16 matrices from shared memory, transposed: lane i supplies the row
+// address of row (i % 8) of matrix (i / 8); register m of lane t receives
+// elements (2(t%4), t/4) and (2(t%4)+1, t/4) of matrix m (low half first).
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t *r) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+
 // fp32 -> tf32 (round to nearest, ties away), kept in an fp32 container
 __device__ __forceinline__ float to_tf32(float x) {
     uint32_t r;
