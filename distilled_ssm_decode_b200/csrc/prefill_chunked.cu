@@ -61,8 +61,10 @@ constexpr int kIm = 16;
 constexpr int kThreads = 192;
 constexpr int kTileBytes = kC * kNC * 2;          // one bf16 [C][128] activation tile
 constexpr int kHalfBytes = kTileBytes / 2;        // [C][64] half tile = one TMA box, 128-byte swizzled
-constexpr int kKVStages = 4;                      // k,v prefetch depth (chunks)
-constexpr int kQStages = 4;                       // q (and staged y) buffers
+constexpr int kKVStages = 2;                      // k,v prefetch depth (chunks)
+constexpr int kQStages = 2;                       // q (and staged y) buffers
+constexpr int kSTBufs = 1;                        // state operand buffers
+constexpr int kCtasPerSM = 2;                     // two CTAs share an SM to hide each other's latency
 constexpr uint32_t kTmemCols = 128;               // D1 x2 (C cols each) + D2 x2 (32 each)
 
 // constant block per head (global, laid out exactly as in shared memory)
@@ -78,15 +80,15 @@ constexpr int kSmAT = kSmTT + kTTBytes;
 constexpr int kSmVT = kSmAT + kATBytes;
 constexpr int kSmUT = kSmVT + kVTBytes;                       // 2 x [128][C] tf32
 constexpr int kUTBytes = kNC * kC * 4;
-constexpr int kSmST = kSmUT + 2 * kUTBytes;                   // 2 x [128][KS] tf32
+constexpr int kSmST = kSmUT + 2 * kUTBytes;                   // kSTBufs x [128][32] tf32
 constexpr int kSTBytes = kNC * kKSMax * 4;
-constexpr int kSmKV = kSmST + 2 * kSTBytes;                   // kKVStages x {k, v}
+constexpr int kSmKV = kSmST + kSTBufs * kSTBytes;             // kKVStages x {k, v}
 constexpr int kSmQ = kSmKV + kKVStages * 2 * kTileBytes;      // kQStages x q (y staged in place)
 constexpr int kSmBar = kSmQ + kQStages * kTileBytes;
 constexpr int kNumBars = 27;
 constexpr int kSmMisc = kSmBar + kNumBars * 8;
 constexpr int kSmemBytes = kSmMisc + 64 + 1024;               // + misc words + alignment slack
-static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+static_assert(kSmemBytes * kCtasPerSM <= 228 * 1024, "shared memory budget");
 
 // barrier slots
 enum : int {
@@ -205,7 +207,7 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
 
 
 // ------------------------------------------------------------------ main kernel
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSM)
 prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_y,
                      const ChunkArgs a) {
@@ -249,7 +251,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         int4 *dst = reinterpret_cast<int4 *>(sm);
         for (int i = tid; i < (kTTBytes + kATBytes + kVTBytes) / 16; i += kThreads) dst[i] = __ldg(src + i);
         int4 *stz = reinterpret_cast<int4 *>(sm + kSmST);
-        for (int i = tid; i < 2 * kSTBytes / 16; i += kThreads) stz[i] = make_int4(0, 0, 0, 0);
+        for (int i = tid; i < kSTBufs * kSTBytes / 16; i += kThreads) stz[i] = make_int4(0, 0, 0, 0);
     }
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
@@ -331,7 +333,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     for (int ks = 0; ks < kC / 8; ++ks)
                         tc::mma_tf32(d1, tc::smem_desc(ut + ks * 256, 128, kC * 32),
                                      tc::smem_desc(sbase + kSmTT + ks * 256, 128, kC * 32), idesc_y, ks > 0);
-                    const uint32_t stb = sbase + kSmST + (j & 1) * kSTBytes;
+                    const uint32_t stb = sbase + kSmST + (j % kSTBufs) * kSTBytes;
                     for (int ks = 0; ks < kKSMax / 8; ++ks)
                         tc::mma_tf32(d1, tc::smem_desc(stb + ks * 256, 128, kKSMax * 32),
                                      tc::smem_desc(sbase + kSmAT + ks * 256, 128, kKSMax * 32), idesc_y, 1);
@@ -394,7 +396,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         };
         // state operand (tf32) for chunk j: column n real part, column 16 + n imaginary part
         auto write_state = [&](int j) {
-            uint8_t *stp = sm + kSmST + (j & 1) * kSTBytes;
+            uint8_t *stp = sm + kSmST + (j % kSTBufs) * kSTBytes;
 #pragma unroll
             for (int n4 = 0; n4 < kMaxModes / 4; ++n4) {
                 const int n = 4 * n4;
@@ -518,10 +520,10 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     if (!(ok = uni(make_u(it + 1, chunk + 1 != a.nchunks - 1)))) break;
                 }
                 if (chunk != a.nchunks - 1) {
-                    // state after this chunk, then the next chunk's state operand, so that the
-                    // next output product can start while this chunk is gated and stored
+                    // state after this chunk; the next chunk's state operand is written as soon as
+                    // the buffer is free (two buffers: now; one buffer: after this output product)
                     if (!(ok = uni(advance_state(it)))) break;
-                    if (j + 1 < nck) write_state(j + 1);
+                    if (kSTBufs == 2 && j + 1 < nck) write_state(j + 1);
                 } else {
                     // last chunk of the prompt (possibly partial): exact fp32 Horner over its
                     // tokens, st <- lambda^rem st + sum_{iota<rem} lambda^(rem-1-iota) u_iota
@@ -555,6 +557,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 // gate: y = q * D1, written in place of q, then one TMA store of the tile
                 if (!(ok = uni(tc::mbar_wait(bar(kBarYDone + (j & 1)), (j >> 1) & 1, abort)))) break;
                 tc::tc_fence_after();
+                if (kSTBufs == 1 && j + 1 < nck && chunk != a.nchunks - 1) write_state(j + 1);
                 const int qs = j % kQStages;
                 if (!(ok = uni(tc::mbar_wait(bar(kBarQFull + qs), (j / kQStages) & 1, abort)))) break;
                 uint8_t *qy = sm + kSmQ + qs * kTileBytes;
@@ -644,8 +647,8 @@ ChunkPlan plan(int B, int L, int Dch, int H, int d) {
     ChunkPlan p{};
     p.nchunks = (L + kC - 1) / kC;
     const long long units = (long long)B * (Dch / kNC);
-    // enough items for ~2 waves of one CTA per SM, segments of at least 4 chunks
-    long long want = (2 * 148 + units - 1) / units;
+    // enough items for ~2 waves of resident CTAs, segments of at least 4 chunks
+    long long want = (2 * 148 * kCtasPerSM + units - 1) / units;
     long long maxseg = (p.nchunks + 3) / 4;
     if (want > maxseg) want = maxseg;
     if (want < 1) want = 1;
