@@ -301,6 +301,25 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             if (*abort)
                 for (int jj = max(0, j - kQStages); jj < j; ++jj)
                     tc::mbar_wait(bar(kBarQFull + jj % kQStages), (jj / kQStages) & 1, never);
+        } else if (lane == 2) {     // y: TMA store of each gated tile, then the buffer goes back to q
+            int j = 0;
+            for (; j < nck; ++j) {
+                if (!tc::mbar_wait(bar(kBarYStaged), j & 1, abort)) {
+                    record_error(a, abort, kErrWait);
+                    break;
+                }
+                const int qs = j % kQStages;
+                for (int h = 0; h < 2; ++h)
+                    tc::tma_store_3d(&tm_y, sbase + kSmQ + qs * kTileBytes + h * kHalfBytes, c0 + 64 * h,
+                                     (ck0 + j) * kC, b);
+                tc::bulk_commit();
+                if (j >= 1) {
+                    // the previous tile's store has read its buffer: hand it back to the q loader
+                    tc::bulk_wait_read<1>();
+                    tc::mbar_arrive(bar(kBarQEmpty + (j - 1) % kQStages));
+                }
+            }
+            tc::bulk_wait<0>();     // every store of this CTA has completed
         }
     } else if (warp == 5) {
         // ------------------------------------------------------------ MMA issuer
@@ -561,6 +580,12 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int qs = j % kQStages;
                 if (!(ok = uni(tc::mbar_wait(bar(kBarQFull + qs), (j / kQStages) & 1, abort)))) break;
                 uint8_t *qy = sm + kSmQ + qs * kTileBytes;
+                // all q of this thread's channel into registers first (independent loads), then
+                // the products, then the stores over the same slots
+                __nv_bfloat16 qv[kC];
+#pragma unroll
+                for (int tau = 0; tau < kC; ++tau)
+                    qv[tau] = *reinterpret_cast<const __nv_bfloat16 *>(qy + act_off(tau, c));
 #pragma unroll
                 for (int k16 = 0; k16 < kC / 16; ++k16) {
                     float z[16];
@@ -569,31 +594,15 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
                     for (int t = 0; t < 16; ++t) {
                         const int tau = k16 * 16 + t;
-                        __nv_bfloat16 *e = reinterpret_cast<__nv_bfloat16 *>(qy + act_off(tau, c));
-                        *e = __float2bfloat16_rn(__bfloat162float(*e) * z[t]);
+                        *reinterpret_cast<__nv_bfloat16 *>(qy + act_off(tau, c)) =
+                            __float2bfloat16_rn(__bfloat162float(qv[tau]) * z[t]);
                     }
                 }
                 tc::tc_fence_before();
                 tc::fence_proxy_async_smem();
-                tc::mbar_arrive(bar(kBarYStaged));
-                if (c == 0) {
-                    ok = tc::mbar_wait(bar(kBarYStaged), j & 1, abort);
-                    if (ok) {
-                        for (int h = 0; h < 2; ++h)
-                            tc::tma_store_3d(&tm_y, sbase + kSmQ + qs * kTileBytes + h * kHalfBytes, c0 + 64 * h,
-                                             chunk * kC, b);
-                        tc::bulk_commit();
-                        if (j >= 1) {
-                            // the previous tile's store has read its buffer: hand it back to the q loader
-                            tc::bulk_wait_read<1>();
-                            tc::mbar_arrive(bar(kBarQEmpty + (j - 1) % kQStages));
-                        }
-                    }
-                }
-                if (!(ok = uni(ok))) break;
+                tc::mbar_arrive(bar(kBarYStaged));     // the store lane of warp 4 takes it from here
             }
             if (!ok) record_error(a, abort, kErrWait);
-            if (c == 0) tc::bulk_wait<0>();
             if (ok && last_seg) {
                 float2 *so = reinterpret_cast<float2 *>(a.state_out) + ((size_t)b * d) * a.Dch + c0 + c;
 #pragma unroll
