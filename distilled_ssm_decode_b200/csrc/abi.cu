@@ -70,6 +70,7 @@ const char *hyena_status_string(int status) {
         case HYENA_ERR_WORKSPACE: return "workspace missing or too small";
         case HYENA_ERR_UNSUPPORTED: return "size outside what this build implements";
         case HYENA_ERR_CUDA: return "CUDA launch or runtime error";
+        case HYENA_ERR_CAPACITY: return "problem needs more scratch than the library's built-in array holds";
         default: return "unknown status";
     }
 }

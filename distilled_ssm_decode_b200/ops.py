@@ -38,6 +38,9 @@ SIGNATURES = {
     "hyena_prefill_chunked_error_offset": (_sz, [_i, _i, _i, _i, _i]),
     "hyena_prefill_chunked": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp, _fp,
                                    _vp, _sz, _vp]),
+    "hyena_prefill_noalloc_capacity": (_sz, []),
+    "hyena_prefill_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp, _fp,
+                                   _vp]),
     "hyena_prompt_state_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "hyena_prompt_state": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _fp, _fp, _vp, _sz, _vp]),
     "hyena_decode_step": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _fp, _fp, _fp, _fp, _vp, _vp]),

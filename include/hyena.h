@@ -65,7 +65,8 @@ typedef enum {
     HYENA_ERR_ALIGN = -3,        /* pointer not aligned as the layout requires */
     HYENA_ERR_WORKSPACE = -4,    /* workspace NULL or smaller than the query says */
     HYENA_ERR_UNSUPPORTED = -5,  /* valid operator, size outside what this build implements */
-    HYENA_ERR_CUDA = -6          /* a CUDA launch/runtime call failed */
+    HYENA_ERR_CUDA = -6,         /* a CUDA launch/runtime call failed */
+    HYENA_ERR_CAPACITY = -7      /* problem needs more than the library's built-in scratch */
 } hyena_status;
 
 typedef enum {
@@ -137,6 +138,31 @@ int hyena_prefill(const void *q, const void *k, const void *v, int dtype,
                   const float *lambda, const float *R, const float *Dskip,
                   void *y, float *state_out,
                   void *workspace, size_t ws_bytes, hyena_stream_t stream);
+
+/*
+ * hyena_prefill without a caller-supplied workspace.  The pages have no
+ * counterpart to this entry point: it exists for callers that cannot allocate
+ * or pass device scratch where they call (a plugin or FFI layer that only sees
+ * the tensors it was given, a latency-critical loop that must not risk the
+ * device synchronisation of cudaMalloc/cudaFree, a fixed start-up memory
+ * budget).  It runs hyena_prefill with its scratch in a fixed array inside the
+ * library: hyena_prefill_noalloc_capacity() bytes (4 MiB), held on every GPU
+ * that loads the library until the process exits.
+ *   Arguments and results as hyena_prefill, minus the workspace.  It never
+ *   calls cudaMalloc, cudaFree or any allocating routine.
+ *   HYENA_ERR_CAPACITY when hyena_prefill_workspace_bytes(...) exceeds the
+ *   capacity (e.g. transforms longer than 16384 points).
+ *   The first call on each device looks up the array's device address (with
+ *   that device current) and may load the module there: make it before any
+ *   stream capture.  Every call uses the same array, so calls whose work
+ *   overlaps on the GPU (other streams, other host threads) race on it; the
+ *   caller must serialise them.  Nothing needs clearing between calls.
+ */
+size_t hyena_prefill_noalloc_capacity(void);
+int hyena_prefill_noalloc(const void *q, const void *k, const void *v, int dtype,
+                          int B, int L, int Dch, int H, int d, int fft_len,
+                          const float *lambda, const float *R, const float *Dskip,
+                          void *y, float *state_out, hyena_stream_t stream);
 
 /*
  * Prefill by chunked modal evaluation on the tensor cores: the same operator
