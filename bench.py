@@ -95,7 +95,8 @@ def source_hash(paths) -> str:
 
 
 def ncu_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch recorded from an ncu capture, if the kernel source is unchanged."""
+    """DRAM bytes per launch recorded from an ncu capture (profiles/traffic.json, keyed by
+    workload name and batch), or None if there is none or the kernel source changed since."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         d = json.load(open(p))[workload][kernel]
@@ -378,7 +379,7 @@ def run_ours(args):
                       "bound": "hbm", "achieved": pre_gbs, "peak": peak, "unit": "GB/s",
                       "frac": pre_gbs / peak, "peak_source": peak_src, "algorithmic_bytes": pb,
                       "launch_ms": pre_ms, "total_ms": pre_ms,
-                      "traffic": ncu_traffic("prefill_fused", w.name)})
+                      "traffic": ncu_traffic("prefill_fused", f"{w.name}/B{w.B}")})
         out_pre = {"tokens_per_s": world * w.B * w.L / (pre_ms / 1e3), "ms": pre_ms,
                    "hbm_frac": pre_gbs / peak}
     if has_dec:
@@ -388,12 +389,12 @@ def run_ours(args):
                       "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak,
                       "peak_source": peak_src, "algorithmic_bytes": db,
                       "launch_ms": dec_launch_ms, "total_ms": dec_ms,
-                      "traffic": ncu_traffic("decode", w.name)})
+                      "traffic": ncu_traffic("decode", f"{w.name}/B{w.B}")})
         out_dec = {"tokens_per_s": world * w.B * w.T / (dec_ms / 1e3),
                    "ms_per_token_step": dec_launch_ms, "hbm_frac": dec_gbs / peak}
     if use_chunked:
         roofs[0]["kernel"] = "hyena_prefill_chunked (tcgen05 chunked conv/gate/state)"
-        roofs[0]["traffic"] = ncu_traffic("prefill_chunk", w.name)
+        roofs[0]["traffic"] = ncu_traffic("prefill_chunk", f"{w.name}/B{w.B}")
         err = ops.chunked_error(ws_c, w.B, w.L, w.Dch, w.H, w.d)
         if err:
             raise SystemExit(f"chunked prefill kernel reported error {err}")
@@ -414,7 +415,7 @@ def run_ours(args):
         fft_route = {"kernel": "hyena_prefill (filter + spectrum + fused FFT conv/gate/state)",
                      "fft_len": w.fft_len, "tokens_per_s": world * w.B * w.L / (fms / 1e3),
                      "ms": fms, "achieved": fgbs, "frac": fgbs / peak, "unit": "GB/s",
-                     "traffic": ncu_traffic("prefill_fused", w.name)}
+                     "traffic": ncu_traffic("prefill_fused", f"{w.name}/B{w.B}")}
     dominant = max(roofs, key=lambda r: r["total_ms"])
 
     # ---- end to end: host (pinned) inputs, copies inside the timed region
