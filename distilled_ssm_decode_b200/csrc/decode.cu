@@ -14,8 +14,8 @@
 // consecutive threads take consecutive pairs, so each mode row is read as
 // contiguous 128-byte lines.  A thread's modes (up to 8 at a time) are loaded
 // before any arithmetic so that they are all in flight together.  When B * Dch is
-// small, NG threads share one pair (each takes every NG-th mode) and combine
-// their partial outputs with warp shuffles, so that small batches still put
+// very small, NG threads share one pair (each takes every NG-th mode) and combine
+// their partial outputs with warp shuffles, so that the few pairs still put
 // enough loads in flight to cover memory latency.
 #include "common.cuh"
 #include "kernels.h"
@@ -34,6 +34,11 @@ decode_vec_kernel(const typename Act::T *__restrict__ q, const typename Act::T *
                   const float2 *__restrict__ lam, const float2 *__restrict__ R,
                   const float *__restrict__ Dskip, float4 *__restrict__ state,
                   typename Act::T *__restrict__ y) {
+    // launched with programmatic stream serialisation: wait until the previous kernel in the
+    // stream (e.g. the previous decode step, which wrote this state) has completed, then let
+    // the next one start its launch while this one runs
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
     const int NG = 1 << lg_ng;
     const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long pair_id = gtid >> lg_ng;
@@ -119,25 +124,45 @@ decode_scalar_kernel(const typename Act::T *__restrict__ q, const typename Act::
     Act::st(y + o, Act::ld(q + o) * fmaf(__ldg(&Dskip[hd]), u, acc));
 }
 
-// Lanes per channel pair (NG) and modes per thread (MPT): enough threads to fill the GPU
-// (148 SMs x 2048), at most 16 lanes per pair, at most 8 modes in registers at once.
+// Lanes per channel pair (NG = 2^lg) and modes per thread (MPT), from a sweep on B200 of
+// one-token steps replayed from a CUDA graph (d = 16):
+//   4096 pairs:  NG = 8..16, MPT = 1 best (2.3 us); one lane per pair is 2.8x slower
+//   32768 pairs: NG = 1, MPT = 4 best (3.6 us); NG = 16 is 2.3x slower
+//   >= 65536:    NG = 1, MPT = 8 best (5.4 us at 65536 pairs, 44.5 us at 524288)
+// Splitting a pair's modes across lanes only pays when there are too few pairs to cover
+// the SMs at all.
 void choose_split(long long pairs, int d, int *lg_ng, int *mpt) {
-    const long long want = 148LL * 2048;
-    int lg = 0;
-    while ((pairs << lg) < want && (1 << (lg + 1)) <= 16 && (1 << (lg + 1)) <= d) ++lg;
-    int per = (d + (1 << lg) - 1) >> lg;        // modes per lane
-    int m = 1;
-    while (m < per && m < 8) m <<= 1;
+    int lg = 0, m = 8;
+    if (pairs < 8192) {
+        while ((1 << (lg + 1)) <= 16 && (1 << (lg + 1)) <= d) ++lg;   // up to 16 lanes, one mode each
+        m = 1;
+    } else if (pairs < 65536) {
+        m = 4;
+    }
+    while (m > 1 && m / 2 >= (d + (1 << lg) - 1) >> lg) m >>= 1;     // no more slots than modes
     *lg_ng = lg;
     *mpt = m;
 }
 
+// Launch with programmatic dependent launch: in a stream (or a graph captured from one) of
+// back-to-back decode steps, each step's grid is scheduled while the previous step runs; the
+// kernel's griddepcontrol.wait keeps the data ordering of an ordinary stream launch.
 template <class Act, int MPT>
 void launch_vec(unsigned blocks, cudaStream_t s, const typename Act::T *q, const typename Act::T *k,
                 const typename Act::T *v, int B, int Dch, int ch, int d, int lg, const float2 *lam,
                 const float2 *R, const float *Dskip, float *state, typename Act::T *y) {
-    decode_vec_kernel<Act, MPT><<<blocks, kThreads, 0, s>>>(q, k, v, B, Dch, ch, d, lg, lam, R, Dskip,
-                                                            reinterpret_cast<float4 *>(state), y);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, decode_vec_kernel<Act, MPT>, q, k, v, B, Dch, ch, d, lg, lam, R, Dskip,
+                       reinterpret_cast<float4 *>(state), y);
 }
 
 template <class Act>
