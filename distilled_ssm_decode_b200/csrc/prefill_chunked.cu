@@ -58,14 +58,19 @@ constexpr int kNC = 128;           // channels per tile (MMA M)
 constexpr int kMaxModes = 16;      // d <= 16
 constexpr int kKSMax = 32;         // state operand width: Re at [0,16), Im at [16,32)
 constexpr int kIm = 16;
-constexpr int kThreads = 192;
 constexpr int kTileBytes = kC * kNC * 2;          // one bf16 [C][128] activation tile
 constexpr int kHalfBytes = kTileBytes / 2;        // [C][64] half tile = one TMA box, 128-byte swizzled
-constexpr int kKVStages = 2;                      // k,v prefetch depth (chunks)
-constexpr int kQStages = 2;                       // q (and staged y) buffers
-constexpr int kSTBufs = 1;                        // state operand buffers
-constexpr int kCtasPerSM = 2;                     // two CTAs share an SM to hide each other's latency
-constexpr uint32_t kTmemCols = 128;               // D1 x2 (C cols each) + D2 x2 (32 each)
+// Ring depths.  A chunk's output product needs the U operand, the state operand and a D1
+// accumulator; each of those is refilled only after the product that used it completes, so a
+// ring of depth n lets n chunks be in flight between those round trips.
+constexpr int kKVStages = 3;                      // k,v tiles
+constexpr int kQStages = 4;                       // q tiles (y staged in place)
+constexpr int kUBufs = 4;                         // U operands
+constexpr int kSTBufs = 4;                        // state operands
+constexpr int kD1Bufs = 4;                        // output accumulators (TMEM)
+constexpr int kD2Bufs = 2;                        // state-product accumulators (TMEM)
+constexpr int kThreads = 512;                     // 16 warps, see the role map below
+constexpr uint32_t kTmemCols = 256;               // D1 (4 x C cols) + D2 (2 x 32 cols), rounded up
 
 // constant block per head (global, laid out exactly as in shared memory)
 constexpr int kTTBytes = kC * kC * 4;             // B operand of the Toeplitz product
@@ -78,32 +83,41 @@ constexpr int kConstStride = (kConstBytes + 255) & ~255;
 constexpr int kSmTT = 0;
 constexpr int kSmAT = kSmTT + kTTBytes;
 constexpr int kSmVT = kSmAT + kATBytes;
-constexpr int kSmUT = kSmVT + kVTBytes;                       // 2 x [128][C] tf32
+constexpr int kSmUT = kSmVT + kVTBytes;                       // kUBufs x [128][C] tf32
 constexpr int kUTBytes = kNC * kC * 4;
-constexpr int kSmST = kSmUT + 2 * kUTBytes;                   // kSTBufs x [128][32] tf32
+constexpr int kSmST = kSmUT + kUBufs * kUTBytes;              // kSTBufs x [128][32] tf32
 constexpr int kSTBytes = kNC * kKSMax * 4;
 constexpr int kSmKV = kSmST + kSTBufs * kSTBytes;             // kKVStages x {k, v}
 constexpr int kSmQ = kSmKV + kKVStages * 2 * kTileBytes;      // kQStages x q (y staged in place)
 constexpr int kSmBar = kSmQ + kQStages * kTileBytes;
-constexpr int kNumBars = 27;
+
+// barrier slots (arrival counts in parentheses; "commit" = tcgen05.commit from the MMA thread)
+enum : int {
+    kBarKVFull = 0,                              // [kKVStages] k,v tile landed (1 + tx)
+    kBarKVEmpty = kBarKVFull + kKVStages,        // [kKVStages] k,v consumed (128: U group, or S group for the prompt's last chunk)
+    kBarQFull = kBarKVEmpty + kKVStages,         // [kQStages] q tile landed (1 + tx)
+    kBarQEmpty = kBarQFull + kQStages,           // [kQStages] q/y buffer free (1: store warp)
+    kBarURdy = kBarQEmpty + kQStages,            // [kUBufs] U operand written (128: U group)
+    kBarUFree = kBarURdy + kUBufs,               // [kUBufs] U operand no longer read (commit)
+    kBarWDone = kBarUFree + kUBufs,              // [kD2Bufs] state product done (commit)
+    kBarD2Free = kBarWDone + kD2Bufs,            // [kD2Bufs] state product read out (128: S group)
+    kBarSRdy = kBarD2Free + kD2Bufs,             // [kSTBufs] state operand written (128: S group)
+    kBarSTFree = kBarSRdy + kSTBufs,             // [kSTBufs] state operand no longer read (commit)
+    kBarYDone = kBarSTFree + kSTBufs,            // [kD1Bufs] output product done (commit)
+    kBarD1Free = kBarYDone + kD1Bufs,            // [kD1Bufs] output product read out (128: E group)
+    kBarYStaged = kBarD1Free + kD1Bufs,          // [kQStages] gated tile staged for the store (128: E group)
+    kBarPub = kBarYStaged + kQStages,            // segment state written to global (128: S group)
+    kBarDrain = kBarPub + 1,                     // every MMA of the CTA finished (commit)
+    kNumBars = kBarDrain + 1
+};
 constexpr int kSmMisc = kSmBar + kNumBars * 8;
 constexpr int kSmemBytes = kSmMisc + 64 + 1024;               // + misc words + alignment slack
-static_assert(kSmemBytes * kCtasPerSM <= 228 * 1024, "shared memory budget");
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
-// barrier slots
-enum : int {
-    kBarKVFull = 0,    // [4] TMA k,v landed (1 arrival + tx)
-    kBarKVEmpty = 4,   // [4] k,v consumed (128)
-    kBarQFull = 8,     // [4] TMA q landed (1 + tx)
-    kBarQEmpty = 12,   // [4] q/y buffer free again (1)
-    kBarURdy = 16,     // [2] U operand written (128)
-    kBarSRdy = 18,     // [2] state operand written (128)
-    kBarWDone = 20,    // [2] state product done (commit)
-    kBarYDone = 22,    // [2] output product done (commit)
-    kBarYStaged = 24,  // gated output staged for the store (128)
-    kBarPub = 25,      // segment state written to global (128)
-    kBarDrain = 26     // every MMA of the CTA finished (commit)
-};
+__host__ __device__ constexpr int bar_count(int i) {
+    return ((i >= kBarKVEmpty && i < kBarQFull) || (i >= kBarURdy && i < kBarUFree) ||
+            (i >= kBarD2Free && i < kBarSTFree) || (i >= kBarD1Free && i < kBarDrain)) ? 128 : 1;
+}
 
 // byte offset of element (row, k) in a K-major, no-swizzle core-matrix tile whose K extent is K
 __host__ __device__ __forceinline__ int cm_off(int row, int k, int K) {
@@ -207,7 +221,15 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
 
 
 // ------------------------------------------------------------------ main kernel
-__global__ void __launch_bounds__(kThreads, kCtasPerSM)
+// Roles (warps):  0-3  U group: u = k*v -> U operand (ldmatrix transpose), one chunk at a time
+//                 4-7  S group: one thread per channel; state chain, segment publish, look-back
+//                 8-11 E group: one thread per channel; gate y = q * D1, stage y for the store
+//                 12   k,v TMA loads    13  q TMA loads    14  y TMA stores (lane 0 each; a
+//                      warp of their own so that one role's blocking wait never holds another)
+//                 15   tensor memory owner and MMA issuer (lane 0)
+// The groups run their own loops over the same chunk sequence and meet only at mbarriers, so
+// the U group forms chunk i+1 while the S group advances chunk i and the E group gates i-1.
+__global__ void __launch_bounds__(kThreads, 1)
 prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_y,
                      const ChunkArgs a) {
@@ -224,12 +246,10 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         misc[0] = atomicAdd(a.sched, 1);
         misc[1] = 0;
         misc[3] = 0;
-        const int counts[kNumBars] = {1, 1, 1, 1, 128, 128, 128, 128, 1, 1, 1, 1, 1, 1, 1, 1,
-                                      128, 128, 128, 128, 1, 1, 1, 1, 128, 128, 1};
-        for (int i = 0; i < kNumBars; ++i) tc::mbar_init(bar(i), counts[i]);
+        for (int i = 0; i < kNumBars; ++i) tc::mbar_init(bar(i), bar_count(i));
         tc::fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 15) {
         tc::tmem_alloc(tc::smem_u32((const void *)(misc + 2)), kTmemCols);
         tc::tmem_relinquish();
     }
@@ -243,9 +263,10 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const bool last_seg = (seg == a.nseg - 1);
     const bool phase1 = !last_seg;
     const int n1 = phase1 ? nck : 0;                  // state-only iterations
+    const int niter = n1 + nck;
     const int d = a.d;
 
-    // per-head constants -> shared memory; zero the state operand (its padding columns stay 0)
+    // per-head constants -> shared memory; zero the state operands (their padding columns stay 0)
     {
         const int4 *src = reinterpret_cast<const int4 *>(a.consts + (size_t)hd * kConstStride);
         int4 *dst = reinterpret_cast<int4 *>(sm);
@@ -258,34 +279,31 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = (uint32_t)misc[2];
+    auto chunk_of = [&](int it) { return ck0 + (it < n1 ? it : it - n1); };
+    auto uni = [&](bool x) -> bool { return __all_sync(0xffffffffu, x && !*abort); };
 
-    if (warp == 4) {
-        // ------------------------------------------------------------ TMA producers
-        if (lane == 0) {            // k, v for every iteration (state-only pass, then full pass)
-            tc::prefetch_tensormap(&tm_k);
-            tc::prefetch_tensormap(&tm_v);
+    if (warp >= 12 && warp <= 14) {
+        // ------------------------------------------------------------ TMA warps
+        if (warp == 12 && lane == 0) {      // k, v for every iteration (state-only pass, then full pass)
             int it = 0;
-            for (; it < n1 + nck; ++it) {
+            for (; it < niter; ++it) {
                 const int s = it % kKVStages;
                 if (!tc::mbar_wait(bar(kBarKVEmpty + s), ((it / kKVStages) & 1) ^ 1, abort)) {
                     record_error(a, abort, kErrWait);
                     break;
                 }
-                const int chunk = ck0 + (it < n1 ? it : it - n1);
                 const uint32_t dst = sbase + kSmKV + s * 2 * kTileBytes;
+                const int t0 = chunk_of(it) * kC;
                 tc::mbar_expect_tx(bar(kBarKVFull + s), 2 * kTileBytes);
                 for (int h = 0; h < 2; ++h) {
-                    tc::tma_load_3d(dst + h * kHalfBytes, &tm_k, bar(kBarKVFull + s), c0 + 64 * h, chunk * kC, b);
-                    tc::tma_load_3d(dst + kTileBytes + h * kHalfBytes, &tm_v, bar(kBarKVFull + s), c0 + 64 * h,
-                                    chunk * kC, b);
+                    tc::tma_load_3d(dst + h * kHalfBytes, &tm_k, bar(kBarKVFull + s), c0 + 64 * h, t0, b);
+                    tc::tma_load_3d(dst + kTileBytes + h * kHalfBytes, &tm_v, bar(kBarKVFull + s), c0 + 64 * h, t0, b);
                 }
             }
             if (*abort)
                 for (int j = max(0, it - kKVStages); j < it; ++j)
                     tc::mbar_wait(bar(kBarKVFull + j % kKVStages), (j / kKVStages) & 1, never);
-        } else if (lane == 1) {     // q for the full pass (the buffer also stages y)
-            tc::prefetch_tensormap(&tm_q);
-            tc::prefetch_tensormap(&tm_y);
+        } else if (warp == 13 && lane == 0) {   // q for the full pass (the buffer then stages y)
             int j = 0;
             for (; j < nck; ++j) {
                 const int s = j % kQStages;
@@ -301,100 +319,87 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             if (*abort)
                 for (int jj = max(0, j - kQStages); jj < j; ++jj)
                     tc::mbar_wait(bar(kBarQFull + jj % kQStages), (jj / kQStages) & 1, never);
-        } else if (lane == 2) {     // y: TMA store of each gated tile, then the buffer goes back to q
-            int j = 0;
-            for (; j < nck; ++j) {
-                if (!tc::mbar_wait(bar(kBarYStaged), j & 1, abort)) {
+        } else if (warp == 14 && lane == 0) {   // y: one TMA store per gated tile, then the buffer goes back to q
+            for (int j = 0; j < nck; ++j) {
+                const int s = j % kQStages;
+                if (!tc::mbar_wait(bar(kBarYStaged + s), (j / kQStages) & 1, abort)) {
                     record_error(a, abort, kErrWait);
                     break;
                 }
-                const int qs = j % kQStages;
                 for (int h = 0; h < 2; ++h)
-                    tc::tma_store_3d(&tm_y, sbase + kSmQ + qs * kTileBytes + h * kHalfBytes, c0 + 64 * h,
+                    tc::tma_store_3d(&tm_y, sbase + kSmQ + s * kTileBytes + h * kHalfBytes, c0 + 64 * h,
                                      (ck0 + j) * kC, b);
                 tc::bulk_commit();
-                if (j >= 1) {
-                    // the previous tile's store has read its buffer: hand it back to the q loader
-                    tc::bulk_wait_read<1>();
-                    tc::mbar_arrive(bar(kBarQEmpty + (j - 1) % kQStages));
-                }
+                tc::bulk_wait_read<0>();
+                tc::mbar_arrive(bar(kBarQEmpty + s));
             }
             tc::bulk_wait<0>();     // every store of this CTA has completed
         }
-    } else if (warp == 5) {
+    } else if (warp == 15) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc_y = tc::idesc_tf32(kNC, kC);
             const uint32_t idesc_w = tc::idesc_tf32(kNC, kKSMax);
-            for (int it = 0; it < n1 + nck && !*abort; ++it) {
-                const int ub = it & 1;
+            for (int it = 0; it < niter && !*abort; ++it) {
+                const int ub = it % kUBufs, wb = it % kD2Bufs;
                 const uint32_t ut = sbase + kSmUT + ub * kUTBytes;
-                if (!tc::mbar_wait(bar(kBarURdy + ub), (it >> 1) & 1, abort)) {
+                if (!tc::mbar_wait(bar(kBarURdy + ub), (it / kUBufs) & 1, abort) ||
+                    !tc::mbar_wait(bar(kBarD2Free + wb), ((it / kD2Bufs) & 1) ^ 1, abort)) {
                     record_error(a, abort, kErrWait);
                     break;
                 }
                 tc::tc_fence_after();
                 // D2 = U V^T: the chunk's contribution to the state
-                const uint32_t d2 = tmem + 2 * kC + ub * kKSMax;
+                const uint32_t d2 = tmem + kD1Bufs * kC + wb * kKSMax;
                 for (int ks = 0; ks < kC / 8; ++ks)
                     tc::mma_tf32(d2, tc::smem_desc(ut + ks * 256, 128, kC * 32),
                                  tc::smem_desc(sbase + kSmVT + ks * 256, 128, kC * 32), idesc_w, ks > 0);
-                tc::mma_commit(bar(kBarWDone + ub));
+                tc::mma_commit(bar(kBarWDone + wb));
                 if (it >= n1) {
-                    const int j = it - n1;
-                    if (!tc::mbar_wait(bar(kBarSRdy + (j & 1)), (j >> 1) & 1, abort)) {
+                    const int j = it - n1, sb = j % kSTBufs, db = j % kD1Bufs;
+                    if (!tc::mbar_wait(bar(kBarSRdy + sb), (j / kSTBufs) & 1, abort) ||
+                        !tc::mbar_wait(bar(kBarD1Free + db), ((j / kD1Bufs) & 1) ^ 1, abort)) {
                         record_error(a, abort, kErrWait);
                         break;
                     }
                     tc::tc_fence_after();
                     // D1 = U T^T + S A^T: intra-chunk Toeplitz product plus the modal carry
-                    const uint32_t d1 = tmem + (j & 1) * kC;
+                    const uint32_t d1 = tmem + db * kC;
+                    const uint32_t stb = sbase + kSmST + sb * kSTBytes;
                     for (int ks = 0; ks < kC / 8; ++ks)
                         tc::mma_tf32(d1, tc::smem_desc(ut + ks * 256, 128, kC * 32),
                                      tc::smem_desc(sbase + kSmTT + ks * 256, 128, kC * 32), idesc_y, ks > 0);
-                    const uint32_t stb = sbase + kSmST + (j % kSTBufs) * kSTBytes;
                     for (int ks = 0; ks < kKSMax / 8; ++ks)
                         tc::mma_tf32(d1, tc::smem_desc(stb + ks * 256, 128, kKSMax * 32),
                                      tc::smem_desc(sbase + kSmAT + ks * 256, 128, kKSMax * 32), idesc_y, 1);
-                    tc::mma_commit(bar(kBarYDone + (j & 1)));
+                    tc::mma_commit(bar(kBarYDone + db));
+                    tc::mma_commit(bar(kBarSTFree + sb));
                 }
+                tc::mma_commit(bar(kBarUFree + ub));
             }
+            // all MMAs issued by this thread have completed once `drain` fires
             tc::mma_commit(bar(kBarDrain));
             tc::mbar_wait(bar(kBarDrain), 0, never);
         }
-    } else {
-        // ------------------------------------------------------------ compute warps
-        const int c = tid;                        // channel within the tile == TMEM lane
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const float2 *lamC = reinterpret_cast<const float2 *>(a.consts + (size_t)hd * kConstStride +
-                                                              kTTBytes + kATBytes + kVTBytes);
-        const float2 *lamS = lamC + kMaxModes;
-        float2 lc[kMaxModes], st[kMaxModes];
-#pragma unroll
-        for (int n = 0; n < kMaxModes; ++n) {
-            lc[n] = n < d ? __ldg(&lamC[n]) : make_float2(0.f, 0.f);
-            st[n] = make_float2(0.f, 0.f);
-        }
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ U group
+        // u = k*v of each chunk -> U operand buffer (it % kUBufs).  ldmatrix transposes the
+        // 128-byte-swizzled k, v tiles: warp w covers channel groups 4w..4w+3 (8 channels each)
+        // and each lane receives token pairs of one channel, the K-major row layout of U.
+        // Tokens past the prompt were zero-filled by TMA.
         bool ok = true;
-        int pub_phase = 0;
-        // keep every compute warp converged (tcgen05.ld is warp-collective): a step
-        // counts as done only if all 32 lanes finished it and nobody aborted
-        auto uni = [&](bool x) -> bool { return __all_sync(0xffffffffu, x && !*abort); };
-
-        // u = k*v of the chunk in kv stage -> U operand buffer (it & 1).  The k, v tiles are
-        // transposed on the way with ldmatrix: warp w covers channel groups 4w..4w+3 (8 channels
-        // each), and each lane receives token pairs of one channel, which is exactly the
-        // K-major row layout of the U operand.  Tokens past the prompt were zero-filled by TMA.
-        auto make_u = [&](int it, bool release) -> bool {
-            if (!tc::mbar_wait(bar(kBarKVFull + it % kKVStages), (it / kKVStages) & 1, abort)) return false;
-            const uint32_t kb = sbase + kSmKV + (it % kKVStages) * 2 * kTileBytes;
-            uint8_t *ut = sm + kSmUT + (it & 1) * kUTBytes;
-            const int r8 = lane & 7, mat = lane >> 3;
+        const int r8 = lane & 7, mat = lane >> 3;
+        for (int it = 0; it < niter && ok; ++it) {
+            const int ub = it % kUBufs, s = it % kKVStages;
+            ok = uni(tc::mbar_wait(bar(kBarUFree + ub), ((it / kUBufs) & 1) ^ 1, abort) &&
+                     tc::mbar_wait(bar(kBarKVFull + s), (it / kKVStages) & 1, abort));
+            if (!ok) break;
+            const uint32_t kb = sbase + kSmKV + s * 2 * kTileBytes;
+            uint8_t *ut = sm + kSmUT + ub * kUTBytes;
 #pragma unroll
             for (int gi = 0; gi < 4; ++gi) {
-                const int g = 4 * warp + gi, cbase = 8 * g;
-                const int tau_row = 8 * mat + r8;               // row address supplied by this lane
-                const uint32_t off = (uint32_t)((cbase >> 6) * kHalfBytes + tau_row * 128 +
+                const int cbase = 8 * (4 * warp + gi);
+                const uint32_t off = (uint32_t)((cbase >> 6) * kHalfBytes + (8 * mat + r8) * 128 +
                                                 ((((cbase & 63) >> 3) ^ r8) << 4));
                 uint32_t kr[4], vr[4];
                 tc::ldsm_x4_trans(kb + off, kr);
@@ -409,77 +414,70 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 }
             }
             tc::fence_proxy_async_smem();
-            tc::mbar_arrive(bar(kBarURdy + (it & 1)));
-            if (release) tc::mbar_arrive(bar(kBarKVEmpty + it % kKVStages));
-            return true;
-        };
-        // state operand (tf32) for chunk j: column n real part, column 16 + n imaginary part
-        auto write_state = [&](int j) {
-            uint8_t *stp = sm + kSmST + (j % kSTBufs) * kSTBytes;
+            tc::mbar_arrive(bar(kBarURdy + ub));
+            // the prompt's last chunk stays until the S group has read it for the final state
+            if (!(it >= n1 && chunk_of(it) == a.nchunks - 1)) tc::mbar_arrive(bar(kBarKVEmpty + s));
+        }
+        if (!ok) record_error(a, abort, kErrWait);
+    } else if (warp < 8) {
+        // ------------------------------------------------------------ S group (state chain)
+        const int c = tid - 128;                     // channel within the tile == TMEM lane
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const float2 *lamC = reinterpret_cast<const float2 *>(a.consts + (size_t)hd * kConstStride +
+                                                              kTTBytes + kATBytes + kVTBytes);
+        const float2 *lamS = lamC + kMaxModes;
+        float2 lc[kMaxModes], st[kMaxModes];
 #pragma unroll
-            for (int n4 = 0; n4 < kMaxModes / 4; ++n4) {
-                const int n = 4 * n4;
-                *reinterpret_cast<float4 *>(stp + cm_off(c, n, kKSMax)) =
-                    make_float4(tc::to_tf32(st[n].x), tc::to_tf32(st[n + 1].x), tc::to_tf32(st[n + 2].x),
-                                tc::to_tf32(st[n + 3].x));
-                *reinterpret_cast<float4 *>(stp + cm_off(c, kIm + n, kKSMax)) =
-                    make_float4(tc::to_tf32(st[n].y), tc::to_tf32(st[n + 1].y), tc::to_tf32(st[n + 2].y),
-                                tc::to_tf32(st[n + 3].y));
-            }
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(bar(kBarSRdy + (j & 1)));
-        };
+        for (int n = 0; n < kMaxModes; ++n) {
+            lc[n] = n < d ? __ldg(&lamC[n]) : make_float2(0.f, 0.f);
+            st[n] = make_float2(0.f, 0.f);
+        }
+        bool ok = true;
+        int pub_phase = 0;
         // st <- lambda^C st + D2 of iteration it
-        auto advance_state = [&](int it) -> bool {
-            if (!tc::mbar_wait(bar(kBarWDone + (it & 1)), (it >> 1) & 1, abort)) return false;
+        auto advance = [&](int it) -> bool {
+            const int wb = it % kD2Bufs;
+            if (!tc::mbar_wait(bar(kBarWDone + wb), (it / kD2Bufs) & 1, abort)) return false;
             tc::tc_fence_after();
             float w[kKSMax];
-            const uint32_t taddr = tmem + lane_base + 2 * kC + (it & 1) * kKSMax;
+            const uint32_t taddr = tmem + lane_base + kD1Bufs * kC + wb * kKSMax;
             tc::tmem_ld16(taddr, w);
             tc::tmem_ld16(taddr + 16, w + 16);
             tc::tmem_wait_ld();
             tc::tc_fence_before();
+            tc::mbar_arrive(bar(kBarD2Free + wb));
 #pragma unroll
             for (int n = 0; n < kMaxModes; ++n) {
-                if (n < d) {
-                    const float2 s = st[n];
-                    st[n] = make_float2(fmaf(lc[n].x, s.x, fmaf(-lc[n].y, s.y, w[n])),
-                                        fmaf(lc[n].x, s.y, fmaf(lc[n].y, s.x, w[kIm + n])));
-                }
+                const float2 sv = st[n];
+                st[n] = make_float2(fmaf(lc[n].x, sv.x, fmaf(-lc[n].y, sv.y, w[n])),
+                                    fmaf(lc[n].x, sv.y, fmaf(lc[n].y, sv.x, w[kIm + n])));
             }
             return true;
         };
-        // publish st to global for other items, then set the status word
         auto publish = [&](float2 *dst, int code) -> bool {
-#pragma unroll
-            for (int n = 0; n < kMaxModes; ++n)
-                if (n < d) dst[(size_t)n * kNC + c] = st[n];
+            for (int n = 0; n < d; ++n) dst[(size_t)n * kNC + c] = st[n];
             __threadfence();
             tc::mbar_arrive(bar(kBarPub));
+            bool r = true;
             if (c == 0) {
-                if (!tc::mbar_wait(bar(kBarPub), pub_phase & 1, abort)) return false;
-                __threadfence();
-                atomicExch(a.status + item, code);
+                r = tc::mbar_wait(bar(kBarPub), pub_phase & 1, abort);
+                if (r) {
+                    __threadfence();
+                    atomicExch(a.status + item, code);
+                }
             }
             ++pub_phase;
-            return true;
+            return r;
         };
 
-        // ---------------- state-only pass over the segment
-        if (phase1) {
-            ok = uni(make_u(0, true));
-            for (int i = 0; i < nck && ok; ++i) {
-                if (i + 1 < nck) ok = uni(make_u(i + 1, true));
-                if (ok) ok = uni(advance_state(i));
-            }
-            if (ok) ok = uni(publish((seg == 0 ? a.inc : a.agg) + (size_t)item * d * kNC, seg == 0 ? 2 : 1));
-            if (!ok) record_error(a, abort, kErrWait);
-        }
+        // state-only pass over the segment, then publish its contribution
+        for (int it = 0; it < n1 && ok; ++it) ok = uni(advance(it));
+        if (ok && phase1) ok = uni(publish((seg == 0 ? a.inc : a.agg) + (size_t)item * d * kNC, seg == 0 ? 2 : 1));
         float2 sloc[kMaxModes];
 #pragma unroll
         for (int n = 0; n < kMaxModes; ++n) { sloc[n] = st[n]; st[n] = make_float2(0.f, 0.f); }
 
-        // ---------------- look-back: the state entering this segment
+        // look-back: the state entering this segment
         if (ok && seg > 0) {
             float2 lsg[kMaxModes], scale[kMaxModes];
 #pragma unroll
@@ -511,6 +509,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 }
                 if (code == 2) break;
             }
+            ok = uni(ok);
             if (ok && phase1) {
                 // inclusive state at the end of this segment: lambda^Lseg s_in + own contribution
                 float2 keep[kMaxModes];
@@ -519,104 +518,104 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     keep[n] = st[n];
                     st[n] = cadd(cmul(lsg[n], st[n]), sloc[n]);
                 }
-                ok = publish(a.inc + (size_t)item * d * kNC, 2);
+                ok = uni(publish(a.inc + (size_t)item * d * kNC, 2));
 #pragma unroll
                 for (int n = 0; n < kMaxModes; ++n) st[n] = keep[n];
-                if (!ok) record_error(a, abort, kErrWait);
             }
         }
-        ok = uni(ok);
 
-        // ---------------- full pass: outputs and state, starting from st = state entering the segment
-        if (ok) {
-            const int it0 = n1;
-            ok = uni(make_u(it0, ck0 != a.nchunks - 1));
-            if (ok) write_state(0);
-            for (int j = 0; j < nck && ok; ++j) {
-                const int it = it0 + j, chunk = ck0 + j;
-                // next chunk's U operand (its buffer was freed when chunk j-1's products finished)
-                if (j + 1 < nck) {
-                    if (!(ok = uni(make_u(it + 1, chunk + 1 != a.nchunks - 1)))) break;
-                }
-                if (chunk != a.nchunks - 1) {
-                    // state after this chunk; the next chunk's state operand is written as soon as
-                    // the buffer is free (two buffers: now; one buffer: after this output product)
-                    if (!(ok = uni(advance_state(it)))) break;
-                    if (kSTBufs == 2 && j + 1 < nck) write_state(j + 1);
-                } else {
-                    // last chunk of the prompt (possibly partial): exact fp32 Horner over its
-                    // tokens, st <- lambda^rem st + sum_{iota<rem} lambda^(rem-1-iota) u_iota
-                    const int rem = a.L - chunk * kC;
-                    const uint8_t *kt = sm + kSmKV + (it % kKVStages) * 2 * kTileBytes;
-                    const uint8_t *vt = kt + kTileBytes;
-                    float2 lm[kMaxModes], acc[kMaxModes];
+        // full pass: state operand for each chunk, then the state after it
+        for (int j = 0; j < nck && ok; ++j) {
+            const int it = n1 + j, sb = j % kSTBufs;
+            if (!(ok = uni(tc::mbar_wait(bar(kBarSTFree + sb), ((j / kSTBufs) & 1) ^ 1, abort)))) break;
+            uint8_t *stp = sm + kSmST + sb * kSTBytes;
 #pragma unroll
-                    for (int n = 0; n < kMaxModes; ++n) {
-                        lm[n] = n < d ? __ldg(&a.lam[(size_t)hd * d + n]) : make_float2(0.f, 0.f);
-                        acc[n] = make_float2(0.f, 0.f);
-                    }
-                    for (int io = 0; io < rem; ++io) {
-                        const int o = act_off(io, c);
-                        const float u = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(kt + o)) *
-                                        __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(vt + o));
-#pragma unroll
-                        for (int n = 0; n < kMaxModes; ++n)
-                            acc[n] = make_float2(fmaf(acc[n].x, lm[n].x, fmaf(-acc[n].y, lm[n].y, u)),
-                                                 fmaf(acc[n].x, lm[n].y, acc[n].y * lm[n].x));
-                    }
-                    tc::mbar_arrive(bar(kBarKVEmpty + it % kKVStages));
-#pragma unroll
-                    for (int n = 0; n < kMaxModes; ++n) {
-                        if (n < d) {
-                            const cd pw = cdpow(cd{lm[n].x, lm[n].y}, rem);
-                            st[n] = cadd(cmul(make_float2((float)pw.x, (float)pw.y), st[n]), acc[n]);
-                        }
-                    }
-                }
-                // gate: y = q * D1, written in place of q, then one TMA store of the tile
-                if (!(ok = uni(tc::mbar_wait(bar(kBarYDone + (j & 1)), (j >> 1) & 1, abort)))) break;
-                tc::tc_fence_after();
-                if (kSTBufs == 1 && j + 1 < nck && chunk != a.nchunks - 1) write_state(j + 1);
-                const int qs = j % kQStages;
-                if (!(ok = uni(tc::mbar_wait(bar(kBarQFull + qs), (j / kQStages) & 1, abort)))) break;
-                uint8_t *qy = sm + kSmQ + qs * kTileBytes;
-                // all q of this thread's channel into registers first (independent loads), then
-                // the products, then the stores over the same slots
-                __nv_bfloat16 qv[kC];
-#pragma unroll
-                for (int tau = 0; tau < kC; ++tau)
-                    qv[tau] = *reinterpret_cast<const __nv_bfloat16 *>(qy + act_off(tau, c));
-#pragma unroll
-                for (int k16 = 0; k16 < kC / 16; ++k16) {
-                    float z[16];
-                    tc::tmem_ld16(tmem + lane_base + (j & 1) * kC + k16 * 16, z);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int t = 0; t < 16; ++t) {
-                        const int tau = k16 * 16 + t;
-                        *reinterpret_cast<__nv_bfloat16 *>(qy + act_off(tau, c)) =
-                            __float2bfloat16_rn(__bfloat162float(qv[tau]) * z[t]);
-                    }
-                }
-                tc::tc_fence_before();
-                tc::fence_proxy_async_smem();
-                tc::mbar_arrive(bar(kBarYStaged));     // the store lane of warp 4 takes it from here
+            for (int n4 = 0; n4 < kMaxModes / 4; ++n4) {
+                const int n = 4 * n4;
+                *reinterpret_cast<float4 *>(stp + cm_off(c, n, kKSMax)) =
+                    make_float4(tc::to_tf32(st[n].x), tc::to_tf32(st[n + 1].x), tc::to_tf32(st[n + 2].x),
+                                tc::to_tf32(st[n + 3].x));
+                *reinterpret_cast<float4 *>(stp + cm_off(c, kIm + n, kKSMax)) =
+                    make_float4(tc::to_tf32(st[n].y), tc::to_tf32(st[n + 1].y), tc::to_tf32(st[n + 2].y),
+                                tc::to_tf32(st[n + 3].y));
             }
-            if (!ok) record_error(a, abort, kErrWait);
-            if (ok && last_seg) {
-                float2 *so = reinterpret_cast<float2 *>(a.state_out) + ((size_t)b * d) * a.Dch + c0 + c;
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(bar(kBarSRdy + sb));
+            const int chunk = ck0 + j;
+            if (chunk != a.nchunks - 1) {
+                if (!(ok = uni(advance(it)))) break;
+            } else {
+                // last chunk of the prompt (possibly partial): exact fp32 Horner over its
+                // tokens, st <- lambda^rem st + sum_{iota<rem} lambda^(rem-1-iota) u_iota
+                const int s = it % kKVStages;
+                if (!(ok = uni(tc::mbar_wait(bar(kBarKVFull + s), (it / kKVStages) & 1, abort)))) break;
+                const int rem = a.L - chunk * kC;
+                const uint8_t *kt = sm + kSmKV + s * 2 * kTileBytes;
+                const uint8_t *vt = kt + kTileBytes;
+                float2 lm[kMaxModes], acc[kMaxModes];
 #pragma unroll
-                for (int n = 0; n < kMaxModes; ++n)
-                    if (n < d) so[(size_t)n * a.Dch] = st[n];
+                for (int n = 0; n < kMaxModes; ++n) {
+                    lm[n] = n < d ? __ldg(&a.lam[(size_t)hd * d + n]) : make_float2(0.f, 0.f);
+                    acc[n] = make_float2(0.f, 0.f);
+                }
+                for (int io = 0; io < rem; ++io) {
+                    const int o = act_off(io, c);
+                    const float u = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(kt + o)) *
+                                    __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(vt + o));
+#pragma unroll
+                    for (int n = 0; n < kMaxModes; ++n)
+                        acc[n] = make_float2(fmaf(acc[n].x, lm[n].x, fmaf(-acc[n].y, lm[n].y, u)),
+                                             fmaf(acc[n].x, lm[n].y, acc[n].y * lm[n].x));
+                }
+                tc::mbar_arrive(bar(kBarKVEmpty + s));
+#pragma unroll
+                for (int n = 0; n < kMaxModes; ++n) {
+                    if (n < d) {
+                        const cd pw = cdpow(cd{lm[n].x, lm[n].y}, rem);
+                        st[n] = cadd(cmul(make_float2((float)pw.x, (float)pw.y), st[n]), acc[n]);
+                    }
+                }
             }
-        } else {
-            record_error(a, abort, kErrWait);
         }
+        if (!ok) record_error(a, abort, kErrWait);
+        if (ok && last_seg) {
+            float2 *so = reinterpret_cast<float2 *>(a.state_out) + ((size_t)b * d) * a.Dch + c0 + c;
+            for (int n = 0; n < d; ++n) so[(size_t)n * a.Dch] = st[n];
+        }
+    } else {
+        // ------------------------------------------------------------ E group (gate and stage y)
+        const int c = tid - 256;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        bool ok = true;
+        for (int j = 0; j < nck && ok; ++j) {
+            const int db = j % kD1Bufs, s = j % kQStages;
+            ok = uni(tc::mbar_wait(bar(kBarYDone + db), (j / kD1Bufs) & 1, abort) &&
+                     tc::mbar_wait(bar(kBarQFull + s), (j / kQStages) & 1, abort));
+            if (!ok) break;
+            tc::tc_fence_after();
+            uint8_t *qy = sm + kSmQ + s * kTileBytes;
+            __nv_bfloat16 qv[kC];
+#pragma unroll
+            for (int tau = 0; tau < kC; ++tau) qv[tau] = *reinterpret_cast<const __nv_bfloat16 *>(qy + act_off(tau, c));
+            float z[kC];
+            tc::tmem_ld16(tmem + lane_base + db * kC, z);
+            tc::tmem_ld16(tmem + lane_base + db * kC + 16, z + 16);
+            tc::tmem_wait_ld();
+            tc::tc_fence_before();
+            tc::mbar_arrive(bar(kBarD1Free + db));
+#pragma unroll
+            for (int tau = 0; tau < kC; ++tau)
+                *reinterpret_cast<__nv_bfloat16 *>(qy + act_off(tau, c)) =
+                    __float2bfloat16_rn(__bfloat162float(qv[tau]) * z[tau]);
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(bar(kBarYStaged + s));
+        }
+        if (!ok) record_error(a, abort, kErrWait);
     }
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    if (warp == 5) tc::tmem_dealloc(tmem, kTmemCols);
+    if (warp == 15) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
 // ------------------------------------------------------------------ host side
@@ -656,8 +655,8 @@ ChunkPlan plan(int B, int L, int Dch, int H, int d) {
     ChunkPlan p{};
     p.nchunks = (L + kC - 1) / kC;
     const long long units = (long long)B * (Dch / kNC);
-    // enough items for ~2 waves of resident CTAs, segments of at least 4 chunks
-    long long want = (2 * 148 * kCtasPerSM + units - 1) / units;
+    // enough items for ~2 waves of one CTA per SM, segments of at least 4 chunks
+    long long want = (2 * 148 + units - 1) / units;
     long long maxseg = (p.nchunks + 3) / 4;
     if (want > maxseg) want = maxseg;
     if (want < 1) want = 1;
