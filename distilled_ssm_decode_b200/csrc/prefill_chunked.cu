@@ -67,23 +67,28 @@ constexpr int kKVStages = 3;                      // k,v tiles
 constexpr int kQStages = 4;                       // q tiles (y staged in place)
 constexpr int kUBufs = 4;                         // U operands
 constexpr int kSTBufs = 4;                        // state operands
-constexpr int kD1Bufs = 4;                        // output accumulators (TMEM)
-constexpr int kD2Bufs = 2;                        // state-product accumulators (TMEM)
+constexpr int kNAcc = 4;                          // accumulators (TMEM): [C output cols | 32 state cols]
+constexpr int kAccCols = kC + kKSMax;
+constexpr int kPrefetch = 8;                      // chunks of q, k, v prefetched into L2 ahead of the loads
 constexpr int kThreads = 512;                     // 16 warps, see the role map below
-constexpr uint32_t kTmemCols = 256;               // D1 (4 x C cols) + D2 (2 x 32 cols), rounded up
+constexpr uint32_t kTmemCols = kNAcc * kAccCols;  // 256
 
-// constant block per head (global, laid out exactly as in shared memory)
-constexpr int kTTBytes = kC * kC * 4;             // B operand of the Toeplitz product
+// constant block per head (global, laid out exactly as in shared memory).  T (Toeplitz) and
+// V (chunk powers) are adjacent so that they form one B operand [T; V] of C + 32 rows: the
+// fused product U [T; V]^T yields the intra-chunk output and the chunk's state contribution
+// in one pass over U (an MMA costs the same for any N <= 128 on B200).
+constexpr int kTTBytes = kC * kC * 4;             // rows 0..C-1 of the fused B operand
+constexpr int kVTBytes = kKSMax * kC * 4;         // rows C..C+31 of the fused B operand
 constexpr int kATBytes = kC * kKSMax * 4;         // B operand of the carry product
-constexpr int kVTBytes = kKSMax * kC * 4;         // B operand of the state product
 constexpr int kConstBytes = kTTBytes + kATBytes + kVTBytes + 2 * kMaxModes * 8;   // + lambda^C, lambda^Lseg
 constexpr int kConstStride = (kConstBytes + 255) & ~255;
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr int kSmTT = 0;
-constexpr int kSmAT = kSmTT + kTTBytes;
-constexpr int kSmVT = kSmAT + kATBytes;
-constexpr int kSmUT = kSmVT + kVTBytes;                       // kUBufs x [128][C] tf32
+constexpr int kSmVT = kSmTT + kTTBytes;
+constexpr int kSmAT = kSmVT + kVTBytes;
+constexpr int kSmLam = kSmAT + kATBytes;                      // lambda^C, lambda^Lseg [16] each (float2)
+constexpr int kSmUT = kSmLam + 1024;                          // kUBufs x [128][C] tf32
 constexpr int kUTBytes = kNC * kC * 4;
 constexpr int kSmST = kSmUT + kUBufs * kUTBytes;              // kSTBufs x [128][32] tf32
 constexpr int kSTBytes = kNC * kKSMax * 4;
@@ -99,13 +104,13 @@ enum : int {
     kBarQEmpty = kBarQFull + kQStages,           // [kQStages] q/y buffer free (1: store warp)
     kBarURdy = kBarQEmpty + kQStages,            // [kUBufs] U operand written (128: U group)
     kBarUFree = kBarURdy + kUBufs,               // [kUBufs] U operand no longer read (commit)
-    kBarWDone = kBarUFree + kUBufs,              // [kD2Bufs] state product done (commit)
-    kBarD2Free = kBarWDone + kD2Bufs,            // [kD2Bufs] state product read out (128: S group)
-    kBarSRdy = kBarD2Free + kD2Bufs,             // [kSTBufs] state operand written (128: S group)
+    kBarWDone = kBarUFree + kUBufs,              // [kNAcc] fused product done (commit)
+    kBarD2Free = kBarWDone + kNAcc,              // [kNAcc] state columns read out (128: S group)
+    kBarSRdy = kBarD2Free + kNAcc,               // [kSTBufs] state operand written (128: S group)
     kBarSTFree = kBarSRdy + kSTBufs,             // [kSTBufs] state operand no longer read (commit)
-    kBarYDone = kBarSTFree + kSTBufs,            // [kD1Bufs] output product done (commit)
-    kBarD1Free = kBarYDone + kD1Bufs,            // [kD1Bufs] output product read out (128: E group)
-    kBarYStaged = kBarD1Free + kD1Bufs,          // [kQStages] gated tile staged for the store (128: E group)
+    kBarYDone = kBarSTFree + kSTBufs,            // [kNAcc] carry product done: output complete (commit)
+    kBarD1Free = kBarYDone + kNAcc,              // [kNAcc] output columns read out (128: E group)
+    kBarYStaged = kBarD1Free + kNAcc,            // [kQStages] gated tile staged for the store (128: E group)
     kBarPub = kBarYStaged + kQStages,            // segment state written to global (128: S group)
     kBarDrain = kBarPub + 1,                     // every MMA of the CTA finished (commit)
     kNumBars = kBarDrain + 1
@@ -158,9 +163,9 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
                     uint8_t *__restrict__ consts) {
     const int hd = blockIdx.x;
     uint8_t *base = consts + (size_t)hd * kConstStride;
-    float *TT = reinterpret_cast<float *>(base);
-    float *AT = reinterpret_cast<float *>(base + kTTBytes);
-    float *VT = reinterpret_cast<float *>(base + kTTBytes + kATBytes);
+    float *TT = reinterpret_cast<float *>(base + kSmTT);
+    float *VT = reinterpret_cast<float *>(base + kSmVT);
+    float *AT = reinterpret_cast<float *>(base + kSmAT);
     float2 *lamC = reinterpret_cast<float2 *>(base + kTTBytes + kATBytes + kVTBytes);
     float2 *lamS = lamC + kMaxModes;
     __shared__ double hs[kC];
@@ -270,7 +275,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     {
         const int4 *src = reinterpret_cast<const int4 *>(a.consts + (size_t)hd * kConstStride);
         int4 *dst = reinterpret_cast<int4 *>(sm);
-        for (int i = tid; i < (kTTBytes + kATBytes + kVTBytes) / 16; i += kThreads) dst[i] = __ldg(src + i);
+        for (int i = tid; i < (kTTBytes + kATBytes + kVTBytes + 2 * kMaxModes * 8) / 16; i += kThreads)
+            dst[i] = __ldg(src + i);      // [T; V], A and lambda^C, lambda^Lseg
         int4 *stz = reinterpret_cast<int4 *>(sm + kSmST);
         for (int i = tid; i < kSTBufs * kSTBytes / 16; i += kThreads) stz[i] = make_int4(0, 0, 0, 0);
     }
@@ -285,8 +291,22 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (warp >= 12 && warp <= 14) {
         // ------------------------------------------------------------ TMA warps
         if (warp == 12 && lane == 0) {      // k, v for every iteration (state-only pass, then full pass)
+            // L2 prefetch runs kPrefetch chunks ahead of the loads, so that many more bytes are in
+            // flight than the shared-memory stages hold (loaded DRAM latency is several us here)
+            for (int it = 0; it < min(kPrefetch, n1 > 0 ? n1 : nck); ++it)
+                for (int h = 0; h < 2; ++h) {
+                    tc::tma_prefetch_3d(&tm_k, c0 + 64 * h, chunk_of(it) * kC, b);
+                    tc::tma_prefetch_3d(&tm_v, c0 + 64 * h, chunk_of(it) * kC, b);
+                }
             int it = 0;
             for (; it < niter; ++it) {
+                // the full pass re-reads k, v that the state-only pass brought into L2
+                const int pf = it + kPrefetch;
+                if (pf < (n1 > 0 ? n1 : nck))
+                    for (int h = 0; h < 2; ++h) {
+                        tc::tma_prefetch_3d(&tm_k, c0 + 64 * h, chunk_of(pf) * kC, b);
+                        tc::tma_prefetch_3d(&tm_v, c0 + 64 * h, chunk_of(pf) * kC, b);
+                    }
                 const int s = it % kKVStages;
                 if (!tc::mbar_wait(bar(kBarKVEmpty + s), ((it / kKVStages) & 1) ^ 1, abort)) {
                     record_error(a, abort, kErrWait);
@@ -304,8 +324,13 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 for (int j = max(0, it - kKVStages); j < it; ++j)
                     tc::mbar_wait(bar(kBarKVFull + j % kKVStages), (j / kKVStages) & 1, never);
         } else if (warp == 13 && lane == 0) {   // q for the full pass (the buffer then stages y)
+            for (int j = 0; j < min(kPrefetch, nck); ++j)
+                for (int h = 0; h < 2; ++h) tc::tma_prefetch_3d(&tm_q, c0 + 64 * h, (ck0 + j) * kC, b);
             int j = 0;
             for (; j < nck; ++j) {
+                if (j + kPrefetch < nck)
+                    for (int h = 0; h < 2; ++h)
+                        tc::tma_prefetch_3d(&tm_q, c0 + 64 * h, (ck0 + j + kPrefetch) * kC, b);
                 const int s = j % kQStages;
                 if (!tc::mbar_wait(bar(kBarQEmpty + s), ((j / kQStages) & 1) ^ 1, abort)) {
                     record_error(a, abort, kErrWait);
@@ -337,45 +362,63 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
     } else if (warp == 15) {
         // ------------------------------------------------------------ MMA issuer
+        // Two streams issued out of order from one thread (polled with non-blocking tests, since
+        // a suspending wait on one stream would hold back the other): the fused product of a chunk
+        // (needs only its U operand and a free accumulator) runs ahead, the carry product
+        // (needs the state entering the chunk) follows when the S group delivers it.  MMAs from
+        // one thread execute in issue order, so a chunk's carry always lands after its fused part.
         if (lane == 0) {
-            const uint32_t idesc_y = tc::idesc_tf32(kNC, kC);
-            const uint32_t idesc_w = tc::idesc_tf32(kNC, kKSMax);
-            for (int it = 0; it < niter && !*abort; ++it) {
-                const int ub = it % kUBufs, wb = it % kD2Bufs;
-                const uint32_t ut = sbase + kSmUT + ub * kUTBytes;
-                if (!tc::mbar_wait(bar(kBarURdy + ub), (it / kUBufs) & 1, abort) ||
-                    !tc::mbar_wait(bar(kBarD2Free + wb), ((it / kD2Bufs) & 1) ^ 1, abort)) {
-                    record_error(a, abort, kErrWait);
-                    break;
+            const uint32_t idesc_f = tc::idesc_tf32(kNC, kAccCols);
+            const uint32_t idesc_c = tc::idesc_tf32(kNC, kC);
+            int ic = 0, jn = 0;
+            unsigned long long t_prog = tc::global_ns();
+            while ((ic < niter || jn < nck) && !*abort) {
+                bool progressed = false;
+                if (jn < nck && n1 + jn < ic) {
+                    const int sb = jn % kSTBufs, ab = (n1 + jn) % kNAcc;
+                    if (tc::mbar_test(bar(kBarSRdy + sb), (jn / kSTBufs) & 1)) {
+                        tc::tc_fence_after();
+                        // carry: D[0:C) += S A^T
+                        const uint32_t d = tmem + ab * kAccCols;
+                        const uint32_t stb = sbase + kSmST + sb * kSTBytes;
+                        for (int ks = 0; ks < kKSMax / 8; ++ks)
+                            tc::mma_tf32(d, tc::smem_desc(stb + ks * 256, 128, kKSMax * 32),
+                                         tc::smem_desc(sbase + kSmAT + ks * 256, 128, kKSMax * 32), idesc_c, 1);
+                        tc::mma_commit(bar(kBarYDone + ab));
+                        tc::mma_commit(bar(kBarSTFree + sb));
+                        ++jn;
+                        progressed = true;
+                    }
                 }
-                tc::tc_fence_after();
-                // D2 = U V^T: the chunk's contribution to the state
-                const uint32_t d2 = tmem + kD1Bufs * kC + wb * kKSMax;
-                for (int ks = 0; ks < kC / 8; ++ks)
-                    tc::mma_tf32(d2, tc::smem_desc(ut + ks * 256, 128, kC * 32),
-                                 tc::smem_desc(sbase + kSmVT + ks * 256, 128, kC * 32), idesc_w, ks > 0);
-                tc::mma_commit(bar(kBarWDone + wb));
-                if (it >= n1) {
-                    const int j = it - n1, sb = j % kSTBufs, db = j % kD1Bufs;
-                    if (!tc::mbar_wait(bar(kBarSRdy + sb), (j / kSTBufs) & 1, abort) ||
-                        !tc::mbar_wait(bar(kBarD1Free + db), ((j / kD1Bufs) & 1) ^ 1, abort)) {
+                if (ic < niter) {
+                    const int ub = ic % kUBufs, ab = ic % kNAcc;
+                    bool ready = tc::mbar_test(bar(kBarURdy + ub), (ic / kUBufs) & 1) &&
+                                 tc::mbar_test(bar(kBarD2Free + ab), ((ic / kNAcc) & 1) ^ 1);
+                    if (ready && ic >= n1)   // phase-2 uses of this accumulator (n1 % kNAcc == 0)
+                        ready = tc::mbar_test(bar(kBarD1Free + ab), (((ic - n1) / kNAcc) & 1) ^ 1);
+                    if (ready) {
+                        tc::tc_fence_after();
+                        // fused: D[0:C+32) = U [T; V]^T  (intra-chunk output | state contribution)
+                        const uint32_t d = tmem + ab * kAccCols;
+                        const uint32_t ut = sbase + kSmUT + ub * kUTBytes;
+                        for (int ks = 0; ks < kC / 8; ++ks)
+                            tc::mma_tf32(d, tc::smem_desc(ut + ks * 256, 128, kC * 32),
+                                         tc::smem_desc(sbase + kSmTT + ks * 256, 128, kC * 32), idesc_f, ks > 0);
+                        tc::mma_commit(bar(kBarWDone + ab));
+                        tc::mma_commit(bar(kBarUFree + ub));
+                        ++ic;
+                        progressed = true;
+                    }
+                }
+                if (progressed) {
+                    t_prog = tc::global_ns();
+                } else {
+                    if (tc::global_ns() - t_prog > tc::kWaitNs) {
                         record_error(a, abort, kErrWait);
                         break;
                     }
-                    tc::tc_fence_after();
-                    // D1 = U T^T + S A^T: intra-chunk Toeplitz product plus the modal carry
-                    const uint32_t d1 = tmem + db * kC;
-                    const uint32_t stb = sbase + kSmST + sb * kSTBytes;
-                    for (int ks = 0; ks < kC / 8; ++ks)
-                        tc::mma_tf32(d1, tc::smem_desc(ut + ks * 256, 128, kC * 32),
-                                     tc::smem_desc(sbase + kSmTT + ks * 256, 128, kC * 32), idesc_y, ks > 0);
-                    for (int ks = 0; ks < kKSMax / 8; ++ks)
-                        tc::mma_tf32(d1, tc::smem_desc(stb + ks * 256, 128, kKSMax * 32),
-                                     tc::smem_desc(sbase + kSmAT + ks * 256, 128, kKSMax * 32), idesc_y, 1);
-                    tc::mma_commit(bar(kBarYDone + db));
-                    tc::mma_commit(bar(kBarSTFree + sb));
+                    __nanosleep(32);      // polling: leave issue slots to the warps sharing the SMSP
                 }
-                tc::mma_commit(bar(kBarUFree + ub));
             }
             // all MMAs issued by this thread have completed once `drain` fires
             tc::mma_commit(bar(kBarDrain));
@@ -423,24 +466,22 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // ------------------------------------------------------------ S group (state chain)
         const int c = tid - 128;                     // channel within the tile == TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const float2 *lamC = reinterpret_cast<const float2 *>(a.consts + (size_t)hd * kConstStride +
-                                                              kTTBytes + kATBytes + kVTBytes);
+        // lambda^C and lambda^Lseg stay in shared memory (broadcast reads) to keep this
+        // group's registers for the state itself
+        const float2 *lamC = reinterpret_cast<const float2 *>(sm + kSmLam);
         const float2 *lamS = lamC + kMaxModes;
-        float2 lc[kMaxModes], st[kMaxModes];
+        float2 st[kMaxModes];
 #pragma unroll
-        for (int n = 0; n < kMaxModes; ++n) {
-            lc[n] = n < d ? __ldg(&lamC[n]) : make_float2(0.f, 0.f);
-            st[n] = make_float2(0.f, 0.f);
-        }
+        for (int n = 0; n < kMaxModes; ++n) st[n] = make_float2(0.f, 0.f);
         bool ok = true;
         int pub_phase = 0;
         // st <- lambda^C st + D2 of iteration it
         auto advance = [&](int it) -> bool {
-            const int wb = it % kD2Bufs;
-            if (!tc::mbar_wait(bar(kBarWDone + wb), (it / kD2Bufs) & 1, abort)) return false;
+            const int wb = it % kNAcc;
+            if (!tc::mbar_wait(bar(kBarWDone + wb), (it / kNAcc) & 1, abort)) return false;
             tc::tc_fence_after();
             float w[kKSMax];
-            const uint32_t taddr = tmem + lane_base + kD1Bufs * kC + wb * kKSMax;
+            const uint32_t taddr = tmem + lane_base + wb * kAccCols + kC;
             tc::tmem_ld16(taddr, w);
             tc::tmem_ld16(taddr + 16, w + 16);
             tc::tmem_wait_ld();
@@ -448,9 +489,9 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             tc::mbar_arrive(bar(kBarD2Free + wb));
 #pragma unroll
             for (int n = 0; n < kMaxModes; ++n) {
-                const float2 sv = st[n];
-                st[n] = make_float2(fmaf(lc[n].x, sv.x, fmaf(-lc[n].y, sv.y, w[n])),
-                                    fmaf(lc[n].x, sv.y, fmaf(lc[n].y, sv.x, w[kIm + n])));
+                const float2 sv = st[n], lc = lamC[n];      // lambda^C is 0 for modes >= d
+                st[n] = make_float2(fmaf(lc.x, sv.x, fmaf(-lc.y, sv.y, w[n])),
+                                    fmaf(lc.x, sv.y, fmaf(lc.y, sv.x, w[kIm + n])));
             }
             return true;
         };
@@ -479,12 +520,9 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 
         // look-back: the state entering this segment
         if (ok && seg > 0) {
-            float2 lsg[kMaxModes], scale[kMaxModes];
+            float2 scale[kMaxModes];
 #pragma unroll
-            for (int n = 0; n < kMaxModes; ++n) {
-                lsg[n] = n < d ? __ldg(&lamS[n]) : make_float2(0.f, 0.f);
-                scale[n] = make_float2(1.f, 0.f);
-            }
+            for (int n = 0; n < kMaxModes; ++n) scale[n] = make_float2(1.f, 0.f);
             for (int p = item - 1; p >= item - seg && ok; --p) {
                 int code = *(volatile int *)(a.status + p);
                 const unsigned long long t0 = tc::global_ns();
@@ -504,7 +542,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     if (n < d) {
                         const float2 v = make_float2(src[(size_t)n * kNC + c].x, src[(size_t)n * kNC + c].y);
                         st[n] = cadd(st[n], cmul(scale[n], v));
-                        scale[n] = cmul(scale[n], lsg[n]);
+                        scale[n] = cmul(scale[n], lamS[n]);
                     }
                 }
                 if (code == 2) break;
@@ -516,7 +554,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
                 for (int n = 0; n < kMaxModes; ++n) {
                     keep[n] = st[n];
-                    st[n] = cadd(cmul(lsg[n], st[n]), sloc[n]);
+                    st[n] = cadd(cmul(lamS[n], st[n]), sloc[n]);
                 }
                 ok = uni(publish(a.inc + (size_t)item * d * kNC, 2));
 #pragma unroll
@@ -588,8 +626,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         bool ok = true;
         for (int j = 0; j < nck && ok; ++j) {
-            const int db = j % kD1Bufs, s = j % kQStages;
-            ok = uni(tc::mbar_wait(bar(kBarYDone + db), (j / kD1Bufs) & 1, abort) &&
+            const int db = j % kNAcc, s = j % kQStages;     // == (n1 + j) % kNAcc since n1 % kNAcc == 0
+            ok = uni(tc::mbar_wait(bar(kBarYDone + db), (j / kNAcc) & 1, abort) &&
                      tc::mbar_wait(bar(kBarQFull + s), (j / kQStages) & 1, abort));
             if (!ok) break;
             tc::tc_fence_after();
@@ -598,8 +636,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
             for (int tau = 0; tau < kC; ++tau) qv[tau] = *reinterpret_cast<const __nv_bfloat16 *>(qy + act_off(tau, c));
             float z[kC];
-            tc::tmem_ld16(tmem + lane_base + db * kC, z);
-            tc::tmem_ld16(tmem + lane_base + db * kC + 16, z + 16);
+            tc::tmem_ld16(tmem + lane_base + db * kAccCols, z);
+            tc::tmem_ld16(tmem + lane_base + db * kAccCols + 16, z + 16);
             tc::tmem_wait_ld();
             tc::tc_fence_before();
             tc::mbar_arrive(bar(kBarD1Free + db));
@@ -661,6 +699,7 @@ ChunkPlan plan(int B, int L, int Dch, int H, int d) {
     if (want > maxseg) want = maxseg;
     if (want < 1) want = 1;
     p.segc = (int)((p.nchunks + want - 1) / want);
+    p.segc = (p.segc + kNAcc - 1) / kNAcc * kNAcc;   // state-only passes cover whole accumulator rings
     p.nseg = (p.nchunks + p.segc - 1) / p.segc;
     p.items = (int)(units * p.nseg);
     p.consts_off = 0;
