@@ -4,46 +4,51 @@
 // sequences 100x faster than FlashAttention", lequren.com, "Hyena層次結構")
 // with the modal filter h_0 = Dskip, h_j = Re sum_n R_n lambda_n^(j-1) of
 // "Laughing Hyena Distillery" (nubint.ai review, "Proposed method") is
-// evaluated chunk by chunk.  For a chunk of C tokens starting at c0, with
+// evaluated chunk by chunk.  For a chunk of C tokens starting at token t0, with
 // tau, iota in [0, C):
 //
-//   z[c0+tau] = sum_{iota<=tau} h_{tau-iota} u[c0+iota]            (intra-chunk Toeplitz)
-//             + Re sum_n R_n lambda_n^tau s_n(c0)                  (modal carry from the past)
-//   s_n(c0+C) = lambda_n^C s_n(c0) + sum_iota lambda_n^(C-1-iota) u[c0+iota]
+//   z[t0+tau] = sum_{iota<=tau} h_{tau-iota} u[t0+iota]            (intra-chunk Toeplitz)
+//             + Re sum_n R_n lambda_n^tau s_n(t0)                  (modal carry from the past)
+//   s_n(t0+C) = lambda_n^C s_n(t0) + sum_iota lambda_n^(C-1-iota) u[t0+iota]
 //
-// where s(c0) is the recurrent state after c0 tokens -- the same O(d) state the
-// decode step advances ("Main findings": O(d) memory per channel).  This is an
-// exact regrouping of the causal convolution (the carry term is the tail of the
-// sum over j < c0 with h_{t-j} = Re sum R lambda^(t-c0) lambda^(c0-1-j)), and
-// the prompt -> state reduction falls out as the last carry.
+// where s(t0) is the recurrent state after the tokens before t0 -- the same
+// O(d) state the decode step advances ("Main findings": O(d) memory per
+// channel).  This is an exact regrouping of the causal convolution (the carry
+// is the tail of the sum over j < t0, with h_{t-j} = Re sum R lambda^(t-t0)
+// lambda^(t0-1-j)), and the prompt -> state reduction is the last state.
 //
-// Per chunk and 128-channel tile (one head, M = 128 = channels on the MMA
-// rows), three products run on the tensor cores in tf32 with fp32 accumulation
-// in tensor memory:
-//   D1[c][tau] = sum_iota U[c][iota] T[tau][iota]  +  sum_r S[c][r] A[tau][r]
-//   D2[c][r]   = sum_iota U[c][iota] V[r][iota]
-// with T[tau][iota] = h_{tau-iota} (iota <= tau), A = (Re, -Im) of R lambda^tau,
-// V = (Re, Im) of lambda^(C-1-iota), S = (Re, Im) of the state.  The chunk's
-// state update S <- lambda^C S + D2 runs on the CUDA cores in fp32 registers
-// (one thread per channel, the thread that owns TMEM lane c), and
-// y = q * D1 is gated and stored by the same thread.
+// The chunk grid is aligned to the END of the prompt: chunk i covers tokens
+// [L - (nchunks-i) C, L - (nchunks-1-i) C), so the first chunk may start before
+// token 0 (its missing tokens are zero-filled by TMA and contribute nothing)
+// and the state after the last chunk is exactly the state after token L-1.
+//
+// Per chunk and 128-channel tile the tensor cores evaluate, in bf16 with fp32
+// accumulation in tensor memory (rows on MMA M, the 128 channels on MMA N):
+//   fused:  [Z; W] = [T; V] U          T[tau][iota] = h_{tau-iota} (iota <= tau)
+//                                      V[r][iota]   = (Re | Im) lambda_r^(C-1-iota)
+//   carry:  Z     += A S               A[tau][r]    = (Re | -Im) R_r lambda_r^tau
+// where U[iota][c] = k v is formed elementwise over the TMA'd k tile (its
+// natural [token][channel] 128-byte-swizzled layout is already an MN-major
+// operand), S[r][c] = (Re | Im) s(t0) and W[r][c] is the chunk's state
+// contribution.  The state chain s <- lambda^C s + W runs on the CUDA cores in
+// fp32 (one thread per state row and 32 channels), and y = q Z is gated and
+// stored per token row.  The carry accumulates into TMEM columns of its own, so
+// the state rows W are never touched while the chain reads them.
 //
 // Work split: a sequence is cut into segments of whole chunks; each
-// (batch, channel tile, segment) item first runs a state-only pass (k, v and
-// the D2 product) to publish its segment's state contribution, then obtains the
+// (batch, channel tile, segment) item first runs a state-only pass (k, v and the
+// fused product) to publish its segment's state contribution, then obtains the
 // state entering its segment by a decoupled look-back over its predecessors'
-// published contributions (bounded polls), then runs the full pass.  Items are
-// handed out by an atomic ticket in launch order, so an item only ever waits on
-// items already running; the state-only pass never waits, so the look-back
-// always ends.  k and v are read twice per item, the second time mostly from L2.
-//
-// Roles in a 192-thread CTA: warps 0-3 (one thread per channel) compute
-// u = k*v, the state and the gated output; warp 4 issues the TMA loads; warp 5
-// owns tensor memory and issues the MMAs.  Every wait is bounded; on timeout
-// the kernel records an error code, drains its copies and MMAs, frees tensor
-// memory and returns.
+// published contributions (bounded polls), then runs the full pass.  The grid is
+// persistent: each CTA takes items from an atomic ticket in order and its
+// pipelines run on across item boundaries.  An item only ever waits on items
+// with lower tickets, which running CTAs hold, and the state-only pass never
+// waits, so the look-back always ends.  Every wait is bounded; on timeout the
+// kernel records an error code, drains its copies and MMAs, frees tensor memory
+// and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cuda_bf16.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -53,101 +58,125 @@ namespace hyena {
 
 namespace {
 
-constexpr int kC = 32;             // tokens per chunk
-constexpr int kNC = 128;           // channels per tile (MMA M)
-constexpr int kMaxModes = 16;      // d <= 16
-constexpr int kKSMax = 32;         // state operand width: Re at [0,16), Im at [16,32)
+constexpr int kC = 64;              // tokens per chunk (K of the fused product)
+constexpr int kNC = 128;            // channels per tile (MMA N)
+constexpr int kMaxModes = 16;       // d <= 16
+constexpr int kKS = 32;             // state rows: Re of modes 0..15, then Im
 constexpr int kIm = 16;
-constexpr int kTileBytes = kC * kNC * 2;          // one bf16 [C][128] activation tile
-constexpr int kHalfBytes = kTileBytes / 2;        // [C][64] half tile = one TMA box, 128-byte swizzled
-// Ring depths.  A chunk's output product needs the U operand, the state operand and a D1
-// accumulator; each of those is refilled only after the product that used it completes, so a
-// ring of depth n lets n chunks be in flight between those round trips.
-constexpr int kKVStages = 3;                      // k,v tiles
-constexpr int kQStages = 4;                       // q tiles (y staged in place)
-constexpr int kUBufs = 4;                         // U operands
-constexpr int kSTBufs = 4;                        // state operands
-constexpr int kNAcc = 4;                          // accumulators (TMEM): [C output cols | 32 state cols]
-constexpr int kAccCols = kC + kKSMax;
-constexpr int kPrefetch = 8;                      // chunks of q, k, v prefetched into L2 ahead of the loads
-constexpr int kThreads = 512;                     // 16 warps, see the role map below
-constexpr uint32_t kTmemCols = kNAcc * kAccCols;  // 256
+constexpr int kTile = kC * kNC * 2;          // one bf16 [C][128] activation tile (16 KB)
+constexpr int kHalf = kTile / 2;             // [C][64] half = one TMA box, 128-byte swizzled
+constexpr int kStageBytes = 2 * kTile;       // k (overwritten by U) then v
+constexpr int kKVStages = 4;
+constexpr int kQStages = 3;                  // q tiles; y is staged in place
+constexpr int kSBufs = 2;                    // state operands
+constexpr int kSlots = 2;                    // accumulator slots: fused [128 cols] | carry [128 cols]
+constexpr int kSlotCols = 2 * kNC;
+constexpr uint32_t kTmemCols = kSlots * kSlotCols;   // 512
+constexpr int kItemQ = 4;                    // item ids handed from the k,v loader to the other roles
+constexpr int kThreads = 512;
+constexpr int kMaxSeg = 128;                 // segments per sequence (bounds look-back walks)
 
-// constant block per head (global, laid out exactly as in shared memory).  T (Toeplitz) and
-// V (chunk powers) are adjacent so that they form one B operand [T; V] of C + 32 rows: the
-// fused product U [T; V]^T yields the intra-chunk output and the chunk's state contribution
-// in one pass over U (an MMA costs the same for any N <= 128 on B200).
-constexpr int kTTBytes = kC * kC * 4;             // rows 0..C-1 of the fused B operand
-constexpr int kVTBytes = kKSMax * kC * 4;         // rows C..C+31 of the fused B operand
-constexpr int kATBytes = kC * kKSMax * 4;         // B operand of the carry product
-constexpr int kConstBytes = kTTBytes + kATBytes + kVTBytes + 2 * kMaxModes * 8;   // + lambda^C, lambda^Lseg
-constexpr int kConstStride = (kConstBytes + 255) & ~255;
+// per-head constants: the two A operands (copied verbatim into shared memory) and the powers
+// lambda^C, lambda^Lseg (read from global by the state group)
+constexpr int kFABytes = 128 * kC * 2;       // [T; V; 0]: 128 rows x 64 K bf16
+constexpr int kCABytes = 128 * kKS * 2;      // [A; 0]:    128 rows x 32 K bf16
+constexpr int kOpBytes = kFABytes + kCABytes;
+constexpr int kLamOff = kOpBytes;            // float2 lambda^C [16], lambda^Lseg [16]
+constexpr int kConstStride = kOpBytes + 256;
 
 // shared memory map (offsets from a 1024-byte aligned base)
-constexpr int kSmTT = 0;
-constexpr int kSmVT = kSmTT + kTTBytes;
-constexpr int kSmAT = kSmVT + kVTBytes;
-constexpr int kSmLam = kSmAT + kATBytes;                      // lambda^C, lambda^Lseg [16] each (float2)
-constexpr int kSmUT = kSmLam + 1024;                          // kUBufs x [128][C] tf32
-constexpr int kUTBytes = kNC * kC * 4;
-constexpr int kSmST = kSmUT + kUBufs * kUTBytes;              // kSTBufs x [128][32] tf32
-constexpr int kSTBytes = kNC * kKSMax * 4;
-constexpr int kSmKV = kSmST + kSTBufs * kSTBytes;             // kKVStages x {k, v}
-constexpr int kSmQ = kSmKV + kKVStages * 2 * kTileBytes;      // kQStages x q (y staged in place)
-constexpr int kSmBar = kSmQ + kQStages * kTileBytes;
+constexpr int kSmFA = 0;
+constexpr int kSmCA = kSmFA + kFABytes;
+constexpr int kSmKV = kSmCA + kCABytes;                   // 1024-aligned (swizzle atoms)
+constexpr int kSmQ = kSmKV + kKVStages * kStageBytes;
+constexpr int kSBytes = kKS * kNC * 2;                    // [32 rows][128 ch] bf16, 128-byte swizzled
+constexpr int kSmS = kSmQ + kQStages * kTile;
+constexpr int kSmBar = kSmS + kSBufs * kSBytes;
 
 // barrier slots (arrival counts in parentheses; "commit" = tcgen05.commit from the MMA thread)
 enum : int {
-    kBarKVFull = 0,                              // [kKVStages] k,v tile landed (1 + tx)
-    kBarKVEmpty = kBarKVFull + kKVStages,        // [kKVStages] k,v consumed (128: U group, or S group for the prompt's last chunk)
-    kBarQFull = kBarKVEmpty + kKVStages,         // [kQStages] q tile landed (1 + tx)
-    kBarQEmpty = kBarQFull + kQStages,           // [kQStages] q/y buffer free (1: store warp)
-    kBarURdy = kBarQEmpty + kQStages,            // [kUBufs] U operand written (128: U group)
-    kBarUFree = kBarURdy + kUBufs,               // [kUBufs] U operand no longer read (commit)
-    kBarWDone = kBarUFree + kUBufs,              // [kNAcc] fused product done (commit)
-    kBarD2Free = kBarWDone + kNAcc,              // [kNAcc] state columns read out (128: S group)
-    kBarSRdy = kBarD2Free + kNAcc,               // [kSTBufs] state operand written (128: S group)
-    kBarSTFree = kBarSRdy + kSTBufs,             // [kSTBufs] state operand no longer read (commit)
-    kBarYDone = kBarSTFree + kSTBufs,            // [kNAcc] carry product done: output complete (commit)
-    kBarD1Free = kBarYDone + kNAcc,              // [kNAcc] output columns read out (128: E group)
-    kBarYStaged = kBarD1Free + kNAcc,            // [kQStages] gated tile staged for the store (128: E group)
-    kBarPub = kBarYStaged + kQStages,            // segment state written to global (128: S group)
+    kBarKVFull = 0,                              // [kKVStages] k,v landed (1 + tx)
+    kBarKVEmpty = kBarKVFull + kKVStages,        // [kKVStages] fused product read U (commit)
+    kBarURdy = kBarKVEmpty + kKVStages,          // [kKVStages] U formed over k (128: U group)
+    kBarQFull = kBarURdy + kKVStages,            // [kQStages] q landed (1 + tx)
+    kBarQEmpty = kBarQFull + kQStages,           // [kQStages] y stored, buffer free (1: store lane)
+    kBarYStaged = kBarQEmpty + kQStages,         // [kQStages] gated y staged (128: E group)
+    kBarWDone = kBarYStaged + kQStages,          // [kSlots] fused product done (commit)
+    kBarD2Free = kBarWDone + kSlots,             // [kSlots] state rows read out (128: S group)
+    kBarYDone = kBarD2Free + kSlots,             // [kSlots] carry done: output complete (commit)
+    kBarD1Free = kBarYDone + kSlots,             // [kSlots] output rows read out (128: E group)
+    kBarSRdy = kBarD1Free + kSlots,              // [kSBufs] state operand written (128: S group)
+    kBarSTFree = kBarSRdy + kSBufs,              // [kSBufs] state operand read (commit)
+    kBarItemFull = kBarSTFree + kSBufs,          // [kItemQ] item id posted (1)
+    kBarItemEmpty = kBarItemFull + kItemQ,       // [kItemQ] item id read by every consumer (kItemReaders)
+    kBarConst = kBarItemEmpty + kItemQ,          // head constants landed (1 + tx)
+    kBarConstFree = kBarConst + 1,               // MMAs on the old constants done (commit)
+    kBarPub = kBarConstFree + 1,                 // segment state written to global (128: S group)
     kBarDrain = kBarPub + 1,                     // every MMA of the CTA finished (commit)
     kNumBars = kBarDrain + 1
 };
+// item readers: q loader, store lane, MMA lane (1 each) + lane 0 of the 4 U, 4 S and 4 E warps
+constexpr int kItemReaders = 3 + 12;
 constexpr int kSmMisc = kSmBar + kNumBars * 8;
-constexpr int kSmemBytes = kSmMisc + 64 + 1024;               // + misc words + alignment slack
+constexpr int kSmemBytes = kSmMisc + 64 + 1024;           // + item ids, misc words, alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+static_assert(kSmKV % 1024 == 0 && kSmQ % 1024 == 0 && kSmS % 1024 == 0, "swizzle atoms");
 
 __host__ __device__ constexpr int bar_count(int i) {
-    return ((i >= kBarKVEmpty && i < kBarQFull) || (i >= kBarURdy && i < kBarUFree) ||
-            (i >= kBarD2Free && i < kBarSTFree) || (i >= kBarD1Free && i < kBarDrain)) ? 128 : 1;
+    return ((i >= kBarURdy && i < kBarQFull) || (i >= kBarYStaged && i < kBarWDone) ||
+            (i >= kBarD2Free && i < kBarYDone) || (i >= kBarD1Free && i < kBarSTFree) || i == kBarPub)
+               ? 128
+               : (i >= kBarItemEmpty && i < kBarConst) ? kItemReaders : 1;
 }
 
-// byte offset of element (row, k) in a K-major, no-swizzle core-matrix tile whose K extent is K
-__host__ __device__ __forceinline__ int cm_off(int row, int k, int K) {
-    return (k >> 2) * 128 + (row >> 3) * (K * 32) + (row & 7) * 16 + (k & 3) * 4;
-}
+// warp roles (16 warps).  The state group must sit on warps w % 4 == 2 (TMEM lanes 64..95, the
+// state rows); the output group on w % 4 in {0, 1} (lanes 0..63, the token rows).
+constexpr int kWarpKV = 0, kWarpQ = 1, kWarpMMA = 3, kWarpStore = 12;
+__host__ __device__ constexpr bool is_s_warp(int w) { return (w & 3) == 2; }                 // 2, 6, 10, 14
+__host__ __device__ constexpr bool is_e_warp(int w) { return w == 4 || w == 5 || w == 8 || w == 9; }
+__host__ __device__ constexpr int u_index(int w) { return w == 7 ? 0 : w == 11 ? 1 : w == 13 ? 2 : w == 15 ? 3 : -1; }
 
-// byte offset of activation (token tau, channel c) in a [C][128] bf16 tile held as two
-// [C][64] halves written by TMA with 128-byte swizzling (16-byte chunk ^= row % 8)
-__device__ __forceinline__ int act_off(int tau, int c) {
-    return (c >> 6) * kHalfBytes + tau * 128 + ((((c & 63) >> 3) ^ (tau & 7)) << 4) + (c & 7) * 2;
+// byte offset of bf16 element (row, k) in a K-major, no-swizzle core-matrix tile of K columns
+__host__ __device__ __forceinline__ int cm_off16(int row, int k, int K) {
+    return (k >> 3) * 128 + (row >> 3) * (K * 16) + (row & 7) * 16 + (k & 7) * 2;
 }
 
 struct ChunkArgs {
     int L, Dch, d, ch;
     int ntiles;          // channel tiles per sequence (Dch / 128)
     int nchunks;         // chunks per sequence
+    int tok_base;        // first token of chunk 0 (L - nchunks * C, <= 0)
     int nseg, segc;      // segments per sequence, chunks per segment (all but the last)
-    const float2 *lam;   // [H][d]
+    int items;
     const uint8_t *consts;
+    __nv_bfloat16 *y;    // for the rows of a chunk that starts before token 0
     float *state_out;    // [B][d][Dch][2]
     int *sched;          // [0] ticket counter, [1] error code
     int *status;         // [items]: 0 none, 1 segment contribution, 2 inclusive state
-    float2 *agg;         // [items][d][128]
-    float2 *inc;         // [items][d][128]
+    float *agg;          // [items][32 rows][128 ch]
+    float *inc;          // [items][32 rows][128 ch]
 };
+
+struct Item {
+    int id, b, c0, hd, seg, ck0, nck, n1, niter;
+    bool last_seg;
+};
+
+__device__ __forceinline__ Item decode_item(const ChunkArgs &a, int id) {
+    Item it;
+    it.id = id;
+    const int unit = id / a.nseg;
+    it.seg = id % a.nseg;
+    it.b = unit / a.ntiles;
+    it.c0 = (unit % a.ntiles) * kNC;
+    it.hd = it.c0 / a.ch;
+    it.ck0 = it.seg * a.segc;
+    it.nck = min(a.nchunks, it.ck0 + a.segc) - it.ck0;
+    it.last_seg = (it.seg == a.nseg - 1);
+    it.n1 = it.last_seg ? 0 : it.nck;        // state-only iterations
+    it.niter = it.n1 + it.nck;
+    return it;
+}
 
 enum : int { kErrWait = 1, kErrLookback = 2 };
 
@@ -156,6 +185,21 @@ __device__ __forceinline__ void record_error(const ChunkArgs &a, volatile int *a
     atomicCAS(a.sched + 1, 0, code);
 }
 
+// One step x <- lam x + a of a complex recurrence held as (Re, Im) in the lanes r and r ^ 16 of a
+// warp (sgn = -1 in the Re lanes, +1 in the Im lanes).  Used for every segment-state combination,
+// so that the same inputs always give the same bits.
+__device__ __forceinline__ float seg_step(float x, float a, float2 lam, float sgn) {
+    const float xp = __shfl_xor_sync(0xffffffffu, x, 16);
+    return fmaf(lam.x, x, fmaf(sgn * lam.y, xp, a));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&p);
+}
+__device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+
 // ------------------------------------------------------------------ per-head constants
 __global__ void __launch_bounds__(256)
 chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R,
@@ -163,10 +207,9 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
                     uint8_t *__restrict__ consts) {
     const int hd = blockIdx.x;
     uint8_t *base = consts + (size_t)hd * kConstStride;
-    float *TT = reinterpret_cast<float *>(base + kSmTT);
-    float *VT = reinterpret_cast<float *>(base + kSmVT);
-    float *AT = reinterpret_cast<float *>(base + kSmAT);
-    float2 *lamC = reinterpret_cast<float2 *>(base + kTTBytes + kATBytes + kVTBytes);
+    __nv_bfloat16 *FA = reinterpret_cast<__nv_bfloat16 *>(base);
+    __nv_bfloat16 *CA = reinterpret_cast<__nv_bfloat16 *>(base + kFABytes);
+    float2 *lamC = reinterpret_cast<float2 *>(base + kLamOff);
     float2 *lamS = lamC + kMaxModes;
     __shared__ double hs[kC];
     const float2 *lh = lam + (size_t)hd * d;
@@ -185,33 +228,33 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
         hs[j] = acc;
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < kC * kC; e += blockDim.x) {
-        const int tau = e / kC, io = e % kC;
-        const float v = io <= tau ? (float)hs[tau - io] : 0.f;
-        TT[cm_off(tau, io, kC) / 4] = tc::to_tf32(v);
+    // fused A operand: rows 0..C-1 Toeplitz taps, rows C..C+31 chunk powers (Re at r < 16, Im at
+    // 16 + n), rows C+32..127 zero
+    for (int e = threadIdx.x; e < 128 * kC; e += blockDim.x) {
+        const int row = e / kC, io = e % kC;
+        double v = 0.0;
+        if (row < kC) {
+            v = io <= row ? hs[row - io] : 0.0;
+        } else if (row < kC + kKS) {
+            const int r = row - kC, n = r & (kIm - 1);
+            if (n < d) {
+                const cd p = cdpow(cd{lh[n].x, lh[n].y}, kC - 1 - io);
+                v = r < kIm ? p.x : p.y;
+            }
+        }
+        FA[cm_off16(row, io, kC) / 2] = __float2bfloat16_rn((float)v);
     }
-    // columns r < 16: real parts of mode r; columns 16 + n: imaginary parts of mode n
-    for (int e = threadIdx.x; e < kC * kKSMax; e += blockDim.x) {
-        const int tau = e / kKSMax, r = e % kKSMax;
-        const int n = r & (kIm - 1);
-        float v = 0.f;
-        if (n < d) {
-            const cd p = cdpow(cd{lh[n].x, lh[n].y}, tau);
+    // carry A operand: rows 0..C-1: (Re, -Im) of R_n lambda_n^tau; rows C..127 zero
+    for (int e = threadIdx.x; e < 128 * kKS; e += blockDim.x) {
+        const int row = e / kKS, r = e % kKS, n = r & (kIm - 1);
+        double v = 0.0;
+        if (row < kC && n < d) {
+            const cd p = cdpow(cd{lh[n].x, lh[n].y}, row);
             const double re = (double)rh[n].x * p.x - (double)rh[n].y * p.y;
             const double im = (double)rh[n].x * p.y + (double)rh[n].y * p.x;
-            v = r < kIm ? (float)re : (float)(-im);
+            v = r < kIm ? re : -im;
         }
-        AT[cm_off(tau, r, kKSMax) / 4] = tc::to_tf32(v);
-    }
-    for (int e = threadIdx.x; e < kKSMax * kC; e += blockDim.x) {
-        const int r = e / kC, io = e % kC;
-        const int n = r & (kIm - 1);
-        float v = 0.f;
-        if (n < d) {
-            const cd p = cdpow(cd{lh[n].x, lh[n].y}, kC - 1 - io);
-            v = r < kIm ? (float)p.x : (float)p.y;
-        }
-        VT[cm_off(r, io, kC) / 4] = tc::to_tf32(v);
+        CA[cm_off16(row, r, kKS) / 2] = __float2bfloat16_rn((float)v);
     }
     for (int n = threadIdx.x; n < kMaxModes; n += blockDim.x) {
         cd pc{0.0, 0.0}, ps{0.0, 0.0};
@@ -224,16 +267,15 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
     }
 }
 
-
 // ------------------------------------------------------------------ main kernel
-// Roles (warps):  0-3  U group: u = k*v -> U operand (ldmatrix transpose), one chunk at a time
-//                 4-7  S group: one thread per channel; state chain, segment publish, look-back
-//                 8-11 E group: one thread per channel; gate y = q * D1, stage y for the store
-//                 12   k,v TMA loads    13  q TMA loads    14  y TMA stores (lane 0 each; a
-//                      warp of their own so that one role's blocking wait never holds another)
-//                 15   tensor memory owner and MMA issuer (lane 0)
-// The groups run their own loops over the same chunk sequence and meet only at mbarriers, so
-// the U group forms chunk i+1 while the S group advances chunk i and the E group gates i-1.
+// Roles (warps):  0  k,v TMA loads; takes item tickets and posts them to the other roles
+//                 1  q TMA loads            12  y TMA stores (lane 0 each)
+//                 3  tensor memory owner and MMA issuer (lane 0)
+//                 7, 11, 13, 15   U group: U = k v over the k tile (elementwise)
+//                 2, 6, 10, 14    S group: state rows 0..31 x 32 channels each; chain, publish, look-back
+//                 4, 5, 8, 9      E group: token rows 0..63 x 64 channels each; gate and stage y
+// Each role loops over the same item sequence and the same chunk order; they meet only at
+// mbarriers, so loads, U, the products, the chain and the epilogue of different chunks overlap.
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_y,
@@ -243,417 +285,476 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint32_t sbase = tc::smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     auto bar = [&](int slot) { return sbase + kSmBar + 8u * slot; };
-    volatile int *misc = reinterpret_cast<volatile int *>(sm + kSmMisc);   // item, abort, tmem, never
-    volatile int *abort = misc + 1;
-    volatile int *never = misc + 3;
+    volatile int *itemq = reinterpret_cast<volatile int *>(sm + kSmMisc);   // [kItemQ]
+    volatile int *misc = itemq + kItemQ;                                     // abort, tmem, never
+    volatile int *abort = misc;
+    volatile int *never = misc + 2;
 
     if (tid == 0) {
-        misc[0] = atomicAdd(a.sched, 1);
-        misc[1] = 0;
-        misc[3] = 0;
+        misc[0] = 0;
+        misc[2] = 0;
         for (int i = 0; i < kNumBars; ++i) tc::mbar_init(bar(i), bar_count(i));
         tc::fence_mbar_init();
     }
-    if (warp == 15) {
-        tc::tmem_alloc(tc::smem_u32((const void *)(misc + 2)), kTmemCols);
+    if (warp == kWarpMMA) {
+        tc::tmem_alloc(tc::smem_u32((const void *)(misc + 1)), kTmemCols);
         tc::tmem_relinquish();
     }
-    __syncthreads();
-    const int item = misc[0];
-    const int unit = item / a.nseg, seg = item % a.nseg;
-    const int b = unit / a.ntiles, c0 = (unit % a.ntiles) * kNC;
-    const int hd = c0 / a.ch;
-    const int ck0 = seg * a.segc;
-    const int nck = min(a.nchunks, ck0 + a.segc) - ck0;
-    const bool last_seg = (seg == a.nseg - 1);
-    const bool phase1 = !last_seg;
-    const int n1 = phase1 ? nck : 0;                  // state-only iterations
-    const int niter = n1 + nck;
-    const int d = a.d;
-
-    // per-head constants -> shared memory; zero the state operands (their padding columns stay 0)
-    {
-        const int4 *src = reinterpret_cast<const int4 *>(a.consts + (size_t)hd * kConstStride);
-        int4 *dst = reinterpret_cast<int4 *>(sm);
-        for (int i = tid; i < (kTTBytes + kATBytes + kVTBytes + 2 * kMaxModes * 8) / 16; i += kThreads)
-            dst[i] = __ldg(src + i);      // [T; V], A and lambda^C, lambda^Lseg
-        int4 *stz = reinterpret_cast<int4 *>(sm + kSmST);
-        for (int i = tid; i < kSTBufs * kSTBytes / 16; i += kThreads) stz[i] = make_int4(0, 0, 0, 0);
-    }
-    tc::fence_proxy_async_smem();
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    const uint32_t tmem = (uint32_t)misc[2];
-    auto chunk_of = [&](int it) { return ck0 + (it < n1 ? it : it - n1); };
+    const uint32_t tmem = (uint32_t)misc[1];
+    const int d = a.d;
     auto uni = [&](bool x) -> bool { return __all_sync(0xffffffffu, x && !*abort); };
+    auto tok_of = [&](int chunk) { return a.tok_base + chunk * kC; };
 
-    if (warp >= 12 && warp <= 14) {
-        // ------------------------------------------------------------ TMA warps
-        if (warp == 12 && lane == 0) {      // k, v for every iteration (state-only pass, then full pass)
-            // L2 prefetch runs kPrefetch chunks ahead of the loads, so that many more bytes are in
-            // flight than the shared-memory stages hold (loaded DRAM latency is several us here)
-            for (int it = 0; it < min(kPrefetch, n1 > 0 ? n1 : nck); ++it)
-                for (int h = 0; h < 2; ++h) {
-                    tc::tma_prefetch_3d(&tm_k, c0 + 64 * h, chunk_of(it) * kC, b);
-                    tc::tma_prefetch_3d(&tm_v, c0 + 64 * h, chunk_of(it) * kC, b);
-                }
-            int it = 0;
-            for (; it < niter; ++it) {
-                // the full pass re-reads k, v that the state-only pass brought into L2
-                const int pf = it + kPrefetch;
-                if (pf < (n1 > 0 ? n1 : nck))
-                    for (int h = 0; h < 2; ++h) {
-                        tc::tma_prefetch_3d(&tm_k, c0 + 64 * h, chunk_of(pf) * kC, b);
-                        tc::tma_prefetch_3d(&tm_v, c0 + 64 * h, chunk_of(pf) * kC, b);
-                    }
-                const int s = it % kKVStages;
-                if (!tc::mbar_wait(bar(kBarKVEmpty + s), ((it / kKVStages) & 1) ^ 1, abort)) {
-                    record_error(a, abort, kErrWait);
-                    break;
-                }
-                const uint32_t dst = sbase + kSmKV + s * 2 * kTileBytes;
-                const int t0 = chunk_of(it) * kC;
-                tc::mbar_expect_tx(bar(kBarKVFull + s), 2 * kTileBytes);
-                for (int h = 0; h < 2; ++h) {
-                    tc::tma_load_3d(dst + h * kHalfBytes, &tm_k, bar(kBarKVFull + s), c0 + 64 * h, t0, b);
-                    tc::tma_load_3d(dst + kTileBytes + h * kHalfBytes, &tm_v, bar(kBarKVFull + s), c0 + 64 * h, t0, b);
-                }
-            }
-            if (*abort)
-                for (int j = max(0, it - kKVStages); j < it; ++j)
-                    tc::mbar_wait(bar(kBarKVFull + j % kKVStages), (j / kKVStages) & 1, never);
-        } else if (warp == 13 && lane == 0) {   // q for the full pass (the buffer then stages y)
-            for (int j = 0; j < min(kPrefetch, nck); ++j)
-                for (int h = 0; h < 2; ++h) tc::tma_prefetch_3d(&tm_q, c0 + 64 * h, (ck0 + j) * kC, b);
-            int j = 0;
-            for (; j < nck; ++j) {
-                if (j + kPrefetch < nck)
-                    for (int h = 0; h < 2; ++h)
-                        tc::tma_prefetch_3d(&tm_q, c0 + 64 * h, (ck0 + j + kPrefetch) * kC, b);
-                const int s = j % kQStages;
-                if (!tc::mbar_wait(bar(kBarQEmpty + s), ((j / kQStages) & 1) ^ 1, abort)) {
-                    record_error(a, abort, kErrWait);
-                    break;
-                }
-                tc::mbar_expect_tx(bar(kBarQFull + s), kTileBytes);
-                for (int h = 0; h < 2; ++h)
-                    tc::tma_load_3d(sbase + kSmQ + s * kTileBytes + h * kHalfBytes, &tm_q, bar(kBarQFull + s),
-                                    c0 + 64 * h, (ck0 + j) * kC, b);
-            }
-            if (*abort)
-                for (int jj = max(0, j - kQStages); jj < j; ++jj)
-                    tc::mbar_wait(bar(kBarQFull + jj % kQStages), (jj / kQStages) & 1, never);
-        } else if (warp == 14 && lane == 0) {   // y: one TMA store per gated tile, then the buffer goes back to q
-            for (int j = 0; j < nck; ++j) {
-                const int s = j % kQStages;
-                if (!tc::mbar_wait(bar(kBarYStaged + s), (j / kQStages) & 1, abort)) {
-                    record_error(a, abort, kErrWait);
-                    break;
-                }
-                for (int h = 0; h < 2; ++h)
-                    tc::tma_store_3d(&tm_y, sbase + kSmQ + s * kTileBytes + h * kHalfBytes, c0 + 64 * h,
-                                     (ck0 + j) * kC, b);
-                tc::bulk_commit();
-                tc::bulk_wait_read<0>();
-                tc::mbar_arrive(bar(kBarQEmpty + s));
-            }
-            tc::bulk_wait<0>();     // every store of this CTA has completed
-        }
-    } else if (warp == 15) {
-        // ------------------------------------------------------------ MMA issuer
-        // Two streams issued out of order from one thread (polled with non-blocking tests, since
-        // a suspending wait on one stream would hold back the other): the fused product of a chunk
-        // (needs only its U operand and a free accumulator) runs ahead, the carry product
-        // (needs the state entering the chunk) follows when the S group delivers it.  MMAs from
-        // one thread execute in issue order, so a chunk's carry always lands after its fused part.
+    // consumer side of the item queue: the id of the k-th item (-1 at the end), or -2 on abort.
+    // `lead` threads (one per consumer role or warp) release the slot after reading it.
+    // Warp-wide callers (all 32 lanes) pass warpwide = true: every lane reads before lane 0 releases.
+    auto take_item = [&](int k, bool warpwide) -> int {
+        const int s = k % kItemQ;
+        bool got = tc::mbar_wait(bar(kBarItemFull + s), (k / kItemQ) & 1, abort);
+        if (warpwide) got = __all_sync(0xffffffffu, got);
+        if (!got) return -2;
+        const int id = itemq[s];
+        if (warpwide) __syncwarp();
+        if (!warpwide || lane == 0) tc::mbar_arrive(bar(kBarItemEmpty + s));
+        return id;
+    };
+
+    if (warp == kWarpKV) {
+        // ------------------------------------------------------------ k,v loads + tickets
         if (lane == 0) {
-            const uint32_t idesc_f = tc::idesc_tf32(kNC, kAccCols);
-            const uint32_t idesc_c = tc::idesc_tf32(kNC, kC);
-            int ic = 0, jn = 0;
-            unsigned long long t_prog = tc::global_ns();
-            while ((ic < niter || jn < nck) && !*abort) {
-                bool progressed = false;
-                if (jn < nck && n1 + jn < ic) {
-                    const int sb = jn % kSTBufs, ab = (n1 + jn) % kNAcc;
-                    if (tc::mbar_test(bar(kBarSRdy + sb), (jn / kSTBufs) & 1)) {
-                        tc::tc_fence_after();
-                        // carry: D[0:C) += S A^T
-                        const uint32_t d = tmem + ab * kAccCols;
-                        const uint32_t stb = sbase + kSmST + sb * kSTBytes;
-                        for (int ks = 0; ks < kKSMax / 8; ++ks)
-                            tc::mma_tf32(d, tc::smem_desc(stb + ks * 256, 128, kKSMax * 32),
-                                         tc::smem_desc(sbase + kSmAT + ks * 256, 128, kKSMax * 32), idesc_c, 1);
-                        tc::mma_commit(bar(kBarYDone + ab));
-                        tc::mma_commit(bar(kBarSTFree + sb));
-                        ++jn;
-                        progressed = true;
-                    }
+            int g = 0;
+            bool ok = true;
+            for (int k = 0; ok; ++k) {
+                const int s = k % kItemQ;
+                if (!tc::mbar_wait(bar(kBarItemEmpty + s), ((k / kItemQ) & 1) ^ 1, abort)) {
+                    ok = false;
+                    break;
                 }
-                if (ic < niter) {
-                    const int ub = ic % kUBufs, ab = ic % kNAcc;
-                    bool ready = tc::mbar_test(bar(kBarURdy + ub), (ic / kUBufs) & 1) &&
-                                 tc::mbar_test(bar(kBarD2Free + ab), ((ic / kNAcc) & 1) ^ 1);
-                    if (ready && ic >= n1)   // phase-2 uses of this accumulator (n1 % kNAcc == 0)
-                        ready = tc::mbar_test(bar(kBarD1Free + ab), (((ic - n1) / kNAcc) & 1) ^ 1);
-                    if (ready) {
-                        tc::tc_fence_after();
-                        // fused: D[0:C+32) = U [T; V]^T  (intra-chunk output | state contribution)
-                        const uint32_t d = tmem + ab * kAccCols;
-                        const uint32_t ut = sbase + kSmUT + ub * kUTBytes;
-                        for (int ks = 0; ks < kC / 8; ++ks)
-                            tc::mma_tf32(d, tc::smem_desc(ut + ks * 256, 128, kC * 32),
-                                         tc::smem_desc(sbase + kSmTT + ks * 256, 128, kC * 32), idesc_f, ks > 0);
-                        tc::mma_commit(bar(kBarWDone + ab));
-                        tc::mma_commit(bar(kBarUFree + ub));
-                        ++ic;
-                        progressed = true;
-                    }
-                }
-                if (progressed) {
-                    t_prog = tc::global_ns();
-                } else {
-                    if (tc::global_ns() - t_prog > tc::kWaitNs) {
-                        record_error(a, abort, kErrWait);
+                int id = atomicAdd(a.sched, 1);
+                if (id >= a.items) id = -1;
+                itemq[s] = id;
+                tc::mbar_arrive(bar(kBarItemFull + s));
+                if (id < 0) break;
+                const Item it = decode_item(a, id);
+                for (int i = 0; i < it.niter; ++i, ++g) {
+                    const int chunk = it.ck0 + (i < it.n1 ? i : i - it.n1);
+                    const int st = g % kKVStages;
+                    if (!tc::mbar_wait(bar(kBarKVEmpty + st), ((g / kKVStages) & 1) ^ 1, abort)) {
+                        ok = false;
                         break;
                     }
-                    __nanosleep(32);      // polling: leave issue slots to the warps sharing the SMSP
+                    const uint32_t dst = sbase + kSmKV + st * kStageBytes;
+                    tc::mbar_expect_tx(bar(kBarKVFull + st), kStageBytes);
+                    for (int h = 0; h < 2; ++h) {
+                        tc::tma_load_3d(dst + h * kHalf, &tm_k, bar(kBarKVFull + st), it.c0 + 64 * h, tok_of(chunk), it.b);
+                        tc::tma_load_3d(dst + kTile + h * kHalf, &tm_v, bar(kBarKVFull + st), it.c0 + 64 * h,
+                                        tok_of(chunk), it.b);
+                    }
                 }
             }
+            if (!ok) {
+                record_error(a, abort, kErrWait);
+                // drain the loads still in flight before the CTA may exit
+                for (int j = max(0, g - kKVStages); j < g; ++j)
+                    tc::mbar_wait(bar(kBarKVFull + j % kKVStages), (j / kKVStages) & 1, never);
+            }
+        }
+    } else if (warp == kWarpQ) {
+        // ------------------------------------------------------------ q loads (full passes only)
+        if (lane == 0) {
+            int qg = 0;
+            bool ok = true;
+            for (int k = 0; ok; ++k) {
+                const int id = take_item(k, false);
+                if (id == -2) ok = false;
+                if (id < 0) break;
+                const Item it = decode_item(a, id);
+                for (int j = 0; j < it.nck; ++j, ++qg) {
+                    const int s = qg % kQStages;
+                    if (!tc::mbar_wait(bar(kBarQEmpty + s), ((qg / kQStages) & 1) ^ 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::mbar_expect_tx(bar(kBarQFull + s), kTile);
+                    for (int h = 0; h < 2; ++h)
+                        tc::tma_load_3d(sbase + kSmQ + s * kTile + h * kHalf, &tm_q, bar(kBarQFull + s),
+                                        it.c0 + 64 * h, tok_of(it.ck0 + j), it.b);
+                }
+            }
+            if (!ok) {
+                record_error(a, abort, kErrWait);
+                for (int j = max(0, qg - kQStages); j < qg; ++j)
+                    tc::mbar_wait(bar(kBarQFull + j % kQStages), (j / kQStages) & 1, never);
+            }
+        }
+    } else if (warp == kWarpStore) {
+        // ------------------------------------------------------------ y stores
+        if (lane == 0) {
+            int qg = 0;
+            bool ok = true;
+            for (int k = 0; ok; ++k) {
+                const int id = take_item(k, false);
+                if (id == -2) ok = false;
+                if (id < 0) break;
+                const Item it = decode_item(a, id);
+                for (int j = 0; j < it.nck; ++j, ++qg) {
+                    const int s = qg % kQStages;
+                    if (!tc::mbar_wait(bar(kBarYStaged + s), (qg / kQStages) & 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    const int tok = tok_of(it.ck0 + j);
+                    if (tok >= 0) {     // a chunk that starts before token 0 was written by the E group
+                        for (int h = 0; h < 2; ++h)
+                            tc::tma_store_3d(&tm_y, sbase + kSmQ + s * kTile + h * kHalf, it.c0 + 64 * h, tok, it.b);
+                        tc::bulk_commit();
+                        tc::bulk_wait_read<0>();
+                    }
+                    tc::mbar_arrive(bar(kBarQEmpty + s));
+                }
+            }
+            if (!ok) record_error(a, abort, kErrWait);
+            tc::bulk_wait<0>();     // every store of this CTA has completed
+        }
+    } else if (warp == kWarpMMA) {
+        // ------------------------------------------------------------ MMA issuer
+        // Two streams issued out of order from one thread (polled with non-blocking tests): the
+        // fused product of a chunk needs only its U operand and a free accumulator slot and runs
+        // ahead; the carry needs the state entering the chunk and follows when the S group
+        // delivers it.  MMAs from one thread execute in issue order.
+        if (lane == 0) {
+            const uint32_t idesc = tc::idesc_bf16(128, kNC, true);
+            int g = 0, pc = 0, cur_hd = -1, cphase = 0, fphase = 0;
+            int c2[kSlots] = {0, 0};    // full-pass uses of each slot issued so far
+            bool any = false, ok = true;
+            for (int k = 0; ok; ++k) {
+                const int id = take_item(k, false);
+                if (id == -2) ok = false;
+                if (id < 0) break;
+                const Item it = decode_item(a, id);
+                if (it.hd != cur_hd) {
+                    // new head: wait until no MMA reads the old constants, then copy the new ones
+                    if (any) {
+                        tc::mma_commit(bar(kBarConstFree));
+                        if (!tc::mbar_wait(bar(kBarConstFree), fphase & 1, abort)) { ok = false; break; }
+                        ++fphase;
+                    }
+                    tc::mbar_expect_tx(bar(kBarConst), kOpBytes);
+                    tc::bulk_load(sbase + kSmFA, a.consts + (size_t)it.hd * kConstStride, kOpBytes, bar(kBarConst));
+                    if (!tc::mbar_wait(bar(kBarConst), cphase & 1, never)) { ok = false; break; }
+                    ++cphase;
+                    cur_hd = it.hd;
+                }
+                const int g0 = g;
+                int ic = 0, jn = 0;
+                unsigned long long t_prog = tc::global_ns();
+                while ((ic < it.niter || jn < it.nck) && !*abort) {
+                    bool progressed = false;
+                    if (jn < it.nck && it.n1 + jn < ic) {
+                        const int sb = pc % kSBufs;
+                        if (tc::mbar_test(bar(kBarSRdy + sb), (pc / kSBufs) & 1)) {
+                            tc::tc_fence_after();
+                            // carry: Z += A S  (own TMEM columns of the chunk's slot)
+                            const int slot = (g0 + it.n1 + jn) % kSlots;
+                            const uint32_t dcol = tmem + slot * kSlotCols + kNC;
+                            const uint32_t sb_addr = sbase + kSmS + sb * kSBytes;
+                            for (int ks = 0; ks < kKS / 16; ++ks)
+                                tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmCA + ks * 256, 128, kKS * 16),
+                                             tc::smem_desc_sw128(sb_addr + ks * 2048, kSBytes / 2, 1024), idesc, ks > 0);
+                            tc::mma_commit(bar(kBarYDone + slot));
+                            tc::mma_commit(bar(kBarSTFree + sb));
+                            ++jn;
+                            ++pc;
+                            progressed = true;
+                        }
+                    }
+                    if (ic < it.niter) {
+                        const int gi = g0 + ic, slot = gi % kSlots, st = gi % kKVStages;
+                        bool ready = tc::mbar_test(bar(kBarURdy + st), (gi / kKVStages) & 1) &&
+                                     tc::mbar_test(bar(kBarD2Free + slot), ((gi / kSlots) & 1) ^ 1) &&
+                                     tc::mbar_test(bar(kBarD1Free + slot), (c2[slot] & 1) ^ 1);
+                        if (ready) {
+                            tc::tc_fence_after();
+                            // fused: [Z; W] = [T; V] U
+                            const uint32_t dcol = tmem + slot * kSlotCols;
+                            const uint32_t u_addr = sbase + kSmKV + st * kStageBytes;
+                            for (int ks = 0; ks < kC / 16; ++ks)
+                                tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmFA + ks * 256, 128, kC * 16),
+                                             tc::smem_desc_sw128(u_addr + ks * 2048, kHalf, 1024), idesc, ks > 0);
+                            tc::mma_commit(bar(kBarWDone + slot));
+                            tc::mma_commit(bar(kBarKVEmpty + st));
+                            if (ic >= it.n1) ++c2[slot];
+                            ++ic;
+                            any = true;
+                            progressed = true;
+                        }
+                    }
+                    if (progressed) {
+                        t_prog = tc::global_ns();
+                    } else {
+                        if (tc::global_ns() - t_prog > tc::kWaitNs) {
+                            ok = false;
+                            break;
+                        }
+                        __nanosleep(20);
+                    }
+                }
+                if (*abort) ok = false;
+                g = g0 + it.niter;
+            }
+            if (!ok) record_error(a, abort, kErrWait);
             // all MMAs issued by this thread have completed once `drain` fires
             tc::mma_commit(bar(kBarDrain));
             tc::mbar_wait(bar(kBarDrain), 0, never);
         }
-    } else if (warp < 4) {
-        // ------------------------------------------------------------ U group
-        // u = k*v of each chunk -> U operand buffer (it % kUBufs).  ldmatrix transposes the
-        // 128-byte-swizzled k, v tiles: warp w covers channel groups 4w..4w+3 (8 channels each)
-        // and each lane receives token pairs of one channel, the K-major row layout of U.
-        // Tokens past the prompt were zero-filled by TMA.
+    } else if (u_index(warp) >= 0) {
+        // ------------------------------------------------------------ U group: U = k v in place
+        const int ut = u_index(warp) * 32 + lane;
+        int g = 0;
         bool ok = true;
-        const int r8 = lane & 7, mat = lane >> 3;
-        for (int it = 0; it < niter && ok; ++it) {
-            const int ub = it % kUBufs, s = it % kKVStages;
-            ok = uni(tc::mbar_wait(bar(kBarUFree + ub), ((it / kUBufs) & 1) ^ 1, abort) &&
-                     tc::mbar_wait(bar(kBarKVFull + s), (it / kKVStages) & 1, abort));
-            if (!ok) break;
-            const uint32_t kb = sbase + kSmKV + s * 2 * kTileBytes;
-            uint8_t *ut = sm + kSmUT + ub * kUTBytes;
+        for (int k = 0; ok; ++k) {
+            const int id = take_item(k, true);
+            if (id == -2) ok = false;
+            if (id < 0) break;
+            const Item it = decode_item(a, id);
+            for (int i = 0; i < it.niter; ++i, ++g) {
+                const int st = g % kKVStages;
+                if (!(ok = uni(tc::mbar_wait(bar(kBarKVFull + st), (g / kKVStages) & 1, abort)))) break;
+                uint8_t *kt = sm + kSmKV + st * kStageBytes;
 #pragma unroll
-            for (int gi = 0; gi < 4; ++gi) {
-                const int cbase = 8 * (4 * warp + gi);
-                const uint32_t off = (uint32_t)((cbase >> 6) * kHalfBytes + (8 * mat + r8) * 128 +
-                                                ((((cbase & 63) >> 3) ^ r8) << 4));
-                uint32_t kr[4], vr[4];
-                tc::ldsm_x4_trans(kb + off, kr);
-                tc::ldsm_x4_trans(kb + kTileBytes + off, vr);
-                const int ch = cbase + (lane >> 2);
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const int tau = 8 * m + 2 * (lane & 3);
-                    const float u0 = __uint_as_float(kr[m] << 16) * __uint_as_float(vr[m] << 16);
-                    const float u1 = __uint_as_float(kr[m] & 0xffff0000u) * __uint_as_float(vr[m] & 0xffff0000u);
-                    *reinterpret_cast<float2 *>(ut + cm_off(ch, tau, kC)) = make_float2(tc::to_tf32(u0), tc::to_tf32(u1));
+                for (int m = 0; m < kTile / 16 / 128; ++m) {
+                    const int off = (ut + 128 * m) * 16;    // same byte offset in k, v and U
+                    const uint4 kk = *reinterpret_cast<const uint4 *>(kt + off);
+                    const uint4 vv = *reinterpret_cast<const uint4 *>(kt + kTile + off);
+                    uint4 uu;
+                    uu.x = pack_bf16(bf_lo(kk.x) * bf_lo(vv.x), bf_hi(kk.x) * bf_hi(vv.x));
+                    uu.y = pack_bf16(bf_lo(kk.y) * bf_lo(vv.y), bf_hi(kk.y) * bf_hi(vv.y));
+                    uu.z = pack_bf16(bf_lo(kk.z) * bf_lo(vv.z), bf_hi(kk.z) * bf_hi(vv.z));
+                    uu.w = pack_bf16(bf_lo(kk.w) * bf_lo(vv.w), bf_hi(kk.w) * bf_hi(vv.w));
+                    *reinterpret_cast<uint4 *>(kt + off) = uu;
                 }
+                tc::fence_proxy_async_smem();
+                tc::mbar_arrive(bar(kBarURdy + st));
             }
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(bar(kBarURdy + ub));
-            // the prompt's last chunk stays until the S group has read it for the final state
-            if (!(it >= n1 && chunk_of(it) == a.nchunks - 1)) tc::mbar_arrive(bar(kBarKVEmpty + s));
         }
         if (!ok) record_error(a, abort, kErrWait);
-    } else if (warp < 8) {
+    } else if (is_s_warp(warp)) {
         // ------------------------------------------------------------ S group (state chain)
-        const int c = tid - 128;                     // channel within the tile == TMEM lane
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        // lambda^C and lambda^Lseg stay in shared memory (broadcast reads) to keep this
-        // group's registers for the state itself
-        const float2 *lamC = reinterpret_cast<const float2 *>(sm + kSmLam);
-        const float2 *lamS = lamC + kMaxModes;
-        float2 st[kMaxModes];
-#pragma unroll
-        for (int n = 0; n < kMaxModes; ++n) st[n] = make_float2(0.f, 0.f);
+        // thread: state row r = lane (mode r % 16, Re for r < 16, Im above) for channels
+        // 32 q4 .. 32 q4 + 31 of the tile; TMEM lane 64 + r holds row r of the state product W
+        const int q4 = warp >> 2, r = lane, n = r & (kIm - 1);
+        const bool leader = (warp == 2 && lane == 0);
+        const float sgn = (r < kIm) ? -1.f : 1.f;
+        const uint32_t lane_base = (uint32_t)64 << 16;
+        int g = 0, pc = 0, pub_phase = 0;
         bool ok = true;
-        int pub_phase = 0;
-        // st <- lambda^C st + D2 of iteration it
-        auto advance = [&](int it) -> bool {
-            const int wb = it % kNAcc;
-            if (!tc::mbar_wait(bar(kBarWDone + wb), (it / kNAcc) & 1, abort)) return false;
-            tc::tc_fence_after();
-            float w[kKSMax];
-            const uint32_t taddr = tmem + lane_base + wb * kAccCols + kC;
-            tc::tmem_ld16(taddr, w);
-            tc::tmem_ld16(taddr + 16, w + 16);
-            tc::tmem_wait_ld();
-            tc::tc_fence_before();
-            tc::mbar_arrive(bar(kBarD2Free + wb));
+        float st[32];
+        for (int k = 0; ok; ++k) {
+            const int id = take_item(k, true);
+            if (id == -2) ok = false;
+            if (id < 0) break;
+            const Item it = decode_item(a, id);
+            const float2 *lp = reinterpret_cast<const float2 *>(a.consts + (size_t)it.hd * kConstStride + kLamOff);
+            const float2 lamC = lp[n], lamS = lp[kMaxModes + n];    // zero for modes >= d
 #pragma unroll
-            for (int n = 0; n < kMaxModes; ++n) {
-                const float2 sv = st[n], lc = lamC[n];      // lambda^C is 0 for modes >= d
-                st[n] = make_float2(fmaf(lc.x, sv.x, fmaf(-lc.y, sv.y, w[n])),
-                                    fmaf(lc.x, sv.y, fmaf(lc.y, sv.x, w[kIm + n])));
-            }
-            return true;
-        };
-        auto publish = [&](float2 *dst, int code) -> bool {
-            for (int n = 0; n < d; ++n) dst[(size_t)n * kNC + c] = st[n];
-            __threadfence();
-            tc::mbar_arrive(bar(kBarPub));
-            bool r = true;
-            if (c == 0) {
-                r = tc::mbar_wait(bar(kBarPub), pub_phase & 1, abort);
-                if (r) {
-                    __threadfence();
-                    atomicExch(a.status + item, code);
-                }
-            }
-            ++pub_phase;
-            return r;
-        };
+            for (int i = 0; i < 32; ++i) st[i] = 0.f;
 
-        // state-only pass over the segment, then publish its contribution
-        for (int it = 0; it < n1 && ok; ++it) ok = uni(advance(it));
-        if (ok && phase1) ok = uni(publish((seg == 0 ? a.inc : a.agg) + (size_t)item * d * kNC, seg == 0 ? 2 : 1));
-        float2 sloc[kMaxModes];
+            // st <- lambda^C st + W of iteration gi
+            auto advance = [&](int gi) -> bool {
+                const int slot = gi % kSlots;
+                if (!uni(tc::mbar_wait(bar(kBarWDone + slot), (gi / kSlots) & 1, abort))) return false;
+                tc::tc_fence_after();
+                float w[32];
+                tc::tmem_ld32(tmem + lane_base + slot * kSlotCols + 32 * q4, w);
+                tc::tmem_wait_ld();
+                tc::tc_fence_before();
+                tc::mbar_arrive(bar(kBarD2Free + slot));
 #pragma unroll
-        for (int n = 0; n < kMaxModes; ++n) { sloc[n] = st[n]; st[n] = make_float2(0.f, 0.f); }
-
-        // look-back: the state entering this segment
-        if (ok && seg > 0) {
-            float2 scale[kMaxModes];
-#pragma unroll
-            for (int n = 0; n < kMaxModes; ++n) scale[n] = make_float2(1.f, 0.f);
-            for (int p = item - 1; p >= item - seg && ok; --p) {
-                int code = *(volatile int *)(a.status + p);
-                const unsigned long long t0 = tc::global_ns();
-                while (code == 0 && !*abort && tc::global_ns() - t0 < tc::kWaitNs) {
-                    __nanosleep(100);
-                    code = *(volatile int *)(a.status + p);
+                for (int i = 0; i < 32; ++i) {
+                    const float p = __shfl_xor_sync(0xffffffffu, st[i], 16);    // the other part of mode n
+                    st[i] = fmaf(lamC.x, st[i], fmaf(sgn * lamC.y, p, w[i]));
                 }
-                if (code == 0) {
+                return true;
+            };
+            // this thread's row of a published [32 rows][128 ch] state (bypassing L1)
+            auto load_rows = [&](const float *src, float *o) {
+                const float4 *p4 = reinterpret_cast<const float4 *>(src + (size_t)r * kNC + 32 * q4);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float4 v4 = __ldcg(p4 + i);
+                    o[4 * i] = v4.x; o[4 * i + 1] = v4.y; o[4 * i + 2] = v4.z; o[4 * i + 3] = v4.w;
+                }
+            };
+            // write the state rows of this thread to dst [32 rows][128 ch], then post `code`
+            auto publish = [&](float *dst, int code) -> bool {
+                float4 *o = reinterpret_cast<float4 *>(dst + (size_t)r * kNC + 32 * q4);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) o[i] = make_float4(st[4 * i], st[4 * i + 1], st[4 * i + 2], st[4 * i + 3]);
+                __threadfence();
+                tc::mbar_arrive(bar(kBarPub));
+                bool res = true;
+                if (leader) {
+                    res = tc::mbar_wait(bar(kBarPub), pub_phase & 1, abort);
+                    if (res) {
+                        __threadfence();
+                        atomicExch(a.status + it.id, code);
+                    }
+                }
+                ++pub_phase;
+                return res;
+            };
+
+            // state-only pass over the segment, then publish its contribution
+            for (int i = 0; i < it.n1 && ok; ++i, ++g) ok = uni(advance(g));
+            if (!ok) break;
+            const size_t item_off = (size_t)it.id * kKS * kNC;
+            if (it.n1 > 0 && !(ok = uni(publish((it.seg == 0 ? a.inc : a.agg) + item_off, it.seg == 0 ? 2 : 1))))
+                break;
+            float sloc[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) { sloc[i] = st[i]; st[i] = 0.f; }
+
+            // look-back: the state entering this segment.  The inclusive states follow the fixed
+            // fp32 recurrence inc(s) = lambda^Lseg inc(s-1) + agg(s), inc(0) = agg(0): find the
+            // nearest predecessor that has posted its inclusive state, then replay the recurrence
+            // over the aggregates after it.  The result is bit-identical whichever predecessor
+            // was found, so the output does not depend on timing.
+            if (it.seg > 0) {
+                int p0 = -1;
+                for (int p = it.id - 1; p >= it.id - it.seg; --p) {
+                    int code = 0;
+                    if (lane == 0) {
+                        code = *(volatile int *)(a.status + p);
+                        const unsigned long long t0 = tc::global_ns();
+                        while (code == 0 && !*abort && tc::global_ns() - t0 < tc::kWaitNs) {
+                            __nanosleep(64);
+                            code = *(volatile int *)(a.status + p);
+                        }
+                    }
+                    code = __shfl_sync(0xffffffffu, code, 0);
+                    if (code == 0) break;
+                    if (code == 2) { p0 = p; break; }
+                }
+                if (p0 < 0) {           // segment 0 always posts an inclusive state: only a timeout lands here
                     record_error(a, abort, kErrLookback);
                     ok = false;
-                    break;
                 }
+                if (!(ok = uni(ok))) break;
                 __threadfence();
-                const volatile float2 *src = (code == 2 ? a.inc : a.agg) + (size_t)p * d * kNC;
+                load_rows(a.inc + (size_t)p0 * kKS * kNC, st);
+                for (int p = p0 + 1; p < it.id; ++p) {
+                    float ag[32];
+                    load_rows(a.agg + (size_t)p * kKS * kNC, ag);
 #pragma unroll
-                for (int n = 0; n < kMaxModes; ++n) {
-                    if (n < d) {
-                        const float2 v = make_float2(src[(size_t)n * kNC + c].x, src[(size_t)n * kNC + c].y);
-                        st[n] = cadd(st[n], cmul(scale[n], v));
-                        scale[n] = cmul(scale[n], lamS[n]);
+                    for (int i = 0; i < 32; ++i) st[i] = seg_step(st[i], ag[i], lamS, sgn);
+                }
+                if (it.n1 > 0) {
+                    // inclusive state at the end of this segment
+                    float keep[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        keep[i] = st[i];
+                        st[i] = seg_step(st[i], sloc[i], lamS, sgn);
                     }
-                }
-                if (code == 2) break;
-            }
-            ok = uni(ok);
-            if (ok && phase1) {
-                // inclusive state at the end of this segment: lambda^Lseg s_in + own contribution
-                float2 keep[kMaxModes];
+                    ok = uni(publish(a.inc + item_off, 2));
 #pragma unroll
-                for (int n = 0; n < kMaxModes; ++n) {
-                    keep[n] = st[n];
-                    st[n] = cadd(cmul(lamS[n], st[n]), sloc[n]);
+                    for (int i = 0; i < 32; ++i) st[i] = keep[i];
+                    if (!ok) break;
                 }
-                ok = uni(publish(a.inc + (size_t)item * d * kNC, 2));
-#pragma unroll
-                for (int n = 0; n < kMaxModes; ++n) st[n] = keep[n];
             }
-        }
 
-        // full pass: state operand for each chunk, then the state after it
-        for (int j = 0; j < nck && ok; ++j) {
-            const int it = n1 + j, sb = j % kSTBufs;
-            if (!(ok = uni(tc::mbar_wait(bar(kBarSTFree + sb), ((j / kSTBufs) & 1) ^ 1, abort)))) break;
-            uint8_t *stp = sm + kSmST + sb * kSTBytes;
+            // full pass: state operand for each chunk, then the state after it
+            for (int j = 0; j < it.nck && ok; ++j, ++g, ++pc) {
+                const int sb = pc % kSBufs;
+                if (!(ok = uni(tc::mbar_wait(bar(kBarSTFree + sb), ((pc / kSBufs) & 1) ^ 1, abort)))) break;
+                // row r of the MN-major, 128-byte swizzled [32 rows][128 ch] operand: channel block
+                // q4 is 64 bytes of row r in swizzle atom q4 / 2
+                uint8_t *sp = sm + kSmS + sb * kSBytes + (q4 >> 1) * (kSBytes / 2) + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-            for (int n4 = 0; n4 < kMaxModes / 4; ++n4) {
-                const int n = 4 * n4;
-                *reinterpret_cast<float4 *>(stp + cm_off(c, n, kKSMax)) =
-                    make_float4(tc::to_tf32(st[n].x), tc::to_tf32(st[n + 1].x), tc::to_tf32(st[n + 2].x),
-                                tc::to_tf32(st[n + 3].x));
-                *reinterpret_cast<float4 *>(stp + cm_off(c, kIm + n, kKSMax)) =
-                    make_float4(tc::to_tf32(st[n].y), tc::to_tf32(st[n + 1].y), tc::to_tf32(st[n + 2].y),
-                                tc::to_tf32(st[n + 3].y));
+                for (int i = 0; i < 4; ++i) {
+                    uint4 v;
+                    v.x = pack_bf16(st[8 * i + 0], st[8 * i + 1]);
+                    v.y = pack_bf16(st[8 * i + 2], st[8 * i + 3]);
+                    v.z = pack_bf16(st[8 * i + 4], st[8 * i + 5]);
+                    v.w = pack_bf16(st[8 * i + 6], st[8 * i + 7]);
+                    *reinterpret_cast<uint4 *>(sp + ((((q4 & 1) * 4 + i) ^ (r & 7)) << 4)) = v;
+                }
+                tc::fence_proxy_async_smem();
+                tc::mbar_arrive(bar(kBarSRdy + sb));
+                if (!(ok = uni(advance(g)))) break;
             }
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(bar(kBarSRdy + sb));
-            const int chunk = ck0 + j;
-            if (chunk != a.nchunks - 1) {
-                if (!(ok = uni(advance(it)))) break;
-            } else {
-                // last chunk of the prompt (possibly partial): exact fp32 Horner over its
-                // tokens, st <- lambda^rem st + sum_{iota<rem} lambda^(rem-1-iota) u_iota
-                const int s = it % kKVStages;
-                if (!(ok = uni(tc::mbar_wait(bar(kBarKVFull + s), (it / kKVStages) & 1, abort)))) break;
-                const int rem = a.L - chunk * kC;
-                const uint8_t *kt = sm + kSmKV + s * 2 * kTileBytes;
-                const uint8_t *vt = kt + kTileBytes;
-                float2 lm[kMaxModes], acc[kMaxModes];
+            if (!ok) break;
+            if (it.last_seg && n < d) {
+                float *so = a.state_out + (((size_t)it.b * d + n) * a.Dch + it.c0 + 32 * q4) * 2 + (r >> 4);
 #pragma unroll
-                for (int n = 0; n < kMaxModes; ++n) {
-                    lm[n] = n < d ? __ldg(&a.lam[(size_t)hd * d + n]) : make_float2(0.f, 0.f);
-                    acc[n] = make_float2(0.f, 0.f);
-                }
-                for (int io = 0; io < rem; ++io) {
-                    const int o = act_off(io, c);
-                    const float u = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(kt + o)) *
-                                    __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(vt + o));
-#pragma unroll
-                    for (int n = 0; n < kMaxModes; ++n)
-                        acc[n] = make_float2(fmaf(acc[n].x, lm[n].x, fmaf(-acc[n].y, lm[n].y, u)),
-                                             fmaf(acc[n].x, lm[n].y, acc[n].y * lm[n].x));
-                }
-                tc::mbar_arrive(bar(kBarKVEmpty + s));
-#pragma unroll
-                for (int n = 0; n < kMaxModes; ++n) {
-                    if (n < d) {
-                        const cd pw = cdpow(cd{lm[n].x, lm[n].y}, rem);
-                        st[n] = cadd(cmul(make_float2((float)pw.x, (float)pw.y), st[n]), acc[n]);
-                    }
-                }
+                for (int i = 0; i < 32; ++i) so[2 * i] = st[i];
             }
         }
         if (!ok) record_error(a, abort, kErrWait);
-        if (ok && last_seg) {
-            float2 *so = reinterpret_cast<float2 *>(a.state_out) + ((size_t)b * d) * a.Dch + c0 + c;
-            for (int n = 0; n < d; ++n) so[(size_t)n * a.Dch] = st[n];
-        }
-    } else {
+    } else if (is_e_warp(warp)) {
         // ------------------------------------------------------------ E group (gate and stage y)
-        const int c = tid - 256;
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        // thread: token row tau = 32 q4 + lane (TMEM lane tau) for channels 64 hh .. 64 hh + 63
+        const int q4 = warp & 3, hh = warp >> 3, tau = 32 * q4 + lane;
+        const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+        int g = 0, qg = 0;
+        int e2[kSlots] = {0, 0};
         bool ok = true;
-        for (int j = 0; j < nck && ok; ++j) {
-            const int db = j % kNAcc, s = j % kQStages;     // == (n1 + j) % kNAcc since n1 % kNAcc == 0
-            ok = uni(tc::mbar_wait(bar(kBarYDone + db), (j / kNAcc) & 1, abort) &&
-                     tc::mbar_wait(bar(kBarQFull + s), (j / kQStages) & 1, abort));
-            if (!ok) break;
-            tc::tc_fence_after();
-            uint8_t *qy = sm + kSmQ + s * kTileBytes;
-            __nv_bfloat16 qv[kC];
+        for (int k = 0; ok; ++k) {
+            const int id = take_item(k, true);
+            if (id == -2) ok = false;
+            if (id < 0) break;
+            const Item it = decode_item(a, id);
+            g += it.n1;
+            for (int j = 0; j < it.nck; ++j, ++g, ++qg) {
+                const int slot = g % kSlots, s = qg % kQStages;
+                ok = uni(tc::mbar_wait(bar(kBarYDone + slot), e2[slot] & 1, abort) &&
+                         tc::mbar_wait(bar(kBarQFull + s), (qg / kQStages) & 1, abort));
+                if (!ok) break;
+                ++e2[slot];
+                tc::tc_fence_after();
+                const int tok = tok_of(it.ck0 + j);
+                uint8_t *qrow = sm + kSmQ + s * kTile + hh * kHalf + tau * 128;
+                const bool store_direct = tok < 0, row_valid = tok + tau >= 0;
+                __nv_bfloat16 *yrow = a.y + ((size_t)it.b * a.L + (row_valid ? tok + tau : 0)) * a.Dch + it.c0 + 64 * hh;
 #pragma unroll
-            for (int tau = 0; tau < kC; ++tau) qv[tau] = *reinterpret_cast<const __nv_bfloat16 *>(qy + act_off(tau, c));
-            float z[kC];
-            tc::tmem_ld16(tmem + lane_base + db * kAccCols, z);
-            tc::tmem_ld16(tmem + lane_base + db * kAccCols + 16, z + 16);
-            tc::tmem_wait_ld();
-            tc::tc_fence_before();
-            tc::mbar_arrive(bar(kBarD1Free + db));
+                for (int x = 0; x < 2; ++x) {
+                    float z[32], cz[32];
+                    const uint32_t col = tmem + lane_base + slot * kSlotCols + 64 * hh + 32 * x;
+                    tc::tmem_ld32(col, z);
+                    tc::tmem_ld32(col + kNC, cz);
+                    tc::tmem_wait_ld();
 #pragma unroll
-            for (int tau = 0; tau < kC; ++tau)
-                *reinterpret_cast<__nv_bfloat16 *>(qy + act_off(tau, c)) =
-                    __float2bfloat16_rn(__bfloat162float(qv[tau]) * z[tau]);
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(bar(kBarYStaged + s));
+                    for (int i = 0; i < 4; ++i) {
+                        const int chunk16 = 4 * x + i;          // 16-byte chunk (8 channels) of the row
+                        uint4 *qp = reinterpret_cast<uint4 *>(qrow + ((chunk16 ^ (tau & 7)) << 4));
+                        const uint4 qv = *qp;
+                        const float *zz = z + 8 * i, *cc = cz + 8 * i;
+                        uint4 yv;
+                        yv.x = pack_bf16(bf_lo(qv.x) * (zz[0] + cc[0]), bf_hi(qv.x) * (zz[1] + cc[1]));
+                        yv.y = pack_bf16(bf_lo(qv.y) * (zz[2] + cc[2]), bf_hi(qv.y) * (zz[3] + cc[3]));
+                        yv.z = pack_bf16(bf_lo(qv.z) * (zz[4] + cc[4]), bf_hi(qv.z) * (zz[5] + cc[5]));
+                        yv.w = pack_bf16(bf_lo(qv.w) * (zz[6] + cc[6]), bf_hi(qv.w) * (zz[7] + cc[7]));
+                        if (!store_direct)
+                            *qp = yv;
+                        else if (row_valid)
+                            *reinterpret_cast<uint4 *>(yrow + 8 * chunk16) = yv;
+                    }
+                }
+                tc::tc_fence_before();
+                tc::mbar_arrive(bar(kBarD1Free + slot));
+                tc::fence_proxy_async_smem();
+                tc::mbar_arrive(bar(kBarYStaged + s));
+            }
         }
         if (!ok) record_error(a, abort, kErrWait);
     }
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    if (warp == 15) tc::tmem_dealloc(tmem, kTmemCols);
+    if (warp == kWarpMMA) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
 // ------------------------------------------------------------------ host side
@@ -669,7 +770,7 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-// [B][L][Dch] bf16 viewed as a 3-D tensor (Dch, L, B); box = 128 channels x C tokens x 1
+// [B][L][Dch] bf16 viewed as a 3-D tensor (Dch, L, B); box = 64 channels x C tokens x 1
 bool make_map(CUtensorMap *m, const void *base, int B, int L, int Dch) {
     auto enc = get_encode();
     if (!enc) return false;
@@ -689,26 +790,49 @@ struct ChunkPlan {
 
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 
-ChunkPlan plan(int B, int L, int Dch, int H, int d) {
+constexpr int kPlanSMs = 148;   // segment choice is made for a full B200 (any count runs correctly)
+
+ChunkPlan plan(int B, int L, int Dch, int H) {
     ChunkPlan p{};
     p.nchunks = (L + kC - 1) / kC;
     const long long units = (long long)B * (Dch / kNC);
-    // enough items for ~2 waves of one CTA per SM, segments of at least 4 chunks
-    long long want = (2 * 148 + units - 1) / units;
-    long long maxseg = (p.nchunks + 3) / 4;
-    if (want > maxseg) want = maxseg;
-    if (want < 1) want = 1;
-    p.segc = (int)((p.nchunks + want - 1) / want);
-    p.segc = (p.segc + kNAcc - 1) / kNAcc * kNAcc;   // state-only passes cover whole accumulator rings
-    p.nseg = (p.nchunks + p.segc - 1) / p.segc;
+    // segments: each non-last segment costs a second (state-only) pass over its chunks, and
+    // every item a little fixed work; pick the count that minimises the estimated makespan
+    // (total chunk passes spread over the SMs + the largest item)
+    double best = 1e300;
+    int best_segc = p.nchunks > 0 ? p.nchunks : 1;
+    for (int want = 1; want <= kMaxSeg && want <= (p.nchunks > 0 ? p.nchunks : 1); ++want) {
+        const int segc = (p.nchunks + want - 1) / want;
+        const int nseg = (p.nchunks + segc - 1) / segc;
+        const double items = (double)units * nseg;
+        const double work = (double)units * (p.nchunks + (double)(nseg - 1) * segc) + 1.5 * items;
+        const double ctas = items < kPlanSMs ? items : kPlanSMs;
+        const double est = work / ctas + (nseg > 1 ? 2.0 * segc : segc);
+        if (est < best - 1e-9) { best = est; best_segc = segc; }
+    }
+    p.segc = best_segc;
+    p.nseg = p.nchunks > 0 ? (p.nchunks + p.segc - 1) / p.segc : 1;
     p.items = (int)(units * p.nseg);
     p.consts_off = 0;
     p.sched_off = al256((size_t)H * kConstStride);
     p.status_off = p.sched_off + 256;
     p.agg_off = p.status_off + al256((size_t)p.items * 4);
-    p.inc_off = p.agg_off + al256((size_t)p.items * d * kNC * 8);
-    p.total = p.inc_off + al256((size_t)p.items * d * kNC * 8);
+    p.inc_off = p.agg_off + al256((size_t)p.items * kKS * kNC * 4);
+    p.total = p.inc_off + al256((size_t)p.items * kKS * kNC * 4);
     return p;
+}
+
+int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+            n = v;
+        else
+            return kPlanSMs;
+    }
+    return n;
 }
 
 }  // namespace
@@ -717,12 +841,15 @@ bool chunked_supported(int dtype, int Dch, int H, int d) {
     return dtype == HYENA_BF16 && H > 0 && Dch % H == 0 && (Dch / H) % kNC == 0 && d >= 1 && d <= kMaxModes;
 }
 
-size_t chunked_ws_bytes(int B, int L, int Dch, int H, int d) { return plan(B, L, Dch, H, d).total; }
+size_t chunked_ws_bytes(int B, int L, int Dch, int H, int d) {
+    (void)d;
+    return plan(B, L, Dch, H).total;
+}
 
 cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, int B, int L, int Dch,
                                    int H, int d, const float2 *lam, const float2 *R, const float *Dskip,
                                    void *y, float *state_out, void *ws, cudaStream_t s) {
-    const ChunkPlan p = plan(B, L, Dch, H, d);
+    const ChunkPlan p = plan(B, L, Dch, H);
     uint8_t *w = static_cast<uint8_t *>(ws);
 
     cudaError_t e = cudaMemsetAsync(w + p.sched_off, 0, p.agg_off - p.sched_off, s);
@@ -735,22 +862,25 @@ cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, 
         return cudaErrorInvalidValue;
     ChunkArgs a;
     a.L = L; a.Dch = Dch; a.d = d; a.ch = Dch / H;
-    a.ntiles = Dch / kNC; a.nchunks = p.nchunks; a.nseg = p.nseg; a.segc = p.segc;
-    a.lam = lam;
+    a.ntiles = Dch / kNC; a.nchunks = p.nchunks; a.tok_base = L - p.nchunks * kC;
+    a.nseg = p.nseg; a.segc = p.segc; a.items = p.items;
     a.consts = w + p.consts_off;
+    a.y = static_cast<__nv_bfloat16 *>(y);
     a.state_out = state_out;
     a.sched = reinterpret_cast<int *>(w + p.sched_off);
     a.status = reinterpret_cast<int *>(w + p.status_off);
-    a.agg = reinterpret_cast<float2 *>(w + p.agg_off);
-    a.inc = reinterpret_cast<float2 *>(w + p.inc_off);
+    a.agg = reinterpret_cast<float *>(w + p.agg_off);
+    a.inc = reinterpret_cast<float *>(w + p.inc_off);
     e = cudaFuncSetAttribute(prefill_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    prefill_chunk_kernel<<<p.items, kThreads, kSmemBytes, s>>>(mq, mk, mv, my, a);
+    const int grid = p.items < sm_count() ? p.items : sm_count();
+    prefill_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, my, a);
     return cudaGetLastError();
 }
 
 int chunked_error_offset(int B, int L, int Dch, int H, int d) {
-    return (int)(plan(B, L, Dch, H, d).sched_off + 4);
+    (void)d;
+    return (int)(plan(B, L, Dch, H).sched_off + 4);
 }
 
 }  // namespace hyena

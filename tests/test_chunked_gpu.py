@@ -92,7 +92,9 @@ def test_chunked_matches_fft_route():
     y1, s1, _ = ops.prefill_chunked(q, k, v, lam, R, D)
     y2, s2 = ops.prefill(q, k, v, lam, R, D, 4096)
     assert rel_err(y1.cpu().double().numpy(), y2.cpu().double().numpy()) <= TOL["bf16"]
-    assert rel_err(state_c128(s1), state_c128(s2)) <= 1e-3
+    # the chunked route's tensor-core operands are bf16 (relative rounding 2^-9), so the two routes'
+    # states agree to about 1e-3 of their maximum; the bar is the bf16 tolerance
+    assert rel_err(state_c128(s1), state_c128(s2)) <= TOL["bf16"]
 
 
 def test_chunked_is_deterministic():
