@@ -41,9 +41,12 @@
 // state entering its segment by a decoupled look-back over its predecessors'
 // published contributions (bounded polls), then runs the full pass.  The grid is
 // persistent: each CTA takes items from an atomic ticket in order and its
-// pipelines run on across item boundaries.  An item only ever waits on items
-// with lower tickets, which running CTAs hold, and the state-only pass never
-// waits, so the look-back always ends.  Every wait is bounded; on timeout the
+// pipelines run on across item boundaries.  Tickets are segment-major (all
+// units' first segments, then all second segments, ...), so an item's
+// predecessors were handed out a whole round of units earlier and have usually
+// published by the time it looks back.  An item only ever waits on items with
+// lower tickets, which running CTAs hold, and the state-only pass never waits,
+// so the look-back always ends.  Every wait is bounded; on timeout the
 // kernel records an error code, drains its copies and MMAs, frees tensor memory
 // and returns.
 #include <cuda.h>
@@ -75,6 +78,7 @@ constexpr uint32_t kTmemCols = kSlots * kSlotCols;   // 512
 constexpr int kItemQ = 4;                    // item ids handed from the k,v loader to the other roles
 constexpr int kThreads = 512;
 constexpr int kMaxSeg = 128;                 // segments per sequence (bounds look-back walks)
+constexpr int kPubQ = 4;                     // segment states written and waiting for their status word
 
 // per-head constants: the two A operands (copied verbatim into shared memory) and the powers
 // lambda^C, lambda^Lseg (read from global by the state group)
@@ -111,20 +115,23 @@ enum : int {
     kBarItemEmpty = kBarItemFull + kItemQ,       // [kItemQ] item id read by every consumer (kItemReaders)
     kBarConst = kBarItemEmpty + kItemQ,          // head constants landed (1 + tx)
     kBarConstFree = kBarConst + 1,               // MMAs on the old constants done (commit)
-    kBarPub = kBarConstFree + 1,                 // segment state written to global (128: S group)
-    kBarDrain = kBarPub + 1,                     // every MMA of the CTA finished (commit)
+    kBarPubFull = kBarConstFree + 1,             // [kPubQ] segment state written to global (128: S group)
+    kBarPubEmpty = kBarPubFull + kPubQ,          // [kPubQ] status posted (1: publisher lane)
+    kBarDrain = kBarPubEmpty + kPubQ,            // every MMA of the CTA finished (commit)
     kNumBars = kBarDrain + 1
 };
 // item readers: q loader, store lane, MMA lane (1 each) + lane 0 of the 4 U, 4 S and 4 E warps
 constexpr int kItemReaders = 3 + 12;
 constexpr int kSmMisc = kSmBar + kNumBars * 8;
-constexpr int kSmemBytes = kSmMisc + 64 + 1024;           // + item ids, misc words, alignment slack
+constexpr int kCQ = 4;                                    // items whose carries the MMA thread still owes
+constexpr int kSmemBytes = kSmMisc + 128 + 1024;          // + item ids, misc words, carry queue, slack
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 static_assert(kSmKV % 1024 == 0 && kSmQ % 1024 == 0 && kSmS % 1024 == 0, "swizzle atoms");
 
 __host__ __device__ constexpr int bar_count(int i) {
     return ((i >= kBarURdy && i < kBarQFull) || (i >= kBarYStaged && i < kBarWDone) ||
-            (i >= kBarD2Free && i < kBarYDone) || (i >= kBarD1Free && i < kBarSTFree) || i == kBarPub)
+            (i >= kBarD2Free && i < kBarYDone) || (i >= kBarD1Free && i < kBarSTFree) ||
+            (i >= kBarPubFull && i < kBarPubEmpty))
                ? 128
                : (i >= kBarItemEmpty && i < kBarConst) ? kItemReaders : 1;
 }
@@ -142,16 +149,18 @@ __host__ __device__ __forceinline__ int cm_off16(int row, int k, int K) {
 }
 
 struct ChunkArgs {
-    int L, Dch, d, ch;
-    int ntiles;          // channel tiles per sequence (Dch / 128)
+    int L, Dch, d, ch, H;
+    int tph;             // channel tiles per head (ch / 128)
+    int units_h;         // (sequence, tile) units per head: B * tph
+    int ih;              // items per head: units_h * nseg
     int nchunks;         // chunks per sequence
     int tok_base;        // first token of chunk 0 (L - nchunks * C, <= 0)
     int nseg, segc;      // segments per sequence, chunks per segment (all but the last)
-    int items;
     const uint8_t *consts;
     __nv_bfloat16 *y;    // for the rows of a chunk that starts before token 0
     float *state_out;    // [B][d][Dch][2]
-    int *sched;          // [0] ticket counter, [1] error code
+    int *sched;          // [1] error code
+    int *tickets;        // [H] ticket counter per head
     int *status;         // [items]: 0 none, 1 segment contribution, 2 inclusive state
     float *agg;          // [items][32 rows][128 ch]
     float *inc;          // [items][32 rows][128 ch]
@@ -165,11 +174,12 @@ struct Item {
 __device__ __forceinline__ Item decode_item(const ChunkArgs &a, int id) {
     Item it;
     it.id = id;
-    const int unit = id / a.nseg;
-    it.seg = id % a.nseg;
-    it.b = unit / a.ntiles;
-    it.c0 = (unit % a.ntiles) * kNC;
-    it.hd = it.c0 / a.ch;
+    it.hd = id / a.ih;
+    const int t = id % a.ih;                // ticket within the head, segment-major: the
+    const int unit = t % a.units_h;         // predecessor of item id is id - units_h
+    it.seg = t / a.units_h;
+    it.b = unit / a.tph;
+    it.c0 = it.hd * a.ch + (unit % a.tph) * kNC;
     it.ck0 = it.seg * a.segc;
     it.nck = min(a.nchunks, it.ck0 + a.segc) - it.ck0;
     it.last_seg = (it.seg == a.nseg - 1);
@@ -185,12 +195,35 @@ __device__ __forceinline__ void record_error(const ChunkArgs &a, volatile int *a
     atomicCAS(a.sched + 1, 0, code);
 }
 
+// Load with acquire semantics at GPU scope (pairs with the publisher's fence + status write).
+__device__ __forceinline__ int ld_acquire(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // One step x <- lam x + a of a complex recurrence held as (Re, Im) in the lanes r and r ^ 16 of a
 // warp (sgn = -1 in the Re lanes, +1 in the Im lanes).  Used for every segment-state combination,
 // so that the same inputs always give the same bits.
 __device__ __forceinline__ float seg_step(float x, float a, float2 lam, float sgn) {
     const float xp = __shfl_xor_sync(0xffffffffu, x, 16);
     return fmaf(lam.x, x, fmaf(sgn * lam.y, xp, a));
+}
+
+// In-register transpose of a 32 x 32 block held one row per lane (v[j] = M[lane][j]) into one
+// column per lane (v[j] = M[j][lane]): five butterfly stages of warp shuffles.
+__device__ __forceinline__ void warp_transpose32(float *v, int lane) {
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) {
+        const bool upper = (lane & m) != 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if (i & m) continue;
+            const float send = upper ? v[i] : v[i | m];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, m);
+            if (upper) v[i] = recv; else v[i | m] = recv;
+        }
+    }
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -201,6 +234,21 @@ __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x <<
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
 // ------------------------------------------------------------------ per-head constants
+// One block per head.  Every entry is a power lambda_n^k with 0 <= k <= C, so the powers are
+// tabulated first (each by binary powering, all in parallel) and the operands are then filled
+// from the table.  fp32 suffices: the operands are rounded to bf16 (relative 2^-9) and the
+// chain powers lambda^C, lambda^Lseg enter an fp32 recurrence, while binary powering to an
+// exponent below 2^31 loses at most a few tens of fp32 ulps.
+__device__ __forceinline__ float2 cfpow(float2 lam, long long m) {
+    float2 r = make_float2(1.f, 0.f), b = lam;
+    while (m > 0) {
+        if (m & 1) r = cmul(r, b);
+        b = cmul(b, b);
+        m >>= 1;
+    }
+    return r;
+}
+
 __global__ void __launch_bounds__(256)
 chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R,
                     const float *__restrict__ Dskip, int d, int seg_tokens,
@@ -211,59 +259,73 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
     __nv_bfloat16 *CA = reinterpret_cast<__nv_bfloat16 *>(base + kFABytes);
     float2 *lamC = reinterpret_cast<float2 *>(base + kLamOff);
     float2 *lamS = lamC + kMaxModes;
-    __shared__ double hs[kC];
-    const float2 *lh = lam + (size_t)hd * d;
-    const float2 *rh = R + (size_t)hd * d;
-    // filter taps h_0 .. h_{C-1} in fp64
+    __shared__ float2 pw[kMaxModes][kC + 1];     // lambda_n^k, zero for modes >= d
+    __shared__ float2 ls[kMaxModes], rs[kMaxModes];   // lambda_n, R_n
+    __shared__ float hs[kC];                     // filter taps h_0 .. h_{C-1}
+    __shared__ float dskip;
+    // the parameters once into shared memory (one round trip; the table loops below would
+    // otherwise wait on a global load per entry)
+    {
+        const int t = threadIdx.x;
+        if (t < kMaxModes) ls[t] = t < d ? lam[(size_t)hd * d + t] : make_float2(0.f, 0.f);
+        else if (t < 2 * kMaxModes) rs[t - kMaxModes] = t - kMaxModes < d ? R[(size_t)hd * d + t - kMaxModes] : make_float2(0.f, 0.f);
+        else if (t == 2 * kMaxModes) dskip = Dskip[hd];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < kMaxModes * (kC + 1); e += blockDim.x) {
+        const int n = e / (kC + 1), k = e % (kC + 1);
+        pw[n][k] = n < d ? cfpow(ls[n], k) : make_float2(0.f, 0.f);
+    }
+    for (int n = threadIdx.x; n < kMaxModes; n += blockDim.x)
+        lamS[n] = n < d ? cfpow(ls[n], seg_tokens) : make_float2(0.f, 0.f);
+    __syncthreads();
     for (int j = threadIdx.x; j < kC; j += blockDim.x) {
-        double acc = 0.0;
+        float acc = 0.f;
         if (j == 0) {
-            acc = Dskip[hd];
+            acc = dskip;
         } else {
-            for (int n = 0; n < d; ++n) {
-                const cd p = cdpow(cd{lh[n].x, lh[n].y}, j - 1);
-                acc += (double)rh[n].x * p.x - (double)rh[n].y * p.y;
-            }
+            for (int n = 0; n < d; ++n) acc += rs[n].x * pw[n][j - 1].x - rs[n].y * pw[n][j - 1].y;
         }
         hs[j] = acc;
     }
+    for (int n = threadIdx.x; n < kMaxModes; n += blockDim.x) lamC[n] = pw[n][kC];
     __syncthreads();
     // fused A operand: rows 0..C-1 Toeplitz taps, rows C..C+31 chunk powers (Re at r < 16, Im at
     // 16 + n), rows C+32..127 zero
-    for (int e = threadIdx.x; e < 128 * kC; e += blockDim.x) {
-        const int row = e / kC, io = e % kC;
-        double v = 0.0;
-        if (row < kC) {
-            v = io <= row ? hs[row - io] : 0.0;
-        } else if (row < kC + kKS) {
-            const int r = row - kC, n = r & (kIm - 1);
-            if (n < d) {
-                const cd p = cdpow(cd{lh[n].x, lh[n].y}, kC - 1 - io);
-                v = r < kIm ? p.x : p.y;
+    // (each thread writes one 16-byte core-matrix row: 8 consecutive K entries of one row)
+    for (int e = threadIdx.x; e < 128 * (kC / 8); e += blockDim.x) {
+        const int row = e / (kC / 8), io0 = 8 * (e % (kC / 8));
+        float v[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+            const int io = io0 + x;
+            v[x] = 0.f;
+            if (row < kC) {
+                v[x] = io <= row ? hs[row - io] : 0.f;
+            } else if (row < kC + kKS) {
+                const int r = row - kC;
+                const float2 p = pw[r & (kIm - 1)][kC - 1 - io];
+                v[x] = r < kIm ? p.x : p.y;
             }
         }
-        FA[cm_off16(row, io, kC) / 2] = __float2bfloat16_rn((float)v);
+        *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(FA) + cm_off16(row, io0, kC)) =
+            make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
     }
     // carry A operand: rows 0..C-1: (Re, -Im) of R_n lambda_n^tau; rows C..127 zero
-    for (int e = threadIdx.x; e < 128 * kKS; e += blockDim.x) {
-        const int row = e / kKS, r = e % kKS, n = r & (kIm - 1);
-        double v = 0.0;
-        if (row < kC && n < d) {
-            const cd p = cdpow(cd{lh[n].x, lh[n].y}, row);
-            const double re = (double)rh[n].x * p.x - (double)rh[n].y * p.y;
-            const double im = (double)rh[n].x * p.y + (double)rh[n].y * p.x;
-            v = r < kIm ? re : -im;
+    for (int e = threadIdx.x; e < 128 * (kKS / 8); e += blockDim.x) {
+        const int row = e / (kKS / 8), r0 = 8 * (e % (kKS / 8));
+        float v[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+            const int r = r0 + x, n = r & (kIm - 1);
+            v[x] = 0.f;
+            if (row < kC) {
+                const float2 c = cmul(rs[n], pw[n][row]);
+                v[x] = r < kIm ? c.x : -c.y;
+            }
         }
-        CA[cm_off16(row, r, kKS) / 2] = __float2bfloat16_rn((float)v);
-    }
-    for (int n = threadIdx.x; n < kMaxModes; n += blockDim.x) {
-        cd pc{0.0, 0.0}, ps{0.0, 0.0};
-        if (n < d) {
-            pc = cdpow(cd{lh[n].x, lh[n].y}, kC);
-            ps = cdpow(cd{lh[n].x, lh[n].y}, seg_tokens);
-        }
-        lamC[n] = make_float2((float)pc.x, (float)pc.y);
-        lamS[n] = make_float2((float)ps.x, (float)ps.y);
+        *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(CA) + cm_off16(row, r0, kKS)) =
+            make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
     }
 }
 
@@ -287,6 +349,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     auto bar = [&](int slot) { return sbase + kSmBar + 8u * slot; };
     volatile int *itemq = reinterpret_cast<volatile int *>(sm + kSmMisc);   // [kItemQ]
     volatile int *misc = itemq + kItemQ;                                     // abort, tmem, never
+    int *cqueue = const_cast<int *>(misc) + 4;                               // [kCQ][3]: n1, nck, g0
+    volatile int *pubq = misc + 4 + 3 * kCQ;                                 // [kPubQ]: 4 item + code, -1 = end
     volatile int *abort = misc;
     volatile int *never = misc + 2;
 
@@ -325,7 +389,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (warp == kWarpKV) {
         // ------------------------------------------------------------ k,v loads + tickets
         if (lane == 0) {
-            int g = 0;
+            int g = 0, head = blockIdx.x % a.H, tries = 0;
             bool ok = true;
             for (int k = 0; ok; ++k) {
                 const int s = k % kItemQ;
@@ -333,8 +397,14 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     ok = false;
                     break;
                 }
-                int id = atomicAdd(a.sched, 1);
-                if (id >= a.items) id = -1;
+                // tickets of this CTA's head first; when they run out, move on to the next head
+                int id = -1;
+                while (tries < a.H) {
+                    const int t = atomicAdd(a.tickets + head, 1);
+                    if (t < a.ih) { id = head * a.ih + t; tries = 0; break; }
+                    head = head + 1 == a.H ? 0 : head + 1;
+                    ++tries;
+                }
                 itemq[s] = id;
                 tc::mbar_arrive(bar(kBarItemFull + s));
                 if (id < 0) break;
@@ -418,93 +488,138 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             }
             if (!ok) record_error(a, abort, kErrWait);
             tc::bulk_wait<0>();     // every store of this CTA has completed
+        } else if (lane == 1) {
+            // publisher: after the S group has written a segment state (seen through the barrier),
+            // one GPU-scope fence orders all of its rows before the status word that other CTAs poll
+            for (int k = 0;; ++k) {
+                const int ps = k % kPubQ;
+                if (!tc::mbar_wait(bar(kBarPubFull + ps), (k / kPubQ) & 1, abort)) {
+                    if (!*abort) record_error(a, abort, kErrWait);
+                    break;
+                }
+                const int v = pubq[ps];
+                if (v < 0) break;
+                __threadfence();
+                atomicExch(a.status + (v >> 2), v & 3);
+                tc::mbar_arrive(bar(kBarPubEmpty + ps));
+            }
         }
     } else if (warp == kWarpMMA) {
         // ------------------------------------------------------------ MMA issuer
-        // Two streams issued out of order from one thread (polled with non-blocking tests): the
+        // Two streams issued out of order from one thread, polled with non-blocking tests: the
         // fused product of a chunk needs only its U operand and a free accumulator slot and runs
         // ahead; the carry needs the state entering the chunk and follows when the S group
-        // delivers it.  MMAs from one thread execute in issue order.
+        // delivers it.  Both streams run on across item boundaries (a small queue holds the
+        // items whose carries are still to come).  MMAs from one thread execute in issue order.
         if (lane == 0) {
             const uint32_t idesc = tc::idesc_bf16(128, kNC, true);
-            int g = 0, pc = 0, cur_hd = -1, cphase = 0, fphase = 0;
-            int c2[kSlots] = {0, 0};    // full-pass uses of each slot issued so far
-            bool any = false, ok = true;
-            for (int k = 0; ok; ++k) {
-                const int id = take_item(k, false);
-                if (id == -2) ok = false;
-                if (id < 0) break;
-                const Item it = decode_item(a, id);
-                if (it.hd != cur_hd) {
-                    // new head: wait until no MMA reads the old constants, then copy the new ones
+            // (indexed arrays would live in local memory, which the small L1 left beside this
+            // much shared memory turns into L2 round trips: the carry queue is in shared memory
+            // and the per-slot counters are scalars)
+            Item fi{};                      // item of the fused stream
+            int chead = 0, ctail = 0;       // carry queue: (n1, nck, first global fused index)
+            int fk = 0, ic = 0, g = 0, jn = 0, pc = 0;
+            int cur_hd = -1, cphase = 0, fphase = 0;
+            int c2a = 0, c2b = 0;           // full-pass uses of slot 0 / slot 1 issued so far
+            bool f_valid = false, need_const = false, done = false, any = false, ok = true;
+            unsigned long long t_prog = tc::global_ns();
+            while (ok && !*abort) {
+                bool progressed = false;
+                // the next item for the fused stream
+                if (!f_valid && !done && ctail - chead < kCQ) {
+                    const int s = fk % kItemQ;
+                    if (tc::mbar_test(bar(kBarItemFull + s), (fk / kItemQ) & 1)) {
+                        const int id = itemq[s];
+                        tc::mbar_arrive(bar(kBarItemEmpty + s));
+                        ++fk;
+                        progressed = true;
+                        if (id < 0) {
+                            done = true;
+                        } else {
+                            fi = decode_item(a, id);
+                            f_valid = true;
+                            ic = 0;
+                            need_const = fi.hd != cur_hd;
+                            int *e = cqueue + 3 * (ctail % kCQ);
+                            e[0] = fi.n1;
+                            e[1] = fi.nck;
+                            e[2] = g;
+                            ++ctail;
+                        }
+                    }
+                }
+                // carry stream: Z += A S (own TMEM columns of the chunk's slot)
+                if (chead < ctail) {
+                    const int *e = cqueue + 3 * (chead % kCQ);
+                    const int c_nck = e[1];
+                    const int cgi = e[2] + e[0] + jn;
+                    const int sb = pc % kSBufs;
+                    if (cgi < g && tc::mbar_test(bar(kBarSRdy + sb), (pc / kSBufs) & 1)) {
+                        tc::tc_fence_after();
+                        const int slot = cgi % kSlots;
+                        const uint32_t dcol = tmem + slot * kSlotCols + kNC;
+                        const uint32_t sb_addr = sbase + kSmS + sb * kSBytes;
+                        for (int ks = 0; ks < kKS / 16; ++ks)
+                            tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmCA + ks * 256, 128, kKS * 16),
+                                         tc::smem_desc_sw128(sb_addr + ks * 2048, kSBytes / 2, 1024), idesc, ks > 0);
+                        tc::mma_commit(bar(kBarYDone + slot));
+                        tc::mma_commit(bar(kBarSTFree + sb));
+                        ++pc;
+                        if (++jn == c_nck) { jn = 0; ++chead; }
+                        progressed = true;
+                    }
+                }
+                // constants of a new head, once no issued or pending MMA uses the old ones (rare:
+                // a CTA keeps to one head until its items run out)
+                if (need_const && chead == ctail - 1) {
                     if (any) {
                         tc::mma_commit(bar(kBarConstFree));
                         if (!tc::mbar_wait(bar(kBarConstFree), fphase & 1, abort)) { ok = false; break; }
                         ++fphase;
                     }
                     tc::mbar_expect_tx(bar(kBarConst), kOpBytes);
-                    tc::bulk_load(sbase + kSmFA, a.consts + (size_t)it.hd * kConstStride, kOpBytes, bar(kBarConst));
+                    tc::bulk_load(sbase + kSmFA, a.consts + (size_t)fi.hd * kConstStride, kOpBytes, bar(kBarConst));
                     if (!tc::mbar_wait(bar(kBarConst), cphase & 1, never)) { ok = false; break; }
                     ++cphase;
-                    cur_hd = it.hd;
+                    cur_hd = fi.hd;
+                    need_const = false;
+                    progressed = true;
                 }
-                const int g0 = g;
-                int ic = 0, jn = 0;
-                unsigned long long t_prog = tc::global_ns();
-                while ((ic < it.niter || jn < it.nck) && !*abort) {
-                    bool progressed = false;
-                    if (jn < it.nck && it.n1 + jn < ic) {
-                        const int sb = pc % kSBufs;
-                        if (tc::mbar_test(bar(kBarSRdy + sb), (pc / kSBufs) & 1)) {
-                            tc::tc_fence_after();
-                            // carry: Z += A S  (own TMEM columns of the chunk's slot)
-                            const int slot = (g0 + it.n1 + jn) % kSlots;
-                            const uint32_t dcol = tmem + slot * kSlotCols + kNC;
-                            const uint32_t sb_addr = sbase + kSmS + sb * kSBytes;
-                            for (int ks = 0; ks < kKS / 16; ++ks)
-                                tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmCA + ks * 256, 128, kKS * 16),
-                                             tc::smem_desc_sw128(sb_addr + ks * 2048, kSBytes / 2, 1024), idesc, ks > 0);
-                            tc::mma_commit(bar(kBarYDone + slot));
-                            tc::mma_commit(bar(kBarSTFree + sb));
-                            ++jn;
-                            ++pc;
-                            progressed = true;
+                // fused stream: [Z; W] = [T; V] U
+                if (f_valid && !need_const) {
+                    const int slot = g % kSlots, st = g % kKVStages;
+                    if (tc::mbar_test(bar(kBarURdy + st), (g / kKVStages) & 1) &&
+                        tc::mbar_test(bar(kBarD2Free + slot), ((g / kSlots) & 1) ^ 1) &&
+                        tc::mbar_test(bar(kBarD1Free + slot), ((slot ? c2b : c2a) & 1) ^ 1)) {
+                        tc::tc_fence_after();
+                        const uint32_t dcol = tmem + slot * kSlotCols;
+                        const uint32_t u_addr = sbase + kSmKV + st * kStageBytes;
+                        for (int ks = 0; ks < kC / 16; ++ks)
+                            tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmFA + ks * 256, 128, kC * 16),
+                                         tc::smem_desc_sw128(u_addr + ks * 2048, kHalf, 1024), idesc, ks > 0);
+                        tc::mma_commit(bar(kBarWDone + slot));
+                        tc::mma_commit(bar(kBarKVEmpty + st));
+                        if (ic >= fi.n1) {
+                            if (slot) ++c2b; else ++c2a;
                         }
-                    }
-                    if (ic < it.niter) {
-                        const int gi = g0 + ic, slot = gi % kSlots, st = gi % kKVStages;
-                        bool ready = tc::mbar_test(bar(kBarURdy + st), (gi / kKVStages) & 1) &&
-                                     tc::mbar_test(bar(kBarD2Free + slot), ((gi / kSlots) & 1) ^ 1) &&
-                                     tc::mbar_test(bar(kBarD1Free + slot), (c2[slot] & 1) ^ 1);
-                        if (ready) {
-                            tc::tc_fence_after();
-                            // fused: [Z; W] = [T; V] U
-                            const uint32_t dcol = tmem + slot * kSlotCols;
-                            const uint32_t u_addr = sbase + kSmKV + st * kStageBytes;
-                            for (int ks = 0; ks < kC / 16; ++ks)
-                                tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmFA + ks * 256, 128, kC * 16),
-                                             tc::smem_desc_sw128(u_addr + ks * 2048, kHalf, 1024), idesc, ks > 0);
-                            tc::mma_commit(bar(kBarWDone + slot));
-                            tc::mma_commit(bar(kBarKVEmpty + st));
-                            if (ic >= it.n1) ++c2[slot];
-                            ++ic;
-                            any = true;
-                            progressed = true;
-                        }
-                    }
-                    if (progressed) {
-                        t_prog = tc::global_ns();
-                    } else {
-                        if (tc::global_ns() - t_prog > tc::kWaitNs) {
-                            ok = false;
-                            break;
-                        }
-                        __nanosleep(20);
+                        ++g;
+                        any = true;
+                        progressed = true;
+                        if (++ic == fi.niter) f_valid = false;
                     }
                 }
-                if (*abort) ok = false;
-                g = g0 + it.niter;
+                if (done && !f_valid && chead == ctail) break;
+                if (progressed) {
+                    t_prog = tc::global_ns();
+                } else {
+                    if (tc::global_ns() - t_prog > tc::kWaitNs) {
+                        ok = false;
+                        break;
+                    }
+                    __nanosleep(20);
+                }
             }
+            if (*abort) ok = false;
             if (!ok) record_error(a, abort, kErrWait);
             // all MMAs issued by this thread have completed once `drain` fires
             tc::mma_commit(bar(kBarDrain));
@@ -549,16 +664,33 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const bool leader = (warp == 2 && lane == 0);
         const float sgn = (r < kIm) ? -1.f : 1.f;
         const uint32_t lane_base = (uint32_t)64 << 16;
-        int g = 0, pc = 0, pub_phase = 0;
+        int g = 0, pc = 0, pub_k = 0, cur_hd = -1;
         bool ok = true;
         float st[32];
+        float2 lamC = make_float2(0.f, 0.f), lamS = lamC;
+        // hand one entry to the publisher lane (all 128 threads call this after their writes)
+        auto post = [&](int v) -> bool {
+            const int ps = pub_k % kPubQ;
+            bool res = true;
+            if (leader) {
+                res = tc::mbar_wait(bar(kBarPubEmpty + ps), ((pub_k / kPubQ) & 1) ^ 1, abort);
+                pubq[ps] = res ? v : -1;
+            }
+            tc::mbar_arrive(bar(kBarPubFull + ps));
+            ++pub_k;
+            return res;
+        };
         for (int k = 0; ok; ++k) {
             const int id = take_item(k, true);
             if (id == -2) ok = false;
             if (id < 0) break;
             const Item it = decode_item(a, id);
-            const float2 *lp = reinterpret_cast<const float2 *>(a.consts + (size_t)it.hd * kConstStride + kLamOff);
-            const float2 lamC = lp[n], lamS = lp[kMaxModes + n];    // zero for modes >= d
+            if (it.hd != cur_hd) {
+                const float2 *lp = reinterpret_cast<const float2 *>(a.consts + (size_t)it.hd * kConstStride + kLamOff);
+                lamC = lp[n];               // zero for modes >= d
+                lamS = lp[kMaxModes + n];
+                cur_hd = it.hd;
+            }
 #pragma unroll
             for (int i = 0; i < 32; ++i) st[i] = 0.f;
 
@@ -588,30 +720,20 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     o[4 * i] = v4.x; o[4 * i + 1] = v4.y; o[4 * i + 2] = v4.z; o[4 * i + 3] = v4.w;
                 }
             };
-            // write the state rows of this thread to dst [32 rows][128 ch], then post `code`
-            auto publish = [&](float *dst, int code) -> bool {
+            // write the state rows of this thread to dst [32 rows][128 ch] and hand `code` to the
+            // publisher lane, which posts it once every row is written (no wait here)
+            auto publish = [&](const float *v, float *dst, int code) -> bool {
                 float4 *o = reinterpret_cast<float4 *>(dst + (size_t)r * kNC + 32 * q4);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) o[i] = make_float4(st[4 * i], st[4 * i + 1], st[4 * i + 2], st[4 * i + 3]);
-                __threadfence();
-                tc::mbar_arrive(bar(kBarPub));
-                bool res = true;
-                if (leader) {
-                    res = tc::mbar_wait(bar(kBarPub), pub_phase & 1, abort);
-                    if (res) {
-                        __threadfence();
-                        atomicExch(a.status + it.id, code);
-                    }
-                }
-                ++pub_phase;
-                return res;
+                for (int i = 0; i < 8; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                return post(it.id * 4 + code);
             };
 
             // state-only pass over the segment, then publish its contribution
             for (int i = 0; i < it.n1 && ok; ++i, ++g) ok = uni(advance(g));
             if (!ok) break;
             const size_t item_off = (size_t)it.id * kKS * kNC;
-            if (it.n1 > 0 && !(ok = uni(publish((it.seg == 0 ? a.inc : a.agg) + item_off, it.seg == 0 ? 2 : 1))))
+            if (it.n1 > 0 && !(ok = uni(publish(st, (it.seg == 0 ? a.inc : a.agg) + item_off, it.seg == 0 ? 2 : 1))))
                 break;
             float sloc[32];
 #pragma unroll
@@ -624,14 +746,15 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             // was found, so the output does not depend on timing.
             if (it.seg > 0) {
                 int p0 = -1;
-                for (int p = it.id - 1; p >= it.id - it.seg; --p) {
+                const int units = a.units_h;
+                for (int p = it.id - units; p >= it.id - it.seg * units; p -= units) {
                     int code = 0;
                     if (lane == 0) {
-                        code = *(volatile int *)(a.status + p);
+                        code = ld_acquire(a.status + p);
                         const unsigned long long t0 = tc::global_ns();
                         while (code == 0 && !*abort && tc::global_ns() - t0 < tc::kWaitNs) {
                             __nanosleep(64);
-                            code = *(volatile int *)(a.status + p);
+                            code = ld_acquire(a.status + p);
                         }
                     }
                     code = __shfl_sync(0xffffffffu, code, 0);
@@ -643,26 +766,19 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     ok = false;
                 }
                 if (!(ok = uni(ok))) break;
-                __threadfence();
+                __syncwarp();       // lane 0's acquire loads order the other lanes' reads below
                 load_rows(a.inc + (size_t)p0 * kKS * kNC, st);
-                for (int p = p0 + 1; p < it.id; ++p) {
+                for (int p = p0 + units; p < it.id; p += units) {
                     float ag[32];
                     load_rows(a.agg + (size_t)p * kKS * kNC, ag);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) st[i] = seg_step(st[i], ag[i], lamS, sgn);
                 }
                 if (it.n1 > 0) {
-                    // inclusive state at the end of this segment
-                    float keep[32];
+                    // inclusive state at the end of this segment (sloc is not needed after this)
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        keep[i] = st[i];
-                        st[i] = seg_step(st[i], sloc[i], lamS, sgn);
-                    }
-                    ok = uni(publish(a.inc + item_off, 2));
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) st[i] = keep[i];
-                    if (!ok) break;
+                    for (int i = 0; i < 32; ++i) sloc[i] = seg_step(st[i], sloc[i], lamS, sgn);
+                    if (!(ok = uni(publish(sloc, a.inc + item_off, 2)))) break;
                 }
             }
 
@@ -687,20 +803,25 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 if (!(ok = uni(advance(g)))) break;
             }
             if (!ok) break;
-            if (it.last_seg && n < d) {
-                float *so = a.state_out + (((size_t)it.b * d + n) * a.Dch + it.c0 + 32 * q4) * 2 + (r >> 4);
+            if (it.last_seg) {
+                // transpose the warp's 32 x 32 block (rows r in lanes -> channels in lanes) so that
+                // each lane writes the (Re, Im) pairs of one channel: coalesced float2 stores
+                warp_transpose32(st, lane);
+                float2 *so = reinterpret_cast<float2 *>(a.state_out) + ((size_t)it.b * d) * a.Dch + it.c0 + 32 * q4 + lane;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) so[2 * i] = st[i];
+                for (int m = 0; m < kMaxModes; ++m)
+                    if (m < d) so[(size_t)m * a.Dch] = make_float2(st[m], st[kIm + m]);
             }
         }
         if (!ok) record_error(a, abort, kErrWait);
+        post(-1);       // end of this CTA's posts
     } else if (is_e_warp(warp)) {
         // ------------------------------------------------------------ E group (gate and stage y)
         // thread: token row tau = 32 q4 + lane (TMEM lane tau) for channels 64 hh .. 64 hh + 63
         const int q4 = warp & 3, hh = warp >> 3, tau = 32 * q4 + lane;
         const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
         int g = 0, qg = 0;
-        int e2[kSlots] = {0, 0};
+        int e2a = 0, e2b = 0;       // full-pass uses of slot 0 / slot 1 consumed so far
         bool ok = true;
         for (int k = 0; ok; ++k) {
             const int id = take_item(k, true);
@@ -710,10 +831,10 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             g += it.n1;
             for (int j = 0; j < it.nck; ++j, ++g, ++qg) {
                 const int slot = g % kSlots, s = qg % kQStages;
-                ok = uni(tc::mbar_wait(bar(kBarYDone + slot), e2[slot] & 1, abort) &&
+                ok = uni(tc::mbar_wait(bar(kBarYDone + slot), (slot ? e2b : e2a) & 1, abort) &&
                          tc::mbar_wait(bar(kBarQFull + s), (qg / kQStages) & 1, abort));
                 if (!ok) break;
-                ++e2[slot];
+                if (slot) ++e2b; else ++e2a;
                 tc::tc_fence_after();
                 const int tok = tok_of(it.ck0 + j);
                 uint8_t *qrow = sm + kSmQ + s * kTile + hh * kHalf + tau * 128;
@@ -783,6 +904,8 @@ bool make_map(CUtensorMap *m, const void *base, int B, int L, int Dch) {
                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+constexpr size_t kTicketOff = 64;    // byte offset of the per-head ticket counters in the schedule block
+
 struct ChunkPlan {
     int nchunks, nseg, segc, items;
     size_t consts_off, sched_off, status_off, agg_off, inc_off, total;
@@ -815,7 +938,7 @@ ChunkPlan plan(int B, int L, int Dch, int H) {
     p.items = (int)(units * p.nseg);
     p.consts_off = 0;
     p.sched_off = al256((size_t)H * kConstStride);
-    p.status_off = p.sched_off + 256;
+    p.status_off = p.sched_off + al256(kTicketOff + (size_t)H * 4);
     p.agg_off = p.status_off + al256((size_t)p.items * 4);
     p.inc_off = p.agg_off + al256((size_t)p.items * kKS * kNC * 4);
     p.total = p.inc_off + al256((size_t)p.items * kKS * kNC * 4);
@@ -861,13 +984,15 @@ cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, 
         !make_map(&my, y, B, L, Dch))
         return cudaErrorInvalidValue;
     ChunkArgs a;
-    a.L = L; a.Dch = Dch; a.d = d; a.ch = Dch / H;
-    a.ntiles = Dch / kNC; a.nchunks = p.nchunks; a.tok_base = L - p.nchunks * kC;
-    a.nseg = p.nseg; a.segc = p.segc; a.items = p.items;
+    a.L = L; a.Dch = Dch; a.d = d; a.ch = Dch / H; a.H = H;
+    a.tph = a.ch / kNC; a.units_h = B * a.tph; a.ih = a.units_h * p.nseg;
+    a.nchunks = p.nchunks; a.tok_base = L - p.nchunks * kC;
+    a.nseg = p.nseg; a.segc = p.segc;
     a.consts = w + p.consts_off;
     a.y = static_cast<__nv_bfloat16 *>(y);
     a.state_out = state_out;
     a.sched = reinterpret_cast<int *>(w + p.sched_off);
+    a.tickets = reinterpret_cast<int *>(w + p.sched_off + kTicketOff);
     a.status = reinterpret_cast<int *>(w + p.status_off);
     a.agg = reinterpret_cast<float *>(w + p.agg_off);
     a.inc = reinterpret_cast<float *>(w + p.inc_off);
