@@ -35,7 +35,7 @@ cudaError_t launch_prefill_fft(const void *q, const void *k, const void *v, int 
                                void *y, float *state_out, void *scratch, size_t scratch_bytes,
                                cudaStream_t s);
 
-// prefill_chunked.cu (bf16 activations, heads of a multiple of 128 channels, d <= 16)
+// prefill_chunked.cu (bf16 activations, heads of a multiple of 64 channels, d <= 16)
 bool chunked_supported(int dtype, int Dch, int H, int d);
 size_t chunked_ws_bytes(int B, int L, int Dch, int H, int d);
 int chunked_error_offset(int B, int L, int Dch, int H, int d);

@@ -62,23 +62,19 @@ namespace hyena {
 namespace {
 
 constexpr int kC = 64;              // tokens per chunk (K of the fused product)
-constexpr int kNC = 128;            // channels per tile (MMA N)
 constexpr int kMaxModes = 16;       // d <= 16
 constexpr int kKS = 32;             // state rows: Re of modes 0..15, then Im
 constexpr int kIm = 16;
-constexpr int kTile = kC * kNC * 2;          // one bf16 [C][128] activation tile (16 KB)
-constexpr int kHalf = kTile / 2;             // [C][64] half = one TMA box, 128-byte swizzled
-constexpr int kStageBytes = 2 * kTile;       // k (overwritten by U) then v
-constexpr int kKVStages = 4;
-constexpr int kQStages = 3;                  // q tiles; y is staged in place
-constexpr int kSBufs = 2;                    // state operands
-constexpr int kSlots = 2;                    // accumulator slots: fused [128 cols] | carry [128 cols]
-constexpr int kSlotCols = 2 * kNC;
-constexpr uint32_t kTmemCols = kSlots * kSlotCols;   // 512
-constexpr int kItemQ = 4;                    // item ids handed from the k,v loader to the other roles
+constexpr int kAtom = kC * 64 * 2;  // one bf16 [C][64] TMA box, 128-byte swizzled (8 KB)
+constexpr int kSBufs = 2;           // state operands
+constexpr int kItemQ = 4;           // item ids handed from the k,v loader to the other roles
 constexpr int kThreads = 512;
-constexpr int kMaxSeg = 128;                 // segments per sequence (bounds look-back walks)
-constexpr int kPubQ = 4;                     // segment states written and waiting for their status word
+constexpr int kMaxSeg = 128;        // segments per sequence (bounds look-back walks)
+constexpr int kPubQ = 4;            // segment states written and waiting for their status word
+constexpr int kCQ = 4;              // items whose carries the MMA thread still owes
+constexpr uint32_t kTmemCols = 512; // all of tensor memory (one CTA per SM)
+// item readers: q loader, store lane, MMA lane (1 each) + lane 0 of the 4 U, 4 S and 4 E warps
+constexpr int kItemReaders = 3 + 12;
 
 // per-head constants: the two A operands (copied verbatim into shared memory) and the powers
 // lambda^C, lambda^Lseg (read from global by the state group)
@@ -88,53 +84,61 @@ constexpr int kOpBytes = kFABytes + kCABytes;
 constexpr int kLamOff = kOpBytes;            // float2 lambda^C [16], lambda^Lseg [16]
 constexpr int kConstStride = kOpBytes + 256;
 
-// shared memory map (offsets from a 1024-byte aligned base)
+// shared memory map (offsets from a 1024-byte aligned base): constants, then the rings
 constexpr int kSmFA = 0;
 constexpr int kSmCA = kSmFA + kFABytes;
 constexpr int kSmKV = kSmCA + kCABytes;                   // 1024-aligned (swizzle atoms)
-constexpr int kSmQ = kSmKV + kKVStages * kStageBytes;
-constexpr int kSBytes = kKS * kNC * 2;                    // [32 rows][128 ch] bf16, 128-byte swizzled
-constexpr int kSmS = kSmQ + kQStages * kTile;
-constexpr int kSmBar = kSmS + kSBufs * kSBytes;
 
-// barrier slots (arrival counts in parentheses; "commit" = tcgen05.commit from the MMA thread)
-enum : int {
-    kBarKVFull = 0,                              // [kKVStages] k,v landed (1 + tx)
-    kBarKVEmpty = kBarKVFull + kKVStages,        // [kKVStages] fused product read U (commit)
-    kBarURdy = kBarKVEmpty + kKVStages,          // [kKVStages] U formed over k (128: U group)
-    kBarQFull = kBarURdy + kKVStages,            // [kQStages] q landed (1 + tx)
-    kBarQEmpty = kBarQFull + kQStages,           // [kQStages] y stored, buffer free (1: store lane)
-    kBarYStaged = kBarQEmpty + kQStages,         // [kQStages] gated y staged (128: E group)
-    kBarWDone = kBarYStaged + kQStages,          // [kSlots] fused product done (commit)
-    kBarD2Free = kBarWDone + kSlots,             // [kSlots] state rows read out (128: S group)
-    kBarYDone = kBarD2Free + kSlots,             // [kSlots] carry done: output complete (commit)
-    kBarD1Free = kBarYDone + kSlots,             // [kSlots] output rows read out (128: E group)
-    kBarSRdy = kBarD1Free + kSlots,              // [kSBufs] state operand written (128: S group)
-    kBarSTFree = kBarSRdy + kSBufs,              // [kSBufs] state operand read (commit)
-    kBarItemFull = kBarSTFree + kSBufs,          // [kItemQ] item id posted (1)
-    kBarItemEmpty = kBarItemFull + kItemQ,       // [kItemQ] item id read by every consumer (kItemReaders)
-    kBarConst = kBarItemEmpty + kItemQ,          // head constants landed (1 + tx)
-    kBarConstFree = kBarConst + 1,               // MMAs on the old constants done (commit)
-    kBarPubFull = kBarConstFree + 1,             // [kPubQ] segment state written to global (128: S group)
-    kBarPubEmpty = kBarPubFull + kPubQ,          // [kPubQ] status posted (1: publisher lane)
-    kBarDrain = kBarPubEmpty + kPubQ,            // every MMA of the CTA finished (commit)
-    kNumBars = kBarDrain + 1
+// Layout for a channel tile of NC = 128 or 64 channels (MMA N).  The narrow tile gives twice
+// the (sequence, tile) units, so that small batches fill the GPU without splitting sequences;
+// its rings are twice as deep (same bytes) and tensor memory holds four accumulator slots.
+template <int NC>
+struct Geo {
+    static_assert(NC == 64 || NC == 128, "channel tile");
+    static constexpr int kTile = kC * NC * 2;                 // one bf16 [C][NC] activation tile
+    static constexpr int kStageBytes = 2 * kTile;             // k (overwritten by U) then v
+    static constexpr int kKVStages = NC == 128 ? 4 : 8;
+    static constexpr int kQStages = NC == 128 ? 3 : 6;        // q tiles; y is staged in place
+    static constexpr int kSlotCols = 2 * NC;                  // fused [NC cols] | carry [NC cols]
+    static constexpr int kSlots = (int)kTmemCols / kSlotCols;
+    static constexpr int kSBytes = kKS * NC * 2;              // [32 rows][NC ch] bf16, 128-byte swizzled
+    static constexpr int kSmQ = kSmKV + kKVStages * kStageBytes;
+    static constexpr int kSmS = kSmQ + kQStages * kTile;
+    static constexpr int kSmBar = kSmS + kSBufs * kSBytes;
+    // barrier slots (arrival counts in parentheses; "commit" = tcgen05.commit from the MMA thread)
+    static constexpr int kBarKVFull = 0;                              // [kKVStages] k,v landed (1 + tx)
+    static constexpr int kBarKVEmpty = kBarKVFull + kKVStages;        // [kKVStages] fused product read U (commit)
+    static constexpr int kBarURdy = kBarKVEmpty + kKVStages;          // [kKVStages] U formed over k (128: U group)
+    static constexpr int kBarQFull = kBarURdy + kKVStages;            // [kQStages] q landed (1 + tx)
+    static constexpr int kBarQEmpty = kBarQFull + kQStages;           // [kQStages] y stored, buffer free (1)
+    static constexpr int kBarYStaged = kBarQEmpty + kQStages;         // [kQStages] gated y staged (128: E group)
+    static constexpr int kBarWDone = kBarYStaged + kQStages;          // [kSlots] fused product done (commit)
+    static constexpr int kBarD2Free = kBarWDone + kSlots;             // [kSlots] state rows read out (128: S)
+    static constexpr int kBarYDone = kBarD2Free + kSlots;             // [kSlots] carry done (commit)
+    static constexpr int kBarD1Free = kBarYDone + kSlots;             // [kSlots] output rows read out (128: E)
+    static constexpr int kBarSRdy = kBarD1Free + kSlots;              // [kSBufs] state operand written (128: S)
+    static constexpr int kBarSTFree = kBarSRdy + kSBufs;              // [kSBufs] state operand read (commit)
+    static constexpr int kBarItemFull = kBarSTFree + kSBufs;          // [kItemQ] item id posted (1)
+    static constexpr int kBarItemEmpty = kBarItemFull + kItemQ;       // [kItemQ] id read by every consumer
+    static constexpr int kBarConst = kBarItemEmpty + kItemQ;          // head constants landed (1 + tx)
+    static constexpr int kBarConstFree = kBarConst + 1;               // MMAs on the old constants done (commit)
+    static constexpr int kBarPubFull = kBarConstFree + 1;             // [kPubQ] segment state written (128: S)
+    static constexpr int kBarPubEmpty = kBarPubFull + kPubQ;          // [kPubQ] status posted (1: publisher)
+    static constexpr int kBarDrain = kBarPubEmpty + kPubQ;            // every MMA of the CTA finished (commit)
+    static constexpr int kNumBars = kBarDrain + 1;
+    static constexpr int kSmMisc = kSmBar + kNumBars * 8;
+    static constexpr int kSmemBytes = kSmMisc + 128 + 1024;           // + ids, misc words, queues, slack
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+    static_assert(kSmQ % 1024 == 0 && kSmS % 1024 == 0, "swizzle atoms");
+
+    __host__ __device__ static constexpr int count(int i) {
+        return ((i >= kBarURdy && i < kBarQFull) || (i >= kBarYStaged && i < kBarWDone) ||
+                (i >= kBarD2Free && i < kBarYDone) || (i >= kBarD1Free && i < kBarSTFree) ||
+                (i >= kBarPubFull && i < kBarPubEmpty))
+                   ? 128
+                   : (i >= kBarItemEmpty && i < kBarConst) ? kItemReaders : 1;
+    }
 };
-// item readers: q loader, store lane, MMA lane (1 each) + lane 0 of the 4 U, 4 S and 4 E warps
-constexpr int kItemReaders = 3 + 12;
-constexpr int kSmMisc = kSmBar + kNumBars * 8;
-constexpr int kCQ = 4;                                    // items whose carries the MMA thread still owes
-constexpr int kSmemBytes = kSmMisc + 128 + 1024;          // + item ids, misc words, carry queue, slack
-static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-static_assert(kSmKV % 1024 == 0 && kSmQ % 1024 == 0 && kSmS % 1024 == 0, "swizzle atoms");
-
-__host__ __device__ constexpr int bar_count(int i) {
-    return ((i >= kBarURdy && i < kBarQFull) || (i >= kBarYStaged && i < kBarWDone) ||
-            (i >= kBarD2Free && i < kBarYDone) || (i >= kBarD1Free && i < kBarSTFree) ||
-            (i >= kBarPubFull && i < kBarPubEmpty))
-               ? 128
-               : (i >= kBarItemEmpty && i < kBarConst) ? kItemReaders : 1;
-}
 
 // warp roles (16 warps).  The state group must sit on warps w % 4 == 2 (TMEM lanes 64..95, the
 // state rows); the output group on w % 4 in {0, 1} (lanes 0..63, the token rows).
@@ -150,7 +154,7 @@ __host__ __device__ __forceinline__ int cm_off16(int row, int k, int K) {
 
 struct ChunkArgs {
     int L, Dch, d, ch, H;
-    int tph;             // channel tiles per head (ch / 128)
+    int tph;             // channel tiles per head (ch / NC)
     int units_h;         // (sequence, tile) units per head: B * tph
     int ih;              // items per head: units_h * nseg
     int nchunks;         // chunks per sequence
@@ -162,8 +166,8 @@ struct ChunkArgs {
     int *sched;          // [1] error code
     int *tickets;        // [H] ticket counter per head
     int *status;         // [items]: 0 none, 1 segment contribution, 2 inclusive state
-    float *agg;          // [items][32 rows][128 ch]
-    float *inc;          // [items][32 rows][128 ch]
+    float *agg;          // [items][32 rows][NC ch]
+    float *inc;          // [items][32 rows][NC ch]
 };
 
 struct Item {
@@ -171,6 +175,7 @@ struct Item {
     bool last_seg;
 };
 
+template <int NC>
 __device__ __forceinline__ Item decode_item(const ChunkArgs &a, int id) {
     Item it;
     it.id = id;
@@ -179,7 +184,7 @@ __device__ __forceinline__ Item decode_item(const ChunkArgs &a, int id) {
     const int unit = t % a.units_h;         // predecessor of item id is id - units_h
     it.seg = t / a.units_h;
     it.b = unit / a.tph;
-    it.c0 = it.hd * a.ch + (unit % a.tph) * kNC;
+    it.c0 = it.hd * a.ch + (unit % a.tph) * NC;
     it.ck0 = it.seg * a.segc;
     it.nck = min(a.nchunks, it.ck0 + a.segc) - it.ck0;
     it.last_seg = (it.seg == a.nseg - 1);
@@ -224,6 +229,28 @@ __device__ __forceinline__ void warp_transpose32(float *v, int lane) {
             if (upper) v[i] = recv; else v[i | m] = recv;
         }
     }
+}
+
+// The same within each half-warp for a 16 x 16 block: lanes 16 h + i hold rows 16 h + i
+// (v[j] = M[16 h + i][j]) and end up with columns (v[j] = M[16 h + j][i]).
+__device__ __forceinline__ void warp_transpose16x2(float *v, int lane) {
+#pragma unroll
+    for (int m = 8; m >= 1; m >>= 1) {
+        const bool upper = (lane & m) != 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (i & m) continue;
+            const float send = upper ? v[i] : v[i | m];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, m);
+            if (upper) v[i] = recv; else v[i | m] = recv;
+        }
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float *v) {
+    if constexpr (N == 32) tc::tmem_ld32(taddr, v);
+    else tc::tmem_ld16(taddr, v);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -338,10 +365,23 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
 //                 4, 5, 8, 9      E group: token rows 0..63 x 64 channels each; gate and stage y
 // Each role loops over the same item sequence and the same chunk order; they meet only at
 // mbarriers, so loads, U, the products, the chain and the epilogue of different chunks overlap.
+template <int NC>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_y,
                      const ChunkArgs a) {
+    using G = Geo<NC>;
+    constexpr int kNC = NC, kTile = G::kTile, kStageBytes = G::kStageBytes, kKVStages = G::kKVStages,
+                  kQStages = G::kQStages, kSlots = G::kSlots, kSlotCols = G::kSlotCols, kSBytes = G::kSBytes,
+                  kSmQ = G::kSmQ, kSmS = G::kSmS, kSmBar = G::kSmBar, kSmMisc = G::kSmMisc;
+    constexpr int kBarKVFull = G::kBarKVFull, kBarKVEmpty = G::kBarKVEmpty, kBarURdy = G::kBarURdy,
+                  kBarQFull = G::kBarQFull, kBarQEmpty = G::kBarQEmpty, kBarYStaged = G::kBarYStaged,
+                  kBarWDone = G::kBarWDone, kBarD2Free = G::kBarD2Free, kBarYDone = G::kBarYDone,
+                  kBarD1Free = G::kBarD1Free, kBarSRdy = G::kBarSRdy, kBarSTFree = G::kBarSTFree,
+                  kBarItemFull = G::kBarItemFull, kBarItemEmpty = G::kBarItemEmpty, kBarConst = G::kBarConst,
+                  kBarConstFree = G::kBarConstFree, kBarPubFull = G::kBarPubFull, kBarPubEmpty = G::kBarPubEmpty,
+                  kBarDrain = G::kBarDrain, kNumBars = G::kNumBars;
+    constexpr int kCh = kNC / 4;        // channels of one S-group thread
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = tc::smem_u32(sm);
@@ -357,7 +397,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (tid == 0) {
         misc[0] = 0;
         misc[2] = 0;
-        for (int i = 0; i < kNumBars; ++i) tc::mbar_init(bar(i), bar_count(i));
+        for (int i = 0; i < kNumBars; ++i) tc::mbar_init(bar(i), G::count(i));
         tc::fence_mbar_init();
     }
     if (warp == kWarpMMA) {
@@ -408,7 +448,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 itemq[s] = id;
                 tc::mbar_arrive(bar(kBarItemFull + s));
                 if (id < 0) break;
-                const Item it = decode_item(a, id);
+                const Item it = decode_item<NC>(a, id);
                 for (int i = 0; i < it.niter; ++i, ++g) {
                     const int chunk = it.ck0 + (i < it.n1 ? i : i - it.n1);
                     const int st = g % kKVStages;
@@ -418,9 +458,9 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     }
                     const uint32_t dst = sbase + kSmKV + st * kStageBytes;
                     tc::mbar_expect_tx(bar(kBarKVFull + st), kStageBytes);
-                    for (int h = 0; h < 2; ++h) {
-                        tc::tma_load_3d(dst + h * kHalf, &tm_k, bar(kBarKVFull + st), it.c0 + 64 * h, tok_of(chunk), it.b);
-                        tc::tma_load_3d(dst + kTile + h * kHalf, &tm_v, bar(kBarKVFull + st), it.c0 + 64 * h,
+                    for (int h = 0; h < kNC / 64; ++h) {
+                        tc::tma_load_3d(dst + h * kAtom, &tm_k, bar(kBarKVFull + st), it.c0 + 64 * h, tok_of(chunk), it.b);
+                        tc::tma_load_3d(dst + kTile + h * kAtom, &tm_v, bar(kBarKVFull + st), it.c0 + 64 * h,
                                         tok_of(chunk), it.b);
                     }
                 }
@@ -441,7 +481,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int id = take_item(k, false);
                 if (id == -2) ok = false;
                 if (id < 0) break;
-                const Item it = decode_item(a, id);
+                const Item it = decode_item<NC>(a, id);
                 for (int j = 0; j < it.nck; ++j, ++qg) {
                     const int s = qg % kQStages;
                     if (!tc::mbar_wait(bar(kBarQEmpty + s), ((qg / kQStages) & 1) ^ 1, abort)) {
@@ -449,8 +489,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         break;
                     }
                     tc::mbar_expect_tx(bar(kBarQFull + s), kTile);
-                    for (int h = 0; h < 2; ++h)
-                        tc::tma_load_3d(sbase + kSmQ + s * kTile + h * kHalf, &tm_q, bar(kBarQFull + s),
+                    for (int h = 0; h < kNC / 64; ++h)
+                        tc::tma_load_3d(sbase + kSmQ + s * kTile + h * kAtom, &tm_q, bar(kBarQFull + s),
                                         it.c0 + 64 * h, tok_of(it.ck0 + j), it.b);
                 }
             }
@@ -469,7 +509,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int id = take_item(k, false);
                 if (id == -2) ok = false;
                 if (id < 0) break;
-                const Item it = decode_item(a, id);
+                const Item it = decode_item<NC>(a, id);
                 for (int j = 0; j < it.nck; ++j, ++qg) {
                     const int s = qg % kQStages;
                     if (!tc::mbar_wait(bar(kBarYStaged + s), (qg / kQStages) & 1, abort)) {
@@ -478,8 +518,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     }
                     const int tok = tok_of(it.ck0 + j);
                     if (tok >= 0) {     // a chunk that starts before token 0 was written by the E group
-                        for (int h = 0; h < 2; ++h)
-                            tc::tma_store_3d(&tm_y, sbase + kSmQ + s * kTile + h * kHalf, it.c0 + 64 * h, tok, it.b);
+                        for (int h = 0; h < kNC / 64; ++h)
+                            tc::tma_store_3d(&tm_y, sbase + kSmQ + s * kTile + h * kAtom, it.c0 + 64 * h, tok, it.b);
                         tc::bulk_commit();
                         tc::bulk_wait_read<0>();
                     }
@@ -520,7 +560,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             int chead = 0, ctail = 0;       // carry queue: (n1, nck, first global fused index)
             int fk = 0, ic = 0, g = 0, jn = 0, pc = 0;
             int cur_hd = -1, cphase = 0, fphase = 0;
-            int c2a = 0, c2b = 0;           // full-pass uses of slot 0 / slot 1 issued so far
+            int c2bits = 0;                 // bit s: parity of the full-pass uses of slot s issued so far
             bool f_valid = false, need_const = false, done = false, any = false, ok = true;
             unsigned long long t_prog = tc::global_ns();
             while (ok && !*abort) {
@@ -536,7 +576,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         if (id < 0) {
                             done = true;
                         } else {
-                            fi = decode_item(a, id);
+                            fi = decode_item<NC>(a, id);
                             f_valid = true;
                             ic = 0;
                             need_const = fi.hd != cur_hd;
@@ -561,7 +601,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         const uint32_t sb_addr = sbase + kSmS + sb * kSBytes;
                         for (int ks = 0; ks < kKS / 16; ++ks)
                             tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmCA + ks * 256, 128, kKS * 16),
-                                         tc::smem_desc_sw128(sb_addr + ks * 2048, kSBytes / 2, 1024), idesc, ks > 0);
+                                         tc::smem_desc_sw128(sb_addr + ks * 2048, kKS * 128, 1024), idesc, ks > 0);
                         tc::mma_commit(bar(kBarYDone + slot));
                         tc::mma_commit(bar(kBarSTFree + sb));
                         ++pc;
@@ -590,18 +630,16 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     const int slot = g % kSlots, st = g % kKVStages;
                     if (tc::mbar_test(bar(kBarURdy + st), (g / kKVStages) & 1) &&
                         tc::mbar_test(bar(kBarD2Free + slot), ((g / kSlots) & 1) ^ 1) &&
-                        tc::mbar_test(bar(kBarD1Free + slot), ((slot ? c2b : c2a) & 1) ^ 1)) {
+                        tc::mbar_test(bar(kBarD1Free + slot), ((c2bits >> slot) & 1) ^ 1)) {
                         tc::tc_fence_after();
                         const uint32_t dcol = tmem + slot * kSlotCols;
                         const uint32_t u_addr = sbase + kSmKV + st * kStageBytes;
                         for (int ks = 0; ks < kC / 16; ++ks)
                             tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmFA + ks * 256, 128, kC * 16),
-                                         tc::smem_desc_sw128(u_addr + ks * 2048, kHalf, 1024), idesc, ks > 0);
+                                         tc::smem_desc_sw128(u_addr + ks * 2048, kAtom, 1024), idesc, ks > 0);
                         tc::mma_commit(bar(kBarWDone + slot));
                         tc::mma_commit(bar(kBarKVEmpty + st));
-                        if (ic >= fi.n1) {
-                            if (slot) ++c2b; else ++c2a;
-                        }
+                        if (ic >= fi.n1) c2bits ^= 1 << slot;
                         ++g;
                         any = true;
                         progressed = true;
@@ -634,7 +672,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const int id = take_item(k, true);
             if (id == -2) ok = false;
             if (id < 0) break;
-            const Item it = decode_item(a, id);
+            const Item it = decode_item<NC>(a, id);
             for (int i = 0; i < it.niter; ++i, ++g) {
                 const int st = g % kKVStages;
                 if (!(ok = uni(tc::mbar_wait(bar(kBarKVFull + st), (g / kKVStages) & 1, abort)))) break;
@@ -659,14 +697,14 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     } else if (is_s_warp(warp)) {
         // ------------------------------------------------------------ S group (state chain)
         // thread: state row r = lane (mode r % 16, Re for r < 16, Im above) for channels
-        // 32 q4 .. 32 q4 + 31 of the tile; TMEM lane 64 + r holds row r of the state product W
+        // kCh q4 .. kCh q4 + kCh - 1 of the tile; TMEM lane 64 + r holds row r of the state product W
         const int q4 = warp >> 2, r = lane, n = r & (kIm - 1);
         const bool leader = (warp == 2 && lane == 0);
         const float sgn = (r < kIm) ? -1.f : 1.f;
         const uint32_t lane_base = (uint32_t)64 << 16;
         int g = 0, pc = 0, pub_k = 0, cur_hd = -1;
         bool ok = true;
-        float st[32];
+        float st[kCh];
         float2 lamC = make_float2(0.f, 0.f), lamS = lamC;
         // hand one entry to the publisher lane (all 128 threads call this after their writes)
         auto post = [&](int v) -> bool {
@@ -684,7 +722,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const int id = take_item(k, true);
             if (id == -2) ok = false;
             if (id < 0) break;
-            const Item it = decode_item(a, id);
+            const Item it = decode_item<NC>(a, id);
             if (it.hd != cur_hd) {
                 const float2 *lp = reinterpret_cast<const float2 *>(a.consts + (size_t)it.hd * kConstStride + kLamOff);
                 lamC = lp[n];               // zero for modes >= d
@@ -692,40 +730,40 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 cur_hd = it.hd;
             }
 #pragma unroll
-            for (int i = 0; i < 32; ++i) st[i] = 0.f;
+            for (int i = 0; i < kCh; ++i) st[i] = 0.f;
 
             // st <- lambda^C st + W of iteration gi
             auto advance = [&](int gi) -> bool {
                 const int slot = gi % kSlots;
                 if (!uni(tc::mbar_wait(bar(kBarWDone + slot), (gi / kSlots) & 1, abort))) return false;
                 tc::tc_fence_after();
-                float w[32];
-                tc::tmem_ld32(tmem + lane_base + slot * kSlotCols + 32 * q4, w);
+                float w[kCh];
+                tmem_ld<kCh>(tmem + lane_base + slot * kSlotCols + kCh * q4, w);
                 tc::tmem_wait_ld();
                 tc::tc_fence_before();
                 tc::mbar_arrive(bar(kBarD2Free + slot));
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
+                for (int i = 0; i < kCh; ++i) {
                     const float p = __shfl_xor_sync(0xffffffffu, st[i], 16);    // the other part of mode n
                     st[i] = fmaf(lamC.x, st[i], fmaf(sgn * lamC.y, p, w[i]));
                 }
                 return true;
             };
-            // this thread's row of a published [32 rows][128 ch] state (bypassing L1)
+            // this thread's row of a published [32 rows][NC ch] state (bypassing L1)
             auto load_rows = [&](const float *src, float *o) {
-                const float4 *p4 = reinterpret_cast<const float4 *>(src + (size_t)r * kNC + 32 * q4);
+                const float4 *p4 = reinterpret_cast<const float4 *>(src + (size_t)r * kNC + kCh * q4);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
+                for (int i = 0; i < kCh / 4; ++i) {
                     const float4 v4 = __ldcg(p4 + i);
                     o[4 * i] = v4.x; o[4 * i + 1] = v4.y; o[4 * i + 2] = v4.z; o[4 * i + 3] = v4.w;
                 }
             };
-            // write the state rows of this thread to dst [32 rows][128 ch] and hand `code` to the
+            // write the state rows of this thread to dst [32 rows][NC ch] and hand `code` to the
             // publisher lane, which posts it once every row is written (no wait here)
             auto publish = [&](const float *v, float *dst, int code) -> bool {
-                float4 *o = reinterpret_cast<float4 *>(dst + (size_t)r * kNC + 32 * q4);
+                float4 *o = reinterpret_cast<float4 *>(dst + (size_t)r * kNC + kCh * q4);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                for (int i = 0; i < kCh / 4; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
                 return post(it.id * 4 + code);
             };
 
@@ -735,9 +773,9 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const size_t item_off = (size_t)it.id * kKS * kNC;
             if (it.n1 > 0 && !(ok = uni(publish(st, (it.seg == 0 ? a.inc : a.agg) + item_off, it.seg == 0 ? 2 : 1))))
                 break;
-            float sloc[32];
+            float sloc[kCh];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) { sloc[i] = st[i]; st[i] = 0.f; }
+            for (int i = 0; i < kCh; ++i) { sloc[i] = st[i]; st[i] = 0.f; }
 
             // look-back: the state entering this segment.  The inclusive states follow the fixed
             // fp32 recurrence inc(s) = lambda^Lseg inc(s-1) + agg(s), inc(0) = agg(0): find the
@@ -769,15 +807,15 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 __syncwarp();       // lane 0's acquire loads order the other lanes' reads below
                 load_rows(a.inc + (size_t)p0 * kKS * kNC, st);
                 for (int p = p0 + units; p < it.id; p += units) {
-                    float ag[32];
+                    float ag[kCh];
                     load_rows(a.agg + (size_t)p * kKS * kNC, ag);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) st[i] = seg_step(st[i], ag[i], lamS, sgn);
+                    for (int i = 0; i < kCh; ++i) st[i] = seg_step(st[i], ag[i], lamS, sgn);
                 }
                 if (it.n1 > 0) {
                     // inclusive state at the end of this segment (sloc is not needed after this)
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) sloc[i] = seg_step(st[i], sloc[i], lamS, sgn);
+                    for (int i = 0; i < kCh; ++i) sloc[i] = seg_step(st[i], sloc[i], lamS, sgn);
                     if (!(ok = uni(publish(sloc, a.inc + item_off, 2)))) break;
                 }
             }
@@ -786,17 +824,20 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             for (int j = 0; j < it.nck && ok; ++j, ++g, ++pc) {
                 const int sb = pc % kSBufs;
                 if (!(ok = uni(tc::mbar_wait(bar(kBarSTFree + sb), ((pc / kSBufs) & 1) ^ 1, abort)))) break;
-                // row r of the MN-major, 128-byte swizzled [32 rows][128 ch] operand: channel block
-                // q4 is 64 bytes of row r in swizzle atom q4 / 2
-                uint8_t *sp = sm + kSmS + sb * kSBytes + (q4 >> 1) * (kSBytes / 2) + (r >> 3) * 1024 + (r & 7) * 128;
+                // row r of the MN-major, 128-byte swizzled [32 rows][NC ch] operand: this thread's
+                // channels are kCh * 2 bytes of row r in swizzle atom (kCh q4) / 64 (atoms of
+                // 64 channels x 32 rows, 4 KB apart)
+                constexpr int kC16 = kCh / 8;                       // 16-byte chunks of the thread
+                const int cb = kCh * q4;
+                uint8_t *sp = sm + kSmS + sb * kSBytes + (cb / 64) * (kKS * 128) + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int i = 0; i < kC16; ++i) {
                     uint4 v;
                     v.x = pack_bf16(st[8 * i + 0], st[8 * i + 1]);
                     v.y = pack_bf16(st[8 * i + 2], st[8 * i + 3]);
                     v.z = pack_bf16(st[8 * i + 4], st[8 * i + 5]);
                     v.w = pack_bf16(st[8 * i + 6], st[8 * i + 7]);
-                    *reinterpret_cast<uint4 *>(sp + ((((q4 & 1) * 4 + i) ^ (r & 7)) << 4)) = v;
+                    *reinterpret_cast<uint4 *>(sp + (((((cb & 63) >> 3) + i) ^ (r & 7)) << 4)) = v;
                 }
                 tc::fence_proxy_async_smem();
                 tc::mbar_arrive(bar(kBarSRdy + sb));
@@ -804,52 +845,64 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             }
             if (!ok) break;
             if (it.last_seg) {
-                // transpose the warp's 32 x 32 block (rows r in lanes -> channels in lanes) so that
-                // each lane writes the (Re, Im) pairs of one channel: coalesced float2 stores
-                warp_transpose32(st, lane);
-                float2 *so = reinterpret_cast<float2 *>(a.state_out) + ((size_t)it.b * d) * a.Dch + it.c0 + 32 * q4 + lane;
+                if constexpr (kCh == 32) {
+                    // transpose the warp's 32 x 32 block (rows r in lanes -> channels in lanes) so
+                    // that each lane writes the (Re, Im) pairs of one channel: coalesced float2 stores
+                    warp_transpose32(st, lane);
+                    float2 *so = reinterpret_cast<float2 *>(a.state_out) + ((size_t)it.b * d) * a.Dch + it.c0 + kCh * q4 + lane;
 #pragma unroll
-                for (int m = 0; m < kMaxModes; ++m)
-                    if (m < d) so[(size_t)m * a.Dch] = make_float2(st[m], st[kIm + m]);
+                    for (int m = 0; m < kMaxModes; ++m)
+                        if (m < d) so[(size_t)m * a.Dch] = make_float2(st[m], st[kIm + m]);
+                } else {
+                    // 16 channels: transpose each half-warp's 16 x 16 block; lane 16 h + i then holds
+                    // part h (Re, Im) of every mode for channel i, and a warp store covers 16
+                    // channels x (Re, Im) = 128 contiguous bytes
+                    warp_transpose16x2(st, lane);
+                    float *so = a.state_out + (((size_t)it.b * d) * a.Dch + it.c0 + kCh * q4 + (lane & 15)) * 2 + (lane >> 4);
+#pragma unroll
+                    for (int m = 0; m < kMaxModes; ++m)
+                        if (m < d) so[(size_t)m * a.Dch * 2] = st[m];
+                }
             }
         }
         if (!ok) record_error(a, abort, kErrWait);
         post(-1);       // end of this CTA's posts
     } else if (is_e_warp(warp)) {
         // ------------------------------------------------------------ E group (gate and stage y)
-        // thread: token row tau = 32 q4 + lane (TMEM lane tau) for channels 64 hh .. 64 hh + 63
+        // thread: token row tau = 32 q4 + lane (TMEM lane tau) for channels NC/2 hh .. NC/2 (hh+1) - 1
         const int q4 = warp & 3, hh = warp >> 3, tau = 32 * q4 + lane;
         const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
         int g = 0, qg = 0;
-        int e2a = 0, e2b = 0;       // full-pass uses of slot 0 / slot 1 consumed so far
+        int e2bits = 0;             // bit s: parity of the full-pass uses of slot s consumed so far
         bool ok = true;
         for (int k = 0; ok; ++k) {
             const int id = take_item(k, true);
             if (id == -2) ok = false;
             if (id < 0) break;
-            const Item it = decode_item(a, id);
+            const Item it = decode_item<NC>(a, id);
             g += it.n1;
             for (int j = 0; j < it.nck; ++j, ++g, ++qg) {
                 const int slot = g % kSlots, s = qg % kQStages;
-                ok = uni(tc::mbar_wait(bar(kBarYDone + slot), (slot ? e2b : e2a) & 1, abort) &&
+                ok = uni(tc::mbar_wait(bar(kBarYDone + slot), (e2bits >> slot) & 1, abort) &&
                          tc::mbar_wait(bar(kBarQFull + s), (qg / kQStages) & 1, abort));
                 if (!ok) break;
-                if (slot) ++e2b; else ++e2a;
+                e2bits ^= 1 << slot;
                 tc::tc_fence_after();
                 const int tok = tok_of(it.ck0 + j);
-                uint8_t *qrow = sm + kSmQ + s * kTile + hh * kHalf + tau * 128;
                 const bool store_direct = tok < 0, row_valid = tok + tau >= 0;
-                __nv_bfloat16 *yrow = a.y + ((size_t)it.b * a.L + (row_valid ? tok + tau : 0)) * a.Dch + it.c0 + 64 * hh;
+                __nv_bfloat16 *yrow = a.y + ((size_t)it.b * a.L + (row_valid ? tok + tau : 0)) * a.Dch + it.c0;
 #pragma unroll
-                for (int x = 0; x < 2; ++x) {
+                for (int x = 0; x < kNC / 64; ++x) {
+                    const int cbase = hh * (kNC / 2) + 32 * x;      // first of 32 channels
+                    uint8_t *qrow = sm + kSmQ + s * kTile + (cbase / 64) * kAtom + tau * 128;
                     float z[32], cz[32];
-                    const uint32_t col = tmem + lane_base + slot * kSlotCols + 64 * hh + 32 * x;
+                    const uint32_t col = tmem + lane_base + slot * kSlotCols + cbase;
                     tc::tmem_ld32(col, z);
                     tc::tmem_ld32(col + kNC, cz);
                     tc::tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const int chunk16 = 4 * x + i;          // 16-byte chunk (8 channels) of the row
+                        const int chunk16 = ((cbase & 63) >> 3) + i;   // 16-byte chunk (8 channels) of the row
                         uint4 *qp = reinterpret_cast<uint4 *>(qrow + ((chunk16 ^ (tau & 7)) << 4));
                         const uint4 qv = *qp;
                         const float *zz = z + 8 * i, *cc = cz + 8 * i;
@@ -861,7 +914,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         if (!store_direct)
                             *qp = yv;
                         else if (row_valid)
-                            *reinterpret_cast<uint4 *>(yrow + 8 * chunk16) = yv;
+                            *reinterpret_cast<uint4 *>(yrow + cbase + 8 * i) = yv;
                     }
                 }
                 tc::tc_fence_before();
@@ -907,41 +960,53 @@ bool make_map(CUtensorMap *m, const void *base, int B, int L, int Dch) {
 constexpr size_t kTicketOff = 64;    // byte offset of the per-head ticket counters in the schedule block
 
 struct ChunkPlan {
-    int nchunks, nseg, segc, items;
+    int nc, nchunks, nseg, segc, items;
     size_t consts_off, sched_off, status_off, agg_off, inc_off, total;
 };
 
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 
-constexpr int kPlanSMs = 148;   // segment choice is made for a full B200 (any count runs correctly)
+constexpr int kPlanSMs = 148;   // the plan is made for a full B200 (any SM count runs correctly)
 
+// Channel tile and segment count.  Costs are in units of one 128-channel chunk pass: a pass of
+// an NC-channel tile costs NC/128 plus a fixed 0.1, an item 1 more, and 6 more when its sequence
+// is split (the state-only pass is counted in the work; the look-back and publication latency
+// is the 6).  The estimated makespan is the larger of the even share and the largest item, plus
+// half an item of tail when there are more items than SMs.  The narrow tile and unsplit
+// sequences are preferred whenever they do not cost more.
 ChunkPlan plan(int B, int L, int Dch, int H) {
     ChunkPlan p{};
     p.nchunks = (L + kC - 1) / kC;
-    const long long units = (long long)B * (Dch / kNC);
-    // segments: each non-last segment costs a second (state-only) pass over its chunks, and
-    // every item a little fixed work; pick the count that minimises the estimated makespan
-    // (total chunk passes spread over the SMs + the largest item)
+    const int ch = Dch / H;
     double best = 1e300;
-    int best_segc = p.nchunks > 0 ? p.nchunks : 1;
-    for (int want = 1; want <= kMaxSeg && want <= (p.nchunks > 0 ? p.nchunks : 1); ++want) {
-        const int segc = (p.nchunks + want - 1) / want;
-        const int nseg = (p.nchunks + segc - 1) / segc;
-        const double items = (double)units * nseg;
-        const double work = (double)units * (p.nchunks + (double)(nseg - 1) * segc) + 1.5 * items;
-        const double ctas = items < kPlanSMs ? items : kPlanSMs;
-        const double est = work / ctas + (nseg > 1 ? 2.0 * segc : segc);
-        if (est < best - 1e-9) { best = est; best_segc = segc; }
+    p.nc = ch % 128 == 0 ? 128 : 64;
+    p.segc = p.nchunks > 0 ? p.nchunks : 1;
+    for (int nc : {128, 64}) {
+        if (ch % nc != 0) continue;
+        const double units = (double)B * (Dch / nc);
+        const double pass = nc / 128.0 + 0.1;
+        const int nch = p.nchunks > 0 ? p.nchunks : 1;
+        for (int want = 1; want <= kMaxSeg && want <= nch; ++want) {
+            const int segc = (nch + want - 1) / want;
+            const int nseg = (nch + segc - 1) / segc;
+            const double items = units * nseg;
+            const double ovh = nseg > 1 ? 7.0 : 1.0;
+            const double work = units * (nch + (double)(nseg - 1) * segc) * pass + items * ovh;
+            const double ctas = items < kPlanSMs ? items : kPlanSMs;
+            const double item_max = (nseg > 1 ? 2.0 * segc : (double)segc) * pass + ovh;
+            double est = work / ctas > item_max ? work / ctas : item_max;
+            if (items > kPlanSMs) est += 0.5 * item_max;
+            if (est < best * (1 - 1e-9)) { best = est; p.nc = nc; p.segc = segc; }
+        }
     }
-    p.segc = best_segc;
     p.nseg = p.nchunks > 0 ? (p.nchunks + p.segc - 1) / p.segc : 1;
-    p.items = (int)(units * p.nseg);
+    p.items = (int)((long long)B * (Dch / p.nc) * p.nseg);
     p.consts_off = 0;
     p.sched_off = al256((size_t)H * kConstStride);
     p.status_off = p.sched_off + al256(kTicketOff + (size_t)H * 4);
     p.agg_off = p.status_off + al256((size_t)p.items * 4);
-    p.inc_off = p.agg_off + al256((size_t)p.items * kKS * kNC * 4);
-    p.total = p.inc_off + al256((size_t)p.items * kKS * kNC * 4);
+    p.inc_off = p.agg_off + al256((size_t)p.items * kKS * p.nc * 4);
+    p.total = p.inc_off + al256((size_t)p.items * kKS * p.nc * 4);
     return p;
 }
 
@@ -961,13 +1026,26 @@ int sm_count() {
 }  // namespace
 
 bool chunked_supported(int dtype, int Dch, int H, int d) {
-    return dtype == HYENA_BF16 && H > 0 && Dch % H == 0 && (Dch / H) % kNC == 0 && d >= 1 && d <= kMaxModes;
+    return dtype == HYENA_BF16 && H > 0 && Dch % H == 0 && (Dch / H) % 64 == 0 && d >= 1 && d <= kMaxModes;
 }
 
 size_t chunked_ws_bytes(int B, int L, int Dch, int H, int d) {
     (void)d;
     return plan(B, L, Dch, H).total;
 }
+
+namespace {
+template <int NC>
+cudaError_t launch_tile(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &my,
+                        const ChunkArgs &a, int items, cudaStream_t s) {
+    constexpr int smem = Geo<NC>::kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(prefill_chunk_kernel<NC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int grid = items < sm_count() ? items : sm_count();
+    prefill_chunk_kernel<NC><<<grid, kThreads, smem, s>>>(mq, mk, mv, my, a);
+    return cudaGetLastError();
+}
+}  // namespace
 
 cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, int B, int L, int Dch,
                                    int H, int d, const float2 *lam, const float2 *R, const float *Dskip,
@@ -985,7 +1063,7 @@ cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, 
         return cudaErrorInvalidValue;
     ChunkArgs a;
     a.L = L; a.Dch = Dch; a.d = d; a.ch = Dch / H; a.H = H;
-    a.tph = a.ch / kNC; a.units_h = B * a.tph; a.ih = a.units_h * p.nseg;
+    a.tph = a.ch / p.nc; a.units_h = B * a.tph; a.ih = a.units_h * p.nseg;
     a.nchunks = p.nchunks; a.tok_base = L - p.nchunks * kC;
     a.nseg = p.nseg; a.segc = p.segc;
     a.consts = w + p.consts_off;
@@ -996,11 +1074,7 @@ cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, 
     a.status = reinterpret_cast<int *>(w + p.status_off);
     a.agg = reinterpret_cast<float *>(w + p.agg_off);
     a.inc = reinterpret_cast<float *>(w + p.inc_off);
-    e = cudaFuncSetAttribute(prefill_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    const int grid = p.items < sm_count() ? p.items : sm_count();
-    prefill_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, my, a);
-    return cudaGetLastError();
+    return p.nc == 128 ? launch_tile<128>(mq, mk, mv, my, a, p.items, s) : launch_tile<64>(mq, mk, mv, my, a, p.items, s);
 }
 
 int chunked_error_offset(int B, int L, int Dch, int H, int d) {

@@ -174,10 +174,12 @@ int hyena_prefill_noalloc(const void *q, const void *k, const void *v, int dtype
  * (s(c0+C) = lambda^C s(c0) + sum_j lambda^(c0+C-1-j) u_j); the last state is
  * the prompt state.  (The "FFT (or chunked)" evaluation of the long
  * convolution; the carry is the distilled recurrence of "Laughing Hyena
- * Distillery", "Main findings".)  Products run in tf32 with fp32 accumulation;
- * the state is carried in fp32.
+ * Distillery", "Main findings".)  The products take bf16 operands (u = k v,
+ * the taps, the powers and the state rounded to bf16) with fp32 accumulation;
+ * the state chain itself runs in fp32.  Chunks are aligned to the end of the
+ * prompt, so the last one ends at token L-1.
  *   Arguments as hyena_prefill, without fft_len.
- *   Implemented for: dtype HYENA_BF16, Dch/H a multiple of 128, d <= 16, all
+ *   Implemented for: dtype HYENA_BF16, Dch/H a multiple of 64, d <= 16, all
  *   activation pointers 16-byte aligned; HYENA_ERR_UNSUPPORTED otherwise.
  *   workspace: >= hyena_prefill_chunked_workspace_bytes() bytes, 256-byte aligned.
  *   The int32 at byte offset hyena_prefill_chunked_error_offset() of the

@@ -45,6 +45,9 @@ CASES = [
     (1, 1000, 384, 3, 1),     # d = 1
     (1, 4096, 128, 1, 16),    # one tile: the sequence is split into many segments (look-back)
     (2, 2048, 256, 2, 12),    # d not a multiple of 8
+    (2, 300, 128, 2, 16),     # 64-channel heads (64-channel tiles), ragged
+    (1, 4096, 128, 2, 16),    # 64-channel tiles, sequences split into segments (look-back)
+    (3, 1000, 192, 3, 5),     # 64-channel heads, three of them
 ]
 
 
@@ -114,7 +117,7 @@ def test_chunked_unsupported_shapes_are_rejected():
     with pytest.raises(ops.HyenaError) as e:
         ops.prefill_chunked(x32, x32, x32, lam, lam, D)          # fp32 activations
     assert e.value.status == -5
-    x = torch.zeros(1, 64, 128, dtype=torch.bfloat16, device="cuda")
+    x = torch.zeros(1, 64, 64, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(ops.HyenaError) as e:
-        ops.prefill_chunked(x, x, x, lam, lam, D)                # 64 channels per head
+        ops.prefill_chunked(x, x, x, lam, lam, D)                # 32 channels per head
     assert e.value.status == -5
