@@ -73,8 +73,10 @@ constexpr int kMaxSeg = 128;        // segments per sequence (bounds look-back w
 constexpr int kPubQ = 4;            // segment states written and waiting for their status word
 constexpr int kCQ = 4;              // items whose carries the MMA thread still owes
 constexpr uint32_t kTmemCols = 512; // all of tensor memory (one CTA per SM)
-// item readers: q loader, store lane, MMA lane (1 each) + lane 0 of the 4 U, 4 S and 4 E warps
-constexpr int kItemReaders = 3 + 12;
+// item readers: q loader, store lane, fused and carry MMA lanes (1 each) + lane 0 of the 3 U,
+// 4 S and 4 E warps
+constexpr int kItemReaders = 4 + 11;
+constexpr int kUThreads = 96;       // U group (3 warps)
 
 // per-head constants: the two A operands (copied verbatim into shared memory) and the powers
 // lambda^C, lambda^Lseg (read from global by the state group)
@@ -124,17 +126,18 @@ struct Geo {
     static constexpr int kBarConstFree = kBarConst + 1;               // MMAs on the old constants done (commit)
     static constexpr int kBarPubFull = kBarConstFree + 1;             // [kPubQ] segment state written (128: S)
     static constexpr int kBarPubEmpty = kBarPubFull + kPubQ;          // [kPubQ] status posted (1: publisher)
-    static constexpr int kBarDrain = kBarPubEmpty + kPubQ;            // every MMA of the CTA finished (commit)
-    static constexpr int kNumBars = kBarDrain + 1;
+    static constexpr int kBarDrain = kBarPubEmpty + kPubQ;            // fused issuer's MMAs finished (commit)
+    static constexpr int kBarDrainC = kBarDrain + 1;                  // carry issuer's MMAs finished (commit)
+    static constexpr int kNumBars = kBarDrainC + 1;
     static constexpr int kSmMisc = kSmBar + kNumBars * 8;
     static constexpr int kSmemBytes = kSmMisc + 128 + 1024;           // + ids, misc words, queues, slack
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
     static_assert(kSmQ % 1024 == 0 && kSmS % 1024 == 0, "swizzle atoms");
 
     __host__ __device__ static constexpr int count(int i) {
-        return ((i >= kBarURdy && i < kBarQFull) || (i >= kBarYStaged && i < kBarWDone) ||
-                (i >= kBarD2Free && i < kBarYDone) || (i >= kBarD1Free && i < kBarSTFree) ||
-                (i >= kBarPubFull && i < kBarPubEmpty))
+        return (i >= kBarURdy && i < kBarQFull) ? kUThreads
+               : ((i >= kBarYStaged && i < kBarWDone) || (i >= kBarD2Free && i < kBarYDone) ||
+                  (i >= kBarD1Free && i < kBarSTFree) || (i >= kBarPubFull && i < kBarPubEmpty))
                    ? 128
                    : (i >= kBarItemEmpty && i < kBarConst) ? kItemReaders : 1;
     }
@@ -142,10 +145,10 @@ struct Geo {
 
 // warp roles (16 warps).  The state group must sit on warps w % 4 == 2 (TMEM lanes 64..95, the
 // state rows); the output group on w % 4 in {0, 1} (lanes 0..63, the token rows).
-constexpr int kWarpKV = 0, kWarpQ = 1, kWarpMMA = 3, kWarpStore = 12;
+constexpr int kWarpKV = 0, kWarpQ = 1, kWarpMMA = 3, kWarpStore = 12, kWarpCarry = 13;
 __host__ __device__ constexpr bool is_s_warp(int w) { return (w & 3) == 2; }                 // 2, 6, 10, 14
 __host__ __device__ constexpr bool is_e_warp(int w) { return w == 4 || w == 5 || w == 8 || w == 9; }
-__host__ __device__ constexpr int u_index(int w) { return w == 7 ? 0 : w == 11 ? 1 : w == 13 ? 2 : w == 15 ? 3 : -1; }
+__host__ __device__ constexpr int u_index(int w) { return w == 7 ? 0 : w == 11 ? 1 : w == 15 ? 2 : -1; }
 
 // byte offset of bf16 element (row, k) in a K-major, no-swizzle core-matrix tile of K columns
 __host__ __device__ __forceinline__ int cm_off16(int row, int k, int K) {
@@ -380,7 +383,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                   kBarD1Free = G::kBarD1Free, kBarSRdy = G::kBarSRdy, kBarSTFree = G::kBarSTFree,
                   kBarItemFull = G::kBarItemFull, kBarItemEmpty = G::kBarItemEmpty, kBarConst = G::kBarConst,
                   kBarConstFree = G::kBarConstFree, kBarPubFull = G::kBarPubFull, kBarPubEmpty = G::kBarPubEmpty,
-                  kBarDrain = G::kBarDrain, kNumBars = G::kNumBars;
+                  kBarDrain = G::kBarDrain, kBarDrainC = G::kBarDrainC, kNumBars = G::kNumBars;
     constexpr int kCh = kNC / 4;        // channels of one S-group thread
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -391,12 +394,14 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     volatile int *misc = itemq + kItemQ;                                     // abort, tmem, never
     int *cqueue = const_cast<int *>(misc) + 4;                               // [kCQ][3]: n1, nck, g0
     volatile int *pubq = misc + 4 + 3 * kCQ;                                 // [kPubQ]: 4 item + code, -1 = end
+    volatile int *carry_issued = pubq + kPubQ;                               // carries issued so far
     volatile int *abort = misc;
     volatile int *never = misc + 2;
 
     if (tid == 0) {
         misc[0] = 0;
         misc[2] = 0;
+        *carry_issued = 0;
         for (int i = 0; i < kNumBars; ++i) tc::mbar_init(bar(i), G::count(i));
         tc::fence_mbar_init();
     }
@@ -545,116 +550,70 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             }
         }
     } else if (warp == kWarpMMA) {
-        // ------------------------------------------------------------ MMA issuer
-        // Two streams issued out of order from one thread, polled with non-blocking tests: the
-        // fused product of a chunk needs only its U operand and a free accumulator slot and runs
-        // ahead; the carry needs the state entering the chunk and follows when the S group
-        // delivers it.  Both streams run on across item boundaries (a small queue holds the
-        // items whose carries are still to come).  MMAs from one thread execute in issue order.
+        // ------------------------------------------------------------ fused-product issuer
+        // [Z; W] = [T; V] U for every iteration, in order.  Its waits only involve the U
+        // operand and a free accumulator slot, so it runs ahead of the state chain; the carries
+        // are issued by their own thread (the carry writes TMEM columns of its own, so the two
+        // need no mutual order).  Waits suspend in hardware (no polling loop on this thread).
         if (lane == 0) {
             const uint32_t idesc = tc::idesc_bf16(128, kNC, true);
-            // (indexed arrays would live in local memory, which the small L1 left beside this
-            // much shared memory turns into L2 round trips: the carry queue is in shared memory
-            // and the per-slot counters are scalars)
-            Item fi{};                      // item of the fused stream
-            int chead = 0, ctail = 0;       // carry queue: (n1, nck, first global fused index)
-            int fk = 0, ic = 0, g = 0, jn = 0, pc = 0;
-            int cur_hd = -1, cphase = 0, fphase = 0;
+            int g = 0, pcf = 0, cur_hd = -1, cphase = 0, fphase = 0;
             int c2bits = 0;                 // bit s: parity of the full-pass uses of slot s issued so far
-            bool f_valid = false, need_const = false, done = false, any = false, ok = true;
-            unsigned long long t_prog = tc::global_ns();
-            while (ok && !*abort) {
-                bool progressed = false;
-                // the next item for the fused stream
-                if (!f_valid && !done && ctail - chead < kCQ) {
-                    const int s = fk % kItemQ;
-                    if (tc::mbar_test(bar(kBarItemFull + s), (fk / kItemQ) & 1)) {
-                        const int id = itemq[s];
-                        tc::mbar_arrive(bar(kBarItemEmpty + s));
-                        ++fk;
-                        progressed = true;
-                        if (id < 0) {
-                            done = true;
-                        } else {
-                            fi = decode_item<NC>(a, id);
-                            f_valid = true;
-                            ic = 0;
-                            need_const = fi.hd != cur_hd;
-                            int *e = cqueue + 3 * (ctail % kCQ);
-                            e[0] = fi.n1;
-                            e[1] = fi.nck;
-                            e[2] = g;
-                            ++ctail;
-                        }
-                    }
-                }
-                // carry stream: Z += A S (own TMEM columns of the chunk's slot)
-                if (chead < ctail) {
-                    const int *e = cqueue + 3 * (chead % kCQ);
-                    const int c_nck = e[1];
-                    const int cgi = e[2] + e[0] + jn;
-                    const int sb = pc % kSBufs;
-                    if (cgi < g && tc::mbar_test(bar(kBarSRdy + sb), (pc / kSBufs) & 1)) {
-                        tc::tc_fence_after();
-                        const int slot = cgi % kSlots;
-                        const uint32_t dcol = tmem + slot * kSlotCols + kNC;
-                        const uint32_t sb_addr = sbase + kSmS + sb * kSBytes;
-                        for (int ks = 0; ks < kKS / 16; ++ks)
-                            tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmCA + ks * 256, 128, kKS * 16),
-                                         tc::smem_desc_sw128(sb_addr + ks * 2048, kKS * 128, 1024), idesc, ks > 0);
-                        tc::mma_commit(bar(kBarYDone + slot));
-                        tc::mma_commit(bar(kBarSTFree + sb));
-                        ++pc;
-                        if (++jn == c_nck) { jn = 0; ++chead; }
-                        progressed = true;
-                    }
-                }
-                // constants of a new head, once no issued or pending MMA uses the old ones (rare:
-                // a CTA keeps to one head until its items run out)
-                if (need_const && chead == ctail - 1) {
+            int c2cnt[kSlots];              // per-slot full-pass uses (const switches only)
+#pragma unroll
+            for (int i = 0; i < kSlots; ++i) c2cnt[i] = 0;
+            bool any = false, ok = true;
+            for (int k = 0; ok; ++k) {
+                const int id = take_item(k, false);
+                if (id == -2) { ok = false; break; }
+                if (id < 0) break;
+                const Item it = decode_item<NC>(a, id);
+                if (it.hd != cur_hd) {
+                    // constants of a new head (rare: a CTA keeps to one head until its items run
+                    // out).  No MMA may still read the old ones: every carry issued so far must be
+                    // issued and finished (each slot then has at most one carry outstanding, so
+                    // its last completion is unambiguous), and so must this thread's own MMAs.
                     if (any) {
+                        const unsigned long long t0 = tc::global_ns();
+                        while (*carry_issued < pcf && !*abort && tc::global_ns() - t0 < tc::kWaitNs) {}
+                        if (*carry_issued < pcf) { ok = false; break; }
+#pragma unroll
+                        for (int sl = 0; sl < kSlots; ++sl)
+                            if (c2cnt[sl] > 0 && !tc::mbar_wait(bar(kBarYDone + sl), (c2cnt[sl] - 1) & 1, abort)) ok = false;
+                        if (!ok) break;
                         tc::mma_commit(bar(kBarConstFree));
                         if (!tc::mbar_wait(bar(kBarConstFree), fphase & 1, abort)) { ok = false; break; }
                         ++fphase;
                     }
                     tc::mbar_expect_tx(bar(kBarConst), kOpBytes);
-                    tc::bulk_load(sbase + kSmFA, a.consts + (size_t)fi.hd * kConstStride, kOpBytes, bar(kBarConst));
+                    tc::bulk_load(sbase + kSmFA, a.consts + (size_t)it.hd * kConstStride, kOpBytes, bar(kBarConst));
                     if (!tc::mbar_wait(bar(kBarConst), cphase & 1, never)) { ok = false; break; }
                     ++cphase;
-                    cur_hd = fi.hd;
-                    need_const = false;
-                    progressed = true;
+                    cur_hd = it.hd;
                 }
-                // fused stream: [Z; W] = [T; V] U
-                if (f_valid && !need_const) {
+                for (int i = 0; i < it.niter; ++i, ++g) {
                     const int slot = g % kSlots, st = g % kKVStages;
-                    if (tc::mbar_test(bar(kBarURdy + st), (g / kKVStages) & 1) &&
-                        tc::mbar_test(bar(kBarD2Free + slot), ((g / kSlots) & 1) ^ 1) &&
-                        tc::mbar_test(bar(kBarD1Free + slot), ((c2bits >> slot) & 1) ^ 1)) {
-                        tc::tc_fence_after();
-                        const uint32_t dcol = tmem + slot * kSlotCols;
-                        const uint32_t u_addr = sbase + kSmKV + st * kStageBytes;
-                        for (int ks = 0; ks < kC / 16; ++ks)
-                            tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmFA + ks * 256, 128, kC * 16),
-                                         tc::smem_desc_sw128(u_addr + ks * 2048, kAtom, 1024), idesc, ks > 0);
-                        tc::mma_commit(bar(kBarWDone + slot));
-                        tc::mma_commit(bar(kBarKVEmpty + st));
-                        if (ic >= fi.n1) c2bits ^= 1 << slot;
-                        ++g;
-                        any = true;
-                        progressed = true;
-                        if (++ic == fi.niter) f_valid = false;
-                    }
-                }
-                if (done && !f_valid && chead == ctail) break;
-                if (progressed) {
-                    t_prog = tc::global_ns();
-                } else {
-                    if (tc::global_ns() - t_prog > tc::kWaitNs) {
+                    if (!tc::mbar_wait(bar(kBarURdy + st), (g / kKVStages) & 1, abort) ||
+                        !tc::mbar_wait(bar(kBarD2Free + slot), ((g / kSlots) & 1) ^ 1, abort) ||
+                        !tc::mbar_wait(bar(kBarD1Free + slot), ((c2bits >> slot) & 1) ^ 1, abort)) {
                         ok = false;
                         break;
                     }
-                    __nanosleep(20);
+                    tc::tc_fence_after();
+                    const uint32_t dcol = tmem + slot * kSlotCols;
+                    const uint32_t u_addr = sbase + kSmKV + st * kStageBytes;
+#pragma unroll
+                    for (int ks = 0; ks < kC / 16; ++ks)
+                        tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmFA + ks * 256, 128, kC * 16),
+                                     tc::smem_desc_sw128(u_addr + ks * 2048, kAtom, 1024), idesc, ks > 0);
+                    tc::mma_commit(bar(kBarWDone + slot));
+                    tc::mma_commit(bar(kBarKVEmpty + st));
+                    if (i >= it.n1) {
+                        c2bits ^= 1 << slot;
+                        ++c2cnt[slot];
+                        ++pcf;
+                    }
+                    any = true;
                 }
             }
             if (*abort) ok = false;
@@ -663,9 +622,48 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             tc::mma_commit(bar(kBarDrain));
             tc::mbar_wait(bar(kBarDrain), 0, never);
         }
+    } else if (warp == kWarpCarry) {
+        // ------------------------------------------------------------ carry issuer
+        // Z += A S for every full-pass chunk, in order, once the S group has written the state
+        // entering the chunk and the chunk's fused product has finished (which also means the
+        // slot's previous contents were read out).
+        if (lane == 0) {
+            const uint32_t idesc = tc::idesc_bf16(128, kNC, true);
+            int g = 0, pc = 0;
+            bool ok = true;
+            for (int k = 0; ok; ++k) {
+                const int id = take_item(k, false);
+                if (id == -2) { ok = false; break; }
+                if (id < 0) break;
+                const Item it = decode_item<NC>(a, id);
+                g += it.n1;
+                for (int j = 0; j < it.nck; ++j, ++g, ++pc) {
+                    const int slot = g % kSlots, sb = pc % kSBufs;
+                    if (!tc::mbar_wait(bar(kBarSRdy + sb), (pc / kSBufs) & 1, abort) ||
+                        !tc::mbar_wait(bar(kBarWDone + slot), (g / kSlots) & 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::tc_fence_after();
+                    const uint32_t dcol = tmem + slot * kSlotCols + kNC;
+                    const uint32_t sb_addr = sbase + kSmS + sb * kSBytes;
+#pragma unroll
+                    for (int ks = 0; ks < kKS / 16; ++ks)
+                        tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmCA + ks * 256, 128, kKS * 16),
+                                     tc::smem_desc_sw128(sb_addr + ks * 2048, kKS * 128, 1024), idesc, ks > 0);
+                    tc::mma_commit(bar(kBarYDone + slot));
+                    tc::mma_commit(bar(kBarSTFree + sb));
+                    *carry_issued = pc + 1;
+                }
+            }
+            if (*abort) ok = false;
+            if (!ok) record_error(a, abort, kErrWait);
+            tc::mma_commit(bar(kBarDrainC));
+            tc::mbar_wait(bar(kBarDrainC), 0, never);
+        }
     } else if (u_index(warp) >= 0) {
         // ------------------------------------------------------------ U group: U = k v in place
-        const int ut = u_index(warp) * 32 + lane;
+        const int ut = u_index(warp) * 32 + lane;       // 0 .. kUThreads - 1
         int g = 0;
         bool ok = true;
         for (int k = 0; ok; ++k) {
@@ -677,9 +675,9 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int st = g % kKVStages;
                 if (!(ok = uni(tc::mbar_wait(bar(kBarKVFull + st), (g / kKVStages) & 1, abort)))) break;
                 uint8_t *kt = sm + kSmKV + st * kStageBytes;
-#pragma unroll
-                for (int m = 0; m < kTile / 16 / 128; ++m) {
-                    const int off = (ut + 128 * m) * 16;    // same byte offset in k, v and U
+#pragma unroll 4
+                for (int c16 = ut; c16 < kTile / 16; c16 += kUThreads) {
+                    const int off = c16 * 16;               // same byte offset in k, v and U
                     const uint4 kk = *reinterpret_cast<const uint4 *>(kt + off);
                     const uint4 vv = *reinterpret_cast<const uint4 *>(kt + kTile + off);
                     uint4 uu;
@@ -884,6 +882,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             for (int j = 0; j < it.nck; ++j, ++g, ++qg) {
                 const int slot = g % kSlots, s = qg % kQStages;
                 ok = uni(tc::mbar_wait(bar(kBarYDone + slot), (e2bits >> slot) & 1, abort) &&
+                         tc::mbar_wait(bar(kBarWDone + slot), (g / kSlots) & 1, abort) &&
                          tc::mbar_wait(bar(kBarQFull + s), (qg / kQStages) & 1, abort));
                 if (!ok) break;
                 e2bits ^= 1 << slot;
