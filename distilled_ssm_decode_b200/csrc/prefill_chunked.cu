@@ -264,7 +264,9 @@ __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x <<
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
 // ------------------------------------------------------------------ per-head constants
-// One block per head.  Every entry is a power lambda_n^k with 0 <= k <= C, so the powers are
+// Blocks (head, part): every block of a head tabulates the head's powers and taps, and writes
+// its part of the operand rows (part 0 also the chain powers).  Every entry is a power
+// lambda_n^k with 0 <= k <= C, so the powers are
 // tabulated first (each by binary powering, all in parallel) and the operands are then filled
 // from the table.  fp32 suffices: the operands are rounded to bf16 (relative 2^-9) and the
 // chain powers lambda^C, lambda^Lseg enter an fp32 recurrence, while binary powering to an
@@ -279,10 +281,19 @@ __device__ __forceinline__ float2 cfpow(float2 lam, long long m) {
     return r;
 }
 
+// It also clears the main kernel's schedule words (`zero`, `nzero` ints: error word, ticket
+// counters, segment status words), and lets the main kernel launch at once (programmatic
+// dependent launch): the main kernel's prologue overlaps this kernel, and its
+// griddepcontrol.wait returns once everything written here is visible.
 __global__ void __launch_bounds__(256)
 chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R,
                     const float *__restrict__ Dskip, int d, int seg_tokens,
-                    uint8_t *__restrict__ consts) {
+                    uint8_t *__restrict__ consts, int *__restrict__ zero, int nzero) {
+    asm volatile("griddepcontrol.launch_dependents;");
+    const int part = blockIdx.y, nparts = gridDim.y;
+    for (int i = (blockIdx.y * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x; i < nzero;
+         i += gridDim.x * gridDim.y * blockDim.x)
+        zero[i] = 0;
     const int hd = blockIdx.x;
     uint8_t *base = consts + (size_t)hd * kConstStride;
     __nv_bfloat16 *FA = reinterpret_cast<__nv_bfloat16 *>(base);
@@ -306,8 +317,9 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
         const int n = e / (kC + 1), k = e % (kC + 1);
         pw[n][k] = n < d ? cfpow(ls[n], k) : make_float2(0.f, 0.f);
     }
-    for (int n = threadIdx.x; n < kMaxModes; n += blockDim.x)
-        lamS[n] = n < d ? cfpow(ls[n], seg_tokens) : make_float2(0.f, 0.f);
+    if (part == 0)
+        for (int n = threadIdx.x; n < kMaxModes; n += blockDim.x)
+            lamS[n] = n < d ? cfpow(ls[n], seg_tokens) : make_float2(0.f, 0.f);
     __syncthreads();
     for (int j = threadIdx.x; j < kC; j += blockDim.x) {
         float acc = 0.f;
@@ -318,12 +330,13 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
         }
         hs[j] = acc;
     }
-    for (int n = threadIdx.x; n < kMaxModes; n += blockDim.x) lamC[n] = pw[n][kC];
+    if (part == 0)
+        for (int n = threadIdx.x; n < kMaxModes; n += blockDim.x) lamC[n] = pw[n][kC];
     __syncthreads();
     // fused A operand: rows 0..C-1 Toeplitz taps, rows C..C+31 chunk powers (Re at r < 16, Im at
     // 16 + n), rows C+32..127 zero
     // (each thread writes one 16-byte core-matrix row: 8 consecutive K entries of one row)
-    for (int e = threadIdx.x; e < 128 * (kC / 8); e += blockDim.x) {
+    for (int e = part * blockDim.x + threadIdx.x; e < 128 * (kC / 8); e += nparts * blockDim.x) {
         const int row = e / (kC / 8), io0 = 8 * (e % (kC / 8));
         float v[8];
 #pragma unroll
@@ -342,7 +355,7 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
             make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
     }
     // carry A operand: rows 0..C-1: (Re, -Im) of R_n lambda_n^tau; rows C..127 zero
-    for (int e = threadIdx.x; e < 128 * (kKS / 8); e += blockDim.x) {
+    for (int e = part * blockDim.x + threadIdx.x; e < 128 * (kKS / 8); e += nparts * blockDim.x) {
         const int row = e / (kKS / 8), r0 = 8 * (e % (kKS / 8));
         float v[8];
 #pragma unroll
@@ -392,7 +405,6 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     auto bar = [&](int slot) { return sbase + kSmBar + 8u * slot; };
     volatile int *itemq = reinterpret_cast<volatile int *>(sm + kSmMisc);   // [kItemQ]
     volatile int *misc = itemq + kItemQ;                                     // abort, tmem, never
-    int *cqueue = const_cast<int *>(misc) + 4;                               // [kCQ][3]: n1, nck, g0
     volatile int *pubq = misc + 4 + 3 * kCQ;                                 // [kPubQ]: 4 item + code, -1 = end
     volatile int *carry_issued = pubq + kPubQ;                               // carries issued so far
     volatile int *abort = misc;
@@ -404,6 +416,11 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         *carry_issued = 0;
         for (int i = 0; i < kNumBars; ++i) tc::mbar_init(bar(i), G::count(i));
         tc::fence_mbar_init();
+    } else if (tid == 32) {
+        tc::prefetch_tensormap(&tm_q);
+        tc::prefetch_tensormap(&tm_k);
+        tc::prefetch_tensormap(&tm_v);
+        tc::prefetch_tensormap(&tm_y);
     }
     if (warp == kWarpMMA) {
         tc::tmem_alloc(tc::smem_u32((const void *)(misc + 1)), kTmemCols);
@@ -412,6 +429,30 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
+    // launched as a programmatic dependent of the constants kernel: the set-up above overlapped
+    // it, and so do L2 prefetches of the first tiles of the item this CTA will most likely take
+    // first (the ticket blockIdx / H of head blockIdx % H; a prefetch has no effect on results,
+    // so a wrong guess costs nothing but bandwidth).  The constants and the cleared schedule
+    // words are visible after the wait.
+    if ((warp == kWarpKV || warp == kWarpQ) && lane == 0 && (int)blockIdx.x / a.H < a.ih) {
+        const Item it = decode_item<NC>(a, (blockIdx.x % a.H) * a.ih + blockIdx.x / a.H);
+        const bool kv = warp == kWarpKV;
+        const int n = kv ? min(it.niter, kKVStages) : min(it.nck, kQStages);
+        for (int i = 0; i < n; ++i) {
+            const int chunk = it.ck0 + (kv && i < it.n1 ? i : (kv ? i - it.n1 : i));
+            const int tok = a.tok_base + chunk * kC;
+            if (tok < 0) continue;
+            for (int h = 0; h < kNC / 64; ++h) {
+                if (kv) {
+                    tc::tma_prefetch_3d(&tm_k, it.c0 + 64 * h, tok, it.b);
+                    tc::tma_prefetch_3d(&tm_v, it.c0 + 64 * h, tok, it.b);
+                } else {
+                    tc::tma_prefetch_3d(&tm_q, it.c0 + 64 * h, tok, it.b);
+                }
+            }
+        }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint32_t tmem = (uint32_t)misc[1];
     const int d = a.d;
     auto uni = [&](bool x) -> bool { return __all_sync(0xffffffffu, x && !*abort); };
@@ -508,7 +549,10 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     } else if (warp == kWarpStore) {
         // ------------------------------------------------------------ y stores
         if (lane == 0) {
-            int qg = 0;
+            // each chunk's stores form one bulk group (empty for a chunk that starts before token 0,
+            // whose rows the E group wrote directly); a staging buffer goes back to the q loader
+            // once its group has been read, checked one chunk later so that two stores overlap
+            int qg = 0, prev = -1;
             bool ok = true;
             for (int k = 0; ok; ++k) {
                 const int id = take_item(k, false);
@@ -522,15 +566,17 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         break;
                     }
                     const int tok = tok_of(it.ck0 + j);
-                    if (tok >= 0) {     // a chunk that starts before token 0 was written by the E group
+                    if (tok >= 0)
                         for (int h = 0; h < kNC / 64; ++h)
                             tc::tma_store_3d(&tm_y, sbase + kSmQ + s * kTile + h * kAtom, it.c0 + 64 * h, tok, it.b);
-                        tc::bulk_commit();
-                        tc::bulk_wait_read<0>();
-                    }
-                    tc::mbar_arrive(bar(kBarQEmpty + s));
+                    tc::bulk_commit();
+                    tc::bulk_wait_read<1>();        // every group but this one has been read
+                    if (prev >= 0) tc::mbar_arrive(bar(kBarQEmpty + prev));
+                    prev = s;
                 }
             }
+            tc::bulk_wait_read<0>();
+            if (prev >= 0) tc::mbar_arrive(bar(kBarQEmpty + prev));
             if (!ok) record_error(a, abort, kErrWait);
             tc::bulk_wait<0>();     // every store of this CTA has completed
         } else if (lane == 1) {
@@ -965,7 +1011,8 @@ struct ChunkPlan {
 
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 
-constexpr int kPlanSMs = 148;   // the plan is made for a full B200 (any SM count runs correctly)
+constexpr int kPlanSMs = 148;
+constexpr int kConstParts = 4;  // blocks per head of the constants kernel   // the plan is made for a full B200 (any SM count runs correctly)
 
 // Channel tile and segment count.  Costs are in units of one 128-channel chunk pass: a pass of
 // an NC-channel tile costs NC/128 plus a fixed 0.1, an item 1 more, and 6 more when its sequence
@@ -1041,7 +1088,18 @@ cudaError_t launch_tile(const CUtensorMap &mq, const CUtensorMap &mk, const CUte
     cudaError_t e = cudaFuncSetAttribute(prefill_chunk_kernel<NC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int grid = items < sm_count() ? items : sm_count();
-    prefill_chunk_kernel<NC><<<grid, kThreads, smem, s>>>(mq, mk, mv, my, a);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, prefill_chunk_kernel<NC>, mq, mk, mv, my, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 }  // namespace
@@ -1052,10 +1110,10 @@ cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, 
     const ChunkPlan p = plan(B, L, Dch, H);
     uint8_t *w = static_cast<uint8_t *>(ws);
 
-    cudaError_t e = cudaMemsetAsync(w + p.sched_off, 0, p.agg_off - p.sched_off, s);
+    chunk_consts_kernel<<<dim3(H, kConstParts), 256, 0, s>>>(lam, R, Dskip, d, p.segc * kC, w + p.consts_off,
+                                          reinterpret_cast<int *>(w + p.sched_off), (int)((p.agg_off - p.sched_off) / 4));
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    chunk_consts_kernel<<<H, 256, 0, s>>>(lam, R, Dskip, d, p.segc * kC, w + p.consts_off);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     CUtensorMap mq, mk, mv, my;
     if (!make_map(&mq, q, B, L, Dch) || !make_map(&mk, k, B, L, Dch) || !make_map(&mv, v, B, L, Dch) ||
         !make_map(&my, y, B, L, Dch))
