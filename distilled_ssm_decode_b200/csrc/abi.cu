@@ -238,4 +238,29 @@ int hyena_decode_step(const void *q, const void *k, const void *v, int dtype, in
                                           (cudaStream_t)stream));
 }
 
+int hyena_decode_step_layers(int layers, const void *const *q, const void *const *k, const void *const *v,
+                             int dtype, int B, int Dch, int H, int d, const float *const *lambda,
+                             const float *const *R, const float *const *Dskip, float *const *state,
+                             void *const *y, hyena_stream_t stream) {
+    if (dtype != HYENA_F32 && dtype != HYENA_BF16) return HYENA_ERR_ARG;
+    if (B < 0 || layers < 0) return HYENA_ERR_SHAPE;
+    if (layers > HYENA_MAX_LAYERS) return HYENA_ERR_UNSUPPORTED;
+    int st = check_common(H, d, Dch);
+    if (st != HYENA_OK) return st;
+    if (layers == 0 || B == 0 || Dch == 0) return HYENA_OK;
+    if (!q || !k || !v || !y || !state || !lambda || !R || !Dskip) return HYENA_ERR_ARG;
+    if (!decode_layers_vec_ok(Dch, H)) return HYENA_ERR_UNSUPPORTED;
+    const size_t ab = (dtype == HYENA_BF16) ? 2 : 4;
+    for (int i = 0; i < layers; ++i) {
+        if (!q[i] || !k[i] || !v[i] || !y[i] || !state[i] || !lambda[i] || !R[i] || !Dskip[i])
+            return HYENA_ERR_ARG;
+        if (!aligned(q[i], 2 * ab) || !aligned(k[i], 2 * ab) || !aligned(v[i], 2 * ab) ||
+            !aligned(y[i], 2 * ab) || !aligned(state[i], 16) || !aligned(lambda[i], 8) ||
+            !aligned(R[i], 8) || !aligned(Dskip[i], 4))
+            return HYENA_ERR_ALIGN;
+    }
+    return cuda_status(launch_decode_layers(layers, q, k, v, dtype, B, Dch, H, d, lambda, R, Dskip, state, y,
+                                            (cudaStream_t)stream));
+}
+
 }  // extern "C"

@@ -53,5 +53,12 @@ cudaError_t launch_prompt_state(const void *k, const void *v, int dtype, int B, 
 cudaError_t launch_decode_step(const void *q, const void *k, const void *v, int dtype,
                                int B, int Dch, int H, int d, const float2 *lam, const float2 *R,
                                const float *Dskip, float *state, void *y, cudaStream_t s);
+// grouped step of `layers` independent layers (host arrays of device pointers); requires the
+// paired-channel layout (decode_layers_vec_ok) and aligned pointers, checked by the caller
+bool decode_layers_vec_ok(int Dch, int H);
+cudaError_t launch_decode_layers(int layers, const void *const *q, const void *const *k, const void *const *v,
+                                 int dtype, int B, int Dch, int H, int d, const float *const *lam,
+                                 const float *const *R, const float *const *Dskip, float *const *state,
+                                 void *const *y, cudaStream_t s);
 
 }  // namespace hyena

@@ -44,6 +44,8 @@ SIGNATURES = {
     "hyena_prompt_state_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "hyena_prompt_state": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _fp, _fp, _vp, _sz, _vp]),
     "hyena_decode_step": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _fp, _fp, _fp, _fp, _vp, _vp]),
+    "hyena_decode_step_layers": (_i, [_i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
+                                      _vp]),
 }
 
 
@@ -228,3 +230,50 @@ def decode_step(q, k, v, lam, R, Dskip, state, y=None):
            lib().hyena_decode_step(_ptr(q), _ptr(k), _ptr(v), dt, B, Dch, H, d, _ptr(lam), _ptr(R),
                                    _ptr(Dskip), _ptr(state), _ptr(y), _stream(q.device)))
     return y
+
+
+class LayerSet:
+    """Host pointer arrays of a fixed set of layers for decode_step_layers (built once, reused
+    every step so that a step costs one library call)."""
+
+    def __init__(self, lams, Rs, Dskips, states):
+        n = len(lams)
+        if not (len(Rs) == len(Dskips) == len(states) == n):
+            raise ValueError("one lam, R, Dskip and state per layer")
+        ps = [_params(l, r, dk) for l, r, dk in zip(lams, Rs, Dskips)]
+        self.H, self.d = ps[0][0].shape[0], ps[0][0].shape[1]
+        if any(p[0].shape != ps[0][0].shape for p in ps):
+            raise ValueError("all layers need the same H and d")
+        self.states = [_cuda(s, "state", torch.float32) for s in states]
+        self.n = n
+        arr = ctypes.c_void_p * max(n, 1)
+        self._keep = ps
+        self.lam = arr(*[p[0].data_ptr() for p in ps])
+        self.R = arr(*[p[1].data_ptr() for p in ps])
+        self.Dskip = arr(*[p[2].data_ptr() for p in ps])
+        self.state = arr(*[s.data_ptr() for s in self.states])
+
+
+def decode_step_layers(layers: LayerSet, qs, ks, vs, ys):
+    """One decode step of every layer in one launch: qs[i], ks[i], vs[i], ys[i] [B][Dch] for
+    layer i; each layer's state is updated in place.  qs..ys are sequences of tensors, or
+    [layers][B][Dch] tensors."""
+    n = layers.n
+    arr = ctypes.c_void_p * max(n, 1)
+    q0 = _cuda(qs[0], "q")
+    dt = _act_dtype(q0)
+    B, Dch = q0.shape
+    for name, ts in (("q", qs), ("k", ks), ("v", vs), ("y", ys)):
+        if len(ts) != n:
+            raise ValueError(f"{name}: one tensor per layer")
+        for t in ts:
+            _cuda(t, name, q0.dtype)
+            if tuple(t.shape) != (B, Dch):
+                raise ValueError(f"{name}: every layer's tensor must be [B][Dch]")
+    pq, pk, pv, py = (arr(*[t.data_ptr() for t in ts]) for ts in (qs, ks, vs, ys))
+    _check("hyena_decode_step_layers",
+           lib().hyena_decode_step_layers(n, pq, pk, pv, dt, B, Dch, layers.H, layers.d, layers.lam,
+                                          layers.R, layers.Dskip, layers.state, py,
+                                          _stream(q0.device)))
+    return ys
+

@@ -228,6 +228,35 @@ int hyena_decode_step(const void *q, const void *k, const void *v, int dtype,
                       const float *lambda, const float *R, const float *Dskip,
                       float *state, void *y, hyena_stream_t stream);
 
+/* Largest number of layers one hyena_decode_step_layers call takes. */
+#define HYENA_MAX_LAYERS 64
+
+/*
+ * One decode step (as hyena_decode_step) for `layers` independent operator
+ * layers in a single launch, e.g. the 24 operator layers of a 1.3B-shaped
+ * generation workload, whose tokens all advance by one at a time.  Layer i
+ * has its own activations q[i], k[i], v[i], y[i] ([B][Dch], dtype), state[i]
+ * ([B][d][Dch][2] fp32, updated in place) and modal parameters lambda[i],
+ * R[i] ([H][d][2] fp32) and Dskip[i] ([H] fp32); B, Dch, H, d and dtype are
+ * shared.  Each layer's results are those of hyena_decode_step on the same
+ * arguments (up to the summation order of Re sum_n R_n s_n).  Per step this
+ * is the O(d) recurrence of the distilled modal SSM ("Laughing Hyena
+ * Distillery", nubint.ai review, "Main findings"), applied layer by layer.
+ *   q, k, v, y, state, lambda, R, Dskip: HOST arrays of `layers` device
+ *   pointers each (read during the call only; the pointers travel to the
+ *   kernel by value, so a captured CUDA graph keeps them).
+ *   0 <= layers <= HYENA_MAX_LAYERS (HYENA_ERR_UNSUPPORTED above).
+ *   Implemented for Dch and Dch/H even (HYENA_ERR_UNSUPPORTED otherwise);
+ *   every state pointer 16-byte aligned and every activation pointer aligned
+ *   to two elements (HYENA_ERR_ALIGN otherwise).  Layers must not share state
+ *   or output buffers.
+ */
+int hyena_decode_step_layers(int layers, const void *const *q, const void *const *k,
+                             const void *const *v, int dtype, int B, int Dch, int H, int d,
+                             const float *const *lambda, const float *const *R,
+                             const float *const *Dskip, float *const *state, void *const *y,
+                             hyena_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

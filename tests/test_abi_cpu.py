@@ -132,3 +132,25 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(ops, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         ops.lib()
+
+
+def test_decode_layers_validation(lib):
+    arr = ctypes.c_void_p * 2
+    good = arr(FAKE, FAKE)
+    mis = arr(FAKE + 8, FAKE)          # state pointer not 16-byte aligned
+
+    def call(layers=2, dtype=1, B=2, Dch=8, H=2, d=4, st=good, q=good):
+        return lib.hyena_decode_step_layers(layers, q, good, good, dtype, B, Dch, H, d, good, good, good,
+                                            st, good, None)
+    assert call(dtype=7) == ERR_ARG
+    assert call(layers=-1) == ERR_SHAPE
+    assert call(layers=65) == ERR_UNSUP
+    assert call(Dch=9, H=3) == ERR_UNSUP       # odd channel count: no channel pairs
+    assert call(Dch=6, H=2) == ERR_UNSUP       # odd channels per head
+    assert call(d=0) == ERR_SHAPE
+    assert call(st=mis) == ERR_ALIGN
+    assert call(q=arr(FAKE + 2, FAKE)) == ERR_ALIGN
+    assert call(layers=0) == OK                # nothing to do, nothing enqueued
+    assert call(B=0) == OK
+    assert lib.hyena_decode_step_layers(2, None, good, good, 1, 2, 8, 2, 4, good, good, good, good, good,
+                                        None) == ERR_ARG
