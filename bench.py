@@ -241,15 +241,17 @@ def run_reference(args):
         dt, t = sample.run_reps(channels, reps)
         total += dt
         tok += t
-    value = tok / total
+    nl = args.layers or w.layers
+    value = tok / total / nl
     cores = oracle.threads()
     desc = (f"fp64 oracle, recurrent mode: all {w.B} sequences x first {channels} of {w.Dch} "
-            f"channels, {w.L}-token prompt + {w.T} decode tokens, {reps} pass(es) per step")
+            f"channels, {w.L}-token prompt + {w.T} decode tokens, {reps} pass(es) per step"
+            + (f"; layer 0 only, tokens/s divided by {nl} layers" if nl > 1 else ""))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(w),
+            "config": dict(workload_config(w), **({"layers": nl} if nl > 1 else {})),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -515,6 +517,152 @@ def run_ours(args):
     return 0
 
 
+def run_layers(args, nl: int):
+    """Every layer of a multi-layer workload: per bench step, the chunked prefill of each layer's
+    prompt, then T decode steps, each one grouped launch over all layers (CUDA graph).  Inputs
+    are drawn on the device (seeded); each layer has its own parameters, state and activations."""
+    import torch
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init("nccl")
+    from distilled_ssm_decode_b200 import build, ops
+    from distilled_ssm_decode_b200 import workloads as W
+    build.build()
+    ops.lib()
+    w = W.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.with_(B=args.batch)
+    if ops.lib().hyena_prefill_chunked_workspace_bytes(w.B, w.L, w.Dch, w.H, w.d) == 0:
+        raise SystemExit(f"chunked prefill does not support workload {w.name}")
+    ps = [W.params(w, layer=l) for l in range(nl)]
+    lams = [p.lam_f32().to(dev) for p in ps]
+    Rs = [p.R_f32().to(dev) for p in ps]
+    Ds = [p.Dskip_f32().to(dev) for p in ps]
+    states = [torch.empty((w.B, w.d, w.Dch, 2), dtype=torch.float32, device=dev) for _ in range(nl)]
+    qkv = [W.prefill_inputs_device(w, l, device=dev) for l in range(nl)]
+    ys = [torch.empty_like(x[0]) for x in qkv]
+    ws = torch.empty(ops.prefill_chunked_workspace_bytes(w.B, w.L, w.Dch, w.H, w.d), dtype=torch.uint8,
+                     device=dev)
+    pool = 8
+    dpool = [W.decode_pool_device(w, pool, device=dev, layer=l) for l in range(nl)]
+    ydec = torch.empty((w.T, nl, w.B, w.Dch), dtype=w.torch_dtype, device=dev)
+    ls = ops.LayerSet(lams, Rs, Ds, states)
+    stream = torch.cuda.Stream(dev)
+
+    def prefill_all():
+        for l in range(nl):
+            q, k, v = qkv[l]
+            ops.prefill_chunked(q, k, v, lams[l], Rs[l], Ds[l], y=ys[l], state=states[l], workspace=ws)
+
+    def decode_all():
+        for t in range(w.T):
+            i = t % pool
+            ops.decode_step_layers(ls, [dpool[l][0][i] for l in range(nl)], [dpool[l][1][i] for l in range(nl)],
+                                   [dpool[l][2][i] for l in range(nl)], [ydec[t][l] for l in range(nl)])
+
+    with torch.cuda.stream(stream):
+        prefill_all()
+        decode_all()
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        decode_all()
+    torch.cuda.synchronize(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        prefill_all()
+        if ev is not None:
+            ev[1].record(stream)
+        g.replay()
+        if ev is not None:
+            ev[2].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(gpu_id_for(dev))
+    clocks.start()
+    time.sleep(0.3)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    clk = clocks.stop()
+    elapsed_ms = reduce_max(t_start.elapsed_time(t_end), dev)
+    pre_ms = reduce_max(sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps, dev)
+    dec_ms = reduce_max(sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps, dev)
+    ms_per_step = elapsed_ms / args.steps
+    err = ops.chunked_error(ws, w.B, w.L, w.Dch, w.H, w.d)
+    if err:
+        raise SystemExit(f"chunked prefill kernel reported error {err}")
+
+    peak, peak_src = load_peaks()
+    pb, db = algorithmic_bytes(w)
+    pb, db = pb * nl, db * nl
+    pre_gbs = pb / (pre_ms / 1e3) / 1e9
+    dec_launch_ms = dec_ms / w.T
+    dec_gbs = db / (dec_launch_ms / 1e3) / 1e9
+    roofs = [{"kernel": f"hyena_prefill_chunked x {nl} layers", "bound": "hbm", "achieved": pre_gbs,
+              "peak": peak, "unit": "GB/s", "frac": pre_gbs / peak, "peak_source": peak_src,
+              "algorithmic_bytes": pb, "launch_ms": pre_ms / nl, "total_ms": pre_ms,
+              "traffic": ncu_traffic("prefill_chunk", f"{w.name}/B{w.B}")},
+             {"kernel": f"hyena_decode_step_layers ({nl} layers per launch)", "bound": "hbm",
+              "achieved": dec_gbs, "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak,
+              "peak_source": peak_src, "algorithmic_bytes": db, "launch_ms": dec_launch_ms,
+              "total_ms": dec_ms, "traffic": ncu_traffic("decode_layers", f"{w.name}/B{w.B}")}]
+    dominant = max(roofs, key=lambda r: r["total_ms"])
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        sample = OracleSample(w)
+        channels, reps = sample.calibrate(12.0)
+        dt, tok = sample.run_reps(channels, reps)
+        cpu = {"value": tok / dt / nl, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+               "sample": (f"fp64 oracle, recurrent mode, layer 0 only: {reps} pass(es) over all {w.B} "
+                          f"sequences x first {channels} of {w.Dch} channels ({w.L}-token prompt + {w.T} "
+                          f"decode tokens), {dt:.1f} s; tokens/s of one layer divided by {nl} layers")}
+    if rank == 0:
+        cfg = workload_config(w)
+        cfg["layers"] = nl
+        cfg["workload"] += f", {nl} independent layers (all timed)"
+        cfg["prefill_route"] = "chunked"
+        cfg["l2"] = ("prefill inputs larger than L2 (3 x %d MiB per layer); decode states %d MiB in total"
+                     % (qkv[0][0].numel() * 2 >> 20, nl * states[0].numel() * 4 >> 20))
+        cfg["decode_inputs"] = f"{pool} distinct device-drawn input sets per layer, cycled"
+        tokens_step = w.B * (w.L + w.T)
+        line = {"metric": METRIC, "value": world * tokens_step / (ms_per_step / 1e3), "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic (device-drawn, seeded)",
+                "config": cfg,
+                "prefill": {"tokens_per_s": world * w.B * w.L / (pre_ms / 1e3), "ms": pre_ms,
+                            "hbm_frac": pre_gbs / peak},
+                "decode": {"tokens_per_s": world * w.B * w.T / (dec_ms / 1e3),
+                           "ms_per_token_step": dec_launch_ms, "hbm_frac": dec_gbs / peak},
+                "roofline": dominant, "roofline_all": roofs, "cpu_baseline": cpu,
+                "e2e": None, "e2e_note": "not measured for the multi-layer workload (9.6 GB of prompt per step)",
+                "gpu_launches": args.steps * (2 * nl + w.T), "clocks": clk}
+        print(json.dumps(line), flush=True)
+    del g
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -529,10 +677,16 @@ def main(argv=None):
                     help="skip the extra timing of the FFT route when the chunked route is used")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="layers of a multi-layer workload to run (default: all; 1 = one layer)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)   # at least 3 untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
+    from distilled_ssm_decode_b200 import workloads as W
+    nl = args.layers or W.WORKLOADS[args.workload].layers
+    if nl > 1:
+        return run_layers(args, nl)
     return run_ours(args)
 
 

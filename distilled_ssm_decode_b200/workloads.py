@@ -173,6 +173,19 @@ def decode_pool_device(w: Workload, pool: int, B: Optional[int] = None, device="
     return tuple(out)
 
 
+def prefill_inputs_device(w: Workload, layer: int = 0, device="cuda"):
+    """q, k, v [B][L][Dch] drawn N(0, 1) on the device by torch's seeded generator (for
+    benchmarking many layers, whose host-drawn inputs would take minutes); parity tests use
+    prefill_inputs()."""
+    g = torch.Generator(device=device)
+    out = []
+    for tid in (T_Q, T_K, T_V):
+        g.manual_seed(_seed(w, layer, tid))
+        x = torch.randn((w.B, w.L, w.Dch), generator=g, device=device, dtype=torch.float32)
+        out.append(x.to(w.torch_dtype))
+    return tuple(out)
+
+
 def to_f64(t: torch.Tensor) -> np.ndarray:
     """Exact widening of a CPU tensor (fp32 / bf16 / complex64) to numpy float64/complex128."""
     if t.is_complex():
