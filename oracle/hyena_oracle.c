@@ -27,7 +27,7 @@
  *   and the state that a length-L prompt leaves behind:
  *       s_n = sum_{j<L} lambda_n^(L-1-j) u_j
  *
- * Readings taken where the pages are silent (each listed in the design doc):
+ * Readings taken where the pages are silent:
  *   - channel c belongs to head c / (Dch / H) (contiguous heads);
  *   - decode emits y_t from the state *before* the update, then updates: the
  *     only order under which prompt state + decode equals the full convolution;
