@@ -269,6 +269,52 @@ def workload_config(w):
 
 
 
+def fir_baseline(ops, W, w, q, k, v, dq, dk, dv, lam, R, D, stream, dev, nsteps, modal_step_ms,
+                 prefill_ms, peak, layers=1):
+    """Generation without the distilled recurrence, on the same inputs: each token convolves the
+    cached history with the long filter (O(t) per token).  Times `nsteps` tokens after the
+    prompt (CUDA graph; `layers` launches per token over one shared history, so every launch
+    streams it from DRAM like a layer of its own would); the re-prefill cost per token is at
+    least one prefill of the prompt."""
+    import torch
+    t_max = w.L + nsteps
+    h = ops.filter_from_modes(lam, R, D, t_max)
+    u = ops.fir_cache_prompt(k, v, t_max)
+    y = torch.empty((w.B, w.Dch), dtype=w.torch_dtype, device=dev)
+
+    def run():
+        for t in range(nsteps):
+            i = t % dq.shape[0]
+            for _ in range(layers):
+                ops.fir_decode_step(dq[i], dk[i], dv[i], h, u, w.L + t, y=y)
+
+    with torch.cuda.stream(stream):
+        run()
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        run()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        g.replay()
+        a.record(stream)
+        for _ in range(3):
+            g.replay()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b) / 3 / nsteps
+    t_mid = w.L + (nsteps - 1) / 2
+    hist_bytes = layers * w.B * w.Dch * (t_mid * 4 + 4 * w.act_bytes + 4)
+    del g
+    return {"fir_decode": {"what": (f"cached-activation long convolution per token (no distillation), tokens "
+                                    f"{w.L}..{w.L + nsteps - 1}" + (f", {layers} layers" if layers > 1 else "")),
+                           "ms_per_token_step": ms, "tokens_per_s": w.B / (ms / 1e3),
+                           "hbm_frac": hist_bytes / (ms / 1e3) / 1e9 / peak,
+                           "modal_decode_speedup": ms / modal_step_ms},
+            "reprefill_per_token": {"what": "lower bound: one chunked prefill of the prompt per generated token",
+                                    "ms_per_token_step": prefill_ms, "modal_decode_speedup": prefill_ms / modal_step_ms}}
+
+
 # ------------------------------------------------------------------ our arm
 def run_ours(args):
     import torch
@@ -434,6 +480,10 @@ def run_ours(args):
                      "ms": fms, "achieved": fgbs, "frac": fgbs / peak, "unit": "GB/s",
                      "traffic": ncu_traffic("prefill_fused", f"{w.name}/B{w.B}")}
     dominant = max(roofs, key=lambda r: r["total_ms"])
+    baselines = None
+    if has_pre and has_dec and not args.no_baselines:
+        baselines = fir_baseline(ops, W, w, q, k, v, dq, dk, dv, lam, R, D, stream, dev, w.T,
+                                 dec_ms / w.T, pre_ms, peak)
 
     # ---- end to end: host (pinned) inputs, copies inside the timed region
     e2e = None
@@ -505,7 +555,7 @@ def run_ours(args):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
                 "data": "synthetic", "config": cfg, "prefill": out_pre, "decode": out_dec,
-                "prefill_fft_route": fft_route,
+                "prefill_fft_route": fft_route, "baselines": baselines,
                 "roofline": dominant, "roofline_all": roofs,
                 "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": args.steps * (pre_launches + w.T), "clocks": clk}
@@ -623,6 +673,17 @@ def run_layers(args, nl: int):
               "peak_source": peak_src, "algorithmic_bytes": db, "launch_ms": dec_launch_ms,
               "total_ms": dec_ms, "traffic": ncu_traffic("decode_layers", f"{w.name}/B{w.B}")}]
     dominant = max(roofs, key=lambda r: r["total_ms"])
+    baselines = None
+    if not args.no_baselines:
+        q0, k0, v0 = qkv[0]
+        dq0, dk0, dv0 = dpool[0]
+        # tokens around the middle of the generation: history of ~L + T/2 tokens per layer
+        wl = w.with_(L=w.L + w.T // 2)
+        k_hist = torch.cat([k0, dk0.transpose(0, 1).repeat(1, w.T // 2 // pool + 1, 1)[:, :w.T // 2]], 1)
+        v_hist = torch.cat([v0, dv0.transpose(0, 1).repeat(1, w.T // 2 // pool + 1, 1)[:, :w.T // 2]], 1)
+        baselines = fir_baseline(ops, W, wl, None, k_hist.contiguous(), v_hist.contiguous(), dq0, dk0, dv0,
+                                 lams[0], Rs[0], Ds[0], stream, dev, 8, dec_ms / w.T, pre_ms, peak, layers=nl)
+        del k_hist, v_hist
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         import oracle
@@ -652,6 +713,7 @@ def run_layers(args, nl: int):
                             "hbm_frac": pre_gbs / peak},
                 "decode": {"tokens_per_s": world * w.B * w.T / (dec_ms / 1e3),
                            "ms_per_token_step": dec_launch_ms, "hbm_frac": dec_gbs / peak},
+                "baselines": baselines,
                 "roofline": dominant, "roofline_all": roofs, "cpu_baseline": cpu,
                 "e2e": None, "e2e_note": "not measured for the multi-layer workload (9.6 GB of prompt per step)",
                 "gpu_launches": args.steps * (2 * nl + w.T), "clocks": clk}
@@ -677,6 +739,8 @@ def main(argv=None):
                     help="skip the extra timing of the FFT route when the chunked route is used")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-baselines", action="store_true",
+                    help="skip the undistilled (FIR / re-prefill) decode baselines")
     ap.add_argument("--layers", type=int, default=0,
                     help="layers of a multi-layer workload to run (default: all; 1 = one layer)")
     args = ap.parse_args(argv)

@@ -263,4 +263,30 @@ int hyena_decode_step_layers(int layers, const void *const *q, const void *const
                                             (cudaStream_t)stream));
 }
 
+int hyena_fir_cache_prompt(const void *k, const void *v, int dtype, int B, int L, int Dch, int t_max,
+                           float *u_cache, hyena_stream_t stream) {
+    if (dtype != HYENA_F32 && dtype != HYENA_BF16) return HYENA_ERR_ARG;
+    if (B < 0 || L < 0 || Dch < 0 || t_max < L) return HYENA_ERR_SHAPE;
+    if ((long long)B * L * Dch == 0) return HYENA_OK;
+    if (!k || !v || !u_cache) return HYENA_ERR_ARG;
+    const size_t ab = (dtype == HYENA_BF16) ? 2 : 4;
+    if (!aligned(k, ab) || !aligned(v, ab) || !aligned(u_cache, 4)) return HYENA_ERR_ALIGN;
+    return cuda_status(launch_fir_fill(k, v, dtype, B, L, Dch, t_max, u_cache, (cudaStream_t)stream));
+}
+
+int hyena_fir_decode_step(const void *q, const void *k, const void *v, int dtype, int B, int Dch, int H, int t,
+                          int t_max, const float *h, float *u_cache, void *y, hyena_stream_t stream) {
+    if (dtype != HYENA_F32 && dtype != HYENA_BF16) return HYENA_ERR_ARG;
+    if (B < 0 || H < 1 || Dch < 0 || Dch % H != 0 || t < 0 || t >= t_max) return HYENA_ERR_SHAPE;
+    if (B > 65535) return HYENA_ERR_UNSUPPORTED;
+    if (B == 0 || Dch == 0) return HYENA_OK;
+    if (!q || !k || !v || !y || !h || !u_cache) return HYENA_ERR_ARG;
+    const size_t ab = (dtype == HYENA_BF16) ? 2 : 4;
+    if (!aligned(q, ab) || !aligned(k, ab) || !aligned(v, ab) || !aligned(y, ab) || !aligned(h, 4) ||
+        !aligned(u_cache, 4))
+        return HYENA_ERR_ALIGN;
+    return cuda_status(launch_fir_step(q, k, v, dtype, B, Dch, H, t, t_max, h, u_cache, y, (cudaStream_t)stream));
+}
+
 }  // extern "C"
+

@@ -61,4 +61,10 @@ cudaError_t launch_decode_layers(int layers, const void *const *q, const void *c
                                  const float *const *R, const float *const *Dskip, float *const *state,
                                  void *const *y, cudaStream_t s);
 
+// fir.cu (undistilled baseline: cached-activation long convolution per token)
+cudaError_t launch_fir_fill(const void *k, const void *v, int dtype, int B, int L, int Dch, int t_max,
+                            float *u_cache, cudaStream_t s);
+cudaError_t launch_fir_step(const void *q, const void *k, const void *v, int dtype, int B, int Dch, int H, int t,
+                            int t_max, const float *h, float *u_cache, void *y, cudaStream_t s);
+
 }  // namespace hyena

@@ -46,6 +46,8 @@ SIGNATURES = {
     "hyena_decode_step": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _fp, _fp, _fp, _fp, _vp, _vp]),
     "hyena_decode_step_layers": (_i, [_i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
                                       _vp]),
+    "hyena_fir_cache_prompt": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _fp, _vp]),
+    "hyena_fir_decode_step": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _fp, _fp, _vp, _vp]),
 }
 
 
@@ -276,4 +278,38 @@ def decode_step_layers(layers: LayerSet, qs, ks, vs, ys):
                                           layers.R, layers.Dskip, layers.state, py,
                                           _stream(q0.device)))
     return ys
+
+
+def fir_cache_prompt(k, v, t_max: int, u_cache=None):
+    """History of a prompt for the undistilled baseline: u_cache float32 [B][t_max][Dch] with
+    rows j < L set to k_j v_j (the rest left as they are)."""
+    k, v = _cuda(k, "k"), _cuda(v, "v")
+    dt = _act_dtype(k)
+    B, L, Dch = k.shape
+    if u_cache is None:
+        u_cache = torch.zeros((B, t_max, Dch), dtype=torch.float32, device=k.device)
+    _cuda(u_cache, "u_cache", torch.float32)
+    _check("hyena_fir_cache_prompt",
+           lib().hyena_fir_cache_prompt(_ptr(k), _ptr(v), dt, B, L, Dch, t_max, _ptr(u_cache),
+                                        _stream(k.device)))
+    return u_cache
+
+
+def fir_decode_step(q, k, v, h, u_cache, t: int, y=None):
+    """Undistilled decode of token t: y = q (sum_{j<=t} h_{t-j} u_j), history in u_cache
+    [B][t_max][Dch] (row t is written); h [H][t_max] float32 taps."""
+    q, k, v = _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v")
+    h = _cuda(h, "h", torch.float32)
+    u_cache = _cuda(u_cache, "u_cache", torch.float32)
+    dt = _act_dtype(q)
+    B, Dch = q.shape
+    H, t_max = h.shape
+    if u_cache.shape != (B, t_max, Dch):
+        raise ValueError("u_cache must be [B][t_max][Dch] with t_max = h.shape[1]")
+    if y is None:
+        y = torch.empty_like(q)
+    _check("hyena_fir_decode_step",
+           lib().hyena_fir_decode_step(_ptr(q), _ptr(k), _ptr(v), dt, B, Dch, H, t, t_max, _ptr(h),
+                                       _ptr(u_cache), _ptr(y), _stream(q.device)))
+    return y
 

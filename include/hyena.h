@@ -257,6 +257,33 @@ int hyena_decode_step_layers(int layers, const void *const *q, const void *const
                              const float *const *Dskip, float *const *state, void *const *y,
                              hyena_stream_t stream);
 
+/*
+ * Undistilled decode baseline: one token by convolving the cached history with
+ * the long filter, as generation works without the distilled recurrence.  Its
+ * cost grows with the sequence (O(t) per token and O(t) cached activations per
+ * channel), against O(d) for hyena_decode_step ("Laughing Hyena Distillery",
+ * nubint.ai review, "Main findings"): it is the comparison point for that
+ * claim, on the same hardware and with the same filter.
+ *
+ * hyena_fir_cache_prompt writes the history of a prompt:
+ *   u_cache[b][j][c] = k[b][j][c] v[b][j][c] for j < L (fp32, exact for bf16 inputs)
+ *   k, v    : [B][L][Dch] (dtype);  u_cache : [B][t_max][Dch] fp32, rows >= L untouched
+ *   Requires t_max >= L.
+ * hyena_fir_decode_step emits token t and appends it to the history:
+ *   y[b][c] = q[b][c] (sum_{j<t} h[hd][t-j] u_cache[b][j][c] + h[hd][0] u),  u = k[b][c] v[b][c]
+ *   then u_cache[b][t][c] = u.
+ *   q, k, v, y : [B][Dch] (dtype);  h : [H][t_max] fp32 filter taps (for example from
+ *   hyena_filter_from_modes with L = t_max);  rows 0..t-1 of u_cache must hold the history.
+ *   Requires 0 <= t < t_max and B <= 65535.  Alignment: activations to their
+ *   element size, h and u_cache to 4 bytes.
+ * The sum over the history runs in fp32 in a fixed order (deterministic).
+ */
+int hyena_fir_cache_prompt(const void *k, const void *v, int dtype, int B, int L, int Dch, int t_max,
+                           float *u_cache, hyena_stream_t stream);
+int hyena_fir_decode_step(const void *q, const void *k, const void *v, int dtype, int B, int Dch, int H,
+                          int t, int t_max, const float *h, float *u_cache, void *y,
+                          hyena_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

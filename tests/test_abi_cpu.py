@@ -154,3 +154,19 @@ def test_decode_layers_validation(lib):
     assert call(B=0) == OK
     assert lib.hyena_decode_step_layers(2, None, good, good, 1, 2, 8, 2, 4, good, good, good, good, good,
                                         None) == ERR_ARG
+
+
+def test_fir_validation(lib):
+    def step(dtype=1, B=2, Dch=8, H=2, t=3, t_max=8, ptr=FAKE):
+        return lib.hyena_fir_decode_step(_p(ptr), _p(FAKE), _p(FAKE), dtype, B, Dch, H, t, t_max, _p(FAKE),
+                                         _p(FAKE), _p(FAKE), None)
+    assert step(dtype=7) == ERR_ARG
+    assert step(t=8) == ERR_SHAPE              # t must be < t_max
+    assert step(t=-1) == ERR_SHAPE
+    assert step(Dch=9, H=2) == ERR_SHAPE
+    assert step(B=70000) == ERR_UNSUP
+    assert step(ptr=FAKE + 1) == ERR_ALIGN
+    assert step(B=0) == OK
+    assert lib.hyena_fir_cache_prompt(_p(), _p(), 1, 2, 9, 8, 8, _p(), None) == ERR_SHAPE   # t_max < L
+    assert lib.hyena_fir_cache_prompt(_p(), _p(), 1, 2, 0, 8, 8, _p(), None) == OK          # empty prompt
+    assert lib.hyena_fir_cache_prompt(_p(FAKE + 1), _p(), 1, 2, 4, 8, 8, _p(), None) == ERR_ALIGN
