@@ -14,6 +14,7 @@ the C file's header:
 * state      s_n = sum_{j<L} lambda_n^(L-1-j) k_j v_j                 (prompt -> state)
 * recurrence y_t = q_t (Dskip u_t + Re sum R s), then s <- lambda s + u (O(d) decode)
 * spectrum   DFT of the zero-padded filter, bins 0..N/2
+* truncation keep the k modes of largest |R|/(1-|lambda|); l1 bound and direct l1/l2 tap errors
 
 Sources: Laughing Hyena Distillery (nubint.ai review), "Proposed method" and
 "Main findings"; Hyena processes long sequences 100x faster than FlashAttention
@@ -63,6 +64,8 @@ def _load():
             lib.oracle_prompt_state.argtypes = [_dp, _dp] + [ctypes.c_int] * 5 + [_dp, _dp]
             lib.oracle_recurrent.argtypes = ([_dp, _dp, _dp] + [ctypes.c_int] * 5 +
                                              [_dp, _dp, _dp, _dp, _dp])
+            lib.oracle_modal_truncate.argtypes = [_dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                  ctypes.c_int, _ip, _dp, _dp, _dp, _dp, _dp]
             _lib = lib
     return _lib
 
@@ -160,3 +163,22 @@ def decode_step(q, k, v, lam, R, Dskip, H: int, state):
     q, k, v = (_f64(a)[:, None, :] for a in (q, k, v))
     y, s = recurrent(q, k, v, lam, R, Dskip, H, state)
     return y[:, 0, :], s
+
+
+def modal_truncate(lam, R, k: int, J: int = 200000):
+    """Keep the k modes of largest |R|/(1-|lambda|) per head (ties: lower index).
+
+    Returns (kept [H][k] int, lam_out [H][k], R_out [H][k] complex, bound [H],
+    err_l1 [H], err_l2 [H]): bound = sum of the dropped scores, err_* the l1 / l2 norms of
+    the dropped modes' filter over taps 1..J by direct summation."""
+    lam2, R2 = _cplx(lam), _cplx(R)
+    H, d = lam2.shape[0], lam2.shape[1]
+    assert 0 <= k <= d <= 256
+    kept = np.zeros((H, max(k, 1)), dtype=np.int32)
+    lo = np.zeros((H, max(k, 1), 2)); ro = np.zeros((H, max(k, 1), 2))
+    b, e1, e2 = np.zeros(H), np.zeros(H), np.zeros(H)
+    _load().oracle_modal_truncate(_ptr(lam2), _ptr(R2), H, d, k, J, kept.ctypes.data_as(_ip), _ptr(lo),
+                                  _ptr(ro), _ptr(b), _ptr(e1), _ptr(e2))
+    kept, lo, ro = kept[:, :k], lo[:, :k], ro[:, :k]
+    return kept, lo[..., 0] + 1j * lo[..., 1], ro[..., 0] + 1j * ro[..., 1], b, e1, e2
+

@@ -221,3 +221,69 @@ void oracle_recurrent(const double *q, const double *k, const double *v,
         }
     }
 }
+
+/* ---------------------------------------------------------------------------
+ * Modal truncation (model-order reduction of the modal SSM: "Laughing Hyena
+ * Distillery", nubint.ai review, "Proposed method", balanced and modal
+ * truncation).  Each mode's share of the filter taps j >= 1 is
+ * Re(R_n lambda_n^(j-1)), whose l1 norm is at most
+ *     score_n = |R_n| / (1 - |lambda_n|)      (+inf when |lambda_n| >= 1).
+ * The k modes with the largest scores are kept, ties going to the lower
+ * index: mode n is kept iff fewer than k modes m have score_m > score_n or
+ * (score_m == score_n and m < n).  Kept modes are written in index order.
+ * Outputs per head: kept[k] (indices), lam_out/R_out [k][2], bound = sum of
+ * the dropped scores, and, by direct summation over taps j = 1..J of the
+ * dropped modes' filter dh_j = Re sum_{n dropped} R_n lambda_n^(j-1) (powers by
+ * repeated multiplication), err_l1 = sum |dh_j| and err_l2 = sqrt(sum dh_j^2).
+ * ------------------------------------------------------------------------- */
+void oracle_modal_truncate(const double *lam, const double *R, int H, int d, int k, int J,
+                           int *kept, double *lam_out, double *R_out,
+                           double *bound, double *err_l1, double *err_l2)
+{
+    for (int hd = 0; hd < H; ++hd) {
+        const double *lh = lam + (size_t)hd * d * 2, *rh = R + (size_t)hd * d * 2;
+        double score[256];
+        int keep[256];
+        for (int n = 0; n < d; ++n) {
+            const double a = sqrt(lh[2 * n] * lh[2 * n] + lh[2 * n + 1] * lh[2 * n + 1]);
+            const double r = sqrt(rh[2 * n] * rh[2 * n] + rh[2 * n + 1] * rh[2 * n + 1]);
+            score[n] = a < 1.0 ? r / (1.0 - a) : INFINITY;
+        }
+        int out = 0;
+        double b = 0.0;
+        for (int n = 0; n < d; ++n) {
+            int ahead = 0;
+            for (int m = 0; m < d; ++m)
+                if (score[m] > score[n] || (score[m] == score[n] && m < n)) ++ahead;
+            keep[n] = ahead < k;
+            if (keep[n]) {
+                kept[(size_t)hd * k + out] = n;
+                lam_out[((size_t)hd * k + out) * 2 + 0] = lh[2 * n];
+                lam_out[((size_t)hd * k + out) * 2 + 1] = lh[2 * n + 1];
+                R_out[((size_t)hd * k + out) * 2 + 0] = rh[2 * n];
+                R_out[((size_t)hd * k + out) * 2 + 1] = rh[2 * n + 1];
+                ++out;
+            } else {
+                b += score[n];
+            }
+        }
+        bound[hd] = b;
+        double l1 = 0.0, l2 = 0.0;
+        double pr[256], pi[256];
+        for (int n = 0; n < d; ++n) { pr[n] = 1.0; pi[n] = 0.0; }
+        for (int j = 1; j <= J; ++j) {
+            double dh = 0.0;
+            for (int n = 0; n < d; ++n) {
+                if (keep[n]) continue;
+                dh += rh[2 * n] * pr[n] - rh[2 * n + 1] * pi[n];
+                const double nr = pr[n] * lh[2 * n] - pi[n] * lh[2 * n + 1];
+                const double ni = pr[n] * lh[2 * n + 1] + pi[n] * lh[2 * n];
+                pr[n] = nr; pi[n] = ni;
+            }
+            l1 += fabs(dh);
+            l2 += dh * dh;
+        }
+        err_l1[hd] = l1;
+        err_l2[hd] = sqrt(l2);
+    }
+}

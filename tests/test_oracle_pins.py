@@ -276,3 +276,57 @@ def test_workload_generator_is_deterministic_and_distributed():
     b = W.decode_inputs(w, step=3, B=2, Dch=16)[0]
     c = W.decode_inputs(w, step=4, B=2, Dch=16)[0]
     assert (a.float() == b.float()).all() and not (a.float() == c.float()).all()
+
+
+# ---------------------------------------------------------------- modal truncation
+def test_truncation_selection_hand_example(oracle):
+    """Scores |R|/(1-|lambda|) worked by hand: lambda = [1/2, 9/10, 0, i/2], R = [1, 1/10, 1/2, 3]
+    give 2, 1, 1/2, 6, so the ranking is modes 3, 0, 1, 2; kept modes come out in index order."""
+    lam = np.array([[0.5, 0.9, 0.0, 0.5j]])
+    R = np.array([[1.0, 0.1, 0.5, 3.0]], dtype=complex)
+    expect = {0: [], 1: [3], 2: [0, 3], 3: [0, 1, 3], 4: [0, 1, 2, 3]}
+    dropped_scores = {0: 9.5, 1: 3.5, 2: 1.5, 3: 0.5, 4: 0.0}
+    for k, ids in expect.items():
+        kept, lo, ro, b, e1, e2 = oracle.modal_truncate(lam, R, k, J=4000)
+        assert kept[0].tolist() == ids
+        assert np.array_equal(lo[0], lam[0, ids]) and np.array_equal(ro[0], R[0, ids])
+        assert b[0] == pytest.approx(dropped_scores[k], rel=1e-15)
+    # equal scores: the lower index wins
+    kept, *_ = oracle.modal_truncate(np.array([[0.5, 0.5]]), np.array([[1.0, -1.0]], dtype=complex), 1)
+    assert kept[0].tolist() == [0]
+
+
+@pytest.mark.parametrize("lam,R", [(0.8, 1.5), (0.6 * cmath.exp(1j), 0.3 - 0.7j), (-0.95j, 2j), (0.0, 1.0)])
+def test_truncation_single_mode_closed_form(oracle, lam, R):
+    """Dropping the only mode leaves dh_j = Re(R lambda^(j-1)).  Closed forms of its norms:
+    sum_j dh_j^2 = Re(R^2 / (1 - lambda^2)) / 2 + |R|^2 / (1 - |lambda|^2) / 2 (from
+    Re(z)^2 = (z^2 + 2|z|^2 + conj(z)^2) / 4 and geometric series), and for a positive real pole
+    and residue sum_j |dh_j| = R / (1 - lambda), which the bound then equals."""
+    lam_a, R_a = np.array([[lam]], dtype=complex), np.array([[R]], dtype=complex)
+    kept, lo, ro, b, e1, e2 = oracle.modal_truncate(lam_a, R_a, 0, J=5000)
+    l2sq = (R * R / (1 - lam * lam)).real / 2 + abs(R) ** 2 / (1 - abs(lam) ** 2) / 2
+    assert e2[0] ** 2 == pytest.approx(l2sq, rel=1e-12)
+    assert b[0] == pytest.approx(abs(R) / (1 - abs(lam)), rel=1e-15)
+    assert e1[0] <= b[0] * (1 + 1e-12)
+    if isinstance(lam, float) and lam > 0:
+        assert e1[0] == pytest.approx(R / (1 - lam), rel=1e-12)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_truncation_splits_the_filter(oracle, seed):
+    """Kept modes' filter + dropped modes' filter = the full filter (brute force), the direct l1/l2
+    errors are the norms of that difference, and the l1 error never exceeds the bound."""
+    rng = np.random.default_rng(seed)
+    H, d, J = 3, 9, 3000
+    lam, R, D = _rand_params(rng, H, d, rmin=0.2, rmax=0.97)
+    h = oracle.filter_from_modes(lam, R, D, J + 1)
+    for k in (0, 3, 8, 9):
+        kept, lo, ro, b, e1, e2 = oracle.modal_truncate(lam, R, k, J=J)
+        hk = oracle.filter_from_modes(lo, ro, D, J + 1) if k else np.tile(D[:, None], (1, J + 1)) * np.eye(1, J + 1)
+        dh = (h - hk)[:, 1:]
+        assert np.allclose(np.abs(dh).sum(1), e1, rtol=1e-10, atol=1e-14)
+        assert np.allclose(np.sqrt((dh ** 2).sum(1)), e2, rtol=1e-10, atol=1e-14)
+        assert np.all(e1 <= b * (1 + 1e-12))
+        assert np.array_equal(hk[:, 0], D)
+        if k == d:
+            assert np.all(e2 == 0) and np.all(b == 0)
