@@ -725,6 +725,33 @@ def run_layers(args, nl: int):
     return 0
 
 
+def run_truncation(args):
+    """Filter error of modal truncation against the number of kept modes, per workload: the l2
+    norm of the tap error relative to the full filter's (taps j >= 1) and the l1 bound relative to
+    its value with every mode dropped (GPU kernel through the C ABI)."""
+    import torch
+    from distilled_ssm_decode_b200 import build, ops
+    from distilled_ssm_decode_b200 import workloads as W
+    build.build()
+    out = {"metric": "modal truncation: relative filter error vs kept modes", "workloads": {}}
+    for name in ("mid_bf16", "gen1p3b_bf16", "long_prefill_bf16"):
+        w = W.WORKLOADS[name]
+        p = W.params(w)
+        lam, R = p.lam_f32().cuda(), p.R_f32().cuda()
+        _, _, _, b0, e0 = ops.modal_truncate(lam, R, 0)
+        rows = []
+        for k in range(1, w.d + 1):
+            _, _, _, b, e = ops.modal_truncate(lam, R, k)
+            rel = (e / e0).cpu().numpy()
+            rb = (b / b0).cpu().numpy()
+            rows.append({"k": k, "l2_rel_mean": float(rel.mean()), "l2_rel_max": float(rel.max()),
+                         "l1_bound_rel_max": float(rb.max())})
+        out["workloads"][name] = {"H": w.H, "d": w.d, "poles": f"|lambda| ~ U[{w.rmin}, {w.rmax}]",
+                                  "rows": rows}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -741,12 +768,16 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-baselines", action="store_true",
                     help="skip the undistilled (FIR / re-prefill) decode baselines")
+    ap.add_argument("--truncation", action="store_true",
+                    help="print the modal-truncation error table instead of benchmarking")
     ap.add_argument("--layers", type=int, default=0,
                     help="layers of a multi-layer workload to run (default: all; 1 = one layer)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)   # at least 3 untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
+    if args.truncation:
+        return run_truncation(args)
     from distilled_ssm_decode_b200 import workloads as W
     nl = args.layers or W.WORKLOADS[args.workload].layers
     if nl > 1:

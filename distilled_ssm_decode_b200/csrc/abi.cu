@@ -288,5 +288,21 @@ int hyena_fir_decode_step(const void *q, const void *k, const void *v, int dtype
     return cuda_status(launch_fir_step(q, k, v, dtype, B, Dch, H, t, t_max, h, u_cache, y, (cudaStream_t)stream));
 }
 
+int hyena_modal_truncate(const float *lambda, const float *R, int H, int d, int k, int *kept,
+                         float *lambda_out, float *R_out, double *bound, double *err_l2,
+                         hyena_stream_t stream) {
+    if (H < 0 || d < 1 || d > HYENA_MAX_MODES || k < 0 || k > d) return HYENA_ERR_SHAPE;
+    if (H == 0) return HYENA_OK;
+    if (!lambda || !R || !bound || !err_l2 || (k > 0 && (!kept || !lambda_out || !R_out))) return HYENA_ERR_ARG;
+    if (!aligned(lambda, 8) || !aligned(R, 8) || !aligned(bound, 8) || !aligned(err_l2, 8) ||
+        (k > 0 && (!aligned(kept, 4) || !aligned(lambda_out, 8) || !aligned(R_out, 8))))
+        return HYENA_ERR_ALIGN;
+    return cuda_status(launch_modal_truncate(reinterpret_cast<const float2 *>(lambda),
+                                             reinterpret_cast<const float2 *>(R), H, d, k, kept,
+                                             reinterpret_cast<float2 *>(lambda_out),
+                                             reinterpret_cast<float2 *>(R_out), bound, err_l2,
+                                             (cudaStream_t)stream));
+}
+
 }  // extern "C"
 

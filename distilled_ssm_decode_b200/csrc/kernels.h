@@ -67,4 +67,8 @@ cudaError_t launch_fir_fill(const void *k, const void *v, int dtype, int B, int 
 cudaError_t launch_fir_step(const void *q, const void *k, const void *v, int dtype, int B, int Dch, int H, int t,
                             int t_max, const float *h, float *u_cache, void *y, cudaStream_t s);
 
+// truncate.cu (modal truncation of each head's SSM)
+cudaError_t launch_modal_truncate(const float2 *lam, const float2 *R, int H, int d, int k, int *kept,
+                                  float2 *lam_out, float2 *R_out, double *bound, double *err_l2, cudaStream_t s);
+
 }  // namespace hyena

@@ -48,6 +48,7 @@ SIGNATURES = {
                                       _vp]),
     "hyena_fir_cache_prompt": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _fp, _vp]),
     "hyena_fir_decode_step": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _fp, _fp, _vp, _vp]),
+    "hyena_modal_truncate": (_i, [_fp, _fp, _i, _i, _i, _vp, _fp, _fp, _vp, _vp, _vp]),
 }
 
 
@@ -312,4 +313,23 @@ def fir_decode_step(q, k, v, h, u_cache, t: int, y=None):
            lib().hyena_fir_decode_step(_ptr(q), _ptr(k), _ptr(v), dt, B, Dch, H, t, t_max, _ptr(h),
                                        _ptr(u_cache), _ptr(y), _stream(q.device)))
     return y
+
+
+def modal_truncate(lam, R, k: int):
+    """Keep the k modes of largest |R|/(1-|lambda|) per head.  Returns (kept int32 [H][k],
+    lam_out, R_out float32 [H][k][2], bound float64 [H], err_l2 float64 [H])."""
+    lam = _cuda(lam, "lam", torch.float32)
+    R = _cuda(R, "R", torch.float32)
+    H, d = lam.shape[0], lam.shape[1]
+    dev = lam.device
+    kept = torch.empty((H, k), dtype=torch.int32, device=dev)
+    lo = torch.empty((H, k, 2), dtype=torch.float32, device=dev)
+    ro = torch.empty((H, k, 2), dtype=torch.float32, device=dev)
+    bound = torch.empty(H, dtype=torch.float64, device=dev)
+    err = torch.empty(H, dtype=torch.float64, device=dev)
+    nul = lambda t: _ptr(t) if k > 0 else None
+    _check("hyena_modal_truncate",
+           lib().hyena_modal_truncate(_ptr(lam), _ptr(R), H, d, k, nul(kept), nul(lo), nul(ro), _ptr(bound),
+                                      _ptr(err), _stream(dev)))
+    return kept, lo, ro, bound, err
 

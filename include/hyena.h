@@ -284,6 +284,29 @@ int hyena_fir_decode_step(const void *q, const void *k, const void *v, int dtype
                           int t, int t_max, const float *h, float *u_cache, void *y,
                           hyena_stream_t stream);
 
+/*
+ * Modal truncation of each head's SSM to k modes (the model-order reduction
+ * step of the distillation: balanced and modal truncation, "Laughing Hyena
+ * Distillery", nubint.ai review, "Proposed method").  Mode n of a head adds
+ * Re(R_n lambda_n^(j-1)) to tap j (j >= 1); the l1 norm of that is at most
+ * score_n = |R_n| / (1 - |lambda_n|).  The k modes with the largest scores are
+ * kept (equal scores: the lower index), in index order, so that
+ * lambda_out, R_out with Dskip unchanged give the truncated filter.
+ *   lambda, R          : [H][d][2] fp32 device (d <= HYENA_MAX_MODES, 0 <= k <= d)
+ *   kept               : [H][k] int32 device, indices of the kept modes
+ *   lambda_out, R_out  : [H][k][2] fp32 device (copies of the kept modes)
+ *   bound              : [H] fp64 device, sum of the dropped scores: an upper
+ *                        bound on sum_j |h_j - h'_j|, hence on max|dy| / max|u|
+ *   err_l2             : [H] fp64 device, the exact l2 norm of the tap error
+ *                        (sqrt sum_{j>=1} (h_j - h'_j)^2, summed in closed form
+ *                        over pairs of dropped modes); +inf if a dropped mode has
+ *                        |lambda| >= 1
+ * kept, lambda_out and R_out may be NULL when k == 0.
+ */
+int hyena_modal_truncate(const float *lambda, const float *R, int H, int d, int k, int *kept,
+                         float *lambda_out, float *R_out, double *bound, double *err_l2,
+                         hyena_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -170,3 +170,17 @@ def test_fir_validation(lib):
     assert lib.hyena_fir_cache_prompt(_p(), _p(), 1, 2, 9, 8, 8, _p(), None) == ERR_SHAPE   # t_max < L
     assert lib.hyena_fir_cache_prompt(_p(), _p(), 1, 2, 0, 8, 8, _p(), None) == OK          # empty prompt
     assert lib.hyena_fir_cache_prompt(_p(FAKE + 1), _p(), 1, 2, 4, 8, 8, _p(), None) == ERR_ALIGN
+
+
+def test_modal_truncate_validation(lib):
+    def call(H=2, d=4, k=2, ptr=FAKE, kept=FAKE):
+        return lib.hyena_modal_truncate(_p(ptr), _p(FAKE), H, d, k, _p(kept), _p(FAKE), _p(FAKE), _p(FAKE),
+                                        _p(FAKE), None)
+    assert call(k=5) == ERR_SHAPE           # k > d
+    assert call(k=-1) == ERR_SHAPE
+    assert call(d=65, k=2) == ERR_SHAPE
+    assert call(H=-1) == ERR_SHAPE
+    assert call(ptr=FAKE + 4) == ERR_ALIGN
+    assert call(kept=FAKE + 2) == ERR_ALIGN
+    assert call(H=0) == OK
+    assert lib.hyena_modal_truncate(_p(), _p(), 2, 4, 2, None, _p(), _p(), _p(), _p(), None) == ERR_ARG
