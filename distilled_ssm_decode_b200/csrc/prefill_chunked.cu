@@ -261,6 +261,14 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&p);
 }
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
+// Two bf16 products rounded to nearest bf16 in one instruction.  The exact product of two bf16
+// values has at most 16 significant bits, so this is the same rounding as an fp32 product
+// followed by a conversion to bf16 (outside the subnormal range).
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
 // ------------------------------------------------------------------ per-head constants
@@ -726,12 +734,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     const int off = c16 * 16;               // same byte offset in k, v and U
                     const uint4 kk = *reinterpret_cast<const uint4 *>(kt + off);
                     const uint4 vv = *reinterpret_cast<const uint4 *>(kt + kTile + off);
-                    uint4 uu;
-                    uu.x = pack_bf16(bf_lo(kk.x) * bf_lo(vv.x), bf_hi(kk.x) * bf_hi(vv.x));
-                    uu.y = pack_bf16(bf_lo(kk.y) * bf_lo(vv.y), bf_hi(kk.y) * bf_hi(vv.y));
-                    uu.z = pack_bf16(bf_lo(kk.z) * bf_lo(vv.z), bf_hi(kk.z) * bf_hi(vv.z));
-                    uu.w = pack_bf16(bf_lo(kk.w) * bf_lo(vv.w), bf_hi(kk.w) * bf_hi(vv.w));
-                    *reinterpret_cast<uint4 *>(kt + off) = uu;
+                    *reinterpret_cast<uint4 *>(kt + off) = make_uint4(mul_bf16x2(kk.x, vv.x), mul_bf16x2(kk.y, vv.y),
+                                                                       mul_bf16x2(kk.z, vv.z), mul_bf16x2(kk.w, vv.w));
                 }
                 tc::fence_proxy_async_smem();
                 tc::mbar_arrive(bar(kBarURdy + st));
