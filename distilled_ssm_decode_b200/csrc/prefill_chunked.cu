@@ -77,6 +77,8 @@ constexpr uint32_t kTmemCols = 512; // all of tensor memory (one CTA per SM)
 // 4 S and 4 E warps
 constexpr int kItemReaders = 4 + 11;
 constexpr int kUThreads = 96;       // U group (3 warps)
+constexpr int kEThreads = 128;      // E group (4 warps); it helps to form U in state-only iterations
+constexpr int kUHelp = kUThreads + kEThreads;
 
 // per-head constants: the two A operands (copied verbatim into shared memory) and the powers
 // lambda^C, lambda^Lseg (read from global by the state group)
@@ -102,7 +104,14 @@ struct Geo {
     static constexpr int kKVStages = NC == 128 ? 4 : 8;
     static constexpr int kQStages = NC == 128 ? 3 : 6;        // q tiles; y is staged in place
     static constexpr int kSlotCols = 2 * NC;                  // fused [NC cols] | carry [NC cols]
-    static constexpr int kSlots = (int)kTmemCols / kSlotCols;
+    // The 64-channel tile keeps both A operands (constant per head) in tensor memory, so the MMAs
+    // read only their B operand from shared memory: 3 accumulator slots + 48 columns of A
+    // (fused A: K = 64 -> 32 columns, carry A: K = 32 -> 16 columns).  The 128-channel tile
+    // needs every column for its 2 slots and reads A from shared memory.
+    static constexpr bool kATmem = NC == 64;
+    static constexpr int kSlots = kATmem ? 3 : (int)kTmemCols / kSlotCols;
+    static constexpr int kACol = kSlots * kSlotCols;          // first column of A (kATmem)
+    static_assert(!kATmem || kACol + 48 <= (int)kTmemCols, "tensor memory budget");
     static constexpr int kSBytes = kKS * NC * 2;              // [32 rows][NC ch] bf16, 128-byte swizzled
     static constexpr int kSmQ = kSmKV + kKVStages * kStageBytes;
     static constexpr int kSmS = kSmQ + kQStages * kTile;
@@ -135,7 +144,7 @@ struct Geo {
     static_assert(kSmQ % 1024 == 0 && kSmS % 1024 == 0, "swizzle atoms");
 
     __host__ __device__ static constexpr int count(int i) {
-        return (i >= kBarURdy && i < kBarQFull) ? kUThreads
+        return (i >= kBarURdy && i < kBarQFull) ? kUHelp
                : ((i >= kBarYStaged && i < kBarWDone) || (i >= kBarD2Free && i < kBarYDone) ||
                   (i >= kBarD1Free && i < kBarSTFree) || (i >= kBarPubFull && i < kBarPubEmpty))
                    ? 128
@@ -149,6 +158,8 @@ constexpr int kWarpKV = 0, kWarpQ = 1, kWarpMMA = 3, kWarpStore = 12, kWarpCarry
 __host__ __device__ constexpr bool is_s_warp(int w) { return (w & 3) == 2; }                 // 2, 6, 10, 14
 __host__ __device__ constexpr bool is_e_warp(int w) { return w == 4 || w == 5 || w == 8 || w == 9; }
 __host__ __device__ constexpr int u_index(int w) { return w == 7 ? 0 : w == 11 ? 1 : w == 15 ? 2 : -1; }
+__host__ __device__ constexpr int e_index(int w) { return w == 4 ? 0 : w == 5 ? 1 : w == 8 ? 2 : 3; }
+
 
 // byte offset of bf16 element (row, k) in a K-major, no-swizzle core-matrix tile of K columns
 __host__ __device__ __forceinline__ int cm_off16(int row, int k, int K) {
@@ -261,6 +272,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&p);
 }
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 // Two bf16 products rounded to nearest bf16 in one instruction.  The exact product of two bf16
 // values has at most 16 significant bits, so this is the same rounding as an fp32 product
 // followed by a conversion to bf16 (outside the subnormal range).
@@ -269,7 +281,20 @@ __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
     asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
-__device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+
+// U = k v in place over the k half of a k,v stage (the same byte offset in k, v and U), 16 bytes
+// per step: thread `t` of `nthreads` takes every nthreads-th 16-byte piece.
+template <int kTileBytes>
+__device__ __forceinline__ void form_u(uint8_t *kt, int t, int nthreads) {
+#pragma unroll 4
+    for (int c16 = t; c16 < kTileBytes / 16; c16 += nthreads) {
+        const int off = c16 * 16;
+        const uint4 kk = *reinterpret_cast<const uint4 *>(kt + off);
+        const uint4 vv = *reinterpret_cast<const uint4 *>(kt + kTileBytes + off);
+        *reinterpret_cast<uint4 *>(kt + off) =
+            make_uint4(mul_bf16x2(kk.x, vv.x), mul_bf16x2(kk.y, vv.y), mul_bf16x2(kk.z, vv.z), mul_bf16x2(kk.w, vv.w));
+    }
+}
 
 // ------------------------------------------------------------------ per-head constants
 // Blocks (head, part): every block of a head tabulates the head's powers and taps, and writes
@@ -382,11 +407,12 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
 
 // ------------------------------------------------------------------ main kernel
 // Roles (warps):  0  k,v TMA loads; takes item tickets and posts them to the other roles
-//                 1  q TMA loads            12  y TMA stores (lane 0 each)
-//                 3  tensor memory owner and MMA issuer (lane 0)
-//                 7, 11, 13, 15   U group: U = k v over the k tile (elementwise)
-//                 2, 6, 10, 14    S group: state rows 0..31 x 32 channels each; chain, publish, look-back
-//                 4, 5, 8, 9      E group: token rows 0..63 x 64 channels each; gate and stage y
+//                 1  q TMA loads            12  y TMA stores, segment-state publisher (lanes 0, 1)
+//                 3  tensor memory owner and fused-product issuer (lane 0)
+//                13  carry-product issuer (lane 0)
+//                 7, 11, 15       U group: U = k v over the k tile (elementwise)
+//                 2, 6, 10, 14    S group: state rows 0..31 x NC/4 channels each; chain, publish, look-back
+//                 4, 5, 8, 9      E group: token rows 0..63 x NC/2 channels each; gate and stage y
 // Each role loops over the same item sequence and the same chunk order; they meet only at
 // mbarriers, so loads, U, the products, the chain and the epilogue of different chunks overlap.
 template <int NC>
@@ -397,6 +423,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     using G = Geo<NC>;
     constexpr int kNC = NC, kTile = G::kTile, kStageBytes = G::kStageBytes, kKVStages = G::kKVStages,
                   kQStages = G::kQStages, kSlots = G::kSlots, kSlotCols = G::kSlotCols, kSBytes = G::kSBytes,
+                  kACol = G::kACol,
                   kSmQ = G::kSmQ, kSmS = G::kSmS, kSmBar = G::kSmBar, kSmMisc = G::kSmMisc;
     constexpr int kBarKVFull = G::kBarKVFull, kBarKVEmpty = G::kBarKVEmpty, kBarURdy = G::kBarURdy,
                   kBarQFull = G::kBarQFull, kBarQEmpty = G::kBarQEmpty, kBarYStaged = G::kBarYStaged,
@@ -485,6 +512,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         if (lane == 0) {
             int g = 0, head = blockIdx.x % a.H, tries = 0;
             bool ok = true;
+            const uint64_t pol_keep = tc::l2_policy_evict_last(), pol_drop = tc::l2_policy_evict_first();
             for (int k = 0; ok; ++k) {
                 const int s = k % kItemQ;
                 if (!tc::mbar_wait(bar(kBarItemEmpty + s), ((k / kItemQ) & 1) ^ 1, abort)) {
@@ -512,10 +540,14 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     }
                     const uint32_t dst = sbase + kSmKV + st * kStageBytes;
                     tc::mbar_expect_tx(bar(kBarKVFull + st), kStageBytes);
+                    // the state-only pass reads k, v that the full pass reads again soon: ask L2 to keep
+                    // them; the full pass reads them for the last time
+                    const uint64_t pol = i < it.n1 ? pol_keep : pol_drop;
                     for (int h = 0; h < kNC / 64; ++h) {
-                        tc::tma_load_3d(dst + h * kAtom, &tm_k, bar(kBarKVFull + st), it.c0 + 64 * h, tok_of(chunk), it.b);
-                        tc::tma_load_3d(dst + kTile + h * kAtom, &tm_v, bar(kBarKVFull + st), it.c0 + 64 * h,
-                                        tok_of(chunk), it.b);
+                        tc::tma_load_3d_hint(dst + h * kAtom, &tm_k, bar(kBarKVFull + st), it.c0 + 64 * h, tok_of(chunk),
+                                             it.b, pol);
+                        tc::tma_load_3d_hint(dst + kTile + h * kAtom, &tm_v, bar(kBarKVFull + st), it.c0 + 64 * h,
+                                             tok_of(chunk), it.b, pol);
                     }
                 }
             }
@@ -531,6 +563,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         if (lane == 0) {
             int qg = 0;
             bool ok = true;
+            const uint64_t pol_drop = tc::l2_policy_evict_first();
             for (int k = 0; ok; ++k) {
                 const int id = take_item(k, false);
                 if (id == -2) ok = false;
@@ -543,9 +576,9 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         break;
                     }
                     tc::mbar_expect_tx(bar(kBarQFull + s), kTile);
-                    for (int h = 0; h < kNC / 64; ++h)
-                        tc::tma_load_3d(sbase + kSmQ + s * kTile + h * kAtom, &tm_q, bar(kBarQFull + s),
-                                        it.c0 + 64 * h, tok_of(it.ck0 + j), it.b);
+                    for (int h = 0; h < kNC / 64; ++h)     // q is read once
+                        tc::tma_load_3d_hint(sbase + kSmQ + s * kTile + h * kAtom, &tm_q, bar(kBarQFull + s),
+                                             it.c0 + 64 * h, tok_of(it.ck0 + j), it.b, pol_drop);
                 }
             }
             if (!ok) {
@@ -644,6 +677,19 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     if (!tc::mbar_wait(bar(kBarConst), cphase & 1, never)) { ok = false; break; }
                     ++cphase;
                     cur_hd = it.hd;
+                    if constexpr (G::kATmem) {
+                        // both A operands into tensor memory, one K = 16 slice (8 columns) per copy; the
+                        // copies run in order with this thread's MMAs, and the commits that follow
+                        // (seen by the carry issuer through WDone) cover them
+                        tc::tc_fence_after();
+#pragma unroll
+                        for (int ks = 0; ks < kC / 16; ++ks)
+                            tc::tmem_cp_128x256b(tmem + kACol + 8 * ks, tc::smem_desc(sbase + kSmFA + ks * 256, 128, kC * 16));
+#pragma unroll
+                        for (int ks = 0; ks < kKS / 16; ++ks)
+                            tc::tmem_cp_128x256b(tmem + kACol + 32 + 8 * ks,
+                                                 tc::smem_desc(sbase + kSmCA + ks * 256, 128, kKS * 16));
+                    }
                 }
                 for (int i = 0; i < it.niter; ++i, ++g) {
                     const int slot = g % kSlots, st = g % kKVStages;
@@ -657,9 +703,13 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     const uint32_t dcol = tmem + slot * kSlotCols;
                     const uint32_t u_addr = sbase + kSmKV + st * kStageBytes;
 #pragma unroll
-                    for (int ks = 0; ks < kC / 16; ++ks)
-                        tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmFA + ks * 256, 128, kC * 16),
-                                     tc::smem_desc_sw128(u_addr + ks * 2048, kAtom, 1024), idesc, ks > 0);
+                    for (int ks = 0; ks < kC / 16; ++ks) {
+                        const uint64_t bdesc = tc::smem_desc_sw128(u_addr + ks * 2048, kAtom, 1024);
+                        if constexpr (G::kATmem)
+                            tc::mma_bf16_ta(dcol, tmem + kACol + 8 * ks, bdesc, idesc, ks > 0);
+                        else
+                            tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmFA + ks * 256, 128, kC * 16), bdesc, idesc, ks > 0);
+                    }
                     tc::mma_commit(bar(kBarWDone + slot));
                     tc::mma_commit(bar(kBarKVEmpty + st));
                     if (i >= it.n1) {
@@ -702,9 +752,13 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     const uint32_t dcol = tmem + slot * kSlotCols + kNC;
                     const uint32_t sb_addr = sbase + kSmS + sb * kSBytes;
 #pragma unroll
-                    for (int ks = 0; ks < kKS / 16; ++ks)
-                        tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmCA + ks * 256, 128, kKS * 16),
-                                     tc::smem_desc_sw128(sb_addr + ks * 2048, kKS * 128, 1024), idesc, ks > 0);
+                    for (int ks = 0; ks < kKS / 16; ++ks) {
+                        const uint64_t bdesc = tc::smem_desc_sw128(sb_addr + ks * 2048, kKS * 128, 1024);
+                        if constexpr (G::kATmem)
+                            tc::mma_bf16_ta(dcol, tmem + kACol + 32 + 8 * ks, bdesc, idesc, ks > 0);
+                        else
+                            tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmCA + ks * 256, 128, kKS * 16), bdesc, idesc, ks > 0);
+                    }
                     tc::mma_commit(bar(kBarYDone + slot));
                     tc::mma_commit(bar(kBarSTFree + sb));
                     *carry_issued = pc + 1;
@@ -729,16 +783,13 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int st = g % kKVStages;
                 if (!(ok = uni(tc::mbar_wait(bar(kBarKVFull + st), (g / kKVStages) & 1, abort)))) break;
                 uint8_t *kt = sm + kSmKV + st * kStageBytes;
-#pragma unroll 4
-                for (int c16 = ut; c16 < kTile / 16; c16 += kUThreads) {
-                    const int off = c16 * 16;               // same byte offset in k, v and U
-                    const uint4 kk = *reinterpret_cast<const uint4 *>(kt + off);
-                    const uint4 vv = *reinterpret_cast<const uint4 *>(kt + kTile + off);
-                    *reinterpret_cast<uint4 *>(kt + off) = make_uint4(mul_bf16x2(kk.x, vv.x), mul_bf16x2(kk.y, vv.y),
-                                                                       mul_bf16x2(kk.z, vv.z), mul_bf16x2(kk.w, vv.w));
-                }
+                // state-only iterations: the E group takes part (it has no epilogue to run there);
+                // full-pass iterations: the U group alone, thread 0 arriving for the E group too
+                const bool shared = i < it.n1;
+                form_u<kTile>(kt, ut, shared ? kUHelp : kUThreads);
                 tc::fence_proxy_async_smem();
-                tc::mbar_arrive(bar(kBarURdy + st));
+                if (!shared && ut == 0) tc::mbar_arrive_cnt(bar(kBarURdy + st), 1 + kEThreads);
+                else tc::mbar_arrive(bar(kBarURdy + st));
             }
         }
         if (!ok) record_error(a, abort, kErrWait);
@@ -928,7 +979,15 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             if (id == -2) ok = false;
             if (id < 0) break;
             const Item it = decode_item<NC>(a, id);
-            g += it.n1;
+            // state-only iterations: help the U group form U (threads kUThreads .. kUHelp - 1)
+            for (int i = 0; i < it.n1 && ok; ++i, ++g) {
+                const int st = g % kKVStages;
+                if (!(ok = uni(tc::mbar_wait(bar(kBarKVFull + st), (g / kKVStages) & 1, abort)))) break;
+                form_u<kTile>(sm + kSmKV + st * kStageBytes, kUThreads + 32 * e_index(warp) + lane, kUHelp);
+                tc::fence_proxy_async_smem();
+                tc::mbar_arrive(bar(kBarURdy + st));
+            }
+            if (!ok) break;
             for (int j = 0; j < it.nck; ++j, ++g, ++qg) {
                 const int slot = g % kSlots, s = qg % kQStages;
                 ok = uni(tc::mbar_wait(bar(kBarYDone + slot), (e2bits >> slot) & 1, abort) &&
