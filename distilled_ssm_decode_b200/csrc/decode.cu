@@ -25,7 +25,6 @@ namespace hyena {
 
 namespace {
 
-constexpr int kMaxThreads = 512;   // vector kernel: 128, 256 or 512 threads per block
 constexpr int kThreads = 256;      // scalar kernel
 constexpr int kMaxLayers = HYENA_MAX_LAYERS;
 
@@ -119,8 +118,10 @@ __device__ __forceinline__ void pdl_enter(const typename Act::T *q, const typena
     asm volatile("griddepcontrol.launch_dependents;");
 }
 
-template <class Act, int MPT>
-__global__ void __launch_bounds__(kMaxThreads)
+// NT: threads per block (128, 256 or 512), fixed at compile time so that register allocation
+// and scheduling are made for the block size each launch shape uses.
+template <class Act, int MPT, int NT>
+__global__ void __launch_bounds__(NT)
 decode_vec_kernel(const typename Act::T *__restrict__ q, const typename Act::T *__restrict__ k,
                   const typename Act::T *__restrict__ v, int B, int Dch, int ch, int d, int lg_ng,
                   const float2 *__restrict__ lam, const float2 *__restrict__ R,
@@ -144,8 +145,8 @@ struct LayerTable {
     LayerPtrs l[kMaxLayers];
 };
 
-template <class Act, int MPT>
-__global__ void __launch_bounds__(kMaxThreads)
+template <class Act, int MPT, int NT>
+__global__ void __launch_bounds__(NT)
 decode_layers_kernel(const __grid_constant__ LayerTable t, int B, int Dch, int ch, int d, int lg_ng) {
     using T = typename Act::T;
     const LayerPtrs &p = t.l[blockIdx.y];
@@ -222,8 +223,9 @@ void launch_vec(unsigned blocks, int threads, cudaStream_t s, const typename Act
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, decode_vec_kernel<Act, MPT>, q, k, v, B, Dch, ch, d, lg, lam, R, Dskip,
-                       reinterpret_cast<float4 *>(state), y);
+    auto kern = threads == 128 ? decode_vec_kernel<Act, MPT, 128>
+                : threads == 256 ? decode_vec_kernel<Act, MPT, 256> : decode_vec_kernel<Act, MPT, 512>;
+    cudaLaunchKernelEx(&cfg, kern, q, k, v, B, Dch, ch, d, lg, lam, R, Dskip, reinterpret_cast<float4 *>(state), y);
 }
 
 template <class Act, int MPT>
@@ -239,7 +241,9 @@ cudaError_t launch_layers(dim3 grid, int threads, cudaStream_t s, const LayerTab
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_layers_kernel<Act, MPT>, t, B, Dch, ch, d, lg);
+    auto kern = threads == 128 ? decode_layers_kernel<Act, MPT, 128>
+                : threads == 256 ? decode_layers_kernel<Act, MPT, 256> : decode_layers_kernel<Act, MPT, 512>;
+    return cudaLaunchKernelEx(&cfg, kern, t, B, Dch, ch, d, lg);
 }
 
 template <class Act>
