@@ -121,3 +121,21 @@ def test_chunked_unsupported_shapes_are_rejected():
     with pytest.raises(ops.HyenaError) as e:
         ops.prefill_chunked(x, x, x, lam, lam, D)                # 32 channels per head
     assert e.value.status == -5
+
+
+def test_chunked_long_prefill_full_size_sampled(oracle):
+    """The long-prefill workload as the bench runs it (B=1, L=65536, Dch=768, 12 heads of 64
+    channels, |lambda| up to 0.999, sequences split into segments joined by the look-back):
+    24 sampled channels against the oracle's recurrence over the whole prompt."""
+    w = W.WORKLOADS["long_prefill_bf16"]
+    p = W.params(w)
+    q, k, v = W.prefill_inputs(w)
+    y, s = _run(q, k, v, p)
+    rng = np.random.default_rng(11)
+    bc = sample_columns(rng, w.B, w.Dch, 24)
+    lam_c, R_c, D_c = column_params(p, w.H, w.Dch, [c for _, c in bc])
+    qc, kc, vc = gather_columns(q, bc), gather_columns(k, bc), gather_columns(v, bc)
+    y_ref, s_ref = oracle.recurrent(qc, kc, vc, lam_c, R_c, D_c, H=len(bc))
+    ey = rel_err(gather_columns(y, bc), y_ref)
+    es = rel_err(np.stack([s[b, :, c] for b, c in bc], -1)[None], s_ref)
+    assert ey <= TOL["bf16"] and es <= TOL["bf16"], (ey, es)

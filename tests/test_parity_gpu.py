@@ -293,6 +293,25 @@ def test_decode_gen_layer_after_prefill(oracle):
     assert rel_err(np.stack([sg[b, :, c] for b, c in bc], -1)[None], s_ref) <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("B,Dch,H", [(8, 1024, 8), (16, 2048, 16), (2, 1024, 8)])
+def test_decode_launch_shapes(oracle, B, Dch, H):
+    """Channel-pair counts that select the launch shapes not covered by the sweep workload
+    (4096 pairs: 8 lanes x 2 modes; 16384: 4 lanes x 2 modes; 1024: 16 lanes x 1 mode), including
+    the mid-size workload's B=8, Dch=1024; 6 steps from a random state, every element compared."""
+    w = W.Workload(600 + B, "case", B=B, L=0, Dch=Dch, H=H, d=16, dtype="bf16", fft_len=0, T=0,
+                   random_state0=True)
+    p = W.params(w)
+    lam, R, D = dev_params(p)
+    s0 = W.initial_state(w)
+    s = torch.view_as_real(s0).contiguous().cuda()
+    steps = [W.decode_inputs(w, t) for t in range(6)]
+    ys = [ops.decode_step(a.cuda(), b.cuda(), c.cuda(), lam, R, D, s).cpu() for a, b, c in steps]
+    qs, ks, vs = (W.to_f64(torch.stack([x[i] for x in steps], 1)) for i in range(3))
+    y_ref, s_ref = oracle.recurrent(qs, ks, vs, p.lam, p.R, p.Dskip, H=H, state=s0.to(torch.complex128).numpy())
+    assert rel_err(torch.stack(ys, 1).double().numpy(), y_ref) <= TOL["bf16"]
+    assert rel_err(state_c128(s), s_ref) <= TOL["bf16"]
+
+
 @pytest.mark.parametrize("Dch,H,dt", [(9, 3, "f32"), (6, 2, "bf16"), (7, 7, "bf16")])
 def test_decode_scalar_layouts(oracle, Dch, H, dt):
     """Odd channel counts take the one-channel-per-thread kernel."""
