@@ -464,30 +464,13 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    // launched as a programmatic dependent of the constants kernel: the set-up above overlapped
-    // it, and so do L2 prefetches of the first tiles of the item this CTA will most likely take
-    // first (the ticket blockIdx / H of head blockIdx % H; a prefetch has no effect on results,
-    // so a wrong guess costs nothing but bandwidth).  The constants and the cleared schedule
-    // words are visible after the wait.
-    if ((warp == kWarpKV || warp == kWarpQ) && lane == 0 && (int)blockIdx.x / a.H < a.ih) {
-        const Item it = decode_item<NC>(a, (blockIdx.x % a.H) * a.ih + blockIdx.x / a.H);
-        const bool kv = warp == kWarpKV;
-        const int n = kv ? min(it.niter, kKVStages) : min(it.nck, kQStages);
-        for (int i = 0; i < n; ++i) {
-            const int chunk = it.ck0 + (kv && i < it.n1 ? i : (kv ? i - it.n1 : i));
-            const int tok = a.tok_base + chunk * kC;
-            if (tok < 0) continue;
-            for (int h = 0; h < kNC / 64; ++h) {
-                if (kv) {
-                    tc::tma_prefetch_3d(&tm_k, it.c0 + 64 * h, tok, it.b);
-                    tc::tma_prefetch_3d(&tm_v, it.c0 + 64 * h, tok, it.b);
-                } else {
-                    tc::tma_prefetch_3d(&tm_q, it.c0 + 64 * h, tok, it.b);
-                }
-            }
-        }
-    }
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // Launched as a programmatic dependent of the constants kernel: the set-up above overlapped it.
+    // The loaders and the U group touch only their inputs and shared memory, so they start at
+    // once: each CTA's first item has a fixed ticket (blockIdx / H of head blockIdx % H), so its
+    // tiles can be loaded and U formed while the constants are still being built.  Every other
+    // role, and the k,v loader before its first counted ticket, waits here until the constants
+    // and the cleared schedule words are visible.
+    if (!(warp == kWarpKV || warp == kWarpQ || u_index(warp) >= 0)) asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint32_t tmem = (uint32_t)misc[1];
     const int d = a.d;
     auto uni = [&](bool x) -> bool { return __all_sync(0xffffffffu, x && !*abort); };
@@ -511,7 +494,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // ------------------------------------------------------------ k,v loads + tickets
         if (lane == 0) {
             int g = 0, head = blockIdx.x % a.H, tries = 0;
-            bool ok = true;
+            bool ok = true, counted = false;
             const uint64_t pol_keep = tc::l2_policy_evict_last(), pol_drop = tc::l2_policy_evict_first();
             for (int k = 0; ok; ++k) {
                 const int s = k % kItemQ;
@@ -519,13 +502,24 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     ok = false;
                     break;
                 }
-                // tickets of this CTA's head first; when they run out, move on to the next head
+                // tickets of this CTA's head first; when they run out, move on to the next head.  The
+                // first item's ticket is fixed (blockIdx / H); the counter of head h hands out the
+                // tickets after the fixed ones of the CTAs assigned to h.
                 int id = -1;
-                while (tries < a.H) {
-                    const int t = atomicAdd(a.tickets + head, 1);
-                    if (t < a.ih) { id = head * a.ih + t; tries = 0; break; }
-                    head = head + 1 == a.H ? 0 : head + 1;
-                    ++tries;
+                if (k == 0 && (int)blockIdx.x / a.H < a.ih) {
+                    id = head * a.ih + (int)blockIdx.x / a.H;
+                } else {
+                    if (!counted) {
+                        asm volatile("griddepcontrol.wait;" ::: "memory");
+                        counted = true;
+                    }
+                    while (tries < a.H) {
+                        const int fixed = head < (int)gridDim.x ? min(a.ih, ((int)gridDim.x - head + a.H - 1) / a.H) : 0;
+                        const int t = atomicAdd(a.tickets + head, 1) + fixed;
+                        if (t < a.ih) { id = head * a.ih + t; tries = 0; break; }
+                        head = head + 1 == a.H ? 0 : head + 1;
+                        ++tries;
+                    }
                 }
                 itemq[s] = id;
                 tc::mbar_arrive(bar(kBarItemFull + s));
