@@ -22,26 +22,30 @@
 // token 0 (its missing tokens are zero-filled by TMA and contribute nothing)
 // and the state after the last chunk is exactly the state after token L-1.
 //
-// Per chunk and 128-channel tile the tensor cores evaluate, in bf16 with fp32
-// accumulation in tensor memory (rows on MMA M, the 128 channels on MMA N):
+// Per chunk and channel tile (NC = 128 or 64 channels) the tensor cores evaluate, in bf16 with
+// fp32 accumulation in tensor memory (rows on MMA M, the NC channels on MMA N):
 //   fused:  [Z; W] = [T; V] U          T[tau][iota] = h_{tau-iota} (iota <= tau)
 //                                      V[r][iota]   = (Re | Im) lambda_r^(C-1-iota)
 //   carry:  Z     += A S               A[tau][r]    = (Re | -Im) R_r lambda_r^tau
-// where U[iota][c] = k v is formed elementwise over the TMA'd k tile (its
-// natural [token][channel] 128-byte-swizzled layout is already an MN-major
-// operand), S[r][c] = (Re | Im) s(t0) and W[r][c] is the chunk's state
-// contribution.  The state chain s <- lambda^C s + W runs on the CUDA cores in
-// fp32 (one thread per state row and 32 channels), and y = q Z is gated and
-// stored per token row.  The carry accumulates into TMEM columns of its own, so
-// the state rows W are never touched while the chain reads them.
+// where U[iota][c] = k v is formed elementwise (packed bf16 products) over the TMA'd k tile
+// (its natural [token][channel] 128-byte-swizzled layout is already an MN-major operand),
+// S[r][c] = (Re | Im) s(t0) and W[r][c] is the chunk's state contribution.  The two A
+// operands are per-head constants: the 64-channel tile keeps them in tensor memory (copied
+// there once per head), the 128-channel tile reads them from shared memory.  The state chain
+// s <- lambda^C s + W runs on the CUDA cores in fp32 (one thread per state row and NC/4
+// channels), and y = q (Z + carry) is gated and stored per token row.  The carry accumulates
+// into tensor-memory columns of its own, so the state rows W are never touched while the chain
+// reads them.
 //
 // Work split: a sequence is cut into segments of whole chunks; each
-// (batch, channel tile, segment) item first runs a state-only pass (k, v and the
-// fused product) to publish its segment's state contribution, then obtains the
+// (batch, channel tile, segment) item but the last of its sequence first runs a
+// state-only pass (k, v and the fused product) to publish its segment's state
+// contribution, then (segments after the first) obtains the
 // state entering its segment by a decoupled look-back over its predecessors'
 // published contributions (bounded polls), then runs the full pass.  The grid is
-// persistent: each CTA takes items from an atomic ticket in order and its
-// pipelines run on across item boundaries.  Tickets are segment-major (all
+// persistent: each CTA's first item has a fixed ticket, later ones come from a
+// per-head atomic ticket counter, and its pipelines run on across item
+// boundaries.  Tickets are segment-major (all
 // units' first segments, then all second segments, ...), so an item's
 // predecessors were handed out a whole round of units earlier and have usually
 // published by the time it looks back.  An item only ever waits on items with
@@ -71,7 +75,6 @@ constexpr int kItemQ = 4;           // item ids handed from the k,v loader to th
 constexpr int kThreads = 512;
 constexpr int kMaxSeg = 128;        // segments per sequence (bounds look-back walks)
 constexpr int kPubQ = 4;            // segment states written and waiting for their status word
-constexpr int kCQ = 4;              // items whose carries the MMA thread still owes
 constexpr uint32_t kTmemCols = 512; // all of tensor memory (one CTA per SM)
 // item readers: q loader, store lane, fused and carry MMA lanes (1 each) + lane 0 of the 3 U,
 // 4 S and 4 E warps
@@ -440,7 +443,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     auto bar = [&](int slot) { return sbase + kSmBar + 8u * slot; };
     volatile int *itemq = reinterpret_cast<volatile int *>(sm + kSmMisc);   // [kItemQ]
     volatile int *misc = itemq + kItemQ;                                     // abort, tmem, never
-    volatile int *pubq = misc + 4 + 3 * kCQ;                                 // [kPubQ]: 4 item + code, -1 = end
+    volatile int *pubq = misc + 16;                                          // [kPubQ]: 4 item + code, -1 = end
     volatile int *carry_issued = pubq + kPubQ;                               // carries issued so far
     volatile int *abort = misc;
     volatile int *never = misc + 2;
