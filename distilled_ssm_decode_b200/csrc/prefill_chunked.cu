@@ -318,9 +318,9 @@ __device__ __forceinline__ float2 cfpow(float2 lam, long long m) {
 }
 
 // It also clears the main kernel's schedule words (`zero`, `nzero` ints: error word, ticket
-// counters, segment status words), and lets the main kernel launch at once (programmatic
-// dependent launch): the main kernel's prologue overlaps this kernel, and its
-// griddepcontrol.wait returns once everything written here is visible.
+// counters, segment status words), and allows the main kernel to launch at once (programmatic
+// dependent launch): where the main kernel's CTAs find room early, their set-up and first loads
+// overlap this kernel; its griddepcontrol.wait returns once everything written here is visible.
 __global__ void __launch_bounds__(256)
 chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R,
                     const float *__restrict__ Dskip, int d, int seg_tokens,

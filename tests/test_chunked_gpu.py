@@ -139,3 +139,18 @@ def test_chunked_long_prefill_full_size_sampled(oracle):
     ey = rel_err(gather_columns(y, bc), y_ref)
     es = rel_err(np.stack([s[b, :, c] for b, c in bc], -1)[None], s_ref)
     assert ey <= TOL["bf16"] and es <= TOL["bf16"], (ey, es)
+
+
+def test_chunked_is_deterministic_with_many_items():
+    """1024 items on the persistent grid (the 1.3B-shaped layer): each CTA's first item has a fixed
+    ticket, the rest are handed out by counters, so which CTA takes which item (and switches heads
+    when) varies from run to run; the outputs must not: repeated runs are bitwise identical."""
+    w = W.WORKLOADS["gen1p3b_bf16"]
+    p = W.params(w)
+    q, k, v = (t.cuda() for t in W.prefill_inputs(w, B=64, L=512))
+    lam, R, D = dev_params(p)
+    y1, s1, ws = ops.prefill_chunked(q, k, v, lam, R, D)
+    for _ in range(3):
+        y2, s2, _ = ops.prefill_chunked(q, k, v, lam, R, D, workspace=ws)
+        assert torch.equal(y1, y2) and torch.equal(s1, s2)
+    assert ops.chunked_error(ws, w.B, w.L, w.Dch, w.H, w.d) == 0
