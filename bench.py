@@ -658,10 +658,22 @@ def run_layers(args, nl: int):
     ls = ops.LayerSet(lams, Rs, Ds, states)
     stream = torch.cuda.Stream(dev)
 
+    # the layers are independent: alternate them over two streams (a workspace each), so that one
+    # layer's start and end overlap its neighbour's instead of idling SMs
+    pstreams = [torch.cuda.Stream(dev) for _ in range(2)]
+    pws = [ws, torch.empty_like(ws)]
+
     def prefill_all():
+        cur = torch.cuda.current_stream(dev)
+        for ps in pstreams:
+            ps.wait_stream(cur)
         for l in range(nl):
             q, k, v = qkv[l]
-            ops.prefill_chunked(q, k, v, lams[l], Rs[l], Ds[l], y=ys[l], state=states[l], workspace=ws)
+            with torch.cuda.stream(pstreams[l % 2]):
+                ops.prefill_chunked(q, k, v, lams[l], Rs[l], Ds[l], y=ys[l], state=states[l],
+                                    workspace=pws[l % 2])
+        for ps in pstreams:
+            cur.wait_stream(ps)
 
     def decode_all():
         for t in range(w.T):
@@ -711,9 +723,10 @@ def run_layers(args, nl: int):
     pre_ms = reduce_max(sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps, dev)
     dec_ms = reduce_max(sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps, dev)
     ms_per_step = elapsed_ms / args.steps
-    err = ops.chunked_error(ws, w.B, w.L, w.Dch, w.H, w.d)
-    if err:
-        raise SystemExit(f"chunked prefill kernel reported error {err}")
+    for wsx in pws:
+        err = ops.chunked_error(wsx, w.B, w.L, w.Dch, w.H, w.d)
+        if err:
+            raise SystemExit(f"chunked prefill kernel reported error {err}")
 
     peak, peak_src = load_peaks()
     pb, db = algorithmic_bytes(w)

@@ -182,6 +182,8 @@ int hyena_prefill_noalloc(const void *q, const void *k, const void *v, int dtype
  *   Implemented for: dtype HYENA_BF16, Dch/H a multiple of 64, d <= 16, all
  *   activation pointers 16-byte aligned; HYENA_ERR_UNSUPPORTED otherwise.
  *   workspace: >= hyena_prefill_chunked_workspace_bytes() bytes, 256-byte aligned.
+ *   Calls on different streams may run at the same time (for instance independent
+ *   layers), each with its own workspace.
  *   The int32 at byte offset hyena_prefill_chunked_error_offset() of the
  *   workspace is 0 after a successful run; a nonzero value means a bounded
  *   wait inside the kernel gave up (the outputs are then invalid).  Read it
