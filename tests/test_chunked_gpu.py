@@ -154,3 +154,62 @@ def test_chunked_is_deterministic_with_many_items():
         y2, s2, _ = ops.prefill_chunked(q, k, v, lam, R, D, workspace=ws)
         assert torch.equal(y1, y2) and torch.equal(s1, s2)
     assert ops.chunked_error(ws, w.B, w.L, w.Dch, w.H, w.d) == 0
+
+
+def test_chunked_empty_inputs():
+    lam = torch.zeros(2, 4, 2, device="cuda")
+    D = torch.zeros(2, device="cuda")
+    # empty prompt: the state is zero
+    x = torch.empty(2, 0, 128, dtype=torch.bfloat16, device="cuda")
+    s = torch.full((2, 4, 128, 2), 7.0, device="cuda")
+    ops.prefill_chunked(x, x, x, lam, lam, D, state=s)
+    assert torch.all(s == 0)
+    # no sequences: nothing to do
+    x = torch.empty(0, 64, 128, dtype=torch.bfloat16, device="cuda")
+    ops.prefill_chunked(x, x, x, lam, lam, D, state=torch.empty(0, 4, 128, 2, device="cuda"))
+    torch.cuda.synchronize()
+
+
+def test_chunked_degenerate_poles(oracle):
+    """Poles at 0 (lambda^0 = 1 only: a two-tap filter, no carry beyond one token) and poles at
+    |lambda| = 0.9999 (almost no decay over the 3000-token prompt, sequence split into segments)
+    mixed in one head; every element against the oracle's recurrence."""
+    w = W.Workload(777, "case", B=1, L=3000, Dch=128, H=1, d=6, dtype="bf16", fft_len=0, T=0)
+    p = W.params(w)
+    lam = p.lam.copy()
+    lam[0, 0] = 0.0
+    lam[0, 1] = 0.0
+    lam[0, 2] = np.complex64(0.9999 * np.exp(0.3j))
+    lam[0, 3] = np.complex64(-0.9999)
+    p = W.Params(lam.astype(np.complex64).astype(np.complex128), p.R, p.Dskip)
+    q, k, v = W.prefill_inputs(w)
+    y, s = _run(q, k, v, p)
+    y_ref, s_ref = oracle.recurrent(W.to_f64(q), W.to_f64(k), W.to_f64(v), p.lam, p.R, p.Dskip, H=1)
+    ey, es = rel_err(y.double().numpy(), y_ref), rel_err(s, s_ref)
+    assert ey <= TOL["bf16"] and es <= TOL["bf16"], (ey, es)
+
+
+def test_mid_workload_flow_chunked_then_decode(oracle):
+    """The default benchmark's flow at full size (B=8, L=4096, Dch=1024, H=8, d=16): chunked
+    prefill, then 8 decode steps from its state; 24 sampled channels against the oracle's
+    recurrence over prompt + generated tokens."""
+    w = W.WORKLOADS["mid_bf16"]
+    p = W.params(w)
+    q, k, v = W.prefill_inputs(w)
+    lam, R, D = dev_params(p)
+    _, s, ws = ops.prefill_chunked(q.cuda(), k.cuda(), v.cuda(), lam, R, D)
+    T = 8
+    bc = sample_columns(np.random.default_rng(5), w.B, w.Dch, 24)
+    ib = torch.tensor([b for b, _ in bc]); ic = torch.tensor([c for _, c in bc])
+    ys, qs, ks, vs = [], [], [], []
+    for t in range(T):
+        a, b, c = W.decode_inputs(w, t)
+        ys.append(ops.decode_step(a.cuda(), b.cuda(), c.cuda(), lam, R, D, s).cpu()[ib, ic])
+        qs.append(a[ib, ic]); ks.append(b[ib, ic]); vs.append(c[ib, ic])
+    assert ops.chunked_error(ws, w.B, w.L, w.Dch, w.H, w.d) == 0
+    lam_c, R_c, D_c = column_params(p, w.H, w.Dch, [c for _, c in bc])
+    qa = np.concatenate([gather_columns(q, bc), W.to_f64(torch.stack(qs))[None]], 1)
+    ka = np.concatenate([gather_columns(k, bc), W.to_f64(torch.stack(ks))[None]], 1)
+    va = np.concatenate([gather_columns(v, bc), W.to_f64(torch.stack(vs))[None]], 1)
+    y_ref, s_ref = oracle.recurrent(qa, ka, va, lam_c, R_c, D_c, H=len(bc))
+    assert rel_err(torch.stack(ys).double().numpy()[None], y_ref[:, w.L:]) <= TOL["bf16"]

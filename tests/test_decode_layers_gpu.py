@@ -134,3 +134,34 @@ def test_layers_rejects_bad_arguments():
     with pytest.raises(ops.HyenaError) as e:          # activations not aligned to a channel pair
         ops.decode_step_layers(ls, mis, q, q, y)
     assert e.value.status == -3
+
+
+def test_layers_flow_chunked_prefill_then_grouped_decode(oracle):
+    """The 24-layer benchmark's flow on 3 small layers: each layer's chunked prefill, then grouped
+    decode steps over all layers from those states; every element against the oracle."""
+    w = W.Workload(480, "case", B=2, L=300, Dch=128, H=2, d=8, dtype="bf16", fft_len=0, T=0)
+    layers, T = 3, 4
+    ps = [W.params(w, layer=l) for l in range(layers)]
+    prompts = [W.prefill_inputs(w, layer=l) for l in range(layers)]
+    steps = [[W.decode_inputs(w, t, layer=l) for t in range(T)] for l in range(layers)]
+    lams, Rs, Ds, states = [], [], [], []
+    for l in range(layers):
+        lam, R, D = dev_params(ps[l])
+        _, s, _ = ops.prefill_chunked(*(x.cuda() for x in prompts[l]), lam, R, D)
+        lams.append(lam); Rs.append(R); Ds.append(D); states.append(s)
+    ls = ops.LayerSet(lams, Rs, Ds, states)
+    ys = []
+    for t in range(T):
+        yo = [torch.empty(w.B, w.Dch, dtype=torch.bfloat16, device="cuda") for _ in range(layers)]
+        ops.decode_step_layers(ls, [steps[l][t][0].cuda() for l in range(layers)],
+                               [steps[l][t][1].cuda() for l in range(layers)],
+                               [steps[l][t][2].cuda() for l in range(layers)], yo)
+        ys.append([y.cpu() for y in yo])
+    for l in range(layers):
+        qa = np.concatenate([W.to_f64(prompts[l][0]), W.to_f64(torch.stack([x[0] for x in steps[l]], 1))], 1)
+        ka = np.concatenate([W.to_f64(prompts[l][1]), W.to_f64(torch.stack([x[1] for x in steps[l]], 1))], 1)
+        va = np.concatenate([W.to_f64(prompts[l][2]), W.to_f64(torch.stack([x[2] for x in steps[l]], 1))], 1)
+        y_ref, s_ref = oracle.recurrent(qa, ka, va, ps[l].lam, ps[l].R, ps[l].Dskip, H=w.H)
+        y_gpu = torch.stack([ys[t][l] for t in range(T)], 1).double().numpy()
+        assert rel_err(y_gpu, y_ref[:, w.L:]) <= TOL["bf16"], l
+        assert rel_err(state_c128(states[l]), s_ref) <= TOL["bf16"], l

@@ -312,6 +312,22 @@ def test_decode_launch_shapes(oracle, B, Dch, H):
     assert rel_err(state_c128(s), s_ref) <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("B,Dch,H,d,dt", [(3, 64, 2, 64, "f32"), (2, 256, 4, 64, "bf16"), (5, 96, 3, 33, "bf16")])
+def test_decode_many_modes(oracle, B, Dch, H, d, dt):
+    """Mode counts up to the maximum (64) and an odd one above 32: every element, 5 steps."""
+    w = W.Workload(650 + d, "case", B=B, L=0, Dch=Dch, H=H, d=d, dtype=dt, fft_len=0, T=0, random_state0=True)
+    p = W.params(w)
+    lam, R, D = dev_params(p)
+    s0 = W.initial_state(w)
+    s = torch.view_as_real(s0).contiguous().cuda()
+    steps = [W.decode_inputs(w, t) for t in range(5)]
+    ys = [ops.decode_step(a.cuda(), b.cuda(), c.cuda(), lam, R, D, s).cpu() for a, b, c in steps]
+    qs, ks, vs = (W.to_f64(torch.stack([x[i] for x in steps], 1)) for i in range(3))
+    y_ref, s_ref = oracle.recurrent(qs, ks, vs, p.lam, p.R, p.Dskip, H=H, state=s0.to(torch.complex128).numpy())
+    assert rel_err(torch.stack(ys, 1).double().numpy(), y_ref) <= TOL[dt]
+    assert rel_err(state_c128(s), s_ref) <= TOL[dt]
+
+
 @pytest.mark.parametrize("Dch,H,dt", [(9, 3, "f32"), (6, 2, "bf16"), (7, 7, "bf16")])
 def test_decode_scalar_layouts(oracle, Dch, H, dt):
     """Odd channel counts take the one-channel-per-thread kernel."""
