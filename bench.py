@@ -453,6 +453,10 @@ def run_ours(args):
                       "peak_source": peak_src, "algorithmic_bytes": db,
                       "launch_ms": dec_launch_ms, "total_ms": dec_ms,
                       "traffic": ncu_traffic("decode", f"{w.name}/B{w.B}")})
+        st_bytes = state.numel() * 4
+        if st_bytes < 100 << 20:
+            roofs[-1]["note"] = (f"the {st_bytes / 2**20:.1f} MiB state stays in L2 between steps, so a step reads "
+                                 "no DRAM and is bound by launch and L2 latency; the HBM fraction is not its bound")
         out_dec = {"tokens_per_s": world * w.B * w.T / (dec_ms / 1e3),
                    "ms_per_token_step": dec_launch_ms, "hbm_frac": dec_gbs / peak}
     if use_chunked:
