@@ -286,16 +286,27 @@ __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
 }
 
 // U = k v in place over the k half of a k,v stage (the same byte offset in k, v and U), 16 bytes
-// per step: thread `t` of `nthreads` takes every nthreads-th 16-byte piece.
-template <int kTileBytes>
-__device__ __forceinline__ void form_u(uint8_t *kt, int t, int nthreads) {
-#pragma unroll 4
-    for (int c16 = t; c16 < kTileBytes / 16; c16 += nthreads) {
-        const int off = c16 * 16;
-        const uint4 kk = *reinterpret_cast<const uint4 *>(kt + off);
-        const uint4 vv = *reinterpret_cast<const uint4 *>(kt + kTileBytes + off);
-        *reinterpret_cast<uint4 *>(kt + off) =
-            make_uint4(mul_bf16x2(kk.x, vv.x), mul_bf16x2(kk.y, vv.y), mul_bf16x2(kk.z, vv.z), mul_bf16x2(kk.w, vv.w));
+// per piece: thread `t` of kThreads takes pieces t, t + kThreads, ...  Every load is issued
+// before the first product, so a thread waits for one shared-memory round trip, not one per
+// piece (the latency is long while TMA and the tensor cores also use shared memory).
+template <int kTileBytes, int kThreads>
+__device__ __forceinline__ void form_u(uint8_t *kt, int t) {
+    constexpr int kPieces = kTileBytes / 16, kPer = (kPieces + kThreads - 1) / kThreads;
+    uint4 kk[kPer], vv[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int off = (t + i * kThreads) * 16;
+        if (i < kPer - 1 || t + i * kThreads < kPieces) {
+            kk[i] = *reinterpret_cast<const uint4 *>(kt + off);
+            vv[i] = *reinterpret_cast<const uint4 *>(kt + kTileBytes + off);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int off = (t + i * kThreads) * 16;
+        if (i < kPer - 1 || t + i * kThreads < kPieces)
+            *reinterpret_cast<uint4 *>(kt + off) = make_uint4(mul_bf16x2(kk[i].x, vv[i].x), mul_bf16x2(kk[i].y, vv[i].y),
+                                                              mul_bf16x2(kk[i].z, vv[i].z), mul_bf16x2(kk[i].w, vv[i].w));
     }
 }
 
@@ -783,7 +794,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 // state-only iterations: the E group takes part (it has no epilogue to run there);
                 // full-pass iterations: the U group alone, thread 0 arriving for the E group too
                 const bool shared = i < it.n1;
-                form_u<kTile>(kt, ut, shared ? kUHelp : kUThreads);
+                if (shared) form_u<kTile, kUHelp>(kt, ut);
+                else form_u<kTile, kUThreads>(kt, ut);
                 tc::fence_proxy_async_smem();
                 if (!shared && ut == 0) tc::mbar_arrive_cnt(bar(kBarURdy + st), 1 + kEThreads);
                 else tc::mbar_arrive(bar(kBarURdy + st));
@@ -980,7 +992,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             for (int i = 0; i < it.n1 && ok; ++i, ++g) {
                 const int st = g % kKVStages;
                 if (!(ok = uni(tc::mbar_wait(bar(kBarKVFull + st), (g / kKVStages) & 1, abort)))) break;
-                form_u<kTile>(sm + kSmKV + st * kStageBytes, kUThreads + 32 * e_index(warp) + lane, kUHelp);
+                form_u<kTile, kUHelp>(sm + kSmKV + st * kStageBytes, kUThreads + 32 * e_index(warp) + lane);
                 tc::fence_proxy_async_smem();
                 tc::mbar_arrive(bar(kBarURdy + st));
             }
@@ -1000,6 +1012,15 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 for (int x = 0; x < kNC / 64; ++x) {
                     const int cbase = hh * (kNC / 2) + 32 * x;      // first of 32 channels
                     uint8_t *qrow = sm + kSmQ + s * kTile + (cbase / 64) * kAtom + tau * 128;
+                    // the four q pieces (16 bytes = 8 channels each) are loaded before the tensor-memory
+                    // reads and before any y piece overwrites its slot, so the round trips overlap
+                    uint4 *qp[4], qvs[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int chunk16 = ((cbase & 63) >> 3) + i;
+                        qp[i] = reinterpret_cast<uint4 *>(qrow + ((chunk16 ^ (tau & 7)) << 4));
+                        qvs[i] = *qp[i];
+                    }
                     float z[32], cz[32];
                     const uint32_t col = tmem + lane_base + slot * kSlotCols + cbase;
                     tc::tmem_ld32(col, z);
@@ -1007,9 +1028,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     tc::tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const int chunk16 = ((cbase & 63) >> 3) + i;   // 16-byte chunk (8 channels) of the row
-                        uint4 *qp = reinterpret_cast<uint4 *>(qrow + ((chunk16 ^ (tau & 7)) << 4));
-                        const uint4 qv = *qp;
+                        const uint4 qv = qvs[i];
                         const float *zz = z + 8 * i, *cc = cz + 8 * i;
                         uint4 yv;
                         yv.x = pack_bf16(bf_lo(qv.x) * (zz[0] + cc[0]), bf_hi(qv.x) * (zz[1] + cc[1]));
@@ -1017,7 +1036,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         yv.z = pack_bf16(bf_lo(qv.z) * (zz[4] + cc[4]), bf_hi(qv.z) * (zz[5] + cc[5]));
                         yv.w = pack_bf16(bf_lo(qv.w) * (zz[6] + cc[6]), bf_hi(qv.w) * (zz[7] + cc[7]));
                         if (!store_direct)
-                            *qp = yv;
+                            *qp[i] = yv;
                         else if (row_valid)
                             *reinterpret_cast<uint4 *>(yrow + cbase + 8 * i) = yv;
                     }
