@@ -112,6 +112,10 @@ struct Geo {
     // (fused A: K = 64 -> 32 columns, carry A: K = 32 -> 16 columns).  The 128-channel tile
     // needs every column for its 2 slots and reads A from shared memory.
     static constexpr bool kATmem = NC == 64;
+    // The 64-channel tile also splits the fused products of a state-only pass between the two
+    // product issuers (there the issue work paces the pass; the 128-channel tile's code is left
+    // as it is, since its longer code measured slower without using the split).
+    static constexpr bool kDualSO = NC == 64;
     static constexpr int kSlots = kATmem ? 3 : (int)kTmemCols / kSlotCols;
     static constexpr int kACol = kSlots * kSlotCols;          // first column of A (kATmem)
     static_assert(!kATmem || kACol + 48 <= (int)kTmemCols, "tensor memory budget");
@@ -140,7 +144,9 @@ struct Geo {
     static constexpr int kBarPubEmpty = kBarPubFull + kPubQ;          // [kPubQ] status posted (1: publisher)
     static constexpr int kBarDrain = kBarPubEmpty + kPubQ;            // fused issuer's MMAs finished (commit)
     static constexpr int kBarDrainC = kBarDrain + 1;                  // carry issuer's MMAs finished (commit)
-    static constexpr int kNumBars = kBarDrainC + 1;
+    static constexpr int kBarSOFin = kBarDrainC + 1;                  // carry issuer's state-only products of an item done (commit)
+    static constexpr int kBarAReady = kBarSOFin + 1;                  // a head's A operands in place (commit, once per head switch)
+    static constexpr int kNumBars = kBarAReady + 1;
     static constexpr int kSmMisc = kSmBar + kNumBars * 8;
     static constexpr int kSmemBytes = kSmMisc + 128 + 1024;           // + ids, misc words, queues, slack
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -423,7 +429,8 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
 // Roles (warps):  0  k,v TMA loads; takes item tickets and posts them to the other roles
 //                 1  q TMA loads            12  y TMA stores, segment-state publisher (lanes 0, 1)
 //                 3  tensor memory owner and fused-product issuer (lane 0)
-//                13  carry-product issuer (lane 0)
+//                13  carry-product issuer (lane 0); with 64-channel tiles also the fused products
+//                    of the odd chunks of a state-only pass
 //                 7, 11, 15       U group: U = k v over the k tile (elementwise)
 //                 2, 6, 10, 14    S group: state rows 0..31 x NC/4 channels each; chain, publish, look-back
 //                 4, 5, 8, 9      E group: token rows 0..63 x NC/2 channels each; gate and stage y
@@ -445,7 +452,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                   kBarD1Free = G::kBarD1Free, kBarSRdy = G::kBarSRdy, kBarSTFree = G::kBarSTFree,
                   kBarItemFull = G::kBarItemFull, kBarItemEmpty = G::kBarItemEmpty, kBarConst = G::kBarConst,
                   kBarConstFree = G::kBarConstFree, kBarPubFull = G::kBarPubFull, kBarPubEmpty = G::kBarPubEmpty,
-                  kBarDrain = G::kBarDrain, kBarDrainC = G::kBarDrainC, kNumBars = G::kNumBars;
+                  kBarDrain = G::kBarDrain, kBarDrainC = G::kBarDrainC, kBarSOFin = G::kBarSOFin,
+                  kBarAReady = G::kBarAReady, kNumBars = G::kNumBars;
     constexpr int kCh = kNC / 4;        // channels of one S-group thread
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -456,6 +464,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     volatile int *misc = itemq + kItemQ;                                     // abort, tmem, never
     volatile int *pubq = misc + 16;                                          // [kPubQ]: 4 item + code, -1 = end
     volatile int *carry_issued = pubq + kPubQ;                               // carries issued so far
+    volatile int *so_items = carry_issued + 1;     // items whose state-only products of the carry issuer are done
     volatile int *abort = misc;
     volatile int *never = misc + 2;
 
@@ -463,6 +472,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         misc[0] = 0;
         misc[2] = 0;
         *carry_issued = 0;
+        *so_items = 0;
         for (int i = 0; i < kNumBars; ++i) tc::mbar_init(bar(i), G::count(i));
         tc::fence_mbar_init();
     } else if (tid == 32) {
@@ -670,8 +680,9 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     // its last completion is unambiguous), and so must this thread's own MMAs.
                     if (any) {
                         const unsigned long long t0 = tc::global_ns();
-                        while (*carry_issued < pcf && !*abort && tc::global_ns() - t0 < tc::kWaitNs) {}
-                        if (*carry_issued < pcf) { ok = false; break; }
+                        const int so_need = G::kDualSO ? k : 0;
+                        while ((*carry_issued < pcf || *so_items < so_need) && !*abort && tc::global_ns() - t0 < tc::kWaitNs) {}
+                        if (*carry_issued < pcf || *so_items < so_need) { ok = false; break; }
 #pragma unroll
                         for (int sl = 0; sl < kSlots; ++sl)
                             if (c2cnt[sl] > 0 && !tc::mbar_wait(bar(kBarYDone + sl), (c2cnt[sl] - 1) & 1, abort)) ok = false;
@@ -698,8 +709,10 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                             tc::tmem_cp_128x256b(tmem + kACol + 32 + 8 * ks,
                                                  tc::smem_desc(sbase + kSmCA + ks * 256, 128, kKS * 16));
                     }
+                    if constexpr (G::kDualSO) tc::mma_commit(bar(kBarAReady));   // for the carry issuer's state-only products
                 }
                 for (int i = 0; i < it.niter; ++i, ++g) {
+                    if (G::kDualSO && i < it.n1 && (i & 1)) continue;     // the carry issuer's (state-only, odd)
                     const int slot = g % kSlots, st = g % kKVStages;
                     if (!tc::mbar_wait(bar(kBarURdy + st), (g / kKVStages) & 1, abort) ||
                         !tc::mbar_wait(bar(kBarD2Free + slot), ((g / kSlots) & 1) ^ 1, abort) ||
@@ -739,15 +752,56 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // Z += A S for every full-pass chunk, in order, once the S group has written the state
         // entering the chunk and the chunk's fused product has finished (which also means the
         // slot's previous contents were read out).
+        //
+        // With the 64-channel tile it also issues the fused products of the odd iterations of a
+        // state-only pass (the fused issuer takes the even ones), so that the two threads' issue
+        // work overlaps.  Before the first of them it waits until the fused issuer has put the
+        // item's head operands in place (one commit per head switch; the next switch cannot
+        // complete before this item's state-only products are counted, so the phase is
+        // unambiguous).  At the end of the pass it waits for its own products and counts the item,
+        // which the fused issuer checks before it replaces the operands.
         if (lane == 0) {
             const uint32_t idesc = tc::idesc_bf16(128, kNC, true);
-            int g = 0, pc = 0;
+            int g = 0, pc = 0, sofin = 0, nsw = 0, cur_hd = -1;
+            int c2bits = 0;                 // as the fused issuer's: parity of the full-pass uses of each slot
             bool ok = true;
             for (int k = 0; ok; ++k) {
                 const int id = take_item(k, false);
                 if (id == -2) { ok = false; break; }
                 if (id < 0) break;
                 const Item it = decode_item<NC>(a, id);
+                if (it.hd != cur_hd) { cur_hd = it.hd; ++nsw; }
+                if (G::kDualSO && it.n1 > 1) {
+                    const int g0 = g;
+                    if (!tc::mbar_wait(bar(kBarAReady), (nsw - 1) & 1, abort)) { ok = false; break; }
+                    for (int i = 1; i < it.n1; i += 2) {
+                        const int gi = g0 + i, slot = gi % kSlots, st = gi % kKVStages;
+                        if (!tc::mbar_wait(bar(kBarURdy + st), (gi / kKVStages) & 1, abort) ||
+                            !tc::mbar_wait(bar(kBarD2Free + slot), ((gi / kSlots) & 1) ^ 1, abort) ||
+                            !tc::mbar_wait(bar(kBarD1Free + slot), ((c2bits >> slot) & 1) ^ 1, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        tc::tc_fence_after();
+                        const uint32_t dcol = tmem + slot * kSlotCols;
+                        const uint32_t u_addr = sbase + kSmKV + st * kStageBytes;
+#pragma unroll
+                        for (int ks = 0; ks < kC / 16; ++ks) {
+                            const uint64_t bdesc = tc::smem_desc_sw128(u_addr + ks * 2048, kAtom, 1024);
+                            if constexpr (G::kATmem)
+                                tc::mma_bf16_ta(dcol, tmem + kACol + 8 * ks, bdesc, idesc, ks > 0);
+                            else
+                                tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmFA + ks * 256, 128, kC * 16), bdesc, idesc, ks > 0);
+                        }
+                        tc::mma_commit(bar(kBarWDone + slot));
+                        tc::mma_commit(bar(kBarKVEmpty + st));
+                    }
+                    if (!ok) break;
+                    tc::mma_commit(bar(kBarSOFin));
+                    if (!tc::mbar_wait(bar(kBarSOFin), sofin & 1, abort)) { ok = false; break; }
+                    ++sofin;
+                }
+                if constexpr (G::kDualSO) *so_items = k + 1;
                 g += it.n1;
                 for (int j = 0; j < it.nck; ++j, ++g, ++pc) {
                     const int slot = g % kSlots, sb = pc % kSBufs;
@@ -770,6 +824,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     tc::mma_commit(bar(kBarYDone + slot));
                     tc::mma_commit(bar(kBarSTFree + sb));
                     *carry_issued = pc + 1;
+                    c2bits ^= 1 << slot;
                 }
             }
             if (*abort) ok = false;

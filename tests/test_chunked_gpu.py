@@ -48,6 +48,13 @@ CASES = [
     (2, 300, 128, 2, 16),     # 64-channel heads (64-channel tiles), ragged
     (1, 4096, 128, 2, 16),    # 64-channel tiles, sequences split into segments (look-back)
     (3, 1000, 192, 3, 5),     # 64-channel heads, three of them
+    # state-only passes of 2, 3, 7 and 10 chunks before the look-back: the two product issuers
+    # take alternate chunks of these passes (an even count, an odd count, both with a single
+    # chunk left over at the end)
+    (1, 8192, 128, 2, 16),
+    (1, 12000, 128, 2, 16),
+    (1, 20000, 192, 3, 16),
+    (3, 5000, 384, 6, 8),
 ]
 
 
