@@ -317,12 +317,12 @@ __device__ __forceinline__ void form_u(uint8_t *kt, int t) {
 }
 
 // ------------------------------------------------------------------ per-head constants
-// Blocks (head, part): every block of a head tabulates the head's powers and taps, and writes
-// its part of the operand rows (part 0 also the chain powers).  Every entry is a power
-// lambda_n^k with 0 <= k <= C, so the powers are
-// tabulated first (each by binary powering, all in parallel) and the operands are then filled
-// from the table.  fp32 suffices: the operands are rounded to bf16 (relative 2^-9) and the
-// chain powers lambda^C, lambda^Lseg enter an fp32 recurrence, while binary powering to an
+// One block of kConstThreads threads per head.  Every entry is a power lambda_n^k with
+// 0 <= k <= C, so the powers are tabulated first (one entry per thread, by binary powering) and
+// the taps and operands are then filled from the table, one tap and one 16-byte operand piece
+// per thread, so that no thread runs a long dependent chain (the whole kernel sits on the
+// prefill's critical path).  fp32 suffices: the operands are rounded to bf16 (relative 2^-9) and
+// the chain powers lambda^C, lambda^Lseg enter an fp32 recurrence, while binary powering to an
 // exponent below 2^31 loses at most a few tens of fp32 ulps.
 __device__ __forceinline__ float2 cfpow(float2 lam, long long m) {
     float2 r = make_float2(1.f, 0.f), b = lam;
@@ -334,63 +334,57 @@ __device__ __forceinline__ float2 cfpow(float2 lam, long long m) {
     return r;
 }
 
+constexpr int kConstThreads = 1024;
+static_assert(kConstThreads == kMaxModes * kC, "one power-table entry per thread");
+static_assert(128 * (kC / 8) == kConstThreads && 128 * (kKS / 8) <= kConstThreads, "one operand piece per thread");
+
 // It also clears the main kernel's schedule words (`zero`, `nzero` ints: error word, ticket
 // counters, segment status words), and allows the main kernel to launch at once (programmatic
 // dependent launch): where the main kernel's CTAs find room early, their set-up and first loads
 // overlap this kernel; its griddepcontrol.wait returns once everything written here is visible.
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kConstThreads)
 chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R,
                     const float *__restrict__ Dskip, int d, int seg_tokens,
                     uint8_t *__restrict__ consts, int *__restrict__ zero, int nzero) {
     asm volatile("griddepcontrol.launch_dependents;");
-    const int part = blockIdx.y, nparts = gridDim.y;
-    for (int i = (blockIdx.y * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x; i < nzero;
-         i += gridDim.x * gridDim.y * blockDim.x)
-        zero[i] = 0;
+    const int t = threadIdx.x;
+    for (int i = blockIdx.x * kConstThreads + t; i < nzero; i += gridDim.x * kConstThreads) zero[i] = 0;
     const int hd = blockIdx.x;
     uint8_t *base = consts + (size_t)hd * kConstStride;
-    __nv_bfloat16 *FA = reinterpret_cast<__nv_bfloat16 *>(base);
-    __nv_bfloat16 *CA = reinterpret_cast<__nv_bfloat16 *>(base + kFABytes);
     float2 *lamC = reinterpret_cast<float2 *>(base + kLamOff);
     float2 *lamS = lamC + kMaxModes;
-    __shared__ float2 pw[kMaxModes][kC + 1];     // lambda_n^k, zero for modes >= d
+    __shared__ float2 pw[kMaxModes][kC];         // lambda_n^k, k < C; zero for modes >= d
     __shared__ float2 ls[kMaxModes], rs[kMaxModes];   // lambda_n, R_n
     __shared__ float hs[kC];                     // filter taps h_0 .. h_{C-1}
     __shared__ float dskip;
-    // the parameters once into shared memory (one round trip; the table loops below would
-    // otherwise wait on a global load per entry)
+    if (t < kMaxModes) ls[t] = t < d ? lam[(size_t)hd * d + t] : make_float2(0.f, 0.f);
+    else if (t < 2 * kMaxModes) rs[t - kMaxModes] = t - kMaxModes < d ? R[(size_t)hd * d + t - kMaxModes] : make_float2(0.f, 0.f);
+    else if (t == 2 * kMaxModes) dskip = Dskip[hd];
+    __syncthreads();
     {
-        const int t = threadIdx.x;
-        if (t < kMaxModes) ls[t] = t < d ? lam[(size_t)hd * d + t] : make_float2(0.f, 0.f);
-        else if (t < 2 * kMaxModes) rs[t - kMaxModes] = t - kMaxModes < d ? R[(size_t)hd * d + t - kMaxModes] : make_float2(0.f, 0.f);
-        else if (t == 2 * kMaxModes) dskip = Dskip[hd];
+        const int n = t / kC, k = t % kC;
+        pw[n][k] = cfpow(ls[n], k);               // ls[n] = 0 for modes >= d: 0^0 = 1 is never read there
+        if (t < kMaxModes) lamC[t] = cfpow(ls[t], kC);
+        else if (t < 2 * kMaxModes) lamS[t - kMaxModes] = cfpow(ls[t - kMaxModes], seg_tokens);
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < kMaxModes * (kC + 1); e += blockDim.x) {
-        const int n = e / (kC + 1), k = e % (kC + 1);
-        pw[n][k] = n < d ? cfpow(ls[n], k) : make_float2(0.f, 0.f);
+    {
+        // tap j (j >= 1) = Re sum_n R_n lambda_n^(j-1): lane group of 16 threads per tap, one mode
+        // each, summed by a fixed shuffle tree (modes >= d contribute zero)
+        const int j = t >> 4, n = t & 15;
+        const float2 p = pw[n][j > 0 ? j - 1 : 0];
+        float v = n < d ? fmaf(rs[n].x, p.x, -rs[n].y * p.y) : 0.f;
+#pragma unroll
+        for (int off = 8; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (n == 0) hs[j] = j == 0 ? dskip : v;
     }
-    if (part == 0)
-        for (int n = threadIdx.x; n < kMaxModes; n += blockDim.x)
-            lamS[n] = n < d ? cfpow(ls[n], seg_tokens) : make_float2(0.f, 0.f);
-    __syncthreads();
-    for (int j = threadIdx.x; j < kC; j += blockDim.x) {
-        float acc = 0.f;
-        if (j == 0) {
-            acc = dskip;
-        } else {
-            for (int n = 0; n < d; ++n) acc += rs[n].x * pw[n][j - 1].x - rs[n].y * pw[n][j - 1].y;
-        }
-        hs[j] = acc;
-    }
-    if (part == 0)
-        for (int n = threadIdx.x; n < kMaxModes; n += blockDim.x) lamC[n] = pw[n][kC];
     __syncthreads();
     // fused A operand: rows 0..C-1 Toeplitz taps, rows C..C+31 chunk powers (Re at r < 16, Im at
-    // 16 + n), rows C+32..127 zero
-    // (each thread writes one 16-byte core-matrix row: 8 consecutive K entries of one row)
-    for (int e = part * blockDim.x + threadIdx.x; e < 128 * (kC / 8); e += nparts * blockDim.x) {
-        const int row = e / (kC / 8), io0 = 8 * (e % (kC / 8));
+    // 16 + n), rows C+32..127 zero; one 16-byte core-matrix row (8 consecutive K entries of one
+    // row) per thread
+    {
+        __nv_bfloat16 *FA = reinterpret_cast<__nv_bfloat16 *>(base);
+        const int row = t / (kC / 8), io0 = 8 * (t % (kC / 8));
         float v[8];
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
@@ -400,16 +394,17 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
                 v[x] = io <= row ? hs[row - io] : 0.f;
             } else if (row < kC + kKS) {
                 const int r = row - kC;
-                const float2 p = pw[r & (kIm - 1)][kC - 1 - io];
-                v[x] = r < kIm ? p.x : p.y;
+                const float2 q = pw[r & (kIm - 1)][kC - 1 - io];
+                v[x] = (r & (kIm - 1)) < d ? (r < kIm ? q.x : q.y) : 0.f;
             }
         }
         *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(FA) + cm_off16(row, io0, kC)) =
             make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
     }
     // carry A operand: rows 0..C-1: (Re, -Im) of R_n lambda_n^tau; rows C..127 zero
-    for (int e = part * blockDim.x + threadIdx.x; e < 128 * (kKS / 8); e += nparts * blockDim.x) {
-        const int row = e / (kKS / 8), r0 = 8 * (e % (kKS / 8));
+    if (t < 128 * (kKS / 8)) {
+        __nv_bfloat16 *CA = reinterpret_cast<__nv_bfloat16 *>(base + kFABytes);
+        const int row = t / (kKS / 8), r0 = 8 * (t % (kKS / 8));
         float v[8];
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
@@ -1146,7 +1141,6 @@ struct ChunkPlan {
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 
 constexpr int kPlanSMs = 148;
-constexpr int kConstParts = 4;  // blocks per head of the constants kernel   // the plan is made for a full B200 (any SM count runs correctly)
 
 // Channel tile and segment count.  Costs are in units of one 128-channel chunk pass: a pass of
 // an NC-channel tile costs NC/128 plus a fixed 0.1, an item 1 more, and 6 more when its sequence
@@ -1244,7 +1238,7 @@ cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, 
     const ChunkPlan p = plan(B, L, Dch, H);
     uint8_t *w = static_cast<uint8_t *>(ws);
 
-    chunk_consts_kernel<<<dim3(H, kConstParts), 256, 0, s>>>(lam, R, Dskip, d, p.segc * kC, w + p.consts_off,
+    chunk_consts_kernel<<<H, kConstThreads, 0, s>>>(lam, R, Dskip, d, p.segc * kC, w + p.consts_off,
                                           reinterpret_cast<int *>(w + p.sched_off), (int)((p.agg_off - p.sched_off) / 4));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
