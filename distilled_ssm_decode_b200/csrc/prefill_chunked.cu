@@ -34,8 +34,10 @@
 // there once per head), the 128-channel tile reads them from shared memory.  The state chain
 // s <- lambda^C s + W runs on the CUDA cores in fp32 (one thread per state row and NC/4
 // channels), and y = q (Z + carry) is gated and stored per token row.  The carry accumulates
-// into tensor-memory columns of its own, so the state rows W are never touched while the chain
-// reads them.
+// onto the fused product in the same tensor-memory columns (A's rows 64..127 are zero, so it
+// adds nothing to the state rows W); the chain reads W out before it posts the state operand
+// that lets the carry start, so the two never overlap.  A slot is thus NC columns, and up to 7
+// (64-channel tile) or 4 chunks are in flight between the products, the chain and the gate.
 //
 // Work split: a sequence is cut into segments of whole chunks; each
 // (batch, channel tile, segment) item but the last of its sequence first runs a
@@ -106,17 +108,21 @@ struct Geo {
     static constexpr int kStageBytes = 2 * kTile;             // k (overwritten by U) then v
     static constexpr int kKVStages = NC == 128 ? 4 : 8;
     static constexpr int kQStages = NC == 128 ? 3 : 6;        // q tiles; y is staged in place
-    static constexpr int kSlotCols = 2 * NC;                  // fused [NC cols] | carry [NC cols]
+    // One accumulator slot per chunk in flight: NC columns, into which the fused product writes
+    // [Z; W] and the carry product then adds A S.  The carry operand's rows 64..127 are zero, so
+    // it leaves the state rows W as they are; the S group reads them out before it posts the
+    // state operand that lets the carry start, so the two never overlap.
+    static constexpr int kSlotCols = NC;
     // The 64-channel tile keeps both A operands (constant per head) in tensor memory, so the MMAs
-    // read only their B operand from shared memory: 3 accumulator slots + 48 columns of A
+    // read only their B operand from shared memory: 7 accumulator slots + 48 columns of A
     // (fused A: K = 64 -> 32 columns, carry A: K = 32 -> 16 columns).  The 128-channel tile
-    // needs every column for its 2 slots and reads A from shared memory.
+    // gives every column to its 4 slots and reads A from shared memory.
     static constexpr bool kATmem = NC == 64;
     // The 64-channel tile also splits the fused products of a state-only pass between the two
     // product issuers (there the issue work paces the pass; the 128-channel tile's code is left
     // as it is, since its longer code measured slower without using the split).
     static constexpr bool kDualSO = NC == 64;
-    static constexpr int kSlots = kATmem ? 3 : (int)kTmemCols / kSlotCols;
+    static constexpr int kSlots = kATmem ? ((int)kTmemCols - 48) / kSlotCols : (int)kTmemCols / kSlotCols;
     static constexpr int kACol = kSlots * kSlotCols;          // first column of A (kATmem)
     static_assert(!kATmem || kACol + 48 <= (int)kTmemCols, "tensor memory budget");
     static constexpr int kSBytes = kKS * NC * 2;              // [32 rows][NC ch] bf16, 128-byte swizzled
@@ -806,15 +812,15 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         break;
                     }
                     tc::tc_fence_after();
-                    const uint32_t dcol = tmem + slot * kSlotCols + kNC;
+                    const uint32_t dcol = tmem + slot * kSlotCols;     // onto the fused product
                     const uint32_t sb_addr = sbase + kSmS + sb * kSBytes;
 #pragma unroll
                     for (int ks = 0; ks < kKS / 16; ++ks) {
                         const uint64_t bdesc = tc::smem_desc_sw128(sb_addr + ks * 2048, kKS * 128, 1024);
                         if constexpr (G::kATmem)
-                            tc::mma_bf16_ta(dcol, tmem + kACol + 32 + 8 * ks, bdesc, idesc, ks > 0);
+                            tc::mma_bf16_ta(dcol, tmem + kACol + 32 + 8 * ks, bdesc, idesc, 1);
                         else
-                            tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmCA + ks * 256, 128, kKS * 16), bdesc, idesc, ks > 0);
+                            tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmCA + ks * 256, 128, kKS * 16), bdesc, idesc, 1);
                     }
                     tc::mma_commit(bar(kBarYDone + slot));
                     tc::mma_commit(bar(kBarSTFree + sb));
@@ -890,21 +896,29 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
             for (int i = 0; i < kCh; ++i) st[i] = 0.f;
 
-            // st <- lambda^C st + W of iteration gi
-            auto advance = [&](int gi) -> bool {
+            // W of iteration gi out of its slot (then free for the next fused product)
+            auto read_w = [&](int gi, float *w) -> bool {
                 const int slot = gi % kSlots;
                 if (!uni(tc::mbar_wait(bar(kBarWDone + slot), (gi / kSlots) & 1, abort))) return false;
                 tc::tc_fence_after();
-                float w[kCh];
                 tmem_ld<kCh>(tmem + lane_base + slot * kSlotCols + kCh * q4, w);
                 tc::tmem_wait_ld();
                 tc::tc_fence_before();
                 tc::mbar_arrive(bar(kBarD2Free + slot));
+                return true;
+            };
+            // st <- lambda^C st + W
+            auto chain = [&](const float *w) {
 #pragma unroll
                 for (int i = 0; i < kCh; ++i) {
                     const float p = __shfl_xor_sync(0xffffffffu, st[i], 16);    // the other part of mode n
                     st[i] = fmaf(lamC.x, st[i], fmaf(sgn * lamC.y, p, w[i]));
                 }
+            };
+            auto advance = [&](int gi) -> bool {
+                float w[kCh];
+                if (!read_w(gi, w)) return false;
+                chain(w);
                 return true;
             };
             // this thread's row of a published [32 rows][NC ch] state (bypassing L1)
@@ -978,9 +992,12 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 }
             }
 
-            // full pass: state operand for each chunk, then the state after it
+            // full pass: the chunk's W, then the state operand entering the chunk (which lets its
+            // carry product add onto the slot), then the state after the chunk
             for (int j = 0; j < it.nck && ok; ++j, ++g, ++pc) {
                 const int sb = pc % kSBufs;
+                float w[kCh];
+                if (!(ok = read_w(g, w))) break;
                 if (!(ok = uni(tc::mbar_wait(bar(kBarSTFree + sb), ((pc / kSBufs) & 1) ^ 1, abort)))) break;
                 // row r of the MN-major, 128-byte swizzled [32 rows][NC ch] operand: this thread's
                 // channels are kCh * 2 bytes of row r in swizzle atom (kCh q4) / 64 (atoms of
@@ -999,7 +1016,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 }
                 tc::fence_proxy_async_smem();
                 tc::mbar_arrive(bar(kBarSRdy + sb));
-                if (!(ok = uni(advance(g)))) break;
+                chain(w);
             }
             if (!ok) break;
             if (it.last_seg) {
@@ -1071,20 +1088,19 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         qp[i] = reinterpret_cast<uint4 *>(qrow + ((chunk16 ^ (tau & 7)) << 4));
                         qvs[i] = *qp[i];
                     }
-                    float z[32], cz[32];
+                    float z[32];            // Z + carry: the carry product added onto the fused one
                     const uint32_t col = tmem + lane_base + slot * kSlotCols + cbase;
                     tc::tmem_ld32(col, z);
-                    tc::tmem_ld32(col + kNC, cz);
                     tc::tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const uint4 qv = qvs[i];
-                        const float *zz = z + 8 * i, *cc = cz + 8 * i;
+                        const float *zz = z + 8 * i;
                         uint4 yv;
-                        yv.x = pack_bf16(bf_lo(qv.x) * (zz[0] + cc[0]), bf_hi(qv.x) * (zz[1] + cc[1]));
-                        yv.y = pack_bf16(bf_lo(qv.y) * (zz[2] + cc[2]), bf_hi(qv.y) * (zz[3] + cc[3]));
-                        yv.z = pack_bf16(bf_lo(qv.z) * (zz[4] + cc[4]), bf_hi(qv.z) * (zz[5] + cc[5]));
-                        yv.w = pack_bf16(bf_lo(qv.w) * (zz[6] + cc[6]), bf_hi(qv.w) * (zz[7] + cc[7]));
+                        yv.x = pack_bf16(bf_lo(qv.x) * zz[0], bf_hi(qv.x) * zz[1]);
+                        yv.y = pack_bf16(bf_lo(qv.y) * zz[2], bf_hi(qv.y) * zz[3]);
+                        yv.z = pack_bf16(bf_lo(qv.z) * zz[4], bf_hi(qv.z) * zz[5]);
+                        yv.w = pack_bf16(bf_lo(qv.w) * zz[6], bf_hi(qv.w) * zz[7]);
                         if (!store_direct)
                             *qp[i] = yv;
                         else if (row_valid)
