@@ -30,8 +30,12 @@ constexpr int kMaxLayers = HYENA_MAX_LAYERS;
 
 // One decode step for the channel pairs of one layer: the thread's pair and mode slot follow
 // from gtid (its index in the layer's grid).  MPT: modes held in registers per thread per
-// iteration (all loaded before use).
-template <class Act, int MPT>
+// iteration (all loaded before use).  kEarly: the mode parameters and Dskip are loaded in the
+// same batch as the state instead of at their first use.  That shortens the dependent chain of a
+// latency-bound step (few pairs, state in L2; measured 2.03 -> 1.78 us at 4096 pairs) but costs
+// registers that the bandwidth-bound shapes need (3-6% slower there), so only the small launch
+// shapes use it.
+template <class Act, int MPT, bool kEarly>
 __device__ __forceinline__ void decode_pairs(const typename Act::T *__restrict__ q, const typename Act::T *__restrict__ k,
                                              const typename Act::T *__restrict__ v, int B, int Dch, int ch, int d,
                                              int lg_ng, const float2 *__restrict__ lam, const float2 *__restrict__ R,
@@ -56,12 +60,25 @@ __device__ __forceinline__ void decode_pairs(const typename Act::T *__restrict__
     float ua = 0.f, ub = 0.f;
     float2 qq = make_float2(0.f, 0.f);
     float acc_a = 0.f, acc_b = 0.f;
+    float D = 0.f;
+    if (kEarly && valid && g == 0) D = __ldg(&Dskip[hd]);
     for (int n0 = g; n0 < d; n0 += NG * MPT) {
         float4 s[MPT];
+        float2 re[MPT], le[MPT];
 #pragma unroll
         for (int i = 0; i < MPT; ++i) {
             const int n = n0 + i * NG;
             if (valid && n < d) s[i] = sp[(size_t)n * srow];
+        }
+        if constexpr (kEarly) {
+#pragma unroll
+            for (int i = 0; i < MPT; ++i) {
+                const int n = n0 + i * NG;
+                if (valid && n < d) {
+                    re[i] = __ldg(&rh[n]);
+                    le[i] = __ldg(&lh[n]);
+                }
+            }
         }
         if (n0 == g && valid) {   // activations: issued after the first state loads
             const size_t o = (size_t)b * Dch + c;
@@ -74,8 +91,8 @@ __device__ __forceinline__ void decode_pairs(const typename Act::T *__restrict__
         for (int i = 0; i < MPT; ++i) {
             const int n = n0 + i * NG;
             if (valid && n < d) {
-                const float2 r = __ldg(&rh[n]);
-                const float2 l = __ldg(&lh[n]);
+                const float2 r = kEarly ? re[i] : __ldg(&rh[n]);
+                const float2 l = kEarly ? le[i] : __ldg(&lh[n]);
                 acc_a = fmaf(r.x, s[i].x, fmaf(-r.y, s[i].y, acc_a));
                 acc_b = fmaf(r.x, s[i].z, fmaf(-r.y, s[i].w, acc_b));
                 float4 t;
@@ -92,7 +109,7 @@ __device__ __forceinline__ void decode_pairs(const typename Act::T *__restrict__
         acc_b += __shfl_xor_sync(0xffffffffu, acc_b, off);
     }
     if (valid && g == 0) {
-        const float D = __ldg(&Dskip[hd]);
+        if (!kEarly) D = __ldg(&Dskip[hd]);
         Act::st2(y + (size_t)b * Dch + c, qq.x * fmaf(D, ua, acc_a), qq.y * fmaf(D, ub, acc_b));
     }
 }
@@ -120,7 +137,7 @@ __device__ __forceinline__ void pdl_enter(const typename Act::T *q, const typena
 
 // NT: threads per block (128, 256 or 512), fixed at compile time so that register allocation
 // and scheduling are made for the block size each launch shape uses.
-template <class Act, int MPT, int NT>
+template <class Act, int MPT, int NT, bool kEarly>
 __global__ void __launch_bounds__(NT)
 decode_vec_kernel(const typename Act::T *__restrict__ q, const typename Act::T *__restrict__ k,
                   const typename Act::T *__restrict__ v, int B, int Dch, int ch, int d, int lg_ng,
@@ -129,7 +146,7 @@ decode_vec_kernel(const typename Act::T *__restrict__ q, const typename Act::T *
                   typename Act::T *__restrict__ y) {
     const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     pdl_enter<Act>(q, k, v, B, Dch, lg_ng, gtid);
-    decode_pairs<Act, MPT>(q, k, v, B, Dch, ch, d, lg_ng, lam, R, Dskip, state, y, gtid);
+    decode_pairs<Act, MPT, kEarly>(q, k, v, B, Dch, ch, d, lg_ng, lam, R, Dskip, state, y, gtid);
 }
 
 // Several independent layers in one launch: blockIdx.y selects the layer, whose pointers travel
@@ -145,7 +162,7 @@ struct LayerTable {
     LayerPtrs l[kMaxLayers];
 };
 
-template <class Act, int MPT, int NT>
+template <class Act, int MPT, int NT, bool kEarly>
 __global__ void __launch_bounds__(NT)
 decode_layers_kernel(const __grid_constant__ LayerTable t, int B, int Dch, int ch, int d, int lg_ng) {
     using T = typename Act::T;
@@ -153,7 +170,7 @@ decode_layers_kernel(const __grid_constant__ LayerTable t, int B, int Dch, int c
     const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const T *q = static_cast<const T *>(p.q), *k = static_cast<const T *>(p.k), *v = static_cast<const T *>(p.v);
     pdl_enter<Act>(q, k, v, B, Dch, lg_ng, gtid);
-    decode_pairs<Act, MPT>(q, k, v, B, Dch, ch, d, lg_ng, p.lam, p.R, p.Dskip, p.state, static_cast<T *>(p.y), gtid);
+    decode_pairs<Act, MPT, kEarly>(q, k, v, B, Dch, ch, d, lg_ng, p.lam, p.R, p.Dskip, p.state, static_cast<T *>(p.y), gtid);
 }
 
 // General layout (odd channels per head / odd Dch / 8-byte aligned state): one thread per channel.
@@ -223,8 +240,10 @@ void launch_vec(unsigned blocks, int threads, cudaStream_t s, const typename Act
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    auto kern = threads == 128 ? decode_vec_kernel<Act, MPT, 128>
-                : threads == 256 ? decode_vec_kernel<Act, MPT, 256> : decode_vec_kernel<Act, MPT, 512>;
+    // early parameter loads for the shapes with several lanes per pair (at most 16384 pairs)
+    auto kern = (lg >= 2 && threads == 256) ? decode_vec_kernel<Act, MPT, 256, true>
+                : threads == 128 ? decode_vec_kernel<Act, MPT, 128, false>
+                : threads == 256 ? decode_vec_kernel<Act, MPT, 256, false> : decode_vec_kernel<Act, MPT, 512, false>;
     cudaLaunchKernelEx(&cfg, kern, q, k, v, B, Dch, ch, d, lg, lam, R, Dskip, reinterpret_cast<float4 *>(state), y);
 }
 
@@ -241,8 +260,9 @@ cudaError_t launch_layers(dim3 grid, int threads, cudaStream_t s, const LayerTab
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    auto kern = threads == 128 ? decode_layers_kernel<Act, MPT, 128>
-                : threads == 256 ? decode_layers_kernel<Act, MPT, 256> : decode_layers_kernel<Act, MPT, 512>;
+    auto kern = (lg >= 2 && threads == 256) ? decode_layers_kernel<Act, MPT, 256, true>
+                : threads == 128 ? decode_layers_kernel<Act, MPT, 128, false>
+                : threads == 256 ? decode_layers_kernel<Act, MPT, 256, false> : decode_layers_kernel<Act, MPT, 512, false>;
     return cudaLaunchKernelEx(&cfg, kern, t, B, Dch, ch, d, lg);
 }
 
