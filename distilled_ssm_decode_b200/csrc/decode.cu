@@ -32,9 +32,9 @@ constexpr int kMaxLayers = HYENA_MAX_LAYERS;
 // from gtid (its index in the layer's grid).  MPT: modes held in registers per thread per
 // iteration (all loaded before use).  kEarly: the mode parameters and Dskip are loaded in the
 // same batch as the state instead of at their first use.  That shortens the dependent chain of a
-// latency-bound step (few pairs, state in L2; measured 2.03 -> 1.78 us at 4096 pairs) but costs
-// registers that the bandwidth-bound shapes need (3-6% slower there), so only the small launch
-// shapes use it.
+// latency-bound step (few pairs, state in L2; measured 2.03 -> 1.78 us at 4096 pairs, 3.81 -> 3.60
+// us at 32768) but costs registers that the bandwidth-bound shapes need (3-6% slower there), so
+// only the launches of at most 32768 pairs use it.
 template <class Act, int MPT, bool kEarly>
 __device__ __forceinline__ void decode_pairs(const typename Act::T *__restrict__ q, const typename Act::T *__restrict__ k,
                                              const typename Act::T *__restrict__ v, int B, int Dch, int ch, int d,
@@ -240,8 +240,10 @@ void launch_vec(unsigned blocks, int threads, cudaStream_t s, const typename Act
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    // early parameter loads for the shapes with several lanes per pair (at most 16384 pairs)
-    auto kern = (lg >= 2 && threads == 256) ? decode_vec_kernel<Act, MPT, 256, true>
+    // early parameter loads for the latency-bound shapes (at most 32768 pairs)
+    const bool early = (long long)blocks * threads <= (32768ll << lg);
+    auto kern = (early && threads == 256) ? decode_vec_kernel<Act, MPT, 256, true>
+                : (early && threads == 512) ? decode_vec_kernel<Act, MPT, 512, true>
                 : threads == 128 ? decode_vec_kernel<Act, MPT, 128, false>
                 : threads == 256 ? decode_vec_kernel<Act, MPT, 256, false> : decode_vec_kernel<Act, MPT, 512, false>;
     cudaLaunchKernelEx(&cfg, kern, q, k, v, B, Dch, ch, d, lg, lam, R, Dskip, reinterpret_cast<float4 *>(state), y);
