@@ -163,6 +163,25 @@ def test_chunked_is_deterministic_with_many_items():
     assert ops.chunked_error(ws, w.B, w.L, w.Dch, w.H, w.d) == 0
 
 
+@pytest.mark.parametrize("B,L,Dch,H", [(1, 65536, 768, 12), (1, 20000, 192, 3)])
+def test_chunked_is_deterministic_with_segments(B, L, Dch, H):
+    """Sequences split into segments (the long-prefill shape: 12 segments of 86 chunks; and 45
+    segments of 7): which predecessor a look-back finds with an inclusive state, and when the two
+    product issuers finish their shares of a state-only pass, vary from run to run; the outputs
+    must not: repeated runs are bitwise identical."""
+    w = W.Workload(400 + H, "segments", B=B, L=L, Dch=Dch, H=H, d=16, dtype="bf16", fft_len=0, T=0)
+    p = W.params(w)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(11)
+    q, k, v = (torch.randn((B, L, Dch), generator=g, device="cuda").to(torch.bfloat16) for _ in range(3))
+    lam, R, D = dev_params(p)
+    y1, s1, ws = ops.prefill_chunked(q, k, v, lam, R, D)
+    for _ in range(3):
+        y2, s2, _ = ops.prefill_chunked(q, k, v, lam, R, D, workspace=ws)
+        assert torch.equal(y1, y2) and torch.equal(s1, s2)
+    assert ops.chunked_error(ws, B, L, Dch, H, 16) == 0
+
+
 def test_chunked_empty_inputs():
     lam = torch.zeros(2, 4, 2, device="cuda")
     D = torch.zeros(2, device="cuda")
