@@ -19,6 +19,7 @@ from __future__ import annotations
 import argparse
 import datetime
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -91,9 +92,14 @@ LEAD_SPIN_CYCLES = 4_000_000       # ~2 ms at the B200's clock
 
 
 def source_hash(paths) -> str:
+    """Hash of the kernel sources with C/C++ comments removed and white space collapsed: a capture
+    stays valid across comment and layout edits and is dropped as soon as any code changes."""
     h = hashlib.sha256()
     for p in paths:
-        h.update(open(os.path.join(ROOT, p), "rb").read())
+        text = open(os.path.join(ROOT, p), encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

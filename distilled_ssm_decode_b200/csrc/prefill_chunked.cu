@@ -100,7 +100,8 @@ constexpr int kSmKV = kSmCA + kCABytes;                   // 1024-aligned (swizz
 
 // Layout for a channel tile of NC = 128 or 64 channels (MMA N).  The narrow tile gives twice
 // the (sequence, tile) units, so that small batches fill the GPU without splitting sequences;
-// its rings are twice as deep (same bytes) and tensor memory holds four accumulator slots.
+// its rings are twice as deep (same bytes), and it keeps its A operands in tensor memory next
+// to seven accumulator slots (the 128-channel tile has four and reads A from shared memory).
 template <int NC>
 struct Geo {
     static_assert(NC == 64 || NC == 128, "channel tile");
@@ -659,8 +660,9 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // ------------------------------------------------------------ fused-product issuer
         // [Z; W] = [T; V] U for every iteration, in order.  Its waits only involve the U
         // operand and a free accumulator slot, so it runs ahead of the state chain; the carries
-        // are issued by their own thread (the carry writes TMEM columns of its own, so the two
-        // need no mutual order).  Waits suspend in hardware (no polling loop on this thread).
+        // are issued by their own thread (a chunk's carry waits for that chunk's fused product,
+        // onto which it adds, so the two threads need no other mutual order).  Waits suspend in
+        // hardware (no polling loop on this thread).
         if (lane == 0) {
             const uint32_t idesc = tc::idesc_bf16(128, kNC, true);
             int g = 0, pcf = 0, cur_hd = -1, cphase = 0, fphase = 0;
@@ -751,8 +753,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     } else if (warp == kWarpCarry) {
         // ------------------------------------------------------------ carry issuer
         // Z += A S for every full-pass chunk, in order, once the S group has written the state
-        // entering the chunk and the chunk's fused product has finished (which also means the
-        // slot's previous contents were read out).
+        // entering the chunk (after reading the chunk's W out of the slot) and the chunk's fused
+        // product, onto which the carry adds, has finished.
         //
         // With the 64-channel tile it also issues the fused products of the odd iterations of a
         // state-only pass (the fused issuer takes the even ones), so that the two threads' issue
