@@ -68,7 +68,7 @@ const char *hyena_status_string(int status) {
         case HYENA_ERR_SHAPE: return "invalid shape (negative size, Dch % H != 0, d out of range, or bad fft_len)";
         case HYENA_ERR_ALIGN: return "pointer misaligned for the required layout";
         case HYENA_ERR_WORKSPACE: return "workspace missing or too small";
-        case HYENA_ERR_UNSUPPORTED: return "size outside what this build implements";
+        case HYENA_ERR_UNSUPPORTED: return "size outside what the library implements";
         case HYENA_ERR_CUDA: return "CUDA launch or runtime error";
         case HYENA_ERR_CAPACITY: return "problem needs more scratch than the library's built-in array holds";
         default: return "unknown status";

@@ -64,7 +64,7 @@ typedef enum {
     HYENA_ERR_SHAPE = -2,        /* negative size, Dch % H != 0, fft_len too short / not 2^k, d out of range */
     HYENA_ERR_ALIGN = -3,        /* pointer not aligned as the layout requires */
     HYENA_ERR_WORKSPACE = -4,    /* workspace NULL or smaller than the query says */
-    HYENA_ERR_UNSUPPORTED = -5,  /* valid operator, size outside what this build implements */
+    HYENA_ERR_UNSUPPORTED = -5,  /* valid operator, size outside what the library implements */
     HYENA_ERR_CUDA = -6,         /* a CUDA launch/runtime call failed */
     HYENA_ERR_CAPACITY = -7      /* problem needs more than the library's built-in scratch */
 } hyena_status;
@@ -103,7 +103,7 @@ int hyena_filter_from_modes(const float *lambda, const float *R, const float *Ds
  *   spec_out[hd][f] = sum_{j<L} h[hd][j] exp(-2 pi i j f / fft_len),  f = 0..fft_len/2
  *   h        : [H][L] fp32 device
  *   spec_out : [H][fft_len/2+1][2] fp32 device (complex64)
- * fft_len must be a power of two >= L; this build implements 64 <= fft_len
+ * fft_len must be a power of two >= L; the library implements 64 <= fft_len
  * <= 2^17 (HYENA_ERR_UNSUPPORTED otherwise).
  * workspace: device scratch of hyena_filter_spectrum_workspace_bytes() bytes,
  * 256-byte aligned.
@@ -124,7 +124,7 @@ int hyena_filter_spectrum(const float *h, int H, int L, int fft_len, float *spec
  *   fft_len    : power of two, >= 2L-1 (so the circular convolution equals the
  *                linear one on the first L outputs).  Any such length gives the
  *                same result up to rounding; lengths below 64 are raised to 64
- *                internally.  This build implements fft_len <= 2^17, B <= 65535.
+ *                internally.  The library implements fft_len <= 2^17, B <= 65535.
  *                fft_len <= 16384 runs one fused kernel per channel pair with
  *                the whole sequence in shared memory; longer transforms take a
  *                four-step route through the workspace.
