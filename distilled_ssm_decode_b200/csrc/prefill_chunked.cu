@@ -502,6 +502,34 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     auto uni = [&](bool x) -> bool { return __all_sync(0xffffffffu, x && !*abort); };
     auto tok_of = [&](int chunk) { return a.tok_base + chunk * kC; };
 
+    // The fused product [Z; W] = [T; V] U of iteration gi, once its U tile is formed and its slot
+    // has been read out by the S group and, after the slot's last full-pass use, by the E group
+    // (parity bits `c2bits` of the issuing thread); its commits mark the slot's product done and
+    // free the k,v stage.  Issued by one lane (the fused issuer, or the carry issuer for the odd
+    // chunks of a state-only pass); false if a wait gave up.
+    auto fused_product = [&](int gi, int c2bits) -> bool {
+        const int slot = gi % kSlots, st = gi % kKVStages;
+        if (!tc::mbar_wait(bar(kBarURdy + st), (gi / kKVStages) & 1, abort) ||
+            !tc::mbar_wait(bar(kBarD2Free + slot), ((gi / kSlots) & 1) ^ 1, abort) ||
+            !tc::mbar_wait(bar(kBarD1Free + slot), ((c2bits >> slot) & 1) ^ 1, abort))
+            return false;
+        tc::tc_fence_after();
+        const uint32_t idesc = tc::idesc_bf16(128, kNC, true);
+        const uint32_t dcol = tmem + slot * kSlotCols;
+        const uint32_t u_addr = sbase + kSmKV + st * kStageBytes;
+#pragma unroll
+        for (int ks = 0; ks < kC / 16; ++ks) {
+            const uint64_t bdesc = tc::smem_desc_sw128(u_addr + ks * 2048, kAtom, 1024);
+            if constexpr (G::kATmem)
+                tc::mma_bf16_ta(dcol, tmem + kACol + 8 * ks, bdesc, idesc, ks > 0);
+            else
+                tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmFA + ks * 256, 128, kC * 16), bdesc, idesc, ks > 0);
+        }
+        tc::mma_commit(bar(kBarWDone + slot));
+        tc::mma_commit(bar(kBarKVEmpty + st));
+        return true;
+    };
+
     // consumer side of the item queue: the id of the k-th item (-1 at the end), or -2 on abort.
     // `lead` threads (one per consumer role or warp) release the slot after reading it.
     // Warp-wide callers (all 32 lanes) pass warpwide = true: every lane reads before lane 0 releases.
@@ -664,7 +692,6 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // onto which it adds, so the two threads need no other mutual order).  Waits suspend in
         // hardware (no polling loop on this thread).
         if (lane == 0) {
-            const uint32_t idesc = tc::idesc_bf16(128, kNC, true);
             int g = 0, pcf = 0, cur_hd = -1, cphase = 0, fphase = 0;
             int c2bits = 0;                 // bit s: parity of the full-pass uses of slot s issued so far
             int c2cnt[kSlots];              // per-slot full-pass uses (const switches only)
@@ -716,26 +743,11 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 }
                 for (int i = 0; i < it.niter; ++i, ++g) {
                     if (G::kDualSO && i < it.n1 && (i & 1)) continue;     // the carry issuer's (state-only, odd)
-                    const int slot = g % kSlots, st = g % kKVStages;
-                    if (!tc::mbar_wait(bar(kBarURdy + st), (g / kKVStages) & 1, abort) ||
-                        !tc::mbar_wait(bar(kBarD2Free + slot), ((g / kSlots) & 1) ^ 1, abort) ||
-                        !tc::mbar_wait(bar(kBarD1Free + slot), ((c2bits >> slot) & 1) ^ 1, abort)) {
+                    const int slot = g % kSlots;
+                    if (!fused_product(g, c2bits)) {
                         ok = false;
                         break;
                     }
-                    tc::tc_fence_after();
-                    const uint32_t dcol = tmem + slot * kSlotCols;
-                    const uint32_t u_addr = sbase + kSmKV + st * kStageBytes;
-#pragma unroll
-                    for (int ks = 0; ks < kC / 16; ++ks) {
-                        const uint64_t bdesc = tc::smem_desc_sw128(u_addr + ks * 2048, kAtom, 1024);
-                        if constexpr (G::kATmem)
-                            tc::mma_bf16_ta(dcol, tmem + kACol + 8 * ks, bdesc, idesc, ks > 0);
-                        else
-                            tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmFA + ks * 256, 128, kC * 16), bdesc, idesc, ks > 0);
-                    }
-                    tc::mma_commit(bar(kBarWDone + slot));
-                    tc::mma_commit(bar(kBarKVEmpty + st));
                     if (i >= it.n1) {
                         c2bits ^= 1 << slot;
                         ++c2cnt[slot];
@@ -777,28 +789,11 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 if (G::kDualSO && it.n1 > 1) {
                     const int g0 = g;
                     if (!tc::mbar_wait(bar(kBarAReady), (nsw - 1) & 1, abort)) { ok = false; break; }
-                    for (int i = 1; i < it.n1; i += 2) {
-                        const int gi = g0 + i, slot = gi % kSlots, st = gi % kKVStages;
-                        if (!tc::mbar_wait(bar(kBarURdy + st), (gi / kKVStages) & 1, abort) ||
-                            !tc::mbar_wait(bar(kBarD2Free + slot), ((gi / kSlots) & 1) ^ 1, abort) ||
-                            !tc::mbar_wait(bar(kBarD1Free + slot), ((c2bits >> slot) & 1) ^ 1, abort)) {
+                    for (int i = 1; i < it.n1; i += 2)
+                        if (!fused_product(g0 + i, c2bits)) {
                             ok = false;
                             break;
                         }
-                        tc::tc_fence_after();
-                        const uint32_t dcol = tmem + slot * kSlotCols;
-                        const uint32_t u_addr = sbase + kSmKV + st * kStageBytes;
-#pragma unroll
-                        for (int ks = 0; ks < kC / 16; ++ks) {
-                            const uint64_t bdesc = tc::smem_desc_sw128(u_addr + ks * 2048, kAtom, 1024);
-                            if constexpr (G::kATmem)
-                                tc::mma_bf16_ta(dcol, tmem + kACol + 8 * ks, bdesc, idesc, ks > 0);
-                            else
-                                tc::mma_bf16(dcol, tc::smem_desc(sbase + kSmFA + ks * 256, 128, kC * 16), bdesc, idesc, ks > 0);
-                        }
-                        tc::mma_commit(bar(kBarWDone + slot));
-                        tc::mma_commit(bar(kBarKVEmpty + st));
-                    }
                     if (!ok) break;
                     tc::mma_commit(bar(kBarSOFin));
                     if (!tc::mbar_wait(bar(kBarSOFin), sofin & 1, abort)) { ok = false; break; }
