@@ -293,11 +293,13 @@ def test_decode_gen_layer_after_prefill(oracle):
     assert rel_err(np.stack([sg[b, :, c] for b, c in bc], -1)[None], s_ref) <= TOL["bf16"]
 
 
-@pytest.mark.parametrize("B,Dch,H", [(8, 1024, 8), (16, 2048, 16), (2, 1024, 8)])
+@pytest.mark.parametrize("B,Dch,H", [(8, 1024, 8), (16, 2048, 16), (2, 1024, 8), (16, 4096, 32), (17, 4096, 32)])
 def test_decode_launch_shapes(oracle, B, Dch, H):
     """Channel-pair counts that select the launch shapes not covered by the sweep workload
     (4096 pairs: 8 lanes x 2 modes; 16384: 4 lanes x 2 modes; 1024: 16 lanes x 1 mode), including
-    the mid-size workload's B=8, Dch=1024; 6 steps from a random state, every element compared."""
+    the mid-size workload's B=8, Dch=1024, and both sides of the bound of the early parameter loads
+    on the 2-lane shape (32768 pairs: early; 34816: at first use); 6 steps from a random state,
+    every element compared."""
     w = W.Workload(600 + B, "case", B=B, L=0, Dch=Dch, H=H, d=16, dtype="bf16", fft_len=0, T=0,
                    random_state0=True)
     p = W.params(w)
