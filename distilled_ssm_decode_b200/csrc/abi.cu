@@ -191,6 +191,12 @@ int hyena_prefill_chunked(const void *q, const void *k, const void *v, int dtype
                                               workspace, s));
 }
 
+int hyena_test_chunked_inject(int suppress_item, double lookback_limit_s) {
+    if (suppress_item < -1 || !(lookback_limit_s >= 0.0) || lookback_limit_s > 60.0) return HYENA_ERR_ARG;
+    chunked_inject(suppress_item, (unsigned long long)(lookback_limit_s * 1e9));
+    return HYENA_OK;
+}
+
 size_t hyena_prompt_state_workspace_bytes(int B, int L, int Dch, int d) {
     if (B < 0 || L < 0 || Dch < 0 || d < 1 || d > HYENA_MAX_MODES) return 0;
     return align_up(state_ws_bytes(B, L, Dch, d));

@@ -39,6 +39,9 @@ cudaError_t launch_prefill_fft(const void *q, const void *k, const void *v, int 
 bool chunked_supported(int dtype, int Dch, int H, int d);
 size_t chunked_ws_bytes(int B, int L, int Dch, int H, int d);
 int chunked_error_offset(int B, int L, int Dch, int H, int d);
+// fault injection for tests: suppress one item's status word (-1: none) and bound each look-back
+// poll by wait_ns (0: the default bound); applies to every later launch
+void chunked_inject(int suppress_item, unsigned long long wait_ns);
 cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, int B, int L, int Dch,
                                    int H, int d, const float2 *lam, const float2 *R, const float *Dskip,
                                    void *y, float *state_out, void *ws, cudaStream_t s);

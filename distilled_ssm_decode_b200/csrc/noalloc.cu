@@ -12,8 +12,10 @@
 // library holds kNoAllocScratchBytes of it until the process exits.  Host code
 // must not use the array's name as a device address: the address is fetched
 // with cudaGetSymbolAddress once per device (the first call on each device, with
-// that device current) and cached.  That first call may also load the module on
-// the device, so make it before any stream capture.  All calls share the one
+// that device current) and cached for the life of the process (a cudaDeviceReset
+// may move the array, so the entry point must not be used on a device after
+// resetting it).  That first call may also load the module on the device, so
+// make it before any stream capture.  All calls share the one
 // array: calls whose work overlaps on the GPU (different streams, or different
 // host threads on one device) race on it and must be serialised by the caller.
 // The prefill overwrites everything it reads from the scratch, so no contents

@@ -45,16 +45,26 @@
 // contribution, then (segments after the first) obtains the
 // state entering its segment by a decoupled look-back over its predecessors'
 // published contributions (bounded polls), then runs the full pass.  The grid is
-// persistent: each CTA's first item has a fixed ticket, later ones come from a
-// per-head atomic ticket counter, and its pipelines run on across item
-// boundaries.  Tickets are segment-major (all
+// persistent: items come from a per-head atomic ticket counter, and each CTA's
+// pipelines run on across item boundaries.  Tickets are segment-major (all
 // units' first segments, then all second segments, ...), so an item's
 // predecessors were handed out a whole round of units earlier and have usually
-// published by the time it looks back.  An item only ever waits on items with
-// lower tickets, which running CTAs hold, and the state-only pass never waits,
-// so the look-back always ends.  Every wait is bounded; on timeout the
-// kernel records an error code, drains its copies and MMAs, frees tensor memory
-// and returns.
+// published by the time it looks back.
+//
+// Progress does not depend on the order in which CTAs become resident: an item
+// only ever waits on items with lower tickets, and a ticket is only ever held by
+// a CTA that is running (it took the ticket from the counter), whose earlier
+// items have lower tickets still; the state-only pass never waits.  By induction
+// over the tickets every look-back ends, even when other kernels hold most SMs.
+// When sequences are split, the counters are therefore cleared by a memset ahead
+// of the constants kernel, so the loaders can take tickets at once.  When they
+// are not (no item waits on another), each CTA's first item has a fixed ticket
+// (blockIdx / H of head blockIdx % H) and only later tickets come from the
+// counters, which the constants kernel clears.  Every wait is bounded; on
+// timeout the kernel records an error code, drains its copies and MMAs, frees
+// tensor memory and returns.
+#include <atomic>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -198,6 +208,9 @@ struct ChunkArgs {
     int *status;         // [items]: 0 none, 1 segment contribution, 2 inclusive state
     float *agg;          // [items][32 rows][NC ch]
     float *inc;          // [items][32 rows][NC ch]
+    int fixed_first;     // 1: each CTA's first item has a fixed ticket (only when nseg == 1)
+    int suppress_item;   // fault injection for tests: this item's status word is never posted (-1: none)
+    unsigned long long lookback_ns;   // bound of one look-back poll
 };
 
 struct Item {
@@ -225,9 +238,12 @@ __device__ __forceinline__ Item decode_item(const ChunkArgs &a, int id) {
 
 enum : int { kErrWait = 1, kErrLookback = 2 };
 
+// The code is recorded before the CTA's other roles are told to stop, so the error word holds the
+// cause (a role that then gives up on a wait only finds the word already set).
 __device__ __forceinline__ void record_error(const ChunkArgs &a, volatile int *abort, int code) {
-    *abort = 1;
     atomicCAS(a.sched + 1, 0, code);
+    __threadfence();
+    *abort = 1;
 }
 
 // Load with acquire semantics at GPU scope (pairs with the publisher's fence + status write).
@@ -556,19 +572,22 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     ok = false;
                     break;
                 }
-                // tickets of this CTA's head first; when they run out, move on to the next head.  The
-                // first item's ticket is fixed (blockIdx / H); the counter of head h hands out the
-                // tickets after the fixed ones of the CTAs assigned to h.
+                // tickets of this CTA's head first; when they run out, move on to the next head.  With
+                // fixed first tickets (unsplit sequences) the first item's ticket is blockIdx / H and the
+                // counter of head h hands out the tickets after the fixed ones of the CTAs assigned to
+                // h; those counters are cleared by the constants kernel, so the first counted ticket
+                // waits for it.  Otherwise every ticket comes from a counter cleared before this launch.
                 int id = -1;
-                if (k == 0 && (int)blockIdx.x / a.H < a.ih) {
+                if (k == 0 && a.fixed_first && (int)blockIdx.x / a.H < a.ih) {
                     id = head * a.ih + (int)blockIdx.x / a.H;
                 } else {
                     if (!counted) {
-                        asm volatile("griddepcontrol.wait;" ::: "memory");
+                        if (a.fixed_first) asm volatile("griddepcontrol.wait;" ::: "memory");
                         counted = true;
                     }
                     while (tries < a.H) {
-                        const int fixed = head < (int)gridDim.x ? min(a.ih, ((int)gridDim.x - head + a.H - 1) / a.H) : 0;
+                        const int fixed = !a.fixed_first ? 0
+                                          : head < (int)gridDim.x ? min(a.ih, ((int)gridDim.x - head + a.H - 1) / a.H) : 0;
                         const int t = atomicAdd(a.tickets + head, 1) + fixed;
                         if (t < a.ih) { id = head * a.ih + t; tries = 0; break; }
                         head = head + 1 == a.H ? 0 : head + 1;
@@ -680,7 +699,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int v = pubq[ps];
                 if (v < 0) break;
                 __threadfence();
-                atomicExch(a.status + (v >> 2), v & 3);
+                if ((v >> 2) != a.suppress_item) atomicExch(a.status + (v >> 2), v & 3);
                 tc::mbar_arrive(bar(kBarPubEmpty + ps));
             }
         }
@@ -959,7 +978,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     if (lane == 0) {
                         code = ld_acquire(a.status + p);
                         const unsigned long long t0 = tc::global_ns();
-                        while (code == 0 && !*abort && tc::global_ns() - t0 < tc::kWaitNs) {
+                        while (code == 0 && !*abort && tc::global_ns() - t0 < a.lookback_ns) {
                             __nanosleep(64);
                             code = ld_acquire(a.status + p);
                         }
@@ -1197,18 +1216,22 @@ ChunkPlan plan(int B, int L, int Dch, int H) {
     return p;
 }
 
+// SM count of the current device (the persistent grid is at most one CTA per SM), cached per device
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+
 int sm_count() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0, v = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess &&
-            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
-            n = v;
-        else
-            return kPlanSMs;
-    }
-    return n;
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return kPlanSMs;
+    if (dev < kMaxDevices && (v = g_sm_count[dev].load(std::memory_order_relaxed)) > 0) return v;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) return kPlanSMs;
+    if (dev < kMaxDevices) g_sm_count[dev].store(v, std::memory_order_relaxed);
+    return v;
 }
+
+// fault injection for tests (hyena_test_chunked_inject): applied to every later launch
+std::atomic<int> g_inject_item{-1};
+std::atomic<unsigned long long> g_inject_wait_ns{0};
 
 }  // namespace
 
@@ -1250,10 +1273,15 @@ cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, 
                                    void *y, float *state_out, void *ws, cudaStream_t s) {
     const ChunkPlan p = plan(B, L, Dch, H);
     uint8_t *w = static_cast<uint8_t *>(ws);
-
+    // schedule words (error word, ticket counters, status words): with split sequences they are
+    // cleared ahead of the constants kernel, so that every ticket can come from a counter at once
+    const bool fixed_first = p.nseg == 1;
+    const int nzero = (int)((p.agg_off - p.sched_off) / 4);
+    cudaError_t e;
+    if (!fixed_first && (e = cudaMemsetAsync(w + p.sched_off, 0, (size_t)nzero * 4, s)) != cudaSuccess) return e;
     chunk_consts_kernel<<<H, kConstThreads, 0, s>>>(lam, R, Dskip, d, p.segc * kC, w + p.consts_off,
-                                          reinterpret_cast<int *>(w + p.sched_off), (int)((p.agg_off - p.sched_off) / 4));
-    cudaError_t e = cudaGetLastError();
+                                          reinterpret_cast<int *>(w + p.sched_off), fixed_first ? nzero : 0);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     CUtensorMap mq, mk, mv, my;
     if (!make_map(&mq, q, B, L, Dch) || !make_map(&mk, k, B, L, Dch) || !make_map(&mv, v, B, L, Dch) ||
@@ -1272,12 +1300,21 @@ cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, 
     a.status = reinterpret_cast<int *>(w + p.status_off);
     a.agg = reinterpret_cast<float *>(w + p.agg_off);
     a.inc = reinterpret_cast<float *>(w + p.inc_off);
+    a.fixed_first = fixed_first ? 1 : 0;
+    a.suppress_item = g_inject_item.load();
+    const unsigned long long inj_ns = g_inject_wait_ns.load();
+    a.lookback_ns = inj_ns ? inj_ns : tc::kWaitNs;
     return p.nc == 128 ? launch_tile<128>(mq, mk, mv, my, a, p.items, s) : launch_tile<64>(mq, mk, mv, my, a, p.items, s);
 }
 
 int chunked_error_offset(int B, int L, int Dch, int H, int d) {
     (void)d;
     return (int)(plan(B, L, Dch, H).sched_off + 4);
+}
+
+void chunked_inject(int suppress_item, unsigned long long wait_ns) {
+    g_inject_item.store(suppress_item);
+    g_inject_wait_ns.store(wait_ns);
 }
 
 }  // namespace hyena

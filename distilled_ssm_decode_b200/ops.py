@@ -41,6 +41,7 @@ SIGNATURES = {
     "hyena_prefill_noalloc_capacity": (_sz, []),
     "hyena_prefill_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp, _fp,
                                    _vp]),
+    "hyena_test_chunked_inject": (_i, [_i, ctypes.c_double]),
     "hyena_prompt_state_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "hyena_prompt_state": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _fp, _fp, _vp, _sz, _vp]),
     "hyena_decode_step": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _fp, _fp, _fp, _fp, _vp, _vp]),
@@ -200,6 +201,12 @@ def chunked_error(workspace, B, L, Dch, H, d) -> int:
     """The kernel's error word (synchronises): 0 when every bounded wait succeeded."""
     off = int(lib().hyena_prefill_chunked_error_offset(B, L, Dch, H, d))
     return int(workspace[off:off + 4].view(torch.int32).item())
+
+
+def test_chunked_inject(suppress_item: int = -1, lookback_limit_s: float = 0.0):
+    """Test hook: fault injection for the chunked prefill's bounded waits (see hyena.h);
+    (-1, 0) restores normal operation."""
+    _check("hyena_test_chunked_inject", lib().hyena_test_chunked_inject(int(suppress_item), float(lookback_limit_s)))
 
 
 def prompt_state(k, v, lam, H: int, state=None):

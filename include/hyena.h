@@ -151,10 +151,17 @@ int hyena_prefill(const void *q, const void *k, const void *v, int dtype,
  *   Arguments and results as hyena_prefill, minus the workspace.  It never
  *   calls cudaMalloc, cudaFree or any allocating routine.
  *   HYENA_ERR_CAPACITY when hyena_prefill_workspace_bytes(...) exceeds the
- *   capacity (e.g. transforms longer than 16384 points).
+ *   capacity.  For fft_len <= 16384 that size is about 4*H*L + 8*H*fft_len
+ *   bytes (the filter and the head spectra), so the limit depends on H and L
+ *   as well: e.g. fft_len = 8192 and L = 4096 fit up to 51 heads, fft_len =
+ *   16384 and L = 8192 up to 25; transforms longer than 16384 points need far
+ *   more.  Check hyena_prefill_workspace_bytes() against
+ *   hyena_prefill_noalloc_capacity() before relying on it.
  *   The first call on each device looks up the array's device address (with
  *   that device current) and may load the module there: make it before any
- *   stream capture.  Every call uses the same array, so calls whose work
+ *   stream capture.  The address is cached per device for the life of the
+ *   process; after cudaDeviceReset on a device, do not call this entry point
+ *   there again.  Every call uses the same array, so calls whose work
  *   overlaps on the GPU (other streams, other host threads) race on it; the
  *   caller must serialise them.  Nothing needs clearing between calls.
  */
@@ -183,11 +190,14 @@ int hyena_prefill_noalloc(const void *q, const void *k, const void *v, int dtype
  *   activation pointers 16-byte aligned; HYENA_ERR_UNSUPPORTED otherwise.
  *   workspace: >= hyena_prefill_chunked_workspace_bytes() bytes, 256-byte aligned.
  *   Calls on different streams may run at the same time (for instance independent
- *   layers), each with its own workspace.
+ *   layers), each with its own workspace.  Progress does not depend on how many
+ *   SMs other work leaves free: a part of the kernel only waits for parts that
+ *   are already running.
  *   The int32 at byte offset hyena_prefill_chunked_error_offset() of the
  *   workspace is 0 after a successful run; a nonzero value means a bounded
- *   wait inside the kernel gave up (the outputs are then invalid).  Read it
- *   after synchronising the stream if needed.
+ *   wait inside the kernel gave up and the outputs are invalid: 1 = a pipeline
+ *   wait (2 s), 2 = the wait for the state of an earlier segment of the same
+ *   sequence.  Read it after synchronising the stream if needed.
  */
 size_t hyena_prefill_chunked_workspace_bytes(int B, int L, int Dch, int H, int d);
 size_t hyena_prefill_chunked_error_offset(int B, int L, int Dch, int H, int d);
@@ -196,6 +206,20 @@ int hyena_prefill_chunked(const void *q, const void *k, const void *v, int dtype
                           const float *lambda, const float *R, const float *Dskip,
                           void *y, float *state_out,
                           void *workspace, size_t ws_bytes, hyena_stream_t stream);
+
+/*
+ * Test hook (no counterpart in the pages): fault injection for the bounded
+ * waits of hyena_prefill_chunked, so that a test can make a wait run out
+ * without any GPU fault.  Every later hyena_prefill_chunked launch in the
+ * process skips posting the completion word of work item `suppress_item`
+ * (-1: none), and bounds each wait for an earlier segment's state by
+ * `lookback_limit_s` seconds (0: the default 2 s).  A launch whose sequences
+ * are split into segments then ends with error word 2 instead of waiting
+ * forever.  (-1, 0) restores normal operation.  HYENA_ERR_ARG for
+ * suppress_item < -1 or a limit outside [0, 60].  Not thread-safe against
+ * concurrent launches; meant for tests only.
+ */
+int hyena_test_chunked_inject(int suppress_item, double lookback_limit_s);
 
 /*
  * Prompt -> state reduction alone (the Vandermonde contraction over the

@@ -8,6 +8,11 @@ several 128-channel tiles and heads, d from 1 to 16, and sequences split into
 many segments (which exercises the cross-segment state look-back).  Every run
 also checks the kernel's error word (0 = no bounded wait gave up).
 """
+import ctypes
+import os
+import shutil
+import subprocess
+
 import numpy as np
 import pytest
 import torch
@@ -239,3 +244,73 @@ def test_mid_workload_flow_chunked_then_decode(oracle):
     va = np.concatenate([gather_columns(v, bc), W.to_f64(torch.stack(vs))[None]], 1)
     y_ref, s_ref = oracle.recurrent(qa, ka, va, lam_c, R_c, D_c, H=len(bc))
     assert rel_err(torch.stack(ys).double().numpy()[None], y_ref[:, w.L:]) <= TOL["bf16"]
+
+
+ERR_LOOKBACK = 2
+
+
+def test_chunked_lookback_timeout_reports_error_and_recovers(oracle):
+    """Failure detection without a GPU fault: the test hook stops one segment's completion word from
+    ever being posted and bounds the wait for it to 5 ms.  The call must return with error word 2
+    (a look-back gave up) instead of hanging, and the next normal call on the same stream and
+    workspace must pass parity."""
+    w = W.Workload(301, "lookback", B=1, L=4096, Dch=128, H=1, d=16, dtype="bf16", fft_len=0, T=0)
+    p = W.params(w)
+    q, k, v = W.prefill_inputs(w)
+    lam, R, D = dev_params(p)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    ops.test_chunked_inject(0, 0.005)          # item 0: segment 0 of the first sequence
+    try:
+        _, _, ws = ops.prefill_chunked(qd, kd, vd, lam, R, D)
+        torch.cuda.synchronize()
+    finally:
+        ops.test_chunked_inject(-1, 0.0)
+    assert ops.chunked_error(ws, w.B, w.L, w.Dch, w.H, w.d) == ERR_LOOKBACK
+    y, s, _ = ops.prefill_chunked(qd, kd, vd, lam, R, D, workspace=ws)
+    assert ops.chunked_error(ws, w.B, w.L, w.Dch, w.H, w.d) == 0
+    y_ref, s_ref = oracle.recurrent(W.to_f64(q), W.to_f64(k), W.to_f64(v), p.lam, p.R, p.Dskip, H=w.H)
+    ey, es = rel_err(y.cpu().double().numpy(), y_ref), rel_err(state_c128(s), s_ref)
+    assert ey <= TOL["bf16"] and es <= TOL["bf16"], (ey, es)
+
+
+def _hold_sms_lib():
+    """Build (once) and load the test helper that occupies SMs for a bounded time."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = os.path.join(root, "tests", "gpu_aux", "hold_sms.cu")
+    out = os.path.join(root, "_build", "libhyena_test_hold_sms.so")
+    if not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        os.makedirs(os.path.dirname(out), exist_ok=True)
+        nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+        subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O2", "-shared", "-Xcompiler",
+                        "-fPIC", "-o", out, src], check=True, capture_output=True)
+    lib = ctypes.CDLL(out)
+    lib.hold_sms.argtypes = [ctypes.c_int, ctypes.c_ulonglong, ctypes.c_int, ctypes.c_void_p]
+    lib.sm_count.argtypes = []
+    return lib
+
+
+@pytest.mark.parametrize("B,L,Dch,H", [(1, 20000, 192, 3), (1, 65536, 768, 12)])
+def test_chunked_segments_progress_with_most_sms_busy(B, L, Dch, H):
+    """Sequences split into segments, launched while a kernel on another stream holds all but 12 SMs
+    for 20 ms: the items that wait for earlier segments must only ever wait on work that is running,
+    so the call completes with error word 0 and the same bits as an uncontended run."""
+    aux = _hold_sms_lib()
+    w = W.Workload(500 + H, "busy", B=B, L=L, Dch=Dch, H=H, d=16, dtype="bf16", fft_len=0, T=0)
+    p = W.params(w)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(13)
+    q, k, v = (torch.randn((B, L, Dch), generator=g, device="cuda").to(torch.bfloat16) for _ in range(3))
+    lam, R, D = dev_params(p)
+    y1, s1, ws = ops.prefill_chunked(q, k, v, lam, R, D)
+    torch.cuda.synchronize()
+    nsm = aux.sm_count()
+    assert nsm > 12
+    busy, work = torch.cuda.Stream(), torch.cuda.Stream()
+    y2, s2 = torch.empty_like(y1), torch.empty_like(s1)
+    ws2 = torch.empty_like(ws)
+    assert aux.hold_sms(nsm - 12, 20_000_000, 160 * 1024, ctypes.c_void_p(busy.cuda_stream)) == 0
+    with torch.cuda.stream(work):
+        ops.prefill_chunked(q, k, v, lam, R, D, y=y2, state=s2, workspace=ws2)
+    torch.cuda.synchronize()
+    assert ops.chunked_error(ws2, B, L, Dch, H, 16) == 0
+    assert torch.equal(y1, y2) and torch.equal(s1, s2)
