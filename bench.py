@@ -1,27 +1,29 @@
 #!/usr/bin/env python
 """Benchmark of the gated modal long convolution (prefill + O(1) decode) on B200.
 
-One step = one pass of the whole hot path over one batch of synthetic input:
-filter materialisation, filter spectrum, FFT long convolution with gating and
-prompt -> state reduction over a B x L prompt (one hyena_prefill call), then T
-decode steps (one hyena_decode_step call each, replayed from a CUDA graph).
-Default workload: the mid-size operator, B=8, L=4096, Dch=1024, H=8, d=16,
-bf16 activations, complex fp32 state, FFT length 8192, 256 decode steps.
+Default line: the 1.3B-shaped generation workload, 24 independent operator layers, each
+B=64, L=512, Dch=2048, H=16, d=16, bf16 activations, complex fp32 state.  One step = the
+chunked tensor-core prefill of every layer's 512-token prompt, then 512 decode tokens, each
+one grouped decode launch over all 24 layers (replayed from a CUDA graph).  The same run
+adds sub-records, each timed on its own: the mid-size operator (prefill and decode), the
+long prefill (65536 tokens, with its end-to-end time) and the decode batch sweep at
+B = 1, 16, 64, 256 and 1024.  Every sub-record carries its roofline entries.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-subrecords] ...
 
-Under torchrun (N > 1) every rank runs the same workload on its own GPU: the
-sequences are independent, so the data-parallel shards need no collective;
-timing is the max over ranks.  Rank 0 prints one JSON line.
+Under torchrun (N > 1) every rank runs the headline workload on its own GPU: sequences and
+layers are independent, so the data-parallel replicas need no collective; timing is the max
+over ranks and rank 0 prints one JSON line (sub-records are single-GPU figures, N = 1 only).
 """
 from __future__ import annotations
 
 import argparse
 import datetime
 import hashlib
-import re
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -34,6 +36,7 @@ if ROOT not in sys.path:
 
 METRIC = "decode tokens/s and prefill tokens/s on 1 B200; % of HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
+DEFAULT_WORKLOAD = "gen1p3b_bf16"
 
 
 # ------------------------------------------------------------------ multi-rank plumbing
@@ -116,6 +119,18 @@ def ncu_traffic(kernel: str, workload: str):
     return d.get("bytes_per_launch")
 
 
+def roof(kernel, nbytes, launch_ms, peak, peak_src, traffic=None, total_ms=None, note=None):
+    """Roofline entry: algorithmic bytes of one launch over its measured duration."""
+    gbs = nbytes / (launch_ms / 1e3) / 1e9
+    r = {"kernel": kernel, "bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+         "frac": gbs / peak, "peak_source": peak_src, "algorithmic_bytes": nbytes,
+         "launch_ms": launch_ms, "total_ms": launch_ms if total_ms is None else total_ms,
+         "traffic": traffic}
+    if note:
+        r["note"] = note
+    return r
+
+
 # ------------------------------------------------------------------ clocks during the timed region
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -178,6 +193,17 @@ def gpu_id_for(device) -> str:
         return vis.split(",")[device.index] if vis else str(device.index)
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 # ------------------------------------------------------------------ CPU (oracle) timing
 class OracleSample:
     """Inputs of the workload drawn once; the fp64 oracle (recurrent mode: prompt then
@@ -232,6 +258,33 @@ class OracleSample:
         return total, tok
 
 
+def oracle_baseline(w, nl: int, target_s: float):
+    """The fp64 oracle on the host cores: tokens/s of the whole workload (layer 0 timed, divided by
+    the layer count), with a description of the sample."""
+    import oracle
+    oracle.build()
+    sample = OracleSample(w)
+    channels, reps = sample.calibrate(target_s)
+    dt, tok = sample.run_reps(channels, reps)
+    desc = (f"fp64 oracle, recurrent mode: {reps} pass(es) over all {w.B} sequences x first {channels} of "
+            f"{w.Dch} channels ({w.L}-token prompt + {w.T} decode tokens), {dt:.1f} s"
+            + (f"; layer 0 only, tokens/s divided by {nl} layers" if nl > 1 else ""))
+    return {"value": tok / dt / nl, "unit": "tokens/s", "cores": oracle.threads(), "cpu_model": cpu_model(),
+            "kind": "oracle", "sample": desc}, sample, channels, reps
+
+
+# ------------------------------------------------------------------ the line's config (both arms)
+def line_config(w, nl: int):
+    layers = f", {nl} independent layers" if nl > 1 else ""
+    return {"workload": (f"{w.name}: B={w.B} L={w.L} Dch={w.Dch} H={w.H} d={w.d} {w.dtype} activations, "
+                         f"complex fp32 state, FFT length {w.fft_len}, {w.T} decode steps{layers}"),
+            "B": w.B, "L": w.L, "Dch": w.Dch, "H": w.H, "d": w.d, "fft_len": w.fft_len,
+            "decode_steps": w.T, "layers": nl, "activations": w.dtype,
+            "parallelism": "data-parallel replicas",
+            "l2": "inputs larger than L2 (prefill q,k,v per call; decode states of the batch-256+ and "
+                  "multi-layer workloads)"}
+
+
 # ------------------------------------------------------------------ reference arm (the oracle)
 def run_reference(args):
     rank, world = dist_init("gloo")
@@ -241,6 +294,9 @@ def run_reference(args):
     from distilled_ssm_decode_b200 import workloads as W
     oracle.build()
     w = W.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.with_(B=args.batch)
+    nl = args.layers or w.layers
     sample = OracleSample(w)
     channels, reps = sample.calibrate(1.0)
     for _ in range(args.warmup):
@@ -250,9 +306,7 @@ def run_reference(args):
         dt, t = sample.run_reps(channels, reps)
         total += dt
         tok += t
-    nl = args.layers or w.layers
     value = tok / total / nl
-    cores = oracle.threads()
     desc = (f"fp64 oracle, recurrent mode: all {w.B} sequences x first {channels} of {w.Dch} "
             f"channels, {w.L}-token prompt + {w.T} decode tokens, {reps} pass(es) per step"
             + (f"; layer 0 only, tokens/s divided by {nl} layers" if nl > 1 else ""))
@@ -260,22 +314,48 @@ def run_reference(args):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": dict(workload_config(w), **({"layers": nl} if nl > 1 else {})),
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                             "sample": desc},
+            "config": line_config(w, nl),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads(),
+                             "cpu_model": cpu_model(), "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
-def workload_config(w):
-    return {"workload": (f"{w.name}: B={w.B} L={w.L} Dch={w.Dch} H={w.H} d={w.d} "
-                         f"{w.dtype} activations, complex fp32 state, FFT length {w.fft_len}, "
-                         f"{w.T} decode steps"),
-            "B": w.B, "L": w.L, "Dch": w.Dch, "H": w.H, "d": w.d, "fft_len": w.fft_len,
-            "decode_steps": w.T, "activations": w.dtype, "parallelism": "data-parallel replicas"}
+# ------------------------------------------------------------------ shared timing helpers
+def timed_steps(stream, dev, steps: int, warmup: int, step, nsec: int, lead_spin: bool = True):
+    """Run `warmup` untimed steps, then `steps` timed ones on `stream`.  step(ev) records
+    ev[0..nsec] around its sections.  Returns (elapsed ms of all steps, [mean ms per section])."""
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step(None)
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nsec + 1)] for _ in range(steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        if lead_spin:
+            # a short GPU spin ahead of the start event, so that the first step's launches are queued
+            # while the GPU is busy: the timed region then holds device work only, as every later step
+            # does (each is queued while the previous one runs)
+            torch.cuda._sleep(LEAD_SPIN_CYCLES)
+        t_start.record(stream)
+        for i in range(steps):
+            step(evs[i])
+        t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    elapsed = reduce_max(t_start.elapsed_time(t_end), dev)
+    secs = [reduce_max(sum(e[j].elapsed_time(e[j + 1]) for e in evs) / steps, dev) for j in range(nsec)]
+    return elapsed, secs
 
+
+def make_pinned(shape, dtype):
+    import torch
+    return torch.empty(shape, dtype=dtype, pin_memory=True)
 
 
 def fir_baseline(ops, W, w, q, k, v, dq, dk, dv, lam, R, D, stream, dev, nsteps, modal_step_ms,
@@ -324,31 +404,26 @@ def fir_baseline(ops, W, w, q, k, v, dq, dk, dv, lam, R, D, stream, dev, nsteps,
                                     "ms_per_token_step": prefill_ms, "modal_decode_speedup": prefill_ms / modal_step_ms}}
 
 
-# ------------------------------------------------------------------ our arm
-def run_ours(args):
+# ------------------------------------------------------------------ one-layer workloads
+def measure_single(args, w, dev, steps: int, warmup: int, e2e_steps: int, with_fft_route: bool,
+                   with_baselines: bool, with_e2e: bool):
+    """Prefill (chunked route when supported, else FFT) and T decode steps of one workload.
+    Returns a record with separate prefill and decode figures, each with its roofline entry."""
     import torch
 
-    rank, world, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    dist_init("nccl")
-    from distilled_ssm_decode_b200 import build, ops
+    from distilled_ssm_decode_b200 import ops
     from distilled_ssm_decode_b200 import workloads as W
-    build.build()
-    ops.lib()
-
-    w = W.WORKLOADS[args.workload]
-    if args.batch:
-        w = w.with_(B=args.batch)
+    _, world, _ = dist_env()
     has_pre, has_dec = w.L > 0, w.T > 0
     use_chunked = has_pre and args.prefill != "fft" and ops.lib().hyena_prefill_chunked_workspace_bytes(
         w.B, w.L, w.Dch, w.H, w.d) > 0
-    if args.prefill == "chunked" and not use_chunked:
+    if args.prefill == "chunked" and has_pre and not use_chunked:
         raise SystemExit(f"chunked prefill does not support workload {w.name}")
     p = W.params(w)
     lam, R, D = p.lam_f32().to(dev), p.R_f32().to(dev), p.Dskip_f32().to(dev)
     stream = torch.cuda.Stream(dev)
     state = torch.empty((w.B, w.d, w.Dch, 2), dtype=torch.float32, device=dev)
+    key = f"{w.name}/B{w.B}"
 
     # ---- inputs (resident in HBM before the timed region)
     host = {}
@@ -356,7 +431,7 @@ def run_ours(args):
         host["q"], host["k"], host["v"] = W.prefill_inputs(w)
         q, k, v = host["q"].to(dev), host["k"].to(dev), host["v"].to(dev)
         y = torch.empty_like(q)
-        ws = torch.empty(ops.prefill_workspace_bytes(w.B, w.L, w.Dch, w.H, w.d, w.fft_len),
+        ws = torch.empty(max(1, ops.prefill_workspace_bytes(w.B, w.L, w.Dch, w.H, w.d, w.fft_len)),
                          dtype=torch.uint8, device=dev)
         if use_chunked:
             ws_c = torch.empty(ops.prefill_chunked_workspace_bytes(w.B, w.L, w.Dch, w.H, w.d),
@@ -401,7 +476,7 @@ def run_ours(args):
             decode_all()
         torch.cuda.synchronize(dev)
 
-    def step(ev=None):
+    def step(ev):
         if ev is not None:
             ev[0].record(stream)
         if has_pre:
@@ -413,102 +488,66 @@ def run_ours(args):
         if ev is not None:
             ev[2].record(stream)
 
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            step()
-    torch.cuda.synchronize(dev)
-
-    # ---- timed region (device-resident inputs)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(gpu_id_for(dev))
-    clocks.start()
-    time.sleep(0.3)
-    barrier(dev)
-    torch.cuda.synchronize(dev)
-    with torch.cuda.stream(stream):
-        # a short GPU spin ahead of the start event, so that the first step's launches are queued
-        # while the GPU is busy: the timed region then holds device work only, as every later step
-        # does (each is queued while the previous one runs)
-        torch.cuda._sleep(LEAD_SPIN_CYCLES)
-        t_start.record(stream)
-        for i in range(args.steps):
-            step(evs[i])
-        t_end.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(dev)
-    clk = clocks.stop()
-    elapsed_ms = reduce_max(t_start.elapsed_time(t_end), dev)
-    pre_ms = reduce_max(sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps, dev)
-    dec_ms = reduce_max(sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps, dev)
-    ms_per_step = elapsed_ms / args.steps
-
-    tokens_step = w.B * (w.L + w.T)
-    value = world * tokens_step / (ms_per_step / 1e3)
+    elapsed_ms, (pre_ms, dec_ms) = timed_steps(stream, dev, steps, warmup, step, 2)
+    ms_per_step = elapsed_ms / steps
     peak, peak_src = load_peaks()
     pb, db = algorithmic_bytes(w)
+    rec = {"workload": line_config(w, 1)["workload"], "steps": steps, "warmup": warmup,
+           "ms_per_step": ms_per_step,
+           "value": world * w.B * (w.L + w.T) / (ms_per_step / 1e3), "unit": "tokens/s"}
     roofs = []
-    out_pre = out_dec = None
     if has_pre:
-        pre_gbs = pb / (pre_ms / 1e3) / 1e9
-        roofs.append({"kernel": "hyena_prefill (filter + spectrum + fused FFT conv/gate/state)",
-                      "bound": "hbm", "achieved": pre_gbs, "peak": peak, "unit": "GB/s",
-                      "frac": pre_gbs / peak, "peak_source": peak_src, "algorithmic_bytes": pb,
-                      "launch_ms": pre_ms, "total_ms": pre_ms,
-                      "traffic": ncu_traffic("prefill_fused", f"{w.name}/B{w.B}")})
-        out_pre = {"tokens_per_s": world * w.B * w.L / (pre_ms / 1e3), "ms": pre_ms,
-                   "hbm_frac": pre_gbs / peak}
+        name = ("hyena_prefill_chunked (tcgen05 chunked conv/gate/state)" if use_chunked
+                else "hyena_prefill (filter + spectrum + fused FFT conv/gate/state)")
+        r = roof(name, pb, pre_ms, peak, peak_src,
+                 ncu_traffic("prefill_chunk" if use_chunked else "prefill_fused", key))
+        roofs.append(r)
+        rec["prefill"] = {"route": "chunked" if use_chunked else "fft",
+                          "tokens_per_s": world * w.B * w.L / (pre_ms / 1e3), "ms": pre_ms,
+                          "hbm_frac": r["frac"], "roofline": r,
+                          "inputs": "q, k, v of %d MiB each (larger than L2)" % (w.B * w.L * w.Dch * w.act_bytes >> 20)}
+        if use_chunked:
+            err = ops.chunked_error(ws_c, w.B, w.L, w.Dch, w.H, w.d)
+            if err:
+                raise SystemExit(f"chunked prefill kernel reported error {err}")
     if has_dec:
-        dec_launch_ms = dec_ms / w.T
-        dec_gbs = db / (dec_launch_ms / 1e3) / 1e9
-        roofs.append({"kernel": "hyena_decode_step", "bound": "hbm", "achieved": dec_gbs,
-                      "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak,
-                      "peak_source": peak_src, "algorithmic_bytes": db,
-                      "launch_ms": dec_launch_ms, "total_ms": dec_ms,
-                      "traffic": ncu_traffic("decode", f"{w.name}/B{w.B}")})
-        st_bytes = state.numel() * 4
-        if st_bytes < 100 << 20:
-            roofs[-1]["note"] = (f"the {st_bytes / 2**20:.1f} MiB state stays in L2 between steps, so a step reads "
-                                 "no DRAM and is bound by launch and L2 latency; the HBM fraction is not its bound")
-        out_dec = {"tokens_per_s": world * w.B * w.T / (dec_ms / 1e3),
-                   "ms_per_token_step": dec_launch_ms, "hbm_frac": dec_gbs / peak}
-    if use_chunked:
-        roofs[0]["kernel"] = "hyena_prefill_chunked (tcgen05 chunked conv/gate/state)"
-        roofs[0]["traffic"] = ncu_traffic("prefill_chunk", f"{w.name}/B{w.B}")
-        err = ops.chunked_error(ws_c, w.B, w.L, w.Dch, w.H, w.d)
-        if err:
-            raise SystemExit(f"chunked prefill kernel reported error {err}")
+        launch_ms = dec_ms / w.T
+        st_mib = state.numel() * 4 / 2 ** 20
+        l2_res = st_mib < 100
+        note = (f"the {st_mib:.1f} MiB state stays in L2 between steps, so a step reads no DRAM and is bound by "
+                "launch and L2 latency; the HBM fraction is not its bound") if l2_res else None
+        r = roof("hyena_decode_step", db, launch_ms, peak, peak_src, ncu_traffic("decode", key), dec_ms, note)
+        roofs.append(r)
+        rec["decode"] = {"tokens_per_s": world * w.B * w.T / (dec_ms / 1e3), "ms_per_token_step": launch_ms,
+                         "hbm_frac": r["frac"], "roofline": r,
+                         "state": "%.1f MiB, %s" % (st_mib, "L2-resident between steps" if l2_res else "larger than L2"),
+                         "inputs": ("%d distinct input sets, cycled" % dq.shape[0]) if dq.shape[0] != w.T
+                         else "one input set per step"}
     # the FFT route (zero-padded FFT long convolution) timed on the same inputs
-    fft_route = None
-    if has_pre and use_chunked and not args.no_fft_route:
-        fe = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        with torch.cuda.stream(stream):
-            for _ in range(2):
-                prefill_fft()
-            fe[0].record(stream)
-            for _ in range(args.steps):
-                prefill_fft()
-            fe[1].record(stream)
-        torch.cuda.synchronize(dev)
-        fms = reduce_max(fe[0].elapsed_time(fe[1]) / args.steps, dev)
-        fgbs = pb / (fms / 1e3) / 1e9
-        fft_route = {"kernel": "hyena_prefill (filter + spectrum + fused FFT conv/gate/state)",
-                     "fft_len": w.fft_len, "tokens_per_s": world * w.B * w.L / (fms / 1e3),
-                     "ms": fms, "achieved": fgbs, "frac": fgbs / peak, "unit": "GB/s",
-                     "traffic": ncu_traffic("prefill_fused", f"{w.name}/B{w.B}")}
-    dominant = max(roofs, key=lambda r: r["total_ms"])
-    baselines = None
-    if has_pre and has_dec and not args.no_baselines:
-        baselines = fir_baseline(ops, W, w, q, k, v, dq, dk, dv, lam, R, D, stream, dev, w.T,
-                                 dec_ms / w.T, pre_ms, peak)
+    if has_pre and use_chunked and with_fft_route:
+        def fstep(ev):
+            if ev is not None:
+                ev[0].record(stream)
+            prefill_fft()
+            if ev is not None:
+                ev[1].record(stream)
+        _, (fms,) = timed_steps(stream, dev, steps, 3, fstep, 1)
+        r = roof("hyena_prefill (filter + spectrum + fused FFT conv/gate/state)", pb, fms, peak, peak_src,
+                 ncu_traffic("prefill_fused", key))
+        rec["prefill_fft_route"] = {"fft_len": w.fft_len, "tokens_per_s": world * w.B * w.L / (fms / 1e3),
+                                    "ms": fms, "hbm_frac": r["frac"], "roofline": r}
+    rec["roofline_all"] = roofs
+    rec["roofline"] = max(roofs, key=lambda x: x["total_ms"])
+    rec["launches_per_step"] = (0 if not has_pre else (2 if use_chunked else (3 if w.fft_len <= 16384 else 8))) + w.T
+    if has_pre and has_dec and with_baselines:
+        rec["baselines"] = fir_baseline(ops, W, w, q, k, v, dq, dk, dv, lam, R, D, stream, dev, w.T,
+                                        dec_ms / w.T, pre_ms, peak)
 
     # ---- end to end: host (pinned) inputs, copies inside the timed region.  Every step copies its
     # inputs in from pinned host memory and its results (prefill y and every decode y) out to
     # pinned host memory.  Two buffer sets let step i+1's inputs travel in, and step i-1's results
     # travel out, while step i computes (copy-in, compute and copy-out streams; PCIe is full duplex).
-    e2e = None
-    if not args.no_e2e and all(x in host for x in ("q", "k", "v")) and \
-            (not has_dec or "dq" in host):
+    if with_e2e and all(x in host for x in ("q", "k", "v")) and (not has_dec or "dq" in host):
         pins = {n: t.pin_memory() for n, t in host.items()}
         sets = []
         for j in range(2):
@@ -583,81 +622,34 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier(dev)
-        e2e_run(args.steps, a, b)
+        e2e_run(e2e_steps, a, b)
         torch.cuda.synchronize(dev)
-        e2e_ms = reduce_max(a.elapsed_time(b), dev) / args.steps
+        e2e_ms = reduce_max(a.elapsed_time(b), dev) / e2e_steps
         if use_chunked:
             err = ops.chunked_error(ws_c, w.B, w.L, w.Dch, w.H, w.d)
             if err:
                 raise SystemExit(f"chunked prefill kernel reported error {err} (end-to-end run)")
-        e2e = {"value": world * tokens_step / (e2e_ms / 1e3), "unit": "tokens/s",
-               "ms_per_step": e2e_ms, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
-               "overlap": "two buffer sets; copy-in, compute and copy-out streams"}
+        rec["e2e"] = {"value": world * w.B * (w.L + w.T) / (e2e_ms / 1e3), "unit": "tokens/s",
+                      "ms_per_step": e2e_ms, "steps": e2e_steps, "h2d_bytes_per_step": bi,
+                      "d2h_bytes_per_step": bo,
+                      "overlap": "two buffer sets; copy-in, compute and copy-out streams"}
         for bs in sets:
             bs.pop("graph", None)
-
-    # ---- CPU baseline: the oracle on the host cores (rank 0, N = 1 only)
-    cpu = None
-    if world == 1 and not args.no_cpu_baseline and has_pre:
-        import oracle
-        oracle.build()
-        sample = OracleSample(w)
-        channels, reps = sample.calibrate(12.0)
-        dt, tok = sample.run_reps(channels, reps)
-        cpu = {"value": tok / dt, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
-               "sample": (f"fp64 oracle, recurrent mode, {reps} pass(es) over all {w.B} sequences "
-                          f"x first {channels} of {w.Dch} channels ({w.L}-token prompt + {w.T} "
-                          f"decode tokens); {dt:.1f} s")}
-
-    # our kernels per step: chunked = constants + main; FFT = filter + spectrum + fused
-    # (four-step FFT beyond 16384 points: filter, 2 spectrum, 3 convolution, 2 state kernels)
-    pre_launches = 0 if not has_pre else (2 if use_chunked else (3 if w.fft_len <= 16384 else 8))
-    if rank == 0:
-        cfg = workload_config(w)
-        if has_pre:
-            cfg["prefill_route"] = "chunked" if use_chunked else "fft"
-            cfg["l2"] = ("prefill inputs larger than L2 (3 x %d MiB)"
-                         % (q.numel() * q.element_size() >> 20))
-        if has_dec:
-            st_mib = state.numel() * 4 / 2 ** 20
-            cfg["l2_decode"] = ("decode state %.1f MiB %s" % (
-                st_mib, "stays L2-resident between steps, as in real decoding" if st_mib < 100
-                else "is larger than L2"))
-            if dq.shape[0] != w.T:
-                cfg["decode_inputs"] = f"{dq.shape[0]} distinct device-drawn input sets, cycled"
-        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
-                "data": "synthetic", "config": cfg, "prefill": out_pre, "decode": out_dec,
-                "prefill_fft_route": fft_route, "baselines": baselines,
-                "roofline": dominant, "roofline_all": roofs,
-                "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": args.steps * (pre_launches + w.T), "clocks": clk}
-        print(json.dumps(line), flush=True)
     del g
-    import torch.distributed as dist
-    if dist.is_initialized():
-        dist.destroy_process_group()
-    return 0
+    return rec
 
 
-def run_layers(args, nl: int):
-    """Every layer of a multi-layer workload: per bench step, the chunked prefill of each layer's
-    prompt, then T decode steps, each one grouped launch over all layers (CUDA graph).  Inputs
-    are drawn on the device (seeded); each layer has its own parameters, state and activations."""
+# ------------------------------------------------------------------ multi-layer workload
+def measure_layers(args, w, nl: int, dev, steps: int, warmup: int, e2e_steps: int, with_baselines: bool,
+                   with_e2e: bool, clocks=None):
+    """Every layer of a multi-layer workload: per step, the chunked prefill of each layer's prompt,
+    then T decode steps, each one grouped launch over all layers (CUDA graph).  Inputs are drawn on
+    the device (seeded); each layer has its own parameters, state and activations."""
     import torch
 
-    rank, world, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    dist_init("nccl")
-    from distilled_ssm_decode_b200 import build, ops
+    from distilled_ssm_decode_b200 import ops
     from distilled_ssm_decode_b200 import workloads as W
-    build.build()
-    ops.lib()
-    w = W.WORKLOADS[args.workload]
-    if args.batch:
-        w = w.with_(B=args.batch)
+    _, world, _ = dist_env()
     if ops.lib().hyena_prefill_chunked_workspace_bytes(w.B, w.L, w.Dch, w.H, w.d) == 0:
         raise SystemExit(f"chunked prefill does not support workload {w.name}")
     ps = [W.params(w, layer=l) for l in range(nl)]
@@ -682,15 +674,15 @@ def run_layers(args, nl: int):
 
     def prefill_all():
         cur = torch.cuda.current_stream(dev)
-        for ps in pstreams:
-            ps.wait_stream(cur)
+        for s in pstreams:
+            s.wait_stream(cur)
         for l in range(nl):
             q, k, v = qkv[l]
             with torch.cuda.stream(pstreams[l % 2]):
                 ops.prefill_chunked(q, k, v, lams[l], Rs[l], Ds[l], y=ys[l], state=states[l],
                                     workspace=pws[l % 2])
-        for ps in pstreams:
-            cur.wait_stream(ps)
+        for s in pstreams:
+            cur.wait_stream(s)
 
     def decode_all():
         for t in range(w.T):
@@ -707,7 +699,7 @@ def run_layers(args, nl: int):
         decode_all()
     torch.cuda.synchronize(dev)
 
-    def step(ev=None):
+    def step(ev):
         if ev is not None:
             ev[0].record(stream)
         prefill_all()
@@ -717,99 +709,252 @@ def run_layers(args, nl: int):
         if ev is not None:
             ev[2].record(stream)
 
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            step()
-    torch.cuda.synchronize(dev)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(gpu_id_for(dev))
-    clocks.start()
-    time.sleep(0.3)
-    barrier(dev)
-    torch.cuda.synchronize(dev)
-    with torch.cuda.stream(stream):
-        # a short GPU spin ahead of the start event, so that the first step's launches are queued
-        # while the GPU is busy: the timed region then holds device work only, as every later step
-        # does (each is queued while the previous one runs)
-        torch.cuda._sleep(LEAD_SPIN_CYCLES)
-        t_start.record(stream)
-        for i in range(args.steps):
-            step(evs[i])
-        t_end.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(dev)
-    clk = clocks.stop()
-    elapsed_ms = reduce_max(t_start.elapsed_time(t_end), dev)
-    pre_ms = reduce_max(sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps, dev)
-    dec_ms = reduce_max(sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps, dev)
-    ms_per_step = elapsed_ms / args.steps
+    if clocks is not None:
+        clocks.start()
+        time.sleep(0.3)
+    elapsed_ms, (pre_ms, dec_ms) = timed_steps(stream, dev, steps, warmup, step, 2)
+    clk = clocks.stop() if clocks is not None else None
+    ms_per_step = elapsed_ms / steps
     for wsx in pws:
         err = ops.chunked_error(wsx, w.B, w.L, w.Dch, w.H, w.d)
         if err:
             raise SystemExit(f"chunked prefill kernel reported error {err}")
 
     peak, peak_src = load_peaks()
+    key = f"{w.name}/B{w.B}"
     pb, db = algorithmic_bytes(w)
-    pb, db = pb * nl, db * nl
-    pre_gbs = pb / (pre_ms / 1e3) / 1e9
     dec_launch_ms = dec_ms / w.T
-    dec_gbs = db / (dec_launch_ms / 1e3) / 1e9
-    roofs = [{"kernel": f"hyena_prefill_chunked x {nl} layers", "bound": "hbm", "achieved": pre_gbs,
-              "peak": peak, "unit": "GB/s", "frac": pre_gbs / peak, "peak_source": peak_src,
-              "algorithmic_bytes": pb, "launch_ms": pre_ms / nl, "total_ms": pre_ms,
-              "traffic": ncu_traffic("prefill_chunk", f"{w.name}/B{w.B}")},
-             {"kernel": f"hyena_decode_step_layers ({nl} layers per launch)", "bound": "hbm",
-              "achieved": dec_gbs, "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak,
-              "peak_source": peak_src, "algorithmic_bytes": db, "launch_ms": dec_launch_ms,
-              "total_ms": dec_ms, "traffic": ncu_traffic("decode_layers", f"{w.name}/B{w.B}")}]
-    dominant = max(roofs, key=lambda r: r["total_ms"])
-    baselines = None
-    if not args.no_baselines:
+    r_pre = roof(f"hyena_prefill_chunked x {nl} layers", pb * nl, pre_ms, peak, peak_src,
+                 ncu_traffic("prefill_chunk", key), note="per-layer launch: %.1f us, alternating over two streams"
+                 % (1e3 * pre_ms / nl))
+    r_pre["launch_ms"] = pre_ms / nl
+    r_pre["algorithmic_bytes_per_launch"] = pb
+    t_dec = ncu_traffic("decode_layers", key)
+    r_dec = roof(f"hyena_decode_step_layers ({nl} layers per launch)", db * nl, dec_launch_ms, peak, peak_src,
+                 t_dec, dec_ms)
+    rec = {"workload": line_config(w, nl)["workload"], "steps": steps, "warmup": warmup,
+           "ms_per_step": ms_per_step,
+           "value": world * w.B * (w.L + w.T) / (ms_per_step / 1e3), "unit": "tokens/s",
+           "prefill": {"route": "chunked", "tokens_per_s": world * w.B * w.L / (pre_ms / 1e3), "ms": pre_ms,
+                       "hbm_frac": r_pre["frac"], "roofline": r_pre,
+                       "inputs": "q, k, v of %d MiB per layer (larger than L2), drawn on the device"
+                                 % (w.B * w.L * w.Dch * w.act_bytes >> 20)},
+           "decode": {"tokens_per_s": world * w.B * w.T / (dec_ms / 1e3), "ms_per_token_step": dec_launch_ms,
+                      "hbm_frac": r_dec["frac"], "roofline": r_dec,
+                      "state": "%d MiB over %d layers (larger than L2)" % (nl * states[0].numel() * 4 >> 20, nl),
+                      "inputs": f"{pool} distinct device-drawn input sets per layer, cycled"},
+           "roofline_all": [r_pre, r_dec], "roofline": max([r_pre, r_dec], key=lambda x: x["total_ms"]),
+           "launches_per_step": 2 * nl + w.T, "clocks": clk}
+    if with_baselines:
         q0, k0, v0 = qkv[0]
         dq0, dk0, dv0 = dpool[0]
         # tokens around the middle of the generation: history of ~L + T/2 tokens per layer
         wl = w.with_(L=w.L + w.T // 2)
         k_hist = torch.cat([k0, dk0.transpose(0, 1).repeat(1, w.T // 2 // pool + 1, 1)[:, :w.T // 2]], 1)
         v_hist = torch.cat([v0, dv0.transpose(0, 1).repeat(1, w.T // 2 // pool + 1, 1)[:, :w.T // 2]], 1)
-        baselines = fir_baseline(ops, W, wl, None, k_hist.contiguous(), v_hist.contiguous(), dq0, dk0, dv0,
-                                 lams[0], Rs[0], Ds[0], stream, dev, 8, dec_ms / w.T, pre_ms, peak, layers=nl)
+        rec["baselines"] = fir_baseline(ops, W, wl, None, k_hist.contiguous(), v_hist.contiguous(), dq0, dk0,
+                                        dv0, lams[0], Rs[0], Ds[0], stream, dev, 8, dec_launch_ms, pre_ms, peak,
+                                        layers=nl)
         del k_hist, v_hist
-    cpu = None
-    if world == 1 and not args.no_cpu_baseline:
-        import oracle
-        oracle.build()
-        sample = OracleSample(w)
-        channels, reps = sample.calibrate(12.0)
-        dt, tok = sample.run_reps(channels, reps)
-        cpu = {"value": tok / dt / nl, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
-               "sample": (f"fp64 oracle, recurrent mode, layer 0 only: {reps} pass(es) over all {w.B} "
-                          f"sequences x first {channels} of {w.Dch} channels ({w.L}-token prompt + {w.T} "
-                          f"decode tokens), {dt:.1f} s; tokens/s of one layer divided by {nl} layers")}
-    if rank == 0:
-        cfg = workload_config(w)
-        cfg["layers"] = nl
-        cfg["workload"] += f", {nl} independent layers (all timed)"
-        cfg["prefill_route"] = "chunked"
-        cfg["l2"] = ("prefill inputs larger than L2 (3 x %d MiB per layer); decode states %d MiB in total"
-                     % (qkv[0][0].numel() * 2 >> 20, nl * states[0].numel() * 4 >> 20))
-        cfg["decode_inputs"] = f"{pool} distinct device-drawn input sets per layer, cycled"
-        tokens_step = w.B * (w.L + w.T)
-        line = {"metric": METRIC, "value": world * tokens_step / (ms_per_step / 1e3), "unit": "tokens/s",
-                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic (device-drawn, seeded)",
-                "config": cfg,
-                "prefill": {"tokens_per_s": world * w.B * w.L / (pre_ms / 1e3), "ms": pre_ms,
-                            "hbm_frac": pre_gbs / peak},
-                "decode": {"tokens_per_s": world * w.B * w.T / (dec_ms / 1e3),
-                           "ms_per_token_step": dec_launch_ms, "hbm_frac": dec_gbs / peak},
-                "baselines": baselines,
-                "roofline": dominant, "roofline_all": roofs, "cpu_baseline": cpu,
-                "e2e": None, "e2e_note": "not measured for the multi-layer workload (9.6 GB of prompt per step)",
-                "gpu_launches": args.steps * (2 * nl + w.T), "clocks": clk}
-        print(json.dumps(line), flush=True)
     del g
+
+    # ---- end to end through the C ABI: every step copies every layer's prompt q, k, v in from pinned
+    # host memory and its y out, then every decode token's q, k, v of all layers in and its y out.
+    # Prefill: two device buffer sets, so layer l+1's prompt travels in while layer l computes and
+    # layer l-1's y travels out.  Decode: blocks of S tokens, two device blocks; a block's inputs
+    # (S tokens x all layers, one copy) travel in while the previous block decodes (CUDA graph per
+    # device block), and its outputs travel out after it.
+    if with_e2e:
+        S = 64
+        nblk = (w.T + S - 1) // S
+        # host memory: every layer's prompt (pinned, distinct per layer); one pinned block of S decode
+        # tokens' inputs, tiled from the device input pool and copied in for every block; outputs to
+        # two pinned prompt-y buffers and two pinned decode-y blocks, alternating
+        hp = [[make_pinned(t.shape, t.dtype) for t in qkv[l]] for l in range(nl)]
+        for l in range(nl):
+            for j in range(3):
+                hp[l][j].copy_(qkv[l][j])
+        hblk = make_pinned((S, nl, 3, w.B, w.Dch), w.torch_dtype)
+        for t in range(S):
+            for l in range(nl):
+                for j in range(3):
+                    hblk[t, l, j].copy_(dpool[l][j][t % pool])
+        hy = [make_pinned(qkv[0][0].shape, w.torch_dtype) for _ in range(2)]
+        hyd = [make_pinned((S, nl, w.B, w.Dch), w.torch_dtype) for _ in range(2)]
+        dset = [[torch.empty_like(qkv[0][0]) for _ in range(4)] for _ in range(2)]     # q, k, v, y
+        dblk = [torch.empty((S, nl, 3, w.B, w.Dch), dtype=w.torch_dtype, device=dev) for _ in range(2)]
+        dyb = [torch.empty((S, nl, w.B, w.Dch), dtype=w.torch_dtype, device=dev) for _ in range(2)]
+        torch.cuda.synchronize(dev)
+
+        def dec_block(j):
+            for t in range(S):
+                ops.decode_step_layers(ls, [dblk[j][t, l, 0] for l in range(nl)], [dblk[j][t, l, 1] for l in range(nl)],
+                                       [dblk[j][t, l, 2] for l in range(nl)], [dyb[j][t, l] for l in range(nl)])
+        graphs = []
+        for j in range(2):
+            with torch.cuda.stream(stream):
+                dec_block(j)
+            torch.cuda.synchronize(dev)
+            gj = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gj, stream=stream):
+                dec_block(j)
+            graphs.append(gj)
+        torch.cuda.synchronize(dev)
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev = lambda: torch.cuda.Event()
+        pc, po = [ev(), ev()], [ev(), ev()]       # prompt set j: computed / y copied out
+        dc, do = [ev(), ev()], [ev(), ev()]       # decode block j: decoded / y copied out
+        for e in pc + po + dc + do:
+            e.record(stream)
+        bi = nl * 3 * qkv[0][0].numel() * w.act_bytes + nblk * S * nl * 3 * w.B * w.Dch * w.act_bytes
+        bo = nl * qkv[0][0].numel() * w.act_bytes + nblk * S * nl * w.B * w.Dch * w.act_bytes
+
+        def e2e_step():
+            for l in range(nl):
+                j = l % 2
+                s_in.wait_event(pc[j])
+                with torch.cuda.stream(s_in):
+                    for x in range(3):
+                        dset[j][x].copy_(hp[l][x], non_blocking=True)
+                got = ev()
+                got.record(s_in)
+                stream.wait_event(got)
+                stream.wait_event(po[j])
+                with torch.cuda.stream(stream):
+                    ops.prefill_chunked(dset[j][0], dset[j][1], dset[j][2], lams[l], Rs[l], Ds[l], y=dset[j][3],
+                                        state=states[l], workspace=pws[j])
+                pc[j].record(stream)
+                s_out.wait_event(pc[j])
+                with torch.cuda.stream(s_out):
+                    hy[j].copy_(dset[j][3], non_blocking=True)
+                po[j].record(s_out)
+            for bk in range(nblk):
+                j = bk % 2
+                s_in.wait_event(dc[j])
+                with torch.cuda.stream(s_in):
+                    dblk[j].copy_(hblk, non_blocking=True)
+                got = ev()
+                got.record(s_in)
+                stream.wait_event(got)
+                stream.wait_event(do[j])
+                with torch.cuda.stream(stream):
+                    graphs[j].replay()
+                dc[j].record(stream)
+                s_out.wait_event(dc[j])
+                with torch.cuda.stream(s_out):
+                    hyd[j].copy_(dyb[j], non_blocking=True)
+                do[j].record(s_out)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(dev)
+        torch.cuda.synchronize(dev)
+        s_in.wait_stream(torch.cuda.current_stream(dev))
+        a.record(s_in)
+        for _ in range(e2e_steps):
+            e2e_step()
+        s_out.wait_stream(stream)
+        s_out.wait_stream(s_in)
+        b.record(s_out)
+        torch.cuda.synchronize(dev)
+        e2e_ms = reduce_max(a.elapsed_time(b), dev) / e2e_steps
+        for wsx in pws:
+            err = ops.chunked_error(wsx, w.B, w.L, w.Dch, w.H, w.d)
+            if err:
+                raise SystemExit(f"chunked prefill kernel reported error {err} (end-to-end run)")
+        rec["e2e"] = {"value": world * w.B * (w.L + w.T) / (e2e_ms / 1e3), "unit": "tokens/s",
+                      "ms_per_step": e2e_ms, "steps": e2e_steps, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+                      "overlap": (f"prompt: two device buffer sets, layer l+1 copied in while layer l computes; "
+                                  f"decode: blocks of {S} tokens x {nl} layers, two device blocks; copy-in, compute "
+                                  f"and copy-out streams"),
+                      "host_buffers": ("every layer's prompt distinct in pinned memory; one pinned block of "
+                                       f"{S} tokens' decode inputs, copied in for each of the {nblk} blocks; "
+                                       "outputs to two alternating pinned buffers")}
+        del graphs
+    return rec
+
+
+# ------------------------------------------------------------------ our arm
+SUBRECORDS = [
+    # (name, workload, batch override, steps, e2e, fft route, baselines)
+    ("mid_bf16", "mid_bf16", 0, None, True, True, True),
+    ("long_prefill_bf16", "long_prefill_bf16", 0, None, True, True, False),
+    ("decode_sweep_bf16/B1", "decode_sweep_bf16", 1, 5, False, False, False),
+    ("decode_sweep_bf16/B16", "decode_sweep_bf16", 16, 5, False, False, False),
+    ("decode_sweep_bf16/B64", "decode_sweep_bf16", 64, 5, False, False, False),
+    ("decode_sweep_bf16/B256", "decode_sweep_bf16", 256, 5, False, False, False),
+    ("decode_sweep_bf16/B1024", "decode_sweep_bf16", 1024, 5, False, False, False),
+]
+
+
+def run_ours(args):
+    import torch
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init("nccl")
+    from distilled_ssm_decode_b200 import build, ops
+    from distilled_ssm_decode_b200 import workloads as W
+    build.build()
+    ops.lib()
+
+    w = W.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.with_(B=args.batch)
+    nl = args.layers or w.layers
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    clocks = ClockSampler(gpu_id_for(dev))
+    if nl > 1:
+        head = measure_layers(args, w, nl, dev, args.steps, args.warmup, e2e_steps, not args.no_baselines,
+                              not args.no_e2e, clocks)
+        clk = head.pop("clocks")
+    else:
+        clocks.start()
+        time.sleep(0.3)
+        head = measure_single(args, w, dev, args.steps, args.warmup, e2e_steps, not args.no_fft_route,
+                              not args.no_baselines, not args.no_e2e)
+        clk = clocks.stop()
+    torch.cuda.synchronize(dev)
+
+    # sub-records: the other workloads, each timed on its own (1 GPU only)
+    subs = None
+    if world == 1 and not args.no_subrecords and args.workload == DEFAULT_WORKLOAD and not args.batch:
+        subs = {}
+        for name, wl, batch, steps, e2e, fft, base in SUBRECORDS:
+            ws = W.WORKLOADS[wl]
+            if batch:
+                ws = ws.with_(B=batch)
+            st = steps or args.steps
+            subs[name] = measure_single(args, ws, dev, st, args.warmup, e2e_steps, fft and not args.no_fft_route,
+                                        base and not args.no_baselines, e2e and not args.no_e2e)
+            torch.cuda.empty_cache()
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline and w.L > 0:
+        cpu, _, _, _ = oracle_baseline(w, nl, 12.0)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16" if w.dtype == "bf16" else "f32",
+                "data": "synthetic (seeded; drawn on the device for the multi-layer workload)" if nl > 1 else "synthetic (seeded)",
+                "config": line_config(w, nl),
+                "value_definition": "(prompt + generated) tokens per second through every layer: "
+                                    "B x (L + T) tokens per step / step time, summed over GPUs",
+                "prefill": head.get("prefill"), "decode": head.get("decode"),
+                "roofline": head["roofline"], "roofline_all": head["roofline_all"],
+                "cpu_baseline": cpu, "e2e": head.get("e2e"),
+                "gpu_launches": args.steps * head["launches_per_step"], "clocks": clk}
+        for k in ("prefill_fft_route", "baselines"):
+            if k in head:
+                line[k] = head[k]
+        if subs is not None:
+            line["subrecords"] = subs
+        print(json.dumps(line), flush=True)
     import torch.distributed as dist
     if dist.is_initialized():
         dist.destroy_process_group()
@@ -849,13 +994,16 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mid_bf16")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size")
     ap.add_argument("--prefill", choices=["auto", "chunked", "fft"], default="auto",
                     help="prefill route: chunked tensor-core evaluation (auto when supported) or FFT")
     ap.add_argument("--no-fft-route", action="store_true",
                     help="skip the extra timing of the FFT route when the chunked route is used")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5, help="timed end-to-end steps (at most --steps)")
+    ap.add_argument("--no-subrecords", action="store_true",
+                    help="only the headline workload (the default run adds the other workloads' records)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-baselines", action="store_true",
                     help="skip the undistilled (FIR / re-prefill) decode baselines")
@@ -869,10 +1017,6 @@ def main(argv=None):
         return run_reference(args)
     if args.truncation:
         return run_truncation(args)
-    from distilled_ssm_decode_b200 import workloads as W
-    nl = args.layers or W.WORKLOADS[args.workload].layers
-    if nl > 1:
-        return run_layers(args, nl)
     return run_ours(args)
 
 
