@@ -1,10 +1,14 @@
 """Build libhyena_b200.so in-tree with nvcc for sm_100a.
 
-    python -m distilled_ssm_decode_b200.build [--force] [--verbose]
+    python -m distilled_ssm_decode_b200.build [--force] [--verbose] [--debug-bounds]
 
 Each .cu under csrc/ is compiled to an object in _build/ (in parallel), then
 linked into distilled_ssm_decode_b200/libhyena_b200.so.  The CUDA runtime is
 linked statically, so the library needs only the driver at run time.
+
+--debug-bounds builds the bounds-checked variant, libhyena_b200_dbg.so (objects in
+_build/dbg/, -DHYENA_DEBUG_BOUNDS): every kernel checks the index of each global
+load and store and records the first one out of range instead of making it.
 """
 from __future__ import annotations
 
@@ -20,6 +24,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libhyena_b200.so")
+LIB_DBG = os.path.join(PKG, "libhyena_b200_dbg.so")
 INCLUDE = os.path.join(ROOT, "include")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -49,16 +54,19 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+def build(force: bool = False, verbose: bool = False, extra=(), debug_bounds: bool = False) -> str:
     deps = _deps()
-    if not force and not _stale(LIB, deps + [__file__]):
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+    lib = LIB_DBG if debug_bounds else LIB
+    bdir = os.path.join(BUILD, "dbg") if debug_bounds else BUILD
+    extra = list(extra) + (["-DHYENA_DEBUG_BOUNDS"] if debug_bounds else [])
+    if not force and not _stale(lib, deps + [__file__]):
+        return lib
+    os.makedirs(bdir, exist_ok=True)
     cc = nvcc()
     objs = []
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(bdir, os.path.basename(src)[:-3] + ".o")
         cmd = [cc] + ARCH + NVCC_FLAGS + list(extra) + ["-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
@@ -71,15 +79,15 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
 
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         objs = list(ex.map(compile_one, sources()))
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [cc] + ARCH + ["-shared", "-Xcompiler", "-fPIC", "-cudart", "static", "-o", tmp] + objs
     if verbose:
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 def main(argv=None):
@@ -87,9 +95,11 @@ def main(argv=None):
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-v", action="store_true", help="print register/smem usage")
+    ap.add_argument("--debug-bounds", action="store_true", help="build the bounds-checked variant")
     a = ap.parse_args(argv)
     extra = ["-Xptxas", "-v"] if a.ptxas_v else []
-    print(build(force=a.force or a.ptxas_v, verbose=a.verbose or a.ptxas_v, extra=extra))
+    print(build(force=a.force or a.ptxas_v, verbose=a.verbose or a.ptxas_v, extra=extra,
+                debug_bounds=a.debug_bounds))
 
 
 if __name__ == "__main__":

@@ -191,6 +191,30 @@ int hyena_prefill_chunked(const void *q, const void *k, const void *v, int dtype
                                               workspace, s));
 }
 
+int hyena_debug_bounds_check(long long *record) {
+    if (!record) return HYENA_ERR_ARG;
+    for (int i = 0; i < 4; ++i) record[i] = 0;
+    if (!kBoundsChecked) return HYENA_ERR_UNSUPPORTED;
+    // file ids as documented in hyena.h
+    int (*const readers[])(long long *) = {bounds_read_decode, bounds_read_filter, bounds_read_fir,
+                                           bounds_read_prefill_chunked, bounds_read_prefill_fft,
+                                           bounds_read_state, bounds_read_truncate};
+    int found = 0;
+    for (int f = 0; f < 7; ++f) {
+        long long rec[4];
+        const int r = readers[f](rec);      // every record is read (and cleared), the first one kept
+        if (r < 0) return HYENA_ERR_CUDA;
+        if (r > 0 && !found) {
+            found = 1;
+            record[0] = f + 1;
+            record[1] = rec[1];
+            record[2] = rec[2];
+            record[3] = rec[3];
+        }
+    }
+    return found;
+}
+
 int hyena_test_chunked_inject(int suppress_item, double lookback_limit_s) {
     if (suppress_item < -1 || !(lookback_limit_s >= 0.0) || lookback_limit_s > 60.0) return HYENA_ERR_ARG;
     chunked_inject(suppress_item, (unsigned long long)(lookback_limit_s * 1e9));

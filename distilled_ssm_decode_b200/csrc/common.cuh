@@ -9,6 +9,51 @@
 
 namespace hyena {
 
+// ---------------------------------------------------------------- bounds-checked build
+// Built with -DHYENA_DEBUG_BOUNDS (libhyena_b200_dbg.so), the kernels check the index of each
+// global load and store against the extent their arguments give that buffer.  The first index
+// out of range is recorded in a device record of the source file (source line, index, extent)
+// and the access is skipped: a store is dropped, a load reads element 0 instead.  There is no
+// trap and no fault; the host reads and clears the records with hyena_debug_bounds_check().
+// In the release build both macros are the plain index (no code).
+#ifdef HYENA_DEBUG_BOUNDS
+static __device__ unsigned long long g_hb_rec[4];   // one record per source file (internal linkage)
+__device__ __forceinline__ bool hb_ok(long long i, long long n, int line) {
+    if (i >= 0 && i < n) return true;
+    if (atomicCAS(&g_hb_rec[0], 0ull, 1ull) == 0ull) {
+        g_hb_rec[1] = (unsigned long long)line;
+        g_hb_rec[2] = (unsigned long long)i;
+        g_hb_rec[3] = (unsigned long long)n;
+    }
+    return false;
+}
+#define HB_OK(i, n) (::hyena::hb_ok((long long)(i), (long long)(n), __LINE__))
+#define HB_IDX(i, n) (HB_OK(i, n) ? (i) : 0)
+// reads and clears this file's record: 1 and rec = {1, line, index, extent} if an access was
+// out of range, 0 if none, -1 if the record could not be read
+#define HYENA_BOUNDS_READER(NAME)                                                              \
+    int bounds_read_##NAME(long long *rec) {                                                   \
+        unsigned long long r[4] = {0, 0, 0, 0}, z[4] = {0, 0, 0, 0};                           \
+        if (cudaMemcpyFromSymbol(r, g_hb_rec, sizeof(r)) != cudaSuccess) return -1;            \
+        if (cudaMemcpyToSymbol(g_hb_rec, z, sizeof(z)) != cudaSuccess) return -1;              \
+        for (int i = 0; i < 4; ++i) rec[i] = (long long)r[i];                                  \
+        return r[0] != 0;                                                                      \
+    }
+#else
+#define HB_OK(i, n) true
+#define HB_IDX(i, n) (i)
+#define HYENA_BOUNDS_READER(NAME)                                                              \
+    int bounds_read_##NAME(long long *rec) {                                                   \
+        for (int i = 0; i < 4; ++i) rec[i] = 0;                                                \
+        return 0;                                                                              \
+    }
+#endif
+#ifdef HYENA_DEBUG_BOUNDS
+constexpr bool kBoundsChecked = true;
+#else
+constexpr bool kBoundsChecked = false;
+#endif
+
 // ---------------------------------------------------------------- activations
 // Activation element types.  Loads widen to fp32; stores round to nearest-even.
 struct ActF32 {

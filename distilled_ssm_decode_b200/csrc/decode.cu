@@ -53,35 +53,39 @@ __device__ __forceinline__ void decode_pairs(const typename Act::T *__restrict__
     const int hd = c / ch;
 
     const size_t srow = (size_t)Dch >> 1;                    // float4 per mode row
-    float4 *sp = state + (size_t)b * d * srow + (c >> 1);
+    const size_t sbase = (size_t)b * d * srow + (c >> 1);
+    float4 *sp = state + sbase;
     const float2 *lh = lam + (size_t)hd * d;
     const float2 *rh = R + (size_t)hd * d;
+    // extents for the bounds-checked build: state rows, activations, per-head parameters
+    const long long n_state = (long long)B * d * srow, n_act = (long long)B * Dch, n_par = (long long)(Dch / ch) * d;
+    (void)n_state; (void)n_act; (void)n_par;
 
     float ua = 0.f, ub = 0.f;
     float2 qq = make_float2(0.f, 0.f);
     float acc_a = 0.f, acc_b = 0.f;
     float D = 0.f;
-    if (kEarly && valid && g == 0) D = __ldg(&Dskip[hd]);
+    if (kEarly && valid && g == 0) D = __ldg(&Dskip[HB_IDX(hd, Dch / ch)]);
     for (int n0 = g; n0 < d; n0 += NG * MPT) {
         float4 s[MPT];
         float2 re[MPT], le[MPT];
 #pragma unroll
         for (int i = 0; i < MPT; ++i) {
             const int n = n0 + i * NG;
-            if (valid && n < d) s[i] = sp[(size_t)n * srow];
+            if (valid && n < d) s[i] = sp[HB_IDX((long long)n * srow, n_state - (long long)sbase)];
         }
         if constexpr (kEarly) {
 #pragma unroll
             for (int i = 0; i < MPT; ++i) {
                 const int n = n0 + i * NG;
                 if (valid && n < d) {
-                    re[i] = __ldg(&rh[n]);
-                    le[i] = __ldg(&lh[n]);
+                    re[i] = __ldg(&rh[HB_IDX(n, n_par - (long long)hd * d)]);
+                    le[i] = __ldg(&lh[HB_IDX(n, n_par - (long long)hd * d)]);
                 }
             }
         }
         if (n0 == g && valid) {   // activations: issued after the first state loads
-            const size_t o = (size_t)b * Dch + c;
+            const size_t o = HB_OK((long long)b * Dch + c + 1, n_act) ? (size_t)b * Dch + c : 0;
             const float2 kk = Act::ld2(k + o), vv = Act::ld2(v + o);
             qq = Act::ld2(q + o);
             ua = kk.x * vv.x;
@@ -91,8 +95,8 @@ __device__ __forceinline__ void decode_pairs(const typename Act::T *__restrict__
         for (int i = 0; i < MPT; ++i) {
             const int n = n0 + i * NG;
             if (valid && n < d) {
-                const float2 r = kEarly ? re[i] : __ldg(&rh[n]);
-                const float2 l = kEarly ? le[i] : __ldg(&lh[n]);
+                const float2 r = kEarly ? re[i] : __ldg(&rh[HB_IDX(n, n_par - (long long)hd * d)]);
+                const float2 l = kEarly ? le[i] : __ldg(&lh[HB_IDX(n, n_par - (long long)hd * d)]);
                 acc_a = fmaf(r.x, s[i].x, fmaf(-r.y, s[i].y, acc_a));
                 acc_b = fmaf(r.x, s[i].z, fmaf(-r.y, s[i].w, acc_b));
                 float4 t;
@@ -100,7 +104,7 @@ __device__ __forceinline__ void decode_pairs(const typename Act::T *__restrict__
                 t.y = fmaf(l.x, s[i].y, l.y * s[i].x);
                 t.z = fmaf(l.x, s[i].z, fmaf(-l.y, s[i].w, ub));
                 t.w = fmaf(l.x, s[i].w, l.y * s[i].z);
-                sp[(size_t)n * srow] = t;
+                if (HB_OK((long long)sbase + (long long)n * srow, n_state)) sp[(size_t)n * srow] = t;
             }
         }
     }
@@ -109,8 +113,9 @@ __device__ __forceinline__ void decode_pairs(const typename Act::T *__restrict__
         acc_b += __shfl_xor_sync(0xffffffffu, acc_b, off);
     }
     if (valid && g == 0) {
-        if (!kEarly) D = __ldg(&Dskip[hd]);
-        Act::st2(y + (size_t)b * Dch + c, qq.x * fmaf(D, ua, acc_a), qq.y * fmaf(D, ub, acc_b));
+        if (!kEarly) D = __ldg(&Dskip[HB_IDX(hd, Dch / ch)]);
+        if (HB_OK((long long)b * Dch + c + 1, n_act))
+            Act::st2(y + (size_t)b * Dch + c, qq.x * fmaf(D, ua, acc_a), qq.y * fmaf(D, ub, acc_b));
     }
 }
 
@@ -125,7 +130,8 @@ __device__ __forceinline__ void pdl_enter(const typename Act::T *q, const typena
     const int lane = threadIdx.x & 31, ppw = 32 >> lg_ng;
     const long long pair_id = (gtid >> 5) * ppw + (lane & (ppw - 1));
     constexpr int kPairsPerLine = 128 / (2 * Act::bytes);
-    if ((lane >> (5 - lg_ng)) == 0 && pair_id % kPairsPerLine == 0 && pair_id < (long long)B * (Dch >> 1)) {
+    if ((lane >> (5 - lg_ng)) == 0 && pair_id % kPairsPerLine == 0 && pair_id < (long long)B * (Dch >> 1) &&
+        HB_OK(pair_id * 2 + 1, (long long)B * Dch)) {
         const size_t o = (size_t)pair_id * 2;    // element offset of the pair in [B][Dch]
         asm volatile("prefetch.global.L2 [%0];" ::"l"(q + o));
         asm volatile("prefetch.global.L2 [%0];" ::"l"(k + o));
@@ -184,19 +190,23 @@ decode_scalar_kernel(const typename Act::T *__restrict__ q, const typename Act::
     const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (gtid >= (long long)B * Dch) return;
     const int b = (int)(gtid / Dch), c = (int)(gtid % Dch);
-    const int hd = c / ch;
-    const size_t o = (size_t)b * Dch + c;
+    const int hd = c / ch, H = Dch / ch;
+    const long long n_act = (long long)B * Dch, n_state = (long long)B * d * Dch, n_par = (long long)H * d;
+    (void)n_state; (void)n_par;
+    const size_t o = HB_IDX((size_t)b * Dch + c, n_act);
     const float u = Act::ld(k + o) * Act::ld(v + o);
     float acc = 0.f;
-    float2 *sp = state + (size_t)b * d * Dch + c;
+    const size_t sbase = (size_t)b * d * Dch + c;
     for (int n = 0; n < d; ++n) {
-        const float2 s = sp[(size_t)n * Dch];
-        const float2 r = __ldg(&R[(size_t)hd * d + n]);
-        const float2 l = __ldg(&lam[(size_t)hd * d + n]);
+        const size_t si = HB_IDX(sbase + (size_t)n * Dch, n_state);
+        const float2 s = state[si];
+        const float2 r = __ldg(&R[HB_IDX((size_t)hd * d + n, n_par)]);
+        const float2 l = __ldg(&lam[HB_IDX((size_t)hd * d + n, n_par)]);
         acc = fmaf(r.x, s.x, fmaf(-r.y, s.y, acc));
-        sp[(size_t)n * Dch] = make_float2(fmaf(l.x, s.x, fmaf(-l.y, s.y, u)), fmaf(l.x, s.y, l.y * s.x));
+        if (HB_OK(sbase + (size_t)n * Dch, n_state))
+            state[si] = make_float2(fmaf(l.x, s.x, fmaf(-l.y, s.y, u)), fmaf(l.x, s.y, l.y * s.x));
     }
-    Act::st(y + o, Act::ld(q + o) * fmaf(__ldg(&Dskip[hd]), u, acc));
+    if (HB_OK(o, n_act)) Act::st(y + o, Act::ld(q + o) * fmaf(__ldg(&Dskip[HB_IDX(hd, H)]), u, acc));
 }
 
 // Lanes per pair (NG = 2^lg), modes per thread (MPT) and block size, from a sweep on B200 of
@@ -300,6 +310,8 @@ cudaError_t decode_launch(const void *q, const void *k, const void *v, int B, in
 }
 
 }  // namespace
+
+HYENA_BOUNDS_READER(decode)
 
 cudaError_t launch_decode_step(const void *q, const void *k, const void *v, int dtype,
                                int B, int Dch, int H, int d, const float2 *lam, const float2 *R,

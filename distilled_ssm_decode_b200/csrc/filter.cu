@@ -20,7 +20,8 @@ constexpr int kRun = 16;
 __global__ void __launch_bounds__(128)
 filter_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R,
               const float *__restrict__ Dskip, int d, int L, float *__restrict__ h) {
-    const int hd = blockIdx.y;
+    const int hd = blockIdx.y, H = gridDim.y;
+    (void)H;
     const long long j0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * kRun;
     if (j0 >= L) return;
     double acc[kRun];
@@ -29,8 +30,8 @@ filter_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R,
     // tap j >= 1 uses lambda^(j-1); the run starts at power max(j0-1, 0)
     const long long p0 = j0 > 0 ? j0 - 1 : 0;
     for (int n = 0; n < d; ++n) {
-        const float2 lf = __ldg(&lam[(size_t)hd * d + n]);
-        const float2 rf = __ldg(&R[(size_t)hd * d + n]);
+        const float2 lf = __ldg(&lam[HB_IDX((size_t)hd * d + n, (long long)H * d)]);
+        const float2 rf = __ldg(&R[HB_IDX((size_t)hd * d + n, (long long)H * d)]);
         const cd l{lf.x, lf.y};
         cd p = cdpow(l, p0);
 #pragma unroll
@@ -46,10 +47,12 @@ filter_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R,
 #pragma unroll
     for (int r = 0; r < kRun; ++r) {
         const long long j = j0 + r;
-        if (j < L) out[j] = (j == 0) ? Dskip[hd] : (float)acc[r];
+        if (j < L && HB_OK((long long)hd * L + j, (long long)H * L)) out[j] = (j == 0) ? Dskip[HB_IDX(hd, H)] : (float)acc[r];
     }
 }
 }  // namespace
+
+HYENA_BOUNDS_READER(filter)
 
 cudaError_t launch_filter(const float2 *lam, const float2 *R, const float *Dskip,
                           int H, int d, int L, float *h, cudaStream_t s) {

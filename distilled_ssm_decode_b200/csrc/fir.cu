@@ -36,7 +36,8 @@ fir_fill_kernel(const typename Act::T *__restrict__ k, const typename Act::T *__
     for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
          e += (long long)gridDim.x * blockDim.x) {
         const long long b = e / row, r = e - b * row;
-        u_cache[b * t_max * Dch + r] = Act::ld(k + e) * Act::ld(v + e);
+        if (HB_OK(b * t_max * Dch + r, (long long)B * t_max * Dch))
+            u_cache[b * t_max * Dch + r] = Act::ld(k + HB_IDX(e, n)) * Act::ld(v + HB_IDX(e, n));
     }
 }
 
@@ -52,6 +53,10 @@ fir_step_kernel(const typename Act::T *__restrict__ q, const typename Act::T *__
     const int hd = valid ? c / ch : 0;
     const float *hh = h + (size_t)hd * t_max;            // taps of this channel's head
     float *uc = u_cache + (size_t)b * t_max * Dch + c;
+    // extents (bounds-checked build), relative to hh and uc
+    const long long n_h = (long long)(Dch / ch) * t_max - (long long)hd * t_max;
+    const long long n_u = (long long)gridDim.y * t_max * Dch - ((long long)b * t_max * Dch + c);
+    (void)n_h; (void)n_u;
     float acc = 0.f;
     if (valid) {
         // rows j < t come from the cache; row t (this token) is added below from registers
@@ -60,13 +65,13 @@ fir_step_kernel(const typename Act::T *__restrict__ q, const typename Act::T *__
             float u[kUnroll], w[kUnroll];
 #pragma unroll
             for (int i = 0; i < kUnroll; ++i) {
-                u[i] = __ldcs(uc + (size_t)(j + i * kSlices) * Dch);
-                w[i] = __ldg(hh + (t - j - i * kSlices));
+                u[i] = __ldcs(uc + HB_IDX((size_t)(j + i * kSlices) * Dch, n_u));
+                w[i] = __ldg(hh + HB_IDX(t - j - i * kSlices, n_h));
             }
 #pragma unroll
             for (int i = 0; i < kUnroll; ++i) acc = fmaf(w[i], u[i], acc);
         }
-        for (; j < t; j += kSlices) acc = fmaf(__ldg(hh + (t - j)), __ldcs(uc + (size_t)j * Dch), acc);
+        for (; j < t; j += kSlices) acc = fmaf(__ldg(hh + HB_IDX(t - j, n_h)), __ldcs(uc + HB_IDX((size_t)j * Dch, n_u)), acc);
     }
     part[slice][lane] = acc;
     __syncthreads();
@@ -74,14 +79,17 @@ fir_step_kernel(const typename Act::T *__restrict__ q, const typename Act::T *__
         float s = 0.f;
 #pragma unroll
         for (int w = 0; w < kSlices; ++w) s += part[w][lane];
-        const size_t o = (size_t)b * Dch + c;
+        const size_t o = HB_IDX((size_t)b * Dch + c, (long long)gridDim.y * Dch);
         const float u = Act::ld(k + o) * Act::ld(v + o);
-        uc[(size_t)t * Dch] = u;                              // append this token to the history
-        Act::st(y + o, Act::ld(q + o) * fmaf(__ldg(hh), u, s));
+        if (HB_OK((size_t)t * Dch, n_u)) uc[(size_t)t * Dch] = u;     // append this token to the history
+        if (HB_OK((size_t)b * Dch + c, (long long)gridDim.y * Dch))
+            Act::st(y + o, Act::ld(q + o) * fmaf(__ldg(hh + HB_IDX(0, n_h)), u, s));
     }
 }
 
 }  // namespace
+
+HYENA_BOUNDS_READER(fir)
 
 cudaError_t launch_fir_fill(const void *k, const void *v, int dtype, int B, int L, int Dch, int t_max,
                             float *u_cache, cudaStream_t s) {

@@ -74,4 +74,14 @@ cudaError_t launch_fir_step(const void *q, const void *k, const void *v, int dty
 cudaError_t launch_modal_truncate(const float2 *lam, const float2 *R, int H, int d, int k, int *kept,
                                   float2 *lam_out, float2 *R_out, double *bound, double *err_l2, cudaStream_t s);
 
+// bounds-checked build: per source file, read and clear the record of the first global access
+// out of range (see common.cuh); in the release build they report nothing
+int bounds_read_decode(long long *rec);
+int bounds_read_filter(long long *rec);
+int bounds_read_fir(long long *rec);
+int bounds_read_prefill_chunked(long long *rec);
+int bounds_read_prefill_fft(long long *rec);
+int bounds_read_state(long long *rec);
+int bounds_read_truncate(long long *rec);
+
 }  // namespace hyena

@@ -380,9 +380,11 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
     __shared__ float2 ls[kMaxModes], rs[kMaxModes];   // lambda_n, R_n
     __shared__ float hs[kC];                     // filter taps h_0 .. h_{C-1}
     __shared__ float dskip;
-    if (t < kMaxModes) ls[t] = t < d ? lam[(size_t)hd * d + t] : make_float2(0.f, 0.f);
-    else if (t < 2 * kMaxModes) rs[t - kMaxModes] = t - kMaxModes < d ? R[(size_t)hd * d + t - kMaxModes] : make_float2(0.f, 0.f);
-    else if (t == 2 * kMaxModes) dskip = Dskip[hd];
+    const long long n_par = (long long)gridDim.x * d;
+    (void)n_par;
+    if (t < kMaxModes) ls[t] = t < d ? lam[HB_IDX((size_t)hd * d + t, n_par)] : make_float2(0.f, 0.f);
+    else if (t < 2 * kMaxModes) rs[t - kMaxModes] = t - kMaxModes < d ? R[HB_IDX((size_t)hd * d + t - kMaxModes, n_par)] : make_float2(0.f, 0.f);
+    else if (t == 2 * kMaxModes) dskip = Dskip[HB_IDX(hd, gridDim.x)];
     __syncthreads();
     {
         const int n = t / kC, k = t % kC;
@@ -421,8 +423,9 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
                 v[x] = (r & (kIm - 1)) < d ? (r < kIm ? q.x : q.y) : 0.f;
             }
         }
-        *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(FA) + cm_off16(row, io0, kC)) =
-            make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+        if (HB_OK(cm_off16(row, io0, kC) + 15, kFABytes))
+            *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(FA) + cm_off16(row, io0, kC)) =
+                make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
     }
     // carry A operand: rows 0..C-1: (Re, -Im) of R_n lambda_n^tau; rows C..127 zero
     if (t < 128 * (kKS / 8)) {
@@ -438,8 +441,9 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
                 v[x] = r < kIm ? c.x : -c.y;
             }
         }
-        *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(CA) + cm_off16(row, r0, kKS)) =
-            make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+        if (HB_OK(cm_off16(row, r0, kKS) + 15, kCABytes))
+            *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(CA) + cm_off16(row, r0, kKS)) =
+                make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
     }
 }
 
@@ -699,7 +703,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int v = pubq[ps];
                 if (v < 0) break;
                 __threadfence();
-                if ((v >> 2) != a.suppress_item) atomicExch(a.status + (v >> 2), v & 3);
+                if ((v >> 2) != a.suppress_item && HB_OK(v >> 2, (long long)a.H * a.ih)) atomicExch(a.status + (v >> 2), v & 3);
                 tc::mbar_arrive(bar(kBarPubEmpty + ps));
             }
         }
@@ -741,7 +745,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         ++fphase;
                     }
                     tc::mbar_expect_tx(bar(kBarConst), kOpBytes);
-                    tc::bulk_load(sbase + kSmFA, a.consts + (size_t)it.hd * kConstStride, kOpBytes, bar(kBarConst));
+                    tc::bulk_load(sbase + kSmFA, a.consts + (size_t)HB_IDX(it.hd, a.H) * kConstStride, kOpBytes, bar(kBarConst));
                     if (!tc::mbar_wait(bar(kBarConst), cphase & 1, never)) { ok = false; break; }
                     ++cphase;
                     cur_hd = it.hd;
@@ -904,7 +908,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             if (id < 0) break;
             const Item it = decode_item<NC>(a, id);
             if (it.hd != cur_hd) {
-                const float2 *lp = reinterpret_cast<const float2 *>(a.consts + (size_t)it.hd * kConstStride + kLamOff);
+                const float2 *lp = reinterpret_cast<const float2 *>(a.consts + (size_t)HB_IDX(it.hd, a.H) * kConstStride + kLamOff);
                 lamC = lp[n];               // zero for modes >= d
                 lamS = lp[kMaxModes + n];
                 cur_hd = it.hd;
@@ -937,8 +941,10 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 chain(w);
                 return true;
             };
-            // this thread's row of a published [32 rows][NC ch] state (bypassing L1)
-            auto load_rows = [&](const float *src, float *o) {
+            // this thread's row of a published [32 rows][NC ch] state (bypassing L1); `item` is the
+            // publishing item (checked against the item count in the bounds-checked build)
+            auto load_rows = [&](const float *base, long long item, float *o) {
+                const float *src = base + (size_t)HB_IDX(item, (long long)a.H * a.ih) * kKS * kNC;
                 const float4 *p4 = reinterpret_cast<const float4 *>(src + (size_t)r * kNC + kCh * q4);
 #pragma unroll
                 for (int i = 0; i < kCh / 4; ++i) {
@@ -948,7 +954,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             };
             // write the state rows of this thread to dst [32 rows][NC ch] and hand `code` to the
             // publisher lane, which posts it once every row is written (no wait here)
-            auto publish = [&](const float *v, float *dst, int code) -> bool {
+            auto publish = [&](const float *v, float *base, int code) -> bool {
+                float *dst = base + (size_t)HB_IDX(it.id, (long long)a.H * a.ih) * kKS * kNC;
                 float4 *o = reinterpret_cast<float4 *>(dst + (size_t)r * kNC + kCh * q4);
 #pragma unroll
                 for (int i = 0; i < kCh / 4; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
@@ -958,8 +965,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             // state-only pass over the segment, then publish its contribution
             for (int i = 0; i < it.n1 && ok; ++i, ++g) ok = uni(advance(g));
             if (!ok) break;
-            const size_t item_off = (size_t)it.id * kKS * kNC;
-            if (it.n1 > 0 && !(ok = uni(publish(st, (it.seg == 0 ? a.inc : a.agg) + item_off, it.seg == 0 ? 2 : 1))))
+            if (it.n1 > 0 && !(ok = uni(publish(st, it.seg == 0 ? a.inc : a.agg, it.seg == 0 ? 2 : 1))))
                 break;
             float sloc[kCh];
 #pragma unroll
@@ -975,7 +981,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int units = a.units_h;
                 for (int p = it.id - units; p >= it.id - it.seg * units; p -= units) {
                     int code = 0;
-                    if (lane == 0) {
+                    if (lane == 0 && HB_OK(p, (long long)a.H * a.ih)) {
                         code = ld_acquire(a.status + p);
                         const unsigned long long t0 = tc::global_ns();
                         while (code == 0 && !*abort && tc::global_ns() - t0 < a.lookback_ns) {
@@ -993,10 +999,10 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 }
                 if (!(ok = uni(ok))) break;
                 __syncwarp();       // lane 0's acquire loads order the other lanes' reads below
-                load_rows(a.inc + (size_t)p0 * kKS * kNC, st);
+                load_rows(a.inc, p0, st);
                 for (int p = p0 + units; p < it.id; p += units) {
                     float ag[kCh];
-                    load_rows(a.agg + (size_t)p * kKS * kNC, ag);
+                    load_rows(a.agg, p, ag);
 #pragma unroll
                     for (int i = 0; i < kCh; ++i) st[i] = seg_step(st[i], ag[i], lamS, sgn);
                 }
@@ -1004,7 +1010,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     // inclusive state at the end of this segment (sloc is not needed after this)
 #pragma unroll
                     for (int i = 0; i < kCh; ++i) sloc[i] = seg_step(st[i], sloc[i], lamS, sgn);
-                    if (!(ok = uni(publish(sloc, a.inc + item_off, 2)))) break;
+                    if (!(ok = uni(publish(sloc, a.inc, 2)))) break;
                 }
             }
 
@@ -1040,19 +1046,23 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     // transpose the warp's 32 x 32 block (rows r in lanes -> channels in lanes) so
                     // that each lane writes the (Re, Im) pairs of one channel: coalesced float2 stores
                     warp_transpose32(st, lane);
-                    float2 *so = reinterpret_cast<float2 *>(a.state_out) + ((size_t)it.b * d) * a.Dch + it.c0 + kCh * q4 + lane;
+                    const size_t s0 = ((size_t)it.b * d) * a.Dch + it.c0 + kCh * q4 + lane;
+                    float2 *so = reinterpret_cast<float2 *>(a.state_out) + s0;
 #pragma unroll
                     for (int m = 0; m < kMaxModes; ++m)
-                        if (m < d) so[(size_t)m * a.Dch] = make_float2(st[m], st[kIm + m]);
+                        if (m < d && HB_OK(s0 + (size_t)m * a.Dch, (long long)(a.units_h / a.tph) * d * a.Dch))
+                            so[(size_t)m * a.Dch] = make_float2(st[m], st[kIm + m]);
                 } else {
                     // 16 channels: transpose each half-warp's 16 x 16 block; lane 16 h + i then holds
                     // part h (Re, Im) of every mode for channel i, and a warp store covers 16
                     // channels x (Re, Im) = 128 contiguous bytes
                     warp_transpose16x2(st, lane);
-                    float *so = a.state_out + (((size_t)it.b * d) * a.Dch + it.c0 + kCh * q4 + (lane & 15)) * 2 + (lane >> 4);
+                    const size_t s0 = (((size_t)it.b * d) * a.Dch + it.c0 + kCh * q4 + (lane & 15)) * 2 + (lane >> 4);
+                    float *so = a.state_out + s0;
 #pragma unroll
                     for (int m = 0; m < kMaxModes; ++m)
-                        if (m < d) so[(size_t)m * a.Dch * 2] = st[m];
+                        if (m < d && HB_OK(s0 + (size_t)m * a.Dch * 2, (long long)(a.units_h / a.tph) * d * a.Dch * 2))
+                            so[(size_t)m * a.Dch * 2] = st[m];
                 }
             }
         }
@@ -1119,7 +1129,8 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         yv.w = pack_bf16(bf_lo(qv.w) * zz[6], bf_hi(qv.w) * zz[7]);
                         if (!store_direct)
                             *qp[i] = yv;
-                        else if (row_valid)
+                        else if (row_valid && HB_OK(((long long)it.b * a.L + tok + tau) * a.Dch + it.c0 + cbase + 8 * i + 7,
+                                                    (long long)(a.units_h / a.tph) * a.L * a.Dch))
                             *reinterpret_cast<uint4 *>(yrow + cbase + 8 * i) = yv;
                     }
                 }
@@ -1234,6 +1245,8 @@ std::atomic<int> g_inject_item{-1};
 std::atomic<unsigned long long> g_inject_wait_ns{0};
 
 }  // namespace
+
+HYENA_BOUNDS_READER(prefill_chunked)
 
 bool chunked_supported(int dtype, int Dch, int H, int d) {
     return dtype == HYENA_BF16 && H > 0 && Dch % H == 0 && (Dch / H) % 64 == 0 && d >= 1 && d <= kMaxModes;

@@ -49,16 +49,18 @@ __global__ void __launch_bounds__(kFusedThreads)
 spectrum_fused_kernel(const float *__restrict__ h, int L, int N, float scale,
                       float2 *__restrict__ spec_perm) {
     extern __shared__ float2 buf[];
-    const int hd = blockIdx.x;
+    const int hd = blockIdx.x, H = gridDim.x;
+    (void)H;
     const float *hh = h + (size_t)hd * L;
     const bool half_zero = (L <= N / 2);
     const int fill = half_zero ? N / 2 : N;
     for (int t = threadIdx.x; t < fill; t += blockDim.x)
-        buf[pad(t)] = make_float2(t < L ? hh[t] : 0.f, 0.f);
+        buf[pad(t)] = make_float2(t < L ? hh[HB_IDX(t, (long long)(H - hd) * L)] : 0.f, 0.f);
     __syncthreads();
     fft::forward(buf, N, half_zero);
     float2 *out = spec_perm + (size_t)hd * N;
-    for (int p = threadIdx.x; p < N; p += blockDim.x) out[p] = cscale(buf[pad(p)], scale);
+    for (int p = threadIdx.x; p < N; p += blockDim.x)
+        if (HB_OK((long long)hd * N + p, (long long)H * N)) out[p] = cscale(buf[pad(p)], scale);
 }
 
 // natural-order bins 0..N/2 from the digit-reversed layout
@@ -74,7 +76,8 @@ __global__ void spectrum_natural_kernel(const float2 *__restrict__ spec_perm, in
         const int N1 = N / N2;
         f = (p / N2) + N1 * fft::freq_of_pos(p % N2, N2);
     }
-    if (f <= N / 2) out[(size_t)hd * (N / 2 + 1) + f] = spec_perm[(size_t)hd * N + p];
+    if (f <= N / 2 && HB_OK((long long)hd * (N / 2 + 1) + f, (long long)gridDim.y * (N / 2 + 1)))
+        out[(size_t)hd * (N / 2 + 1) + f] = spec_perm[HB_IDX((size_t)hd * N + p, (long long)gridDim.y * N)];
 }
 
 // ------------------------------------------------------------------ fused prefill
@@ -96,6 +99,10 @@ prefill_fused_kernel(const typename Act::T *__restrict__ q, const typename Act::
     const int hd = c0 / ch;
     const typename Act::T *kb = k + (size_t)b * L * Dch + c0;
     const typename Act::T *vb = v + (size_t)b * L * Dch + c0;
+    // extents (bounds-checked build): activations from kb, state, spectra, poles
+    const long long n_act = (long long)gridDim.y * L * Dch - ((long long)b * L * Dch + c0);
+    const long long H = Dch / ch;
+    (void)n_act; (void)H;
 
     // 1. gate-in: x_t = (k_a v_a, k_b v_b), zero padding up to N/2; four rows per
     //    thread are loaded before any is used so that their latencies overlap
@@ -106,7 +113,7 @@ prefill_fused_kernel(const typename Act::T *__restrict__ q, const typename Act::
         for (int r = 0; r < U; ++r) {
             const int t = t0 + r * nthr;
             kk[r] = vv[r] = make_float2(0.f, 0.f);
-            if (t < L) {
+            if (t < L && HB_OK((long long)t * Dch + paired, n_act)) {
                 const size_t o = (size_t)t * Dch;
                 if (paired) { kk[r] = Act::ld2(kb + o); vv[r] = Act::ld2(vb + o); }
                 else { kk[r].x = Act::ld(kb + o); vv[r].x = Act::ld(vb + o); }
@@ -123,7 +130,7 @@ prefill_fused_kernel(const typename Act::T *__restrict__ q, const typename Act::
     // 2. prompt -> state: s_n = sum_j lambda_n^(L-1-j) x_j over the last W tokens
     //    (older ones weigh < 2^-40 max|u|), by segments: Horner inside a segment,
     //    then scaled by lambda^(L - segment end) (fp64 power), segments summed in order.
-    const float2 *lh = lam + (size_t)hd * d;
+    const float2 *lh = lam + (size_t)HB_IDX(hd, H) * d;
     const int jstart = L - state_window(lh, d, L);
     const int nseg = max(1, nthr / d);
     const int seglen = (L - jstart + nseg - 1) / nseg;
@@ -154,14 +161,16 @@ prefill_fused_kernel(const typename Act::T *__restrict__ q, const typename Act::
             s.x += p.x; s.y += p.y; s.z += p.z; s.w += p.w;
         }
         float *so = state_out + (((size_t)b * d + n) * Dch + c0) * 2;
-        *reinterpret_cast<float2 *>(so) = make_float2(s.x, s.y);   // state is 8-byte aligned
-        if (paired) *reinterpret_cast<float2 *>(so + 2) = make_float2(s.z, s.w);
+        const long long si = (((long long)b * d + n) * Dch + c0) * 2, n_state = (long long)gridDim.y * d * Dch * 2;
+        (void)si; (void)n_state;
+        if (HB_OK(si + 1, n_state)) *reinterpret_cast<float2 *>(so) = make_float2(s.x, s.y);   // state is 8-byte aligned
+        if (paired && HB_OK(si + 3, n_state)) *reinterpret_cast<float2 *>(so + 2) = make_float2(s.z, s.w);
     }
 
     // 3. forward transform, product with the head's spectrum (scaled by 1/N), inverse
     fft::forward(buf, N, true);
     const float2 *hs = spec_perm + (size_t)hd * N;
-    for (int p = tid; p < N; p += nthr) buf[pad(p)] = cmul(buf[pad(p)], __ldg(&hs[p]));
+    for (int p = tid; p < N; p += nthr) buf[pad(p)] = cmul(buf[pad(p)], __ldg(&hs[HB_IDX(p, (H - hd) * N)]));
     __syncthreads();
     fft::inverse(buf, N, L);
 
@@ -174,7 +183,7 @@ prefill_fused_kernel(const typename Act::T *__restrict__ q, const typename Act::
         for (int r = 0; r < U; ++r) {
             const int t = t0 + r * nthr;
             qq[r] = make_float2(0.f, 0.f);
-            if (t < L) {
+            if (t < L && HB_OK((long long)t * Dch + paired, n_act)) {
                 if (paired) qq[r] = Act::ld2(qb + (size_t)t * Dch);
                 else qq[r].x = Act::ld(qb + (size_t)t * Dch);
             }
@@ -182,7 +191,7 @@ prefill_fused_kernel(const typename Act::T *__restrict__ q, const typename Act::
 #pragma unroll
         for (int r = 0; r < U; ++r) {
             const int t = t0 + r * nthr;
-            if (t < L) {
+            if (t < L && HB_OK((long long)t * Dch + paired, n_act)) {
                 const float2 z = buf[pad(t)];
                 if (paired) Act::st2(yb + (size_t)t * Dch, qq[r].x * z.x, qq[r].y * z.y);
                 else Act::st(yb + (size_t)t * Dch, qq[r].x * z.x);
@@ -234,7 +243,8 @@ fourstep_fwd1_kernel(Src src, int N2, float2 *__restrict__ Y) {
 #pragma unroll
     for (int k1 = 0; k1 < N1; ++k1) {
         const float2 w = fft::expi_neg(n2 * k1, (int)N);
-        out[(size_t)k1 * N2] = k1 ? cmul(x[k1], w) : x[k1];
+        if (HB_OK((long long)col * N + (long long)k1 * N2 + n2, (long long)gridDim.y * N))
+            out[(size_t)k1 * N2] = k1 ? cmul(x[k1], w) : x[k1];
     }
 }
 
@@ -248,11 +258,14 @@ fourstep_inner_kernel(float2 *__restrict__ Y, int N1, int N2, int mode, float sc
     const int col = blockIdx.y, k1 = blockIdx.x;
     const long long N = (long long)N1 * N2;
     float2 *row = Y + (size_t)col * N + (size_t)k1 * N2;
-    for (int t = threadIdx.x; t < N2; t += blockDim.x) buf[pad(t)] = row[t];
+    const long long n_row = (long long)gridDim.y * N - ((long long)col * N + (long long)k1 * N2);
+    (void)n_row;
+    for (int t = threadIdx.x; t < N2; t += blockDim.x) buf[pad(t)] = row[HB_IDX(t, n_row)];
     __syncthreads();
     fft::forward(buf, N2, false);
     if (mode == 0) {
-        for (int p = threadIdx.x; p < N2; p += blockDim.x) row[p] = cscale(buf[pad(p)], scale);
+        for (int p = threadIdx.x; p < N2; p += blockDim.x)
+            if (HB_OK(p, n_row)) row[p] = cscale(buf[pad(p)], scale);
         return;
     }
     const int slot = col % nslots;
@@ -261,7 +274,8 @@ fourstep_inner_kernel(float2 *__restrict__ Y, int N1, int N2, int mode, float sc
     for (int p = threadIdx.x; p < N2; p += blockDim.x) buf[pad(p)] = cmul(buf[pad(p)], __ldg(&hs[p]));
     __syncthreads();
     fft::inverse(buf, N2, -1);
-    for (int t = threadIdx.x; t < N2; t += blockDim.x) row[t] = buf[pad(t)];
+    for (int t = threadIdx.x; t < N2; t += blockDim.x)
+        if (HB_OK(t, n_row)) row[t] = buf[pad(t)];
 }
 
 // step 3: inverse across the long stride, gate-out, store the first L outputs
@@ -274,11 +288,13 @@ fourstep_inv1_kernel(const float2 *__restrict__ Y, int N2, int L, int Dch, int n
     if (n2 >= N2) return;
     const long long N = (long long)N1 * N2;
     const float2 *in = Y + (size_t)col * N + n2;
+    const long long n_in = (long long)gridDim.y * N - ((long long)col * N + n2);
+    (void)n_in;
     float2 x[N1];
 #pragma unroll
     for (int k1 = 0; k1 < N1; ++k1) {
         const float2 w = fft::expi_neg(n2 * k1, (int)N);
-        x[k1] = k1 ? cmulc(in[(size_t)k1 * N2], w) : in[0];
+        x[k1] = k1 ? cmulc(in[HB_IDX((long long)k1 * N2, n_in)], w) : in[0];
     }
     fft::dftR<N1, true>(x);
     const int b = col / nslots, slot = col % nslots;
@@ -286,7 +302,7 @@ fourstep_inv1_kernel(const float2 *__restrict__ Y, int N2, int L, int Dch, int n
 #pragma unroll
     for (int n1 = 0; n1 < N1; ++n1) {
         const long long t = (long long)N2 * n1 + n2;
-        if (t < L) {
+        if (t < L && HB_OK(((long long)b * L + t) * Dch + c0 + paired, (long long)(gridDim.y / nslots) * L * Dch)) {
             const size_t o = ((size_t)b * L + t) * Dch + c0;
             if (paired) {
                 const float2 qq = Act::ld2(q + o);
@@ -379,6 +395,8 @@ cudaError_t prefill_fourstep(const void *q, const void *k, const void *v, int B,
 }
 
 }  // namespace
+
+HYENA_BOUNDS_READER(prefill_fft)
 
 size_t spectrum_ws_bytes(int H, int N) { return (size_t)H * N * sizeof(float2); }
 

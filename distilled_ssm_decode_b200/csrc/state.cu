@@ -41,7 +41,9 @@ state_partial_kernel(const typename Act::T *__restrict__ k, const typename Act::
     const int c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= Dch) return;
     const int g = blockIdx.y, b = blockIdx.z, nseg = gridDim.y;
-    const int hd = c / ch;
+    const int hd = c / ch, H = Dch / ch;
+    const long long n_act = (long long)gridDim.z * L * Dch, n_part = (long long)gridDim.z * nseg * d * Dch;
+    (void)H; (void)n_act; (void)n_part;
     // the nseg segments cover this head's window [L - W, L)
     const int W = state_window(lam + (size_t)hd * d, d, L);
     const int jstart = L - W;
@@ -51,11 +53,11 @@ state_partial_kernel(const typename Act::T *__restrict__ k, const typename Act::
         float2 l[kModeChunk], a[kModeChunk];
 #pragma unroll
         for (int i = 0; i < kModeChunk; ++i) {
-            l[i] = (n0 + i < d) ? __ldg(&lam[(size_t)hd * d + n0 + i]) : make_float2(0.f, 0.f);
+            l[i] = (n0 + i < d) ? __ldg(&lam[HB_IDX((size_t)hd * d + n0 + i, (long long)H * d)]) : make_float2(0.f, 0.f);
             a[i] = make_float2(0.f, 0.f);
         }
         for (int j = j0; j < j1; ++j) {
-            const size_t o = ((size_t)b * L + j) * Dch + c;
+            const size_t o = HB_IDX(((size_t)b * L + j) * Dch + c, n_act);
             const float u = Act::ld(k + o) * Act::ld(v + o);
 #pragma unroll
             for (int i = 0; i < kModeChunk; ++i)
@@ -71,7 +73,8 @@ state_partial_kernel(const typename Act::T *__restrict__ k, const typename Act::
                 const cd pw = cdpow(cd{l[i].x, l[i].y}, (long long)(L - j1));
                 r = cmul(a[i], make_float2((float)pw.x, (float)pw.y));
             }
-            part[(((size_t)b * nseg + g) * d + n) * Dch + c] = r;
+            const size_t pi = (((size_t)b * nseg + g) * d + n) * Dch + c;
+            if (HB_OK(pi, n_part)) part[pi] = r;
         }
     }
 }
@@ -81,12 +84,16 @@ __global__ void state_sum_kernel(const float2 *__restrict__ part, int nseg, int 
     const int c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= Dch) return;
     const int n = blockIdx.y, b = blockIdx.z;
+    const long long n_part = (long long)gridDim.z * nseg * d * Dch, n_state = (long long)gridDim.z * d * Dch;
+    (void)n_part; (void)n_state;
     float2 s = make_float2(0.f, 0.f);
-    for (int g = 0; g < nseg; ++g) s = cadd(s, part[(((size_t)b * nseg + g) * d + n) * Dch + c]);
-    state[((size_t)b * d + n) * Dch + c] = s;
+    for (int g = 0; g < nseg; ++g) s = cadd(s, part[HB_IDX((((size_t)b * nseg + g) * d + n) * Dch + c, n_part)]);
+    if (HB_OK(((size_t)b * d + n) * Dch + c, n_state)) state[((size_t)b * d + n) * Dch + c] = s;
 }
 
 }  // namespace
+
+HYENA_BOUNDS_READER(state)
 
 size_t state_ws_bytes(int B, int L, int Dch, int d) {
     if (L <= 0) return 0;

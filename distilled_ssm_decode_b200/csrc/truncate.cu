@@ -37,9 +37,10 @@ truncate_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R, in
     __shared__ double score[HYENA_MAX_MODES], row[HYENA_MAX_MODES];
     __shared__ int keep[HYENA_MAX_MODES];
     __shared__ cd c[HYENA_MAX_MODES], mu[HYENA_MAX_MODES];
-    const int hd = blockIdx.x, n = threadIdx.x;
+    const int hd = blockIdx.x, n = threadIdx.x, H = gridDim.x;
+    (void)H;
     if (n < d) {
-        const float2 l = lam[(size_t)hd * d + n], r = R[(size_t)hd * d + n];
+        const float2 l = lam[HB_IDX((size_t)hd * d + n, (long long)H * d)], r = R[HB_IDX((size_t)hd * d + n, (long long)H * d)];
         mu[n] = cd{l.x, l.y};
         c[n] = cd{r.x, r.y};
         const double a = sqrt((double)l.x * l.x + (double)l.y * l.y);
@@ -58,9 +59,11 @@ truncate_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R, in
             int pos = 0;
             for (int m = 0; m < n; ++m) pos += keep[m];
             const size_t o = (size_t)hd * k + pos;
-            kept[o] = n;
-            lam_out[o] = lam[(size_t)hd * d + n];
-            R_out[o] = R[(size_t)hd * d + n];
+            if (HB_OK(o, (long long)H * k)) {
+                kept[o] = n;
+                lam_out[o] = lam[HB_IDX((size_t)hd * d + n, (long long)H * d)];
+                R_out[o] = R[HB_IDX((size_t)hd * d + n, (long long)H * d)];
+            }
             row[n] = 0.0;
         } else {
             // row n of the pair sums over the dropped modes m
@@ -86,12 +89,16 @@ truncate_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R, in
             inf |= isinf(score[m]);
             e += row[m];
         }
-        bound[hd] = b;
-        err_l2[hd] = inf ? INFINITY : sqrt(fmax(e, 0.0));
+        if (HB_OK(hd, H)) {
+            bound[hd] = b;
+            err_l2[hd] = inf ? INFINITY : sqrt(fmax(e, 0.0));
+        }
     }
 }
 
 }  // namespace
+
+HYENA_BOUNDS_READER(truncate)
 
 cudaError_t launch_modal_truncate(const float2 *lam, const float2 *R, int H, int d, int k, int *kept,
                                   float2 *lam_out, float2 *R_out, double *bound, double *err_l2, cudaStream_t s) {

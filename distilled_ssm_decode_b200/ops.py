@@ -7,6 +7,7 @@ missing or cannot be loaded, every call raises.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -42,6 +43,7 @@ SIGNATURES = {
     "hyena_prefill_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp, _fp,
                                    _vp]),
     "hyena_test_chunked_inject": (_i, [_i, ctypes.c_double]),
+    "hyena_debug_bounds_check": (_i, [_vp]),
     "hyena_prompt_state_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "hyena_prompt_state": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _fp, _fp, _vp, _sz, _vp]),
     "hyena_decode_step": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _fp, _fp, _fp, _fp, _vp, _vp]),
@@ -59,22 +61,50 @@ class HyenaError(RuntimeError):
         self.status = status
 
 
+def _load(path: str):
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{os.path.basename(path)} not found at {path}; build it with "
+            "`python -m distilled_ssm_decode_b200.build` (there is no CPU fallback)")
+    L = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L
+
+
 def lib():
     """The loaded ctypes library (raises if the CUDA library is missing)."""
     global _lib
     with _lock:
         if _lib is None:
-            if not os.path.exists(LIB_PATH):
-                raise RuntimeError(
-                    f"libhyena_b200.so not found at {LIB_PATH}; build it with "
-                    "`python -m distilled_ssm_decode_b200.build` (there is no CPU fallback)")
-            L = ctypes.CDLL(LIB_PATH)
-            for name, (res, args) in SIGNATURES.items():
-                f = getattr(L, name)
-                f.restype = res
-                f.argtypes = args
-            _lib = L
+            _lib = _load(LIB_PATH)
     return _lib
+
+
+@contextlib.contextmanager
+def using_library(path: str):
+    """Route every call of this module through another build of the library (for instance the
+    bounds-checked libhyena_b200_dbg.so) inside the `with` block."""
+    global _lib
+    other = _load(path)
+    with _lock:
+        prev = _lib
+        _lib = other
+    try:
+        yield other
+    finally:
+        with _lock:
+            _lib = prev
+
+
+def bounds_check():
+    """Bounds-checked build only: (status, record) of the first global access out of range since
+    the last check; status 0 = none, 1 = record = (file id, source line, index, extent)."""
+    rec = (ctypes.c_longlong * 4)()
+    st = lib().hyena_debug_bounds_check(ctypes.cast(rec, ctypes.c_void_p))
+    return st, tuple(rec)
 
 
 def status_string(status: int) -> str:

@@ -208,6 +208,20 @@ int hyena_prefill_chunked(const void *q, const void *k, const void *v, int dtype
                           void *workspace, size_t ws_bytes, hyena_stream_t stream);
 
 /*
+ * Bounds-checked build (no counterpart in the pages): libhyena_b200_dbg.so is
+ * the same library compiled with every kernel checking the index of each
+ * global load and store against the extent its arguments give that buffer.
+ * The first index out of range in each source file is recorded and the access
+ * is skipped (no trap, no fault).  This call waits for the device, then reads
+ * and clears the records.  Returns 0 when no access was out of range, 1 when
+ * one was, with record = {file, source line, index, extent} (file: 1 decode.cu,
+ * 2 filter.cu, 3 fir.cu, 4 prefill_chunked.cu, 5 prefill_fft.cu, 6 state.cu,
+ * 7 truncate.cu); HYENA_ERR_UNSUPPORTED from the release build, which has no
+ * checks; HYENA_ERR_ARG for a NULL record.
+ */
+int hyena_debug_bounds_check(long long *record);
+
+/*
  * Test hook (no counterpart in the pages): fault injection for the bounded
  * waits of hyena_prefill_chunked, so that a test can make a wait run out
  * without any GPU fault.  Every later hyena_prefill_chunked launch in the

@@ -184,3 +184,28 @@ def test_modal_truncate_validation(lib):
     assert call(kept=FAKE + 2) == ERR_ALIGN
     assert call(H=0) == OK
     assert lib.hyena_modal_truncate(_p(), _p(), 2, 4, 2, None, _p(), _p(), _p(), _p(), None) == ERR_ARG
+
+
+def test_bounds_checked_build_exports_every_declared_symbol():
+    """The bounds-checked variant (libhyena_b200_dbg.so, -DHYENA_DEBUG_BOUNDS) has the same ABI."""
+    from distilled_ssm_decode_b200 import build
+    path = build.build(debug_bounds=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (hyena_\w+)", out))
+    assert not [n for n in declared_functions() if n not in exported]
+
+
+def test_release_build_reports_no_bounds_checks(lib):
+    """hyena_debug_bounds_check answers from the host in the release build (no CUDA call)."""
+    rec = (ctypes.c_longlong * 4)(7, 7, 7, 7)
+    assert lib.hyena_debug_bounds_check(ctypes.cast(rec, ctypes.c_void_p)) == ERR_UNSUP
+    assert tuple(rec) == (0, 0, 0, 0)
+    assert lib.hyena_debug_bounds_check(None) == ERR_ARG
+
+
+def test_fault_injection_hook_validates_its_arguments(lib):
+    assert lib.hyena_test_chunked_inject(-2, 0.0) == ERR_ARG
+    assert lib.hyena_test_chunked_inject(0, -1.0) == ERR_ARG
+    assert lib.hyena_test_chunked_inject(0, 61.0) == ERR_ARG
+    assert lib.hyena_test_chunked_inject(-1, 0.0) == OK
