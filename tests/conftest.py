@@ -18,3 +18,17 @@ def oracle():
     import oracle as _oracle
     _oracle.build()
     return _oracle
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Print the parity errors that tests recorded (record_property), one line per test."""
+    rows = []
+    for rep in terminalreporter.stats.get("passed", []) + terminalreporter.stats.get("failed", []):
+        props = [(k, v) for k, v in getattr(rep, "user_properties", []) if k.endswith("_err")]
+        if props and rep.when == "call":
+            rows.append((rep.nodeid, props))
+    if rows:
+        terminalreporter.write_sep("-", "recorded parity errors (max|err| / max|oracle|)")
+        for nodeid, props in rows:
+            terminalreporter.write_line(nodeid.split("::", 1)[-1] + "  " +
+                                        "  ".join(f"{k}={v:.2e}" for k, v in props))

@@ -23,6 +23,22 @@ from parity_util import TOL, column_params, dev_params, gather_columns, rel_err,
 
 pytestmark = pytest.mark.gpu
 
+# The chunked route rounds its tensor-core operands to bf16 (u = k v, the taps, the powers and the
+# carried state; relative 2^-9 each) and accumulates in fp32.  Measured on B200 over every case
+# below and the full-size workloads: max|y - oracle| / max|oracle| from 2.8e-3 to 6.5e-3 (the FFT
+# route on the same inputs: 1.3e-3 to 3.3e-3, its bf16 output rounding), and the prompt state from
+# 1.6e-3 to 3.9e-3 (FFT route ~1e-7).  Besides the bf16 bar (2e-2) every case must stay within
+# these measured margins, so a change that loses accuracy shows even while the bar still holds.
+Y_MARGIN = 1e-2
+S_MARGIN = 6e-3
+
+
+def _check_errors(record_property, ey, es):
+    record_property("chunked_y_err", float(ey))
+    record_property("chunked_state_err", float(es))
+    assert ey <= TOL["bf16"] and es <= TOL["bf16"], (ey, es)
+    assert ey <= Y_MARGIN and es <= S_MARGIN, (ey, es)
+
 
 @pytest.fixture(scope="module", autouse=True)
 def _cuda():
@@ -64,7 +80,7 @@ CASES = [
 
 
 @pytest.mark.parametrize("B,L,Dch,H,d", CASES)
-def test_chunked_small_cases_full_compare(oracle, B, L, Dch, H, d):
+def test_chunked_small_cases_full_compare(oracle, record_property, B, L, Dch, H, d):
     w = W.Workload(300 + L + d, "case", B=B, L=L, Dch=Dch, H=H, d=d, dtype="bf16", fft_len=0, T=0)
     p = W.params(w)
     q, k, v = W.prefill_inputs(w)
@@ -77,11 +93,11 @@ def test_chunked_small_cases_full_compare(oracle, B, L, Dch, H, d):
     else:
         y_ref, s_ref = oracle.recurrent(qf, kf, vf, p.lam, p.R, p.Dskip, H=H)
     ey, es = rel_err(y.double().numpy(), y_ref), rel_err(s, s_ref)
-    assert ey <= TOL["bf16"] and es <= TOL["bf16"], (ey, es)
+    _check_errors(record_property, ey, es)
 
 
 @pytest.mark.parametrize("name,ncols", [("mid_bf16", 24), ("gen1p3b_bf16", 32)])
-def test_chunked_full_size_sampled(oracle, name, ncols):
+def test_chunked_full_size_sampled(oracle, record_property, name, ncols):
     w = W.WORKLOADS[name]
     p = W.params(w)
     q, k, v = W.prefill_inputs(w)
@@ -95,7 +111,7 @@ def test_chunked_full_size_sampled(oracle, name, ncols):
     s_ref = oracle.prompt_state(kc, vc, lam_c, H=len(bc))
     ey = rel_err(gather_columns(y, bc), y_ref)
     es = rel_err(np.stack([s[b, :, c] for b, c in bc], -1)[None], s_ref)
-    assert ey <= TOL["bf16"] and es <= TOL["bf16"], (ey, es)
+    _check_errors(record_property, ey, es)
 
 
 def test_chunked_matches_fft_route():
@@ -106,10 +122,10 @@ def test_chunked_matches_fft_route():
     lam, R, D = dev_params(p.__class__(p.lam[:2], p.R[:2], p.Dskip[:2]))
     y1, s1, _ = ops.prefill_chunked(q, k, v, lam, R, D)
     y2, s2 = ops.prefill(q, k, v, lam, R, D, 4096)
-    assert rel_err(y1.cpu().double().numpy(), y2.cpu().double().numpy()) <= TOL["bf16"]
-    # the chunked route's tensor-core operands are bf16 (relative rounding 2^-9), so the two routes'
-    # states agree to about 1e-3 of their maximum; the bar is the bf16 tolerance
-    assert rel_err(state_c128(s1), state_c128(s2)) <= TOL["bf16"]
+    # the FFT route's state is fp32 throughout (~1e-7 of the oracle), so this measures the chunked
+    # route's own state error (bf16 operands): within the bf16 bar and the measured margin
+    assert rel_err(y1.cpu().double().numpy(), y2.cpu().double().numpy()) <= Y_MARGIN
+    assert rel_err(state_c128(s1), state_c128(s2)) <= S_MARGIN
 
 
 def test_chunked_is_deterministic():
@@ -135,7 +151,7 @@ def test_chunked_unsupported_shapes_are_rejected():
     assert e.value.status == -5
 
 
-def test_chunked_long_prefill_full_size_sampled(oracle):
+def test_chunked_long_prefill_full_size_sampled(oracle, record_property):
     """The long-prefill workload as the bench runs it (B=1, L=65536, Dch=768, 12 heads of 64
     channels, |lambda| up to 0.999, sequences split into segments joined by the look-back):
     24 sampled channels against the oracle's recurrence over the whole prompt."""
@@ -150,7 +166,7 @@ def test_chunked_long_prefill_full_size_sampled(oracle):
     y_ref, s_ref = oracle.recurrent(qc, kc, vc, lam_c, R_c, D_c, H=len(bc))
     ey = rel_err(gather_columns(y, bc), y_ref)
     es = rel_err(np.stack([s[b, :, c] for b, c in bc], -1)[None], s_ref)
-    assert ey <= TOL["bf16"] and es <= TOL["bf16"], (ey, es)
+    _check_errors(record_property, ey, es)
 
 
 def test_chunked_is_deterministic_with_many_items():
@@ -201,7 +217,7 @@ def test_chunked_empty_inputs():
     torch.cuda.synchronize()
 
 
-def test_chunked_degenerate_poles(oracle):
+def test_chunked_degenerate_poles(oracle, record_property):
     """Poles at 0 (lambda^0 = 1 only: a two-tap filter, no carry beyond one token) and poles at
     |lambda| = 0.9999 (almost no decay over the 3000-token prompt, sequence split into segments)
     mixed in one head; every element against the oracle's recurrence."""
@@ -217,7 +233,7 @@ def test_chunked_degenerate_poles(oracle):
     y, s = _run(q, k, v, p)
     y_ref, s_ref = oracle.recurrent(W.to_f64(q), W.to_f64(k), W.to_f64(v), p.lam, p.R, p.Dskip, H=1)
     ey, es = rel_err(y.double().numpy(), y_ref), rel_err(s, s_ref)
-    assert ey <= TOL["bf16"] and es <= TOL["bf16"], (ey, es)
+    _check_errors(record_property, ey, es)
 
 
 def test_mid_workload_flow_chunked_then_decode(oracle):
