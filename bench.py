@@ -661,28 +661,21 @@ def measure_layers(args, w, nl: int, dev, steps: int, warmup: int, e2e_steps: in
     ys = [torch.empty_like(x[0]) for x in qkv]
     ws = torch.empty(ops.prefill_chunked_workspace_bytes(w.B, w.L, w.Dch, w.H, w.d), dtype=torch.uint8,
                      device=dev)
+    # every layer's prefill in one launch (the layers' work items share the persistent grid)
+    pset = ops.PrefillLayerSet([x[0] for x in qkv], [x[1] for x in qkv], [x[2] for x in qkv], ys, states,
+                               lams, Rs, Ds)
+    ws_all = torch.empty(pset.workspace_bytes(), dtype=torch.uint8, device=dev)
     pool = 8
     dpool = [W.decode_pool_device(w, pool, device=dev, layer=l) for l in range(nl)]
     ydec = torch.empty((w.T, nl, w.B, w.Dch), dtype=w.torch_dtype, device=dev)
     ls = ops.LayerSet(lams, Rs, Ds, states)
     stream = torch.cuda.Stream(dev)
 
-    # the layers are independent: alternate them over two streams (a workspace each), so that one
-    # layer's start and end overlap its neighbour's instead of idling SMs
-    pstreams = [torch.cuda.Stream(dev) for _ in range(2)]
+    # workspaces of the end-to-end leg's per-layer calls
     pws = [ws, torch.empty_like(ws)]
 
     def prefill_all():
-        cur = torch.cuda.current_stream(dev)
-        for s in pstreams:
-            s.wait_stream(cur)
-        for l in range(nl):
-            q, k, v = qkv[l]
-            with torch.cuda.stream(pstreams[l % 2]):
-                ops.prefill_chunked(q, k, v, lams[l], Rs[l], Ds[l], y=ys[l], state=states[l],
-                                    workspace=pws[l % 2])
-        for s in pstreams:
-            cur.wait_stream(s)
+        ops.prefill_chunked_layers(pset, workspace=ws_all)
 
     def decode_all():
         for t in range(w.T):
@@ -715,20 +708,16 @@ def measure_layers(args, w, nl: int, dev, steps: int, warmup: int, e2e_steps: in
     elapsed_ms, (pre_ms, dec_ms) = timed_steps(stream, dev, steps, warmup, step, 2)
     clk = clocks.stop() if clocks is not None else None
     ms_per_step = elapsed_ms / steps
-    for wsx in pws:
-        err = ops.chunked_error(wsx, w.B, w.L, w.Dch, w.H, w.d)
-        if err:
-            raise SystemExit(f"chunked prefill kernel reported error {err}")
+    err = pset.error(ws_all)
+    if err:
+        raise SystemExit(f"chunked prefill kernel reported error {err}")
 
     peak, peak_src = load_peaks()
     key = f"{w.name}/B{w.B}"
     pb, db = algorithmic_bytes(w)
     dec_launch_ms = dec_ms / w.T
-    r_pre = roof(f"hyena_prefill_chunked x {nl} layers", pb * nl, pre_ms, peak, peak_src,
-                 ncu_traffic("prefill_chunk", key), note="per-layer launch: %.1f us, alternating over two streams"
-                 % (1e3 * pre_ms / nl))
-    r_pre["launch_ms"] = pre_ms / nl
-    r_pre["algorithmic_bytes_per_launch"] = pb
+    r_pre = roof(f"hyena_prefill_chunked_layers ({nl} layers per launch)", pb * nl, pre_ms, peak, peak_src,
+                 ncu_traffic("prefill_chunk_layers", key))
     t_dec = ncu_traffic("decode_layers", key)
     r_dec = roof(f"hyena_decode_step_layers ({nl} layers per launch)", db * nl, dec_launch_ms, peak, peak_src,
                  t_dec, dec_ms)
@@ -744,7 +733,7 @@ def measure_layers(args, w, nl: int, dev, steps: int, warmup: int, e2e_steps: in
                       "state": "%d MiB over %d layers (larger than L2)" % (nl * states[0].numel() * 4 >> 20, nl),
                       "inputs": f"{pool} distinct device-drawn input sets per layer, cycled"},
            "roofline_all": [r_pre, r_dec], "roofline": max([r_pre, r_dec], key=lambda x: x["total_ms"]),
-           "launches_per_step": 2 * nl + w.T, "clocks": clk}
+           "launches_per_step": 2 + w.T, "clocks": clk}
     if with_baselines:
         q0, k0, v0 = qkv[0]
         dq0, dk0, dv0 = dpool[0]
@@ -760,8 +749,8 @@ def measure_layers(args, w, nl: int, dev, steps: int, warmup: int, e2e_steps: in
 
     # ---- end to end through the C ABI: every step copies every layer's prompt q, k, v in from pinned
     # host memory and its y out, then every decode token's q, k, v of all layers in and its y out.
-    # Prefill: two device buffer sets, so layer l+1's prompt travels in while layer l computes and
-    # layer l-1's y travels out.  Decode: blocks of S tokens, two device blocks; a block's inputs
+    # Prefill: one call per layer (hyena_prefill_chunked) on two device buffer sets, so layer l+1's
+    # prompt travels in while layer l computes and layer l-1's y travels out.  Decode: blocks of S tokens, two device blocks; a block's inputs
     # (S tokens x all layers, one copy) travel in while the previous block decodes (CUDA graph per
     # device block), and its outputs travel out after it.
     if with_e2e:

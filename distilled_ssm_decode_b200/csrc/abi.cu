@@ -221,6 +221,52 @@ int hyena_test_chunked_inject(int suppress_item, double lookback_limit_s) {
     return HYENA_OK;
 }
 
+size_t hyena_prefill_chunked_layers_workspace_bytes(int layers, int B, int L, int Dch, int H, int d) {
+    if (layers < 1 || layers > chunked_max_layers()) return 0;
+    if (check_chunked(HYENA_BF16, B, L, Dch, H, d) != HYENA_OK) return 0;
+    return chunked_ws_bytes(B, L, Dch, H, d, layers);
+}
+
+size_t hyena_prefill_chunked_layers_error_offset(int layers, int B, int L, int Dch, int H, int d) {
+    if (layers < 1 || layers > chunked_max_layers()) return 0;
+    if (check_chunked(HYENA_BF16, B, L, Dch, H, d) != HYENA_OK) return 0;
+    return (size_t)chunked_error_offset(B, L, Dch, H, d, layers);
+}
+
+int hyena_prefill_chunked_layers(int layers, const void *const *q, const void *const *k, const void *const *v,
+                                 int dtype, int B, int L, int Dch, int H, int d, const float *const *lambda,
+                                 const float *const *R, const float *const *Dskip, void *const *y,
+                                 float *const *state_out, void *workspace, size_t ws_bytes, hyena_stream_t stream) {
+    if (layers < 0) return HYENA_ERR_SHAPE;
+    if (layers > chunked_max_layers()) return HYENA_ERR_UNSUPPORTED;
+    int st = check_chunked(dtype, B, L, Dch, H, d);
+    if (st != HYENA_OK) return st;
+    if (layers == 0 || B == 0 || Dch == 0) return HYENA_OK;
+    if (!state_out || !lambda || !R || !Dskip) return HYENA_ERR_ARG;
+    for (int i = 0; i < layers; ++i) {
+        if (!state_out[i] || !lambda[i] || !R[i] || !Dskip[i]) return HYENA_ERR_ARG;
+        if (!aligned(state_out[i], 8) || !aligned(lambda[i], 8) || !aligned(R[i], 8) || !aligned(Dskip[i], 4))
+            return HYENA_ERR_ALIGN;
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    if (L == 0) {
+        for (int i = 0; i < layers; ++i) {
+            const cudaError_t e = cudaMemsetAsync(state_out[i], 0, (size_t)B * d * Dch * 2 * sizeof(float), s);
+            if (e != cudaSuccess) return HYENA_ERR_CUDA;
+        }
+        return HYENA_OK;
+    }
+    if (!q || !k || !v || !y || !workspace) return HYENA_ERR_ARG;
+    for (int i = 0; i < layers; ++i) {
+        if (!q[i] || !k[i] || !v[i] || !y[i]) return HYENA_ERR_ARG;
+        if (!aligned(q[i], 16) || !aligned(k[i], 16) || !aligned(v[i], 16) || !aligned(y[i], 16)) return HYENA_ERR_ALIGN;
+    }
+    if (!aligned(workspace, kAlign)) return HYENA_ERR_ALIGN;
+    if (ws_bytes < chunked_ws_bytes(B, L, Dch, H, d, layers)) return HYENA_ERR_WORKSPACE;
+    return cuda_status(launch_prefill_chunked_layers(layers, q, k, v, B, L, Dch, H, d, lambda, R, Dskip, y, state_out,
+                                                     workspace, s));
+}
+
 size_t hyena_prompt_state_workspace_bytes(int B, int L, int Dch, int d) {
     if (B < 0 || L < 0 || Dch < 0 || d < 1 || d > HYENA_MAX_MODES) return 0;
     return align_up(state_ws_bytes(B, L, Dch, d));

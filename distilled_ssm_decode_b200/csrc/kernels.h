@@ -37,8 +37,14 @@ cudaError_t launch_prefill_fft(const void *q, const void *k, const void *v, int 
 
 // prefill_chunked.cu (bf16 activations, heads of a multiple of 64 channels, d <= 16)
 bool chunked_supported(int dtype, int Dch, int H, int d);
-size_t chunked_ws_bytes(int B, int L, int Dch, int H, int d);
-int chunked_error_offset(int B, int L, int Dch, int H, int d);
+// workspace and error-word offset for `layers` layers of the same shape in one launch
+size_t chunked_ws_bytes(int B, int L, int Dch, int H, int d, int layers = 1);
+int chunked_error_offset(int B, int L, int Dch, int H, int d, int layers = 1);
+int chunked_max_layers();
+cudaError_t launch_prefill_chunked_layers(int layers, const void *const *q, const void *const *k,
+                                          const void *const *v, int B, int L, int Dch, int H, int d,
+                                          const float *const *lam, const float *const *R, const float *const *Dskip,
+                                          void *const *y, float *const *state_out, void *ws, cudaStream_t s);
 // fault injection for tests: suppress one item's status word (-1: none) and bound each look-back
 // poll by wait_ns (0: the default bound); applies to every later launch
 void chunked_inject(int suppress_item, unsigned long long wait_ns);

@@ -45,9 +45,9 @@
 // contribution, then (segments after the first) obtains the
 // state entering its segment by a decoupled look-back over its predecessors'
 // published contributions (bounded polls), then runs the full pass.  The grid is
-// persistent: items come from a per-head atomic ticket counter, and each CTA's
+// persistent: items come from an atomic ticket counter, and each CTA's
 // pipelines run on across item boundaries.  Tickets are segment-major (all
-// units' first segments, then all second segments, ...), so an item's
+// heads' and units' first segments, then all second segments, ...), so an item's
 // predecessors were handed out a whole round of units earlier and have usually
 // published by the time it looks back.
 //
@@ -56,13 +56,16 @@
 // a CTA that is running (it took the ticket from the counter), whose earlier
 // items have lower tickets still; the state-only pass never waits.  By induction
 // over the tickets every look-back ends, even when other kernels hold most SMs.
-// When sequences are split, the counters are therefore cleared by a memset ahead
+// When sequences are split, the counter is therefore cleared by a memset ahead
 // of the constants kernel, so the loaders can take tickets at once.  When they
-// are not (no item waits on another), each CTA's first item has a fixed ticket
-// (blockIdx / H of head blockIdx % H) and only later tickets come from the
-// counters, which the constants kernel clears.  Every wait is bounded; on
-// timeout the kernel records an error code, drains its copies and MMAs, frees
-// tensor memory and returns.
+// are not (no item waits on another), each CTA's first ticket is fixed
+// (blockIdx.x) and only later tickets come from the counter, which the constants
+// kernel clears.  Every wait is bounded; on timeout the kernel records an error
+// code, drains its copies and MMAs, frees tensor memory and returns.
+//
+// Several independent layers of the same shape can share one launch: their heads
+// are the heads of one ticket space (layer = head / heads per layer), each with
+// its own constants and its own tensor maps, y and state.
 #include <atomic>
 
 #include <cuda.h>
@@ -193,7 +196,9 @@ __host__ __device__ __forceinline__ int cm_off16(int row, int k, int K) {
 }
 
 struct ChunkArgs {
-    int L, Dch, d, ch, H;
+    int L, Dch, d, ch;
+    int H;               // heads of the ticket space: layers x Hl (one counter and constant block each)
+    int Hl;              // heads per layer
     int tph;             // channel tiles per head (ch / NC)
     int units_h;         // (sequence, tile) units per head: B * tph
     int ih;              // items per head: units_h * nseg
@@ -201,10 +206,8 @@ struct ChunkArgs {
     int tok_base;        // first token of chunk 0 (L - nchunks * C, <= 0)
     int nseg, segc;      // segments per sequence, chunks per segment (all but the last)
     const uint8_t *consts;
-    __nv_bfloat16 *y;    // for the rows of a chunk that starts before token 0
-    float *state_out;    // [B][d][Dch][2]
     int *sched;          // [1] error code
-    int *tickets;        // [H] ticket counter per head
+    int *tickets;        // [1] ticket counter
     int *status;         // [items]: 0 none, 1 segment contribution, 2 inclusive state
     float *agg;          // [items][32 rows][NC ch]
     float *inc;          // [items][32 rows][NC ch]
@@ -214,26 +217,52 @@ struct ChunkArgs {
 };
 
 struct Item {
-    int id, b, c0, hd, seg, ck0, nck, n1, niter;
+    int id, b, c0, hd, layer, seg, ck0, nck, n1, niter;
     bool last_seg;
 };
+
+// Per-layer tensors of one launch (LMAX = 1 for a single layer, kMaxGroupLayers for a group of
+// independent layers): the TMA maps of q, k, v, y and the y and state pointers.  Passed by value
+// as a __grid_constant__ parameter, so the maps are in parameter space where TMA can read them.
+template <int LMAX>
+struct LayerMaps {
+    CUtensorMap q[LMAX], k[LMAX], v[LMAX], y[LMAX];
+    __nv_bfloat16 *yp[LMAX];   // y, for the rows of a chunk that starts before token 0
+    float *state[LMAX];        // [B][d][Dch][2]
+};
+template <int LMAX>
+struct ParamPtrs {
+    const float2 *lam[LMAX], *R[LMAX];
+    const float *Dskip[LMAX];
+};
+constexpr int kMaxGroupLayers = 32;
 
 template <int NC>
 __device__ __forceinline__ Item decode_item(const ChunkArgs &a, int id) {
     Item it;
     it.id = id;
-    it.hd = id / a.ih;
+    it.hd = id / a.ih;                      // head of the ticket space
+    it.layer = it.hd / a.Hl;
     const int t = id % a.ih;                // ticket within the head, segment-major: the
     const int unit = t % a.units_h;         // predecessor of item id is id - units_h
     it.seg = t / a.units_h;
     it.b = unit / a.tph;
-    it.c0 = it.hd * a.ch + (unit % a.tph) * NC;
+    it.c0 = (it.hd % a.Hl) * a.ch + (unit % a.tph) * NC;
     it.ck0 = it.seg * a.segc;
     it.nck = min(a.nchunks, it.ck0 + a.segc) - it.ck0;
     it.last_seg = (it.seg == a.nseg - 1);
     it.n1 = it.last_seg ? 0 : it.nck;        // state-only iterations
     it.niter = it.n1 + it.nck;
     return it;
+}
+
+// Item of ticket t: tickets run segment-major over all heads (t = (seg * H + head) * units_h + unit),
+// items are numbered head-major (id = head * ih + seg * units_h + unit, so that the predecessor of
+// item id is id - units_h).  Unsplit sequences: the identity.
+__device__ __forceinline__ int ticket_item(const ChunkArgs &a, int t) {
+    const int round = a.H * a.units_h;
+    const int seg = t / round, r = t % round;
+    return (r / a.units_h) * a.ih + seg * a.units_h + r % a.units_h;
 }
 
 enum : int { kErrWait = 1, kErrLookback = 2 };
@@ -365,14 +394,18 @@ static_assert(128 * (kC / 8) == kConstThreads && 128 * (kKS / 8) <= kConstThread
 // counters, segment status words), and allows the main kernel to launch at once (programmatic
 // dependent launch): where the main kernel's CTAs find room early, their set-up and first loads
 // overlap this kernel; its griddepcontrol.wait returns once everything written here is visible.
+// One block per head of the ticket space (layer hd / Hl, head hd % Hl of that layer).
+template <int LMAX>
 __global__ void __launch_bounds__(kConstThreads)
-chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R,
-                    const float *__restrict__ Dskip, int d, int seg_tokens,
+chunk_consts_kernel(const __grid_constant__ ParamPtrs<LMAX> pp, int Hl, int d, int seg_tokens,
                     uint8_t *__restrict__ consts, int *__restrict__ zero, int nzero) {
     asm volatile("griddepcontrol.launch_dependents;");
     const int t = threadIdx.x;
     for (int i = blockIdx.x * kConstThreads + t; i < nzero; i += gridDim.x * kConstThreads) zero[i] = 0;
-    const int hd = blockIdx.x;
+    const int hd = blockIdx.x, layer = hd / Hl, hl = hd % Hl;
+    const float2 *__restrict__ lam = pp.lam[layer];
+    const float2 *__restrict__ R = pp.R[layer];
+    const float *__restrict__ Dskip = pp.Dskip[layer];
     uint8_t *base = consts + (size_t)hd * kConstStride;
     float2 *lamC = reinterpret_cast<float2 *>(base + kLamOff);
     float2 *lamS = lamC + kMaxModes;
@@ -380,11 +413,11 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
     __shared__ float2 ls[kMaxModes], rs[kMaxModes];   // lambda_n, R_n
     __shared__ float hs[kC];                     // filter taps h_0 .. h_{C-1}
     __shared__ float dskip;
-    const long long n_par = (long long)gridDim.x * d;
+    const long long n_par = (long long)Hl * d;
     (void)n_par;
-    if (t < kMaxModes) ls[t] = t < d ? lam[HB_IDX((size_t)hd * d + t, n_par)] : make_float2(0.f, 0.f);
-    else if (t < 2 * kMaxModes) rs[t - kMaxModes] = t - kMaxModes < d ? R[HB_IDX((size_t)hd * d + t - kMaxModes, n_par)] : make_float2(0.f, 0.f);
-    else if (t == 2 * kMaxModes) dskip = Dskip[HB_IDX(hd, gridDim.x)];
+    if (t < kMaxModes) ls[t] = t < d ? lam[HB_IDX((size_t)hl * d + t, n_par)] : make_float2(0.f, 0.f);
+    else if (t < 2 * kMaxModes) rs[t - kMaxModes] = t - kMaxModes < d ? R[HB_IDX((size_t)hl * d + t - kMaxModes, n_par)] : make_float2(0.f, 0.f);
+    else if (t == 2 * kMaxModes) dskip = Dskip[HB_IDX(hl, Hl)];
     __syncthreads();
     {
         const int n = t / kC, k = t % kC;
@@ -458,11 +491,9 @@ chunk_consts_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R
 //                 4, 5, 8, 9      E group: token rows 0..63 x NC/2 channels each; gate and stage y
 // Each role loops over the same item sequence and the same chunk order; they meet only at
 // mbarriers, so loads, U, the products, the chain and the epilogue of different chunks overlap.
-template <int NC>
+template <int NC, int LMAX>
 __global__ void __launch_bounds__(kThreads, 1)
-prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_y,
-                     const ChunkArgs a) {
+prefill_chunk_kernel(const __grid_constant__ LayerMaps<LMAX> m, const ChunkArgs a) {
     using G = Geo<NC>;
     constexpr int kNC = NC, kTile = G::kTile, kStageBytes = G::kStageBytes, kKVStages = G::kKVStages,
                   kQStages = G::kQStages, kSlots = G::kSlots, kSlotCols = G::kSlotCols, kSBytes = G::kSBytes,
@@ -498,10 +529,12 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         for (int i = 0; i < kNumBars; ++i) tc::mbar_init(bar(i), G::count(i));
         tc::fence_mbar_init();
     } else if (tid == 32) {
-        tc::prefetch_tensormap(&tm_q);
-        tc::prefetch_tensormap(&tm_k);
-        tc::prefetch_tensormap(&tm_v);
-        tc::prefetch_tensormap(&tm_y);
+        // the maps of the layer of this CTA's first head (fetched on first use for the others)
+        const int l0 = ((int)blockIdx.x % a.H) / a.Hl;
+        tc::prefetch_tensormap(&m.q[l0]);
+        tc::prefetch_tensormap(&m.k[l0]);
+        tc::prefetch_tensormap(&m.v[l0]);
+        tc::prefetch_tensormap(&m.y[l0]);
     }
     if (warp == kWarpMMA) {
         tc::tmem_alloc(tc::smem_u32((const void *)(misc + 1)), kTmemCols);
@@ -567,37 +600,33 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (warp == kWarpKV) {
         // ------------------------------------------------------------ k,v loads + tickets
         if (lane == 0) {
-            int g = 0, head = blockIdx.x % a.H, tries = 0;
+            int g = 0;
             bool ok = true, counted = false;
             const uint64_t pol_keep = tc::l2_policy_evict_last(), pol_drop = tc::l2_policy_evict_first();
+            const int n_items = a.H * a.ih;
             for (int k = 0; ok; ++k) {
                 const int s = k % kItemQ;
                 if (!tc::mbar_wait(bar(kBarItemEmpty + s), ((k / kItemQ) & 1) ^ 1, abort)) {
                     ok = false;
                     break;
                 }
-                // tickets of this CTA's head first; when they run out, move on to the next head.  With
-                // fixed first tickets (unsplit sequences) the first item's ticket is blockIdx / H and the
-                // counter of head h hands out the tickets after the fixed ones of the CTAs assigned to
-                // h; those counters are cleared by the constants kernel, so the first counted ticket
-                // waits for it.  Otherwise every ticket comes from a counter cleared before this launch.
-                int id = -1;
-                if (k == 0 && a.fixed_first && (int)blockIdx.x / a.H < a.ih) {
-                    id = head * a.ih + (int)blockIdx.x / a.H;
+                // One ticket counter for all items, handed out segment-major: all heads' first segments,
+                // then all second segments, ..., so an item's predecessors always have lower tickets.
+                // With unsplit sequences each CTA's first ticket is fixed (blockIdx.x) and the counter,
+                // which the constants kernel clears, hands out the tickets after them; the first counted
+                // ticket waits for that kernel.  With split sequences every ticket comes from the
+                // counter, cleared before this launch.
+                int t = -1;
+                if (a.fixed_first && k == 0) {
+                    t = (int)blockIdx.x;
                 } else {
                     if (!counted) {
                         if (a.fixed_first) asm volatile("griddepcontrol.wait;" ::: "memory");
                         counted = true;
                     }
-                    while (tries < a.H) {
-                        const int fixed = !a.fixed_first ? 0
-                                          : head < (int)gridDim.x ? min(a.ih, ((int)gridDim.x - head + a.H - 1) / a.H) : 0;
-                        const int t = atomicAdd(a.tickets + head, 1) + fixed;
-                        if (t < a.ih) { id = head * a.ih + t; tries = 0; break; }
-                        head = head + 1 == a.H ? 0 : head + 1;
-                        ++tries;
-                    }
+                    t = atomicAdd(a.tickets, 1) + (a.fixed_first ? (int)gridDim.x : 0);
                 }
+                const int id = t < n_items ? ticket_item(a, t) : -1;
                 itemq[s] = id;
                 tc::mbar_arrive(bar(kBarItemFull + s));
                 if (id < 0) break;
@@ -615,9 +644,9 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     // them; the full pass reads them for the last time
                     const uint64_t pol = i < it.n1 ? pol_keep : pol_drop;
                     for (int h = 0; h < kNC / 64; ++h) {
-                        tc::tma_load_3d_hint(dst + h * kAtom, &tm_k, bar(kBarKVFull + st), it.c0 + 64 * h, tok_of(chunk),
+                        tc::tma_load_3d_hint(dst + h * kAtom, &m.k[it.layer], bar(kBarKVFull + st), it.c0 + 64 * h, tok_of(chunk),
                                              it.b, pol);
-                        tc::tma_load_3d_hint(dst + kTile + h * kAtom, &tm_v, bar(kBarKVFull + st), it.c0 + 64 * h,
+                        tc::tma_load_3d_hint(dst + kTile + h * kAtom, &m.v[it.layer], bar(kBarKVFull + st), it.c0 + 64 * h,
                                              tok_of(chunk), it.b, pol);
                     }
                 }
@@ -648,7 +677,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     }
                     tc::mbar_expect_tx(bar(kBarQFull + s), kTile);
                     for (int h = 0; h < kNC / 64; ++h)     // q is read once
-                        tc::tma_load_3d_hint(sbase + kSmQ + s * kTile + h * kAtom, &tm_q, bar(kBarQFull + s),
+                        tc::tma_load_3d_hint(sbase + kSmQ + s * kTile + h * kAtom, &m.q[it.layer], bar(kBarQFull + s),
                                              it.c0 + 64 * h, tok_of(it.ck0 + j), it.b, pol_drop);
                 }
             }
@@ -680,7 +709,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     const int tok = tok_of(it.ck0 + j);
                     if (tok >= 0)
                         for (int h = 0; h < kNC / 64; ++h)
-                            tc::tma_store_3d(&tm_y, sbase + kSmQ + s * kTile + h * kAtom, it.c0 + 64 * h, tok, it.b);
+                            tc::tma_store_3d(&m.y[it.layer], sbase + kSmQ + s * kTile + h * kAtom, it.c0 + 64 * h, tok, it.b);
                     tc::bulk_commit();
                     tc::bulk_wait_read<1>();        // every group but this one has been read
                     if (prev >= 0) tc::mbar_arrive(bar(kBarQEmpty + prev));
@@ -727,8 +756,9 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 if (id < 0) break;
                 const Item it = decode_item<NC>(a, id);
                 if (it.hd != cur_hd) {
-                    // constants of a new head (rare: a CTA keeps to one head until its items run
-                    // out).  No MMA may still read the old ones: every carry issued so far must be
+                    // constants of a new head (consecutive tickets of a CTA may belong to different
+                    // heads; the switch costs about one chunk's MMA issue, measured cheaper than
+                    // keeping CTAs on one head).  No MMA may still read the old ones: every carry issued so far must be
                     // issued and finished (each slot then has at most one carry outstanding, so
                     // its last completion is unambiguous), and so must this thread's own MMAs.
                     if (any) {
@@ -1047,7 +1077,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     // that each lane writes the (Re, Im) pairs of one channel: coalesced float2 stores
                     warp_transpose32(st, lane);
                     const size_t s0 = ((size_t)it.b * d) * a.Dch + it.c0 + kCh * q4 + lane;
-                    float2 *so = reinterpret_cast<float2 *>(a.state_out) + s0;
+                    float2 *so = reinterpret_cast<float2 *>(m.state[it.layer]) + s0;
 #pragma unroll
                     for (int m = 0; m < kMaxModes; ++m)
                         if (m < d && HB_OK(s0 + (size_t)m * a.Dch, (long long)(a.units_h / a.tph) * d * a.Dch))
@@ -1058,7 +1088,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     // channels x (Re, Im) = 128 contiguous bytes
                     warp_transpose16x2(st, lane);
                     const size_t s0 = (((size_t)it.b * d) * a.Dch + it.c0 + kCh * q4 + (lane & 15)) * 2 + (lane >> 4);
-                    float *so = a.state_out + s0;
+                    float *so = m.state[it.layer] + s0;
 #pragma unroll
                     for (int m = 0; m < kMaxModes; ++m)
                         if (m < d && HB_OK(s0 + (size_t)m * a.Dch * 2, (long long)(a.units_h / a.tph) * d * a.Dch * 2))
@@ -1100,7 +1130,7 @@ prefill_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 tc::tc_fence_after();
                 const int tok = tok_of(it.ck0 + j);
                 const bool store_direct = tok < 0, row_valid = tok + tau >= 0;
-                __nv_bfloat16 *yrow = a.y + ((size_t)it.b * a.L + (row_valid ? tok + tau : 0)) * a.Dch + it.c0;
+                __nv_bfloat16 *yrow = m.yp[it.layer] + ((size_t)it.b * a.L + (row_valid ? tok + tau : 0)) * a.Dch + it.c0;
 #pragma unroll
                 for (int x = 0; x < kNC / 64; ++x) {
                     const int cbase = hh * (kNC / 2) + 32 * x;      // first of 32 channels
@@ -1174,7 +1204,7 @@ bool make_map(CUtensorMap *m, const void *base, int B, int L, int Dch) {
                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr size_t kTicketOff = 64;    // byte offset of the per-head ticket counters in the schedule block
+constexpr size_t kTicketOff = 64;    // byte offset of the ticket counter in the schedule block
 
 struct ChunkPlan {
     int nc, nchunks, nseg, segc, items;
@@ -1190,8 +1220,9 @@ constexpr int kPlanSMs = 148;
 // is split (the state-only pass is counted in the work; the look-back and publication latency
 // is the 6).  The estimated makespan is the larger of the even share and the largest item, plus
 // half an item of tail when there are more items than SMs.  The narrow tile and unsplit
-// sequences are preferred whenever they do not cost more.
-ChunkPlan plan(int B, int L, int Dch, int H) {
+// sequences are preferred whenever they do not cost more.  `layers` independent layers of the
+// same shape share one launch: their (sequence, tile) units add up.
+ChunkPlan plan(int B, int L, int Dch, int H, int layers = 1) {
     ChunkPlan p{};
     p.nchunks = (L + kC - 1) / kC;
     const int ch = Dch / H;
@@ -1200,7 +1231,7 @@ ChunkPlan plan(int B, int L, int Dch, int H) {
     p.segc = p.nchunks > 0 ? p.nchunks : 1;
     for (int nc : {128, 64}) {
         if (ch % nc != 0) continue;
-        const double units = (double)B * (Dch / nc);
+        const double units = (double)layers * B * (Dch / nc);
         const double pass = nc / 128.0 + 0.1;
         const int nch = p.nchunks > 0 ? p.nchunks : 1;
         for (int want = 1; want <= kMaxSeg && want <= nch; ++want) {
@@ -1217,13 +1248,15 @@ ChunkPlan plan(int B, int L, int Dch, int H) {
         }
     }
     p.nseg = p.nchunks > 0 ? (p.nchunks + p.segc - 1) / p.segc : 1;
-    p.items = (int)((long long)B * (Dch / p.nc) * p.nseg);
+    p.items = (int)((long long)layers * B * (Dch / p.nc) * p.nseg);
+    // status words and published segment states exist only when sequences are split
+    const size_t split_items = p.nseg > 1 ? (size_t)p.items : 0;
     p.consts_off = 0;
-    p.sched_off = al256((size_t)H * kConstStride);
-    p.status_off = p.sched_off + al256(kTicketOff + (size_t)H * 4);
-    p.agg_off = p.status_off + al256((size_t)p.items * 4);
-    p.inc_off = p.agg_off + al256((size_t)p.items * kKS * p.nc * 4);
-    p.total = p.inc_off + al256((size_t)p.items * kKS * p.nc * 4);
+    p.sched_off = al256((size_t)layers * H * kConstStride);
+    p.status_off = p.sched_off + al256(kTicketOff + 4);
+    p.agg_off = p.status_off + al256(split_items * 4);
+    p.inc_off = p.agg_off + al256(split_items * kKS * p.nc * 4);
+    p.total = p.inc_off + al256(split_items * kKS * p.nc * 4);
     return p;
 }
 
@@ -1252,17 +1285,16 @@ bool chunked_supported(int dtype, int Dch, int H, int d) {
     return dtype == HYENA_BF16 && H > 0 && Dch % H == 0 && (Dch / H) % 64 == 0 && d >= 1 && d <= kMaxModes;
 }
 
-size_t chunked_ws_bytes(int B, int L, int Dch, int H, int d) {
+size_t chunked_ws_bytes(int B, int L, int Dch, int H, int d, int layers) {
     (void)d;
-    return plan(B, L, Dch, H).total;
+    return plan(B, L, Dch, H, layers).total;
 }
 
 namespace {
-template <int NC>
-cudaError_t launch_tile(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &my,
-                        const ChunkArgs &a, int items, cudaStream_t s) {
+template <int NC, int LMAX>
+cudaError_t launch_tile(const LayerMaps<LMAX> &m, const ChunkArgs &a, int items, cudaStream_t s) {
     constexpr int smem = Geo<NC>::kSmemBytes;
-    cudaError_t e = cudaFuncSetAttribute(prefill_chunk_kernel<NC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(prefill_chunk_kernel<NC, LMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int grid = items < sm_count() ? items : sm_count();
     cudaLaunchConfig_t cfg = {};
@@ -1275,16 +1307,17 @@ cudaError_t launch_tile(const CUtensorMap &mq, const CUtensorMap &mk, const CUte
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, prefill_chunk_kernel<NC>, mq, mk, mv, my, a);
+    e = cudaLaunchKernelEx(&cfg, prefill_chunk_kernel<NC, LMAX>, m, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
-}  // namespace
 
-cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, int B, int L, int Dch,
-                                   int H, int d, const float2 *lam, const float2 *R, const float *Dskip,
-                                   void *y, float *state_out, void *ws, cudaStream_t s) {
-    const ChunkPlan p = plan(B, L, Dch, H);
+// The constants kernel, then the main kernel, for `layers` layers of the same shape (LMAX >= layers).
+template <int LMAX>
+cudaError_t launch_group(int layers, const void *const *q, const void *const *k, const void *const *v, int B, int L,
+                         int Dch, int H, int d, const float2 *const *lam, const float2 *const *R,
+                         const float *const *Dskip, void *const *y, float *const *state_out, void *ws, cudaStream_t s) {
+    const ChunkPlan p = plan(B, L, Dch, H, layers);
     uint8_t *w = static_cast<uint8_t *>(ws);
     // schedule words (error word, ticket counters, status words): with split sequences they are
     // cleared ahead of the constants kernel, so that every ticket can come from a counter at once
@@ -1292,22 +1325,36 @@ cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, 
     const int nzero = (int)((p.agg_off - p.sched_off) / 4);
     cudaError_t e;
     if (!fixed_first && (e = cudaMemsetAsync(w + p.sched_off, 0, (size_t)nzero * 4, s)) != cudaSuccess) return e;
-    chunk_consts_kernel<<<H, kConstThreads, 0, s>>>(lam, R, Dskip, d, p.segc * kC, w + p.consts_off,
-                                          reinterpret_cast<int *>(w + p.sched_off), fixed_first ? nzero : 0);
+    ParamPtrs<LMAX> pp;
+    LayerMaps<LMAX> m;
+    for (int l = 0; l < LMAX; ++l) {
+        const int j = l < layers ? l : 0;       // unused entries repeat layer 0
+        pp.lam[l] = lam[j];
+        pp.R[l] = R[j];
+        pp.Dskip[l] = Dskip[j];
+        m.yp[l] = static_cast<__nv_bfloat16 *>(y[j]);
+        m.state[l] = state_out[j];
+        if (l < layers && (!make_map(&m.q[l], q[l], B, L, Dch) || !make_map(&m.k[l], k[l], B, L, Dch) ||
+                           !make_map(&m.v[l], v[l], B, L, Dch) || !make_map(&m.y[l], y[l], B, L, Dch)))
+            return cudaErrorInvalidValue;
+        if (l >= layers) {
+            m.q[l] = m.q[0];
+            m.k[l] = m.k[0];
+            m.v[l] = m.v[0];
+            m.y[l] = m.y[0];
+        }
+    }
+    chunk_consts_kernel<LMAX><<<layers * H, kConstThreads, 0, s>>>(pp, H, d, p.segc * kC, w + p.consts_off,
+                                                                 reinterpret_cast<int *>(w + p.sched_off),
+                                                                 fixed_first ? nzero : 0);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    CUtensorMap mq, mk, mv, my;
-    if (!make_map(&mq, q, B, L, Dch) || !make_map(&mk, k, B, L, Dch) || !make_map(&mv, v, B, L, Dch) ||
-        !make_map(&my, y, B, L, Dch))
-        return cudaErrorInvalidValue;
     ChunkArgs a;
-    a.L = L; a.Dch = Dch; a.d = d; a.ch = Dch / H; a.H = H;
+    a.L = L; a.Dch = Dch; a.d = d; a.ch = Dch / H; a.H = layers * H; a.Hl = H;
     a.tph = a.ch / p.nc; a.units_h = B * a.tph; a.ih = a.units_h * p.nseg;
     a.nchunks = p.nchunks; a.tok_base = L - p.nchunks * kC;
     a.nseg = p.nseg; a.segc = p.segc;
     a.consts = w + p.consts_off;
-    a.y = static_cast<__nv_bfloat16 *>(y);
-    a.state_out = state_out;
     a.sched = reinterpret_cast<int *>(w + p.sched_off);
     a.tickets = reinterpret_cast<int *>(w + p.sched_off + kTicketOff);
     a.status = reinterpret_cast<int *>(w + p.status_off);
@@ -1317,12 +1364,34 @@ cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, 
     a.suppress_item = g_inject_item.load();
     const unsigned long long inj_ns = g_inject_wait_ns.load();
     a.lookback_ns = inj_ns ? inj_ns : tc::kWaitNs;
-    return p.nc == 128 ? launch_tile<128>(mq, mk, mv, my, a, p.items, s) : launch_tile<64>(mq, mk, mv, my, a, p.items, s);
+    return p.nc == 128 ? launch_tile<128, LMAX>(m, a, p.items, s) : launch_tile<64, LMAX>(m, a, p.items, s);
+}
+}  // namespace
+
+cudaError_t launch_prefill_chunked(const void *q, const void *k, const void *v, int B, int L, int Dch,
+                                   int H, int d, const float2 *lam, const float2 *R, const float *Dskip,
+                                   void *y, float *state_out, void *ws, cudaStream_t s) {
+    return launch_group<1>(1, &q, &k, &v, B, L, Dch, H, d, &lam, &R, &Dskip, &y, &state_out, ws, s);
 }
 
-int chunked_error_offset(int B, int L, int Dch, int H, int d) {
+int chunked_max_layers() { return kMaxGroupLayers; }
+
+cudaError_t launch_prefill_chunked_layers(int layers, const void *const *q, const void *const *k,
+                                          const void *const *v, int B, int L, int Dch, int H, int d,
+                                          const float *const *lam, const float *const *R, const float *const *Dskip,
+                                          void *const *y, float *const *state_out, void *ws, cudaStream_t s) {
+    if (layers < 1 || layers > kMaxGroupLayers) return cudaErrorInvalidValue;
+    const float2 *lam2[kMaxGroupLayers], *R2[kMaxGroupLayers];
+    for (int l = 0; l < layers; ++l) {
+        lam2[l] = reinterpret_cast<const float2 *>(lam[l]);
+        R2[l] = reinterpret_cast<const float2 *>(R[l]);
+    }
+    return launch_group<kMaxGroupLayers>(layers, q, k, v, B, L, Dch, H, d, lam2, R2, Dskip, y, state_out, ws, s);
+}
+
+int chunked_error_offset(int B, int L, int Dch, int H, int d, int layers) {
     (void)d;
-    return (int)(plan(B, L, Dch, H).sched_off + 4);
+    return (int)(plan(B, L, Dch, H, layers).sched_off + 4);
 }
 
 void chunked_inject(int suppress_item, unsigned long long wait_ns) {

@@ -39,6 +39,10 @@ SIGNATURES = {
     "hyena_prefill_chunked_error_offset": (_sz, [_i, _i, _i, _i, _i]),
     "hyena_prefill_chunked": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp, _fp,
                                    _vp, _sz, _vp]),
+    "hyena_prefill_chunked_layers_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "hyena_prefill_chunked_layers_error_offset": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "hyena_prefill_chunked_layers": (_i, [_i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
+                                          _vp, _sz, _vp]),
     "hyena_prefill_noalloc_capacity": (_sz, []),
     "hyena_prefill_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp, _fp,
                                    _vp]),
@@ -225,6 +229,61 @@ def prefill_chunked(q, k, v, lam, R, Dskip, y=None, state=None, workspace=None):
                                        _ptr(R), _ptr(Dskip), _ptr(y), _ptr(state), _ptr(workspace),
                                        workspace.numel(), _stream(q.device)))
     return y, state, workspace
+
+
+class PrefillLayerSet:
+    """Host pointer arrays of a fixed set of layers for prefill_chunked_layers (built once, so that
+    a call costs one library call): per layer q, k, v, y [B][L][Dch] bf16, state [B][d][Dch][2]
+    float32 and the modal parameters."""
+
+    def __init__(self, qs, ks, vs, ys, states, lams, Rs, Dskips):
+        n = len(qs)
+        if not all(len(x) == n for x in (ks, vs, ys, states, lams, Rs, Dskips)):
+            raise ValueError("one tensor of each kind per layer")
+        q0 = _cuda(qs[0], "q")
+        self.dt = _act_dtype(q0)
+        self.B, self.L, self.Dch = q0.shape
+        ps = [_params(l, r, dk) for l, r, dk in zip(lams, Rs, Dskips)]
+        self.H, self.d = ps[0][0].shape[0], ps[0][0].shape[1]
+        for name, ts in (("q", qs), ("k", ks), ("v", vs), ("y", ys)):
+            for t in ts:
+                _cuda(t, name, q0.dtype)
+                if tuple(t.shape) != (self.B, self.L, self.Dch):
+                    raise ValueError(f"{name}: every layer's tensor must be [B][L][Dch]")
+        for st in states:
+            _cuda(st, "state", torch.float32)
+        if any(p[0].shape != ps[0][0].shape for p in ps):
+            raise ValueError("all layers need the same H and d")
+        self.n = n
+        self._keep = (list(qs), list(ks), list(vs), list(ys), list(states), ps)
+        arr = ctypes.c_void_p * max(n, 1)
+        self.q, self.k, self.v, self.y, self.state = (arr(*[t.data_ptr() for t in ts]) for ts in (qs, ks, vs, ys, states))
+        self.lam = arr(*[p[0].data_ptr() for p in ps])
+        self.R = arr(*[p[1].data_ptr() for p in ps])
+        self.Dskip = arr(*[p[2].data_ptr() for p in ps])
+        self.device = q0.device
+
+    def workspace_bytes(self) -> int:
+        return int(lib().hyena_prefill_chunked_layers_workspace_bytes(self.n, self.B, self.L, self.Dch, self.H, self.d))
+
+    def error(self, workspace) -> int:
+        """The kernel's error word (synchronises): 0 when every bounded wait succeeded."""
+        off = int(lib().hyena_prefill_chunked_layers_error_offset(self.n, self.B, self.L, self.Dch, self.H, self.d))
+        return int(workspace[off:off + 4].view(torch.int32).item())
+
+
+def prefill_chunked_layers(layers: PrefillLayerSet, workspace=None):
+    """Chunked prefill of every layer of the set in one launch (writes each layer's y and state).
+    Returns the workspace."""
+    nbytes = layers.workspace_bytes()
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=layers.device)
+    _check("hyena_prefill_chunked_layers",
+           lib().hyena_prefill_chunked_layers(layers.n, layers.q, layers.k, layers.v, layers.dt, layers.B, layers.L,
+                                              layers.Dch, layers.H, layers.d, layers.lam, layers.R, layers.Dskip,
+                                              layers.y, layers.state, _ptr(workspace), workspace.numel(),
+                                              _stream(layers.device)))
+    return workspace
 
 
 def chunked_error(workspace, B, L, Dch, H, d) -> int:

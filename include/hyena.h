@@ -207,6 +207,35 @@ int hyena_prefill_chunked(const void *q, const void *k, const void *v, int dtype
                           void *y, float *state_out,
                           void *workspace, size_t ws_bytes, hyena_stream_t stream);
 
+/* Largest number of layers one hyena_prefill_chunked_layers call takes. */
+#define HYENA_MAX_PREFILL_LAYERS 32
+
+/*
+ * hyena_prefill_chunked for `layers` independent operator layers of the same
+ * shape in one launch (e.g. the 24 operator layers of a 1.3B-shaped
+ * generation workload, each with its own prompt activations, modal filter and
+ * state).  The results of layer i are those of hyena_prefill_chunked on layer
+ * i's arguments; the layers' work items share one persistent grid, so no layer
+ * pays its own start and end.  (The prefill of the "Laughing Hyena Distillery"
+ * review, "Main findings": every layer hands its O(d) state to generation.)
+ *   q, k, v, y, state_out, lambda, R, Dskip: HOST arrays of `layers` device
+ *   pointers each, as hyena_prefill_chunked's arguments of each layer (read
+ *   during the call only).  B, L, Dch, H, d and dtype are shared.
+ *   0 <= layers <= HYENA_MAX_PREFILL_LAYERS (HYENA_ERR_UNSUPPORTED above).
+ *   Implemented and aligned as hyena_prefill_chunked.  Layers must not share
+ *   output buffers.
+ *   workspace: >= hyena_prefill_chunked_layers_workspace_bytes() bytes, 256-byte
+ *   aligned; its error word (hyena_prefill_chunked_layers_error_offset()) is 0
+ *   after a successful run, as for hyena_prefill_chunked.
+ */
+size_t hyena_prefill_chunked_layers_workspace_bytes(int layers, int B, int L, int Dch, int H, int d);
+size_t hyena_prefill_chunked_layers_error_offset(int layers, int B, int L, int Dch, int H, int d);
+int hyena_prefill_chunked_layers(int layers, const void *const *q, const void *const *k, const void *const *v,
+                                 int dtype, int B, int L, int Dch, int H, int d,
+                                 const float *const *lambda, const float *const *R, const float *const *Dskip,
+                                 void *const *y, float *const *state_out,
+                                 void *workspace, size_t ws_bytes, hyena_stream_t stream);
+
 /*
  * Bounds-checked build (no counterpart in the pages): libhyena_b200_dbg.so is
  * the same library compiled with every kernel checking the index of each

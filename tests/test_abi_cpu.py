@@ -209,3 +209,19 @@ def test_fault_injection_hook_validates_its_arguments(lib):
     assert lib.hyena_test_chunked_inject(0, -1.0) == ERR_ARG
     assert lib.hyena_test_chunked_inject(0, 61.0) == ERR_ARG
     assert lib.hyena_test_chunked_inject(-1, 0.0) == OK
+
+
+def test_prefill_chunked_layers_validation(lib):
+    arr = (ctypes.c_void_p * 1)(FAKE)
+    call = lambda layers, dtype=1, B=2, L=64, Dch=128, H=2, d=4, ws=1 << 30: lib.hyena_prefill_chunked_layers(
+        layers, arr, arr, arr, dtype, B, L, Dch, H, d, arr, arr, arr, arr, arr, _p(), ws, None)
+    assert call(-1) == ERR_SHAPE
+    assert call(33) == ERR_UNSUP
+    assert call(1, dtype=0) == ERR_UNSUP          # fp32 activations: FFT route only
+    assert call(1, Dch=64, H=2) == ERR_UNSUP      # 32 channels per head
+    assert call(1, d=17) == ERR_UNSUP
+    assert call(1, ws=0) == ERR_WS
+    assert call(0) == OK
+    assert lib.hyena_prefill_chunked_layers_workspace_bytes(33, 2, 64, 128, 2, 4) == 0
+    assert lib.hyena_prefill_chunked_layers_workspace_bytes(24, 64, 512, 2048, 16, 16) > \
+        lib.hyena_prefill_chunked_workspace_bytes(64, 512, 2048, 16, 16)

@@ -330,3 +330,47 @@ def test_chunked_segments_progress_with_most_sms_busy(B, L, Dch, H):
     torch.cuda.synchronize()
     assert ops.chunked_error(ws2, B, L, Dch, H, 16) == 0
     assert torch.equal(y1, y2) and torch.equal(s1, s2)
+
+
+@pytest.mark.parametrize("nl,B,L,Dch,hd_ch,d", [(3, 2, 300, 256, 128, 16), (2, 1, 4096, 128, 64, 16),
+                                                  (5, 1, 65, 192, 64, 5)])
+def test_chunked_layers_match_oracle(oracle, record_property, nl, B, L, Dch, hd_ch, d):
+    """Several independent layers in one launch (their work items share the persistent grid; with one
+    sequence and 64-channel heads the sequences are split into segments): every layer's y and
+    state against the oracle."""
+    H = Dch // hd_ch
+    w = W.Workload(700 + L + d, "layers", B=B, L=L, Dch=Dch, H=H, d=d, dtype="bf16", fft_len=0, T=0)
+    ps = [W.params(w, layer=l) for l in range(nl)]
+    qkv = [W.prefill_inputs(w, layer=l) for l in range(nl)]
+    dev = [dev_params(p) for p in ps]
+    qs, ks, vs = ([x[j].cuda() for x in qkv] for j in range(3))
+    ys = [torch.empty_like(q) for q in qs]
+    sts = [torch.empty((B, d, Dch, 2), device="cuda") for _ in range(nl)]
+    ls = ops.PrefillLayerSet(qs, ks, vs, ys, sts, [x[0] for x in dev], [x[1] for x in dev], [x[2] for x in dev])
+    ws = ops.prefill_chunked_layers(ls)
+    assert ls.error(ws) == 0
+    for l in range(nl):
+        qf, kf, vf = (W.to_f64(t) for t in qkv[l])
+        y_ref, s_ref = oracle.recurrent(qf, kf, vf, ps[l].lam, ps[l].R, ps[l].Dskip, H=H)
+        ey, es = rel_err(ys[l].cpu().double().numpy(), y_ref), rel_err(state_c128(sts[l]), s_ref)
+        _check_errors(record_property, ey, es)
+
+
+def test_chunked_layers_equal_single_layer_calls_1p3b():
+    """The 24 layers of the 1.3B-shaped workload in one launch give the same bits as 24 single-layer
+    calls (the same plan: 128-channel tiles, sequences not split)."""
+    w = W.WORKLOADS["gen1p3b_bf16"]
+    nl = w.layers
+    ps = [W.params(w, layer=l) for l in range(nl)]
+    dev = [dev_params(p) for p in ps]
+    qkv = [W.prefill_inputs_device(w, l) for l in range(nl)]
+    ys = [torch.empty_like(x[0]) for x in qkv]
+    sts = [torch.empty((w.B, w.d, w.Dch, 2), device="cuda") for _ in range(nl)]
+    ls = ops.PrefillLayerSet([x[0] for x in qkv], [x[1] for x in qkv], [x[2] for x in qkv], ys, sts,
+                             [x[0] for x in dev], [x[1] for x in dev], [x[2] for x in dev])
+    ws = ops.prefill_chunked_layers(ls)
+    assert ls.error(ws) == 0
+    for l in range(nl):
+        y1, s1, ws1 = ops.prefill_chunked(*qkv[l], *dev[l])
+        assert ops.chunked_error(ws1, w.B, w.L, w.Dch, w.H, w.d) == 0
+        assert torch.equal(y1, ys[l]) and torch.equal(s1, sts[l]), l
