@@ -756,11 +756,13 @@ def measure_layers(args, w, nl: int, dev, steps: int, warmup: int, e2e_steps: in
     if with_e2e:
         S = 64
         nblk = (w.T + S - 1) // S
-        # host memory: every layer's prompt (pinned, distinct per layer); one pinned block of S decode
-        # tokens' inputs, tiled from the device input pool and copied in for every block; outputs to
-        # two pinned prompt-y buffers and two pinned decode-y blocks, alternating
-        hp = [[make_pinned(t.shape, t.dtype) for t in qkv[l]] for l in range(nl)]
-        for l in range(nl):
+        # host memory (pinned): the prompts of 4 layers, which the 24 layers' copies cycle through (each
+        # layer's prompt still crosses PCIe every step; the pool only bounds pinned memory, ~4 GB per
+        # GPU in all); one block of S decode tokens' inputs, tiled from the device input pool and copied
+        # in for every block; outputs to two prompt-y buffers and two decode-y blocks, alternating
+        P = min(4, nl)
+        hp = [[make_pinned(t.shape, t.dtype) for t in qkv[l]] for l in range(P)]
+        for l in range(P):
             for j in range(3):
                 hp[l][j].copy_(qkv[l][j])
         hblk = make_pinned((S, nl, 3, w.B, w.Dch), w.torch_dtype)
@@ -804,7 +806,7 @@ def measure_layers(args, w, nl: int, dev, steps: int, warmup: int, e2e_steps: in
                 s_in.wait_event(pc[j])
                 with torch.cuda.stream(s_in):
                     for x in range(3):
-                        dset[j][x].copy_(hp[l][x], non_blocking=True)
+                        dset[j][x].copy_(hp[l % P][x], non_blocking=True)
                 got = ev()
                 got.record(s_in)
                 stream.wait_event(got)
@@ -858,9 +860,9 @@ def measure_layers(args, w, nl: int, dev, steps: int, warmup: int, e2e_steps: in
                       "overlap": (f"prompt: two device buffer sets, layer l+1 copied in while layer l computes; "
                                   f"decode: blocks of {S} tokens x {nl} layers, two device blocks; copy-in, compute "
                                   f"and copy-out streams"),
-                      "host_buffers": ("every layer's prompt distinct in pinned memory; one pinned block of "
-                                       f"{S} tokens' decode inputs, copied in for each of the {nblk} blocks; "
-                                       "outputs to two alternating pinned buffers")}
+                      "host_buffers": (f"pinned prompts of {P} layers, cycled over the {nl} layers' copies; one "
+                                       f"pinned block of {S} tokens' decode inputs, copied in for each of the "
+                                       f"{nblk} blocks; outputs to two alternating pinned buffers")}
         del graphs
     return rec
 

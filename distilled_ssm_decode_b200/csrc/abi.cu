@@ -5,6 +5,8 @@
 // entry point allocates, frees or synchronises; all work goes on `stream`.
 #include <stdint.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -19,6 +21,19 @@ bool is_pow2(long long x) { return x > 0 && (x & (x - 1)) == 0; }
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA; }
+
+// Test hook (hyena_test_fail_next_launches): the next n calls that pass validation report a CUDA
+// failure instead of enqueuing anything, as a failed launch would.
+std::atomic<int> g_fail_launches{0};
+bool injected_launch_failure() {
+    int n = g_fail_launches.load();
+    while (n > 0 && !g_fail_launches.compare_exchange_weak(n, n - 1)) {}
+    return n > 0;
+}
+#define HYENA_LAUNCH_GUARD() \
+    do {                     \
+        if (injected_launch_failure()) return HYENA_ERR_CUDA; \
+    } while (0)
 
 int check_common(int H, int d, int Dch) {
     if (H < 1 || Dch < 0) return HYENA_ERR_SHAPE;
@@ -85,6 +100,7 @@ int hyena_filter_from_modes(const float *lambda, const float *R, const float *Ds
     if (!lambda || !R || !Dskip || !h_out) return HYENA_ERR_ARG;
     if (!aligned(lambda, 8) || !aligned(R, 8) || !aligned(Dskip, 4) || !aligned(h_out, 4))
         return HYENA_ERR_ALIGN;
+    HYENA_LAUNCH_GUARD();
     return cuda_status(launch_filter(reinterpret_cast<const float2 *>(lambda),
                                      reinterpret_cast<const float2 *>(R), Dskip, H, d, L, h_out,
                                      (cudaStream_t)stream));
@@ -105,6 +121,7 @@ int hyena_filter_spectrum(const float *h, int H, int L, int fft_len, float *spec
     if (ws_bytes < hyena_filter_spectrum_workspace_bytes(H, L, fft_len)) return HYENA_ERR_WORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
     float2 *perm = static_cast<float2 *>(workspace);
+    HYENA_LAUNCH_GUARD();
     cudaError_t e = launch_spectrum_perm(h, H, L, fft_len, perm, 1.0f, s);
     if (e != cudaSuccess) return HYENA_ERR_CUDA;
     return cuda_status(launch_spectrum_natural(perm, H, fft_len, reinterpret_cast<float2 *>(spec_out), s));
@@ -127,8 +144,10 @@ int hyena_prefill(const void *q, const void *k, const void *v, int dtype, int B,
     if (!state_out || !lambda || !R || !Dskip) return HYENA_ERR_ARG;
     if (!aligned(state_out, 8) || !aligned(lambda, 8) || !aligned(R, 8) || !aligned(Dskip, 4))
         return HYENA_ERR_ALIGN;
-    if (L == 0)
+    if (L == 0) {
+        HYENA_LAUNCH_GUARD();
         return cuda_status(cudaMemsetAsync(state_out, 0, (size_t)B * d * Dch * 2 * sizeof(float), s));
+    }
     if (!q || !k || !v || !y || !workspace) return HYENA_ERR_ARG;
     const size_t ab = (dtype == HYENA_BF16) ? 2 : 4;
     if (!aligned(q, 2 * ab) || !aligned(k, 2 * ab) || !aligned(v, 2 * ab) || !aligned(y, 2 * ab) ||
@@ -141,6 +160,7 @@ int hyena_prefill(const void *q, const void *k, const void *v, int dtype, int B,
     float2 *spec = reinterpret_cast<float2 *>(ws + w.spec_off);
     const int N = fft_internal_len(fft_len);
     const float2 *lam2 = reinterpret_cast<const float2 *>(lambda);
+    HYENA_LAUNCH_GUARD();
     cudaError_t e = launch_filter(lam2, reinterpret_cast<const float2 *>(R), Dskip, H, d, L, h, s);
     if (e != cudaSuccess) return HYENA_ERR_CUDA;
     // the inverse transform is unnormalised: fold its 1/N into the spectrum
@@ -180,12 +200,15 @@ int hyena_prefill_chunked(const void *q, const void *k, const void *v, int dtype
     if (!state_out || !lambda || !R || !Dskip) return HYENA_ERR_ARG;
     if (!aligned(state_out, 8) || !aligned(lambda, 8) || !aligned(R, 8) || !aligned(Dskip, 4))
         return HYENA_ERR_ALIGN;
-    if (L == 0)
+    if (L == 0) {
+        HYENA_LAUNCH_GUARD();
         return cuda_status(cudaMemsetAsync(state_out, 0, (size_t)B * d * Dch * 2 * sizeof(float), s));
+    }
     if (!q || !k || !v || !y || !workspace) return HYENA_ERR_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(y, 16) || !aligned(workspace, kAlign))
         return HYENA_ERR_ALIGN;
     if (ws_bytes < chunked_ws_bytes(B, L, Dch, H, d)) return HYENA_ERR_WORKSPACE;
+    HYENA_LAUNCH_GUARD();
     return cuda_status(launch_prefill_chunked(q, k, v, B, L, Dch, H, d, reinterpret_cast<const float2 *>(lambda),
                                               reinterpret_cast<const float2 *>(R), Dskip, y, state_out,
                                               workspace, s));
@@ -213,6 +236,12 @@ int hyena_debug_bounds_check(long long *record) {
         }
     }
     return found;
+}
+
+int hyena_test_fail_next_launches(int n) {
+    if (n < 0) return HYENA_ERR_ARG;
+    g_fail_launches.store(n);
+    return HYENA_OK;
 }
 
 int hyena_test_chunked_inject(int suppress_item, double lookback_limit_s) {
@@ -250,6 +279,7 @@ int hyena_prefill_chunked_layers(int layers, const void *const *q, const void *c
     }
     cudaStream_t s = (cudaStream_t)stream;
     if (L == 0) {
+        HYENA_LAUNCH_GUARD();
         for (int i = 0; i < layers; ++i) {
             const cudaError_t e = cudaMemsetAsync(state_out[i], 0, (size_t)B * d * Dch * 2 * sizeof(float), s);
             if (e != cudaSuccess) return HYENA_ERR_CUDA;
@@ -263,6 +293,7 @@ int hyena_prefill_chunked_layers(int layers, const void *const *q, const void *c
     }
     if (!aligned(workspace, kAlign)) return HYENA_ERR_ALIGN;
     if (ws_bytes < chunked_ws_bytes(B, L, Dch, H, d, layers)) return HYENA_ERR_WORKSPACE;
+    HYENA_LAUNCH_GUARD();
     return cuda_status(launch_prefill_chunked_layers(layers, q, k, v, B, L, Dch, H, d, lambda, R, Dskip, y, state_out,
                                                      workspace, s));
 }
@@ -284,12 +315,15 @@ int hyena_prompt_state(const void *k, const void *v, int dtype, int B, int L, in
     if (!state_out || !lambda) return HYENA_ERR_ARG;
     if (!aligned(state_out, 8) || !aligned(lambda, 8)) return HYENA_ERR_ALIGN;
     cudaStream_t s = (cudaStream_t)stream;
-    if (L == 0)
+    if (L == 0) {
+        HYENA_LAUNCH_GUARD();
         return cuda_status(cudaMemsetAsync(state_out, 0, (size_t)B * d * Dch * 2 * sizeof(float), s));
+    }
     if (!k || !v || !workspace) return HYENA_ERR_ARG;
     const size_t ab = (dtype == HYENA_BF16) ? 2 : 4;
     if (!aligned(k, ab) || !aligned(v, ab) || !aligned(workspace, kAlign)) return HYENA_ERR_ALIGN;
     if (ws_bytes < hyena_prompt_state_workspace_bytes(B, L, Dch, d)) return HYENA_ERR_WORKSPACE;
+    HYENA_LAUNCH_GUARD();
     return cuda_status(launch_prompt_state(k, v, dtype, B, L, Dch, H, d,
                                            reinterpret_cast<const float2 *>(lambda), state_out,
                                            workspace, s));
@@ -308,6 +342,7 @@ int hyena_decode_step(const void *q, const void *k, const void *v, int dtype, in
     if (!aligned(q, ab) || !aligned(k, ab) || !aligned(v, ab) || !aligned(y, ab) ||
         !aligned(state, 8) || !aligned(lambda, 8) || !aligned(R, 8) || !aligned(Dskip, 4))
         return HYENA_ERR_ALIGN;
+    HYENA_LAUNCH_GUARD();
     return cuda_status(launch_decode_step(q, k, v, dtype, B, Dch, H, d,
                                           reinterpret_cast<const float2 *>(lambda),
                                           reinterpret_cast<const float2 *>(R), Dskip, state, y,
@@ -335,6 +370,7 @@ int hyena_decode_step_layers(int layers, const void *const *q, const void *const
             !aligned(R[i], 8) || !aligned(Dskip[i], 4))
             return HYENA_ERR_ALIGN;
     }
+    HYENA_LAUNCH_GUARD();
     return cuda_status(launch_decode_layers(layers, q, k, v, dtype, B, Dch, H, d, lambda, R, Dskip, state, y,
                                             (cudaStream_t)stream));
 }
@@ -347,6 +383,7 @@ int hyena_fir_cache_prompt(const void *k, const void *v, int dtype, int B, int L
     if (!k || !v || !u_cache) return HYENA_ERR_ARG;
     const size_t ab = (dtype == HYENA_BF16) ? 2 : 4;
     if (!aligned(k, ab) || !aligned(v, ab) || !aligned(u_cache, 4)) return HYENA_ERR_ALIGN;
+    HYENA_LAUNCH_GUARD();
     return cuda_status(launch_fir_fill(k, v, dtype, B, L, Dch, t_max, u_cache, (cudaStream_t)stream));
 }
 
@@ -361,6 +398,7 @@ int hyena_fir_decode_step(const void *q, const void *k, const void *v, int dtype
     if (!aligned(q, ab) || !aligned(k, ab) || !aligned(v, ab) || !aligned(y, ab) || !aligned(h, 4) ||
         !aligned(u_cache, 4))
         return HYENA_ERR_ALIGN;
+    HYENA_LAUNCH_GUARD();
     return cuda_status(launch_fir_step(q, k, v, dtype, B, Dch, H, t, t_max, h, u_cache, y, (cudaStream_t)stream));
 }
 
@@ -373,6 +411,7 @@ int hyena_modal_truncate(const float *lambda, const float *R, int H, int d, int 
     if (!aligned(lambda, 8) || !aligned(R, 8) || !aligned(bound, 8) || !aligned(err_l2, 8) ||
         (k > 0 && (!aligned(kept, 4) || !aligned(lambda_out, 8) || !aligned(R_out, 8))))
         return HYENA_ERR_ALIGN;
+    HYENA_LAUNCH_GUARD();
     return cuda_status(launch_modal_truncate(reinterpret_cast<const float2 *>(lambda),
                                              reinterpret_cast<const float2 *>(R), H, d, k, kept,
                                              reinterpret_cast<float2 *>(lambda_out),

@@ -47,6 +47,7 @@ SIGNATURES = {
     "hyena_prefill_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp, _fp,
                                    _vp]),
     "hyena_test_chunked_inject": (_i, [_i, ctypes.c_double]),
+    "hyena_test_fail_next_launches": (_i, [_i]),
     "hyena_debug_bounds_check": (_i, [_vp]),
     "hyena_prompt_state_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "hyena_prompt_state": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _fp, _fp, _vp, _sz, _vp]),

@@ -251,6 +251,15 @@ int hyena_prefill_chunked_layers(int layers, const void *const *q, const void *c
 int hyena_debug_bounds_check(long long *record);
 
 /*
+ * Test hook (no counterpart in the pages): the next `n` calls of any entry
+ * point that pass argument validation return HYENA_ERR_CUDA without enqueuing
+ * anything, as if their launch had failed; 0 disarms it.  Lets a caller test
+ * its handling of launch failures without a GPU fault (or without a GPU).
+ * HYENA_ERR_ARG for n < 0.  Process-wide; meant for tests only.
+ */
+int hyena_test_fail_next_launches(int n);
+
+/*
  * Test hook (no counterpart in the pages): fault injection for the bounded
  * waits of hyena_prefill_chunked, so that a test can make a wait run out
  * without any GPU fault.  Every later hyena_prefill_chunked launch in the

@@ -225,3 +225,32 @@ def test_prefill_chunked_layers_validation(lib):
     assert lib.hyena_prefill_chunked_layers_workspace_bytes(33, 2, 64, 128, 2, 4) == 0
     assert lib.hyena_prefill_chunked_layers_workspace_bytes(24, 64, 512, 2048, 16, 16) > \
         lib.hyena_prefill_chunked_workspace_bytes(64, 512, 2048, 16, 16)
+
+
+def test_injected_launch_failure_is_reported_before_any_cuda_call(lib):
+    """A launch failure, simulated on the host (no GPU needed): valid calls of several entry points
+    report HYENA_ERR_CUDA while the hook is armed, and nothing is enqueued."""
+    arr = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    calls = [
+        lambda: lib.hyena_decode_step(_p(), _p(), _p(), 1, 2, 8, 2, 4, _p(), _p(), _p(), _p(), _p(), None),
+        lambda: prefill(lib),
+        lambda: lib.hyena_prefill_chunked(_p(), _p(), _p(), 1, 2, 64, 128, 2, 4, _p(), _p(), _p(), _p(), _p(),
+                                          _p(), 1 << 30, None),
+        lambda: lib.hyena_prefill_chunked_layers(2, arr, arr, arr, 1, 2, 64, 128, 2, 4, arr, arr, arr, arr, arr,
+                                                 _p(), 1 << 30, None),
+        lambda: lib.hyena_filter_from_modes(_p(), _p(), _p(), 2, 4, 16, _p(), None),
+        lambda: lib.hyena_decode_step_layers(2, arr, arr, arr, 1, 2, 8, 2, 4, arr, arr, arr, arr, arr, None),
+    ]
+    assert lib.hyena_test_fail_next_launches(-1) == ERR_ARG
+    assert lib.hyena_test_fail_next_launches(len(calls)) == OK
+    try:
+        for c in calls:
+            assert c() == ERR_CUDA
+    finally:
+        lib.hyena_test_fail_next_launches(0)
+    # validation still comes first: an invalid call is reported as such and does not use up the hook
+    assert lib.hyena_test_fail_next_launches(1) == OK
+    try:
+        assert prefill(lib, dtype=7) == ERR_ARG
+    finally:
+        lib.hyena_test_fail_next_launches(0)

@@ -155,3 +155,25 @@ def test_decode_layers_in_bounds(dbg):
         assert rel_err(a.cpu().double().numpy(), b.cpu().double().numpy()) <= 1e-2
     for a, b in zip(st, ref_st):
         assert rel_err(a.cpu().double().numpy(), b.cpu().double().numpy()) <= 1e-5
+
+
+@pytest.mark.parametrize("L", [1, 17, 3000])
+def test_chunked_layers_in_bounds(dbg, oracle, L):
+    """Three layers in one launch (with L = 3000 and one 64-channel head per layer the sequences are
+    split into segments: look-back across the layers' items) in the bounds-checked build."""
+    nl, B, Dch, H, d = 3, 1, 64, 1, 2
+    cases = [_case(B, L, Dch, H, d, "bf16", 200 + 10 * l + L % 7) for l in range(nl)]
+    qkv = [W.prefill_inputs(w) for w, _ in cases]
+    dev = [dev_params(p) for _, p in cases]
+    qs, ks, vs = ([x[j].cuda() for x in qkv] for j in range(3))
+    ys = [torch.empty_like(q) for q in qs]
+    sts = [torch.empty((B, d, Dch, 2), device="cuda") for _ in range(nl)]
+    ls = ops.PrefillLayerSet(qs, ks, vs, ys, sts, [x[0] for x in dev], [x[1] for x in dev], [x[2] for x in dev])
+    ws = ops.prefill_chunked_layers(ls)
+    _clean()
+    assert ls.error(ws) == 0
+    for l, (w, p) in enumerate(cases):
+        qf, kf, vf = (W.to_f64(t) for t in qkv[l])
+        y_ref, s_ref = oracle.recurrent(qf, kf, vf, p.lam, p.R, p.Dskip, H=H)
+        assert rel_err(ys[l].cpu().double().numpy(), y_ref) <= TOL["bf16"]
+        assert rel_err(state_c128(sts[l]), s_ref) <= TOL["bf16"]
