@@ -529,8 +529,9 @@ prefill_chunk_kernel(const __grid_constant__ LayerMaps<LMAX> m, const ChunkArgs 
         for (int i = 0; i < kNumBars; ++i) tc::mbar_init(bar(i), G::count(i));
         tc::fence_mbar_init();
     } else if (tid == 32) {
-        // the maps of the layer of this CTA's first head (fetched on first use for the others)
-        const int l0 = ((int)blockIdx.x % a.H) / a.Hl;
+        // the maps of the layer of this CTA's first item if its ticket is fixed, else of layer 0
+        // (the others are fetched on first use)
+        const int l0 = a.fixed_first ? (ticket_item(a, (int)blockIdx.x) / a.ih) / a.Hl : 0;
         tc::prefetch_tensormap(&m.q[l0]);
         tc::prefetch_tensormap(&m.k[l0]);
         tc::prefetch_tensormap(&m.v[l0]);

@@ -374,3 +374,39 @@ def test_chunked_layers_equal_single_layer_calls_1p3b():
         y1, s1, ws1 = ops.prefill_chunked(*qkv[l], *dev[l])
         assert ops.chunked_error(ws1, w.B, w.L, w.Dch, w.H, w.d) == 0
         assert torch.equal(y1, ys[l]) and torch.equal(s1, sts[l]), l
+
+
+def test_chunked_layers_lookback_timeout_and_empty_prompt():
+    """The grouped launch shares the single-layer error path: with one item's completion word
+    suppressed (test hook, 5 ms bound) a split-sequence launch of two layers ends with error word 2,
+    and the next normal call passes; an empty prompt writes zero states for every layer."""
+    nl, B, L, Dch, H, d = 2, 1, 4096, 64, 1, 8
+    w = W.Workload(711, "layers", B=B, L=L, Dch=Dch, H=H, d=d, dtype="bf16", fft_len=0, T=0)
+    ps = [W.params(w, layer=l) for l in range(nl)]
+    dev = [dev_params(p) for p in ps]
+    g = torch.Generator(device="cuda")
+    g.manual_seed(21)
+    qs, ks, vs = ([torch.randn((B, L, Dch), generator=g, device="cuda").to(torch.bfloat16) for _ in range(nl)]
+                  for _ in range(3))
+    ys = [torch.empty_like(q) for q in qs]
+    sts = [torch.empty((B, d, Dch, 2), device="cuda") for _ in range(nl)]
+    ls = ops.PrefillLayerSet(qs, ks, vs, ys, sts, [x[0] for x in dev], [x[1] for x in dev], [x[2] for x in dev])
+    ops.test_chunked_inject(0, 0.005)
+    try:
+        ws = ops.prefill_chunked_layers(ls)
+        torch.cuda.synchronize()
+    finally:
+        ops.test_chunked_inject(-1, 0.0)
+    assert ls.error(ws) == ERR_LOOKBACK
+    ops.prefill_chunked_layers(ls, workspace=ws)
+    assert ls.error(ws) == 0
+    for l in range(nl):
+        y1, s1, _ = ops.prefill_chunked(qs[l], ks[l], vs[l], *dev[l])
+        assert rel_err(ys[l].cpu().double().numpy(), y1.cpu().double().numpy()) <= Y_MARGIN
+    empty = [torch.empty((B, 0, Dch), dtype=torch.bfloat16, device="cuda") for _ in range(nl)]
+    sts0 = [torch.full((B, d, Dch, 2), 7.0, device="cuda") for _ in range(nl)]
+    ls0 = ops.PrefillLayerSet(empty, empty, empty, empty, sts0, [x[0] for x in dev], [x[1] for x in dev],
+                              [x[2] for x in dev])
+    ops.prefill_chunked_layers(ls0)
+    torch.cuda.synchronize()
+    assert all(torch.all(st == 0) for st in sts0)
