@@ -58,3 +58,32 @@ def test_traffic_figure_is_dropped_once_the_code_changes(tmp_path, monkeypatch):
     _write(tmp_path, "k.cu", KERNEL.replace("2.f", "4.f"))
     assert bench.ncu_traffic("kern", "wl/B1") is None
 
+
+
+def test_both_arms_report_the_same_config():
+    """The reference arm (the oracle) and our arm build the line's config from the same function, for
+    the default workload and the others, so the driver sees the same config on both lines."""
+    import argparse
+    from distilled_ssm_decode_b200 import workloads as W
+    w = W.WORKLOADS[bench.DEFAULT_WORKLOAD]
+    assert bench.DEFAULT_WORKLOAD == "gen1p3b_bf16" and w.layers == 24
+    cfg = bench.line_config(w, w.layers)
+    assert cfg["layers"] == 24 and cfg["B"] == 64 and cfg["L"] == 512 and cfg["Dch"] == 2048
+    assert "24 independent layers" in cfg["workload"]
+    for name, wl in W.WORKLOADS.items():
+        assert bench.line_config(wl, wl.layers) == bench.line_config(wl, wl.layers)
+    src = open(os.path.join(ROOT, "bench.py")).read()
+    # both arms print config=line_config(w, nl) and nothing else under "config"
+    assert src.count('"config": line_config(w, nl)') == 2
+
+
+def test_algorithmic_bytes_match_the_documented_figures():
+    from distilled_ssm_decode_b200 import workloads as W
+    pre, dec = bench.algorithmic_bytes(W.WORKLOADS["mid_bf16"])
+    assert pre == 269_484_032 and dec == 2_162_688
+    pre, dec = bench.algorithmic_bytes(W.WORKLOADS["gen1p3b_bf16"])
+    assert pre * 24 == 13_287_555_072 and dec * 24 == 830_472_192
+    pre, _ = bench.algorithmic_bytes(W.WORKLOADS["long_prefill_bf16"])
+    assert pre == 402_751_488
+    _, dec = bench.algorithmic_bytes(W.WORKLOADS["decode_sweep_bf16"].with_(B=1024))
+    assert dec == 1_107_296_256
