@@ -3,11 +3,12 @@
 
 Default line: the 1.3B-shaped generation workload, 24 independent operator layers, each
 B=64, L=512, Dch=2048, H=16, d=16, bf16 activations, complex fp32 state.  One step = the
-chunked tensor-core prefill of every layer's 512-token prompt, then 512 decode tokens, each
-one grouped decode launch over all 24 layers (replayed from a CUDA graph).  The same run
-adds sub-records, each timed on its own: the mid-size operator (prefill and decode), the
-long prefill (65536 tokens, with its end-to-end time) and the decode batch sweep at
-B = 1, 16, 64, 256 and 1024.  Every sub-record carries its roofline entries.
+chunked tensor-core prefill of every layer's 512-token prompt (one launch), then 512 decode
+tokens, each one grouped decode launch over all 24 layers (replayed from a CUDA graph).  The
+same run adds sub-records, each timed on its own: the tiny fp32 operator (FFT prefill and 32
+decode steps), the mid-size operator (prefill and decode), the long prefill (65536 tokens,
+with its end-to-end time) and the decode batch sweep at B = 1, 16, 64, 256 and 1024.  Every
+sub-record carries its roofline entries.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--no-subrecords] ...
@@ -870,6 +871,7 @@ def measure_layers(args, w, nl: int, dev, steps: int, warmup: int, e2e_steps: in
 # ------------------------------------------------------------------ our arm
 SUBRECORDS = [
     # (name, workload, batch override, steps, e2e, fft route, baselines)
+    ("tiny_f32", "tiny_f32", 0, None, True, False, False),
     ("mid_bf16", "mid_bf16", 0, None, True, True, True),
     ("long_prefill_bf16", "long_prefill_bf16", 0, None, True, True, False),
     ("decode_sweep_bf16/B1", "decode_sweep_bf16", 1, 5, False, False, False),
