@@ -183,8 +183,10 @@ int hyena_prefill_noalloc(const void *q, const void *k, const void *v, int dtype
  * convolution; the carry is the distilled recurrence of "Laughing Hyena
  * Distillery", "Main findings".)  The products take bf16 operands (u = k v,
  * the taps, the powers and the state rounded to bf16) with fp32 accumulation;
- * the state chain itself runs in fp32.  Chunks are aligned to the end of the
- * prompt, so the last one ends at token L-1.
+ * the state chain itself runs in fp32.  Measured against an fp64 evaluation on
+ * the library's test shapes: y within 6.5e-3 of max|y| (hyena_prefill: 3.3e-3,
+ * its bf16 output rounding), the prompt state within 4e-3 of its maximum.
+ * Chunks are aligned to the end of the prompt, so the last one ends at token L-1.
  *   Arguments as hyena_prefill, without fft_len.
  *   Implemented for: dtype HYENA_BF16, Dch/H a multiple of 64, d <= 16, all
  *   activation pointers 16-byte aligned; HYENA_ERR_UNSUPPORTED otherwise.
