@@ -33,7 +33,8 @@ using fft::padded_len;
 namespace {
 
 constexpr int kFusedThreads = 256;
-constexpr int kFusedMinBlocks = 3;   // three CTAs per SM: one loads while others compute
+constexpr int kFusedMinBlocks = 2;   // two CTAs per SM: one loads while the other computes; the
+                                      // 128-register cap keeps the radix-16 passes' loads in flight
 
 int fused_threads(int N) {
     int t = N / 32;
