@@ -43,8 +43,9 @@ int check_common(int H, int d, int Dch) {
 }
 
 // Prefill workspace layout: [h: H*L f32][spectra: H*N c64][four-step planes][state partials]
+// [error word of the tensor-core route]
 struct PrefillWs {
-    size_t h_off, spec_off, four_off, state_off, total;
+    size_t h_off, spec_off, four_off, state_off, err_off, total;
 };
 
 PrefillWs prefill_ws(int B, int L, int Dch, int H, int d, int fft_len) {
@@ -55,7 +56,8 @@ PrefillWs prefill_ws(int B, int L, int Dch, int H, int d, int fft_len) {
     w.spec_off = align_up((size_t)H * L * sizeof(float));
     w.four_off = w.spec_off + align_up(spectrum_ws_bytes(H, N));
     w.state_off = w.four_off + align_up(fourstep_ws_bytes(B, Dch, ch, N));
-    w.total = w.state_off + (N > kFusedMaxN ? align_up(state_ws_bytes(B, L, Dch, d)) : 0);
+    w.err_off = w.state_off + (N > kFusedMaxN ? align_up(state_ws_bytes(B, L, Dch, d)) : 0);
+    w.total = w.err_off + kAlign;
     return w;
 }
 
@@ -160,15 +162,36 @@ int hyena_prefill(const void *q, const void *k, const void *v, int dtype, int B,
     float2 *spec = reinterpret_cast<float2 *>(ws + w.spec_off);
     const int N = fft_internal_len(fft_len);
     const float2 *lam2 = reinterpret_cast<const float2 *>(lambda);
+    int *err = reinterpret_cast<int *>(ws + w.err_off);
     HYENA_LAUNCH_GUARD();
-    cudaError_t e = launch_filter(lam2, reinterpret_cast<const float2 *>(R), Dskip, H, d, L, h, s);
+    // the filter kernel also clears the error word
+    cudaError_t e = launch_filter(lam2, reinterpret_cast<const float2 *>(R), Dskip, H, d, L, h, s, err);
     if (e != cudaSuccess) return HYENA_ERR_CUDA;
     // the inverse transform is unnormalised: fold its 1/N into the spectrum
+    const int r3 = monarch_r3(dtype, B, L, Dch, H, N, q, k, v, y);
+    if (r3) {
+        // tensor-core route: spectrum in its frequency order
+        e = launch_spectrum_monarch(h, H, L, N, spec, 1.0f / (float)N, s);
+        if (e != cudaSuccess) return HYENA_ERR_CUDA;
+        return cuda_status(launch_prefill_monarch(r3, q, k, v, B, L, Dch, H, d, spec, lam2, y, state_out,
+                                                  err, s));
+    }
     e = launch_spectrum_perm(h, H, L, N, spec, 1.0f / (float)N, s);
     if (e != cudaSuccess) return HYENA_ERR_CUDA;
     e = launch_prefill_fft(q, k, v, dtype, B, L, Dch, H, d, N, spec, lam2, y, state_out,
-                           ws + w.four_off, w.total - w.four_off, s);
+                           ws + w.four_off, w.err_off - w.four_off, s);
     return cuda_status(e);
+}
+
+size_t hyena_prefill_error_offset(int B, int L, int Dch, int H, int d, int fft_len) {
+    if (check_prefill_shape(B, L, Dch, H, d, fft_len) != HYENA_OK) return 0;
+    return prefill_ws(B, L, Dch, H, d, fft_len).err_off;
+}
+
+int hyena_test_fft_tensor_cores(int enable) {
+    if (enable != 0 && enable != 1) return HYENA_ERR_ARG;
+    monarch_enable(enable);
+    return HYENA_OK;
 }
 
 static int check_chunked(int dtype, int B, int L, int Dch, int H, int d) {
@@ -221,9 +244,10 @@ int hyena_debug_bounds_check(long long *record) {
     // file ids as documented in hyena.h
     int (*const readers[])(long long *) = {bounds_read_decode, bounds_read_filter, bounds_read_fir,
                                            bounds_read_prefill_chunked, bounds_read_prefill_fft,
-                                           bounds_read_state, bounds_read_truncate};
+                                           bounds_read_state, bounds_read_truncate,
+                                           bounds_read_prefill_monarch};
     int found = 0;
-    for (int f = 0; f < 7; ++f) {
+    for (int f = 0; f < 8; ++f) {
         long long rec[4];
         const int r = readers[f](rec);      // every record is read (and cleared), the first one kept
         if (r < 0) return HYENA_ERR_CUDA;

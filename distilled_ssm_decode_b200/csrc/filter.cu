@@ -19,8 +19,9 @@ constexpr int kRun = 16;
 
 __global__ void __launch_bounds__(128)
 filter_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R,
-              const float *__restrict__ Dskip, int d, int L, float *__restrict__ h) {
+              const float *__restrict__ Dskip, int d, int L, float *__restrict__ h, int *clear) {
     const int hd = blockIdx.y, H = gridDim.y;
+    if (clear && hd == 0 && blockIdx.x == 0 && threadIdx.x == 0) *clear = 0;
     (void)H;
     const long long j0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * kRun;
     if (j0 >= L) return;
@@ -55,12 +56,12 @@ filter_kernel(const float2 *__restrict__ lam, const float2 *__restrict__ R,
 HYENA_BOUNDS_READER(filter)
 
 cudaError_t launch_filter(const float2 *lam, const float2 *R, const float *Dskip,
-                          int H, int d, int L, float *h, cudaStream_t s) {
+                          int H, int d, int L, float *h, cudaStream_t s, int *clear) {
     if (H == 0 || L == 0) return cudaSuccess;
     const int threads = 128;
     const long long runs = (L + kRun - 1) / kRun;
     dim3 grid((unsigned)((runs + threads - 1) / threads), (unsigned)H);
-    filter_kernel<<<grid, threads, 0, s>>>(lam, R, Dskip, d, L, h);
+    filter_kernel<<<grid, threads, 0, s>>>(lam, R, Dskip, d, L, h, clear);
     return cudaGetLastError();
 }
 

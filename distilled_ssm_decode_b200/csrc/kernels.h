@@ -18,8 +18,9 @@ constexpr int kMinFFT = 64;
 inline int fft_internal_len(int fft_len) { return fft_len < kMinFFT ? kMinFFT : fft_len; }
 
 // filter.cu
+// (block 0 also clears *clear when it is given)
 cudaError_t launch_filter(const float2 *lam, const float2 *R, const float *Dskip,
-                          int H, int d, int L, float *h, cudaStream_t s);
+                          int H, int d, int L, float *h, cudaStream_t s, int *clear = nullptr);
 
 // prefill_fft.cu
 size_t spectrum_ws_bytes(int H, int N);               // digit-reversed spectra (+ four-step scratch)
@@ -34,6 +35,20 @@ cudaError_t launch_prefill_fft(const void *q, const void *k, const void *v, int 
                                const float2 *spec_perm, const float2 *lam,
                                void *y, float *state_out, void *scratch, size_t scratch_bytes,
                                cudaStream_t s);
+
+// spectrum for the tensor-core route: frequency k = k1 + 64 k2 + 4096 k3 stored at
+// [k2][k1][k3] per head (N = 4096, 8192 or 16384)
+cudaError_t launch_spectrum_monarch(const float *h, int H, int L, int N, float2 *spec, float scale,
+                                    cudaStream_t s);
+
+// prefill_monarch.cu (FFT route on the tensor cores; bf16 activations)
+// R3 = N / 4096 when the tensor-core route takes this call, else 0 (the CUDA-core route)
+int monarch_r3(int dtype, int B, int L, int Dch, int H, int N, const void *q, const void *k, const void *v,
+               const void *y);
+void monarch_enable(int enable);
+cudaError_t launch_prefill_monarch(int r3, const void *q, const void *k, const void *v, int B, int L, int Dch,
+                                   int H, int d, const float2 *spec, const float2 *lam, void *y,
+                                   float *state_out, int *err, cudaStream_t s);
 
 // prefill_chunked.cu (bf16 activations, heads of a multiple of 64 channels, d <= 16)
 bool chunked_supported(int dtype, int Dch, int H, int d);
@@ -87,6 +102,7 @@ int bounds_read_filter(long long *rec);
 int bounds_read_fir(long long *rec);
 int bounds_read_prefill_chunked(long long *rec);
 int bounds_read_prefill_fft(long long *rec);
+int bounds_read_prefill_monarch(long long *rec);
 int bounds_read_state(long long *rec);
 int bounds_read_truncate(long long *rec);
 

@@ -45,10 +45,12 @@ int fused_threads(int N) {
 
 // ------------------------------------------------------------------ spectrum
 // One CTA per head: forward transform of the zero-padded filter, times scale,
-// stored in the transform's digit-reversed order.
+// stored in the transform's digit-reversed order (mon_r3 == 0), or, for the
+// tensor-core route, at frequency k = k1 + 64 k2 + 4096 k3 in the order
+// [k2][k1][k3] (mon_r3 = N / 4096).
 __global__ void __launch_bounds__(kFusedThreads)
 spectrum_fused_kernel(const float *__restrict__ h, int L, int N, float scale,
-                      float2 *__restrict__ spec_perm) {
+                      float2 *__restrict__ spec_perm, int mon_r3) {
     extern __shared__ float2 buf[];
     const int hd = blockIdx.x, H = gridDim.x;
     (void)H;
@@ -60,8 +62,14 @@ spectrum_fused_kernel(const float *__restrict__ h, int L, int N, float scale,
     __syncthreads();
     fft::forward(buf, N, half_zero);
     float2 *out = spec_perm + (size_t)hd * N;
-    for (int p = threadIdx.x; p < N; p += blockDim.x)
-        if (HB_OK((long long)hd * N + p, (long long)H * N)) out[p] = cscale(buf[pad(p)], scale);
+    for (int p = threadIdx.x; p < N; p += blockDim.x) {
+        int o = p;
+        if (mon_r3) {
+            const int f = fft::freq_of_pos(p, N);
+            o = (((f >> 6) & 63) * 64 + (f & 63)) * mon_r3 + (f >> 12);
+        }
+        if (HB_OK((long long)hd * N + o, (long long)H * N)) out[o] = cscale(buf[pad(p)], scale);
+    }
 }
 
 // natural-order bins 0..N/2 from the digit-reversed layout
@@ -408,7 +416,7 @@ cudaError_t launch_spectrum_perm(const float *h, int H, int L, int N, float2 *sp
         const size_t smem = inner_smem_bytes(N);
         cudaError_t e = set_smem((const void *)spectrum_fused_kernel, smem);
         if (e != cudaSuccess) return e;
-        spectrum_fused_kernel<<<H, fused_threads(N), smem, s>>>(h, L, N, scale, spec_perm);
+        spectrum_fused_kernel<<<H, fused_threads(N), smem, s>>>(h, L, N, scale, spec_perm, 0);
         return cudaGetLastError();
     }
     const int N2 = kFourStepN2, N1 = N / N2;
@@ -419,6 +427,17 @@ cudaError_t launch_spectrum_perm(const float *h, int H, int L, int N, float2 *sp
     if (e != cudaSuccess) return e;
     fourstep_inner_kernel<<<dim3(N1, H), kFusedThreads, smem, s>>>(spec_perm, N1, N2, 0, scale,
                                                                   nullptr, 1, 0, 1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_spectrum_monarch(const float *h, int H, int L, int N, float2 *spec, float scale,
+                                    cudaStream_t s) {
+    if (H == 0) return cudaSuccess;
+    if (N != 4096 && N != 8192 && N != 16384) return cudaErrorInvalidValue;
+    const size_t smem = inner_smem_bytes(N);
+    cudaError_t e = set_smem((const void *)spectrum_fused_kernel, smem);
+    if (e != cudaSuccess) return e;
+    spectrum_fused_kernel<<<H, fused_threads(N), smem, s>>>(h, L, N, scale, spec, N / 4096);
     return cudaGetLastError();
 }
 

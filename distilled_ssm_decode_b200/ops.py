@@ -33,6 +33,7 @@ SIGNATURES = {
     "hyena_filter_spectrum_workspace_bytes": (_sz, [_i, _i, _i]),
     "hyena_filter_spectrum": (_i, [_fp, _i, _i, _i, _fp, _vp, _sz, _vp]),
     "hyena_prefill_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "hyena_prefill_error_offset": (_sz, [_i, _i, _i, _i, _i, _i]),
     "hyena_prefill": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp, _fp,
                            _vp, _sz, _vp]),
     "hyena_prefill_chunked_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
@@ -48,6 +49,7 @@ SIGNATURES = {
                                    _vp]),
     "hyena_test_chunked_inject": (_i, [_i, ctypes.c_double]),
     "hyena_test_fail_next_launches": (_i, [_i]),
+    "hyena_test_fft_tensor_cores": (_i, [_i]),
     "hyena_debug_bounds_check": (_i, [_vp]),
     "hyena_prompt_state_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "hyena_prompt_state": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _fp, _fp, _vp, _sz, _vp]),
@@ -291,6 +293,25 @@ def chunked_error(workspace, B, L, Dch, H, d) -> int:
     """The kernel's error word (synchronises): 0 when every bounded wait succeeded."""
     off = int(lib().hyena_prefill_chunked_error_offset(B, L, Dch, H, d))
     return int(workspace[off:off + 4].view(torch.int32).item())
+
+
+def prefill_error(workspace, B, L, Dch, H, d, fft_len) -> int:
+    """Error word of the FFT prefill's tensor-core route (synchronises): 0 when its bounded
+    waits all succeeded (and always 0 after a call that took the CUDA-core route)."""
+    off = int(lib().hyena_prefill_error_offset(B, L, Dch, H, d, fft_len))
+    return int(workspace[off:off + 4].view(torch.int32).item())
+
+
+@contextlib.contextmanager
+def fft_tensor_cores(enable: bool):
+    """Test hook: inside the block every FFT prefill call runs its transforms on the tensor
+    cores where that route applies (enable=True, the default outside) or on the CUDA cores
+    only (enable=False)."""
+    _check("hyena_test_fft_tensor_cores", lib().hyena_test_fft_tensor_cores(1 if enable else 0))
+    try:
+        yield
+    finally:
+        _check("hyena_test_fft_tensor_cores", lib().hyena_test_fft_tensor_cores(1))
 
 
 def test_chunked_inject(suppress_item: int = -1, lookback_limit_s: float = 0.0):

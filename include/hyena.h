@@ -131,8 +131,23 @@ int hyena_filter_spectrum(const float *h, int H, int L, int fft_len, float *spec
  *   workspace  : device scratch, >= hyena_prefill_workspace_bytes(...) bytes,
  *                256-byte aligned; contents on entry are ignored.
  * Alignment: all activation pointers 4-byte aligned (bf16) / 8-byte (f32).
+ * Routes.  bf16 activations with an internal FFT length of 4096, 8192 or 16384,
+ * an even number of channels per head, Dch a multiple of 8 (of 4 at 16384)
+ * and q, k, v, y aligned to 16 bytes (8 at 16384) run on the tensor cores: each
+ * transform is factored as 64 x 64 x (N/4096) and its two 64-point DFT stages
+ * are dense matrix products (a Monarch-style factorisation; bf16 operands,
+ * fp32 accumulation, twiddles and the spectral product in fp32).  Measured on
+ * the library's test shapes: y within about 5e-3 of max|y| (the bar for bf16
+ * activations is 2e-2); the state is summed in fp32 from fp32 u over the last
+ * 1024 prompt tokens and from bf16-rounded u before them.  Every other call
+ * (fp32 activations, other lengths or layouts) runs the transforms on the CUDA
+ * cores in fp32.  The tensor-core route waits on its own products with bounded
+ * waits; if one gives up, the int at hyena_prefill_error_offset(...) bytes into
+ * the workspace is nonzero after the call and y and state_out are not valid
+ * (every call with L > 0 clears it first, whichever route it takes).
  */
 size_t hyena_prefill_workspace_bytes(int B, int L, int Dch, int H, int d, int fft_len);
+size_t hyena_prefill_error_offset(int B, int L, int Dch, int H, int d, int fft_len);
 int hyena_prefill(const void *q, const void *k, const void *v, int dtype,
                   int B, int L, int Dch, int H, int d, int fft_len,
                   const float *lambda, const float *R, const float *Dskip,
@@ -247,7 +262,7 @@ int hyena_prefill_chunked_layers(int layers, const void *const *q, const void *c
  * and clears the records.  Returns 0 when no access was out of range, 1 when
  * one was, with record = {file, source line, index, extent} (file: 1 decode.cu,
  * 2 filter.cu, 3 fir.cu, 4 prefill_chunked.cu, 5 prefill_fft.cu, 6 state.cu,
- * 7 truncate.cu); HYENA_ERR_UNSUPPORTED from the release build, which has no
+ * 7 truncate.cu, 8 prefill_monarch.cu); HYENA_ERR_UNSUPPORTED from the release build, which has no
  * checks; HYENA_ERR_ARG for a NULL record.
  */
 int hyena_debug_bounds_check(long long *record);
@@ -274,6 +289,16 @@ int hyena_test_fail_next_launches(int n);
  * concurrent launches; meant for tests only.
  */
 int hyena_test_chunked_inject(int suppress_item, double lookback_limit_s);
+
+/*
+ * Test hook (no counterpart in the pages): enable = 0 makes every later
+ * hyena_prefill / hyena_prefill_noalloc call run its transforms on the CUDA
+ * cores, also where the tensor-core route would apply (so that both routes
+ * can be tested and timed on the same inputs); 1 (the default) restores the
+ * automatic choice.  HYENA_ERR_ARG for other values.  Process-wide; meant for
+ * tests and benchmarks only.
+ */
+int hyena_test_fft_tensor_cores(int enable);
 
 /*
  * Prompt -> state reduction alone (the Vandermonde contraction over the

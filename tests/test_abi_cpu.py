@@ -211,6 +211,17 @@ def test_fault_injection_hook_validates_its_arguments(lib):
     assert lib.hyena_test_chunked_inject(-1, 0.0) == OK
 
 
+def test_fft_route_hook_and_error_offset(lib):
+    assert lib.hyena_test_fft_tensor_cores(2) == ERR_ARG
+    assert lib.hyena_test_fft_tensor_cores(-1) == ERR_ARG
+    assert lib.hyena_test_fft_tensor_cores(0) == OK
+    assert lib.hyena_test_fft_tensor_cores(1) == OK
+    ws = lib.hyena_prefill_workspace_bytes(8, 4096, 1024, 8, 16, 8192)
+    off = lib.hyena_prefill_error_offset(8, 4096, 1024, 8, 16, 8192)
+    assert 0 < off and off + 4 <= ws and off % 4 == 0
+    assert lib.hyena_prefill_error_offset(8, 4096, 1024, 8, 16, 4096) == 0    # fft_len < 2L-1
+
+
 def test_prefill_chunked_layers_validation(lib):
     arr = (ctypes.c_void_p * 1)(FAKE)
     call = lambda layers, dtype=1, B=2, L=64, Dch=128, H=2, d=4, ws=1 << 30: lib.hyena_prefill_chunked_layers(
