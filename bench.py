@@ -454,6 +454,12 @@ def measure_single(args, w, dev, steps: int, warmup: int, e2e_steps: int, with_f
     def prefill_fft():
         ops.prefill(q, k, v, lam, R, D, w.fft_len, y=y, state=state, workspace=ws)
 
+    # which FFT route the library takes for these tensors (tensor cores for bf16 at 4096..16384)
+    fft_tc = has_pre and ops.prefill_uses_tensor_cores(q, k, v, w.H, w.d, w.fft_len, y=y)
+    fft_label = ("hyena_prefill (filter + spectrum + tensor-core FFT conv/gate/state)" if fft_tc
+                 else "hyena_prefill (filter + spectrum + fused FFT conv/gate/state)")
+    fft_kernel = "prefill_monarch" if fft_tc else "prefill_fused"
+
     def prefill_chunked():
         ops.prefill_chunked(q, k, v, lam, R, D, y=y, state=state, workspace=ws_c)
 
@@ -498,12 +504,11 @@ def measure_single(args, w, dev, steps: int, warmup: int, e2e_steps: int, with_f
            "value": world * w.B * (w.L + w.T) / (ms_per_step / 1e3), "unit": "tokens/s"}
     roofs = []
     if has_pre:
-        name = ("hyena_prefill_chunked (tcgen05 chunked conv/gate/state)" if use_chunked
-                else "hyena_prefill (filter + spectrum + fused FFT conv/gate/state)")
+        name = "hyena_prefill_chunked (tcgen05 chunked conv/gate/state)" if use_chunked else fft_label
         r = roof(name, pb, pre_ms, peak, peak_src,
-                 ncu_traffic("prefill_chunk" if use_chunked else "prefill_fused", key))
+                 ncu_traffic("prefill_chunk" if use_chunked else fft_kernel, key))
         roofs.append(r)
-        rec["prefill"] = {"route": "chunked" if use_chunked else "fft",
+        rec["prefill"] = {"route": "chunked" if use_chunked else ("fft, tensor cores" if fft_tc else "fft"),
                           "tokens_per_s": world * w.B * w.L / (pre_ms / 1e3), "ms": pre_ms,
                           "hbm_frac": r["frac"], "roofline": r,
                           "inputs": "q, k, v of %d MiB each (larger than L2)" % (w.B * w.L * w.Dch * w.act_bytes >> 20)}
@@ -533,9 +538,9 @@ def measure_single(args, w, dev, steps: int, warmup: int, e2e_steps: int, with_f
             if ev is not None:
                 ev[1].record(stream)
         _, (fms,) = timed_steps(stream, dev, steps, 3, fstep, 1)
-        r = roof("hyena_prefill (filter + spectrum + fused FFT conv/gate/state)", pb, fms, peak, peak_src,
-                 ncu_traffic("prefill_fused", key))
-        rec["prefill_fft_route"] = {"fft_len": w.fft_len, "tokens_per_s": world * w.B * w.L / (fms / 1e3),
+        r = roof(fft_label, pb, fms, peak, peak_src, ncu_traffic(fft_kernel, key))
+        rec["prefill_fft_route"] = {"fft_len": w.fft_len, "tensor_cores": bool(fft_tc),
+                                    "tokens_per_s": world * w.B * w.L / (fms / 1e3),
                                     "ms": fms, "hbm_frac": r["frac"], "roofline": r}
     rec["roofline_all"] = roofs
     rec["roofline"] = max(roofs, key=lambda x: x["total_ms"])

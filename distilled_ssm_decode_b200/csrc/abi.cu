@@ -183,6 +183,14 @@ int hyena_prefill(const void *q, const void *k, const void *v, int dtype, int B,
     return cuda_status(e);
 }
 
+int hyena_prefill_uses_tensor_cores(int dtype, int B, int L, int Dch, int H, int d, int fft_len,
+                                    const void *q, const void *k, const void *v, const void *y) {
+    if (dtype != HYENA_F32 && dtype != HYENA_BF16) return HYENA_ERR_ARG;
+    const int st = check_prefill_shape(B, L, Dch, H, d, fft_len);
+    if (st != HYENA_OK) return st;
+    return monarch_r3(dtype, B, L, Dch, H, fft_internal_len(fft_len), q, k, v, y) != 0 ? 1 : 0;
+}
+
 size_t hyena_prefill_error_offset(int B, int L, int Dch, int H, int d, int fft_len) {
     if (check_prefill_shape(B, L, Dch, H, d, fft_len) != HYENA_OK) return 0;
     return prefill_ws(B, L, Dch, H, d, fft_len).err_off;

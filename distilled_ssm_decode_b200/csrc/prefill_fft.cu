@@ -47,7 +47,7 @@ int fused_threads(int N) {
 // One CTA per head: forward transform of the zero-padded filter, times scale,
 // stored in the transform's digit-reversed order (mon_r3 == 0), or, for the
 // tensor-core route, at frequency k = k1 + 64 k2 + 4096 k3 in the order
-// [k2][k1][k3] (mon_r3 = N / 4096).
+// [k2][k1 % 2][k1 / 2][k3] (mon_r3 = N / 4096).
 __global__ void __launch_bounds__(kFusedThreads)
 spectrum_fused_kernel(const float *__restrict__ h, int L, int N, float scale,
                       float2 *__restrict__ spec_perm, int mon_r3) {
@@ -66,7 +66,7 @@ spectrum_fused_kernel(const float *__restrict__ h, int L, int N, float scale,
         int o = p;
         if (mon_r3) {
             const int f = fft::freq_of_pos(p, N);
-            o = (((f >> 6) & 63) * 64 + (f & 63)) * mon_r3 + (f >> 12);
+            o = ((((f >> 6) & 63) * 2 + (f & 1)) * 32 + ((f & 63) >> 1)) * mon_r3 + (f >> 12);
         }
         if (HB_OK((long long)hd * N + o, (long long)H * N)) out[o] = cscale(buf[pad(p)], scale);
     }

@@ -77,7 +77,8 @@ struct Mon {
     static constexpr int kSmB = 128 * 128 * 2;   // P B operands (also the gate-out staging)
     static constexpr int kSmU = kSmB + P * kBop; // [G][kUWin] fp32
     static constexpr int kSmBar = kSmU + G * kUWin * 4;
-    static constexpr int kSmBytes = kSmBar + 64;
+    static constexpr int kSmBytes = kSmBar + 64;   // P barriers, tensor-memory slot, abort, P windows
+    static_assert(8 * P + 8 + 4 * P <= 64, "control block");
     static constexpr int kTmemCols = P * C;
     static_assert(kTmemCols == 256 || kTmemCols == 512, "tensor memory allocation");
     static_assert(kSmB % 1024 == 0 && kBop % 1024 == 0, "swizzle atoms are 1024-byte aligned");
@@ -122,6 +123,17 @@ __device__ __forceinline__ void small_dft(float2 *x) {
     else if constexpr (R == 4) fft::dft4<INV>(x[0], x[1], x[2], x[3]);
 }
 
+// Trailing prompt tokens the state needs, from r2 = max_n |lambda_n|^2 of a head (the rule of
+// state_window: the older tokens weigh at most 2^-40 max|u|).
+__device__ __forceinline__ int window_of(float r2, int L) {
+    if (r2 == 0.f) return L < 1 ? L : 1;
+    if (r2 >= 1.f) return L;
+    const double r = sqrt((double)r2);
+    const double m = (-40.0 * 0.69314718055994530942 + log1p(-r)) / log(r);
+    if (!(m < (double)L)) return L;
+    return (int)ceil(m) + 1;
+}
+
 __device__ __forceinline__ void wg_sync(int p) {
     asm volatile("bar.sync %0, 128;" ::"r"(p + 1) : "memory");
 }
@@ -142,6 +154,7 @@ prefill_monarch_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 
     uint64_t *bars = reinterpret_cast<uint64_t *>(sp + M::kSmBar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sp + M::kSmBar + 8 * P);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sp + M::kSmBar + 8 * P + 4);
+    int *wwin = reinterpret_cast<int *>(sp + M::kSmBar + 8 * P + 8);     // [P] state windows
     float *us = reinterpret_cast<float *>(sp + M::kSmU);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -224,6 +237,7 @@ prefill_monarch_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 
         const int b = (int)(grp / ngc), c0 = (int)(grp % ngc) * G;
 
         // ---- 1. gate-in (CTA-wide): u = k v for the G channels, rows of 8 tokens per thread
+        //      (each row is G * 2 bytes of a token's channels: loaded through L2 only)
         for (int it = tid; it < N / 16; it += blockDim.x) {
             const int t0 = it * 8;
             RowT kr[8], vr[8];
@@ -232,8 +246,8 @@ prefill_monarch_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 
                 const int t = t0 + s;
                 const long long o = ((long long)b * L + t) * Dch + c0;
                 if (t < L && HB_OK(o + G - 1, n_act)) {
-                    kr[s] = __ldg(reinterpret_cast<const RowT *>(k + o));
-                    vr[s] = __ldg(reinterpret_cast<const RowT *>(v + o));
+                    kr[s] = __ldcg(reinterpret_cast<const RowT *>(k + o));
+                    vr[s] = __ldcg(reinterpret_cast<const RowT *>(v + o));
                 } else {
                     kr[s] = RowT{};
                     vr[s] = RowT{};
@@ -257,6 +271,18 @@ prefill_monarch_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 
                 *reinterpret_cast<uint4 *>(sp + M::kSmB + (chl >> 1) * M::kBop + bop_off(row, j0)) = pk;
             }
         }
+        // the state window of each pair's head (the rule of state_window), one warp per pair
+        if (warp < P) {
+            const float2 *lw = lam + (size_t)HB_IDX((c0 + 2 * warp) / ch, H) * d;
+            float r2 = 0.f;
+            for (int n = lane; n < d; n += 32) {
+                const float2 l = __ldg(&lw[n]);
+                r2 = fmaxf(r2, l.x * l.x + l.y * l.y);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) r2 = fmaxf(r2, __shfl_xor_sync(0xffffffffu, r2, off));
+            if (lane == 0) wwin[warp] = window_of(r2, L);
+        }
         tc::fence_proxy_async_smem();
         __syncthreads();
 
@@ -268,7 +294,7 @@ prefill_monarch_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 
         // prompt -> state reduction for the pair while the product runs
         {
             const float2 *lh = lam + (size_t)HB_IDX(hd, H) * d;
-            const int W = state_window(lh, d, L);
+            const int W = wwin[p];
             const int jstart = L - W;
             int nseg = 1;
             while (nseg * 2 * 2 * d <= 128 && nseg < 32) nseg *= 2;
@@ -281,12 +307,48 @@ prefill_monarch_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 
                 const int seglen = (W + nseg - 1) / nseg;
                 const int j0 = jstart + g * seglen;
                 const int j1 = min(L, j0 + seglen);
+                auto u_at = [&](int t) -> float {
+                    if (t >= L - Wf) return us[(2 * p + cc) * M::kUWin + (t - (L - Wf))];
+                    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(bop + bop_off(kappa(t / C, cc), t % C)));
+                };
+                // Horner over blocks of 8 tokens: acc <- acc lambda^8 + sum_i lambda^(7-i) u(t+i)
+                float2 lp[8];
+                lp[0] = make_float2(1.f, 0.f);
+#pragma unroll
+                for (int i = 1; i < 8; ++i) lp[i] = cmul(lp[i - 1], l);
+                const float2 l8 = cmul(lp[7], l);
                 float2 aa = make_float2(0.f, 0.f);
-                for (int t = j0; t < j1; ++t) {
-                    float x;
-                    if (t >= L - Wf) x = us[(2 * p + cc) * M::kUWin + (t - (L - Wf))];
-                    else x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(bop + bop_off(kappa(t / C, cc), t % C)));
+                const int cnt = j1 > j0 ? j1 - j0 : 0;   // the last segments can be empty
+                int t = j0;
+                for (; t < j0 + (cnt & 7); ++t) {
+                    const float x = u_at(t);
                     aa = make_float2(fmaf(aa.x, l.x, fmaf(-aa.y, l.y, x)), fmaf(aa.x, l.y, aa.y * l.x));
+                }
+                if (t >= L - Wf) {
+                    // the whole rest of the segment has fp32 u: straight reads, no per-token test
+                    const float *ur = us + (2 * p + cc) * M::kUWin + (t - (L - Wf));
+                    for (; t < j0 + cnt; t += 8, ur += 8) {
+                        float x[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) x[i] = ur[i];
+                        float bx = 0.f, by = 0.f;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            bx = fmaf(lp[7 - i].x, x[i], bx);
+                            by = fmaf(lp[7 - i].y, x[i], by);
+                        }
+                        aa = make_float2(fmaf(aa.x, l8.x, fmaf(-aa.y, l8.y, bx)), fmaf(aa.x, l8.y, fmaf(aa.y, l8.x, by)));
+                    }
+                }
+                for (; t < j0 + cnt; t += 8) {
+                    float bx = 0.f, by = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float x = u_at(t + i);
+                        bx = fmaf(lp[7 - i].x, x, bx);
+                        by = fmaf(lp[7 - i].y, x, by);
+                    }
+                    aa = make_float2(fmaf(aa.x, l8.x, fmaf(-aa.y, l8.y, bx)), fmaf(aa.x, l8.y, fmaf(aa.y, l8.x, by)));
                 }
                 if (j1 > j0) {
                     const cd pw = cdpow(cd{l.x, l.y}, (long long)(L - j1));
@@ -336,51 +398,77 @@ prefill_monarch_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 
                 }
             }
         }
+        // the spectrum of this row's first two T2 chunks, loaded while stage B runs: row (k2, c)
+        // reads the k1 with k1 % 2 == c, stored contiguously ([k2][k1 % 2][k1 / 2][k3])
+        const float4 *hrow4 = reinterpret_cast<const float4 *>(
+            spec + ((size_t)HB_IDX(hd, H) * N + (size_t)((r >> 1) * 2 + c) * 32 * R3));
+        float4 ha[4], hb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            ha[i] = __ldg(&hrow4[i]);
+            hb[i] = __ldg(&hrow4[4 + i]);
+        }
         step_done();
         if (issuer) issue(8);                         // stage B
         wait_product();
 
         // T2: rows (k2, c), columns R3 k1 + n3: twiddle, R3-point DFT, spectrum, inverse
-        //     R3-point DFT, conjugate twiddle; conj(Z) to K-row kappa(k2, c), same columns
+        //     R3-point DFT, conjugate twiddle; conj(Z) to K-row kappa(k2, c), same columns.
+        //     The two lanes of a row pair split the work: lane c computes the complex chain of
+        //     the k1 with k1 % 2 == c (one shuffle brings in the other part of its inputs, one
+        //     more hands back the partner's part of its outputs), and loads only those k1's
+        //     spectrum (8 values per 16-column chunk), two chunks ahead.
         {
+            constexpr int CW = 16, KPC = CW / R3, OWN = KPC / 2;
+            static_assert(OWN * R3 == 8, "eight spectrum values per chunk");
             const int k2 = r >> 1;
             float2 tw[R3];
 #pragma unroll
             for (int n3 = 0; n3 < R3; ++n3) tw[n3] = fft::expi_neg(n3 * k2, 64 * R3);
-            const float2 *hrow = spec + ((size_t)HB_IDX(hd, H) * N + (size_t)k2 * 64 * R3);
             const int row = kappa(k2, c);
 #pragma unroll 1
-            for (int m0 = 0; m0 < C; m0 += 32) {
-                float x[32], px[32];
-                tc::tmem_ld32(trow + m0, x);
+            for (int m0 = 0; m0 < C; m0 += CW) {
+                float4 h4[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    h4[i] = ha[i];
+                    ha[i] = hb[i];
+                }
+                if (m0 + 2 * CW < C) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) hb[i] = __ldg(&hrow4[(m0 + 2 * CW) / 4 + i]);
+                }
+                const float2 *hc = reinterpret_cast<const float2 *>(h4);
+                float x[CW];
+                tc::tmem_ld16(trow + m0, x);
                 tc::tmem_wait_ld();
+                float o[CW];
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) px[jj] = __shfl_xor_sync(0xffffffffu, x[jj], 1);
-                float o[32];
-#pragma unroll
-                for (int gq = 0; gq < 32 / R3; ++gq) {
-                    const int k1 = m0 / R3 + gq;
+                for (int i = 0; i < OWN; ++i) {
                     float2 V[R3];
 #pragma unroll
                     for (int n3 = 0; n3 < R3; ++n3) {
-                        const int jj = gq * R3 + n3;
-                        V[n3] = c ? make_float2(px[jj], x[jj]) : make_float2(x[jj], px[jj]);
+                        const int je = (2 * i) * R3 + n3, jo = (2 * i + 1) * R3 + n3;
+                        const float rcv = __shfl_xor_sync(0xffffffffu, c ? x[je] : x[jo], 1);
+                        V[n3] = c ? make_float2(rcv, x[jo]) : make_float2(x[je], rcv);
                         if (n3) V[n3] = cmul(V[n3], tw[n3]);
                     }
                     small_dft<R3, false>(V);
 #pragma unroll
-                    for (int k3 = 0; k3 < R3; ++k3) V[k3] = cmul(V[k3], __ldg(&hrow[k1 * R3 + k3]));
+                    for (int k3 = 0; k3 < R3; ++k3) V[k3] = cmul(V[k3], hc[i * R3 + k3]);
                     small_dft<R3, true>(V);
 #pragma unroll
                     for (int n3 = 0; n3 < R3; ++n3) {
-                        float2 z = V[n3];
-                        if (n3) z = cmulc(z, tw[n3]);
-                        o[gq * R3 + n3] = c ? -z.y : z.x;
+                        const float2 z = n3 ? cmulc(V[n3], tw[n3]) : V[n3];
+                        const int je = (2 * i) * R3 + n3, jo = (2 * i + 1) * R3 + n3;
+                        const float rcv = __shfl_xor_sync(0xffffffffu, c ? z.x : -z.y, 1);
+                        o[je] = c ? rcv : z.x;
+                        o[jo] = c ? -z.y : rcv;
                     }
                 }
                 uint8_t *drow = bop + (m0 >> 6) * M::kAtom + row * 128;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int i = 0; i < CW / 8; ++i) {
                     const int chunk = ((m0 & 63) >> 3) + i;
                     *reinterpret_cast<uint4 *>(drow + ((chunk ^ (row & 7)) << 4)) =
                         make_uint4(pack2(o[8 * i], o[8 * i + 1]), pack2(o[8 * i + 2], o[8 * i + 3]),
@@ -463,7 +551,7 @@ prefill_monarch_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
                 const long long o = ((long long)b * L + t0 + s) * Dch + c0;
-                qr[s] = (t0 + s < L && HB_OK(o + G - 1, n_act)) ? __ldg(reinterpret_cast<const RowT *>(q + o)) : RowT{};
+                qr[s] = (t0 + s < L && HB_OK(o + G - 1, n_act)) ? __ldcg(reinterpret_cast<const RowT *>(q + o)) : RowT{};
             }
             float yv[G][8];
 #pragma unroll

@@ -34,6 +34,7 @@ SIGNATURES = {
     "hyena_filter_spectrum": (_i, [_fp, _i, _i, _i, _fp, _vp, _sz, _vp]),
     "hyena_prefill_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "hyena_prefill_error_offset": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "hyena_prefill_uses_tensor_cores": (_i, [_i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "hyena_prefill": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp, _fp,
                            _vp, _sz, _vp]),
     "hyena_prefill_chunked_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
@@ -293,6 +294,16 @@ def chunked_error(workspace, B, L, Dch, H, d) -> int:
     """The kernel's error word (synchronises): 0 when every bounded wait succeeded."""
     off = int(lib().hyena_prefill_chunked_error_offset(B, L, Dch, H, d))
     return int(workspace[off:off + 4].view(torch.int32).item())
+
+
+def prefill_uses_tensor_cores(q, k, v, H: int, d: int, fft_len: int, y=None) -> bool:
+    """Whether prefill(q, k, v, ...) with these tensors runs its transforms on the tensor cores."""
+    B, L, Dch = q.shape
+    st = lib().hyena_prefill_uses_tensor_cores(_act_dtype(q), B, L, Dch, H, d, fft_len, _ptr(q), _ptr(k), _ptr(v),
+                                              _ptr(q if y is None else y))
+    if st < 0:
+        _check("hyena_prefill_uses_tensor_cores", st)
+    return st == 1
 
 
 def prefill_error(workspace, B, L, Dch, H, d, fft_len) -> int:

@@ -148,6 +148,12 @@ int hyena_filter_spectrum(const float *h, int H, int L, int fft_len, float *spec
  */
 size_t hyena_prefill_workspace_bytes(int B, int L, int Dch, int H, int d, int fft_len);
 size_t hyena_prefill_error_offset(int B, int L, int Dch, int H, int d, int fft_len);
+/* 1 if hyena_prefill with these arguments runs on the tensor cores, 0 if on the
+ * CUDA cores; HYENA_ERR_ARG / HYENA_ERR_SHAPE / HYENA_ERR_UNSUPPORTED as
+ * hyena_prefill would return for invalid arguments.  Pointers are only
+ * inspected for alignment.  Host-only (no CUDA call). */
+int hyena_prefill_uses_tensor_cores(int dtype, int B, int L, int Dch, int H, int d, int fft_len,
+                                    const void *q, const void *k, const void *v, const void *y);
 int hyena_prefill(const void *q, const void *k, const void *v, int dtype,
                   int B, int L, int Dch, int H, int d, int fft_len,
                   const float *lambda, const float *R, const float *Dskip,

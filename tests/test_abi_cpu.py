@@ -222,6 +222,25 @@ def test_fft_route_hook_and_error_offset(lib):
     assert lib.hyena_prefill_error_offset(8, 4096, 1024, 8, 16, 4096) == 0    # fft_len < 2L-1
 
 
+def test_route_query_follows_the_documented_rule(lib):
+    BF16, F32 = 1, 0
+    a = ctypes.c_void_p(1 << 20)                       # 16-byte aligned (inspected only)
+    assert lib.hyena_prefill_uses_tensor_cores(BF16, 8, 4096, 1024, 8, 16, 8192, a, a, a, a) == 1
+    assert lib.hyena_prefill_uses_tensor_cores(F32, 8, 4096, 1024, 8, 16, 8192, a, a, a, a) == 0
+    assert lib.hyena_prefill_uses_tensor_cores(BF16, 8, 4096, 1020, 4, 16, 8192, a, a, a, a) == 0   # Dch % 8
+    assert lib.hyena_prefill_uses_tensor_cores(BF16, 1, 9000, 16, 2, 16, 32768, a, a, a, a) == 0    # four-step
+    assert lib.hyena_prefill_uses_tensor_cores(BF16, 1, 900, 16, 2, 16, 2048, a, a, a, a) == 0      # too short
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    assert lib.hyena_prefill_uses_tensor_cores(BF16, 8, 4096, 1024, 8, 16, 8192, a, odd, a, a) == 0
+    assert lib.hyena_prefill_uses_tensor_cores(BF16, 8, 4096, 1024, 8, 16, 4096, a, a, a, a) == ERR_SHAPE
+    assert lib.hyena_prefill_uses_tensor_cores(7, 8, 4096, 1024, 8, 16, 8192, a, a, a, a) == ERR_ARG
+    assert lib.hyena_test_fft_tensor_cores(0) == OK
+    try:
+        assert lib.hyena_prefill_uses_tensor_cores(BF16, 8, 4096, 1024, 8, 16, 8192, a, a, a, a) == 0
+    finally:
+        assert lib.hyena_test_fft_tensor_cores(1) == OK
+
+
 def test_prefill_chunked_layers_validation(lib):
     arr = (ctypes.c_void_p * 1)(FAKE)
     call = lambda layers, dtype=1, B=2, L=64, Dch=128, H=2, d=4, ws=1 << 30: lib.hyena_prefill_chunked_layers(
