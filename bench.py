@@ -996,6 +996,9 @@ def main(argv=None):
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size")
     ap.add_argument("--prefill", choices=["auto", "chunked", "fft"], default="auto",
                     help="prefill route: chunked tensor-core evaluation (auto when supported) or FFT")
+    ap.add_argument("--fft-cuda-cores", action="store_true",
+                    help="run the FFT route's transforms on the CUDA cores also where the tensor-core "
+                         "route applies (bf16 at FFT lengths 4096..16384); for comparisons")
     ap.add_argument("--no-fft-route", action="store_true",
                     help="skip the extra timing of the FFT route when the chunked route is used")
     ap.add_argument("--no-e2e", action="store_true")
@@ -1015,6 +1018,9 @@ def main(argv=None):
         return run_reference(args)
     if args.truncation:
         return run_truncation(args)
+    if args.fft_cuda_cores:
+        from distilled_ssm_decode_b200 import ops
+        ops.lib().hyena_test_fft_tensor_cores(0)
     return run_ours(args)
 
 

@@ -371,23 +371,28 @@ prefill_monarch_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 
         wg_sync(p);                                   // the state's reads of the operand are done
 
         // T1: rows (k1, c), columns j = R3 n2 + n3: times w_N^(j k1); to K-row kappa(n2, c),
-        //     columns R3 k1 + n3
+        //     columns R3 k1 + n3.  Lane c forms the complex products of the columns j % 2 == c
+        //     (twiddle chain stepping by w_N^(2 k1)); two shuffles per column pair swap the parts.
         {
             const int k1 = r >> 1;
-            const float2 st = fft::expi_neg(k1, N);
+            const float2 st = fft::expi_neg((2 * k1) % N, N);
             const int col = R3 * k1;
 #pragma unroll 1
             for (int j0 = 0; j0 < C; j0 += 32) {
                 float x[32];
                 tc::tmem_ld32(trow + j0, x);
                 tc::tmem_wait_ld();
-                float2 w = fft::expi_neg((j0 * k1) % N, N);
+                float2 w = fft::expi_neg(((j0 + c) * k1) % N, N);
                 float o[32];
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const float pv = __shfl_xor_sync(0xffffffffu, x[jj], 1);
-                    o[jj] = fmaf(x[jj], w.x, (c ? pv : -pv) * w.y);
+                for (int i = 0; i < 16; ++i) {
+                    const float rcv = __shfl_xor_sync(0xffffffffu, c ? x[2 * i] : x[2 * i + 1], 1);
+                    const float2 V = c ? make_float2(rcv, x[2 * i + 1]) : make_float2(x[2 * i], rcv);
+                    const float2 z = cmul(V, w);
                     w = cmul(w, st);
+                    const float back = __shfl_xor_sync(0xffffffffu, c ? z.x : z.y, 1);
+                    o[2 * i] = c ? back : z.x;
+                    o[2 * i + 1] = c ? z.y : back;
                 }
 #pragma unroll
                 for (int gq = 0; gq < 32 / R3; ++gq) {
@@ -403,13 +408,13 @@ prefill_monarch_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 
         const float4 *hrow4 = reinterpret_cast<const float4 *>(
             spec + ((size_t)HB_IDX(hd, H) * N + (size_t)((r >> 1) * 2 + c) * 32 * R3));
         float4 ha[4], hb[4];
+        step_done();
+        if (issuer) issue(8);                         // stage B
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             ha[i] = __ldg(&hrow4[i]);
             hb[i] = __ldg(&hrow4[4 + i]);
         }
-        step_done();
-        if (issuer) issue(8);                         // stage B
         wait_product();
 
         // T2: rows (k2, c), columns R3 k1 + n3: twiddle, R3-point DFT, spectrum, inverse
@@ -481,12 +486,20 @@ prefill_monarch_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 
         wait_product();
 
         // T3: rows (n2, c), columns R3 k1 + n3: times w_N^((R3 n2 + n3) k1); to K-row
-        //     kappa(k1, c), columns R3 n2 + n3
+        //     kappa(k1, c), columns R3 n2 + n3.  Lane c forms the complex products of the columns
+        //     m % 2 == c, as in T1 (chains per n3 residue: one, or two for R3 = 4).
         {
             const int n2 = r >> 1;
-            float2 st[R3];
+            constexpr int NCH = (R3 == 4) ? 2 : 1;
+            constexpr int KSTEP = (R3 == 1) ? 2 : 1;       // k1 advance of a chain per use
+            float2 st[NCH];
+            int ex[NCH];                                    // R3 n2 + n3 of each chain
 #pragma unroll
-            for (int n3 = 0; n3 < R3; ++n3) st[n3] = fft::expi_neg(R3 * n2 + n3, N);
+            for (int q2 = 0; q2 < NCH; ++q2) {
+                const int n3q = (R3 == 1) ? 0 : c + 2 * q2;
+                ex[q2] = R3 * n2 + n3q;
+                st[q2] = fft::expi_neg((ex[q2] * KSTEP) % N, N);
+            }
             const int col = R3 * n2;
 #pragma unroll 1
             for (int m0 = 0; m0 < C; m0 += 32) {
@@ -494,19 +507,21 @@ prefill_monarch_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 
                 tc::tmem_ld32(trow + m0, x);
                 tc::tmem_wait_ld();
                 const int k10 = m0 / R3;
-                float2 w[R3];
+                const int k1f = (R3 == 1) ? m0 + c : k10;      // first k1 of each chain in the chunk
+                float2 w[NCH];
 #pragma unroll
-                for (int n3 = 0; n3 < R3; ++n3) w[n3] = fft::expi_neg(((R3 * n2 + n3) * k10) % N, N);
+                for (int q2 = 0; q2 < NCH; ++q2) w[q2] = fft::expi_neg((ex[q2] * k1f) % N, N);
                 float o[32];
 #pragma unroll
-                for (int gq = 0; gq < 32 / R3; ++gq) {
-#pragma unroll
-                    for (int n3 = 0; n3 < R3; ++n3) {
-                        const int jj = gq * R3 + n3;
-                        const float pv = __shfl_xor_sync(0xffffffffu, x[jj], 1);
-                        o[jj] = fmaf(x[jj], w[n3].x, (c ? pv : -pv) * w[n3].y);
-                        w[n3] = cmul(w[n3], st[n3]);
-                    }
+                for (int i = 0; i < 16; ++i) {
+                    const int q2 = (R3 == 4) ? (i & 1) : 0;
+                    const float rcv = __shfl_xor_sync(0xffffffffu, c ? x[2 * i] : x[2 * i + 1], 1);
+                    const float2 V = c ? make_float2(rcv, x[2 * i + 1]) : make_float2(x[2 * i], rcv);
+                    const float2 z = cmul(V, w[q2]);
+                    w[q2] = cmul(w[q2], st[q2]);
+                    const float back = __shfl_xor_sync(0xffffffffu, c ? z.x : z.y, 1);
+                    o[2 * i] = c ? back : z.x;
+                    o[2 * i + 1] = c ? z.y : back;
                 }
 #pragma unroll
                 for (int gq = 0; gq < 32 / R3; ++gq) {
