@@ -36,8 +36,8 @@ cudaError_t launch_prefill_fft(const void *q, const void *k, const void *v, int 
                                void *y, float *state_out, void *scratch, size_t scratch_bytes,
                                cudaStream_t s);
 
-// spectrum for the tensor-core route: frequency k = k1 + 64 k2 + 4096 k3 stored at
-// [k2][k1 % 2][k1 / 2][k3] per head (N = 4096, 8192 or 16384)
+// spectrum for the tensor-core route: frequency k = k1 + 64 k2 + 4096 k3 stored per head in the
+// order its lanes read it (N = 4096, 8192 or 16384; see spectrum_fused_kernel)
 cudaError_t launch_spectrum_monarch(const float *h, int H, int L, int N, float2 *spec, float scale,
                                     cudaStream_t s);
 

@@ -46,8 +46,10 @@ int fused_threads(int N) {
 // ------------------------------------------------------------------ spectrum
 // One CTA per head: forward transform of the zero-padded filter, times scale,
 // stored in the transform's digit-reversed order (mon_r3 == 0), or, for the
-// tensor-core route, at frequency k = k1 + 64 k2 + 4096 k3 in the order
-// [k2][k1 % 2][k1 / 2][k3] (mon_r3 = N / 4096).
+// tensor-core route, at frequency k = k1 + 64 k2 + 4096 k3 in the order its lanes read it
+// (mon_r3 = N / 4096): with c = k1 % 2 and f8 = (k1 / 2) R3 + k3, the float2 index is
+// ((((f8 / 8) * 4 + (f8 % 8) / 2) * 64 + k2) * 2 + c) * 2 + f8 % 2, so that the 32 lanes of a
+// warp (16 values of k2, two of c) read one contiguous 512-byte run per 16-byte load.
 __global__ void __launch_bounds__(kFusedThreads)
 spectrum_fused_kernel(const float *__restrict__ h, int L, int N, float scale,
                       float2 *__restrict__ spec_perm, int mon_r3) {
@@ -66,7 +68,8 @@ spectrum_fused_kernel(const float *__restrict__ h, int L, int N, float scale,
         int o = p;
         if (mon_r3) {
             const int f = fft::freq_of_pos(p, N);
-            o = ((((f >> 6) & 63) * 2 + (f & 1)) * 32 + ((f & 63) >> 1)) * mon_r3 + (f >> 12);
+            const int k1 = f & 63, k2 = (f >> 6) & 63, f8 = (k1 >> 1) * mon_r3 + (f >> 12);
+            o = (((((f8 >> 3) * 4 + ((f8 & 7) >> 1)) * 64 + k2) * 2 + (k1 & 1)) * 2) + (f8 & 1);
         }
         if (HB_OK((long long)hd * N + o, (long long)H * N)) out[o] = cscale(buf[pad(p)], scale);
     }

@@ -404,16 +404,16 @@ prefill_monarch_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 
             }
         }
         // the spectrum of this row's first two T2 chunks, loaded while stage B runs: row (k2, c)
-        // reads the k1 with k1 % 2 == c, stored contiguously ([k2][k1 % 2][k1 / 2][k3])
-        const float4 *hrow4 = reinterpret_cast<const float4 *>(
-            spec + ((size_t)HB_IDX(hd, H) * N + (size_t)((r >> 1) * 2 + c) * 32 * R3));
+        // reads the k1 with k1 % 2 == c, 8 values per 16-column chunk as 4 float4; float4 i of
+        // chunk q sits at ((q * 4 + i) * 64 + k2) * 2 + c, so a warp's loads are contiguous
+        const float4 *hrow4 = reinterpret_cast<const float4 *>(spec + (size_t)HB_IDX(hd, H) * N) + r;
         float4 ha[4], hb[4];
         step_done();
         if (issuer) issue(8);                         // stage B
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            ha[i] = __ldg(&hrow4[i]);
-            hb[i] = __ldg(&hrow4[4 + i]);
+            ha[i] = __ldg(&hrow4[i * 128]);
+            hb[i] = __ldg(&hrow4[(4 + i) * 128]);
         }
         wait_product();
 
@@ -422,7 +422,7 @@ prefill_monarch_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 
         //     The two lanes of a row pair split the work: lane c computes the complex chain of
         //     the k1 with k1 % 2 == c (one shuffle brings in the other part of its inputs, one
         //     more hands back the partner's part of its outputs), and loads only those k1's
-        //     spectrum (8 values per 16-column chunk), two chunks ahead.
+        //     spectrum (8 values per 16-column chunk, contiguous across the warp), two chunks ahead.
         {
             constexpr int CW = 16, KPC = CW / R3, OWN = KPC / 2;
             static_assert(OWN * R3 == 8, "eight spectrum values per chunk");
@@ -441,7 +441,7 @@ prefill_monarch_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 
                 }
                 if (m0 + 2 * CW < C) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) hb[i] = __ldg(&hrow4[(m0 + 2 * CW) / 4 + i]);
+                    for (int i = 0; i < 4; ++i) hb[i] = __ldg(&hrow4[(((m0 + 2 * CW) / CW) * 4 + i) * 128]);
                 }
                 const float2 *hc = reinterpret_cast<const float2 *>(h4);
                 float x[CW];
