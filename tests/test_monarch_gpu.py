@@ -102,8 +102,12 @@ def test_route_is_taken_and_both_routes_agree():
     """Same inputs through both routes: different roundings (so the tensor-core route ran),
     the same operator within the bf16 bar; the states agree to fp32 rounding."""
     w, p = _case(5, 2, 4096, 32, 4, 16)
-    _, y_tc, s_tc = _run(w, p, 8192, tensor_cores=True)
+    (q, k, v), y_tc, s_tc = _run(w, p, 8192, tensor_cores=True)
     _, y_cc, s_cc = _run(w, p, 8192, tensor_cores=False)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    assert ops.prefill_uses_tensor_cores(qd, kd, vd, w.H, w.d, 8192)
+    with ops.fft_tensor_cores(False):
+        assert not ops.prefill_uses_tensor_cores(qd, kd, vd, w.H, w.d, 8192)
     assert not torch.equal(y_tc, y_cc)
     assert rel_err(y_tc.cpu().double().numpy(), y_cc.cpu().double().numpy()) <= Y_MARGIN
     assert rel_err(state_c128(s_tc), state_c128(s_cc)) <= 1e-5
@@ -120,6 +124,7 @@ def test_layouts_outside_the_route_fall_back_to_cuda_cores(oracle):
     """Dch not a multiple of 8 at FFT length 8192: the CUDA-core route, still within the bar."""
     w, p = _case(7, 1, 2000, 12, 2, 8)
     (q, k, v), y, s = _run(w, p, 8192)
+    assert not ops.prefill_uses_tensor_cores(q.cuda(), k.cuda(), v.cuda(), w.H, w.d, 8192)
     y_ref, s_ref = _oracle(oracle, w, p, q, k, v)
     assert rel_err(y.cpu().double().numpy(), y_ref) <= TOL["bf16"]
     assert rel_err(state_c128(s), s_ref) <= 1e-4
