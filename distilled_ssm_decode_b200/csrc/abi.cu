@@ -56,7 +56,8 @@ PrefillWs prefill_ws(int B, int L, int Dch, int H, int d, int fft_len) {
     w.spec_off = align_up((size_t)H * L * sizeof(float));
     w.four_off = w.spec_off + align_up(spectrum_ws_bytes(H, N));
     w.state_off = w.four_off + align_up(fourstep_ws_bytes(B, Dch, ch, N));
-    w.err_off = w.state_off + (N > kFusedMaxN ? align_up(state_ws_bytes(B, L, Dch, d)) : 0);
+    // beyond 16384 points: the state partials, then the spectrum rows of the tensor-core inner kernel
+    w.err_off = w.state_off + (N > kFusedMaxN ? align_up(state_ws_bytes(B, L, Dch, d)) + align_up(spectrum_ws_bytes(H, N)) : 0);
     w.total = w.err_off + kAlign;
     return w;
 }
@@ -179,7 +180,7 @@ int hyena_prefill(const void *q, const void *k, const void *v, int dtype, int B,
     e = launch_spectrum_perm(h, H, L, N, spec, 1.0f / (float)N, s);
     if (e != cudaSuccess) return HYENA_ERR_CUDA;
     e = launch_prefill_fft(q, k, v, dtype, B, L, Dch, H, d, N, spec, lam2, y, state_out,
-                           ws + w.four_off, w.err_off - w.four_off, s);
+                           ws + w.four_off, w.err_off - w.four_off, err, s);
     return cuda_status(e);
 }
 
@@ -188,7 +189,10 @@ int hyena_prefill_uses_tensor_cores(int dtype, int B, int L, int Dch, int H, int
     if (dtype != HYENA_F32 && dtype != HYENA_BF16) return HYENA_ERR_ARG;
     const int st = check_prefill_shape(B, L, Dch, H, d, fft_len);
     if (st != HYENA_OK) return st;
-    return monarch_r3(dtype, B, L, Dch, H, fft_internal_len(fft_len), q, k, v, y) != 0 ? 1 : 0;
+    const int N = fft_internal_len(fft_len);
+    if (monarch_r3(dtype, B, L, Dch, H, N, q, k, v, y) != 0) return 1;
+    // beyond 16384 points the four-step route's inner transforms run on the tensor cores for bf16
+    return (N > kFusedMaxN && dtype == HYENA_BF16 && fourstep_tc_enabled()) ? 1 : 0;
 }
 
 size_t hyena_prefill_error_offset(int B, int L, int Dch, int H, int d, int fft_len) {

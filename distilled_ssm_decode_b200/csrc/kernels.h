@@ -34,7 +34,7 @@ cudaError_t launch_prefill_fft(const void *q, const void *k, const void *v, int 
                                int B, int L, int Dch, int H, int d, int N,
                                const float2 *spec_perm, const float2 *lam,
                                void *y, float *state_out, void *scratch, size_t scratch_bytes,
-                               cudaStream_t s);
+                               int *err, cudaStream_t s);
 
 // spectrum for the tensor-core route: frequency k = k1 + 64 k2 + 4096 k3 stored per head in the
 // order its lanes read it (N = 4096, 8192 or 16384; see spectrum_fused_kernel)
@@ -46,6 +46,11 @@ cudaError_t launch_spectrum_monarch(const float *h, int H, int L, int N, float2 
 int monarch_r3(int dtype, int B, int L, int Dch, int H, int N, const void *q, const void *k, const void *v,
                const void *y);
 void monarch_enable(int enable);
+// the four-step route's inner 8192-point rows on the tensor cores (bf16 activations); specm holds
+// each (head, k1) row's spectrum in the order fourstep_spec_tc_kernel writes
+bool fourstep_tc_enabled();
+cudaError_t launch_fourstep_inner_tc(float2 *Y, int N1, int ncols, int nslots, int paired, int ch, int H,
+                                     const float2 *specm, int *err, cudaStream_t s);
 cudaError_t launch_prefill_monarch(int r3, const void *q, const void *k, const void *v, int B, int L, int Dch,
                                    int H, int d, const float2 *spec, const float2 *lam, void *y,
                                    float *state_out, int *err, cudaStream_t s);

@@ -290,6 +290,26 @@ fourstep_inner_kernel(float2 *__restrict__ Y, int N1, int N2, int mode, float sc
         if (HB_OK(t, n_row)) row[t] = buf[pad(t)];
 }
 
+// The four-step spectrum rows (row k1 of a head: the spectrum at k1 + N1 f2, f2 in the inner
+// transform's digit-reversed order) reordered for the tensor-core inner kernel: inner frequency
+// f2 = a1 + 64 a2 + 4096 a3 goes where its lanes read it (the order of spectrum_fused_kernel's
+// tensor-core layout at 8192 points).
+__global__ void fourstep_spec_tc_kernel(const float2 *__restrict__ spec_perm, int N1, int N2,
+                                        float2 *__restrict__ out) {
+    const int k1 = blockIdx.x, hd = blockIdx.y;
+    const long long N = (long long)N1 * N2;
+    const long long n_all = (long long)gridDim.y * N;
+    (void)n_all;
+    for (int p = threadIdx.x; p < N2; p += blockDim.x) {
+        const int f = fft::freq_of_pos(p, N2);
+        const int a1 = f & 63, a2 = (f >> 6) & 63, f8 = (a1 >> 1) * 2 + (f >> 12);
+        const int o = (((((f8 >> 3) * 4 + ((f8 & 7) >> 1)) * 64 + a2) * 2 + (a1 & 1)) * 2) + (f8 & 1);
+        const long long dst = ((long long)hd * N1 + k1) * N2 + o;
+        if (HB_OK(dst, n_all))
+            out[dst] = spec_perm[HB_IDX((long long)hd * N + (long long)k1 * N2 + p, n_all)];
+    }
+}
+
 // step 3: inverse across the long stride, gate-out, store the first L outputs
 template <int N1, class Act>
 __global__ void __launch_bounds__(256)
@@ -383,7 +403,7 @@ template <class Act>
 cudaError_t prefill_fourstep(const void *q, const void *k, const void *v, int B, int L, int Dch,
                              int H, int ch, int d, int N, int paired, const float2 *spec_perm,
                              const float2 *lam, void *y, float *state_out, void *scratch,
-                             cudaStream_t s) {
+                             int *err, cudaStream_t s) {
     using T = typename Act::T;
     const int N2 = kFourStepN2, N1 = N / N2;
     const int nslots = paired ? Dch / 2 : Dch;
@@ -393,12 +413,22 @@ cudaError_t prefill_fourstep(const void *q, const void *k, const void *v, int B,
     ActSrc<Act> src{static_cast<const T *>(k), static_cast<const T *>(v), L, Dch, nslots, paired};
     cudaError_t e = launch_fwd1(N1, src, N2, ncols, Y, s);
     if (e != cudaSuccess) return e;
-    const size_t smem = inner_smem_bytes(N2);
-    e = set_smem((const void *)fourstep_inner_kernel, smem);
+    if (Act::bytes == 2 && fourstep_tc_enabled()) {
+        // bf16 activations: the inner transforms on the tensor cores, with the spectrum rows in the
+        // order that kernel reads them (after the state partials in the scratch)
+        float2 *specm = reinterpret_cast<float2 *>(after + ((state_ws_bytes(B, L, Dch, d) + 255) & ~size_t(255)));
+        fourstep_spec_tc_kernel<<<dim3(N1, H), 256, 0, s>>>(spec_perm, N1, N2, specm);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = launch_fourstep_inner_tc(Y, N1, ncols, nslots, paired, ch, H, specm, err, s);
+    } else {
+        const size_t smem = inner_smem_bytes(N2);
+        e = set_smem((const void *)fourstep_inner_kernel, smem);
+        if (e != cudaSuccess) return e;
+        fourstep_inner_kernel<<<dim3(N1, ncols), kFusedThreads, smem, s>>>(Y, N1, N2, 1, 1.f, spec_perm,
+                                                                          nslots, paired, ch);
+        e = cudaGetLastError();
+    }
     if (e != cudaSuccess) return e;
-    fourstep_inner_kernel<<<dim3(N1, ncols), kFusedThreads, smem, s>>>(Y, N1, N2, 1, 1.f, spec_perm,
-                                                                      nslots, paired, ch);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     e = launch_inv1<Act>(N1, Y, N2, L, Dch, nslots, paired, ncols, q, y, s);
     if (e != cudaSuccess) return e;
     // the state comes from the standalone reduction (u is never whole in one CTA here)
@@ -462,7 +492,7 @@ cudaError_t launch_prefill_fft(const void *q, const void *k, const void *v, int 
                                int B, int L, int Dch, int H, int d, int N,
                                const float2 *spec_perm, const float2 *lam,
                                void *y, float *state_out, void *scratch, size_t scratch_bytes,
-                               cudaStream_t s) {
+                               int *err, cudaStream_t s) {
     (void)scratch_bytes;
     const int ch = Dch / H;
     const int paired = (ch % 2 == 0) ? 1 : 0;
@@ -472,8 +502,8 @@ cudaError_t launch_prefill_fft(const void *q, const void *k, const void *v, int 
                    : prefill_fused<ActF32>(q, k, v, B, L, Dch, ch, d, N, paired, spec_perm, lam, y, state_out, s);
     }
     return dtype == HYENA_BF16
-               ? prefill_fourstep<ActBF16>(q, k, v, B, L, Dch, H, ch, d, N, paired, spec_perm, lam, y, state_out, scratch, s)
-               : prefill_fourstep<ActF32>(q, k, v, B, L, Dch, H, ch, d, N, paired, spec_perm, lam, y, state_out, scratch, s);
+               ? prefill_fourstep<ActBF16>(q, k, v, B, L, Dch, H, ch, d, N, paired, spec_perm, lam, y, state_out, scratch, err, s)
+               : prefill_fourstep<ActF32>(q, k, v, B, L, Dch, H, ch, d, N, paired, spec_perm, lam, y, state_out, scratch, err, s);
 }
 
 }  // namespace hyena

@@ -598,6 +598,294 @@ prefill_monarch_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 
     if (warp == 0) tc::tmem_dealloc(tmem, M::kTmemCols);
 }
 
+// ------------------------------------------------------------------ four-step inner rows
+// The inner 8192-point transforms of the four-step route (transforms longer than 16384 points,
+// bf16 activations) on the tensor cores: each row of the complex plane Y (one column and one
+// residue k1 of the outer factor) goes through the same 64 x 64 x 2 factorisation and products
+// as prefill_monarch_kernel -- forward, times the row's spectrum, inverse -- and back in place.
+// The rows are contiguous complex fp32, so every warpgroup loads and stores its own row with
+// coalesced 16-byte accesses and the four warpgroups of a CTA run independently (no CTA-wide
+// step inside the loop).  Stage A takes the full K (the row has no zero half); the output is
+// staged in two halves of 64 columns through the free operand buffer.
+__global__ void __launch_bounds__(512, 1)
+fourstep_inner_tc_kernel(float2 *__restrict__ Y, int N1, int ncols, int nslots, int paired, int ch,
+                         int H, const float2 *__restrict__ specm, int *err) {
+    using M = Mon<2>;
+    constexpr int N2 = M::N, C = M::C, P = M::P, R3 = 2;
+    constexpr int kSmBarI = M::kSmB + P * M::kBop;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = tc::smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    uint8_t *sp = smem_raw + (sbase - raw);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sp + kSmBarI);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sp + kSmBarI + 8 * P);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sp + kSmBarI + 8 * P + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int p = warp >> 2, qd = warp & 3, r = 32 * qd + lane, c = r & 1, wt = tid - 128 * p;
+    const uint32_t bar_p = tc::smem_u32(&bars[p]);
+    uint8_t *bop = sp + M::kSmB + p * M::kBop;
+    const uint32_t bop_s = sbase + M::kSmB + p * M::kBop;
+    const long long rows = (long long)ncols * N1;
+    const long long n_y = rows * N2;
+    (void)n_y; (void)H;
+
+    if (tid == 0) {
+        for (int i = 0; i < P; ++i) tc::mbar_init(tc::smem_u32(&bars[i]), 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(tc::smem_u32(tmem_slot), M::kTmemCols);
+        tc::tmem_relinquish();
+    }
+    for (int e = tid; e < 128 * 128; e += blockDim.x) {
+        const int row = e >> 7, kk = e & 127;
+        const int kf = row >> 1, co = row & 1;
+        const int n = 4 * (kk >> 3) + (kk & 3), ci = (kk >> 2) & 1;
+        float s, cs;
+        sincospif((float)((kf * n) & 63) / 32.0f, &s, &cs);
+        const float val = co == 0 ? (ci == 0 ? cs : s) : (ci == 0 ? -s : cs);
+        *reinterpret_cast<__nv_bfloat16 *>(sp + M::kSmA + amat_off(row, kk)) = __float2bfloat16_rn(val);
+    }
+    tc::fence_proxy_async_smem();
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t dcol = tmem + p * C;
+    const uint32_t trow = tmem + ((uint32_t)(32 * qd) << 16) + p * C;
+    const bool issuer = (qd == 0 && lane == 0);
+    uint32_t ph = 0;
+    bool ok = true;
+    auto issue = [&](int nks) {
+        tc::tc_fence_after();
+        if (ok) {
+            const uint32_t idesc = tc::idesc_bf16(128, C, true);
+#pragma unroll 1
+            for (int ks = 0; ks < nks; ++ks) {
+                const uint64_t ad = tc::smem_desc(sbase + M::kSmA + ks * 256, 128, 2048);
+                const uint64_t bd = tc::smem_desc_sw128(bop_s + ks * 2048, M::kAtom, 1024);
+                tc::mma_bf16(dcol, ad, bd, idesc, ks > 0);
+            }
+            tc::mma_commit(bar_p);
+        }
+    };
+    auto wait_product = [&]() {
+        if (ok && !tc::mbar_wait(bar_p, ph, abort_flag)) {
+            ok = false;
+            *abort_flag = 1;
+            atomicCAS(err, 0, 1);
+        }
+        ph ^= 1;
+        tc::tc_fence_after();
+    };
+    auto step_done = [&]() {
+        tc::tmem_wait_ld();
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        wg_sync(p);
+    };
+
+#pragma unroll 1
+    for (long long rw = (long long)blockIdx.x * P + p; rw < rows; rw += (long long)gridDim.x * P) {
+        const int col = (int)(rw / N1), k1o = (int)(rw % N1);
+        const int slot = col % nslots;
+        const int hd = (paired ? 2 * slot : slot) / ch;
+        float2 *rowp = Y + rw * N2;
+
+        // gate-in: the row (8 complex values per thread and step) as Re / Im K-rows of the operand
+#pragma unroll 1
+        for (int it = wt; it < N2 / 8; it += 128) {
+            const int t0 = it * 8;
+            float4 a[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = __ldcg(reinterpret_cast<const float4 *>(rowp + HB_IDX(t0 + 2 * i, n_y - rw * N2)));
+            const int n1 = t0 / C, j0 = t0 % C;
+            *reinterpret_cast<uint4 *>(bop + bop_off(kappa(n1, 0), j0)) =
+                make_uint4(pack2(a[0].x, a[0].z), pack2(a[1].x, a[1].z), pack2(a[2].x, a[2].z), pack2(a[3].x, a[3].z));
+            *reinterpret_cast<uint4 *>(bop + bop_off(kappa(n1, 1), j0)) =
+                make_uint4(pack2(a[0].y, a[0].w), pack2(a[1].y, a[1].w), pack2(a[2].y, a[2].w), pack2(a[3].y, a[3].w));
+        }
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        wg_sync(p);
+        if (issuer) issue(8);                         // stage A (full K)
+        wait_product();
+
+        // T1 (as in prefill_monarch_kernel)
+        {
+            const int k1 = r >> 1;
+            const float2 st = fft::expi_neg((2 * k1) % N2, N2);
+            const int colo = R3 * k1;
+#pragma unroll 1
+            for (int j0 = 0; j0 < C; j0 += 32) {
+                float x[32];
+                tc::tmem_ld32(trow + j0, x);
+                tc::tmem_wait_ld();
+                float2 w = fft::expi_neg(((j0 + c) * k1) % N2, N2);
+                float o[32];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float rcv = __shfl_xor_sync(0xffffffffu, c ? x[2 * i] : x[2 * i + 1], 1);
+                    const float2 V = c ? make_float2(rcv, x[2 * i + 1]) : make_float2(x[2 * i], rcv);
+                    const float2 z = cmul(V, w);
+                    w = cmul(w, st);
+                    const float back = __shfl_xor_sync(0xffffffffu, c ? z.x : z.y, 1);
+                    o[2 * i] = c ? back : z.x;
+                    o[2 * i + 1] = c ? z.y : back;
+                }
+#pragma unroll
+                for (int gq = 0; gq < 16; ++gq)
+                    *reinterpret_cast<uint32_t *>(bop + bop_off(kappa(j0 / R3 + gq, c), colo)) = pack2(o[2 * gq], o[2 * gq + 1]);
+            }
+        }
+        const float4 *hrow4 = reinterpret_cast<const float4 *>(specm + ((size_t)HB_IDX(hd, H) * N1 + k1o) * N2) + r;
+        float4 ha[4], hb[4];
+        step_done();
+        if (issuer) issue(8);                         // stage B
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            ha[i] = __ldg(&hrow4[i * 128]);
+            hb[i] = __ldg(&hrow4[(4 + i) * 128]);
+        }
+        wait_product();
+
+        // T2 (as in prefill_monarch_kernel, R3 = 2)
+        {
+            constexpr int CW = 16, OWN = 4;
+            const int k2 = r >> 1;
+            const float2 tw1 = fft::expi_neg(k2, 64 * R3);
+            const int row = kappa(k2, c);
+#pragma unroll 1
+            for (int m0 = 0; m0 < C; m0 += CW) {
+                float4 h4[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    h4[i] = ha[i];
+                    ha[i] = hb[i];
+                }
+                if (m0 + 2 * CW < C) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) hb[i] = __ldg(&hrow4[(((m0 + 2 * CW) / CW) * 4 + i) * 128]);
+                }
+                const float2 *hc = reinterpret_cast<const float2 *>(h4);
+                float x[CW];
+                tc::tmem_ld16(trow + m0, x);
+                tc::tmem_wait_ld();
+                float o[CW];
+#pragma unroll
+                for (int i = 0; i < OWN; ++i) {
+                    float2 V[2];
+#pragma unroll
+                    for (int n3 = 0; n3 < 2; ++n3) {
+                        const int je = (2 * i) * 2 + n3, jo = (2 * i + 1) * 2 + n3;
+                        const float rcv = __shfl_xor_sync(0xffffffffu, c ? x[je] : x[jo], 1);
+                        V[n3] = c ? make_float2(rcv, x[jo]) : make_float2(x[je], rcv);
+                    }
+                    V[1] = cmul(V[1], tw1);
+                    fft::dft2<false>(V[0], V[1]);
+                    V[0] = cmul(V[0], hc[i * 2]);
+                    V[1] = cmul(V[1], hc[i * 2 + 1]);
+                    fft::dft2<true>(V[0], V[1]);
+                    V[1] = cmulc(V[1], tw1);
+#pragma unroll
+                    for (int n3 = 0; n3 < 2; ++n3) {
+                        const float2 z = V[n3];
+                        const int je = (2 * i) * 2 + n3, jo = (2 * i + 1) * 2 + n3;
+                        const float rcv = __shfl_xor_sync(0xffffffffu, c ? z.x : -z.y, 1);
+                        o[je] = c ? rcv : z.x;
+                        o[jo] = c ? -z.y : rcv;
+                    }
+                }
+                uint8_t *drow = bop + (m0 >> 6) * M::kAtom + row * 128;
+#pragma unroll
+                for (int i = 0; i < CW / 8; ++i) {
+                    const int chunk = ((m0 & 63) >> 3) + i;
+                    *reinterpret_cast<uint4 *>(drow + ((chunk ^ (row & 7)) << 4)) =
+                        make_uint4(pack2(o[8 * i], o[8 * i + 1]), pack2(o[8 * i + 2], o[8 * i + 3]),
+                                   pack2(o[8 * i + 4], o[8 * i + 5]), pack2(o[8 * i + 6], o[8 * i + 7]));
+                }
+            }
+        }
+        step_done();
+        if (issuer) issue(8);                         // stage B, inverse direction
+        wait_product();
+
+        // T3 (as in prefill_monarch_kernel, R3 = 2)
+        {
+            const int n2 = r >> 1;
+            const int ex = R3 * n2 + c;
+            const float2 st = fft::expi_neg(ex % N2, N2);
+            const int colo = R3 * n2;
+#pragma unroll 1
+            for (int m0 = 0; m0 < C; m0 += 32) {
+                float x[32];
+                tc::tmem_ld32(trow + m0, x);
+                tc::tmem_wait_ld();
+                const int k10 = m0 / R3;
+                float2 w = fft::expi_neg((ex * k10) % N2, N2);
+                float o[32];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float rcv = __shfl_xor_sync(0xffffffffu, c ? x[2 * i] : x[2 * i + 1], 1);
+                    const float2 V = c ? make_float2(rcv, x[2 * i + 1]) : make_float2(x[2 * i], rcv);
+                    const float2 z = cmul(V, w);
+                    w = cmul(w, st);
+                    const float back = __shfl_xor_sync(0xffffffffu, c ? z.x : z.y, 1);
+                    o[2 * i] = c ? back : z.x;
+                    o[2 * i + 1] = c ? z.y : back;
+                }
+#pragma unroll
+                for (int gq = 0; gq < 16; ++gq)
+                    *reinterpret_cast<uint32_t *>(bop + bop_off(kappa(k10 + gq, c), colo)) = pack2(o[2 * gq], o[2 * gq + 1]);
+            }
+        }
+        step_done();
+        if (issuer) issue(8);                         // stage A, inverse direction
+        wait_product();
+
+        // T4: the row out (conjugate of the product), two halves of 64 columns staged as Re / Im
+        // planes [n1][64] fp32 (16-byte chunks XOR-ed by n1 % 8), then written back coalesced
+        {
+            const int n1 = r >> 1;
+            const float sg = c ? -1.f : 1.f;
+            float *plane = reinterpret_cast<float *>(bop + c * 64 * 64 * 4) + n1 * 64;
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+#pragma unroll 1
+                for (int j0 = 0; j0 < 64; j0 += 32) {
+                    float x[32];
+                    tc::tmem_ld32(trow + 64 * h + j0, x);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        *reinterpret_cast<float4 *>(plane + ((((j0 >> 2) + i) ^ (n1 & 7)) << 2)) =
+                            make_float4(sg * x[4 * i], sg * x[4 * i + 1], sg * x[4 * i + 2], sg * x[4 * i + 3]);
+                }
+                wg_sync(p);
+                const float *pr = reinterpret_cast<const float *>(bop), *pi = pr + 64 * 64;
+#pragma unroll 4
+                for (int e = wt; e < 64 * 32; e += 128) {
+                    const int m = e >> 5, jp = (e & 31) * 2;
+                    const int off = m * 64 + ((((jp >> 2)) ^ (m & 7)) << 2) + (jp & 3);
+                    const float2 re = *reinterpret_cast<const float2 *>(pr + off);
+                    const float2 im = *reinterpret_cast<const float2 *>(pi + off);
+                    const long long t = 128LL * m + 64 * h + jp;
+                    if (HB_OK(rw * N2 + t + 1, n_y))
+                        *reinterpret_cast<float4 *>(rowp + t) = make_float4(re.x, im.x, re.y, im.y);
+                }
+                wg_sync(p);
+            }
+        }
+        tc::tmem_wait_ld();
+        tc::tc_fence_before();
+    }
+    tc::tc_fence_after();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, M::kTmemCols);
+}
+
 int sm_count_now() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -652,6 +940,23 @@ cudaError_t launch_prefill_monarch(int r3, const void *q, const void *k, const v
         case 4: return launch_r<4>(q, k, v, B, L, Dch, H, d, spec, lam, y, state_out, err, s);
         default: return cudaErrorInvalidValue;
     }
+}
+
+bool fourstep_tc_enabled() { return g_tensor_core_fft.load() != 0; }
+
+cudaError_t launch_fourstep_inner_tc(float2 *Y, int N1, int ncols, int nslots, int paired, int ch, int H,
+                                     const float2 *specm, int *err, cudaStream_t s) {
+    using M = Mon<2>;
+    const size_t smem = (size_t)(M::kSmB + M::P * M::kBop) + 64 + 1024;
+    cudaError_t e = cudaFuncSetAttribute((const void *)fourstep_inner_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const long long rows = (long long)ncols * N1;
+    const long long ctas = (rows + M::P - 1) / M::P;
+    const long long grid = ctas < sm_count_now() ? ctas : sm_count_now();
+    if (grid < 1) return cudaSuccess;
+    fourstep_inner_tc_kernel<<<(unsigned)grid, 512, smem, s>>>(Y, N1, ncols, nslots, paired, ch, H, specm, err);
+    return cudaGetLastError();
 }
 
 }  // namespace hyena

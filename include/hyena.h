@@ -131,7 +131,9 @@ int hyena_filter_spectrum(const float *h, int H, int L, int fft_len, float *spec
  *   workspace  : device scratch, >= hyena_prefill_workspace_bytes(...) bytes,
  *                256-byte aligned; contents on entry are ignored.
  * Alignment: all activation pointers 4-byte aligned (bf16) / 8-byte (f32).
- * Routes.  bf16 activations with an internal FFT length of 4096, 8192 or 16384,
+ * Routes.  Beyond 16384 points (the four-step route), the inner 8192-point
+ * transforms of bf16 activations run on the tensor cores the same way.
+ * bf16 activations with an internal FFT length of 4096, 8192 or 16384,
  * an even number of channels per head, Dch a multiple of 8 (of 4 at 16384)
  * and q, k, v, y aligned to 16 bytes (8 at 16384) run on the tensor cores: each
  * transform is factored as 64 x 64 x (N/4096) and its two 64-point DFT stages
@@ -148,8 +150,9 @@ int hyena_filter_spectrum(const float *h, int H, int L, int fft_len, float *spec
  */
 size_t hyena_prefill_workspace_bytes(int B, int L, int Dch, int H, int d, int fft_len);
 size_t hyena_prefill_error_offset(int B, int L, int Dch, int H, int d, int fft_len);
-/* 1 if hyena_prefill with these arguments runs on the tensor cores, 0 if on the
- * CUDA cores; HYENA_ERR_ARG / HYENA_ERR_SHAPE / HYENA_ERR_UNSUPPORTED as
+/* 1 if hyena_prefill with these arguments runs its DFT stages on the tensor cores
+ * (all of them up to 16384 points; the inner 8192-point transforms of the
+ * four-step route beyond), 0 if on the CUDA cores; HYENA_ERR_ARG / HYENA_ERR_SHAPE / HYENA_ERR_UNSUPPORTED as
  * hyena_prefill would return for invalid arguments.  Pointers are only
  * inspected for alignment.  Host-only (no CUDA call). */
 int hyena_prefill_uses_tensor_cores(int dtype, int B, int L, int Dch, int H, int d, int fft_len,

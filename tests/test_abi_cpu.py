@@ -228,7 +228,8 @@ def test_route_query_follows_the_documented_rule(lib):
     assert lib.hyena_prefill_uses_tensor_cores(BF16, 8, 4096, 1024, 8, 16, 8192, a, a, a, a) == 1
     assert lib.hyena_prefill_uses_tensor_cores(F32, 8, 4096, 1024, 8, 16, 8192, a, a, a, a) == 0
     assert lib.hyena_prefill_uses_tensor_cores(BF16, 8, 4096, 1020, 4, 16, 8192, a, a, a, a) == 0   # Dch % 8
-    assert lib.hyena_prefill_uses_tensor_cores(BF16, 1, 9000, 16, 2, 16, 32768, a, a, a, a) == 0    # four-step
+    assert lib.hyena_prefill_uses_tensor_cores(BF16, 1, 9000, 16, 2, 16, 32768, a, a, a, a) == 1    # four-step inner
+    assert lib.hyena_prefill_uses_tensor_cores(F32, 1, 9000, 16, 2, 16, 32768, a, a, a, a) == 0
     assert lib.hyena_prefill_uses_tensor_cores(BF16, 1, 900, 16, 2, 16, 2048, a, a, a, a) == 0      # too short
     odd = ctypes.c_void_p((1 << 20) + 4)
     assert lib.hyena_prefill_uses_tensor_cores(BF16, 8, 4096, 1024, 8, 16, 8192, a, odd, a, a) == 0

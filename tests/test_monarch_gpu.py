@@ -130,8 +130,33 @@ def test_layouts_outside_the_route_fall_back_to_cuda_cores(oracle):
     assert rel_err(state_c128(s), s_ref) <= 1e-4
 
 
+FOURSTEP = [
+    # B, L, Dch, H, d, fft_len: the four-step route, inner 8192-point rows on the tensor cores
+    (1, 9000, 6, 3, 4, 32768),       # ragged, heads of 2 channels
+    (2, 20000, 8, 2, 16, 65536),     # two sequences, N1 = 8
+    (1, 40000, 4, 1, 8, 131072),     # N1 = 16 (the long prefill's length)
+]
+
+
+@pytest.mark.parametrize("B,L,Dch,H,d,N", FOURSTEP)
+def test_four_step_inner_rows_on_tensor_cores(oracle, record_property, B, L, Dch, H, d, N):
+    w, p = _case(L % 97 + d, B, L, Dch, H, d)
+    (q, k, v), y, s = _run(w, p, N)
+    assert ops.prefill_uses_tensor_cores(q.cuda(), k.cuda(), v.cuda(), H, d, N)
+    y_ref, s_ref = oracle.recurrent(W.to_f64(q), W.to_f64(k), W.to_f64(v), p.lam, p.R, p.Dskip, H=H)
+    ey = rel_err(y.cpu().double().numpy(), y_ref)
+    es = rel_err(state_c128(s), s_ref)
+    record_property("y_err", ey)
+    record_property("state_err", es)
+    assert ey <= TOL["bf16"] and es <= 1e-4, (ey, es)
+    assert ey <= Y_MARGIN, ey
+    with ops.fft_tensor_cores(False):
+        _, y_cc, _ = _run(w, p, N, tensor_cores=False)
+    assert not torch.equal(y, y_cc)
+
+
 @pytest.mark.parametrize("L", [1, 2, 3, 17, 200])
-@pytest.mark.parametrize("N,Dch,H", [(4096, 8, 2), (8192, 16, 8), (16384, 4, 1)])
+@pytest.mark.parametrize("N,Dch,H", [(4096, 8, 2), (8192, 16, 8), (16384, 4, 1), (32768, 6, 3)])
 def test_tensor_core_prefill_in_bounds(oracle, L, N, Dch, H):
     """The bounds-checked build: no global access out of range, results as in the release build."""
     from distilled_ssm_decode_b200 import build
