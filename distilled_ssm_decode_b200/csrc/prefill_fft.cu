@@ -239,24 +239,42 @@ struct ActSrc {
     }
 };
 
+// Thread -> (column, n2) of the outer steps.  COLS8: a block takes 8 adjacent columns x 32 values
+// of n2, the column fastest, so that 8 lanes read (or write) one 32-byte piece of an activation row
+// (8 channel pairs) instead of 8 separate 4-byte pieces; else a block takes 256 values of n2 of one
+// column.
+template <bool COLS8>
+__device__ __forceinline__ void outer_index(int &col, int &n2) {
+    if constexpr (COLS8) {
+        col = blockIdx.y * 8 + (threadIdx.x & 7);
+        n2 = blockIdx.x * 32 + (threadIdx.x >> 3);
+    } else {
+        col = blockIdx.y;
+        n2 = blockIdx.x * blockDim.x + threadIdx.x;
+    }
+}
+
 // step 1: Y[col][k1][n2] = w_N^(n2 k1) * DFT_N1 over n1 of x[N2 n1 + n2]
-template <int N1, class Src>
+template <int N1, class Src, bool COLS8>
 __global__ void __launch_bounds__(256)
-fourstep_fwd1_kernel(Src src, int N2, float2 *__restrict__ Y) {
-    const int col = blockIdx.y;
-    const int n2 = blockIdx.x * blockDim.x + threadIdx.x;
-    if (n2 >= N2) return;
+fourstep_fwd1_kernel(Src src, int N2, float2 *__restrict__ Y, int ncols) {
+    int col, n2;
+    outer_index<COLS8>(col, n2);
+    if (n2 >= N2 || col >= ncols) return;
     const long long N = (long long)N1 * N2;
     float2 x[N1];
 #pragma unroll
     for (int n1 = 0; n1 < N1; ++n1) x[n1] = src(col, (long long)N2 * n1 + n2);
     fft::dftR<N1, false>(x);
     float2 *out = Y + (size_t)col * N + n2;
+    // twiddles w_N^(n2 k1) as powers of one exactly reduced w_N^(n2) (at most 15 products)
+    const float2 w1 = fft::expi_neg(n2, (int)N);
+    float2 w = w1;
 #pragma unroll
     for (int k1 = 0; k1 < N1; ++k1) {
-        const float2 w = fft::expi_neg(n2 * k1, (int)N);
-        if (HB_OK((long long)col * N + (long long)k1 * N2 + n2, (long long)gridDim.y * N))
+        if (HB_OK((long long)col * N + (long long)k1 * N2 + n2, (long long)ncols * N))
             out[(size_t)k1 * N2] = k1 ? cmul(x[k1], w) : x[k1];
+        if (k1) w = cmul(w, w1);
     }
 }
 
@@ -311,22 +329,24 @@ __global__ void fourstep_spec_tc_kernel(const float2 *__restrict__ spec_perm, in
 }
 
 // step 3: inverse across the long stride, gate-out, store the first L outputs
-template <int N1, class Act>
+template <int N1, class Act, bool COLS8>
 __global__ void __launch_bounds__(256)
 fourstep_inv1_kernel(const float2 *__restrict__ Y, int N2, int L, int Dch, int nslots, int paired,
-                     const typename Act::T *__restrict__ q, typename Act::T *__restrict__ y) {
-    const int col = blockIdx.y;
-    const int n2 = blockIdx.x * blockDim.x + threadIdx.x;
-    if (n2 >= N2) return;
+                     const typename Act::T *__restrict__ q, typename Act::T *__restrict__ y, int ncols) {
+    int col, n2;
+    outer_index<COLS8>(col, n2);
+    if (n2 >= N2 || col >= ncols) return;
     const long long N = (long long)N1 * N2;
     const float2 *in = Y + (size_t)col * N + n2;
-    const long long n_in = (long long)gridDim.y * N - ((long long)col * N + n2);
+    const long long n_in = (long long)ncols * N - ((long long)col * N + n2);
     (void)n_in;
     float2 x[N1];
+    const float2 w1 = fft::expi_neg(n2, (int)N);
+    float2 w = w1;
 #pragma unroll
     for (int k1 = 0; k1 < N1; ++k1) {
-        const float2 w = fft::expi_neg(n2 * k1, (int)N);
         x[k1] = k1 ? cmulc(in[HB_IDX((long long)k1 * N2, n_in)], w) : in[0];
+        if (k1) w = cmul(w, w1);
     }
     fft::dftR<N1, true>(x);
     const int b = col / nslots, slot = col % nslots;
@@ -334,7 +354,7 @@ fourstep_inv1_kernel(const float2 *__restrict__ Y, int N2, int L, int Dch, int n
 #pragma unroll
     for (int n1 = 0; n1 < N1; ++n1) {
         const long long t = (long long)N2 * n1 + n2;
-        if (t < L && HB_OK(((long long)b * L + t) * Dch + c0 + paired, (long long)(gridDim.y / nslots) * L * Dch)) {
+        if (t < L && HB_OK(((long long)b * L + t) * Dch + c0 + paired, (long long)(ncols / nslots) * L * Dch)) {
             const size_t o = ((size_t)b * L + t) * Dch + c0;
             if (paired) {
                 const float2 qq = Act::ld2(q + o);
@@ -346,31 +366,36 @@ fourstep_inv1_kernel(const float2 *__restrict__ Y, int N2, int L, int Dch, int n
     }
 }
 
-template <class Src>
-cudaError_t launch_fwd1(int N1, Src src, int N2, int ncols, float2 *Y, cudaStream_t s) {
-    dim3 grid((N2 + 255) / 256, ncols);
+template <class Src, bool COLS8>
+cudaError_t launch_fwd1_t(int N1, Src src, int N2, int ncols, float2 *Y, cudaStream_t s) {
+    const dim3 grid = COLS8 ? dim3((N2 + 31) / 32, (ncols + 7) / 8) : dim3((N2 + 255) / 256, ncols);
     switch (N1) {
-        case 2: fourstep_fwd1_kernel<2><<<grid, 256, 0, s>>>(src, N2, Y); break;
-        case 4: fourstep_fwd1_kernel<4><<<grid, 256, 0, s>>>(src, N2, Y); break;
-        case 8: fourstep_fwd1_kernel<8><<<grid, 256, 0, s>>>(src, N2, Y); break;
-        case 16: fourstep_fwd1_kernel<16><<<grid, 256, 0, s>>>(src, N2, Y); break;
+        case 2: fourstep_fwd1_kernel<2, Src, COLS8><<<grid, 256, 0, s>>>(src, N2, Y, ncols); break;
+        case 4: fourstep_fwd1_kernel<4, Src, COLS8><<<grid, 256, 0, s>>>(src, N2, Y, ncols); break;
+        case 8: fourstep_fwd1_kernel<8, Src, COLS8><<<grid, 256, 0, s>>>(src, N2, Y, ncols); break;
+        case 16: fourstep_fwd1_kernel<16, Src, COLS8><<<grid, 256, 0, s>>>(src, N2, Y, ncols); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
+}
+// activation columns (channel pairs or channels) take the 8-column blocks; the filter's do not
+template <class Src>
+cudaError_t launch_fwd1(int N1, Src src, int N2, int ncols, float2 *Y, cudaStream_t s, bool cols8 = false) {
+    return cols8 ? launch_fwd1_t<Src, true>(N1, src, N2, ncols, Y, s) : launch_fwd1_t<Src, false>(N1, src, N2, ncols, Y, s);
 }
 
 template <class Act>
 cudaError_t launch_inv1(int N1, const float2 *Y, int N2, int L, int Dch, int nslots, int paired,
                         int ncols, const void *q, void *y, cudaStream_t s) {
-    dim3 grid((N2 + 255) / 256, ncols);
+    const dim3 grid((N2 + 31) / 32, (ncols + 7) / 8);          // 8-column blocks
     using T = typename Act::T;
     const T *qq = static_cast<const T *>(q);
     T *yy = static_cast<T *>(y);
     switch (N1) {
-        case 2: fourstep_inv1_kernel<2, Act><<<grid, 256, 0, s>>>(Y, N2, L, Dch, nslots, paired, qq, yy); break;
-        case 4: fourstep_inv1_kernel<4, Act><<<grid, 256, 0, s>>>(Y, N2, L, Dch, nslots, paired, qq, yy); break;
-        case 8: fourstep_inv1_kernel<8, Act><<<grid, 256, 0, s>>>(Y, N2, L, Dch, nslots, paired, qq, yy); break;
-        case 16: fourstep_inv1_kernel<16, Act><<<grid, 256, 0, s>>>(Y, N2, L, Dch, nslots, paired, qq, yy); break;
+        case 2: fourstep_inv1_kernel<2, Act, true><<<grid, 256, 0, s>>>(Y, N2, L, Dch, nslots, paired, qq, yy, ncols); break;
+        case 4: fourstep_inv1_kernel<4, Act, true><<<grid, 256, 0, s>>>(Y, N2, L, Dch, nslots, paired, qq, yy, ncols); break;
+        case 8: fourstep_inv1_kernel<8, Act, true><<<grid, 256, 0, s>>>(Y, N2, L, Dch, nslots, paired, qq, yy, ncols); break;
+        case 16: fourstep_inv1_kernel<16, Act, true><<<grid, 256, 0, s>>>(Y, N2, L, Dch, nslots, paired, qq, yy, ncols); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
@@ -411,7 +436,7 @@ cudaError_t prefill_fourstep(const void *q, const void *k, const void *v, int B,
     float2 *Y = static_cast<float2 *>(scratch);
     char *after = static_cast<char *>(scratch) + (size_t)ncols * N * sizeof(float2);
     ActSrc<Act> src{static_cast<const T *>(k), static_cast<const T *>(v), L, Dch, nslots, paired};
-    cudaError_t e = launch_fwd1(N1, src, N2, ncols, Y, s);
+    cudaError_t e = launch_fwd1(N1, src, N2, ncols, Y, s, true);
     if (e != cudaSuccess) return e;
     if (Act::bytes == 2 && fourstep_tc_enabled()) {
         // bf16 activations: the inner transforms on the tensor cores, with the spectrum rows in the
