@@ -1,4 +1,5 @@
-"""FFT prefill on the tensor cores (bf16 activations; FFT lengths 4096, 8192, 16384).
+"""FFT prefill on the tensor cores (bf16 activations; FFT lengths 4096, 8192, 16384, and the
+inner 8192-point rows of the four-step route beyond).
 
 hyena_prefill runs these calls with each transform factored as 64 x 64 x (N/4096): the two
 64-point DFT stages are dense matrix products on the tensor cores (bf16 operands, fp32
